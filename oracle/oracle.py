@@ -1,0 +1,271 @@
+"""ctypes wrapper of the CPU oracle (liboracle.so).  TEST INFRASTRUCTURE ONLY.
+
+Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline / reference
+legs may import this module.  It imports nothing from the CUDA package; scenes
+come from the shared seeded generator, which holds no splatting arithmetic.
+
+Every function restates one step of the packed 3DGS step in plain serial form
+(see oracle.cpp for the per-step citations):
+  project      packed projection + both compactions (plain flag scan and bitmask)
+  intersect    tile intersections by the per-tile overlap test, range form checked
+  sort         std::stable_sort by key
+  tile_ranges  per-tile [start, end) by counting
+  rasterize_fwd / rasterize_bwd / project_bwd  one pixel / one row at a time
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+PAIRS_PER_BLOCK = 128
+TILE = 16
+ROW = 12
+
+
+class Dims(ct.Structure):
+    _fields_ = [("C", ct.c_int32), ("W", ct.c_int32), ("H", ct.c_int32), ("sh_degree", ct.c_int32),
+                ("N", ct.c_int64), ("near_plane", ct.c_float), ("far_plane", ct.c_float)]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ct.CDLL(path)
+        P = ct.c_void_p
+        i64, i32 = ct.c_int64, ct.c_int
+        L.orc_exp_fp32.argtypes = [ct.c_float]
+        L.orc_exp_fp32.restype = ct.c_float
+        L.orc_exp_fp32_vec.argtypes = [P, P, i64]
+        L.orc_sh_basis_f64.argtypes = [i32, ct.c_double, ct.c_double, ct.c_double, P]
+        L.orc_sh_basis_grad_f64.argtypes = [i32, ct.c_double, ct.c_double, ct.c_double, P]
+        L.orc_geometry.argtypes = [P, P]
+        L.orc_project.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, P, P, P, P, P, i64, i32]
+        L.orc_row_boxes.argtypes = [P, P, P, P, P, P, P, P, i64, P]
+        L.orc_count_tiles.argtypes = [P, P, i64, P, P]
+        L.orc_intersect.argtypes = [P, P, P, P, i64, i32, P, P, i64, P]
+        L.orc_sort.argtypes = [P, P, i64]
+        L.orc_tile_ranges.argtypes = [P, i64, i64, P]
+        L.orc_rasterize_fwd.argtypes = [P, P, P, P, i32, P, P, P, i32]
+        L.orc_rasterize_bwd.argtypes = [P, P, P, P, P, P, i32, i64, P, i32]
+        L.orc_project_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i64, P, i32, P, P, P, P, P]
+        for f in ("orc_project", "orc_row_boxes", "orc_count_tiles", "orc_intersect", "orc_sort",
+                  "orc_tile_ranges", "orc_rasterize_fwd", "orc_rasterize_bwd", "orc_project_bwd"):
+            getattr(L, f).restype = ct.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ct.c_void_p)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def dims_of(scene) -> Dims:
+    return Dims(scene.C, scene.W, scene.H, scene.sh_degree, scene.N, scene.near, scene.far)
+
+
+def geometry(scene) -> dict:
+    out = np.zeros(6, np.int64)
+    d = dims_of(scene)
+    lib().orc_geometry(ct.byref(d), _p(out))
+    keys = ("tiles_x", "tiles_y", "tiles_per_cam", "n_pad", "words_per_cam", "blocks_per_cam")
+    g = {k: int(v) for k, v in zip(keys, out)}
+    g["n_tiles"] = g["tiles_per_cam"] * scene.C
+    g["mask_words"] = g["words_per_cam"] * scene.C
+    g["mask_blocks"] = g["blocks_per_cam"] * scene.C
+    return g
+
+
+def exp_fp32(x: float) -> float:
+    return float(lib().orc_exp_fp32(ct.c_float(x)))
+
+
+def exp_fp32_vec(x) -> np.ndarray:
+    x = _c(x, np.float32)
+    y = np.empty_like(x)
+    lib().orc_exp_fp32_vec(_p(x), _p(y), x.size)
+    return y
+
+
+def sh_basis(degree: int, d) -> np.ndarray:
+    out = np.zeros(16)
+    lib().orc_sh_basis_f64(degree, float(d[0]), float(d[1]), float(d[2]), _p(out))
+    return out[: (degree + 1) ** 2]
+
+
+def sh_basis_grad(degree: int, d) -> np.ndarray:
+    out = np.zeros((16, 3))
+    lib().orc_sh_basis_grad_f64(degree, float(d[0]), float(d[1]), float(d[2]), _p(out))
+    return out[: (degree + 1) ** 2]
+
+
+def _inputs(scene):
+    """All oracle inputs are fp64; fp32 scene arrays convert exactly."""
+    return dict(cams=_c(scene.cams, np.float64), means=_c(scene.means, np.float64),
+                quats=_c(scene.quats, np.float64), scales=_c(scene.scales, np.float64),
+                opac=_c(scene.opacities, np.float64), sh=_c(scene.sh, np.float64))
+
+
+def project(scene, precision: int = 0, nthreads: int = 0, rows: bool = True) -> dict:
+    g = geometry(scene)
+    d = dims_of(scene)
+    x = _inputs(scene)
+    mask = np.zeros(g["mask_words"], np.uint32)
+    bc = np.zeros(g["mask_blocks"], np.uint32)
+    bo = np.zeros(g["mask_blocks"] + 1, np.int64)
+    nnz = ct.c_int64(0)
+    L = lib()
+    args = [ct.byref(d), _p(x["cams"]), _p(x["means"]), _p(x["quats"]), _p(x["scales"]), _p(x["opac"]),
+            _p(x["sh"]), precision, _p(mask), _p(bc), _p(bo), ct.byref(nnz)]
+    rc = L.orc_project(*args, None, None, None, None, None, 0, nthreads)
+    if rc != 0:
+        raise RuntimeError(f"oracle projection: compactions disagree (rc={rc})")
+    out = dict(mask=mask, block_count=bc, block_off=bo, nnz=int(nnz.value))
+    if not rows:
+        return out
+    n = out["nnz"]
+    screen = np.zeros((max(n, 1), ROW), np.float64)
+    aabb = np.zeros((max(n, 1), 2), np.uint32)
+    row_cam = np.zeros(max(n, 1), np.int32)
+    row_gauss = np.zeros(max(n, 1), np.int64)
+    rgb_cl = np.zeros((max(n, 1), 3), np.uint8)
+    rc = L.orc_project(*args, _p(screen), _p(aabb), _p(row_cam), _p(row_gauss), _p(rgb_cl), n, nthreads)
+    if rc != 0:
+        raise RuntimeError(f"oracle projection failed (rc={rc})")
+    out.update(screen=screen[:n], aabb=aabb[:n], row_cam=row_cam[:n], row_gauss=row_gauss[:n],
+               rgb_clamped=rgb_cl[:n])
+    return out
+
+
+def row_boxes(scene, proj) -> np.ndarray:
+    d = dims_of(scene)
+    x = _inputs(scene)
+    n = proj["nnz"]
+    box = np.zeros((max(n, 1), 4), np.float32)
+    rc = lib().orc_row_boxes(ct.byref(d), _p(x["cams"]), _p(x["means"]), _p(x["quats"]), _p(x["scales"]),
+                             _p(x["opac"]), _p(_c(proj["row_cam"], np.int32)),
+                             _p(_c(proj["row_gauss"], np.int64)), n, _p(box))
+    if rc != 0:
+        raise RuntimeError("row_boxes: row not visible")
+    return box[:n]
+
+
+def count_tiles(scene, aabb) -> tuple[np.ndarray, int]:
+    d = dims_of(scene)
+    n = len(aabb)
+    per = np.zeros(max(n, 1), np.int64)
+    tot = ct.c_uint64(0)
+    lib().orc_count_tiles(ct.byref(d), _p(_c(aabb, np.uint32)), n, _p(per), ct.byref(tot))
+    return per[:n], int(tot.value)
+
+
+def intersect(scene, proj, all_pairs: bool | None = None) -> dict:
+    g = geometry(scene)
+    d = dims_of(scene)
+    n = proj["nnz"]
+    _, total = count_tiles(scene, proj["aabb"])
+    if all_pairs is None:
+        all_pairs = n * g["tiles_per_cam"] <= 200_000_000
+    keys = np.zeros(max(total, 1), np.uint64)
+    vals = np.zeros(max(total, 1), np.uint32)
+    tot = ct.c_uint64(0)
+    rc = lib().orc_intersect(ct.byref(d), _p(_c(proj["screen"], np.float64)), _p(_c(proj["aabb"], np.uint32)),
+                             _p(_c(proj["row_cam"], np.int32)), n, int(all_pairs), _p(keys), _p(vals), total,
+                             ct.byref(tot))
+    if rc != 0:
+        raise RuntimeError(f"oracle intersect: range form and overlap test disagree (rc={rc})")
+    return dict(keys=keys[:total], vals=vals[:total], n_isects=int(tot.value))
+
+
+def sort(keys, vals) -> tuple[np.ndarray, np.ndarray]:
+    k = np.array(keys, np.uint64, copy=True)
+    v = np.array(vals, np.uint32, copy=True)
+    lib().orc_sort(_p(k), _p(v), len(k))
+    return k, v
+
+
+def tile_ranges(keys, n_tiles: int) -> np.ndarray:
+    off = np.zeros(n_tiles + 1, np.int64)
+    k = _c(keys, np.uint64)
+    if lib().orc_tile_ranges(_p(k), len(k), n_tiles, _p(off)) != 0:
+        raise RuntimeError("tile id out of range")
+    return off
+
+
+def rasterize_fwd(scene, screen, vals_sorted, tile_off, precision: int = 0, nthreads: int = 0):
+    d = dims_of(scene)
+    npix = scene.C * scene.H * scene.W
+    img = np.zeros((scene.C, scene.H, scene.W, 3))
+    T = np.zeros((scene.C, scene.H, scene.W))
+    last = np.zeros((scene.C, scene.H, scene.W), np.int64)
+    lib().orc_rasterize_fwd(ct.byref(d), _p(_c(screen, np.float64)), _p(_c(vals_sorted, np.uint32)),
+                            _p(_c(tile_off, np.int64)), precision, _p(img), _p(T), _p(last), nthreads)
+    assert img.size == 3 * npix
+    return img, T, last
+
+
+def rasterize_bwd(scene, screen, vals_sorted, tile_off, v_img, v_T=None, precision: int = 0,
+                  nthreads: int = 0) -> np.ndarray:
+    d = dims_of(scene)
+    n = len(screen)
+    vs = np.zeros((max(n, 1), ROW))
+    vT = None if v_T is None else _c(v_T, np.float64)
+    lib().orc_rasterize_bwd(ct.byref(d), _p(_c(screen, np.float64)), _p(_c(vals_sorted, np.uint32)),
+                            _p(_c(tile_off, np.int64)), _p(_c(v_img, np.float64)), _p(vT), precision, n,
+                            _p(vs), nthreads)
+    return vs[:n]
+
+
+def project_bwd(scene, proj, v_screen, precision: int = 0) -> dict:
+    d = dims_of(scene)
+    x = _inputs(scene)
+    N, K = scene.N, scene.K
+    out = dict(v_means=np.zeros((N, 3)), v_quats=np.zeros((N, 4)), v_scales=np.zeros((N, 3)),
+               v_opacities=np.zeros(N), v_sh=np.zeros((N, K, 3)))
+    lib().orc_project_bwd(ct.byref(d), _p(x["cams"]), _p(x["means"]), _p(x["quats"]), _p(x["scales"]),
+                          _p(x["opac"]), _p(x["sh"]), _p(_c(proj["row_cam"], np.int32)),
+                          _p(_c(proj["row_gauss"], np.int64)), proj["nnz"], _p(_c(v_screen, np.float64)),
+                          precision, _p(out["v_means"]), _p(out["v_quats"]), _p(out["v_scales"]),
+                          _p(out["v_opacities"]), _p(out["v_sh"]))
+    return out
+
+
+def upstream(scene, img) -> np.ndarray:
+    """dL/dimage of the scene: the given uniform field, or the L1 gradient
+    sign(img - target) / (3 W H C) against the scene's target."""
+    if scene.upstream == "uniform":
+        return np.asarray(scene.v_img, np.float32)
+    return (np.sign(np.asarray(img, np.float64) - scene.target) * scene.l1_scale).astype(np.float32)
+
+
+def forward(scene, precision: int = 0, nthreads: int = 0) -> dict:
+    g = geometry(scene)
+    proj = project(scene, precision, nthreads)
+    isect = intersect(scene, proj)
+    ks, vs = sort(isect["keys"], isect["vals"])
+    toff = tile_ranges(ks, g["n_tiles"])
+    img, T, last = rasterize_fwd(scene, proj["screen"], vs, toff, precision, nthreads)
+    return dict(proj=proj, isect=isect, keys_sorted=ks, vals_sorted=vs, tile_off=toff, img=img, T=T,
+                last=last, geo=g)
+
+
+def step(scene, precision: int = 0, nthreads: int = 0, v_img=None, v_T=None) -> dict:
+    """One forward+backward pass; gradients in fp64."""
+    f = forward(scene, precision, nthreads)
+    if v_img is None:
+        v_img = upstream(scene, f["img"])
+    v_screen = rasterize_bwd(scene, f["proj"]["screen"], f["vals_sorted"], f["tile_off"], v_img, v_T, precision,
+                             nthreads)
+    grads = project_bwd(scene, f["proj"], v_screen, precision)
+    f.update(v_img=v_img, v_screen=v_screen, grads=grads)
+    return f

@@ -1,0 +1,392 @@
+"""Pins of the CPU oracle against what the pages and mathematics fix.
+
+Nothing here calls the CUDA path.  Each test targets a mistake that could hide
+in the oracle (a dropped term, a wrong sign or index, a transposed operand):
+
+* exp:         error bound against fp64 exp on a dense sweep;
+* SH basis:    the library's complex spherical harmonics (scipy) in real form,
+               and finite differences of the basis for its gradient;
+* projection:  closed forms (pinhole mean, isotropic 2D covariance, the
+               off-axis Jacobian limit), quaternion rotation from scipy, matrix
+               inverse from numpy;
+* compaction:  the plain flag scan and the bitmask scan agree (checked inside the
+               oracle) and the popcount bookkeeping reproduces the pages' sizes;
+* AABB16:      the decoded box contains the float box exactly and the step
+               sizes the page prints;
+* intersect:   the all-tiles overlap test equals the range form; tile sets only
+               grow by at most one tile per side;
+* sort/ranges: numpy's stable lexsort and bincount;
+* rasterizer:  closed form of one Gaussian, telescoping sum, the 0.99 clamp
+               hand count;
+* backward:    central finite differences of the fp64 instantiation.
+"""
+import math
+
+import numpy as np
+import pytest
+from scipy.spatial.transform import Rotation
+from scipy.special import sph_harm_y
+
+from conftest import golden
+from gaussian_splatting_differentiable_packed_b200 import scenes
+from oracle import oracle as orc
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def make(means, quats, scales, opac, sh, cams, W, H, sh_degree=0, v_img=None):
+    N = len(means)
+    C = len(cams)
+    return scenes.Scene(0, C, W, H, sh_degree, N, 0.01, 1e10, np.asarray(cams, np.float32),
+                        np.asarray(means, np.float32), np.asarray(quats, np.float32),
+                        np.asarray(scales, np.float32), np.asarray(opac, np.float32),
+                        np.asarray(sh, np.float32).reshape(N, (sh_degree + 1) ** 2, 3), "uniform",
+                        v_img, None, "pin")
+
+
+def ident_cam(fx, fy, cx, cy):
+    return np.concatenate([np.eye(4).reshape(16), [fx, fy, cx, cy]]).astype(np.float32)
+
+
+# ---------------------------------------------------------------- exp
+def test_exp_error_bound_and_monotone():
+    x = -np.linspace(0.0, 87.0, 2_000_001).astype(np.float32)
+    y = orc.exp_fp32_vec(x).astype(np.float64)
+    exact = np.exp(x.astype(np.float64))
+    ulp = np.spacing(exact.astype(np.float32)).astype(np.float64)
+    err = np.abs(y - exact) / ulp
+    assert err.max() <= 2.0, err.max()
+    assert orc.exp_fp32(0.0) == 1.0
+    assert np.all(np.diff(y) <= 0.0)  # x decreasing -> non-increasing
+    # early-out safety used by a rasterizer: o <= 1 and sigma > 5.6 can never reach 1/255
+    assert orc.exp_fp32(-5.6) < np.float32(1.0) / np.float32(255.0)
+    assert orc.exp_fp32(-88.0) == 0.0
+
+
+# ---------------------------------------------------------------- SH
+def real_sh_scipy(l, m, d):
+    """Real SH from scipy's complex SH (Condon-Shortley phase included):
+    m<0 -> sqrt2 Im Y_l^|m|, m=0 -> Y_l^0, m>0 -> sqrt2 Re Y_l^m."""
+    x, y, z = d
+    theta = math.acos(max(-1.0, min(1.0, z)))
+    phi = math.atan2(y, x)
+    if m < 0:
+        return math.sqrt(2) * sph_harm_y(l, -m, theta, phi).imag
+    if m == 0:
+        return sph_harm_y(l, 0, theta, phi).real
+    return math.sqrt(2) * sph_harm_y(l, m, theta, phi).real
+
+
+def test_sh_basis_matches_library():
+    rng = np.random.default_rng(7)
+    for _ in range(50):
+        d = rng.normal(size=3)
+        d /= np.linalg.norm(d)
+        got = orc.sh_basis(3, d)
+        want = [real_sh_scipy(l, m, d) for l in range(4) for m in range(-l, l + 1)]
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_sh_basis_gradient_finite_difference():
+    rng = np.random.default_rng(8)
+    for _ in range(20):
+        d = rng.normal(size=3)
+        g = orc.sh_basis_grad(3, d)
+        for ax in range(3):
+            e = np.zeros(3)
+            e[ax] = 1e-6
+            fd = (orc.sh_basis(3, d + e) - orc.sh_basis(3, d - e)) / 2e-6
+            np.testing.assert_allclose(g[:, ax], fd, rtol=1e-6, atol=1e-8)
+
+
+# ---------------------------------------------------------------- projection
+def test_pinhole_mean_and_isotropic_covariance_closed_form():
+    fx, fy, cx, cy = 50.0, 60.0, 32.0, 24.0
+    p = np.array([0.5, -0.25, 2.0])
+    s = 0.04
+    sc = make([p], [[1, 0, 0, 0]], [[s, s, s]], [0.8], [[0.0, 0.0, 0.0]], [ident_cam(fx, fy, cx, cy)], 64, 48)
+    for prec in (0, 1):
+        pr = orc.project(sc, precision=prec)
+        assert pr["nnz"] == 1
+        row = pr["screen"][0]
+        u, v = p[0] / p[2], p[1] / p[2]
+        np.testing.assert_allclose(row[:2], [fx * u + cx, fy * v + cy], rtol=1e-6)
+        J = np.array([[fx / p[2], 0, -fx * u / p[2]], [0, fy / p[2], -fy * v / p[2]]])
+        S2 = s * s * J @ J.T + 0.3 * np.eye(2)
+        Q = np.linalg.inv(S2)
+        np.testing.assert_allclose(row[2:5], [Q[0, 0], Q[0, 1], Q[1, 1]], rtol=2e-6)
+        assert row[5] == np.float32(0.8)
+        assert row[9] == np.float32(2.0)
+
+
+def test_off_axis_jacobian_limit():
+    # u = x/z beyond 1.3 * (W/2)/fx: the Jacobian uses the clamped value, the mean does not
+    fx = fy = 40.0
+    W = H = 64
+    lim = 1.3 * (0.5 * W) / fx
+    z = 1.0
+    x = (lim + 0.5) * z
+    s = 0.3
+    sc = make([[x, 0.0, z]], [[1, 0, 0, 0]], [[s, s, s]], [0.9], [[0.0, 0.0, 0.0]],
+              [ident_cam(fx, fy, -20.0, 32.0)], W, H)
+    pr = orc.project(sc, precision=1)
+    assert pr["nnz"] == 1
+    row = pr["screen"][0]
+    J = np.array([[fx / z, 0, -fx * lim / z], [0, fy / z, 0.0]])
+    S2 = s * s * J @ J.T + 0.3 * np.eye(2)
+    Q = np.linalg.inv(S2)
+    np.testing.assert_allclose(row[2:5], [Q[0, 0], Q[0, 1], Q[1, 1]], rtol=1e-6)
+    assert abs(row[0] - (fx * x / z - 20.0)) < 1e-4
+
+
+def test_anisotropic_covariance_against_library_rotation():
+    sc = scenes.random_tiny(3, N=40, W=48, H=40, C=2, sh_degree=0)
+    pr = orc.project(sc, precision=1)
+    assert pr["nnz"] > 10
+    for r in range(pr["nnz"]):
+        c, n = pr["row_cam"][r], pr["row_gauss"][r]
+        V = sc.cams[c, :16].astype(np.float64).reshape(4, 4)
+        fx, fy = sc.cams[c, 16:18].astype(np.float64)
+        q = sc.quats[n].astype(np.float64)
+        Rq = Rotation.from_quat([q[1], q[2], q[3], q[0]]).as_matrix()
+        S = Rq @ np.diag(sc.scales[n].astype(np.float64) ** 2) @ Rq.T
+        p = V[:3, :3] @ sc.means[n].astype(np.float64) + V[:3, 3]
+        limx, limy = 1.3 * 0.5 * sc.W / fx, 1.3 * 0.5 * sc.H / fy
+        ux = np.clip(p[0] / p[2], -limx, limx)
+        uy = np.clip(p[1] / p[2], -limy, limy)
+        J = np.array([[fx / p[2], 0, -fx * ux / p[2]], [0, fy / p[2], -fy * uy / p[2]]])
+        S2 = J @ V[:3, :3] @ S @ V[:3, :3].T @ J.T + 0.3 * np.eye(2)
+        Q = np.linalg.inv(S2)
+        np.testing.assert_allclose(pr["screen"][r][2:5], [Q[0, 0], Q[0, 1], Q[1, 1]], rtol=1e-8)
+
+
+def test_visibility_edges():
+    fx = fy = 50.0
+    W = H = 64
+    cam = ident_cam(fx, fy, 32.0, 32.0)
+    s = 0.02
+    # behind the camera, in front but far off-image, and just overlapping the left edge
+    sc = make([[0, 0, -2.0], [10.0, 0, 2.0], [-1.33, 0, 2.0]], [[1, 0, 0, 0]] * 3, [[s, s, s]] * 3,
+              [0.5] * 3, [[0.0, 0.0, 0.0]] * 3, [cam], W, H)
+    pr = orc.project(sc, precision=0)
+    assert pr["nnz"] == 1 and pr["row_gauss"][0] == 2
+
+
+# ---------------------------------------------------------------- compaction and sizes
+def test_compaction_routes_agree_on_random_scenes():
+    for seed in range(6):
+        sc = scenes.random_tiny(seed, N=300 + 37 * seed, W=40, H=32, C=3, sh_degree=1)
+        pr = orc.project(sc)  # raises if the plain and bitmask compactions disagree
+        g = orc.geometry(sc)
+        assert g["n_pad"] % 128 == 0
+        assert pr["block_off"][-1] == pr["nnz"]
+        assert int(np.unpackbits(pr["mask"].view(np.uint8)).sum()) == pr["nnz"]
+
+
+def test_page_buffer_sizes():
+    gd = golden("page_figures.txt")
+    P = gd["pairs_C_times_N"]
+    mib = 1024.0 * 1024.0
+    assert round(P * gd["old_bridge_bytes_per_pair"] / mib, 2) == gd["old_bridge_mib"]
+    per_pair = gd["mask_bytes_per_pair"] + gd["block_count_bytes_per_pair"] + gd["scan_bytes_per_pair"]
+    assert per_pair == 1.0 / 8 + 2 * 4.0 / gd["pairs_per_popcount"]  # one u32 per 128 pairs, twice
+    assert abs(P * per_pair / mib - gd["bitmask_bridge_mib"]) < 0.015
+    # this layout: 5 cameras x 15M Gaussians padded to the 128-pair block
+    sc = make(np.zeros((1, 3)), [[1, 0, 0, 0]], [[1, 1, 1]], [0.5], [[0, 0, 0]],
+              [ident_cam(1, 1, 0, 0)] * 5, 1600, 1067)
+    sc.N = 15_000_000
+    g = orc.geometry(sc)
+    mask_b = g["mask_words"] * 4
+    bc_b = g["mask_blocks"] * 4
+    assert abs((mask_b + 2 * bc_b) / mib - gd["bitmask_bridge_mib"]) < 0.015
+    # AABB rows 16 B -> 8 B at nnz ~ 15.1M
+    nnz = gd["nnz_art_gallery"]
+    assert abs(16 * nnz / mib - gd["aabb_old_mib"]) < 1.0
+    assert abs(8 * nnz / mib - gd["aabb_new_mib"]) < 1.0
+    # 64-bit keys cross 4 GiB at 2^32 / 8 intersections
+    assert abs(2**32 / gd["key_bytes"] - gd["four_gib_crossing_isects"]) < 1e6
+
+
+# ---------------------------------------------------------------- AABB16
+def test_aabb16_contains_float_box_and_step():
+    gd = golden("page_figures.txt")
+    assert round(608 / 65535, 3) == gd["aabb_step_px_608"]
+    assert round(6000 / 65535, 2) == gd["aabb_step_px_6000"]
+    for seed in range(4):
+        sc = scenes.random_tiny(seed, N=400, W=608 if seed % 2 == 0 else 97, H=57, C=2, sh_degree=0)
+        pr = orc.project(sc)
+        box = orc.row_boxes(sc, pr).astype(np.float64)
+        a = pr["aabb"]
+        qx0, qy0 = (a[:, 0] & 0xFFFF).astype(np.int64), (a[:, 0] >> 16).astype(np.int64)
+        qx1, qy1 = (a[:, 1] & 0xFFFF).astype(np.int64), (a[:, 1] >> 16).astype(np.int64)
+        # exact: q*extent/65535 <= v  <=>  q*extent <= v*65535 (both exact in fp64)
+        assert np.all(qx0 * sc.W <= box[:, 0] * 65535.0)
+        assert np.all(qx1 * sc.W >= box[:, 1] * 65535.0)
+        assert np.all(qy0 * sc.H <= box[:, 2] * 65535.0)
+        assert np.all(qy1 * sc.H >= box[:, 3] * 65535.0)
+        # at most one grid step wider per side
+        assert np.all((qx0 + 1) * sc.W > box[:, 0] * 65535.0)
+        assert np.all((qx1 - 1) * sc.W < box[:, 1] * 65535.0)
+
+
+# ---------------------------------------------------------------- intersections, sort, ranges
+def test_intersect_range_form_equals_overlap_test_and_only_grows():
+    for seed in range(4):
+        sc = scenes.random_tiny(seed, N=250, W=80, H=48, C=2, sh_degree=0)
+        pr = orc.project(sc)
+        it = orc.intersect(sc, pr, all_pairs=True)  # raises on any disagreement
+        it2 = orc.intersect(sc, pr, all_pairs=False)
+        np.testing.assert_array_equal(it["keys"], it2["keys"])
+        box = orc.row_boxes(sc, pr).astype(np.float64)
+        per, total = orc.count_tiles(sc, pr["aabb"])
+        assert total == it["n_isects"] == per.sum()
+        # float-box tile count <= decoded-box count <= float-box count widened by one tile per side
+        fx = np.ceil(box[:, 1] / 16) - np.floor(box[:, 0] / 16)
+        fy = np.ceil(box[:, 3] / 16) - np.floor(box[:, 2] / 16)
+        assert np.all(per >= fx * fy)
+        assert np.all(per <= (fx + 2) * (fy + 2))
+
+
+def test_keys_layout_and_sort_against_lexsort():
+    sc = scenes.random_tiny(11, N=300, W=64, H=64, C=3, sh_degree=0)
+    pr = orc.project(sc)
+    it = orc.intersect(sc, pr)
+    g = orc.geometry(sc)
+    k, v = it["keys"], it["vals"]
+    tiles = (k >> np.uint64(32)).astype(np.int64)
+    cams = tiles // g["tiles_per_cam"]
+    np.testing.assert_array_equal(cams, pr["row_cam"][v])
+    depth = (k & np.uint64(0xFFFFFFFF)).astype(np.uint32).view(np.float32)
+    np.testing.assert_array_equal(depth, pr["screen"][v, 9].astype(np.float32))
+    assert np.all(np.diff(v.astype(np.int64)) >= 0)  # written row-major
+    ks, vs = orc.sort(k, v)
+    order = np.lexsort((np.arange(len(k)), k))
+    np.testing.assert_array_equal(ks, k[order])
+    np.testing.assert_array_equal(vs, v[order])
+    off = orc.tile_ranges(ks, g["n_tiles"])
+    np.testing.assert_array_equal(np.diff(off), np.bincount(tiles, minlength=g["n_tiles"]))
+
+
+# ---------------------------------------------------------------- rasterizer
+def render(sc, precision=0):
+    return orc.forward(sc, precision)
+
+
+def test_single_gaussian_closed_form():
+    fx = fy = 50.0
+    W = H = 64
+    z, s, o = 2.0, 0.04, 0.7
+    q = Rotation.from_euler("xyz", [0.3, -0.4, 0.9]).as_quat()  # (x, y, z, w)
+    scl = np.array([0.05, 0.02, 0.03])
+    sc = make([[0.0, 0.0, z]], [[q[3], q[0], q[1], q[2]]], [scl], [o], [[0.0, 0.0, 0.0]],
+              [ident_cam(fx, fy, 32.0, 32.0)], W, H)
+    f = render(sc)
+    Rq = Rotation.from_quat(q).as_matrix()
+    S = Rq @ np.diag(scl ** 2) @ Rq.T
+    S2 = (fx / z) ** 2 * S[:2, :2] + 0.3 * np.eye(2)
+    Q = np.linalg.inv(S2)
+    jj, ii = np.mgrid[0:H, 0:W]
+    d = np.stack([32.0 - (ii + 0.5), 32.0 - (jj + 0.5)], -1)
+    sig = 0.5 * np.einsum("...i,ij,...j->...", d, Q, d)
+    alpha = np.minimum(0.99, o * np.exp(-sig))
+    keep = alpha >= 1.0 / 255.0
+    safe = np.abs(alpha - 1.0 / 255.0) > 1e-6
+    want = np.where(keep, 0.5 * alpha, 0.0)
+    np.testing.assert_allclose(f["img"][0, ..., 0][safe], want[safe], atol=1e-6)
+    np.testing.assert_allclose(f["T"][0][safe], np.where(keep, 1 - alpha, 1.0)[safe], atol=1e-6)
+    # the Gaussian is the only entry of each tile list: last_id = that tile's start
+    g = f["geo"]
+    t = (jj // 16) * g["tiles_x"] + ii // 16
+    np.testing.assert_array_equal(f["last"][0][keep & safe], f["tile_off"][t][keep & safe])
+    assert np.all(f["last"][0][~keep & safe] == -1)
+
+
+def test_weights_telescope_to_one():
+    rng = np.random.default_rng(5)
+    N = 60
+    dc = np.full((N, 1, 3), scenes.SQRT_PI)  # rgb = C0 * sqrt(pi) + 0.5 = 1
+    for prec, tol in ((0, 2e-5), (1, 1e-12)):
+        sc = make(rng.uniform(-0.5, 0.5, (N, 3)) + [0, 0, 3.0], rng.normal(size=(N, 4)),
+                  np.exp(rng.uniform(-3.0, -1.5, (N, 3))), rng.uniform(0.2, 0.95, N), dc,
+                  [ident_cam(40, 40, 24, 20)], 48, 40)
+        f = render(sc, prec)
+        for ch in range(3):
+            np.testing.assert_allclose(f["img"][..., ch] + f["T"], 1.0, atol=tol)
+        assert np.all((f["T"] >= 0) & (f["T"] <= 1))
+        # last_id lies inside the pixel's tile range
+        g = f["geo"]
+        jj, ii = np.mgrid[0:sc.H, 0:sc.W]
+        t = (jj // 16) * g["tiles_x"] + ii // 16
+        lo, hi = f["tile_off"][t], f["tile_off"][t + 1]
+        L = f["last"][0]
+        assert np.all((L == -1) | ((L >= lo) & (L < hi)))
+
+
+def test_clamped_opacity_stops_after_one():
+    # every alpha clamps at 0.99: T = 1 - 0.99f after the first, the second would
+    # take T below 1e-4, so exactly one Gaussian is composited per pixel
+    N = 3
+    sc = make([[0, 0, 2.0], [0.1, 0, 3.0], [0, -0.1, 4.0]], [[1, 0, 0, 0]] * N, [[100.0] * 3] * N,
+              [1.0] * N, [[0.0, 0.0, 0.0]] * N, [ident_cam(20, 20, 16, 16)], 32, 32)
+    f = render(sc)
+    one = np.float32(1.0) - np.float32(0.99)
+    assert np.all(f["T"] == one)
+    g = f["geo"]
+    jj, ii = np.mgrid[0:32, 0:32]
+    t = (jj // 16) * g["tiles_x"] + ii // 16
+    np.testing.assert_array_equal(f["last"][0], f["tile_off"][t])
+    np.testing.assert_allclose(f["img"][0], 0.5 * 0.99, rtol=1e-6)
+
+
+def test_fp32_forward_close_to_fp64():
+    sc = scenes.make_scene(1)
+    a = render(sc, 0)
+    b = render(sc, 1)
+    assert a["proj"]["nnz"] == b["proj"]["nnz"]
+    diff = np.abs(a["img"] - b["img"])
+    assert np.mean(diff < 1e-4) > 0.995
+
+
+# ---------------------------------------------------------------- backward vs finite differences
+def loss(sc, v_img, v_T):
+    f = orc.forward(sc, precision=1)
+    return float(np.sum(f["img"] * v_img) + np.sum(f["T"] * v_T))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_backward_central_differences(seed):
+    sc = scenes.random_tiny(seed, N=5, W=32, H=32, C=2 if seed % 2 else 1, sh_degree=seed % 4,
+                            opacity_range=(0.1, 0.9))
+    # fp64 parameters so the differences are not quantised to fp32
+    for name in ("means", "quats", "scales", "opacities", "sh"):
+        setattr(sc, name, getattr(sc, name).astype(np.float64))
+    rng = np.random.default_rng(seed)
+    v_img = rng.uniform(-1, 1, (sc.C, sc.H, sc.W, 3))
+    v_T = rng.uniform(-1, 1, (sc.C, sc.H, sc.W))
+    r = orc.step(sc, precision=1, v_img=v_img, v_T=v_T)
+    gr = r["grads"]
+    names = {"means": "v_means", "quats": "v_quats", "scales": "v_scales", "opacities": "v_opacities",
+             "sh": "v_sh"}
+    checked = skipped = 0
+    for pname, gname in names.items():
+        arr = getattr(sc, pname)
+        flat = arr.reshape(-1)
+        an = gr[gname].reshape(-1)
+        for i in range(flat.size):
+            x0 = flat[i]
+            vals = []
+            for h in (1e-6, 5e-7):
+                hh = h * max(1.0, abs(x0))
+                flat[i] = x0 + hh
+                lp = loss(sc, v_img, v_T)
+                flat[i] = x0 - hh
+                lm = loss(sc, v_img, v_T)
+                flat[i] = x0
+                vals.append((lp - lm) / (2 * hh))
+            # two step sizes that disagree mean a threshold (1/255, 3-sigma tile edge) was crossed
+            if abs(vals[0] - vals[1]) > 1e-5 * max(1.0, abs(vals[0])):
+                skipped += 1
+                continue
+            checked += 1
+            assert abs(vals[0] - an[i]) <= 1e-4 * max(1.0, abs(an[i])), (pname, i, vals, an[i])
+    assert checked > 10 * skipped

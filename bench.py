@@ -1,0 +1,404 @@
+"""Benchmark of the packed 3DGS forward+backward step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
+
+A step is one pass of the whole path over the workload: ss_project_packed,
+ss_intersect_tiles, ss_sort_isects, ss_rasterize_fwd, ss_rasterize_bwd,
+ss_project_bwd.  The upstream dL/dimage is an input of the step (the L1
+gradient against the workload's seeded target, computed once from the forward
+image before timing; the step's work does not depend on its values).
+
+Default workload: configuration 4 (15M Gaussians x 5 cameras at 1600x1067,
+SH degree 3; 75M pairs, ~15M visible, ~33M tile intersections), the shape of
+the pages' art_gallery measurement.  Inputs (3.5 GB of parameters) are larger
+than L2, so no flush is needed between steps.
+
+Multi-GPU: the step does not shard on one GPU's problem; N ranks run N
+independent replicas (weak scaling), timed on the device, max over ranks.
+
+--impl reference times the CPU oracle (as it stands) on a bounded sample of
+the same workload on the host cores; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd step ms at 1 B200; isects/s; per-stage % of HBM/FP32 roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), sm_max_mhz=float(p.get("sm_max_mhz", 1965.0)), src="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, src="fallback")
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return dict(sm_mhz=float(np.median(sm)) if sm else None, sm_max_mhz=mx, reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+# ---------------------------------------------------------------------------- roofline model
+def stage_model(d, K, nnz, n_isects, passes, n_tiles, work):
+    """Algorithmic bytes (HBM) and FP32 instruction counts per call.
+
+    bytes: every input read once and every output written once, at the
+    stage's own layout; instr: FP32-pipe instructions of the canonical
+    per-item sequences (counted from the source), for the ALU-bound stages.
+    """
+    C, N, W, H = d.C, d.N, d.W, d.H
+    P = C * N
+    X = C * W * H
+    row = 48
+    par = 40  # means 12 + quats 16 + scales 12
+    shb = 12 * K
+    m = {}
+    m["project_packed"] = dict(bytes=par * N + P / 8 + P / 32 + P / 16 + (par + 4 + shb) * N + (row + 8) * nnz,
+                               instr=P * 140.0 + nnz * 160.0)
+    m["intersect_tiles"] = dict(bytes=8 * nnz * 2 + 8 * nnz + 4 * nnz + 12 * n_isects, instr=0.0)
+    m["sort_isects"] = dict(bytes=n_isects * (8 + 24) * passes + 8 * (n_tiles + 1), instr=0.0)
+    m["rasterize_fwd"] = dict(bytes=n_isects * (4 + row) + X * 20 + 8 * (n_tiles + 1),
+                              instr=work["evals"] * 12.0 + work["exps"] * 22.0 + work["comps"] * 9.0)
+    m["rasterize_bwd"] = dict(bytes=n_isects * (4 + row) + X * 24 + nnz * row * 2,
+                              instr=work["bwd_evals"] * 12.0 + work["bwd_exps"] * 22.0 + work["comps"] * 60.0)
+    m["project_bwd"] = dict(bytes=(par + shb) * N + row * nnz + P / 8 + P / 16 + (par + 4 + shb) * N,
+                            instr=nnz * 700.0)
+    return m
+
+
+def fp32_peak_instr_per_s(sm_mhz: float) -> float:
+    # 148 SMs x 128 FP32 lanes, one instruction per lane per clock
+    return 148 * 128 * sm_mhz * 1e6
+
+
+# ---------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from gaussian_splatting_differentiable_packed_b200 import scenes, ss
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    dev = torch.device("cuda", local)
+
+    sc = scenes.make_scene(args.config, n=args.n)
+    d = ss.scene_dims(sc)
+    inputs = ss.scene_tensors(sc, dev)
+    step = ss.PackedStep(d, dev)
+    step.forward(*inputs)
+    torch.cuda.synchronize()
+    # capacities with headroom, then the upstream gradient from this forward
+    step._rows(int(step.nnz * 1.05) + 1)
+    step._isects(int(step.n_isects * 1.05) + 1)
+    img = step.forward(*inputs)
+    if sc.upstream == "l1":
+        target = torch.from_numpy(sc.target).to(dev)
+        v_img = (torch.sign(img - target) * sc.l1_scale).contiguous()
+        del target
+    else:
+        v_img = torch.from_numpy(sc.v_img).to(dev)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+
+    names = ["project_packed", "intersect_tiles", "sort_isects", "rasterize_fwd", "rasterize_bwd", "project_bwd"]
+
+    def run_step(ev=None):
+        if ev is not None:
+            ev[0].record(st)
+        step.forward(*inputs, stream=None) if ev is None else _timed_forward(ev)
+        if ev is None:
+            step.backward(v_img)
+        else:
+            ss.ss_rasterize_bwd(d, step.screen, step.vals, step.tile_off, step.T, step.last, v_img, None,
+                                step.v_screen, step.nnz)
+            ev[5].record(st)
+            ss.ss_project_bwd(d, *inputs, step.mask, step.block_off, step.v_screen, step.v_means, step.v_quats,
+                              step.v_scales, step.v_opacities, step.v_sh)
+            ev[6].record(st)
+
+    def _timed_forward(ev):
+        cams, means, quats, scales, opac, sh = inputs
+        nnz = ss.ss_project_packed(d, cams, means, quats, scales, opac, sh, step.mask, step.block_count,
+                                   step.block_off, step.screen, step.aabb16, step.cap_rows, step.temp_project)
+        ev[1].record(st)
+        n = ss.ss_intersect_tiles(d, step.screen, step.aabb16, step.block_off, nnz, step.isect_off, step.keys_a,
+                                  step.vals_a, step.cap_isects, step.temp_isect)
+        ev[2].record(st)
+        in_b = ss.ss_sort_isects(d, step.keys_a, step.vals_a, step.keys_b, step.vals_b, n, step.temp_sort,
+                                 step.tile_off)
+        step.vals = step.vals_b if in_b else step.vals_a
+        ev[3].record(st)
+        ss.ss_rasterize_fwd(d, step.screen, step.vals, step.tile_off, step.img, step.T, step.last)
+        ev[4].record(st)
+        step.nnz, step.n_isects = nnz, n
+
+    for _ in range(args.warmup):
+        step.forward(*inputs)
+        step.backward(v_img)
+    torch.cuda.synchronize()
+
+    # ---- headline: K whole steps, device-timed, max over ranks
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for _ in range(args.steps):
+        step.forward(*inputs)
+        step.backward(v_img)
+    t1.record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    # ---- per-stage times (separate pass, events between the calls)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        run_step(evs[k])
+    torch.cuda.synchronize()
+    stage_ms = {nm: float(np.mean([evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)]))
+                for i, nm in enumerate(names)}
+
+    # ---- work counts for the ALU roofline (outside every timed region)
+    work = ss.raster_work(d, step) if hasattr(ss, "raster_work") else dict(
+        evals=0.0, exps=0.0, comps=0.0, bwd_evals=0.0, bwd_exps=0.0)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.cpu().pin_memory() for t in inputs]
+        host_vimg = v_img.cpu().pin_memory()
+        host_out = {k: torch.empty(tuple(getattr(step, k).shape), dtype=torch.float32).pin_memory()
+                    for k in ("v_means", "v_quats", "v_scales", "v_opacities", "v_sh")}
+        dev_in = [torch.empty_like(t) for t in inputs]
+        dev_vimg = torch.empty_like(v_img)
+        h2d = sum(t.numel() * 4 for t in host_in) + host_vimg.numel() * 4
+        d2h = sum(t.numel() * 4 for t in host_out.values())
+        ke = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            for a, b in zip(dev_in, host_in):
+                a.copy_(b, non_blocking=True)
+            dev_vimg.copy_(host_vimg, non_blocking=True)
+            step.forward(*dev_in)
+            g = step.backward(dev_vimg)
+            for k, h in host_out.items():
+                h.copy_(g[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(st)
+        for _ in range(ke):
+            e2e_step()
+        a1.record(st)
+        torch.cuda.synchronize()
+        e_ms = a0.elapsed_time(a1) / ke
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = dict(value=world * step.n_isects / (e_ms / 1e3), unit="isects/s", ms_per_step=e_ms,
+                   h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h))
+
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks = load_peaks()
+    passes = ss.sort_passes(d)
+    model = stage_model(d, (d.sh_degree + 1) ** 2, step.nnz, step.n_isects, passes, ss.size(d, ss.SIZE_N_TILES),
+                        work)
+    sm_mhz = clocks["sm_mhz"] or peaks["sm_max_mhz"]
+    stages = {}
+    for nm in names:
+        t = stage_ms[nm] / 1e3
+        b = model[nm]["bytes"]
+        ins = model[nm]["instr"]
+        hbm = b / t / 1e9
+        alu = ins / t
+        f_hbm = hbm / peaks["hbm_gbs"]
+        f_alu = alu / fp32_peak_instr_per_s(sm_mhz) if ins else 0.0
+        stages[nm] = dict(ms=round(stage_ms[nm], 4), hbm_gbs=round(hbm, 1), hbm_frac=round(f_hbm, 4),
+                          alu_frac=round(f_alu, 4), bound="alu" if f_alu > f_hbm else "hbm")
+    dom = max(names, key=lambda k: stage_ms[k])
+    sd = stages[dom]
+    if sd["bound"] == "hbm":
+        roof = dict(bound="hbm", achieved=sd["hbm_gbs"], peak=peaks["hbm_gbs"], unit="GB/s", frac=sd["hbm_frac"],
+                    traffic=None, kernel=dom, peak_source=peaks["src"])
+    else:
+        ach = model[dom]["instr"] / (stage_ms[dom] / 1e3) / 1e12
+        pk = fp32_peak_instr_per_s(sm_mhz) / 1e12
+        roof = dict(bound="alu", achieved=round(ach, 3), peak=round(pk, 3), unit="T FP32 instr/s",
+                    frac=round(ach / pk, 4), traffic=None, kernel=dom,
+                    peak_source=f"148 SMs x 128 FP32 lanes x {sm_mhz:.0f} MHz (median SM clock under load)")
+    launches = ss.launches_per_step(d, step.nnz, step.n_isects) * args.steps
+    out = dict(metric=METRIC, value=world * step.n_isects / (ms / 1e3), unit="isects/s", n_gpus=world,
+               steps=args.steps, warmup=args.warmup, ms_per_step=round(ms, 4), higher_is_better=True,
+               scaling="weak", vs_baseline=None, dtype="f32", data="synthetic",
+               config=dict(workload=f"config {args.config}: {sc.name}", C=d.C, N=d.N, W=d.W, H=d.H,
+                           sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
+                           sort_passes=passes, l2="inputs larger than L2 (3.5 GB parameters), no flush",
+                           parallelism=f"replicas x{world}"),
+               pairs_per_s=world * d.C * d.N / (ms / 1e3), stages=stages, roofline=roof, clocks=clocks,
+               e2e=e2e, gpu_launches=launches)
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_sample)
+    print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_sample(config: int, n: int):
+    from gaussian_splatting_differentiable_packed_b200 import scenes
+    return scenes.make_scene(config, n=n)
+
+
+def cpu_baseline(config: int, n_sample: int, repeats: int = 1):
+    from oracle import oracle as orc
+    cores = os.cpu_count() or 1
+    sc = oracle_sample(config, n_sample)
+    t = time.perf_counter()
+    isects = 0
+    for _ in range(repeats):
+        r = orc.step(sc, precision=0, nthreads=cores)
+        isects += r["isect"]["n_isects"]
+    dt = time.perf_counter() - t
+    return dict(value=isects / dt, unit="isects/s", cores=cores, kind="oracle",
+                sample=f"config {config} distributions and cameras with N={n_sample} Gaussians "
+                       f"({r['isect']['n_isects']} intersections, full image size), {repeats} step(s) "
+                       f"in {dt:.1f} s")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    cores = os.cpu_count() or 1
+    sc = oracle_sample(args.config, args.cpu_sample)
+    for _ in range(min(args.warmup, 1)):
+        orc.step(sc, precision=0, nthreads=cores)
+    t = time.perf_counter()
+    isects = 0
+    for _ in range(args.steps):
+        r = orc.step(sc, precision=0, nthreads=cores)
+        isects += r["isect"]["n_isects"]
+    dt = time.perf_counter() - t
+    v = isects / dt
+    out = dict(impl="reference", metric=METRIC, value=v, unit="isects/s", n_gpus=world, steps=args.steps,
+               warmup=args.warmup, ms_per_step=1e3 * dt / args.steps, higher_is_better=True, scaling="weak",
+               vs_baseline=None, dtype="f32", data="synthetic",
+               config=dict(workload=f"config {args.config} (bounded sample, N={args.cpu_sample})"),
+               cpu_baseline=dict(value=v, unit="isects/s", cores=cores, kind="oracle",
+                                 sample=f"config {args.config} with N={args.cpu_sample} Gaussians per step"),
+               e2e=dict(value=v, unit="isects/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--n", type=int, default=None, help="override the Gaussian count (profiling captures)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample", type=int, default=300_000)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

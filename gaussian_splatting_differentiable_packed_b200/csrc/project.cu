@@ -1,0 +1,198 @@
+// Packed projection ("Spirula Studio VRAM deep-dive", section "bitmask
+// compaction"; "16-bit packed AABB"; projection chain from the "Spirula Studio
+// backward pass" page, section 5).
+//
+// Pass 1 (k_project_mask): one thread per Gaussian, 128 threads per CTA, loops
+// over the cameras so each Gaussian's parameters are read once.  For camera c
+// the CTA's 128 pairs are bits [c*n_pad + 128*blk, +128) of the mask: each warp
+// writes its ballot word and the CTA writes one popcount (block_count).
+// Scan: block_off = exclusive scan of block_count (int64), nnz at the end.
+// Pass 2 (k_project_rows): same geometry; a thread whose bit is set re-projects
+// its pair and writes row = block_off[block] + popc(earlier words of the block)
+// + popc(bits below it in its word).
+#include "ss_common.cuh"
+#include "ss_math.cuh"
+
+namespace ss {
+
+constexpr int kCamChunk = 32;
+
+struct GaussIn {
+  float mx, my, mz;
+  Cov3 S;
+};
+
+__device__ __forceinline__ GaussIn load_gauss(const float* means, const float* quats, const float* scales, int64_t n) {
+  GaussIn g;
+  g.mx = means[3 * n]; g.my = means[3 * n + 1]; g.mz = means[3 * n + 2];
+  float4 q = reinterpret_cast<const float4*>(quats)[n];
+  QuatRot r = quat_rot(q.x, q.y, q.z, q.w);
+  g.S = cov3(r, scales[3 * n], scales[3 * n + 1], scales[3 * n + 2]);
+  return g;
+}
+
+__global__ __launch_bounds__(kBlock) void k_project_mask(Geo g, const float* __restrict__ cams,
+                                                         const float* __restrict__ means,
+                                                         const float* __restrict__ quats,
+                                                         const float* __restrict__ scales, uint32_t* __restrict__ mask,
+                                                         uint32_t* __restrict__ block_count) {
+  __shared__ Cam scam[kCamChunk];
+  __shared__ uint32_t wcnt[kCamChunk][kBlock / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t blk = blockIdx.x;
+  const int64_t n = blk * kBlock + threadIdx.x;
+  const bool valid = n < g.N;
+  GaussIn gi{};
+  if (valid) gi = load_gauss(means, quats, scales, n);
+  for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
+    const int nc = min(kCamChunk, g.C - c0);
+    __syncthreads();
+    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
+    __syncthreads();
+    for (int cc = 0; cc < nc; ++cc) {
+      bool vis = false;
+      if (valid) {
+        const Cam& k = scam[cc];
+        Proj P;
+        cam_point(k, gi.mx, gi.my, gi.mz, P.px, P.py, P.pz);
+        if (g.near_plane < P.pz && P.pz < g.far_plane) {
+          project_rest(k, gi.S, g.W, g.H, P);
+          vis = P.vis;
+        }
+      }
+      const uint32_t word = __ballot_sync(0xffffffffu, vis);
+      if (lane == 0) {
+        const int64_t c = c0 + cc;
+        mask[(c * g.n_pad + blk * kBlock) / 32 + warp] = word;
+        wcnt[cc][warp] = __popc(word);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < nc) {
+      const int64_t c = c0 + threadIdx.x;
+      uint32_t s = 0;
+#pragma unroll
+      for (int w = 0; w < kBlock / 32; ++w) s += wcnt[threadIdx.x][w];
+      block_count[c * g.blocks_per_cam + blk] = s;
+    }
+  }
+}
+
+__global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __restrict__ cams,
+                                                         const float* __restrict__ means,
+                                                         const float* __restrict__ quats,
+                                                         const float* __restrict__ scales,
+                                                         const float* __restrict__ opacities,
+                                                         const float* __restrict__ sh,
+                                                         const uint32_t* __restrict__ mask,
+                                                         const int64_t* __restrict__ block_off,
+                                                         float* __restrict__ screen, uint32_t* __restrict__ aabb16) {
+  __shared__ Cam scam[kCamChunk];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t blk = blockIdx.x;
+  const int64_t n = blk * kBlock + threadIdx.x;
+  const bool valid = n < g.N;
+  GaussIn gi{};
+  float opac = 0.0f;
+  if (valid) {
+    gi = load_gauss(means, quats, scales, n);
+    opac = opacities[n];
+  }
+  const float* shn = sh + (int64_t)g.K * 3 * (valid ? n : 0);
+  for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
+    const int nc = min(kCamChunk, g.C - c0);
+    __syncthreads();
+    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
+    __syncthreads();
+    for (int cc = 0; cc < nc; ++cc) {
+      const int64_t c = c0 + cc;
+      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
+      const uint32_t word = mask[wbase + warp];
+      if (!((word >> lane) & 1u)) continue;
+      int64_t row = block_off[c * g.blocks_per_cam + blk];
+      for (int w = 0; w < warp; ++w) row += __popc(mask[wbase + w]);
+      row += __popc(word & ((1u << lane) - 1u));
+      const Cam& k = scam[cc];
+      Proj P;
+      cam_point(k, gi.mx, gi.my, gi.mz, P.px, P.py, P.pz);
+      project_rest(k, gi.S, g.W, g.H, P);
+      const float idet = div_(1.0f, P.det);
+      const float ca = mul(P.c, idet), cb = -mul(P.b, idet), cc2 = mul(P.a, idet);
+      // colour
+      float b[16];
+      float X = 0.0f, Y = 0.0f, Z = 0.0f, il;
+      if (g.deg > 0) view_dir(k, gi.mx, gi.my, gi.mz, X, Y, Z, il);
+      sh_basis(g.deg, X, Y, Z, b);
+      float rgb[3];
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) {
+        float acc = mul(shn[ch], b[0]);
+        for (int kk = 1; kk < g.K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], b[kk]));
+        rgb[ch] = fmaxf(add(acc, 0.5f), 0.0f);
+      }
+      float4* out = reinterpret_cast<float4*>(screen + row * kRowF);
+      out[0] = make_float4(P.mx, P.my, ca, cb);
+      out[1] = make_float4(cc2, opac, rgb[0], rgb[1]);
+      out[2] = make_float4(rgb[2], P.pz, 0.0f, 0.0f);
+      const float x0 = fmaxf(sub(P.mx, P.r), 0.0f), x1 = fminf(add(P.mx, P.r), (float)g.W);
+      const float y0 = fmaxf(sub(P.my, P.r), 0.0f), y1 = fminf(add(P.my, P.r), (float)g.H);
+      uint2 q;
+      q.x = q16_floor(x0, g.W) | (q16_floor(y0, g.H) << 16);
+      q.y = q16_ceil(x1, g.W) | (q16_ceil(y1, g.H) << 16);
+      reinterpret_cast<uint2*>(aabb16)[row] = q;
+    }
+  }
+}
+
+}  // namespace ss
+
+using namespace ss;
+
+extern "C" ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float* means,
+                                       const float* quats, const float* scales, const float* opacities,
+                                       const float* sh, uint32_t* mask, uint32_t* block_count, int64_t* block_off,
+                                       float* screen, uint32_t* aabb16, int64_t cap_rows, void* temp,
+                                       size_t temp_bytes, int64_t* nnz_out, void* stream) {
+  if (!dims_ok(dims)) return invalid("dims");
+  if (!nnz_out) return invalid("nnz_out is NULL");
+  const Geo g = geometry(*dims);
+  cudaStream_t st = as_stream(stream);
+  if (!block_off) return invalid("block_off is NULL");
+  if (g.N == 0) {
+    ss_status s = cuda_status(cudaMemsetAsync(block_off, 0, sizeof(int64_t), st), "memset");
+    if (s) return s;
+    *nnz_out = 0;
+    return SS_OK;
+  }
+  if (!cams || !means || !quats || !scales || !mask || !block_count) return invalid("null input");
+  if (((uintptr_t)quats & 15) != 0) return invalid("quats must be 16-byte aligned");
+  if (!temp || temp_bytes < ss_workspace_bytes(dims, SS_WS_PROJECT, 0)) return invalid("temp too small");
+  const unsigned grid = (unsigned)g.blocks_per_cam;
+  k_project_mask<<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, mask, block_count);
+  ss_status s = cuda_status(cudaGetLastError(), "project pass 1");
+  if (s) return s;
+  ScanSrc src{};
+  src.kind = SCAN_U32;
+  src.u32 = block_count;
+  s = scan_phase1(src, g.mask_blocks, temp, block_off + g.mask_blocks, st);
+  if (s) return s;
+  s = scan_phase2<int64_t>(src, g.mask_blocks, temp, block_off, st);
+  if (s) return s;
+  int64_t nnz = 0;
+  s = cuda_status(cudaMemcpyAsync(&nnz, block_off + g.mask_blocks, sizeof(int64_t), cudaMemcpyDeviceToHost, st),
+                  "copy nnz");
+  if (s) return s;
+  s = cuda_status(cudaStreamSynchronize(st), "project pass 1 / scan");
+  if (s) return s;
+  *nnz_out = nnz;
+  if (!screen) return SS_OK;
+  if (nnz > cap_rows) {
+    set_error("ss_project_packed: nnz exceeds cap_rows");
+    return SS_ERR_CAPACITY;
+  }
+  if (!opacities || !sh || !aabb16) return invalid("null row input/output");
+  if (((uintptr_t)screen & 15) != 0 || ((uintptr_t)aabb16 & 7) != 0) return invalid("row buffers misaligned");
+  k_project_rows<<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, opacities, sh, mask, block_off, screen,
+                                          aabb16);
+  return cuda_status(cudaGetLastError(), "project pass 2");
+}

@@ -1,0 +1,278 @@
+// Projection backward ("Spirula Studio backward pass", section 5: each
+// Gaussian's screen-space gradient goes back through the intrinsics and
+// extrinsics to its six attributes: means, rotation, scale, opacity, DC and
+// higher SH coefficients).
+//
+// One thread per Gaussian, 128 per CTA, looping over the cameras exactly as
+// the packed projection does; a set mask bit gives the row by the same
+// popcount arithmetic, so no (camera, Gaussian) ids are stored.  The gradient
+// of the 3D covariance is summed over cameras first and taken through
+// Sigma = M M^T, the scale and the quaternion once per Gaussian.
+// Deterministic: no atomics.  Decisions that gate gradients (the Jacobian's
+// off-axis clamp, the colour clamp) are re-taken with the forward's
+// canonical arithmetic.
+#include "ss_common.cuh"
+#include "ss_math.cuh"
+
+namespace ss {
+
+constexpr int kCamChunkB = 32;
+
+template <int DEG>
+__device__ __forceinline__ void sh_grads(float X, float Y, float Z, const float* __restrict__ shn, const float vr[3],
+                                         const bool cl[3], float* gsh, float vdir[3]) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  float b[16];
+  sh_basis(DEG, X, Y, Z, b);
+  // d b_k / d(X, Y, Z)
+  float dX[16], dY[16], dZ[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) dX[k] = dY[k] = dZ[k] = 0.0f;
+  if (DEG >= 1) {
+    dY[1] = -SS_SH_C1; dZ[2] = SS_SH_C1; dX[3] = -SS_SH_C1;
+  }
+  if (DEG >= 2) {
+    dX[4] = SS_SH_C2A * Y; dY[4] = SS_SH_C2A * X;
+    dY[5] = -SS_SH_C2A * Z; dZ[5] = -SS_SH_C2A * Y;
+    dX[6] = -2.0f * SS_SH_C2C * X; dY[6] = -2.0f * SS_SH_C2C * Y; dZ[6] = 4.0f * SS_SH_C2C * Z;
+    dX[7] = -SS_SH_C2A * Z; dZ[7] = -SS_SH_C2A * X;
+    dX[8] = 2.0f * SS_SH_C2E * X; dY[8] = -2.0f * SS_SH_C2E * Y;
+  }
+  if (DEG >= 3) {
+    const float XX = X * X, YY = Y * Y, ZZ = Z * Z;
+    dX[9] = -SS_SH_C3A * 6.0f * X * Y; dY[9] = -SS_SH_C3A * (3.0f * XX - 3.0f * YY);
+    dX[10] = SS_SH_C3B * Y * Z; dY[10] = SS_SH_C3B * X * Z; dZ[10] = SS_SH_C3B * X * Y;
+    dX[11] = 2.0f * SS_SH_C3C * X * Y; dY[11] = -SS_SH_C3C * (4.0f * ZZ - XX - 3.0f * YY);
+    dZ[11] = -8.0f * SS_SH_C3C * Y * Z;
+    dX[12] = -6.0f * SS_SH_C3D * X * Z; dY[12] = -6.0f * SS_SH_C3D * Y * Z;
+    dZ[12] = SS_SH_C3D * (6.0f * ZZ - 3.0f * XX - 3.0f * YY);
+    dX[13] = -SS_SH_C3C * (4.0f * ZZ - 3.0f * XX - YY); dY[13] = 2.0f * SS_SH_C3C * X * Y;
+    dZ[13] = -8.0f * SS_SH_C3C * X * Z;
+    dX[14] = 2.0f * SS_SH_C3F * X * Z; dY[14] = -2.0f * SS_SH_C3F * Y * Z; dZ[14] = SS_SH_C3F * (XX - YY);
+    dX[15] = -SS_SH_C3A * (3.0f * XX - 3.0f * YY); dY[15] = SS_SH_C3A * 6.0f * X * Y;
+  }
+#pragma unroll
+  for (int ch = 0; ch < 3; ++ch) {
+    if (cl[ch]) continue;
+    const float v = vr[ch];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      gsh[3 * k + ch] += b[k] * v;
+      if (DEG >= 1) {
+        const float sv = shn[3 * k + ch] * v;
+        vdir[0] += sv * dX[k];
+        vdir[1] += sv * dY[k];
+        vdir[2] += sv * dZ[k];
+      }
+    }
+  }
+}
+
+template <int DEG>
+__global__ __launch_bounds__(kBlock) void k_project_bwd(Geo g, const float* __restrict__ cams,
+                                                        const float* __restrict__ means,
+                                                        const float* __restrict__ quats,
+                                                        const float* __restrict__ scales,
+                                                        const float* __restrict__ sh,
+                                                        const uint32_t* __restrict__ mask,
+                                                        const int64_t* __restrict__ block_off,
+                                                        const float* __restrict__ v_screen, float* __restrict__ v_means,
+                                                        float* __restrict__ v_quats, float* __restrict__ v_scales,
+                                                        float* __restrict__ v_opac, float* __restrict__ v_sh) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  __shared__ Cam scam[kCamChunkB];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t blk = blockIdx.x;
+  const int64_t n = blk * kBlock + threadIdx.x;
+  const bool valid = n < g.N;
+  const int64_t nn = valid ? n : 0;
+  const float mx = means[3 * nn], my = means[3 * nn + 1], mz = means[3 * nn + 2];
+  const float4 q4 = reinterpret_cast<const float4*>(quats)[nn];
+  const QuatRot qr = quat_rot(q4.x, q4.y, q4.z, q4.w);
+  const float s0 = scales[3 * nn], s1 = scales[3 * nn + 1], s2 = scales[3 * nn + 2];
+  const Cov3 S = cov3(qr, s0, s1, s2);
+  const float* shn = sh + (int64_t)K * 3 * nn;
+  float gmu[3] = {0.f, 0.f, 0.f}, go = 0.f;
+  float gS[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // dL/dSigma, full-matrix convention (00 01 02 11 12 22)
+  float gsh[3 * K];
+#pragma unroll
+  for (int q = 0; q < 3 * K; ++q) gsh[q] = 0.f;
+  for (int c0 = 0; c0 < g.C; c0 += kCamChunkB) {
+    const int nc = min(kCamChunkB, g.C - c0);
+    __syncthreads();
+    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
+    __syncthreads();
+    if (!valid) continue;
+    for (int cc = 0; cc < nc; ++cc) {
+      const int64_t c = c0 + cc;
+      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
+      const uint32_t word = mask[wbase + warp];
+      if (!((word >> lane) & 1u)) continue;
+      int64_t row = block_off[c * g.blocks_per_cam + blk];
+      for (int w = 0; w < warp; ++w) row += __popc(mask[wbase + w]);
+      row += __popc(word & ((1u << lane) - 1u));
+      const float4* vrp = reinterpret_cast<const float4*>(v_screen + row * kRowF);
+      const float4 v0 = vrp[0], v1 = vrp[1], v2 = vrp[2];
+      const Cam& k = scam[cc];
+      Proj P;
+      cam_point(k, mx, my, mz, P.px, P.py, P.pz);
+      project_rest(k, S, g.W, g.H, P);
+      // conic (c, -b, a)/det -> dilated covariance (a, b, c)
+      const float a = P.a, b = P.b, cq = P.c;
+      const float id = 1.0f / P.det, id2 = id * id;
+      const float vca = v0.z, vcb = v0.w, vcc = v1.x;
+      const float va = (-vca * cq * cq + vcb * b * cq - vcc * b * b) * id2;
+      const float vb = (2.0f * vca * b * cq - vcb * (a * cq + b * b) + 2.0f * vcc * a * b) * id2;
+      const float vc = (-vca * b * b + vcb * a * b - vcc * a * a) * id2;
+      const float hb = 0.5f * vb;
+      const float* T = P.T;
+      // TS = T Sigma (2x3)
+      const float Sm[3][3] = {{S.s00, S.s01, S.s02}, {S.s01, S.s11, S.s12}, {S.s02, S.s12, S.s22}};
+      float TS[2][3];
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int m = 0; m < 3; ++m) TS[r][m] = T[3 * r] * Sm[0][m] + T[3 * r + 1] * Sm[1][m] + T[3 * r + 2] * Sm[2][m];
+      // dL/dT = 2 V2 T Sigma
+      float GT[2][3];
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        GT[0][m] = 2.0f * (va * TS[0][m] + hb * TS[1][m]);
+        GT[1][m] = 2.0f * (hb * TS[0][m] + vc * TS[1][m]);
+      }
+      // dL/dSigma += T^T V2 T
+      {
+        float VT[2][3];
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          VT[0][m] = va * T[m] + hb * T[3 + m];
+          VT[1][m] = hb * T[m] + vc * T[3 + m];
+        }
+        gS[0] += T[0] * VT[0][0] + T[3] * VT[1][0];
+        gS[1] += T[0] * VT[0][1] + T[3] * VT[1][1];
+        gS[2] += T[0] * VT[0][2] + T[3] * VT[1][2];
+        gS[3] += T[1] * VT[0][1] + T[4] * VT[1][1];
+        gS[4] += T[1] * VT[0][2] + T[4] * VT[1][2];
+        gS[5] += T[2] * VT[0][2] + T[5] * VT[1][2];
+      }
+      // T = J R -> dL/dJ = dL/dT R^T (entries 00, 02, 11, 12)
+      const float* R = k.R;
+      const float gj00 = GT[0][0] * R[0] + GT[0][1] * R[1] + GT[0][2] * R[2];
+      const float gj02 = GT[0][0] * R[6] + GT[0][1] * R[7] + GT[0][2] * R[8];
+      const float gj11 = GT[1][0] * R[3] + GT[1][1] * R[4] + GT[1][2] * R[5];
+      const float gj12 = GT[1][0] * R[6] + GT[1][1] * R[7] + GT[1][2] * R[8];
+      const float iz = 1.0f / P.pz, iz2 = iz * iz;
+      float gx = 0.f, gy = 0.f;
+      float gz = -k.fx * iz2 * gj00 + k.fx * P.ux * iz2 * gj02 - k.fy * iz2 * gj11 + k.fy * P.uy * iz2 * gj12;
+      const float gux = -k.fx * iz * gj02, guy = -k.fy * iz * gj12;
+      if (!(P.u < -k.limx || P.u > k.limx)) { gx += gux * iz; gz -= gux * P.px * iz2; }
+      if (!(P.v < -k.limy || P.v > k.limy)) { gy += guy * iz; gz -= guy * P.py * iz2; }
+      const float vmx = v0.x, vmy = v0.y;
+      gx += vmx * k.fx * iz; gz -= vmx * k.fx * P.px * iz2;
+      gy += vmy * k.fy * iz; gz -= vmy * k.fy * P.py * iz2;
+      gz += v2.y;  // depth
+      gmu[0] += R[0] * gx + R[3] * gy + R[6] * gz;
+      gmu[1] += R[1] * gx + R[4] * gy + R[7] * gz;
+      gmu[2] += R[2] * gx + R[5] * gy + R[8] * gz;
+      go += v1.y;
+      // colour: clamp decisions in the forward's canonical arithmetic
+      float X = 0.f, Y = 0.f, Z = 0.f, il = 0.f;
+      if (DEG > 0) view_dir(k, mx, my, mz, X, Y, Z, il);
+      bool cl[3];
+      {
+        float bb[16];
+        sh_basis(DEG, X, Y, Z, bb);
+#pragma unroll
+        for (int ch = 0; ch < 3; ++ch) {
+          float acc = mul(shn[ch], bb[0]);
+#pragma unroll
+          for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], bb[kk]));
+          cl[ch] = !(add(acc, 0.5f) >= 0.0f);
+        }
+      }
+      const float vr[3] = {v1.z, v1.w, v2.x};
+      float vdir[3] = {0.f, 0.f, 0.f};
+      sh_grads<DEG>(X, Y, Z, shn, vr, cl, gsh, vdir);
+      if (DEG > 0) {
+        const float dd = X * vdir[0] + Y * vdir[1] + Z * vdir[2];
+        gmu[0] += (vdir[0] - X * dd) * il;
+        gmu[1] += (vdir[1] - Y * dd) * il;
+        gmu[2] += (vdir[2] - Z * dd) * il;
+      }
+    }
+  }
+  if (!valid) return;
+  // Sigma = M M^T: dL/dM = 2 gS M, M = R_q diag(s)
+  const float Gs[3][3] = {{gS[0], gS[1], gS[2]}, {gS[1], gS[3], gS[4]}, {gS[2], gS[4], gS[5]}};
+  const float sv[3] = {s0, s1, s2};
+  float M[9];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 3; ++jj) M[3 * i + jj] = qr.R[3 * i + jj] * sv[jj];
+  float gsc[3] = {0.f, 0.f, 0.f}, GR[9];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 3; ++jj) {
+      const float gm = 2.0f * (Gs[i][0] * M[jj] + Gs[i][1] * M[3 + jj] + Gs[i][2] * M[6 + jj]);
+      gsc[jj] += gm * qr.R[3 * i + jj];
+      GR[3 * i + jj] = gm * sv[jj];
+    }
+  const float w = qr.w, x = qr.x, y = qr.y, z = qr.z;
+  float vw = 0.f, vx = 0.f, vy = 0.f, vz = 0.f;
+  vy += -4.f * y * GR[0]; vz += -4.f * z * GR[0];
+  vw += -2.f * z * GR[1]; vx += 2.f * y * GR[1]; vy += 2.f * x * GR[1]; vz += -2.f * w * GR[1];
+  vw += 2.f * y * GR[2]; vx += 2.f * z * GR[2]; vy += 2.f * w * GR[2]; vz += 2.f * x * GR[2];
+  vw += 2.f * z * GR[3]; vx += 2.f * y * GR[3]; vy += 2.f * x * GR[3]; vz += 2.f * w * GR[3];
+  vx += -4.f * x * GR[4]; vz += -4.f * z * GR[4];
+  vw += -2.f * x * GR[5]; vx += -2.f * w * GR[5]; vy += 2.f * z * GR[5]; vz += 2.f * y * GR[5];
+  vw += -2.f * y * GR[6]; vx += 2.f * z * GR[6]; vy += -2.f * w * GR[6]; vz += 2.f * x * GR[6];
+  vw += 2.f * x * GR[7]; vx += 2.f * w * GR[7]; vy += 2.f * z * GR[7]; vz += 2.f * y * GR[7];
+  vx += -4.f * x * GR[8]; vy += -4.f * y * GR[8];
+  const float dq = w * vw + x * vx + y * vy + z * vz;
+  v_means[3 * n] = gmu[0];
+  v_means[3 * n + 1] = gmu[1];
+  v_means[3 * n + 2] = gmu[2];
+  reinterpret_cast<float4*>(v_quats)[n] =
+      make_float4((vw - w * dq) * qr.inv, (vx - x * dq) * qr.inv, (vy - y * dq) * qr.inv, (vz - z * dq) * qr.inv);
+  v_scales[3 * n] = gsc[0];
+  v_scales[3 * n + 1] = gsc[1];
+  v_scales[3 * n + 2] = gsc[2];
+  v_opac[n] = go;
+  float* o = v_sh + (int64_t)K * 3 * n;
+#pragma unroll
+  for (int q = 0; q < 3 * K; ++q) o[q] = gsh[q];
+}
+
+}  // namespace ss
+
+using namespace ss;
+
+extern "C" ss_status ss_project_bwd(const ss_dims* dims, const float* cams, const float* means, const float* quats,
+                                    const float* scales, const float* opacities, const float* sh,
+                                    const uint32_t* mask, const int64_t* block_off, const float* v_screen,
+                                    float* v_means, float* v_quats, float* v_scales, float* v_opacities, float* v_sh,
+                                    void* stream) {
+  if (!dims_ok(dims)) return invalid("dims");
+  const Geo g = geometry(*dims);
+  if (g.N == 0) return SS_OK;
+  if (!cams || !means || !quats || !scales || !sh || !mask || !block_off || !v_screen) return invalid("null input");
+  if (!v_means || !v_quats || !v_scales || !v_opacities || !v_sh) return invalid("null output");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)v_quats & 15) || ((uintptr_t)v_screen & 15))
+    return invalid("quats, v_quats and v_screen must be 16-byte aligned");
+  (void)opacities;
+  cudaStream_t st = as_stream(stream);
+  const unsigned grid = (unsigned)g.blocks_per_cam;
+  switch (g.deg) {
+    case 0: k_project_bwd<0><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                                      v_means, v_quats, v_scales, v_opacities, v_sh); break;
+    case 1: k_project_bwd<1><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                                      v_means, v_quats, v_scales, v_opacities, v_sh); break;
+    case 2: k_project_bwd<2><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                                      v_means, v_quats, v_scales, v_opacities, v_sh); break;
+    default: k_project_bwd<3><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                                       v_means, v_quats, v_scales, v_opacities, v_sh); break;
+  }
+  return cuda_status(cudaGetLastError(), "project bwd");
+}

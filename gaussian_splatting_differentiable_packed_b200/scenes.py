@@ -92,7 +92,7 @@ def _sh(rng, n, degree, dc_low, dc_high, rest_sigma):
     sh = np.empty((n, K, 3), np.float32)
     sh[:, 0, :] = rng.uniform(dc_low, dc_high, (n, 3))
     if K > 1:
-        sh[:, 1:, :] = rng.normal(0.0, rest_sigma, (n, K - 1, 3))
+        sh[:, 1:, :] = rng.standard_normal((n, K - 1, 3), dtype=np.float32) * np.float32(rest_sigma)
     return sh
 
 
@@ -105,16 +105,25 @@ def _ball(rng, n, sigma, radius):
     return out[:n]
 
 
-# Camera placements found once on the CPU (see the calibration notes in the
-# design document); frozen here so every run sees the same scene.
-CFG4_CAMS = (
-    ((-7.0, 0.5, -6.5), (2.0, -0.5, 3.0)),
-    ((7.0, 1.0, 6.5), (-1.0, -0.5, -2.0)),
-    ((6.5, -1.0, -7.0), (-2.0, 0.0, 2.5)),
-    ((-6.5, 1.5, 7.0), (2.5, -1.0, -1.5)),
-    ((0.0, 2.0, -7.5), (0.0, -1.0, 4.0)),
-)
-CFG5_EYE = (0.0, 4.2, 6.3)
+# Camera placements found once on the CPU with the oracle's visibility and
+# tile counts on subsampled scenes; frozen here so every run sees the same
+# scene.  Workload 3: ring of radius 8, each camera turned 47 degrees away from
+# the centre (about 30% of pairs visible).  Workload 4: five cameras on a
+# radius-22 ring around the room at height 1.5, turned +-41.5 degrees away from
+# the centre (about 20% of pairs visible, about 2.2 tiles per row).
+# Workload 5: camera 13.8 from the origin (about 5.9e8 intersections).
+CFG3_YAW_DEG = 47.0
+CFG4_RING = (22.0, 1.5, 41.5)
+CFG5_EYE_DIR = (0.0, 4.2, 6.3)
+CFG5_DIST = 13.8
+
+
+def _yawed(eye, yaw_deg):
+    eye = np.asarray(eye, np.float64)
+    fwd = -eye / np.linalg.norm(eye)
+    a = np.deg2rad(yaw_deg)
+    R = np.array([[np.cos(a), 0, np.sin(a)], [0, 1, 0], [-np.sin(a), 0, np.cos(a)]])
+    return look_at(eye, eye + R @ fwd)
 
 
 def make_scene(cfg: int, n: int | None = None, seed: int | None = None) -> Scene:
@@ -166,7 +175,7 @@ def make_scene(cfg: int, n: int | None = None, seed: int | None = None) -> Scene
         cams = []
         for k in range(4):
             th = np.deg2rad(90.0 * k)
-            cams.append(_cam(look_at((8 * np.sin(th), 0.0, 8 * np.cos(th)), (0, 0, 0)), 900, 900, 640, 360))
+            cams.append(_cam(_yawed((8 * np.sin(th), 0.0, 8 * np.cos(th)), CFG3_YAW_DEG), 900, 900, 640, 360))
         trng = np.random.Generator(np.random.PCG64(100 + (cfg - 1 if seed is None else seed)))
         target = trng.uniform(0.0, 1.0, (4, H, W, 3)).astype(np.float32)
         return Scene(cfg, 4, W, H, 3, N, near, far, np.stack(cams), means.astype(np.float32), quats,
@@ -193,7 +202,13 @@ def make_scene(cfg: int, n: int | None = None, seed: int | None = None) -> Scene
         opac = _sigmoid(rng.normal(0.0, 1.5, N))
         sh = _sh(rng, N, 3, 0.0, 1.0, 0.05)
         W, H = 1600, 1067
-        cams = np.stack([_cam(look_at(e, t), 1400, 1400, 800, 533.5) for e, t in CFG4_CAMS])
+        D, h, yaw = CFG4_RING
+        cams = []
+        for k in range(5):
+            th = np.deg2rad(72.0 * k + 10.0)
+            cams.append(_cam(_yawed((D * np.sin(th), h, D * np.cos(th)), yaw if k % 2 else -yaw),
+                             1400, 1400, 800, 533.5))
+        cams = np.stack(cams)
         trng = np.random.Generator(np.random.PCG64(100 + (cfg - 1 if seed is None else seed)))
         target = trng.uniform(0.0, 1.0, (5, H, W, 3)).astype(np.float32)
         return Scene(cfg, 5, W, H, 3, N, near, far, cams, means.astype(np.float32), quats,
@@ -212,7 +227,8 @@ def make_scene(cfg: int, n: int | None = None, seed: int | None = None) -> Scene
         opac = _sigmoid(rng.normal(0.0, 1.5, N))
         sh = _sh(rng, N, 3, 0.0, 1.0, 0.05)
         W = H = 7680
-        cams = np.stack([_cam(look_at(CFG5_EYE, (0, 0, 0)), 6000, 6000, 3840, 3840)])
+        eye = np.asarray(CFG5_EYE_DIR) / np.linalg.norm(CFG5_EYE_DIR) * CFG5_DIST
+        cams = np.stack([_cam(look_at(eye, (0, 0, 0)), 6000, 6000, 3840, 3840)])
         trng = np.random.Generator(np.random.PCG64(100 + (cfg - 1 if seed is None else seed)))
         v_img = (trng.uniform(-1.0, 1.0, (1, H, W, 3)) / (3.0 * W * H)).astype(np.float32)
         return Scene(cfg, 1, W, H, 3, N, near, far, cams, means.astype(np.float32), quats,

@@ -1,0 +1,307 @@
+"""ctypes binding of libss.so (include/ss.h) — argument marshalling only.
+
+Every function here forwards torch CUDA tensors' device pointers and the
+current CUDA stream to the C entry point of the same name and raises SSError
+on a non-zero status.  No step of the splatting path runs in Python or on the
+CPU: if libss.so is missing the import of the library fails loudly.
+PyTorch only allocates device memory and provides the stream.
+
+`PackedStep` strings the six calls into one forward+backward step with
+buffers owned by torch (the counts returned by the two synchronising calls
+size the later buffers; capacities grow with headroom when exceeded).
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libss.so")
+
+SS_OK, SS_ERR_INVALID_ARG, SS_ERR_CAPACITY, SS_ERR_OVERFLOW, SS_ERR_CUDA, SS_ERR_DEVICE_CHECK = range(6)
+SIZE_MASK_WORDS, SIZE_MASK_BLOCKS, SIZE_TILES_X, SIZE_TILES_Y, SIZE_N_TILES, SIZE_N_PAD = range(6)
+WS_PROJECT, WS_INTERSECT, WS_SORT = range(3)
+ROW = 12
+PMASK_BLOCK = 128
+TILE = 16
+
+EXPORTS = ("ss_size", "ss_workspace_bytes", "ss_status_string", "ss_last_error", "ss_project_packed",
+           "ss_intersect_tiles", "ss_sort_isects", "ss_rasterize_fwd", "ss_rasterize_bwd", "ss_project_bwd")
+
+
+class ss_dims(ct.Structure):
+    _fields_ = [("C", ct.c_int32), ("W", ct.c_int32), ("H", ct.c_int32), ("sh_degree", ct.c_int32),
+                ("N", ct.c_int64), ("near_plane", ct.c_float), ("far_plane", ct.c_float)]
+
+
+class SSError(RuntimeError):
+    def __init__(self, status: int, call: str, msg: str, count: int | None = None):
+        super().__init__(f"{call}: {msg} (status {status})")
+        self.status = status
+        self.count = count
+
+
+_lib = None
+
+
+def lib() -> ct.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m gaussian_splatting_differentiable_packed_b200.build`")
+        L = ct.CDLL(LIB_PATH)
+        P, i64, i32, sz = ct.c_void_p, ct.c_int64, ct.c_int, ct.c_size_t
+        D = ct.POINTER(ss_dims)
+        L.ss_size.argtypes = [D, i32]
+        L.ss_size.restype = i64
+        L.ss_workspace_bytes.argtypes = [D, i32, i64]
+        L.ss_workspace_bytes.restype = sz
+        L.ss_status_string.argtypes = [i32]
+        L.ss_status_string.restype = ct.c_char_p
+        L.ss_last_error.argtypes = []
+        L.ss_last_error.restype = ct.c_char_p
+        L.ss_project_packed.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, i64, P, sz, ct.POINTER(i64), P]
+        L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
+        L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, P, sz, P, ct.POINTER(i32), P]
+        L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P]
+        L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, i64, P]
+        L.ss_project_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_rasterize_fwd",
+                  "ss_rasterize_bwd", "ss_project_bwd"):
+            getattr(L, f).restype = i32
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ct.c_void_p(t)
+    return ct.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ct.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ct.c_void_p(stream)
+    return ct.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, call: str, count=None):
+    if status != SS_OK:
+        msg = lib().ss_last_error().decode() or lib().ss_status_string(status).decode()
+        raise SSError(status, call, msg, count)
+
+
+def make_dims(C, W, H, sh_degree, N, near=0.01, far=1e10) -> ss_dims:
+    return ss_dims(C, W, H, sh_degree, N, near, far)
+
+
+def size(d: ss_dims, what: int) -> int:
+    v = lib().ss_size(ct.byref(d), what)
+    if v < 0:
+        raise SSError(SS_ERR_INVALID_ARG, "ss_size", "invalid dims")
+    return int(v)
+
+
+def workspace_bytes(d: ss_dims, which: int, count: int = 0) -> int:
+    return int(lib().ss_workspace_bytes(ct.byref(d), which, count))
+
+
+def ss_project_packed(d, cams, means, quats, scales, opacities, sh, mask, block_count, block_off, screen, aabb16,
+                      cap_rows, temp, stream=None) -> int:
+    nnz = ct.c_int64(0)
+    st = lib().ss_project_packed(ct.byref(d), _p(cams), _p(means), _p(quats), _p(scales), _p(opacities), _p(sh),
+                                 _p(mask), _p(block_count), _p(block_off), _p(screen), _p(aabb16), int(cap_rows),
+                                 _p(temp), 0 if temp is None else temp.numel() * temp.element_size(),
+                                 ct.byref(nnz), _stream(stream))
+    _check(st, "ss_project_packed", int(nnz.value))
+    return int(nnz.value)
+
+
+def ss_intersect_tiles(d, screen, aabb16, block_off, nnz, isect_off, keys, vals, cap_isects, temp,
+                       stream=None) -> int:
+    n = ct.c_uint64(0)
+    st = lib().ss_intersect_tiles(ct.byref(d), _p(screen), _p(aabb16), _p(block_off), int(nnz), _p(isect_off),
+                                  _p(keys), _p(vals), int(cap_isects), _p(temp),
+                                  0 if temp is None else temp.numel() * temp.element_size(), ct.byref(n),
+                                  _stream(stream))
+    _check(st, "ss_intersect_tiles", int(n.value))
+    return int(n.value)
+
+
+def ss_sort_isects(d, keys_a, vals_a, keys_b, vals_b, n, temp, tile_off, stream=None) -> bool:
+    in_b = ct.c_int(0)
+    st = lib().ss_sort_isects(ct.byref(d), _p(keys_a), _p(vals_a), _p(keys_b), _p(vals_b), int(n), _p(temp),
+                              0 if temp is None else temp.numel() * temp.element_size(), _p(tile_off),
+                              ct.byref(in_b), _stream(stream))
+    _check(st, "ss_sort_isects")
+    return bool(in_b.value)
+
+
+def ss_rasterize_fwd(d, screen, vals, tile_off, img, T_final, last_id, stream=None):
+    _check(lib().ss_rasterize_fwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(img), _p(T_final),
+                                  _p(last_id), _stream(stream)), "ss_rasterize_fwd")
+
+
+def ss_rasterize_bwd(d, screen, vals, tile_off, T_final, last_id, v_img, v_T, v_screen, nnz, stream=None):
+    _check(lib().ss_rasterize_bwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(T_final), _p(last_id),
+                                  _p(v_img), _p(v_T), _p(v_screen), int(nnz), _stream(stream)), "ss_rasterize_bwd")
+
+
+def ss_project_bwd(d, cams, means, quats, scales, opacities, sh, mask, block_off, v_screen, v_means, v_quats,
+                   v_scales, v_opacities, v_sh, stream=None):
+    _check(lib().ss_project_bwd(ct.byref(d), _p(cams), _p(means), _p(quats), _p(scales), _p(opacities), _p(sh),
+                                _p(mask), _p(block_off), _p(v_screen), _p(v_means), _p(v_quats), _p(v_scales),
+                                _p(v_opacities), _p(v_sh), _stream(stream)), "ss_project_bwd")
+
+
+def _u32(n, dev):
+    return torch.empty(max(int(n), 1), dtype=torch.int32, device=dev)
+
+
+class PackedStep:
+    """One forward+backward step over fixed dims, buffers owned by torch.
+
+    forward() runs ss_project_packed, ss_intersect_tiles, ss_sort_isects and
+    ss_rasterize_fwd; backward(v_img, v_T=None) runs ss_rasterize_bwd and
+    ss_project_bwd.  Intermediate buffers are kept as attributes so callers
+    (tests) can inspect every stage.
+    """
+
+    def __init__(self, d: ss_dims, device="cuda", cap_rows: int = 0, cap_isects: int = 0, headroom: float = 1.25):
+        self.d = d
+        self.dev = torch.device(device)
+        self.headroom = headroom
+        C, N = d.C, d.N
+        self.K = (d.sh_degree + 1) ** 2
+        self.mask_words = size(d, SIZE_MASK_WORDS)
+        self.mask_blocks = size(d, SIZE_MASK_BLOCKS)
+        self.n_tiles = size(d, SIZE_N_TILES)
+        dev = self.dev
+        self.mask = _u32(self.mask_words, dev)
+        self.block_count = _u32(self.mask_blocks, dev)
+        self.block_off = torch.empty(self.mask_blocks + 1, dtype=torch.int64, device=dev)
+        self.temp_project = torch.empty(workspace_bytes(d, WS_PROJECT), dtype=torch.uint8, device=dev)
+        self.tile_off = torch.empty(self.n_tiles + 1, dtype=torch.int64, device=dev)
+        self.img = torch.empty((C, d.H, d.W, 3), dtype=torch.float32, device=dev)
+        self.T = torch.empty((C, d.H, d.W), dtype=torch.float32, device=dev)
+        self.last = torch.empty((C, d.H, d.W), dtype=torch.int32, device=dev)
+        self.v_means = torch.empty((N, 3), dtype=torch.float32, device=dev)
+        self.v_quats = torch.empty((N, 4), dtype=torch.float32, device=dev)
+        self.v_scales = torch.empty((N, 3), dtype=torch.float32, device=dev)
+        self.v_opacities = torch.empty((N,), dtype=torch.float32, device=dev)
+        self.v_sh = torch.empty((N, self.K, 3), dtype=torch.float32, device=dev)
+        self.cap_rows = 0
+        self.cap_isects = 0
+        self._rows(cap_rows)
+        self._isects(cap_isects)
+        self.nnz = 0
+        self.n_isects = 0
+        self.result_in_b = False
+
+    def _rows(self, cap):
+        cap = max(int(cap), 1)
+        if cap <= self.cap_rows:
+            return
+        dev = self.dev
+        self.screen = torch.empty((cap, ROW), dtype=torch.float32, device=dev)
+        self.aabb16 = torch.empty((cap, 2), dtype=torch.int32, device=dev)
+        self.isect_off = torch.empty(cap + 1, dtype=torch.int64, device=dev)
+        self.v_screen = torch.empty((cap, ROW), dtype=torch.float32, device=dev)
+        self.temp_isect = torch.empty(workspace_bytes(self.d, WS_INTERSECT, cap), dtype=torch.uint8, device=dev)
+        self.cap_rows = cap
+
+    def _isects(self, cap):
+        cap = max(int(cap), 1)
+        if cap <= self.cap_isects:
+            return
+        dev = self.dev
+        self.keys_a = torch.empty(cap, dtype=torch.int64, device=dev)
+        self.vals_a = torch.empty(cap, dtype=torch.int32, device=dev)
+        self.keys_b = torch.empty(cap, dtype=torch.int64, device=dev)
+        self.vals_b = torch.empty(cap, dtype=torch.int32, device=dev)
+        self.temp_sort = torch.empty(workspace_bytes(self.d, WS_SORT, cap), dtype=torch.uint8, device=dev)
+        self.cap_isects = cap
+
+    def forward(self, cams, means, quats, scales, opacities, sh, stream=None):
+        self.inputs = (cams, means, quats, scales, opacities, sh)
+        d = self.d
+        try:
+            nnz = ss_project_packed(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_count,
+                                    self.block_off, self.screen, self.aabb16, self.cap_rows, self.temp_project,
+                                    stream)
+        except SSError as e:
+            if e.status != SS_ERR_CAPACITY:
+                raise
+            self._rows(int(e.count * self.headroom) + 1)
+            nnz = ss_project_packed(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_count,
+                                    self.block_off, self.screen, self.aabb16, self.cap_rows, self.temp_project,
+                                    stream)
+        self.nnz = nnz
+        try:
+            n = ss_intersect_tiles(d, self.screen, self.aabb16, self.block_off, nnz, self.isect_off, self.keys_a,
+                                   self.vals_a, self.cap_isects, self.temp_isect, stream)
+        except SSError as e:
+            if e.status != SS_ERR_CAPACITY:
+                raise
+            self._isects(int(e.count * self.headroom) + 1)
+            n = ss_intersect_tiles(d, self.screen, self.aabb16, self.block_off, nnz, self.isect_off, self.keys_a,
+                                   self.vals_a, self.cap_isects, self.temp_isect, stream)
+        self.n_isects = n
+        self.unsorted_keys = self.keys_a
+        self.unsorted_vals = self.vals_a
+        self.result_in_b = ss_sort_isects(d, self.keys_a, self.vals_a, self.keys_b, self.vals_b, n, self.temp_sort,
+                                          self.tile_off, stream)
+        self.keys = self.keys_b if self.result_in_b else self.keys_a
+        self.vals = self.vals_b if self.result_in_b else self.vals_a
+        ss_rasterize_fwd(d, self.screen, self.vals, self.tile_off, self.img, self.T, self.last, stream)
+        return self.img
+
+    def backward(self, v_img, v_T=None, stream=None):
+        cams, means, quats, scales, opacities, sh = self.inputs
+        d = self.d
+        ss_rasterize_bwd(d, self.screen, self.vals, self.tile_off, self.T, self.last, v_img, v_T, self.v_screen,
+                         self.nnz, stream)
+        ss_project_bwd(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_off, self.v_screen,
+                       self.v_means, self.v_quats, self.v_scales, self.v_opacities, self.v_sh, stream)
+        return dict(v_means=self.v_means, v_quats=self.v_quats, v_scales=self.v_scales,
+                    v_opacities=self.v_opacities, v_sh=self.v_sh)
+
+
+def scene_tensors(scene, device="cuda"):
+    """Device copies of a scenes.Scene's inputs (cams, means, quats, scales, opacities, sh)."""
+    f = lambda a: torch.from_numpy(a).to(device=device, dtype=torch.float32).contiguous()
+    return (f(scene.cams), f(scene.means), f(scene.quats), f(scene.scales), f(scene.opacities), f(scene.sh))
+
+
+def scene_dims(scene) -> ss_dims:
+    return make_dims(scene.C, scene.W, scene.H, scene.sh_degree, scene.N, scene.near, scene.far)
+
+
+def sort_passes(d: ss_dims) -> int:
+    """8-bit digit passes of ss_sort_isects: 4 over the 31 depth bits, then
+    ceil(bits(n_tiles) / 8) over the tile id."""
+    n_tiles = size(d, SIZE_N_TILES)
+    tb = max(0, (n_tiles - 1).bit_length())
+    return 4 + (tb + 7) // 8
+
+
+def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
+    """Kernels libss launches in one forward+backward step (memsets excluded):
+    projection 5 (pass 1, three scan kernels, pass 2), intersection 4 (three
+    scan kernels, write), sort 5 per pass + tile ranges, rasterizer 1 + 1,
+    projection backward 1."""
+    if d.N == 0:
+        return 0
+    n = 5
+    if nnz > 0:
+        n += 4 if n_isects > 0 else 3
+    if n_isects > 0:
+        n += 5 * sort_passes(d) + 1
+    return n + 3

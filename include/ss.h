@@ -1,0 +1,195 @@
+/*
+ * ss.h — C ABI of the packed 3D Gaussian Splatting training step (libss.so).
+ *
+ * One forward+backward step over C cameras x N Gaussians, as described on the
+ * "Spirula Studio" pages:
+ *   ss_project_packed   packed projection (visibility bitmask, block-count scan,
+ *                       compaction into screen rows and 16-bit AABBs)
+ *   ss_intersect_tiles  tile intersections with an exact 64-bit count
+ *   ss_sort_isects      radix sort of (tile_id << 32 | depth) keys + tile ranges
+ *   ss_rasterize_fwd    16x16-tile front-to-back alpha compositing
+ *   ss_rasterize_bwd    per-pixel reverse replay -> screen-space gradients
+ *   ss_project_bwd      screen-space gradients -> means, quats, scales,
+ *                       opacities, SH coefficients
+ *
+ * Conventions (all entry points):
+ *   - Every array pointer is a DEVICE pointer owned by the caller unless the
+ *     parameter name ends in _out (host scalar).  The library never allocates
+ *     or frees memory and keeps no state between calls.  Calls that need
+ *     scratch take (temp, temp_bytes), sized by ss_workspace_bytes().
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).  Only ss_project_packed and ss_intersect_tiles
+ *     synchronise the stream, to return the counts that size later buffers.
+ *   - Outputs are overwritten, never accumulated into.
+ *   - Floating point is IEEE fp32; integer outputs are deterministic.
+ *   - Errors are returned as ss_status; a failing call writes no element
+ *     outside the caller's stated capacities.  Device-side checks never trap.
+ *   - All sizes and offsets are 64-bit; buffers may exceed 4 GiB.
+ *
+ * Layouts:
+ *   cams      float [C][20]: world-to-camera 4x4 view matrix, row-major, OpenCV
+ *             axes (x right, y down, z forward), then fx, fy, cx, cy (pixels)
+ *   means     float [N][3]      quats  float [N][4] (w,x,y,z; normalised inside)
+ *   scales    float [N][3] activated (exp of the log-scale)
+ *   opacities float [N]    activated (sigmoid of the logit)
+ *   sh        float [N][K][3], K = (sh_degree+1)^2, real SH, degree-major
+ *   mask      uint32 [ss_size(SS_SIZE_MASK_WORDS)]: bit (c*n_pad + n), LSB
+ *             first, n_pad = N rounded up to SS_PMASK_BLOCK; padding bits are 0
+ *   block_count uint32 [ss_size(SS_SIZE_MASK_BLOCKS)]: set bits per 128-pair block
+ *   block_off int64 [blocks + 1]: exclusive scan of block_count; last = nnz
+ *   screen    float [cap_rows][12]: x, y, conic a, conic b, conic c, opacity,
+ *             r, g, b, depth, 0, 0 (48-byte rows: three 16-byte vectors)
+ *   aabb16    uint32 [cap_rows][2]: word0 = qx0 | qy0 << 16, word1 = qx1 | qy1 << 16,
+ *             edges on the grid extent/65535, min floored, max ceiled
+ *   keys      uint64 [cap_isects]: (c*tiles_per_cam + ty*tiles_x + tx) << 32 | bits(depth)
+ *   vals      uint32 [cap_isects]: screen row index
+ *   tile_off  int64 [n_tiles + 1]: tile t owns sorted entries [tile_off[t], tile_off[t+1])
+ *   img       float [C][H][W][3]   T_final float [C][H][W]   last_id int32 [C][H][W]
+ *   v_screen  float [nnz][12]: d/d(x, y, a, b, c, opacity, r, g, b, depth), 0, 0
+ */
+#ifndef SS_H
+#define SS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Pairs per visibility block: each 128-pair block of the mask gets one
+ * popcount ("Spirula Studio VRAM deep-dive", section "bitmask compaction":
+ * both passes must agree on this constant). */
+#define SS_PMASK_BLOCK 128
+/* Rasterizer tile edge in pixels. */
+#define SS_TILE 16
+/* Floats per screen row and per screen-gradient row. */
+#define SS_ROW_FLOATS 12
+
+typedef int ss_status;
+#define SS_OK 0
+#define SS_ERR_INVALID_ARG 1   /* bad dims, null pointer, short temp buffer */
+#define SS_ERR_CAPACITY 2      /* output capacity too small; the exact count is still returned */
+#define SS_ERR_OVERFLOW 3      /* n_isects >= 2^31 (values and last_id are 32-bit) */
+#define SS_ERR_CUDA 4          /* a CUDA runtime error; see ss_last_error() */
+#define SS_ERR_DEVICE_CHECK 5  /* a device-side check failed (reported, never trapped) */
+
+typedef struct ss_dims {
+  int32_t C;          /* cameras, >= 1 */
+  int32_t W, H;       /* image size in pixels, >= 1 */
+  int32_t sh_degree;  /* 0..3 */
+  int64_t N;          /* Gaussians, >= 0 */
+  float near_plane;   /* > 0 */
+  float far_plane;    /* > near_plane */
+} ss_dims;
+
+/* Sizes derived from dims (element counts, not bytes). */
+#define SS_SIZE_MASK_WORDS 0   /* C * n_pad / 32 */
+#define SS_SIZE_MASK_BLOCKS 1  /* C * n_pad / 128 */
+#define SS_SIZE_TILES_X 2
+#define SS_SIZE_TILES_Y 3
+#define SS_SIZE_N_TILES 4      /* C * tiles_x * tiles_y */
+#define SS_SIZE_N_PAD 5
+int64_t ss_size(const ss_dims* dims, int what);
+
+/* Scratch bytes needed by a call: which = SS_WS_PROJECT (count ignored),
+ * SS_WS_INTERSECT (count = nnz), SS_WS_SORT (count = number of keys). */
+#define SS_WS_PROJECT 0
+#define SS_WS_INTERSECT 1
+#define SS_WS_SORT 2
+size_t ss_workspace_bytes(const ss_dims* dims, int which, int64_t count);
+
+const char* ss_status_string(ss_status status);
+/* Message of the last failing call on this host thread ("" if none). */
+const char* ss_last_error(void);
+
+/*
+ * Packed projection ("Spirula Studio VRAM deep-dive", sections "bitmask
+ * compaction" and "16-bit packed AABB"; "Spirula Studio backward pass",
+ * section 5 for the projection chain).
+ *
+ * Pass 1 projects every (camera, Gaussian) pair (EWA covariance from quat and
+ * scale, 0.3 dilation, 3-sigma radius) and writes the visibility bitmask and
+ * one popcount per 128-pair block; the block counts are scanned into block_off
+ * and nnz = block_off[blocks] is copied to *nnz_out (stream sync).  If screen
+ * is NULL the call stops there (count-only).  If nnz > cap_rows it returns
+ * SS_ERR_CAPACITY with *nnz_out exact and writes no row.  Otherwise pass 2
+ * re-projects the survivors only: row = block_off[block] + set bits before the
+ * pair, writing the screen row (SH colour evaluated toward the camera centre)
+ * and the 16-bit AABB.  Rows are ordered camera-major, Gaussian-minor.
+ */
+ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float* means, const float* quats,
+                            const float* scales, const float* opacities, const float* sh, uint32_t* mask,
+                            uint32_t* block_count, int64_t* block_off, float* screen, uint32_t* aabb16,
+                            int64_t cap_rows, void* temp, size_t temp_bytes, int64_t* nnz_out, void* stream);
+
+/*
+ * Tile intersections ("Spirula Studio VRAM deep-dive", section "4 GiB rule and
+ * 2^31 limit": exact 64-bit count, host check before the scan, write window
+ * clamped to the allocation; key format from the buffer-cost table).
+ *
+ * Counts the tiles of each row from its AABB16 (integer arithmetic), sums them
+ * exactly in 64 bits and returns the total in *n_isects_out (stream sync).
+ * Returns SS_ERR_CAPACITY if the total exceeds cap_isects and
+ * SS_ERR_OVERFLOW if it is >= 2^31, writing nothing else in either case.
+ * Otherwise writes isect_off[nnz+1] (exclusive per-row offsets) and one
+ * (key, row) per covered tile, row-major over (row, ty, tx).  block_off is the
+ * array ss_project_packed wrote (it gives each camera's first row).
+ */
+ss_status ss_intersect_tiles(const ss_dims* dims, const float* screen, const uint32_t* aabb16,
+                             const int64_t* block_off, int64_t nnz, int64_t* isect_off, uint64_t* keys,
+                             uint32_t* vals, int64_t cap_isects, void* temp, size_t temp_bytes,
+                             uint64_t* n_isects_out, void* stream);
+
+/*
+ * Stable LSD radix sort of n (key, value) pairs by key, 8-bit digits over the
+ * 31 depth bits and the tile-id bits only ("Spirula Studio VRAM deep-dive",
+ * buffer table: double-buffered isect.ids_a/b).  Ping-pongs between (keys_a,
+ * vals_a) and (keys_b, vals_b); *result_in_b_out (host) says which pair holds
+ * the result (known from dims alone; no sync).  Then writes tile_off[n_tiles+1].
+ * n >= 2^31 returns SS_ERR_OVERFLOW.  Equal keys keep their input order.
+ */
+ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
+                         uint32_t* vals_b, int64_t n, void* temp, size_t temp_bytes, int64_t* tile_off,
+                         int* result_in_b_out, void* stream);
+
+/*
+ * Forward rasterizer ("Spirula Studio backward pass", section 4: the forward
+ * keeps tile offsets, the intersection list, each pixel's last Gaussian and
+ * its transmittance for the backward pass).  One CTA per 16x16 tile, front to
+ * back over the tile's sorted entries: alpha = min(0.99, o*exp(-sigma)),
+ * entries with alpha < 1/255 skipped, stop before the entry that would take
+ * T below 1e-4.  Writes img, T_final and last_id (the sorted index of the last
+ * composited entry, -1 if none).  vals are the sorted values.
+ */
+ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, const uint32_t* vals, const int64_t* tile_off,
+                           float* img, float* T_final, int32_t* last_id, void* stream);
+
+/*
+ * Backward rasterizer ("Spirula Studio backward pass", section 4): per pixel,
+ * reverse replay from last_id using the saved state (no re-intersection),
+ * splitting v_img (and v_T, may be NULL) by each entry's alpha contribution.
+ * Gradients are reduced over the tile's pixels and added with atomics into
+ * v_screen[nnz][12], which the call zeroes first.
+ */
+ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, const uint32_t* vals, const int64_t* tile_off,
+                           const float* T_final, const int32_t* last_id, const float* v_img, const float* v_T,
+                           float* v_screen, int64_t nnz, void* stream);
+
+/*
+ * Projection backward ("Spirula Studio backward pass", section 5): for each
+ * Gaussian, over the cameras whose mask bit is set, the screen-row gradient is
+ * taken back through the conic, the EWA Jacobian, the camera transform, the
+ * covariance and the SH colour.  Deterministic (one thread per Gaussian, no
+ * atomics).  Writes every element of the five outputs (zero where invisible).
+ */
+ss_status ss_project_bwd(const ss_dims* dims, const float* cams, const float* means, const float* quats,
+                         const float* scales, const float* opacities, const float* sh, const uint32_t* mask,
+                         const int64_t* block_off, const float* v_screen, float* v_means, float* v_quats,
+                         float* v_scales, float* v_opacities, float* v_sh, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS_H */

@@ -117,10 +117,14 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work):
                                instr=P * 140.0 + nnz * 160.0)
     m["intersect_tiles"] = dict(bytes=8 * nnz * 2 + 8 * nnz + 4 * nnz + 12 * n_isects, instr=0.0)
     m["sort_isects"] = dict(bytes=n_isects * (8 + 24) * passes + 8 * (n_tiles + 1), instr=0.0)
+    # per-pixel FP32 instructions of the canonical sequences: 11 per evaluated
+    # entry (offsets, sigma, tests), 16 per exp (range reduction, degree-7
+    # polynomial, scaling, alpha), 7 per composite; backward: 11 per replayed
+    # entry, 17 per exp, 30 per contributing entry (T recovery, nine gradients)
     m["rasterize_fwd"] = dict(bytes=n_isects * (4 + row) + X * 20 + 8 * (n_tiles + 1),
-                              instr=work["evals"] * 12.0 + work["exps"] * 22.0 + work["comps"] * 9.0)
+                              instr=work["evals"] * 11.0 + work["exps"] * 16.0 + work["comps"] * 7.0)
     m["rasterize_bwd"] = dict(bytes=n_isects * (4 + row) + X * 24 + nnz * row * 2,
-                              instr=work["bwd_evals"] * 12.0 + work["bwd_exps"] * 22.0 + work["comps"] * 60.0)
+                              instr=work["bwd_evals"] * 11.0 + work["bwd_exps"] * 17.0 + work["comps"] * 30.0)
     m["project_bwd"] = dict(bytes=(par + shb) * N + row * nnz + P / 8 + P / 16 + (par + 4 + shb) * N,
                             instr=nnz * 700.0)
     return m
@@ -315,6 +319,7 @@ def run_ours(args):
                     frac=round(ach / pk, 4), traffic=None, kernel=dom,
                     peak_source=f"148 SMs x 128 FP32 lanes x {sm_mhz:.0f} MHz (median SM clock under load)")
     launches = ss.launches_per_step(d, step.nnz, step.n_isects) * args.steps
+    out_work = dict(work)
     out = dict(metric=METRIC, value=world * step.n_isects / (ms / 1e3), unit="isects/s", n_gpus=world,
                steps=args.steps, warmup=args.warmup, ms_per_step=round(ms, 4), higher_is_better=True,
                scaling="weak", vs_baseline=None, dtype="f32", data="synthetic",
@@ -322,7 +327,8 @@ def run_ours(args):
                            sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
                            sort_passes=passes, l2="inputs larger than L2 (3.5 GB parameters), no flush",
                            parallelism=f"replicas x{world}"),
-               pairs_per_s=world * d.C * d.N / (ms / 1e3), stages=stages, roofline=roof, clocks=clocks,
+               pairs_per_s=world * d.C * d.N / (ms / 1e3), raster_work=out_work, stages=stages, roofline=roof,
+               clocks=clocks,
                e2e=e2e, gpu_launches=launches)
     if not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_sample)

@@ -78,6 +78,13 @@ __global__ __launch_bounds__(kBlock) void k_project_mask(Geo g, const float* __r
   }
 }
 
+// Shared-memory stride per Gaussian for an SH block (odd: conflict-free).
+template <int DEG>
+__host__ __device__ constexpr int rows_sh_stride() {
+  return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
+}
+
+template <int DEG>
 __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __restrict__ cams,
                                                          const float* __restrict__ means,
                                                          const float* __restrict__ quats,
@@ -87,18 +94,31 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
                                                          const uint32_t* __restrict__ mask,
                                                          const int64_t* __restrict__ block_off,
                                                          float* __restrict__ screen, uint32_t* __restrict__ aabb16) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  constexpr int K3 = 3 * K;
+  constexpr int KP = rows_sh_stride<DEG>();
   __shared__ Cam scam[kCamChunk];
+  __shared__ float sh_s[kBlock * KP];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t blk = blockIdx.x;
-  const int64_t n = blk * kBlock + threadIdx.x;
+  const int64_t n0 = blk * kBlock;
+  const int64_t n = n0 + threadIdx.x;
   const bool valid = n < g.N;
+  const int cnt = (int)min64(kBlock, g.N - n0);
+  {
+    const float* src = sh + n0 * K3;
+    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+      const int gi = f / K3, q = f - gi * K3;
+      sh_s[gi * KP + q] = src[f];
+    }
+  }
+  const float* shn = sh_s + threadIdx.x * KP;
   GaussIn gi{};
   float opac = 0.0f;
   if (valid) {
     gi = load_gauss(means, quats, scales, n);
     opac = opacities[n];
   }
-  const float* shn = sh + (int64_t)g.K * 3 * (valid ? n : 0);
   for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
     const int nc = min(kCamChunk, g.C - c0);
     __syncthreads();
@@ -121,13 +141,14 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
       // colour
       float b[16];
       float X = 0.0f, Y = 0.0f, Z = 0.0f, il;
-      if (g.deg > 0) view_dir(k, gi.mx, gi.my, gi.mz, X, Y, Z, il);
-      sh_basis(g.deg, X, Y, Z, b);
+      if (DEG > 0) view_dir(k, gi.mx, gi.my, gi.mz, X, Y, Z, il);
+      sh_basis(DEG, X, Y, Z, b);
       float rgb[3];
 #pragma unroll
       for (int ch = 0; ch < 3; ++ch) {
         float acc = mul(shn[ch], b[0]);
-        for (int kk = 1; kk < g.K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], b[kk]));
+#pragma unroll
+        for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], b[kk]));
         rgb[ch] = fmaxf(add(acc, 0.5f), 0.0f);
       }
       float4* out = reinterpret_cast<float4*>(screen + row * kRowF);
@@ -142,6 +163,14 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
       reinterpret_cast<uint2*>(aabb16)[row] = q;
     }
   }
+}
+
+template <int DEG>
+void launch_rows(const Geo& g, unsigned grid, cudaStream_t st, const float* cams, const float* means,
+                 const float* quats, const float* scales, const float* opacities, const float* sh,
+                 const uint32_t* mask, const int64_t* block_off, float* screen, uint32_t* aabb16) {
+  k_project_rows<DEG><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, opacities, sh, mask, block_off, screen,
+                                               aabb16);
 }
 
 }  // namespace ss
@@ -192,7 +221,14 @@ extern "C" ss_status ss_project_packed(const ss_dims* dims, const float* cams, c
   }
   if (!opacities || !sh || !aabb16) return invalid("null row input/output");
   if (((uintptr_t)screen & 15) != 0 || ((uintptr_t)aabb16 & 7) != 0) return invalid("row buffers misaligned");
-  k_project_rows<<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, opacities, sh, mask, block_off, screen,
-                                          aabb16);
+  switch (g.deg) {
+    case 0: launch_rows<0>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+            break;
+    case 1: launch_rows<1>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+            break;
+    case 2: launch_rows<2>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+            break;
+    default: launch_rows<3>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+  }
   return cuda_status(cudaGetLastError(), "project pass 2");
 }

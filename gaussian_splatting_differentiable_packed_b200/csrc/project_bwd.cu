@@ -68,35 +68,57 @@ __device__ __forceinline__ void sh_grads(float X, float Y, float Z, const float*
   }
 }
 
+// Shared-memory stride per Gaussian for SH blocks (odd, so that thread t's
+// word k sits in bank (t*stride + k) mod 32: conflict-free across a warp).
 template <int DEG>
-__global__ __launch_bounds__(kBlock) void k_project_bwd(Geo g, const float* __restrict__ cams,
-                                                        const float* __restrict__ means,
-                                                        const float* __restrict__ quats,
-                                                        const float* __restrict__ scales,
-                                                        const float* __restrict__ sh,
-                                                        const uint32_t* __restrict__ mask,
-                                                        const int64_t* __restrict__ block_off,
-                                                        const float* __restrict__ v_screen, float* __restrict__ v_means,
-                                                        float* __restrict__ v_quats, float* __restrict__ v_scales,
-                                                        float* __restrict__ v_opac, float* __restrict__ v_sh) {
+__host__ __device__ constexpr int sh_stride() {
+  return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
+}
+
+template <int DEG>
+__global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* __restrict__ cams,
+                                                           const float* __restrict__ means,
+                                                           const float* __restrict__ quats,
+                                                           const float* __restrict__ scales,
+                                                           const float* __restrict__ sh,
+                                                           const uint32_t* __restrict__ mask,
+                                                           const int64_t* __restrict__ block_off,
+                                                           const float* __restrict__ v_screen,
+                                                           float* __restrict__ v_means, float* __restrict__ v_quats,
+                                                           float* __restrict__ v_scales, float* __restrict__ v_opac,
+                                                           float* __restrict__ v_sh) {
   constexpr int K = (DEG + 1) * (DEG + 1);
+  constexpr int K3 = 3 * K;
+  constexpr int KP = sh_stride<DEG>();
   __shared__ Cam scam[kCamChunkB];
+  extern __shared__ float smem[];
+  float* sh_s = smem;                 // [kBlock][KP] SH coefficients of the CTA's Gaussians
+  float* gsh_s = smem + kBlock * KP;  // [kBlock][KP] their gradient accumulators
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t blk = blockIdx.x;
-  const int64_t n = blk * kBlock + threadIdx.x;
+  const int64_t n0 = blk * kBlock;
+  const int64_t n = n0 + threadIdx.x;
   const bool valid = n < g.N;
+  const int cnt = (int)min64(kBlock, g.N - n0);
+  // coalesced staging of the CTA's contiguous SH block
+  {
+    const float* src = sh + n0 * K3;
+    for (int f = threadIdx.x; f < kBlock * K3; f += kBlock) {
+      const int gi = f / K3, q = f - gi * K3;
+      sh_s[gi * KP + q] = f < cnt * K3 ? src[f] : 0.0f;
+      gsh_s[gi * KP + q] = 0.0f;
+    }
+  }
+  const float* shn = sh_s + threadIdx.x * KP;
+  float* gsh = gsh_s + threadIdx.x * KP;
   const int64_t nn = valid ? n : 0;
   const float mx = means[3 * nn], my = means[3 * nn + 1], mz = means[3 * nn + 2];
   const float4 q4 = reinterpret_cast<const float4*>(quats)[nn];
   const QuatRot qr = quat_rot(q4.x, q4.y, q4.z, q4.w);
   const float s0 = scales[3 * nn], s1 = scales[3 * nn + 1], s2 = scales[3 * nn + 2];
   const Cov3 S = cov3(qr, s0, s1, s2);
-  const float* shn = sh + (int64_t)K * 3 * nn;
   float gmu[3] = {0.f, 0.f, 0.f}, go = 0.f;
-  float gS[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // dL/dSigma, full-matrix convention (00 01 02 11 12 22)
-  float gsh[3 * K];
-#pragma unroll
-  for (int q = 0; q < 3 * K; ++q) gsh[q] = 0.f;
+  double gS[6] = {0., 0., 0., 0., 0., 0.};  // dL/dSigma, full-matrix convention (00 01 02 11 12 22)
   for (int c0 = 0; c0 < g.C; c0 += kCamChunkB) {
     const int nc = min(kCamChunkB, g.C - c0);
     __syncthreads();
@@ -114,62 +136,75 @@ __global__ __launch_bounds__(kBlock) void k_project_bwd(Geo g, const float* __re
       const float4* vrp = reinterpret_cast<const float4*>(v_screen + row * kRowF);
       const float4 v0 = vrp[0], v1 = vrp[1], v2 = vrp[2];
       const Cam& k = scam[cc];
-      Proj P;
-      cam_point(k, mx, my, mz, P.px, P.py, P.pz);
-      project_rest(k, S, g.W, g.H, P);
-      // conic (c, -b, a)/det -> dilated covariance (a, b, c)
-      const float a = P.a, b = P.b, cq = P.c;
-      const float id = 1.0f / P.det, id2 = id * id;
-      const float vca = v0.z, vcb = v0.w, vcc = v1.x;
-      const float va = (-vca * cq * cq + vcb * b * cq - vcc * b * b) * id2;
-      const float vb = (2.0f * vca * b * cq - vcb * (a * cq + b * b) + 2.0f * vcc * a * b) * id2;
-      const float vc = (-vca * b * b + vcb * a * b - vcc * a * a) * id2;
-      const float hb = 0.5f * vb;
-      const float* T = P.T;
-      // TS = T Sigma (2x3)
-      const float Sm[3][3] = {{S.s00, S.s01, S.s02}, {S.s01, S.s11, S.s12}, {S.s02, S.s12, S.s22}};
-      float TS[2][3];
+      const float* R = k.R;
+      // camera point and the projection's gating decision in canonical arithmetic
+      float px, py, pz;
+      cam_point(k, mx, my, mz, px, py, pz);
+      const float izc = div_(1.0f, pz);
+      const float u = mul(px, izc), v = mul(py, izc);
+      const bool clx = (u < -k.limx) || (u > k.limx);
+      const bool cly = (v < -k.limy) || (v > k.limy);
+      const float ux = fminf(fmaxf(u, -k.limx), k.limx), uy = fminf(fmaxf(v, -k.limy), k.limy);
+      // gradient arithmetic (any rounding order)
+      const float iz = 1.0f / pz, iz2 = iz * iz;
+      const float j00 = k.fx * iz, j02 = -j00 * ux, j11 = k.fy * iz, j12 = -j11 * uy;
+      float T[6];
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        T[m] = j00 * R[m] + j02 * R[6 + m];
+        T[3 + m] = j11 * R[3 + m] + j12 * R[6 + m];
+      }
+      // conic -> 2D covariance -> (T, Sigma) in fp64: the terms are of size
+      // (f/z)^2 * |V2| and cancel down to small rotation/scale gradients
+      const double Sm[3][3] = {{S.s00, S.s01, S.s02}, {S.s01, S.s11, S.s12}, {S.s02, S.s12, S.s22}};
+      double Td[6];
+#pragma unroll
+      for (int m = 0; m < 6; ++m) Td[m] = T[m];
+      double TS[2][3];
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int m = 0; m < 3; ++m) TS[r][m] = T[3 * r] * Sm[0][m] + T[3 * r + 1] * Sm[1][m] + T[3 * r + 2] * Sm[2][m];
-      // dL/dT = 2 V2 T Sigma
+        for (int m = 0; m < 3; ++m)
+          TS[r][m] = Td[3 * r] * Sm[0][m] + Td[3 * r + 1] * Sm[1][m] + Td[3 * r + 2] * Sm[2][m];
+      const double a = TS[0][0] * Td[0] + TS[0][1] * Td[1] + TS[0][2] * Td[2] + 0.3;
+      const double b = TS[0][0] * Td[3] + TS[0][1] * Td[4] + TS[0][2] * Td[5];
+      const double cq = TS[1][0] * Td[3] + TS[1][1] * Td[4] + TS[1][2] * Td[5] + 0.3;
+      // conic (c, -b, a)/det -> dilated covariance (a, b, c)
+      const double id = 1.0 / (a * cq - b * b), id2 = id * id;
+      const double vca = v0.z, vcb = v0.w, vcc = v1.x;
+      const double va = (-vca * cq * cq + vcb * b * cq - vcc * b * b) * id2;
+      const double vb = (2.0 * vca * b * cq - vcb * (a * cq + b * b) + 2.0 * vcc * a * b) * id2;
+      const double vc = (-vca * b * b + vcb * a * b - vcc * a * a) * id2;
+      const double hb = 0.5 * vb;
+      // dL/dT = 2 V2 T Sigma;  dL/dSigma += T^T V2 T
       float GT[2][3];
+      double VT[2][3];
 #pragma unroll
       for (int m = 0; m < 3; ++m) {
-        GT[0][m] = 2.0f * (va * TS[0][m] + hb * TS[1][m]);
-        GT[1][m] = 2.0f * (hb * TS[0][m] + vc * TS[1][m]);
+        GT[0][m] = (float)(2.0 * (va * TS[0][m] + hb * TS[1][m]));
+        GT[1][m] = (float)(2.0 * (hb * TS[0][m] + vc * TS[1][m]));
+        VT[0][m] = va * Td[m] + hb * Td[3 + m];
+        VT[1][m] = hb * Td[m] + vc * Td[3 + m];
       }
-      // dL/dSigma += T^T V2 T
-      {
-        float VT[2][3];
-#pragma unroll
-        for (int m = 0; m < 3; ++m) {
-          VT[0][m] = va * T[m] + hb * T[3 + m];
-          VT[1][m] = hb * T[m] + vc * T[3 + m];
-        }
-        gS[0] += T[0] * VT[0][0] + T[3] * VT[1][0];
-        gS[1] += T[0] * VT[0][1] + T[3] * VT[1][1];
-        gS[2] += T[0] * VT[0][2] + T[3] * VT[1][2];
-        gS[3] += T[1] * VT[0][1] + T[4] * VT[1][1];
-        gS[4] += T[1] * VT[0][2] + T[4] * VT[1][2];
-        gS[5] += T[2] * VT[0][2] + T[5] * VT[1][2];
-      }
+      gS[0] += Td[0] * VT[0][0] + Td[3] * VT[1][0];
+      gS[1] += Td[0] * VT[0][1] + Td[3] * VT[1][1];
+      gS[2] += Td[0] * VT[0][2] + Td[3] * VT[1][2];
+      gS[3] += Td[1] * VT[0][1] + Td[4] * VT[1][1];
+      gS[4] += Td[1] * VT[0][2] + Td[4] * VT[1][2];
+      gS[5] += Td[2] * VT[0][2] + Td[5] * VT[1][2];
       // T = J R -> dL/dJ = dL/dT R^T (entries 00, 02, 11, 12)
-      const float* R = k.R;
       const float gj00 = GT[0][0] * R[0] + GT[0][1] * R[1] + GT[0][2] * R[2];
       const float gj02 = GT[0][0] * R[6] + GT[0][1] * R[7] + GT[0][2] * R[8];
       const float gj11 = GT[1][0] * R[3] + GT[1][1] * R[4] + GT[1][2] * R[5];
       const float gj12 = GT[1][0] * R[6] + GT[1][1] * R[7] + GT[1][2] * R[8];
-      const float iz = 1.0f / P.pz, iz2 = iz * iz;
       float gx = 0.f, gy = 0.f;
-      float gz = -k.fx * iz2 * gj00 + k.fx * P.ux * iz2 * gj02 - k.fy * iz2 * gj11 + k.fy * P.uy * iz2 * gj12;
+      float gz = -k.fx * iz2 * gj00 + k.fx * ux * iz2 * gj02 - k.fy * iz2 * gj11 + k.fy * uy * iz2 * gj12;
       const float gux = -k.fx * iz * gj02, guy = -k.fy * iz * gj12;
-      if (!(P.u < -k.limx || P.u > k.limx)) { gx += gux * iz; gz -= gux * P.px * iz2; }
-      if (!(P.v < -k.limy || P.v > k.limy)) { gy += guy * iz; gz -= guy * P.py * iz2; }
+      if (!clx) { gx += gux * iz; gz -= gux * px * iz2; }
+      if (!cly) { gy += guy * iz; gz -= guy * py * iz2; }
       const float vmx = v0.x, vmy = v0.y;
-      gx += vmx * k.fx * iz; gz -= vmx * k.fx * P.px * iz2;
-      gy += vmy * k.fy * iz; gz -= vmy * k.fy * P.py * iz2;
+      gx += vmx * k.fx * iz; gz -= vmx * k.fx * px * iz2;
+      gy += vmy * k.fy * iz; gz -= vmy * k.fy * py * iz2;
       gz += v2.y;  // depth
       gmu[0] += R[0] * gx + R[3] * gy + R[6] * gz;
       gmu[1] += R[1] * gx + R[4] * gy + R[7] * gz;
@@ -201,48 +236,68 @@ __global__ __launch_bounds__(kBlock) void k_project_bwd(Geo g, const float* __re
       }
     }
   }
-  if (!valid) return;
-  // Sigma = M M^T: dL/dM = 2 gS M, M = R_q diag(s)
-  const float Gs[3][3] = {{gS[0], gS[1], gS[2]}, {gS[1], gS[3], gS[4]}, {gS[2], gS[4], gS[5]}};
-  const float sv[3] = {s0, s1, s2};
-  float M[9];
+  if (valid) {
+    // Sigma = M M^T: dL/dM = 2 gS M, M = R_q diag(s)  (fp64, see above)
+    const double Gs[3][3] = {{gS[0], gS[1], gS[2]}, {gS[1], gS[3], gS[4]}, {gS[2], gS[4], gS[5]}};
+    const double sv[3] = {s0, s1, s2};
+    double M[9];
 #pragma unroll
-  for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < 3; ++i)
 #pragma unroll
-    for (int jj = 0; jj < 3; ++jj) M[3 * i + jj] = qr.R[3 * i + jj] * sv[jj];
-  float gsc[3] = {0.f, 0.f, 0.f}, GR[9];
+      for (int jj = 0; jj < 3; ++jj) M[3 * i + jj] = (double)qr.R[3 * i + jj] * sv[jj];
+    double gsc[3] = {0., 0., 0.}, GR[9];
 #pragma unroll
-  for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < 3; ++i)
 #pragma unroll
-    for (int jj = 0; jj < 3; ++jj) {
-      const float gm = 2.0f * (Gs[i][0] * M[jj] + Gs[i][1] * M[3 + jj] + Gs[i][2] * M[6 + jj]);
-      gsc[jj] += gm * qr.R[3 * i + jj];
-      GR[3 * i + jj] = gm * sv[jj];
-    }
-  const float w = qr.w, x = qr.x, y = qr.y, z = qr.z;
-  float vw = 0.f, vx = 0.f, vy = 0.f, vz = 0.f;
-  vy += -4.f * y * GR[0]; vz += -4.f * z * GR[0];
-  vw += -2.f * z * GR[1]; vx += 2.f * y * GR[1]; vy += 2.f * x * GR[1]; vz += -2.f * w * GR[1];
-  vw += 2.f * y * GR[2]; vx += 2.f * z * GR[2]; vy += 2.f * w * GR[2]; vz += 2.f * x * GR[2];
-  vw += 2.f * z * GR[3]; vx += 2.f * y * GR[3]; vy += 2.f * x * GR[3]; vz += 2.f * w * GR[3];
-  vx += -4.f * x * GR[4]; vz += -4.f * z * GR[4];
-  vw += -2.f * x * GR[5]; vx += -2.f * w * GR[5]; vy += 2.f * z * GR[5]; vz += 2.f * y * GR[5];
-  vw += -2.f * y * GR[6]; vx += 2.f * z * GR[6]; vy += -2.f * w * GR[6]; vz += 2.f * x * GR[6];
-  vw += 2.f * x * GR[7]; vx += 2.f * w * GR[7]; vy += 2.f * z * GR[7]; vz += 2.f * y * GR[7];
-  vx += -4.f * x * GR[8]; vy += -4.f * y * GR[8];
-  const float dq = w * vw + x * vx + y * vy + z * vz;
-  v_means[3 * n] = gmu[0];
-  v_means[3 * n + 1] = gmu[1];
-  v_means[3 * n + 2] = gmu[2];
-  reinterpret_cast<float4*>(v_quats)[n] =
-      make_float4((vw - w * dq) * qr.inv, (vx - x * dq) * qr.inv, (vy - y * dq) * qr.inv, (vz - z * dq) * qr.inv);
-  v_scales[3 * n] = gsc[0];
-  v_scales[3 * n + 1] = gsc[1];
-  v_scales[3 * n + 2] = gsc[2];
-  v_opac[n] = go;
-  float* o = v_sh + (int64_t)K * 3 * n;
-#pragma unroll
-  for (int q = 0; q < 3 * K; ++q) o[q] = gsh[q];
+      for (int jj = 0; jj < 3; ++jj) {
+        const double gm = 2.0 * (Gs[i][0] * M[jj] + Gs[i][1] * M[3 + jj] + Gs[i][2] * M[6 + jj]);
+        gsc[jj] += gm * qr.R[3 * i + jj];
+        GR[3 * i + jj] = gm * sv[jj];
+      }
+    const double w = qr.w, x = qr.x, y = qr.y, z = qr.z;
+    double vw = 0., vx = 0., vy = 0., vz = 0.;
+    vy += -4.f * y * GR[0]; vz += -4.f * z * GR[0];
+    vw += -2.f * z * GR[1]; vx += 2.f * y * GR[1]; vy += 2.f * x * GR[1]; vz += -2.f * w * GR[1];
+    vw += 2.f * y * GR[2]; vx += 2.f * z * GR[2]; vy += 2.f * w * GR[2]; vz += 2.f * x * GR[2];
+    vw += 2.f * z * GR[3]; vx += 2.f * y * GR[3]; vy += 2.f * x * GR[3]; vz += 2.f * w * GR[3];
+    vx += -4.f * x * GR[4]; vz += -4.f * z * GR[4];
+    vw += -2.f * x * GR[5]; vx += -2.f * w * GR[5]; vy += 2.f * z * GR[5]; vz += 2.f * y * GR[5];
+    vw += -2.f * y * GR[6]; vx += 2.f * z * GR[6]; vy += -2.f * w * GR[6]; vz += 2.f * x * GR[6];
+    vw += 2.f * x * GR[7]; vx += 2.f * w * GR[7]; vy += 2.f * z * GR[7]; vz += 2.f * y * GR[7];
+    vx += -4.f * x * GR[8]; vy += -4.f * y * GR[8];
+    const double dq = w * vw + x * vx + y * vy + z * vz;
+    const double qi = qr.inv;
+    v_means[3 * n] = gmu[0];
+    v_means[3 * n + 1] = gmu[1];
+    v_means[3 * n + 2] = gmu[2];
+    reinterpret_cast<float4*>(v_quats)[n] = make_float4((float)((vw - w * dq) * qi), (float)((vx - x * dq) * qi),
+                                                        (float)((vy - y * dq) * qi), (float)((vz - z * dq) * qi));
+    v_scales[3 * n] = (float)gsc[0];
+    v_scales[3 * n + 1] = (float)gsc[1];
+    v_scales[3 * n + 2] = (float)gsc[2];
+    v_opac[n] = go;
+  }
+  __syncthreads();
+  // coalesced write-back of the CTA's SH gradient block
+  float* dst = v_sh + n0 * K3;
+  for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+    const int gi = f / K3, q = f - gi * K3;
+    dst[f] = gsh_s[gi * KP + q];
+  }
+}
+
+template <int DEG>
+ss_status launch_pbwd(const Geo& g, unsigned grid, cudaStream_t st, const float* cams, const float* means,
+                      const float* quats, const float* scales, const float* sh, const uint32_t* mask,
+                      const int64_t* block_off, const float* v_screen, float* v_means, float* v_quats,
+                      float* v_scales, float* v_opacities, float* v_sh) {
+  const size_t smem = 2 * sizeof(float) * kBlock * sh_stride<DEG>();
+  ss_status s = cuda_status(
+      cudaFuncSetAttribute(k_project_bwd<DEG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "smem attr");
+  if (s) return s;
+  k_project_bwd<DEG><<<grid, kBlock, smem, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                                 v_means, v_quats, v_scales, v_opacities, v_sh);
+  return cuda_status(cudaGetLastError(), "project bwd");
 }
 
 }  // namespace ss
@@ -265,14 +320,13 @@ extern "C" ss_status ss_project_bwd(const ss_dims* dims, const float* cams, cons
   cudaStream_t st = as_stream(stream);
   const unsigned grid = (unsigned)g.blocks_per_cam;
   switch (g.deg) {
-    case 0: k_project_bwd<0><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                                      v_means, v_quats, v_scales, v_opacities, v_sh); break;
-    case 1: k_project_bwd<1><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                                      v_means, v_quats, v_scales, v_opacities, v_sh); break;
-    case 2: k_project_bwd<2><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                                      v_means, v_quats, v_scales, v_opacities, v_sh); break;
-    default: k_project_bwd<3><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                                       v_means, v_quats, v_scales, v_opacities, v_sh); break;
+    case 0: return launch_pbwd<0>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
+                                  v_quats, v_scales, v_opacities, v_sh);
+    case 1: return launch_pbwd<1>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
+                                  v_quats, v_scales, v_opacities, v_sh);
+    case 2: return launch_pbwd<2>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
+                                  v_quats, v_scales, v_opacities, v_sh);
+    default: return launch_pbwd<3>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
+                                   v_quats, v_scales, v_opacities, v_sh);
   }
-  return cuda_status(cudaGetLastError(), "project bwd");
 }

@@ -2,13 +2,25 @@
 // keys ("Spirula Studio VRAM deep-dive", buffer-cost table: double-buffered
 // isect.ids_a/b; the reference's CUDA backend calls a library sort, this one is
 // written here).  8-bit digits over the 31 depth bits (depth > 0, so bit 31 is
-// zero) and over the bits the tile ids need.  Per pass, reduce-then-scan:
-//   k_radix_hist     per 4096-key tile: digit histogram -> counts[digit][tile]
-//   scan             exclusive scan of counts (digit-major) -> offsets
-//   k_radix_scatter  per tile: stable rank of each key among equal digits
-//                    (warp match + per-warp counters), keys staged in shared
-//                    memory in digit order, then written out in contiguous runs
-// No CTA waits on another.  Equal keys keep their input order.
+// zero) and over the bits the tile ids need.
+//
+//   k_hist_all   one read of the keys: the global digit histogram of every pass
+//                (a permutation does not change them)
+//   k_bases      exclusive scan of each pass's 256 counts
+//   k_onesweep   per pass, one kernel: each CTA takes the next 4096-key tile by
+//                ticket, ranks its keys stably among equal digits (warp match +
+//                per-warp counters), publishes its digit counts and looks back
+//                over earlier tiles' published counts (decoupled look-back) for
+//                its global offsets, then writes the keys in contiguous runs
+//                from shared memory.  12 B read + 12 B written per key per pass.
+//
+// The look-back spin is bounded: after kSpinLimit polls it records an error
+// flag (reported by the call as SS_ERR_DEVICE_CHECK) and goes on.  Tiles are
+// handed out by ticket, so every tile a CTA waits on belongs to a CTA that is
+// already running and never waits on a later tile.
+//
+// The per-pass reduce-then-scan kernels below (k_radix_hist, k_radix_scatter)
+// are the simpler variant kept for reference; they are not launched.
 #include <algorithm>
 #include <utility>
 
@@ -136,6 +148,181 @@ __global__ __launch_bounds__(kSortThreads) void k_radix_scatter(const uint64_t* 
   }
 }
 
+constexpr int kMaxPasses = 8;
+constexpr uint64_t kFlagAgg = 1ull << 54;
+constexpr uint64_t kFlagPre = 2ull << 54;
+constexpr uint64_t kValMask = (1ull << 54) - 1;
+constexpr int kSpinLimit = 1 << 20;
+
+struct SortPlan {
+  int passes;
+  int shift[kMaxPasses];
+};
+
+__global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __restrict__ keys, int64_t n, SortPlan plan,
+                                                           uint32_t* __restrict__ hist) {
+  __shared__ uint32_t h[kMaxPasses][kRadix];
+  for (int i = threadIdx.x; i < kMaxPasses * kRadix; i += kSortThreads) (&h[0][0])[i] = 0;
+  __syncthreads();
+  for (int64_t i = (int64_t)blockIdx.x * kSortThreads + threadIdx.x; i < n; i += (int64_t)gridDim.x * kSortThreads) {
+    const uint64_t k = keys[i];
+    for (int p = 0; p < plan.passes; ++p) atomicAdd(&h[p][(uint32_t)(k >> plan.shift[p]) & 0xFFu], 1u);
+  }
+  __syncthreads();
+  for (int p = 0; p < plan.passes; ++p) {
+    const uint32_t v = h[p][threadIdx.x];
+    if (v) atomicAdd(&hist[p * kRadix + threadIdx.x], v);
+  }
+}
+
+// hist[p][d] -> exclusive scan over d, in place (one CTA of 256 threads).
+__global__ __launch_bounds__(kRadix) void k_bases(uint32_t* __restrict__ hist, int passes) {
+  __shared__ uint32_t wt[kRadix / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int p = 0; p < passes; ++p) {
+    const uint32_t v = hist[p * kRadix + threadIdx.x];
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += x;
+    }
+    if (lane == 31) wt[warp] = inc;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += wt[w];
+    hist[p * kRadix + threadIdx.x] = before + inc - v;
+    __syncthreads();
+  }
+}
+
+struct OnesweepSmem {
+  uint32_t wcnt[kSortWarps][kRadix];
+  uint32_t dstart[kRadix];
+  int64_t gbase[kRadix];
+  uint32_t wtot[kSortWarps + 1];
+  uint32_t tile;
+  uint64_t k[kSortTile];
+  uint32_t v[kSortTile];
+};
+
+__device__ __forceinline__ uint64_t ld_status(const uint64_t* p) {
+  return *reinterpret_cast<const volatile unsigned long long*>(p);
+}
+
+__global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __restrict__ kin,
+                                                           const uint32_t* __restrict__ vin,
+                                                           uint64_t* __restrict__ kout, uint32_t* __restrict__ vout,
+                                                           int64_t n, int shift, uint64_t epoch,
+                                                           const uint32_t* __restrict__ bases,
+                                                           uint64_t* __restrict__ status,
+                                                           uint32_t* __restrict__ ticket, uint32_t* __restrict__ err) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  OnesweepSmem& S = *reinterpret_cast<OnesweepSmem*>(smem_raw);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) S.tile = atomicAdd(ticket, 1u);
+  for (int i = threadIdx.x; i < kSortWarps * kRadix; i += kSortThreads) (&S.wcnt[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t tile = S.tile;
+  const int64_t tile0 = tile * kSortTile;
+  const int64_t base = tile0 + warp * (kSortTile / kSortWarps);
+  const uint32_t lt = (1u << lane) - 1u;
+  uint64_t kk[kSortItems];
+  uint32_t vv[kSortItems];
+  uint32_t pos[kSortItems];
+#pragma unroll
+  for (int r = 0; r < kSortItems; ++r) {
+    const int64_t i = base + r * 32 + lane;
+    const bool valid = i < n;
+    kk[r] = valid ? kin[i] : 0ull;
+    vv[r] = valid ? vin[i] : 0u;
+    const uint32_t d = valid ? (uint32_t)(kk[r] >> shift) & 0xFFu : 0x100u;
+    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+    const uint32_t before = valid ? S.wcnt[warp][d] : 0u;
+    __syncwarp();
+    if (valid && lane == 31 - __clz(peers)) S.wcnt[warp][d] = before + __popc(peers);
+    __syncwarp();
+    pos[r] = valid ? before + __popc(peers & lt) : 0xFFFFFFFFu;
+  }
+  __syncthreads();
+  {
+    const int d = threadIdx.x;
+    uint32_t run = 0;
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t t = S.wcnt[w][d];
+      S.wcnt[w][d] = run;
+      run += t;
+    }
+    // publish this tile's count of digit d, then look back for its prefix
+    uint64_t* st = status + tile * kRadix + d;
+    if (tile == 0) {
+      atomicExch(reinterpret_cast<unsigned long long*>(st), epoch | kFlagPre | run);
+    } else {
+      atomicExch(reinterpret_cast<unsigned long long*>(st), epoch | kFlagAgg | run);
+    }
+    uint64_t prefix = 0;
+    if (tile > 0) {
+      int64_t t = tile - 1;
+      int spins = 0;
+      while (true) {
+        const uint64_t sv = ld_status(status + t * kRadix + d);
+        const bool ready = (sv & ~(kValMask | kFlagAgg | kFlagPre)) == epoch && (sv & (kFlagAgg | kFlagPre));
+        if (!ready) {
+          if (++spins > kSpinLimit) {
+            atomicOr(err, 1u);
+            break;
+          }
+          __nanosleep(64);
+          continue;
+        }
+        prefix += sv & kValMask;
+        if (sv & kFlagPre) break;
+        if (--t < 0) break;
+      }
+      atomicExch(reinterpret_cast<unsigned long long*>(st), epoch | kFlagPre | (prefix + run));
+    }
+    S.gbase[d] = (int64_t)bases[d] + (int64_t)prefix;
+    // exclusive scan of the tile's digit counts -> local digit starts
+    uint32_t inc = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += x;
+    }
+    if (lane == 31) S.wtot[warp] = inc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t a = 0;
+      for (int w = 0; w < kSortWarps; ++w) {
+        const uint32_t t = S.wtot[w];
+        S.wtot[w] = a;
+        a += t;
+      }
+    }
+    __syncthreads();
+    S.dstart[d] = S.wtot[warp] + inc - run;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kSortItems; ++r) {
+    if (pos[r] == 0xFFFFFFFFu) continue;
+    const uint32_t d = (uint32_t)(kk[r] >> shift) & 0xFFu;
+    const uint32_t lp = S.dstart[d] + S.wcnt[warp][d] + pos[r];
+    S.k[lp] = kk[r];
+    S.v[lp] = vv[r];
+  }
+  __syncthreads();
+  const int cnt = (int)min64(kSortTile, n - tile0);
+  for (int i = threadIdx.x; i < cnt; i += kSortThreads) {
+    const uint64_t key = S.k[i];
+    const uint32_t d = (uint32_t)(key >> shift) & 0xFFu;
+    const int64_t gpos = S.gbase[d] + (i - (int64_t)S.dstart[d]);
+    kout[gpos] = key;
+    vout[gpos] = S.v[i];
+  }
+}
+
 // tile_off[t] = first sorted index whose tile id is >= t; tile_off[ntiles] = n.
 __global__ void k_tile_ranges(const uint64_t* __restrict__ keys, int64_t n, int64_t ntiles,
                               int64_t* __restrict__ tile_off) {
@@ -154,10 +341,13 @@ int tile_bits(int64_t ntiles) {
 
 int sort_passes(int64_t ntiles) { return 4 + (tile_bits(ntiles) + 7) / 8; }
 
+// Scratch layout: hist [kMaxPasses][256] u32 | tickets [kMaxPasses] u32 |
+// error flag u32 | look-back status [tiles][256] u64.
+size_t sort_status_offset() { return align_up(kMaxPasses * kRadix * 4 + kMaxPasses * 4 + 4, 256); }
+
 size_t sort_temp_bytes(int64_t n) {
   const int64_t tiles = ceil_div(max64(n, 1), kSortTile);
-  const size_t counts = align_up((size_t)tiles * kRadix * 4, 256);
-  return 2 * counts + scan_temp_bytes(tiles * kRadix) + 256;
+  return sort_status_offset() + (size_t)tiles * kRadix * 8;
 }
 
 }  // namespace ss
@@ -181,46 +371,51 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   if (n == 0) return cuda_status(cudaMemsetAsync(tile_off, 0, sizeof(int64_t) * (g.n_tiles + 1), st), "memset");
   if (!keys_a || !vals_a || !keys_b || !vals_b) return invalid("null keys/vals");
   if (!temp || temp_bytes < sort_temp_bytes(n)) return invalid("temp too small");
-  static bool attr_set = false;
-  if (!attr_set) {
-    ss_status s = cuda_status(cudaFuncSetAttribute(k_radix_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)sizeof(ScatterSmem)),
-                              "set smem attribute");
-    if (s) return s;
-    attr_set = true;
-  }
+  ss_status s = cuda_status(cudaFuncSetAttribute(k_onesweep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)sizeof(OnesweepSmem)),
+                            "set smem attribute");
+  if (s) return s;
   const int64_t tiles = ceil_div(n, kSortTile);
-  const size_t counts_b = align_up((size_t)tiles * kRadix * 4, 256);
-  uint32_t* counts = reinterpret_cast<uint32_t*>(temp);
-  uint32_t* offs = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(temp) + counts_b);
-  char* scan_tmp = reinterpret_cast<char*>(temp) + 2 * counts_b;
-  int64_t* scan_total = reinterpret_cast<int64_t*>(scan_tmp + scan_temp_bytes(tiles * kRadix));
+  char* tb = reinterpret_cast<char*>(temp);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(tb);
+  uint32_t* tickets = hist + kMaxPasses * kRadix;
+  uint32_t* err = tickets + kMaxPasses;
+  uint64_t* status = reinterpret_cast<uint64_t*>(tb + sort_status_offset());
+  s = cuda_status(cudaMemsetAsync(temp, 0, sort_status_offset() + (size_t)tiles * kRadix * 8, st), "memset");
+  if (s) return s;
+  SortPlan plan{};
+  plan.passes = passes;
+  for (int p = 0; p < passes; ++p) plan.shift[p] = p < 4 ? 8 * p : 32 + 8 * (p - 4);
+  const unsigned hgrid = (unsigned)min64(tiles, 148 * 8);
+  k_hist_all<<<hgrid, kSortThreads, 0, st>>>(keys_a, n, plan, hist);
+  k_bases<<<1, kRadix, 0, st>>>(hist, passes);
+  s = cuda_status(cudaGetLastError(), "radix histogram");
+  if (s) return s;
   uint64_t* kin = keys_a;
   uint32_t* vin = vals_a;
   uint64_t* kout = keys_b;
   uint32_t* vout = vals_b;
-  const int tb = tile_bits(g.n_tiles);
   for (int p = 0; p < passes; ++p) {
-    const int shift = p < 4 ? 8 * p : 32 + 8 * (p - 4);
-    (void)tb;
-    k_radix_hist<<<(unsigned)tiles, kSortThreads, 0, st>>>(kin, n, shift, counts, tiles);
-    ss_status s = cuda_status(cudaGetLastError(), "radix histogram");
-    if (s) return s;
-    ScanSrc src{};
-    src.kind = SCAN_U32;
-    src.u32 = counts;
-    s = scan_phase1(src, tiles * kRadix, scan_tmp, scan_total, st);
-    if (s) return s;
-    s = scan_phase2<uint32_t>(src, tiles * kRadix, scan_tmp, offs, st);
-    if (s) return s;
-    k_radix_scatter<<<(unsigned)tiles, kSortThreads, sizeof(ScatterSmem), st>>>(kin, vin, kout, vout, n, shift,
-                                                                                offs, tiles);
-    s = cuda_status(cudaGetLastError(), "radix scatter");
+    const uint64_t epoch = (uint64_t)(p + 1) << 56;
+    k_onesweep<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
+        kin, vin, kout, vout, n, plan.shift[p], epoch, hist + p * kRadix, status, tickets + p, err);
+    s = cuda_status(cudaGetLastError(), "radix pass");
     if (s) return s;
     std::swap(kin, kout);
     std::swap(vin, vout);
   }
   const unsigned grid = (unsigned)ceil_div(n + 1, 256);
   k_tile_ranges<<<grid, 256, 0, st>>>(kin, n, g.n_tiles, tile_off);
-  return cuda_status(cudaGetLastError(), "tile ranges");
+  s = cuda_status(cudaGetLastError(), "tile ranges");
+  if (s) return s;
+  uint32_t herr = 0;
+  s = cuda_status(cudaMemcpyAsync(&herr, err, 4, cudaMemcpyDeviceToHost, st), "copy sort flag");
+  if (s) return s;
+  s = cuda_status(cudaStreamSynchronize(st), "sort");
+  if (s) return s;
+  if (herr) {
+    set_error("ss_sort_isects: look-back wait exceeded its limit");
+    return SS_ERR_DEVICE_CHECK;
+  }
+  return SS_OK;
 }

@@ -28,7 +28,8 @@ PMASK_BLOCK = 128
 TILE = 16
 
 EXPORTS = ("ss_size", "ss_workspace_bytes", "ss_status_string", "ss_last_error", "ss_project_packed",
-           "ss_intersect_tiles", "ss_sort_isects", "ss_rasterize_fwd", "ss_rasterize_bwd", "ss_project_bwd")
+           "ss_intersect_tiles", "ss_sort_isects", "ss_rasterize_fwd", "ss_rasterize_fwd_counts",
+           "ss_rasterize_bwd", "ss_project_bwd")
 
 
 class ss_dims(ct.Structure):
@@ -67,10 +68,11 @@ def lib() -> ct.CDLL:
         L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
         L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, P, sz, P, ct.POINTER(i32), P]
         L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P]
+        L.ss_rasterize_fwd_counts.argtypes = [D, P, P, P, P, P, P, P, P]
         L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, i64, P]
         L.ss_project_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
         for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_rasterize_fwd",
-                  "ss_rasterize_bwd", "ss_project_bwd"):
+                  "ss_rasterize_fwd_counts", "ss_rasterize_bwd", "ss_project_bwd"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -147,6 +149,20 @@ def ss_sort_isects(d, keys_a, vals_a, keys_b, vals_b, n, temp, tile_off, stream=
 def ss_rasterize_fwd(d, screen, vals, tile_off, img, T_final, last_id, stream=None):
     _check(lib().ss_rasterize_fwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(img), _p(T_final),
                                   _p(last_id), _stream(stream)), "ss_rasterize_fwd")
+
+
+def ss_rasterize_fwd_counts(d, screen, vals, tile_off, img, T_final, last_id, counts, stream=None):
+    _check(lib().ss_rasterize_fwd_counts(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(img), _p(T_final),
+                                         _p(last_id), _p(counts), _stream(stream)), "ss_rasterize_fwd_counts")
+
+
+def raster_work(d, step) -> dict:
+    """Exact per-launch work counts of the rasterizers for the step's last
+    forward (runs the counting forward once; not part of any timed region)."""
+    counts = torch.zeros(5, dtype=torch.int64, device=step.dev)
+    ss_rasterize_fwd_counts(d, step.screen, step.vals, step.tile_off, step.img, step.T, step.last, counts)
+    c = [int(x) for x in counts.cpu().tolist()]
+    return dict(evals=c[0], exps=c[1], comps=c[2], bwd_evals=c[3], bwd_exps=c[4])
 
 
 def ss_rasterize_bwd(d, screen, vals, tile_off, T_final, last_id, v_img, v_T, v_screen, nnz, stream=None):

@@ -166,6 +166,18 @@ ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, const uint3
                            float* img, float* T_final, int32_t* last_id, void* stream);
 
 /*
+ * Measurement helper, not part of the step: ss_rasterize_fwd plus exact work
+ * counts summed over all pixels into counts[5] (device uint64, zeroed by the
+ * call): [0] entries evaluated (up to and including the one that stopped the
+ * pixel), [1] entries whose exp was evaluated, [2] entries composited,
+ * [3] entries the backward replays (tile start to last_id), [4] exps among
+ * those.  Used to state the rasterizers' arithmetic work for a roofline.
+ */
+ss_status ss_rasterize_fwd_counts(const ss_dims* dims, const float* screen, const uint32_t* vals,
+                                  const int64_t* tile_off, float* img, float* T_final, int32_t* last_id,
+                                  uint64_t* counts, void* stream);
+
+/*
  * Backward rasterizer ("Spirula Studio backward pass", section 4): per pixel,
  * reverse replay from last_id using the saved state (no re-intersection),
  * splitting v_img (and v_T, may be NULL) by each entry's alpha contribution.

@@ -383,7 +383,7 @@ struct Contrib {
 template <typename R>
 void composite_pixel(const double* screen, const uint32_t* vals, int64_t beg, int64_t end, R px, R py,
                      R* rgb_out, R* T_out, int64_t* last_out, std::vector<Contrib>* list,
-                     int64_t* n_eval = nullptr) {
+                     int64_t* n_eval = nullptr, int64_t* n_comp = nullptr) {
   R T = R(1), Cc[3] = {R(0), R(0), R(0)};
   int64_t last = -1;
   const R alpha_min = R(1) / R(255);
@@ -403,6 +403,7 @@ void composite_pixel(const double* screen, const uint32_t* vals, int64_t beg, in
     for (int ch = 0; ch < 3; ++ch) Cc[ch] = fmaR(g.rgb[ch], w, Cc[ch]);
     T = Tn;
     last = i;
+    if (n_comp) ++*n_comp;
     if (list) list->push_back({i, !(oe < R(0.99))});
   }
   for (int ch = 0; ch < 3; ++ch) rgb_out[ch] = Cc[ch];
@@ -839,17 +840,19 @@ int orc_tile_ranges(const uint64_t* keys, int64_t n, int64_t n_tiles, int64_t* t
 // Forward rasterizer, one pixel at a time.  img [C][H][W][3], T_final and
 // last_id [C][H][W].  precision 0: fp32 (canonical), 1: fp64.
 // Optional evals[npix]: entries each pixel evaluated (up to and including the
-// one that stopped it).
+// one that stopped it); comps[npix]: entries composited.
 int orc_rasterize_fwd(const orc_dims* d, const double* screen, const uint32_t* vals, const int64_t* tile_off,
                       int precision, double* img, double* T_final, int64_t* last_id, int64_t* evals,
-                      int nthreads) {
+                      int64_t* comps, int nthreads) {
   set_threads(nthreads);
   Geo geo = geometry(d);
   const int64_t npix = (int64_t)d->C * d->H * d->W;
 #pragma omp parallel for schedule(dynamic, 1024)
   for (int64_t p = 0; p < npix; ++p) {
     int64_t* ev = evals ? evals + p : nullptr;
+    int64_t* cp = comps ? comps + p : nullptr;
     if (ev) *ev = 0;
+    if (cp) *cp = 0;
     int64_t c = p / ((int64_t)d->H * d->W), rem = p % ((int64_t)d->H * d->W);
     int64_t j = rem / d->W, i = rem % d->W;
     int64_t t = c * geo.tiles_per_cam + (j / kTile) * geo.tiles_x + (i / kTile);
@@ -857,13 +860,13 @@ int orc_rasterize_fwd(const orc_dims* d, const double* screen, const uint32_t* v
     if (precision == 0) {
       float rgb[3], T;
       composite_pixel<float>(screen, vals, tile_off[t], tile_off[t + 1], (float)i + 0.5f, (float)j + 0.5f, rgb, &T,
-                             &last, nullptr, ev);
+                             &last, nullptr, ev, cp);
       for (int ch = 0; ch < 3; ++ch) img[3 * p + ch] = rgb[ch];
       T_final[p] = T;
     } else {
       double rgb[3], T;
       composite_pixel<double>(screen, vals, tile_off[t], tile_off[t + 1], (double)i + 0.5, (double)j + 0.5, rgb,
-                              &T, &last, nullptr, ev);
+                              &T, &last, nullptr, ev, cp);
       for (int ch = 0; ch < 3; ++ch) img[3 * p + ch] = rgb[ch];
       T_final[p] = T;
     }

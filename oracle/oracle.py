@@ -52,7 +52,7 @@ def lib():
         L.orc_intersect.argtypes = [P, P, P, P, i64, i32, P, P, i64, P]
         L.orc_sort.argtypes = [P, P, i64]
         L.orc_tile_ranges.argtypes = [P, i64, i64, P]
-        L.orc_rasterize_fwd.argtypes = [P, P, P, P, i32, P, P, P, P, i32]
+        L.orc_rasterize_fwd.argtypes = [P, P, P, P, i32, P, P, P, P, P, i32]
         L.orc_rasterize_bwd.argtypes = [P, P, P, P, P, P, i32, i64, P, i32]
         L.orc_project_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i64, P, i32, P, P, P, P, P]
         for f in ("orc_project", "orc_row_boxes", "orc_count_tiles", "orc_intersect", "orc_sort",
@@ -209,10 +209,12 @@ def rasterize_fwd(scene, screen, vals_sorted, tile_off, precision: int = 0, nthr
     T = np.zeros((scene.C, scene.H, scene.W))
     last = np.zeros((scene.C, scene.H, scene.W), np.int64)
     ev = np.zeros((scene.C, scene.H, scene.W), np.int64) if evals else None
+    cp = np.zeros((scene.C, scene.H, scene.W), np.int64) if evals else None
     lib().orc_rasterize_fwd(ct.byref(d), _p(_c(screen, np.float64)), _p(_c(vals_sorted, np.uint32)),
-                            _p(_c(tile_off, np.int64)), precision, _p(img), _p(T), _p(last), _p(ev), nthreads)
+                            _p(_c(tile_off, np.int64)), precision, _p(img), _p(T), _p(last), _p(ev), _p(cp),
+                            nthreads)
     if evals:
-        return img, T, last, ev
+        return img, T, last, ev, cp
     return img, T, last
 
 

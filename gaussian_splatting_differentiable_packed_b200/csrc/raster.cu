@@ -4,39 +4,50 @@
 // reuses them without re-intersecting, splits each pixel's gradient by alpha
 // contribution and sums per Gaussian with atomics).
 //
-// One CTA per 16x16 tile, one thread per pixel.  Each batch of the tile's
-// sorted entries is gathered once into shared memory (three 16-byte loads per
-// 48-byte screen row) and evaluated by all 256 pixels.
+// One CTA of 128 threads per 16x16 tile.  Each thread owns a vertical pair of
+// pixels (same column, rows j and j+1), so the pair shares dx and the sigma and
+// exp arithmetic runs on packed fp32 pairs (FFMA2/FMUL2/FADD2: each lane of the
+// pair is rounded exactly like the scalar operation, so the canonical order is
+// kept bit for bit).  Warp w owns the 16x4 region of rows 4w..4w+3.  Each batch
+// of 256 sorted entries is gathered once into shared memory (three 16-byte
+// loads per 48-byte screen row) and each warp builds its own candidate list by
+// ballot, skipping entries that provably miss its region (see warp_culled).
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 
 namespace ss {
 
-constexpr int kPix = kTile * kTile;  // 256 threads
-constexpr int kFwdBatch = 256;
-constexpr int kBwdBatch = 64;
+constexpr int kRThreads = 128;
+constexpr int kBatch = 256;
+constexpr int kRedF = 12;
 
-__device__ __forceinline__ void tile_coords(const Geo& g, int64_t tile, int& c, int& i, int& j) {
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 f2s(float a) { return make_float2(a, a); }
+
+// Pixel-pair coordinates of this thread: column i, rows j and j+1.
+__device__ __forceinline__ void tile_coords(const Geo& g, int64_t tile, int& c, int& tx0, int& ty0, int& i, int& j) {
   c = (int)(tile / g.tiles_per_cam);
   const int rem = (int)(tile - (int64_t)c * g.tiles_per_cam);
   const int ty = rem / g.tiles_x, tx = rem - ty * g.tiles_x;
-  i = tx * kTile + (threadIdx.x & (kTile - 1));
-  j = ty * kTile + (threadIdx.x >> 4);
+  tx0 = tx * kTile;
+  ty0 = ty * kTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  i = tx0 + (lane & 15);
+  j = ty0 + 4 * warp + 2 * (lane >> 4);
 }
 
 // ---------------------------------------------------------------------------
-// Warp culling.  A warp owns a 16x2 strip of the tile (rows 2w, 2w+1).  For an
-// entry with o <= 1 every pixel whose computed sigma exceeds 5.6 is skipped by
-// the per-pixel test anyway (o*exp(-sigma) < 1/255).  The staged half-extents
-// (hx, hy) bound the ellipse {sigma <= 5.7} of the stored conic exactly
-// (computed in fp64 with a margin); a strip outside that box has exact sigma
-// > 5.7 at every pixel, and when kterm*(Dx^2 + Dy^2) <= 1e5 the fp32 rounding
-// of the canonical sigma is below 0.04, so the computed sigma exceeds 5.6 too:
-// skipping the entry for the whole warp takes exactly the per-pixel decision.
+// Staged entry.  thr = 5.6 when o <= 1 (then sigma > 5.6 implies
+// o*exp(-sigma) < 1/255: the pixel skips the entry without the exp), +inf
+// otherwise.  (hx, hy) bound the ellipse {sigma <= 5.7} of the stored conic
+// (fp64 with a margin; +inf when o > 1 or the conic is not positive definite).
 struct Stage {
   float4 a;  // x, y, 0.5*ca, cb
   float4 b;  // 0.5*cc, o, r, g
-  float4 c;  // b, hx, hy, kterm
+  float4 c;  // b, hx, hy, kterm = |ha| + |hc| + |cb|
+  float thr;
+  uint32_t row;
+  float pad0, pad1;
 };
 
 __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint32_t r, Stage& st) {
@@ -44,7 +55,8 @@ __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint
   const float4 r0 = row[0], r1 = row[1], r2 = row[2];
   st.a = make_float4(r0.x, r0.y, mul(0.5f, r0.z), r0.w);
   st.b = make_float4(mul(0.5f, r1.x), r1.y, r1.z, r1.w);
-  float hx = __int_as_float(0x7f800000), hy = hx;
+  const float inf = __int_as_float(0x7f800000);
+  float hx = inf, hy = inf;
   const double dq = (double)r0.z * (double)r1.x - (double)r0.w * (double)r0.w;
   if (r1.y <= 1.0f && dq > 0.0) {
     hx = (float)(sqrt(11.4 * (double)r1.x / dq) * 1.001 + 1e-3);
@@ -52,9 +64,17 @@ __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint
   }
   const float kterm = 0.5f * fabsf(r0.z) + 0.5f * fabsf(r1.x) + fabsf(r0.w);
   st.c = make_float4(r2.x, hx, hy, kterm);
+  st.thr = r1.y <= 1.0f ? SS_SIGMA_SKIP : inf;
+  st.row = r;
 }
 
-// True when the entry can be skipped by the whole warp (see above).
+// Warp culling.  For an entry with o <= 1 every pixel whose computed sigma
+// exceeds 5.6 skips the entry.  A region outside the box (hx, hy) of the
+// ellipse {sigma <= 5.7} has exact sigma > 5.7 at every pixel centre; when
+// kterm*(Dx^2 + Dy^2) <= 1e5 (D: largest offset from the mean to the region)
+// the canonical fp32 sigma differs from the exact one by less than 0.04, so
+// every pixel of the region computes sigma > 5.6 and would skip the entry:
+// skipping it for the whole warp takes exactly the per-pixel decision.
 __device__ __forceinline__ bool warp_culled(const Stage& st, float x_lo, float x_hi, float y_lo, float y_hi) {
   const float mx = st.a.x, my = st.a.y;
   const float ex = fmaxf(fmaxf(x_lo - mx, mx - x_hi), 0.0f);
@@ -65,86 +85,151 @@ __device__ __forceinline__ bool warp_culled(const Stage& st, float x_lo, float x
   return st.c.w * (Dx * Dx + Dy * Dy) <= 1e5f;
 }
 
-// COUNT adds per-pixel work counters (measurement helper): entries evaluated,
-// exps evaluated, entries composited; and for the backward replay (entries up
-// to last_id): entries replayed and exps evaluated.  The counts follow the
-// per-pixel definition (warp culling does not change them).
+// sigma of the pixel pair in the canonical order (see gauss_sigma).
+__device__ __forceinline__ float2 sigma_pair(const Stage& st, float dx, float2 dy) {
+  const float t = mul(st.a.w, dx);                       // cb*dx
+  float2 s = __fmul2_rn(f2s(t), dy);                     // (cb*dx)*dy
+  s = __ffma2_rn(__fmul2_rn(f2s(st.b.x), dy), dy, s);    // fma(hc*dy, dy, s)
+  const float v = mul(st.a.z, dx);                       // ha*dx
+  return __ffma2_rn(f2s(v), f2s(dx), s);                 // fma(ha*dx, dx, s)
+}
+
+// exp_neg on a pair, each lane exactly as the scalar version.
+__device__ __forceinline__ float2 exp_neg_pair(float2 x) {
+  const float2 t = __fmul2_rn(x, f2s(0x1.715476p+0f));
+  const float2 kf = f2(rintf(t.x), rintf(t.y));
+  float2 r = __ffma2_rn(kf, f2s(-0x1.62e4p-1f), x);
+  r = __ffma2_rn(kf, f2s(-0x1.7f7d1cp-20f), r);
+  float2 p = f2s(0x1.a01a02p-13f);
+  p = __ffma2_rn(p, r, f2s(0x1.6c16c2p-10f));
+  p = __ffma2_rn(p, r, f2s(0x1.111112p-7f));
+  p = __ffma2_rn(p, r, f2s(0x1.555556p-5f));
+  p = __ffma2_rn(p, r, f2s(0x1.555556p-3f));
+  p = __ffma2_rn(p, r, f2s(0.5f));
+  p = __ffma2_rn(p, r, f2s(1.0f));
+  p = __ffma2_rn(p, r, f2s(1.0f));
+  const uint32_t ex = ((uint32_t)((int)kf.x + 127)) << 23, ey = ((uint32_t)((int)kf.y + 127)) << 23;
+  float2 e = __fmul2_rn(p, f2(__uint_as_float(ex), __uint_as_float(ey)));
+  if (x.x < -87.0f) e.x = 0.0f;
+  if (x.y < -87.0f) e.y = 0.0f;
+  return e;
+}
+
+// One pixel's front-to-back step for an entry whose sigma passed the tests.
+__device__ __forceinline__ void composite(const Stage& st, float oe, float amin, int64_t idx, float& T, float& C0,
+                                          float& C1, float& C2, int64_t& last, bool& done, unsigned long long& ncomp) {
+  const float alpha = fminf(SS_ALPHA_MAX, oe);
+  if (alpha < amin) return;
+  const float Tn = mul(T, sub(1.0f, alpha));
+  if (Tn < SS_T_STOP) {
+    done = true;
+    return;
+  }
+  const float w = mul(alpha, T);
+  C0 = fma_(st.b.z, w, C0);
+  C1 = fma_(st.b.w, w, C1);
+  C2 = fma_(st.c.x, w, C2);
+  T = Tn;
+  last = idx;
+  ++ncomp;
+}
+
+// COUNT adds work counters (measurement helper): entries evaluated per pixel
+// (up to and including the stopping one), exps evaluated, entries composited,
+// entries the backward replays (tile start to last_id) and exps among those.
+// In COUNT mode no entry is culled, so the counts follow the per-pixel
+// definition.
 template <bool COUNT>
-__global__ __launch_bounds__(kPix) void k_raster_fwd(Geo g, const float* __restrict__ screen,
-                                                     const uint32_t* __restrict__ vals,
-                                                     const int64_t* __restrict__ tile_off, float* __restrict__ img,
-                                                     float* __restrict__ T_final, int32_t* __restrict__ last_id,
-                                                     unsigned long long* __restrict__ counts) {
-  __shared__ Stage s_e[kFwdBatch];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__global__ __launch_bounds__(kRThreads) void k_raster_fwd(Geo g, const float* __restrict__ screen,
+                                                          const uint32_t* __restrict__ vals,
+                                                          const int64_t* __restrict__ tile_off,
+                                                          float* __restrict__ img, float* __restrict__ T_final,
+                                                          int32_t* __restrict__ last_id,
+                                                          unsigned long long* __restrict__ counts) {
+  __shared__ Stage s_e[kBatch];
+  const int lane = threadIdx.x & 31;
   const int64_t tile = blockIdx.x;
-  int c, i, j;
-  tile_coords(g, tile, c, i, j);
-  const bool inside = i < g.W && j < g.H;
-  const float px = add((float)i, 0.5f), py = add((float)j, 0.5f);
-  const float x_lo = (float)(i - (i & (kTile - 1))) + 0.5f, x_hi = x_lo + 15.0f;
-  const float y_lo = (float)(j - (j & 1)) + 0.5f, y_hi = y_lo + 1.0f;
+  int c, tx0, ty0, i, j;
+  tile_coords(g, tile, c, tx0, ty0, i, j);
+  const bool inA = i < g.W && j < g.H, inB = i < g.W && j + 1 < g.H;
+  const float px = add((float)i, 0.5f);
+  const float2 npy = f2(-add((float)j, 0.5f), -add((float)(j + 1), 0.5f));
+  const float x_lo = (float)tx0 + 0.5f, x_hi = x_lo + 15.0f;
+  const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f, y_hi = y_lo + 3.0f;
   const int64_t beg = tile_off[tile], end = tile_off[tile + 1];
   const float amin = alpha_min();
-  float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
-  int64_t last = -1;
-  bool done = !inside;
-  unsigned long long n_eval = 0, n_exp = 0, n_comp = 0, n_exp_last = 0;
-  for (int64_t b0 = beg; b0 < end; b0 += kFwdBatch) {
-    if (__syncthreads_count(done) == kPix) break;
-    const int64_t idx = b0 + threadIdx.x;
-    if (idx < end) stage_row(screen, vals[idx], s_e[threadIdx.x]);
+  float TA = 1.0f, A0 = 0.0f, A1 = 0.0f, A2 = 0.0f, TB = 1.0f, B0 = 0.0f, B1 = 0.0f, B2 = 0.0f;
+  int64_t lastA = -1, lastB = -1;
+  bool doneA = !inA, doneB = !inB;
+  unsigned long long n_eval = 0, n_exp = 0, n_comp = 0, n_expA_last = 0, n_expB_last = 0, n_expA = 0, n_expB = 0;
+  for (int64_t b0 = beg; b0 < end; b0 += kBatch) {
+    if (__syncthreads_count(doneA && doneB) == kRThreads) break;
+    for (int t = threadIdx.x; t < kBatch; t += kRThreads)
+      if (b0 + t < end) stage_row(screen, vals[b0 + t], s_e[t]);
     __syncthreads();
-    if (__all_sync(0xffffffffu, done)) continue;
-    const int cnt = (int)min64(kFwdBatch, end - b0);
-    for (int q = 0; q < kFwdBatch / 32; ++q) {
-      if (q * 32 >= cnt) break;
+    if (__all_sync(0xffffffffu, doneA && doneB)) continue;
+    const int cnt = (int)min64(kBatch, end - b0);
+    for (int q = 0; q * 32 < cnt; ++q) {
       const int e = q * 32 + lane;
-      uint32_t bits = __ballot_sync(0xffffffffu, e < cnt && (COUNT || !warp_culled(s_e[e], x_lo, x_hi, y_lo, y_hi)));
+      uint32_t bits =
+          __ballot_sync(0xffffffffu, e < cnt && (COUNT || !warp_culled(s_e[e], x_lo, x_hi, y_lo, y_hi)));
       while (bits) {
         const int k = q * 32 + __ffs(bits) - 1;
         bits &= bits - 1;
-        if (done) continue;
-        if (COUNT) ++n_eval;
+        if (doneA && doneB) continue;
         const Stage& st = s_e[k];
-        const float dx = sub(st.a.x, px), dy = sub(st.a.y, py);
-        const float sig = gauss_sigma(st.a.z, st.a.w, st.b.x, dx, dy);
-        if (sig < 0.0f) continue;
-        if (sig > SS_SIGMA_SKIP && st.b.y <= 1.0f) continue;  // o*exp(-sig) < 1/255 guaranteed
-        if (COUNT) ++n_exp;
-        const float ev = exp_neg(-sig);
-        const float alpha = fminf(SS_ALPHA_MAX, mul(st.b.y, ev));
-        if (alpha < amin) continue;
-        const float Tn = mul(T, sub(1.0f, alpha));
-        if (Tn < SS_T_STOP) {
-          done = true;
-          continue;
+        if (COUNT) n_eval += (doneA ? 0 : 1) + (doneB ? 0 : 1);
+        const float dx = sub(st.a.x, px);
+        const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
+        const float2 sig = sigma_pair(st, dx, dy);
+        const bool needA = !doneA && !(sig.x < 0.0f) && !(sig.x > st.thr);
+        const bool needB = !doneB && !(sig.y < 0.0f) && !(sig.y > st.thr);
+        if (!(needA || needB)) continue;
+        const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
+        const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
+        const int64_t idx = b0 + k;
+        if (needA) {
+          if (COUNT) {
+            ++n_exp;
+            ++n_expA;
+          }
+          const int64_t before = lastA;
+          composite(st, oe.x, amin, idx, TA, A0, A1, A2, lastA, doneA, n_comp);
+          if (COUNT && lastA != before) n_expA_last = n_expA;
         }
-        const float w = mul(alpha, T);
-        C0 = fma_(st.b.z, w, C0);
-        C1 = fma_(st.b.w, w, C1);
-        C2 = fma_(st.c.x, w, C2);
-        T = Tn;
-        last = b0 + k;
-        if (COUNT) {
-          ++n_comp;
-          n_exp_last = n_exp;
+        if (needB) {
+          if (COUNT) {
+            ++n_exp;
+            ++n_expB;
+          }
+          const int64_t before = lastB;
+          composite(st, oe.y, amin, idx, TB, B0, B1, B2, lastB, doneB, n_comp);
+          if (COUNT && lastB != before) n_expB_last = n_expB;
         }
       }
-      if (__all_sync(0xffffffffu, done)) break;
+      if (__all_sync(0xffffffffu, doneA && doneB)) break;
     }
   }
-  if (inside) {
-    const int64_t pix = ((int64_t)c * g.H + j) * g.W + i;
-    img[3 * pix] = C0;
-    img[3 * pix + 1] = C1;
-    img[3 * pix + 2] = C2;
-    T_final[pix] = T;
-    last_id[pix] = (int32_t)last;
+  const int64_t pixA = ((int64_t)c * g.H + j) * g.W + i;
+  if (inA) {
+    img[3 * pixA] = A0;
+    img[3 * pixA + 1] = A1;
+    img[3 * pixA + 2] = A2;
+    T_final[pixA] = TA;
+    last_id[pixA] = (int32_t)lastA;
+  }
+  if (inB) {
+    const int64_t pixB = pixA + g.W;
+    img[3 * pixB] = B0;
+    img[3 * pixB + 1] = B1;
+    img[3 * pixB + 2] = B2;
+    T_final[pixB] = TB;
+    last_id[pixB] = (int32_t)lastB;
   }
   if (COUNT) {
-    const unsigned long long replay = last >= 0 ? (unsigned long long)(last - beg + 1) : 0ull;
-    unsigned long long v[5] = {n_eval, n_exp, n_comp, replay, n_exp_last};
+    const unsigned long long replay = (lastA >= 0 ? (unsigned long long)(lastA - beg + 1) : 0ull) +
+                                      (lastB >= 0 ? (unsigned long long)(lastB - beg + 1) : 0ull);
+    unsigned long long v[5] = {n_eval, n_exp, n_comp, replay, n_expA_last + n_expB_last};
 #pragma unroll
     for (int q = 0; q < 5; ++q) {
       unsigned long long x = v[q];
@@ -152,6 +237,153 @@ __global__ __launch_bounds__(kPix) void k_raster_fwd(Geo g, const float* __restr
       for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
       if (lane == 0 && x) atomicAdd(&counts[q], x);
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-pixel candidate masks.  For a block of 32 staged entries (one per lane)
+// each lane computes which of the warp's 64 pixels its entry can reach: a
+// pixel is left out only if its computed sigma provably exceeds 5.6 for an
+// entry with o <= 1 (exact sigma > 5.7 outside the fp64 chord of the ellipse
+// {sigma <= 5.7}, widened by 1e-3 px, and kterm*D^2 <= 8e4 bounds the fp32
+// rounding of the canonical sigma by 0.04); such pixels skip the entry in the
+// per-pixel definition too.  A 32x32 bit transpose across the warp then gives
+// each lane the entries of the block that reach each of its two pixels.
+
+// Lane i receives bit j = bit i of lane j's word.
+template <int S, uint32_t M>
+__device__ __forceinline__ uint32_t transpose_step(uint32_t x, int lane) {
+  const uint32_t y = __shfl_xor_sync(0xffffffffu, x, S);
+  return (lane & S) ? ((x & ~M) | ((y >> S) & M)) : ((x & M) | ((y << S) & ~M));
+}
+
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+  x = transpose_step<16, 0x0000FFFFu>(x, lane);
+  x = transpose_step<8, 0x00FF00FFu>(x, lane);
+  x = transpose_step<4, 0x0F0F0F0Fu>(x, lane);
+  x = transpose_step<2, 0x33333333u>(x, lane);
+  return transpose_step<1, 0x55555555u>(x, lane);
+}
+
+// 16-bit column mask of the pixels of row centre yc (columns x_lo + c, c =
+// 0..15) inside the widened chord of {sigma <= 5.7}.
+__device__ __forceinline__ uint32_t chord_span(const Stage& st, float yc, float x_lo) {
+  const double A = st.a.z;                       // 0.5*ca
+  const double dy = (double)st.a.y - (double)yc;  // exact
+  const double B = (double)st.a.w * dy;
+  const double Cq = (double)st.b.x * dy * dy - 5.7;
+  const double disc = B * B - 4.0 * A * Cq;
+  if (disc < 0.0) return 0u;
+  const double sq = sqrt(disc);
+  const double dx1 = (-B - sq) / (2.0 * A), dx2 = (-B + sq) / (2.0 * A);
+  // pixel centre px = x_lo + c covers when mx - dx2 <= px <= mx - dx1
+  const double lo = (double)st.a.x - dx2 - (double)x_lo - 1e-3;
+  const double hi = (double)st.a.x - dx1 - (double)x_lo + 1e-3;
+  if (hi < 0.0 || lo > 15.0) return 0u;
+  const int c0 = lo <= 0.0 ? 0 : (int)ceil(lo);
+  const int c1 = hi >= 15.0 ? 15 : (int)floor(hi);
+  if (c1 < c0) return 0u;
+  return ((0xFFFFu >> (15 - c1)) >> c0) << c0;
+}
+
+// Coverage of this lane's entry over the warp's region: bit L of covA (covB)
+// set when the entry can reach lane L's upper (lower) pixel.
+__device__ __forceinline__ void entry_coverage(const Stage& st, float x_lo, float y_lo, uint32_t& covA,
+                                               uint32_t& covB) {
+  const float x_hi = x_lo + 15.0f, y_hi = y_lo + 3.0f;
+  const float mx = st.a.x, my = st.a.y;
+  const float Dx = fmaxf(fabsf(x_lo - mx), fabsf(x_hi - mx));
+  const float Dy = fmaxf(fabsf(y_lo - my), fabsf(y_hi - my));
+  const bool bounded = st.b.y <= 1.0f && st.a.z > 0.0f && st.c.w * (Dx * Dx + Dy * Dy) <= 8e4f;
+  if (!bounded) {
+    covA = covB = 0xFFFFFFFFu;
+    return;
+  }
+  const float ex = fmaxf(fmaxf(x_lo - mx, mx - x_hi), 0.0f);
+  const float ey = fmaxf(fmaxf(y_lo - my, my - y_hi), 0.0f);
+  if (ex > st.c.y || ey > st.c.z) {
+    covA = covB = 0u;
+    return;
+  }
+  const uint32_t s0 = chord_span(st, y_lo, x_lo), s1 = chord_span(st, y_lo + 1.0f, x_lo);
+  const uint32_t s2 = chord_span(st, y_lo + 2.0f, x_lo), s3 = chord_span(st, y_lo + 3.0f, x_lo);
+  covA = s0 | (s2 << 16);
+  covB = s1 | (s3 << 16);
+}
+
+__global__ __launch_bounds__(kRThreads) void k_raster_fwd_masked(Geo g, const float* __restrict__ screen,
+                                                                 const uint32_t* __restrict__ vals,
+                                                                 const int64_t* __restrict__ tile_off,
+                                                                 float* __restrict__ img, float* __restrict__ T_final,
+                                                                 int32_t* __restrict__ last_id) {
+  __shared__ Stage s_e[kBatch];
+  const int lane = threadIdx.x & 31;
+  const int64_t tile = blockIdx.x;
+  int c, tx0, ty0, i, j;
+  tile_coords(g, tile, c, tx0, ty0, i, j);
+  const bool inA = i < g.W && j < g.H, inB = i < g.W && j + 1 < g.H;
+  const float px = add((float)i, 0.5f);
+  const float2 npy = f2(-add((float)j, 0.5f), -add((float)(j + 1), 0.5f));
+  const float x_lo = (float)tx0 + 0.5f;
+  const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f;
+  const int64_t beg = tile_off[tile], end = tile_off[tile + 1];
+  const float amin = alpha_min();
+  float TA = 1.0f, A0 = 0.0f, A1 = 0.0f, A2 = 0.0f, TB = 1.0f, B0 = 0.0f, B1 = 0.0f, B2 = 0.0f;
+  int64_t lastA = -1, lastB = -1;
+  bool doneA = !inA, doneB = !inB;
+  unsigned long long ncomp = 0;
+  for (int64_t b0 = beg; b0 < end; b0 += kBatch) {
+    if (__syncthreads_count(doneA && doneB) == kRThreads) break;
+    for (int t = threadIdx.x; t < kBatch; t += kRThreads)
+      if (b0 + t < end) stage_row(screen, vals[b0 + t], s_e[t]);
+    __syncthreads();
+    if (__all_sync(0xffffffffu, doneA && doneB)) continue;
+    const int cnt = (int)min64(kBatch, end - b0);
+    for (int q = 0; q * 32 < cnt; ++q) {
+      const int e = q * 32 + lane;
+      uint32_t covA = 0u, covB = 0u;
+      if (e < cnt) entry_coverage(s_e[e], x_lo, y_lo, covA, covB);
+      uint32_t mA = warp_transpose32(covA, lane), mB = warp_transpose32(covB, lane);
+      if (doneA) mA = 0u;
+      if (doneB) mB = 0u;
+      uint32_t m = mA | mB;
+      while (m) {
+        const int b = __ffs(m) - 1;
+        m &= m - 1;
+        const bool cA = !doneA && ((mA >> b) & 1u), cB = !doneB && ((mB >> b) & 1u);
+        if (!(cA || cB)) continue;
+        const int k = q * 32 + b;
+        const Stage& st = s_e[k];
+        const float dx = sub(st.a.x, px);
+        const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
+        const float2 sig = sigma_pair(st, dx, dy);
+        const bool needA = cA && !(sig.x < 0.0f) && !(sig.x > st.thr);
+        const bool needB = cB && !(sig.y < 0.0f) && !(sig.y > st.thr);
+        if (!(needA || needB)) continue;
+        const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
+        const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
+        const int64_t idx = b0 + k;
+        if (needA) composite(st, oe.x, amin, idx, TA, A0, A1, A2, lastA, doneA, ncomp);
+        if (needB) composite(st, oe.y, amin, idx, TB, B0, B1, B2, lastB, doneB, ncomp);
+      }
+      if (__all_sync(0xffffffffu, doneA && doneB)) break;
+    }
+  }
+  const int64_t pixA = ((int64_t)c * g.H + j) * g.W + i;
+  if (inA) {
+    img[3 * pixA] = A0;
+    img[3 * pixA + 1] = A1;
+    img[3 * pixA + 2] = A2;
+    T_final[pixA] = TA;
+    last_id[pixA] = (int32_t)lastA;
+  }
+  if (inB) {
+    const int64_t pixB = pixA + g.W;
+    img[3 * pixB] = B0;
+    img[3 * pixB + 1] = B1;
+    img[3 * pixB + 2] = B2;
+    T_final[pixB] = TB;
+    last_id[pixB] = (int32_t)lastB;
   }
 }
 
@@ -189,63 +421,97 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Gradient slots per entry in the shared reduction buffer (12 = 3 float4).
-constexpr int kRedF = 12;
+// Per-pixel backward state.
+struct PixB {
+  float T, Sg, g0, g1, g2, vTT;
+  int64_t last;
+};
 
-__global__ __launch_bounds__(kPix) void k_raster_bwd(Geo g, const float* __restrict__ screen,
-                                                     const uint32_t* __restrict__ vals,
-                                                     const int64_t* __restrict__ tile_off,
-                                                     const float* __restrict__ T_final,
-                                                     const int32_t* __restrict__ last_id,
-                                                     const float* __restrict__ v_img, const float* __restrict__ v_T,
-                                                     float* __restrict__ v_screen) {
-  __shared__ Stage s_e[kBwdBatch];
-  __shared__ uint32_t s_row[kBwdBatch];
-  __shared__ uint32_t s_wmask[kBwdBatch];  // warps that contributed to each entry
-  __shared__ __align__(16) float red[kPix / 32][kBwdBatch][kRedF];
+// Reverse step of one pixel for a replayed entry (sigma already computed and
+// below the skip threshold); adds this pixel's contribution to gr[0..8].
+__device__ __forceinline__ bool pixel_grad(const Stage& st, float dx, float dy, float ev, float amin, PixB& p,
+                                           float* gr) {
+  const float oe = mul(st.b.y, ev);
+  const float alpha = fminf(SS_ALPHA_MAX, oe);
+  if (alpha < amin) return false;
+  const float ra = 1.0f / (1.0f - alpha);
+  const float Ti = p.T * ra;
+  const float w = alpha * Ti;
+  gr[6] += w * p.g0;
+  gr[7] += w * p.g1;
+  gr[8] += w * p.g2;
+  const float rgbg = st.b.z * p.g0 + st.b.w * p.g1 + st.c.x * p.g2;
+  const float v_alpha = Ti * rgbg - ra * (p.Sg + p.vTT);
+  p.Sg += w * rgbg;
+  p.T = Ti;
+  if (oe < SS_ALPHA_MAX) {
+    const float v_sig = -alpha * v_alpha;
+    gr[5] += ev * v_alpha;
+    gr[2] += v_sig * 0.5f * dx * dx;
+    gr[3] += v_sig * dx * dy;
+    gr[4] += v_sig * 0.5f * dy * dy;
+    gr[0] += v_sig * (2.0f * st.a.z * dx + st.a.w * dy);
+    gr[1] += v_sig * (st.a.w * dx + 2.0f * st.b.x * dy);
+  }
+  return true;
+}
+
+__global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __restrict__ screen,
+                                                          const uint32_t* __restrict__ vals,
+                                                          const int64_t* __restrict__ tile_off,
+                                                          const float* __restrict__ T_final,
+                                                          const int32_t* __restrict__ last_id,
+                                                          const float* __restrict__ v_img,
+                                                          const float* __restrict__ v_T,
+                                                          float* __restrict__ v_screen) {
+  __shared__ Stage s_e[kBatch];
+  __shared__ __align__(16) float red[kBatch][kRedF];  // per-entry sums over the CTA's warps
+  __shared__ uint32_t s_any[kBatch];
   __shared__ int s_maxlast;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const int64_t tile = blockIdx.x;
-  int c, i, j;
-  tile_coords(g, tile, c, i, j);
-  const bool inside = i < g.W && j < g.H;
-  const float px = add((float)i, 0.5f), py = add((float)j, 0.5f);
-  const float x_lo = (float)(i - (i & (kTile - 1))) + 0.5f, x_hi = x_lo + 15.0f;
-  const float y_lo = (float)(j - (j & 1)) + 0.5f, y_hi = y_lo + 1.0f;
+  int c, tx0, ty0, i, j;
+  tile_coords(g, tile, c, tx0, ty0, i, j);
+  const bool inA = i < g.W && j < g.H, inB = i < g.W && j + 1 < g.H;
+  const float px = add((float)i, 0.5f);
+  const float2 npy = f2(-add((float)j, 0.5f), -add((float)(j + 1), 0.5f));
+  const float x_lo = (float)tx0 + 0.5f, x_hi = x_lo + 15.0f;
+  const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f, y_hi = y_lo + 3.0f;
   const int64_t beg = tile_off[tile];
   const float amin = alpha_min();
-  float T = 1.0f, Tfin = 1.0f, g0 = 0.0f, g1 = 0.0f, g2 = 0.0f, vT = 0.0f, Sg = 0.0f;
-  int64_t last = -1;
+  for (int t = threadIdx.x; t < kBatch * kRedF; t += kRThreads) (&red[0][0])[t] = 0.0f;
+  for (int t = threadIdx.x; t < kBatch; t += kRThreads) s_any[t] = 0u;
   if (threadIdx.x == 0) s_maxlast = -1;
   __syncthreads();
-  if (inside) {
-    const int64_t pix = ((int64_t)c * g.H + j) * g.W + i;
-    last = last_id[pix];
-    Tfin = T_final[pix];
-    T = Tfin;
-    g0 = v_img[3 * pix];
-    g1 = v_img[3 * pix + 1];
-    g2 = v_img[3 * pix + 2];
-    vT = v_T ? v_T[pix] : 0.0f;
-    if (last >= 0) atomicMax(&s_maxlast, (int)last);
+  PixB pa{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1}, pb{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1};
+  const int64_t pixA = ((int64_t)c * g.H + j) * g.W + i, pixB = pixA + g.W;
+  if (inA) {
+    pa.last = last_id[pixA];
+    pa.T = T_final[pixA];
+    pa.g0 = v_img[3 * pixA];
+    pa.g1 = v_img[3 * pixA + 1];
+    pa.g2 = v_img[3 * pixA + 2];
+    pa.vTT = mul(v_T ? v_T[pixA] : 0.0f, pa.T);
+    if (pa.last >= 0) atomicMax(&s_maxlast, (int)pa.last);
+  }
+  if (inB) {
+    pb.last = last_id[pixB];
+    pb.T = T_final[pixB];
+    pb.g0 = v_img[3 * pixB];
+    pb.g1 = v_img[3 * pixB + 1];
+    pb.g2 = v_img[3 * pixB + 2];
+    pb.vTT = mul(v_T ? v_T[pixB] : 0.0f, pb.T);
+    if (pb.last >= 0) atomicMax(&s_maxlast, (int)pb.last);
   }
   __syncthreads();
   const int64_t stop = (int64_t)s_maxlast + 1;  // entries [beg, stop) can matter
-  // the warp's own last entry: entries above it need no work from this warp
-  int64_t wlast = last;
+  int64_t wlast = max64(pa.last, pb.last);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wlast = max64(wlast, __shfl_xor_sync(0xffffffffu, wlast, o));
-  const float vTT = mul(vT, Tfin);
-  for (int64_t b1 = stop; b1 > beg; b1 -= kBwdBatch) {
-    const int64_t b0 = max64(beg, b1 - kBwdBatch);
+  for (int64_t b1 = stop; b1 > beg; b1 -= kBatch) {
+    const int64_t b0 = max64(beg, b1 - kBatch);
     const int cnt = (int)(b1 - b0);
-    __syncthreads();
-    if (threadIdx.x < cnt) {
-      const uint32_t r = vals[b0 + threadIdx.x];
-      stage_row(screen, r, s_e[threadIdx.x]);
-      s_row[threadIdx.x] = r;
-      s_wmask[threadIdx.x] = 0u;
-    }
+    for (int t = threadIdx.x; t < cnt; t += kRThreads) stage_row(screen, vals[b0 + t], s_e[t]);
     __syncthreads();
     if (b0 <= wlast) {
       for (int q = (cnt - 1) / 32; q >= 0; --q) {
@@ -257,73 +523,49 @@ __global__ __launch_bounds__(kPix) void k_raster_bwd(Geo g, const float* __restr
           bits &= ~(1u << hb);
           const int k = q * 32 + hb;
           const int64_t idx = b0 + k;
+          const Stage& st = s_e[k];
           float gr[9];
 #pragma unroll
           for (int t = 0; t < 9; ++t) gr[t] = 0.0f;
           bool contrib = false;
-          if (idx <= last) {
-            const Stage& st = s_e[k];
-            const float dx = sub(st.a.x, px), dy = sub(st.a.y, py);
-            const float sig = gauss_sigma(st.a.z, st.a.w, st.b.x, dx, dy);
-            if (sig >= 0.0f && !(sig > SS_SIGMA_SKIP && st.b.y <= 1.0f)) {
-              const float ev = exp_neg(-sig);
-              const float oe = mul(st.b.y, ev);
-              const float alpha = fminf(SS_ALPHA_MAX, oe);
-              if (alpha >= amin) {
-                contrib = true;
-                const float ra = 1.0f / (1.0f - alpha);
-                const float Ti = T * ra;
-                const float w = alpha * Ti;
-                gr[6] = w * g0;
-                gr[7] = w * g1;
-                gr[8] = w * g2;
-                const float rgbg = st.b.z * g0 + st.b.w * g1 + st.c.x * g2;
-                const float v_alpha = Ti * rgbg - ra * (Sg + vTT);
-                Sg += w * rgbg;
-                T = Ti;
-                if (oe < SS_ALPHA_MAX) {
-                  const float v_sig = -alpha * v_alpha;
-                  gr[5] = ev * v_alpha;
-                  gr[2] = v_sig * 0.5f * dx * dx;
-                  gr[3] = v_sig * dx * dy;
-                  gr[4] = v_sig * 0.5f * dy * dy;
-                  gr[0] = v_sig * (2.0f * st.a.z * dx + st.a.w * dy);
-                  gr[1] = v_sig * (st.a.w * dx + 2.0f * st.b.x * dy);
-                }
-              }
+          const bool liveA = idx <= pa.last, liveB = idx <= pb.last;
+          if (liveA || liveB) {
+            const float dx = sub(st.a.x, px);
+            const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
+            const float2 sig = sigma_pair(st, dx, dy);
+            const bool needA = liveA && !(sig.x < 0.0f) && !(sig.x > st.thr);
+            const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.thr);
+            if (needA || needB) {
+              const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
+              if (needA) contrib |= pixel_grad(st, dx, dy.x, ev.x, amin, pa, gr);
+              if (needB) contrib |= pixel_grad(st, dx, dy.y, ev.y, amin, pb, gr);
             }
           }
           if (__any_sync(0xffffffffu, contrib)) {
             const float s8 = warp_reduce8(gr, lane);
             const float sb = warp_sum(gr[8]);
-            if ((lane & 3) == 0) red[warp][k][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = s8;
+            if ((lane & 3) == 0)
+              atomicAdd(&red[k][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)], s8);
             if (lane == 0) {
-              red[warp][k][8] = sb;
-              atomicOr(&s_wmask[k], 1u << warp);
+              atomicAdd(&red[k][8], sb);
+              s_any[k] = 1u;
             }
           }
         }
       }
     }
     __syncthreads();
-    // cross-warp sum over the contributing warps, one vector atomic per (entry, 16-byte quarter)
-    for (int t = threadIdx.x; t < cnt * 3; t += kPix) {
+    // one vector atomic per (entry, 16-byte quarter); the buffer is re-zeroed
+    for (int t = threadIdx.x; t < cnt * 3; t += kRThreads) {
       const int k = t / 3, q = t - 3 * k;
-      uint32_t m = s_wmask[k];
-      if (!m) continue;
-      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-      while (m) {
-        const int w = __ffs(m) - 1;
-        m &= m - 1;
-        if (q < 2) {
-          const float4 v = *reinterpret_cast<const float4*>(&red[w][k][4 * q]);
-          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-        } else {
-          sum.x += red[w][k][8];
-        }
-      }
-      atomicAdd(reinterpret_cast<float4*>(v_screen + (int64_t)s_row[k] * kRowF + 4 * q), sum);
+      if (!s_any[k]) continue;
+      float4* src = reinterpret_cast<float4*>(&red[k][4 * q]);
+      const float4 v = *src;
+      *src = make_float4(0.f, 0.f, 0.f, 0.f);
+      atomicAdd(reinterpret_cast<float4*>(v_screen + (int64_t)s_e[k].row * kRowF + 4 * q), v);
     }
+    __syncthreads();
+    for (int t = threadIdx.x; t < cnt; t += kRThreads) s_any[t] = 0u;
   }
 }
 
@@ -339,8 +581,7 @@ extern "C" ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, 
   if (((uintptr_t)screen & 15) != 0) return invalid("screen must be 16-byte aligned");
   const Geo g = geometry(*dims);
   cudaStream_t st = as_stream(stream);
-  k_raster_fwd<false><<<(unsigned)g.n_tiles, kPix, 0, st>>>(g, screen, vals, tile_off, img, T_final, last_id,
-                                                            nullptr);
+  k_raster_fwd_masked<<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, img, T_final, last_id);
   return cuda_status(cudaGetLastError(), "rasterize fwd");
 }
 
@@ -354,8 +595,8 @@ extern "C" ss_status ss_rasterize_fwd_counts(const ss_dims* dims, const float* s
   cudaStream_t st = as_stream(stream);
   ss_status s = cuda_status(cudaMemsetAsync(counts, 0, 5 * sizeof(uint64_t), st), "memset");
   if (s) return s;
-  k_raster_fwd<true><<<(unsigned)g.n_tiles, kPix, 0, st>>>(g, screen, vals, tile_off, img, T_final, last_id,
-                                                           reinterpret_cast<unsigned long long*>(counts));
+  k_raster_fwd<true><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, img, T_final, last_id,
+                                                                reinterpret_cast<unsigned long long*>(counts));
   return cuda_status(cudaGetLastError(), "rasterize fwd (counted)");
 }
 
@@ -373,7 +614,7 @@ extern "C" ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, 
     ss_status s = cuda_status(cudaMemsetAsync(v_screen, 0, (size_t)nnz * kRowF * sizeof(float), st), "memset");
     if (s) return s;
   }
-  k_raster_bwd<<<(unsigned)g.n_tiles, kPix, 0, st>>>(g, screen, vals, tile_off, T_final, last_id, v_img, v_T,
-                                                    v_screen);
+  k_raster_bwd<<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, T_final, last_id, v_img, v_T,
+                                                         v_screen);
   return cuda_status(cudaGetLastError(), "rasterize bwd");
 }

@@ -162,11 +162,21 @@ struct SortPlan {
 __global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __restrict__ keys, int64_t n, SortPlan plan,
                                                            uint32_t* __restrict__ hist) {
   __shared__ uint32_t h[kMaxPasses][kRadix];
+  const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kMaxPasses * kRadix; i += kSortThreads) (&h[0][0])[i] = 0;
   __syncthreads();
-  for (int64_t i = (int64_t)blockIdx.x * kSortThreads + threadIdx.x; i < n; i += (int64_t)gridDim.x * kSortThreads) {
-    const uint64_t k = keys[i];
-    for (int p = 0; p < plan.passes; ++p) atomicAdd(&h[p][(uint32_t)(k >> plan.shift[p]) & 0xFFu], 1u);
+  // neighbouring keys share digits (rows write adjacent tiles at one depth):
+  // one shared atomic per distinct digit per warp
+  const int64_t stride = (int64_t)gridDim.x * kSortThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kSortThreads; base < n; base += stride) {
+    const int64_t i = base + threadIdx.x;
+    const bool valid = i < n;
+    const uint64_t k = valid ? keys[i] : 0ull;
+    for (int p = 0; p < plan.passes; ++p) {
+      const uint32_t d = valid ? (uint32_t)(k >> plan.shift[p]) & 0xFFu : 0x100u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, d);
+      if (valid && lane == __ffs(peers) - 1) atomicAdd(&h[p][d], (uint32_t)__popc(peers));
+    }
   }
   __syncthreads();
   for (int p = 0; p < plan.passes; ++p) {

@@ -956,4 +956,197 @@ int orc_project_bwd(const orc_dims* d, const double* cams, const double* means, 
   return 0;
 }
 
+// ---------------------------------------------------------------------------
+// Sampled checks at full size.  These restate the same definitions for a
+// chosen subset of tiles or rows, so that outputs can be compared one by one
+// where the whole step is too large for the oracle.
+
+// Exact number of entries per tile (row-major walk over every row's range).
+int orc_tile_counts(const orc_dims* d, const uint32_t* aabb, const int32_t* row_cam, int64_t nnz, int64_t* counts) {
+  Geo geo = geometry(d);
+  const int64_t T = geo.tiles_per_cam * d->C;
+  for (int64_t t = 0; t < T; ++t) counts[t] = 0;
+  for (int64_t r = 0; r < nnz; ++r) {
+    int64_t tx0, tx1, ty0, ty1;
+    tile_range(aabb[2 * r] & 0xFFFFu, aabb[2 * r + 1] & 0xFFFFu, d->W, geo.tiles_x, &tx0, &tx1);
+    tile_range(aabb[2 * r] >> 16, aabb[2 * r + 1] >> 16, d->H, geo.tiles_y, &ty0, &ty1);
+    const int64_t base = (int64_t)row_cam[r] * geo.tiles_per_cam;
+    for (int64_t ty = ty0; ty < ty1; ++ty)
+      for (int64_t tx = tx0; tx < tx1; ++tx) counts[base + ty * geo.tiles_x + tx]++;
+  }
+  return 0;
+}
+
+// Sorted (key, row) lists of the selected tiles: every row whose decoded box
+// overlaps the tile, ordered by key then row.  out_off[nsel+1] gives each
+// selected tile's slice of out_keys/out_vals (capacity cap); returns -2 if cap
+// is too small (out_off still complete).
+int orc_tile_lists(const orc_dims* d, const double* screen, const uint32_t* aabb, const int32_t* row_cam,
+                   int64_t nnz, const int64_t* sel, int64_t nsel, int64_t* out_off, uint64_t* out_keys,
+                   uint32_t* out_vals, int64_t cap) {
+  Geo geo = geometry(d);
+  const int64_t T = geo.tiles_per_cam * d->C;
+  std::vector<int64_t> slot((size_t)T, -1);
+  for (int64_t i = 0; i < nsel; ++i) slot[sel[i]] = i;
+  std::vector<std::vector<std::pair<uint64_t, uint32_t>>> lists((size_t)nsel);
+  for (int64_t r = 0; r < nnz; ++r) {
+    int64_t tx0, tx1, ty0, ty1;
+    tile_range(aabb[2 * r] & 0xFFFFu, aabb[2 * r + 1] & 0xFFFFu, d->W, geo.tiles_x, &tx0, &tx1);
+    tile_range(aabb[2 * r] >> 16, aabb[2 * r + 1] >> 16, d->H, geo.tiles_y, &ty0, &ty1);
+    const int64_t base = (int64_t)row_cam[r] * geo.tiles_per_cam;
+    for (int64_t ty = ty0; ty < ty1; ++ty)
+      for (int64_t tx = tx0; tx < tx1; ++tx) {
+        const int64_t t = base + ty * geo.tiles_x + tx;
+        const int64_t s = slot[t];
+        if (s < 0) continue;
+        float depth32 = (float)screen[r * kRow + 9];
+        uint32_t dbits;
+        std::memcpy(&dbits, &depth32, 4);
+        lists[s].push_back({((uint64_t)t << 32) | dbits, (uint32_t)r});
+      }
+  }
+  out_off[0] = 0;
+  for (int64_t i = 0; i < nsel; ++i) {
+    std::stable_sort(lists[i].begin(), lists[i].end(),
+                     [](const std::pair<uint64_t, uint32_t>& a, const std::pair<uint64_t, uint32_t>& b) {
+                       return a.first < b.first;
+                     });
+    out_off[i + 1] = out_off[i] + (int64_t)lists[i].size();
+  }
+  if (out_off[nsel] > cap) return -2;
+  for (int64_t i = 0; i < nsel; ++i)
+    for (size_t k = 0; k < lists[i].size(); ++k) {
+      out_keys[out_off[i] + k] = lists[i][k].first;
+      out_vals[out_off[i] + k] = lists[i][k].second;
+    }
+  return 0;
+}
+
+// Forward rasterizer of the selected tiles from their lists (list i is
+// vals[off[i]..off[i+1]) and starts at global sorted index start[i]).
+// Outputs per selected tile: img [nsel][256][3], T [nsel][256], last [nsel][256]
+// (pixels outside the image: T = 1, last = -2).
+int orc_rasterize_tiles(const orc_dims* d, const double* screen, const uint32_t* vals, const int64_t* off,
+                        const int64_t* sel, const int64_t* start, int64_t nsel, double* img, double* T_out,
+                        int64_t* last_out, int nthreads) {
+  set_threads(nthreads);
+  Geo geo = geometry(d);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t q = 0; q < nsel * kTile * kTile; ++q) {
+    const int64_t s = q / (kTile * kTile), pix = q % (kTile * kTile);
+    const int64_t t = sel[s];
+    const int64_t tr = t % geo.tiles_per_cam;
+    const int64_t i = (tr % geo.tiles_x) * kTile + pix % kTile, j = (tr / geo.tiles_x) * kTile + pix / kTile;
+    if (i >= d->W || j >= d->H) {
+      for (int ch = 0; ch < 3; ++ch) img[3 * q + ch] = 0.0;
+      T_out[q] = 1.0;
+      last_out[q] = -2;
+      continue;
+    }
+    float rgb[3], T;
+    int64_t last;
+    composite_pixel<float>(screen, vals, off[s], off[s + 1], (float)i + 0.5f, (float)j + 0.5f, rgb, &T, &last,
+                           nullptr);
+    for (int ch = 0; ch < 3; ++ch) img[3 * q + ch] = rgb[ch];
+    T_out[q] = T;
+    last_out[q] = last < 0 ? -1 : start[s] + (last - off[s]);
+  }
+  return 0;
+}
+
+// Backward rasterizer restricted to the selected rows: every pixel of the
+// listed tiles (which must include all tiles those rows cover) is replayed in
+// fp64 on top of its fp32 decisions, and only the selected rows' gradients are
+// kept: v_rows [nrows][12].  row_slot[nnz] maps a row to its slot or -1.
+int orc_raster_bwd_rows(const orc_dims* d, const double* screen, const uint32_t* vals, const int64_t* off,
+                        const int64_t* sel, int64_t nsel, const double* v_img, const double* v_T,
+                        const int64_t* row_slot, int64_t nrows, double* v_rows, int nthreads) {
+  set_threads(nthreads);
+  Geo geo = geometry(d);
+  int nt = 1;
+#ifdef _OPENMP
+  nt = std::max(1, nthreads > 0 ? nthreads : omp_get_max_threads());
+#endif
+  std::vector<std::vector<double>> part((size_t)nt, std::vector<double>((size_t)nrows * kRow, 0.0));
+#pragma omp parallel num_threads(nt)
+  {
+    int tid = 0;
+#ifdef _OPENMP
+    tid = omp_get_thread_num();
+#endif
+    std::vector<Contrib> list;
+    std::vector<double> acc, lscreen;
+    std::vector<uint32_t> local;
+    std::vector<Contrib> ll;
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t s = 0; s < nsel; ++s) {
+      const int64_t t = sel[s];
+      const int64_t c = t / geo.tiles_per_cam, tr = t % geo.tiles_per_cam;
+      for (int64_t pix = 0; pix < kTile * kTile; ++pix) {
+        const int64_t i = (tr % geo.tiles_x) * kTile + pix % kTile, j = (tr / geo.tiles_x) * kTile + pix / kTile;
+        if (i >= d->W || j >= d->H) continue;
+        float rgb[3], T;
+        int64_t last;
+        list.clear();
+        composite_pixel<float>(screen, vals, off[s], off[s + 1], (float)i + 0.5f, (float)j + 0.5f, rgb, &T, &last,
+                               &list);
+        bool any = false;
+        for (const Contrib& cb : list)
+          if (row_slot[vals[cb.idx]] >= 0) any = true;
+        if (!any) continue;
+        const int64_t p = (c * d->H + j) * d->W + i;
+        double g[3] = {v_img[3 * p], v_img[3 * p + 1], v_img[3 * p + 2]};
+        double vT = v_T ? v_T[p] : 0.0;
+        // replay this pixel's list on a local copy of its rows
+        acc.assign(list.size() * kRow, 0.0);
+        local.resize(list.size());
+        ll.resize(list.size());
+        lscreen.resize(list.size() * kRow);
+        for (size_t k = 0; k < list.size(); ++k) {
+          const uint32_t row = vals[list[k].idx];
+          for (int q = 0; q < kRow; ++q) lscreen[k * kRow + q] = screen[(int64_t)row * kRow + q];
+          local[k] = (uint32_t)k;
+          ll[k] = {(int64_t)k, list[k].clamped};
+        }
+        pixel_backward(lscreen.data(), local.data(), ll, (double)i + 0.5, (double)j + 0.5, g, vT, acc.data());
+        for (size_t k = 0; k < list.size(); ++k) {
+          const int64_t sl = row_slot[vals[list[k].idx]];
+          if (sl < 0) continue;
+          for (int q = 0; q < kRow; ++q) part[tid][sl * kRow + q] += acc[k * kRow + q];
+        }
+      }
+    }
+  }
+  for (int64_t q = 0; q < nrows * kRow; ++q) {
+    double sum = 0.0;
+    for (int t = 0; t < nt; ++t) sum += part[t][q];
+    v_rows[q] = sum;
+  }
+  return 0;
+}
+
+// Projection backward of single rows: per-row gradient contributions
+// [nrows][3+4+3+1+3K] (means, quats, scales, opacity, sh) in fp64, with the
+// gates decided in fp32.  Summing a Gaussian's rows gives its gradient.
+int orc_project_bwd_rows(const orc_dims* d, const double* cams, const double* means, const double* quats,
+                         const double* scales, const double* opac, const double* sh, const int32_t* cam_of,
+                         const int64_t* gauss_of, int64_t nrows, const double* v_rows, double* out) {
+  const int K = (d->sh_degree + 1) * (d->sh_degree + 1);
+  const int64_t w = 11 + 3 * K;
+  for (int64_t q = 0; q < nrows * w; ++q) out[q] = 0.0;
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t c = cam_of[r], n = gauss_of[r];
+    const double* cam = cams + 20 * c;
+    const double *mu = means + 3 * n, *q = quats + 4 * n, *s = scales + 3 * n, *shn = sh + (int64_t)K * 3 * n;
+    Gates gt = decide_gates<float>(cam, d, mu, q, s, opac[n], shn);
+    Camera<double> k = make_camera<double>(cam, d->W, d->H);
+    Gauss<double> g = make_gauss<double>(mu, q, s, opac[n]);
+    Pair<double> P;
+    project_pair<double>(k, g, d->W, d->H, d->near_plane, d->far_plane, P);
+    double* o = out + r * w;
+    pair_backward(k, g, P, gt, d->sh_degree, shn, v_rows + r * kRow, o, o + 3, o + 7, o + 10, o + 11);
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -55,8 +55,15 @@ def lib():
         L.orc_rasterize_fwd.argtypes = [P, P, P, P, i32, P, P, P, P, P, i32]
         L.orc_rasterize_bwd.argtypes = [P, P, P, P, P, P, i32, i64, P, i32]
         L.orc_project_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i64, P, i32, P, P, P, P, P]
+        L.orc_tile_counts.argtypes = [P, P, P, i64, P]
+        L.orc_tile_lists.argtypes = [P, P, P, P, i64, P, i64, P, P, P, i64]
+        L.orc_rasterize_tiles.argtypes = [P, P, P, P, P, P, i64, P, P, P, i32]
+        L.orc_raster_bwd_rows.argtypes = [P, P, P, P, P, i64, P, P, P, i64, P, i32]
+        L.orc_project_bwd_rows.argtypes = [P, P, P, P, P, P, P, P, P, i64, P, P]
         for f in ("orc_project", "orc_row_boxes", "orc_count_tiles", "orc_intersect", "orc_sort",
-                  "orc_tile_ranges", "orc_rasterize_fwd", "orc_rasterize_bwd", "orc_project_bwd"):
+                  "orc_tile_ranges", "orc_rasterize_fwd", "orc_rasterize_bwd", "orc_project_bwd",
+                  "orc_tile_counts", "orc_tile_lists", "orc_rasterize_tiles", "orc_raster_bwd_rows",
+                  "orc_project_bwd_rows"):
             getattr(L, f).restype = ct.c_int
         _lib = L
     return _lib
@@ -273,3 +280,72 @@ def step(scene, precision: int = 0, nthreads: int = 0, v_img=None, v_T=None) -> 
     grads = project_bwd(scene, f["proj"], v_screen, precision)
     f.update(v_img=v_img, v_screen=v_screen, grads=grads)
     return f
+
+
+# ---------------------------------------------------------------------------- sampled checks at full size
+def tile_counts(scene, proj) -> np.ndarray:
+    g = geometry(scene)
+    d = dims_of(scene)
+    out = np.zeros(g["n_tiles"], np.int64)
+    lib().orc_tile_counts(ct.byref(d), _p(_c(proj["aabb"], np.uint32)), _p(_c(proj["row_cam"], np.int32)),
+                          proj["nnz"], _p(out))
+    return out
+
+
+def tile_lists(scene, proj, tiles) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Sorted (key, row) lists of the given tiles: (offsets, keys, vals)."""
+    d = dims_of(scene)
+    sel = _c(tiles, np.int64)
+    off = np.zeros(len(sel) + 1, np.int64)
+    cap = 1
+    while True:
+        keys = np.zeros(cap, np.uint64)
+        vals = np.zeros(cap, np.uint32)
+        rc = lib().orc_tile_lists(ct.byref(d), _p(_c(proj["screen"], np.float64)), _p(_c(proj["aabb"], np.uint32)),
+                                  _p(_c(proj["row_cam"], np.int32)), proj["nnz"], _p(sel), len(sel), _p(off),
+                                  _p(keys), _p(vals), cap)
+        if rc == 0:
+            return off, keys[: off[-1]], vals[: off[-1]]
+        cap = int(off[-1]) + 1
+
+
+def rasterize_tiles(scene, proj, tiles, off, vals, starts, nthreads: int = 0):
+    """Pixels of the selected tiles: img [n][256][3], T [n][256], last [n][256]
+    (global sorted index; -2 outside the image)."""
+    d = dims_of(scene)
+    n = len(tiles)
+    img = np.zeros((n, 256, 3))
+    T = np.zeros((n, 256))
+    last = np.zeros((n, 256), np.int64)
+    lib().orc_rasterize_tiles(ct.byref(d), _p(_c(proj["screen"], np.float64)), _p(_c(vals, np.uint32)),
+                              _p(_c(off, np.int64)), _p(_c(tiles, np.int64)), _p(_c(starts, np.int64)), n, _p(img),
+                              _p(T), _p(last), nthreads)
+    return img, T, last
+
+
+def raster_bwd_rows(scene, proj, tiles, off, vals, v_img, v_T, rows, nthreads: int = 0) -> np.ndarray:
+    """Screen-row gradients [len(rows)][12] of the selected rows; `tiles` must
+    cover every tile those rows touch."""
+    d = dims_of(scene)
+    slot = np.full(proj["nnz"], -1, np.int64)
+    slot[np.asarray(rows, np.int64)] = np.arange(len(rows))
+    out = np.zeros((len(rows), ROW))
+    vT = None if v_T is None else _c(v_T, np.float64)
+    lib().orc_raster_bwd_rows(ct.byref(d), _p(_c(proj["screen"], np.float64)), _p(_c(vals, np.uint32)),
+                              _p(_c(off, np.int64)), _p(_c(tiles, np.int64)), len(tiles),
+                              _p(_c(v_img, np.float64)), _p(vT), _p(slot), len(rows), _p(out), nthreads)
+    return out
+
+
+def project_bwd_rows(scene, proj, rows, v_rows) -> np.ndarray:
+    """Per-row gradient contributions [len(rows)][11 + 3K]: means(3) quats(4)
+    scales(3) opacity(1) sh(3K)."""
+    d = dims_of(scene)
+    x = _inputs(scene)
+    rows = np.asarray(rows, np.int64)
+    out = np.zeros((len(rows), 11 + 3 * scene.K))
+    lib().orc_project_bwd_rows(ct.byref(d), _p(x["cams"]), _p(x["means"]), _p(x["quats"]), _p(x["scales"]),
+                               _p(x["opac"]), _p(x["sh"]), _p(_c(proj["row_cam"][rows], np.int32)),
+                               _p(_c(proj["row_gauss"][rows], np.int64)), len(rows), _p(_c(v_rows, np.float64)),
+                               _p(out))
+    return out

@@ -84,6 +84,19 @@ __host__ __device__ constexpr int rows_sh_stride() {
   return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
 }
 
+// A visible (camera, Gaussian) pair waiting in the CTA's work queue.
+struct RowItem {
+  int64_t row;
+  int cam;  // camera within the current chunk
+  int g;    // Gaussian within the CTA
+};
+constexpr int kQueue = 2 * kBlock;
+
+// Pass 2 keeps its 128 threads busy whatever the visibility pattern: the
+// visible pairs of the CTA's Gaussians are appended camera by camera to a
+// shared queue (row = block_off of the camera's block + rank among the set
+// bits) and processed 128 at a time by any thread, with the Gaussians'
+// parameters and SH blocks in shared memory.
 template <int DEG>
 __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __restrict__ cams,
                                                          const float* __restrict__ means,
@@ -99,26 +112,60 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   constexpr int KP = rows_sh_stride<DEG>();
   __shared__ Cam scam[kCamChunk];
   __shared__ float sh_s[kBlock * KP];
+  __shared__ GaussIn s_g[kBlock];
+  __shared__ float s_o[kBlock];
+  __shared__ RowItem q[kQueue];
+  __shared__ int q_len;
+  __shared__ uint32_t s_wc[kBlock / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t blk = blockIdx.x;
   const int64_t n0 = blk * kBlock;
   const int64_t n = n0 + threadIdx.x;
-  const bool valid = n < g.N;
   const int cnt = (int)min64(kBlock, g.N - n0);
   {
     const float* src = sh + n0 * K3;
     for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-      const int gi = f / K3, q = f - gi * K3;
-      sh_s[gi * KP + q] = src[f];
+      const int gi = f / K3, qq = f - gi * K3;
+      sh_s[gi * KP + qq] = src[f];
     }
   }
-  const float* shn = sh_s + threadIdx.x * KP;
-  GaussIn gi{};
-  float opac = 0.0f;
-  if (valid) {
-    gi = load_gauss(means, quats, scales, n);
-    opac = opacities[n];
+  if (n < g.N) {
+    s_g[threadIdx.x] = load_gauss(means, quats, scales, n);
+    s_o[threadIdx.x] = opacities[n];
   }
+  if (threadIdx.x == 0) q_len = 0;
+  auto process = [&](const RowItem& it) {
+    const Cam& k = scam[it.cam];
+    const GaussIn& gi = s_g[it.g];
+    const float* shn = sh_s + it.g * KP;
+    Proj P;
+    cam_point(k, gi.mx, gi.my, gi.mz, P.px, P.py, P.pz);
+    project_rest(k, gi.S, g.W, g.H, P);
+    const float idet = div_(1.0f, P.det);
+    const float ca = mul(P.c, idet), cb = -mul(P.b, idet), cc2 = mul(P.a, idet);
+    float b[16];
+    float X = 0.0f, Y = 0.0f, Z = 0.0f, il;
+    if (DEG > 0) view_dir(k, gi.mx, gi.my, gi.mz, X, Y, Z, il);
+    sh_basis(DEG, X, Y, Z, b);
+    float rgb[3];
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) {
+      float acc = mul(shn[ch], b[0]);
+#pragma unroll
+      for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], b[kk]));
+      rgb[ch] = fmaxf(add(acc, 0.5f), 0.0f);
+    }
+    float4* out = reinterpret_cast<float4*>(screen + it.row * kRowF);
+    out[0] = make_float4(P.mx, P.my, ca, cb);
+    out[1] = make_float4(cc2, s_o[it.g], rgb[0], rgb[1]);
+    out[2] = make_float4(rgb[2], P.pz, 0.0f, 0.0f);
+    const float x0 = fmaxf(sub(P.mx, P.r), 0.0f), x1 = fminf(add(P.mx, P.r), (float)g.W);
+    const float y0 = fmaxf(sub(P.my, P.r), 0.0f), y1 = fminf(add(P.my, P.r), (float)g.H);
+    uint2 qq;
+    qq.x = q16_floor(x0, g.W) | (q16_floor(y0, g.H) << 16);
+    qq.y = q16_ceil(x1, g.W) | (q16_ceil(y1, g.H) << 16);
+    reinterpret_cast<uint2*>(aabb16)[it.row] = qq;
+  };
   for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
     const int nc = min(kCamChunk, g.C - c0);
     __syncthreads();
@@ -128,40 +175,41 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
       const int64_t c = c0 + cc;
       const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
       const uint32_t word = mask[wbase + warp];
-      if (!((word >> lane) & 1u)) continue;
-      int64_t row = block_off[c * g.blocks_per_cam + blk];
-      for (int w = 0; w < warp; ++w) row += __popc(mask[wbase + w]);
-      row += __popc(word & ((1u << lane) - 1u));
-      const Cam& k = scam[cc];
-      Proj P;
-      cam_point(k, gi.mx, gi.my, gi.mz, P.px, P.py, P.pz);
-      project_rest(k, gi.S, g.W, g.H, P);
-      const float idet = div_(1.0f, P.det);
-      const float ca = mul(P.c, idet), cb = -mul(P.b, idet), cc2 = mul(P.a, idet);
-      // colour
-      float b[16];
-      float X = 0.0f, Y = 0.0f, Z = 0.0f, il;
-      if (DEG > 0) view_dir(k, gi.mx, gi.my, gi.mz, X, Y, Z, il);
-      sh_basis(DEG, X, Y, Z, b);
-      float rgb[3];
+      if (lane == 0) s_wc[warp] = __popc(word);
+      __syncthreads();
+      int before = 0, total = 0;
 #pragma unroll
-      for (int ch = 0; ch < 3; ++ch) {
-        float acc = mul(shn[ch], b[0]);
-#pragma unroll
-        for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], b[kk]));
-        rgb[ch] = fmaxf(add(acc, 0.5f), 0.0f);
+      for (int w = 0; w < kBlock / 32; ++w) {
+        before += w < warp ? (int)s_wc[w] : 0;
+        total += (int)s_wc[w];
       }
-      float4* out = reinterpret_cast<float4*>(screen + row * kRowF);
-      out[0] = make_float4(P.mx, P.my, ca, cb);
-      out[1] = make_float4(cc2, opac, rgb[0], rgb[1]);
-      out[2] = make_float4(rgb[2], P.pz, 0.0f, 0.0f);
-      const float x0 = fmaxf(sub(P.mx, P.r), 0.0f), x1 = fminf(add(P.mx, P.r), (float)g.W);
-      const float y0 = fmaxf(sub(P.my, P.r), 0.0f), y1 = fminf(add(P.my, P.r), (float)g.H);
-      uint2 q;
-      q.x = q16_floor(x0, g.W) | (q16_floor(y0, g.H) << 16);
-      q.y = q16_ceil(x1, g.W) | (q16_ceil(y1, g.H) << 16);
-      reinterpret_cast<uint2*>(aabb16)[row] = q;
+      const int base = q_len;
+      if ((word >> lane) & 1u) {
+        const int r = before + __popc(word & ((1u << lane) - 1u));
+        RowItem it;
+        it.row = block_off[c * g.blocks_per_cam + blk] + r;
+        it.cam = cc;
+        it.g = threadIdx.x;
+        q[base + r] = it;
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) q_len = base + total;
+      __syncthreads();
+      if (q_len >= kBlock) {  // a full round: every thread takes one item
+        const int len = q_len;
+        process(q[threadIdx.x]);
+        __syncthreads();
+        for (int t = kBlock + threadIdx.x; t < len; t += kBlock) q[t - kBlock] = q[t];
+        __syncthreads();
+        if (threadIdx.x == 0) q_len = len - kBlock;
+        __syncthreads();
+      }
     }
+    // the queue refers to this chunk's cameras: drain it before the next chunk
+    const int len = q_len;
+    if (threadIdx.x < len) process(q[threadIdx.x]);
+    __syncthreads();
+    if (threadIdx.x == 0) q_len = 0;
   }
 }
 

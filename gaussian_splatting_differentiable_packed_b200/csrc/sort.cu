@@ -22,6 +22,7 @@
 // The per-pass reduce-then-scan kernels below (k_radix_hist, k_radix_scatter)
 // are the simpler variant kept for reference; they are not launched.
 #include <algorithm>
+#include <mutex>
 #include <utility>
 
 #include "ss_common.cuh"
@@ -428,4 +429,57 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
     return SS_ERR_DEVICE_CHECK;
   }
   return SS_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Some callers cannot call cudaMalloc at all (for
+// example code running inside another runtime's allocator callbacks, or a
+// host that hands out only fixed device buffers), so this entry point keeps
+// the sort's scratch in a file-scope device array instead of a caller buffer.
+// The array is part of the loaded module: every GPU that loads the library
+// holds it until the process exits.
+
+namespace ss {
+
+constexpr size_t kNoAllocScratchBytes = size_t(24) << 20;  // 24 MiB
+__device__ __align__(256) unsigned char g_sort_scratch[kNoAllocScratchBytes];
+
+// Host code may not use g_sort_scratch as a device address: the symbol's host
+// side is only a stand-in.  The device address is looked up once per device.
+std::mutex g_scratch_mu;
+void* g_scratch_addr[256] = {};
+
+ss_status noalloc_scratch(void** out) {
+  int dev = 0;
+  ss_status s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s) return s;
+  if (dev < 0 || dev >= 256) return invalid("device ordinal out of range");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    s = cuda_status(cudaGetSymbolAddress(&p, g_sort_scratch), "cudaGetSymbolAddress");
+    if (s) return s;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return SS_OK;
+}
+
+}  // namespace ss
+
+extern "C" ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a,
+                                            uint64_t* keys_b, uint32_t* vals_b, int64_t n, int64_t* tile_off,
+                                            int* result_in_b_out, void* stream) {
+  if (n < 0) return invalid("n < 0");
+  if (n > 0 && sort_temp_bytes(n) > kNoAllocScratchBytes) {
+    set_error("ss_sort_isects_noalloc: n exceeds the 24 MiB static scratch (at most 50311168 keys)");
+    return SS_ERR_INVALID_ARG;
+  }
+  void* scratch = nullptr;
+  if (n > 0) {
+    ss_status s = noalloc_scratch(&scratch);
+    if (s) return s;
+  }
+  return ss_sort_isects(dims, keys_a, vals_a, keys_b, vals_b, n, scratch, kNoAllocScratchBytes, tile_off,
+                        result_in_b_out, stream);
 }

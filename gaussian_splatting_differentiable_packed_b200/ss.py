@@ -28,7 +28,8 @@ PMASK_BLOCK = 128
 TILE = 16
 
 EXPORTS = ("ss_size", "ss_workspace_bytes", "ss_status_string", "ss_last_error", "ss_project_packed",
-           "ss_intersect_tiles", "ss_sort_isects", "ss_rasterize_fwd", "ss_rasterize_fwd_counts",
+           "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc", "ss_rasterize_fwd",
+           "ss_rasterize_fwd_counts",
            "ss_rasterize_bwd", "ss_project_bwd")
 
 
@@ -67,11 +68,13 @@ def lib() -> ct.CDLL:
         L.ss_project_packed.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, i64, P, sz, ct.POINTER(i64), P]
         L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
         L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, P, sz, P, ct.POINTER(i32), P]
+        L.ss_sort_isects_noalloc.argtypes = [D, P, P, P, P, i64, P, ct.POINTER(i32), P]
         L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P]
         L.ss_rasterize_fwd_counts.argtypes = [D, P, P, P, P, P, P, P, P]
         L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, i64, P]
         L.ss_project_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
-        for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_rasterize_fwd",
+        for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc",
+                  "ss_rasterize_fwd",
                   "ss_rasterize_fwd_counts", "ss_rasterize_bwd", "ss_project_bwd"):
             getattr(L, f).restype = i32
         _lib = L
@@ -143,6 +146,15 @@ def ss_sort_isects(d, keys_a, vals_a, keys_b, vals_b, n, temp, tile_off, stream=
                               0 if temp is None else temp.numel() * temp.element_size(), _p(tile_off),
                               ct.byref(in_b), _stream(stream))
     _check(st, "ss_sort_isects")
+    return bool(in_b.value)
+
+
+def ss_sort_isects_noalloc(d, keys_a, vals_a, keys_b, vals_b, n, tile_off, stream=None) -> bool:
+    """ss_sort_isects with the library's static scratch (no caller temp buffer)."""
+    in_b = ct.c_int(0)
+    st = lib().ss_sort_isects_noalloc(ct.byref(d), _p(keys_a), _p(vals_a), _p(keys_b), _p(vals_b), int(n),
+                                      _p(tile_off), ct.byref(in_b), _stream(stream))
+    _check(st, "ss_sort_isects_noalloc")
     return bool(in_b.value)
 
 

@@ -154,6 +154,26 @@ ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a
                          int* result_in_b_out, void* stream);
 
 /*
+ * Allocation-free variant of ss_sort_isects (the pages have no counterpart:
+ * this is an addition of this library).  For callers that cannot allocate
+ * device memory themselves (code that runs inside another runtime's
+ * allocator or capture, or a host that only hands out fixed buffers): the
+ * sort's scratch lives in a file-scope device array of 24 MiB that the
+ * library holds on every GPU that loads it, until the process exits.  The
+ * caller still passes the key/value buffers and tile_off; no cudaMalloc,
+ * cudaFree or allocating routine is called.  n may be at most 50,311,168
+ * keys; a larger n returns SS_ERR_INVALID_ARG before any device work.  The
+ * first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call shares the one array (cleared at the
+ * start of each call), so calls that overlap on the GPU race with each other:
+ * serialise them, e.g. on one stream.  Results equal ss_sort_isects'.
+ */
+ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
+                                 uint32_t* vals_b, int64_t n, int64_t* tile_off, int* result_in_b_out,
+                                 void* stream);
+
+/*
  * Forward rasterizer ("Spirula Studio backward pass", section 4: the forward
  * keeps tile offsets, the intersection list, each pixel's last Gaussian and
  * its transmittance for the backward pass).  One CTA per 16x16 tile, front to

@@ -39,39 +39,51 @@ __device__ __forceinline__ void tile_coords(const Geo& g, int64_t tile, int& c, 
 // ---------------------------------------------------------------------------
 // Staged entry.  thr = 5.6 when o <= 1 (then sigma > 5.6 implies
 // o*exp(-sigma) < 1/255: the pixel skips the entry without the exp), +inf
-// otherwise.  (hx, hy) bound the ellipse {sigma <= 5.7} of the stored conic
-// (fp64 with a margin; +inf when o > 1 or the conic is not positive definite).
+// otherwise.  The remaining fields bound where the entry can matter, all
+// computed in fp32 and rounded outward: dql underestimates ca*cc - cb^2 (the
+// fma error bound subtracted), so (hx, hy) over-cover the ellipse
+// {sigma <= 5.8} of the stored conic and the row chords below over-cover it
+// too; +inf / "everything" when o > 1 or the conic is not safely positive
+// definite.
+constexpr float kCullT = 5.8f;
+
 struct Stage {
   float4 a;  // x, y, 0.5*ca, cb
   float4 b;  // 0.5*cc, o, r, g
   float4 c;  // b, hx, hy, kterm = |ha| + |hc| + |cb|
-  float thr;
-  uint32_t row;
-  float pad0, pad1;
+  float4 d;  // thr, row (bits), P = 2*ca*kCullT, dql
+  float4 e;  // 1/ca, cb/ca, bounded (1/0), 0
 };
 
 __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint32_t r, Stage& st) {
   const float4* row = reinterpret_cast<const float4*>(screen + (int64_t)r * kRowF);
   const float4 r0 = row[0], r1 = row[1], r2 = row[2];
-  st.a = make_float4(r0.x, r0.y, mul(0.5f, r0.z), r0.w);
-  st.b = make_float4(mul(0.5f, r1.x), r1.y, r1.z, r1.w);
+  const float ca = r0.z, cb = r0.w, cc = r1.x, o = r1.y;
+  st.a = make_float4(r0.x, r0.y, mul(0.5f, ca), cb);
+  st.b = make_float4(mul(0.5f, cc), o, r1.z, r1.w);
   const float inf = __int_as_float(0x7f800000);
-  float hx = inf, hy = inf;
-  const double dq = (double)r0.z * (double)r1.x - (double)r0.w * (double)r0.w;
-  if (r1.y <= 1.0f && dq > 0.0) {
-    hx = (float)(sqrt(11.4 * (double)r1.x / dq) * 1.001 + 1e-3);
-    hy = (float)(sqrt(11.4 * (double)r0.z / dq) * 1.001 + 1e-3);
+  const float bb = cb * cb;
+  const float dq = fmaf(ca, cc, -bb);
+  const float dql = dq - 2e-7f * (bb + fabsf(dq)) - 1e-30f;
+  float hx = inf, hy = inf, P = 0.0f, ica = 0.0f, cbr = 0.0f, bounded = 0.0f;
+  if (o <= 1.0f && ca > 0.0f && cc > 0.0f && dql > 0.0f) {
+    hx = sqrtf(2.0f * kCullT * cc / dql) * 1.00001f + 1e-3f;
+    hy = sqrtf(2.0f * kCullT * ca / dql) * 1.00001f + 1e-3f;
+    P = 2.0f * kCullT * ca;
+    ica = 1.0f / ca;
+    cbr = cb * ica;
+    bounded = 1.0f;
   }
-  const float kterm = 0.5f * fabsf(r0.z) + 0.5f * fabsf(r1.x) + fabsf(r0.w);
+  const float kterm = 0.5f * fabsf(ca) + 0.5f * fabsf(cc) + fabsf(cb);
   st.c = make_float4(r2.x, hx, hy, kterm);
-  st.thr = r1.y <= 1.0f ? SS_SIGMA_SKIP : inf;
-  st.row = r;
+  st.d = make_float4(o <= 1.0f ? SS_SIGMA_SKIP : inf, __uint_as_float(r), P, dql);
+  st.e = make_float4(ica, cbr, bounded, 0.0f);
 }
 
 // Warp culling.  For an entry with o <= 1 every pixel whose computed sigma
 // exceeds 5.6 skips the entry.  A region outside the box (hx, hy) of the
-// ellipse {sigma <= 5.7} has exact sigma > 5.7 at every pixel centre; when
-// kterm*(Dx^2 + Dy^2) <= 1e5 (D: largest offset from the mean to the region)
+// ellipse {sigma <= 5.8} has exact sigma > 5.8 at every pixel centre; when
+// kterm*(Dx^2 + Dy^2) <= 8e4 (D: largest offset from the mean to the region)
 // the canonical fp32 sigma differs from the exact one by less than 0.04, so
 // every pixel of the region computes sigma > 5.6 and would skip the entry:
 // skipping it for the whole warp takes exactly the per-pixel decision.
@@ -82,7 +94,7 @@ __device__ __forceinline__ bool warp_culled(const Stage& st, float x_lo, float x
   if (!(ex > st.c.y || ey > st.c.z)) return false;
   const float Dx = fmaxf(fabsf(x_lo - mx), fabsf(x_hi - mx));
   const float Dy = fmaxf(fabsf(y_lo - my), fabsf(y_hi - my));
-  return st.c.w * (Dx * Dx + Dy * Dy) <= 1e5f;
+  return st.c.w * (Dx * Dx + Dy * Dy) <= 8e4f;
 }
 
 // sigma of the pixel pair in the canonical order (see gauss_sigma).
@@ -182,8 +194,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd(Geo g, const float* __
         const float dx = sub(st.a.x, px);
         const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
         const float2 sig = sigma_pair(st, dx, dy);
-        const bool needA = !doneA && !(sig.x < 0.0f) && !(sig.x > st.thr);
-        const bool needB = !doneB && !(sig.y < 0.0f) && !(sig.y > st.thr);
+        const bool needA = !doneA && !(sig.x < 0.0f) && !(sig.x > st.d.x);
+        const bool needB = !doneB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
         if (!(needA || needB)) continue;
         const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
         const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
@@ -265,37 +277,42 @@ __device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
   return transpose_step<1, 0x55555555u>(x, lane);
 }
 
-// 16-bit column mask of the pixels of row centre yc (columns x_lo + c, c =
-// 0..15) inside the widened chord of {sigma <= 5.7}.
+// 16-bit column mask of the pixels of row centre yc (columns x_lo + c,
+// c = 0..15) inside the outward-rounded chord of {sigma <= 5.8}: for a pixel
+// row at offset dy the chord is centred at mx + (cb/ca)*dy with half-width
+// sqrt(2*ca*5.8 - dq*dy^2)/ca; dql <= dq and the margins make every fp32
+// rounding widen it.
 __device__ __forceinline__ uint32_t chord_span(const Stage& st, float yc, float x_lo) {
-  const double A = st.a.z;                       // 0.5*ca
-  const double dy = (double)st.a.y - (double)yc;  // exact
-  const double B = (double)st.a.w * dy;
-  const double Cq = (double)st.b.x * dy * dy - 5.7;
-  const double disc = B * B - 4.0 * A * Cq;
-  if (disc < 0.0) return 0u;
-  const double sq = sqrt(disc);
-  const double dx1 = (-B - sq) / (2.0 * A), dx2 = (-B + sq) / (2.0 * A);
-  // pixel centre px = x_lo + c covers when mx - dx2 <= px <= mx - dx1
-  const double lo = (double)st.a.x - dx2 - (double)x_lo - 1e-3;
-  const double hi = (double)st.a.x - dx1 - (double)x_lo + 1e-3;
-  if (hi < 0.0 || lo > 15.0) return 0u;
-  const int c0 = lo <= 0.0 ? 0 : (int)ceil(lo);
-  const int c1 = hi >= 15.0 ? 15 : (int)floor(hi);
+  const float dy = st.a.y - yc;
+  const float q = st.d.w * dy * dy;
+  const float disc = st.d.z - q + 4e-7f * (st.d.z + q);
+  if (disc < 0.0f) return 0u;
+  if (!(disc >= 0.0f)) return 0xFFFFu;  // NaN: nothing can be concluded
+  const float hw = sqrtf(disc) * st.e.x * 1.00001f + 2e-3f;
+  const float off = st.e.y * dy;
+  const float ctr = st.a.x + off;
+  const float m = 1e-5f * (fabsf(st.a.x) + fabsf(off)) + 2e-3f;
+  const float lo = ctr - hw - m - x_lo, hi = ctr + hw + m - x_lo;
+  if (!(lo == lo && hi == hi)) return 0xFFFFu;
+  if (hi < 0.0f || lo > 15.0f) return 0u;
+  const int c0 = lo <= 0.0f ? 0 : (int)ceilf(lo);
+  const int c1 = hi >= 15.0f ? 15 : (int)floorf(hi);
   if (c1 < c0) return 0u;
   return ((0xFFFFu >> (15 - c1)) >> c0) << c0;
 }
 
 // Coverage of this lane's entry over the warp's region: bit L of covA (covB)
-// set when the entry can reach lane L's upper (lower) pixel.
+// set when the entry can reach lane L's upper (lower) pixel.  A pixel left
+// out has exact sigma > 5.8, and kterm*D^2 <= 8e4 bounds the rounding of the
+// canonical fp32 sigma by 0.04, so its computed sigma exceeds 5.6: it skips
+// the entry in the per-pixel definition as well.
 __device__ __forceinline__ void entry_coverage(const Stage& st, float x_lo, float y_lo, uint32_t& covA,
                                                uint32_t& covB) {
   const float x_hi = x_lo + 15.0f, y_hi = y_lo + 3.0f;
   const float mx = st.a.x, my = st.a.y;
   const float Dx = fmaxf(fabsf(x_lo - mx), fabsf(x_hi - mx));
   const float Dy = fmaxf(fabsf(y_lo - my), fabsf(y_hi - my));
-  const bool bounded = st.b.y <= 1.0f && st.a.z > 0.0f && st.c.w * (Dx * Dx + Dy * Dy) <= 8e4f;
-  if (!bounded) {
+  if (!(st.e.z > 0.0f && st.c.w * (Dx * Dx + Dy * Dy) <= 8e4f)) {
     covA = covB = 0xFFFFFFFFu;
     return;
   }
@@ -357,8 +374,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd_masked(Geo g, const fl
         const float dx = sub(st.a.x, px);
         const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
         const float2 sig = sigma_pair(st, dx, dy);
-        const bool needA = cA && !(sig.x < 0.0f) && !(sig.x > st.thr);
-        const bool needB = cB && !(sig.y < 0.0f) && !(sig.y > st.thr);
+        const bool needA = cA && !(sig.x < 0.0f) && !(sig.x > st.d.x);
+        const bool needB = cB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
         if (!(needA || needB)) continue;
         const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
         const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
@@ -533,8 +550,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
             const float dx = sub(st.a.x, px);
             const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
             const float2 sig = sigma_pair(st, dx, dy);
-            const bool needA = liveA && !(sig.x < 0.0f) && !(sig.x > st.thr);
-            const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.thr);
+            const bool needA = liveA && !(sig.x < 0.0f) && !(sig.x > st.d.x);
+            const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
             if (needA || needB) {
               const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
               if (needA) contrib |= pixel_grad(st, dx, dy.x, ev.x, amin, pa, gr);
@@ -562,7 +579,7 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
       float4* src = reinterpret_cast<float4*>(&red[k][4 * q]);
       const float4 v = *src;
       *src = make_float4(0.f, 0.f, 0.f, 0.f);
-      atomicAdd(reinterpret_cast<float4*>(v_screen + (int64_t)s_e[k].row * kRowF + 4 * q), v);
+      atomicAdd(reinterpret_cast<float4*>(v_screen + (int64_t)__float_as_uint(s_e[k].d.y) * kRowF + 4 * q), v);
     }
     __syncthreads();
     for (int t = threadIdx.x; t < cnt; t += kRThreads) s_any[t] = 0u;

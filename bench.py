@@ -47,6 +47,32 @@ def load_peaks():
         return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, src="fallback")
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def source_digest(paths) -> str:
+    """sha256 over the kernel's source files (the capture is void once they change)."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(stage: str):
+    """DRAM bytes per launch of the stage's kernel from a recorded ncu capture,
+    or None when there is none or the kernel's sources changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[stage]
+        if source_digest(rec["sources"]) != rec["sha256"]:
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -311,12 +337,12 @@ def run_ours(args):
     sd = stages[dom]
     if sd["bound"] == "hbm":
         roof = dict(bound="hbm", achieved=sd["hbm_gbs"], peak=peaks["hbm_gbs"], unit="GB/s", frac=sd["hbm_frac"],
-                    traffic=None, kernel=dom, peak_source=peaks["src"])
+                    traffic=recorded_traffic(dom), kernel=dom, peak_source=peaks["src"])
     else:
         ach = model[dom]["instr"] / (stage_ms[dom] / 1e3) / 1e12
         pk = fp32_peak_instr_per_s(sm_mhz) / 1e12
         roof = dict(bound="alu", achieved=round(ach, 3), peak=round(pk, 3), unit="T FP32 instr/s",
-                    frac=round(ach / pk, 4), traffic=None, kernel=dom,
+                    frac=round(ach / pk, 4), traffic=recorded_traffic(dom), kernel=dom,
                     peak_source=f"148 SMs x 128 FP32 lanes x {sm_mhz:.0f} MHz (median SM clock under load)")
     launches = ss.launches_per_step(d, step.nnz, step.n_isects) * args.steps
     out_work = dict(work)

@@ -3,9 +3,10 @@
 // extrinsics to its six attributes: means, rotation, scale, opacity, DC and
 // higher SH coefficients).
 //
-// One thread per Gaussian, 128 per CTA, looping over the cameras exactly as
-// the packed projection does; a set mask bit gives the row by the same
-// popcount arithmetic, so no (camera, Gaussian) ids are stored.  The gradient
+// One thread per Gaussian, 128 per CTA, looping over the cameras that see
+// its Gaussian (the set bits of the packed projection's mask); a set bit
+// gives the row by the same popcount arithmetic, so no (camera, Gaussian) ids
+// are stored.  The gradient
 // of the 3D covariance is summed over cameras first and taken through
 // Sigma = M M^T, the scale and the quaternion once per Gaussian.
 // Deterministic: no atomics.  Decisions that gate gradients (the Jacobian's
@@ -90,7 +91,10 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = 3 * K;
   constexpr int KP = sh_stride<DEG>();
+  constexpr int kWarps = kBlock / 32;
   __shared__ Cam scam[kCamChunkB];
+  __shared__ uint32_t s_word[kCamChunkB][kWarps];
+  __shared__ int64_t s_row0[kCamChunkB][kWarps];
   extern __shared__ float smem[];
   float* sh_s = smem;                 // [kBlock][KP] SH coefficients of the CTA's Gaussians
   float* gsh_s = smem + kBlock * KP;  // [kBlock][KP] their gradient accumulators
@@ -123,16 +127,26 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     const int nc = min(kCamChunkB, g.C - c0);
     __syncthreads();
     if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
-    __syncthreads();
-    if (!valid) continue;
-    for (int cc = 0; cc < nc; ++cc) {
+    if (threadIdx.x < nc * kWarps) {
+      // each warp's mask word and first row, per camera of the chunk
+      const int cc = threadIdx.x / kWarps, w = threadIdx.x % kWarps;
       const int64_t c = c0 + cc;
       const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
-      const uint32_t word = mask[wbase + warp];
-      if (!((word >> lane) & 1u)) continue;
       int64_t row = block_off[c * g.blocks_per_cam + blk];
-      for (int w = 0; w < warp; ++w) row += __popc(mask[wbase + w]);
-      row += __popc(word & ((1u << lane) - 1u));
+      for (int w2 = 0; w2 < w; ++w2) row += __popc(mask[wbase + w2]);
+      s_word[cc][w] = mask[wbase + w];
+      s_row0[cc][w] = row;
+    }
+    __syncthreads();
+    if (!valid) continue;
+    // Each lane walks its own visible cameras: a warp runs as many rounds as
+    // its busiest Gaussian has cameras, not one round per camera of the chunk.
+    uint32_t vis = 0;
+    for (int cc = 0; cc < nc; ++cc) vis |= ((s_word[cc][warp] >> lane) & 1u) << cc;
+    while (vis) {
+      const int cc = __ffs(vis) - 1;
+      vis &= vis - 1;
+      const int64_t row = s_row0[cc][warp] + __popc(s_word[cc][warp] & ((1u << lane) - 1u));
       const float4* vrp = reinterpret_cast<const float4*>(v_screen + row * kRowF);
       const float4 v0 = vrp[0], v1 = vrp[1], v2 = vrp[2];
       const Cam& k = scam[cc];

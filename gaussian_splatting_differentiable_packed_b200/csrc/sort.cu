@@ -166,17 +166,25 @@ __global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __res
   const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kMaxPasses * kRadix; i += kSortThreads) (&h[0][0])[i] = 0;
   __syncthreads();
-  // neighbouring keys share digits (rows write adjacent tiles at one depth):
-  // one shared atomic per distinct digit per warp
+  // coalesced: a warp reads 32 consecutive keys; neighbouring keys share
+  // digits (a row's keys share the depth and neighbouring tile ids), so each
+  // run of equal digits is counted by its first lane with one shared atomic
   const int64_t stride = (int64_t)gridDim.x * kSortThreads;
   for (int64_t base = (int64_t)blockIdx.x * kSortThreads; base < n; base += stride) {
     const int64_t i = base + threadIdx.x;
     const bool valid = i < n;
     const uint64_t k = valid ? keys[i] : 0ull;
+    const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
     for (int p = 0; p < plan.passes; ++p) {
-      const uint32_t d = valid ? (uint32_t)(k >> plan.shift[p]) & 0xFFu : 0x100u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, d);
-      if (valid && lane == __ffs(peers) - 1) atomicAdd(&h[p][d], (uint32_t)__popc(peers));
+      const uint32_t d = (uint32_t)(k >> plan.shift[p]) & 0xFFu;
+      const uint32_t prev = __shfl_up_sync(0xffffffffu, d, 1);
+      const bool head = valid && (lane == 0 || d != prev);
+      const uint32_t heads = __ballot_sync(0xffffffffu, head);
+      if (head) {
+        const uint32_t after = heads & ~((2u << lane) - 1u);  // heads above this lane
+        const uint32_t end_lane = after ? (uint32_t)(__ffs(after) - 1) : (uint32_t)(32 - __clz(vmask));
+        atomicAdd(&h[p][d], end_lane - (uint32_t)lane);
+      }
     }
   }
   __syncthreads();
@@ -274,22 +282,39 @@ __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __res
     }
     uint64_t prefix = 0;
     if (tile > 0) {
+      // walk back over earlier tiles' published counts, fetching a window of
+      // kLook predecessors per round trip; stop at the first inclusive prefix
+      constexpr int kLook = 8;
       int64_t t = tile - 1;
       int spins = 0;
-      while (true) {
-        const uint64_t sv = ld_status(status + t * kRadix + d);
-        const bool ready = (sv & ~(kValMask | kFlagAgg | kFlagPre)) == epoch && (sv & (kFlagAgg | kFlagPre));
-        if (!ready) {
-          if (++spins > kSpinLimit) {
-            atomicOr(err, 1u);
+      bool found = false;
+      while (!found && t >= 0) {
+        uint64_t w[kLook];
+#pragma unroll
+        for (int j = 0; j < kLook; ++j) w[j] = t - j >= 0 ? ld_status(status + (t - j) * kRadix + d) : 0ull;
+        int j = 0;
+        for (; j < kLook && t - j >= 0; ++j) {
+          const uint64_t sv = w[j];
+          const bool ready = (sv & ~(kValMask | kFlagAgg | kFlagPre)) == epoch && (sv & (kFlagAgg | kFlagPre));
+          if (!ready) break;
+          prefix += sv & kValMask;
+          if (sv & kFlagPre) {
+            found = true;
             break;
           }
-          __nanosleep(64);
+        }
+        if (found) break;
+        if (j == kLook || t - j < 0) {
+          t -= j;
           continue;
         }
-        prefix += sv & kValMask;
-        if (sv & kFlagPre) break;
-        if (--t < 0) break;
+        // predecessor t - j has not published yet: wait for it (bounded)
+        t -= j;
+        if (++spins > kSpinLimit) {
+          atomicOr(err, 1u);
+          break;
+        }
+        __nanosleep(32);
       }
       atomicExch(reinterpret_cast<unsigned long long*>(st), epoch | kFlagPre | (prefix + run));
     }

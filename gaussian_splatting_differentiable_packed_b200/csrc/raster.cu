@@ -444,32 +444,59 @@ struct PixB {
   int64_t last;
 };
 
-// Reverse step of one pixel for a replayed entry (sigma already computed and
-// below the skip threshold); adds this pixel's contribution to gr[0..8].
-__device__ __forceinline__ bool pixel_grad(const Stage& st, float dx, float dy, float ev, float amin, PixB& p,
-                                           float* gr) {
-  const float oe = mul(st.b.y, ev);
-  const float alpha = fminf(SS_ALPHA_MAX, oe);
-  if (alpha < amin) return false;
-  const float ra = 1.0f / (1.0f - alpha);
-  const float Ti = p.T * ra;
-  const float w = alpha * Ti;
-  gr[6] += w * p.g0;
-  gr[7] += w * p.g1;
-  gr[8] += w * p.g2;
-  const float rgbg = st.b.z * p.g0 + st.b.w * p.g1 + st.c.x * p.g2;
-  const float v_alpha = Ti * rgbg - ra * (p.Sg + p.vTT);
-  p.Sg += w * rgbg;
-  p.T = Ti;
-  if (oe < SS_ALPHA_MAX) {
-    const float v_sig = -alpha * v_alpha;
-    gr[5] += ev * v_alpha;
-    gr[2] += v_sig * 0.5f * dx * dx;
-    gr[3] += v_sig * dx * dy;
-    gr[4] += v_sig * 0.5f * dy * dy;
-    gr[0] += v_sig * (2.0f * st.a.z * dx + st.a.w * dy);
-    gr[1] += v_sig * (st.a.w * dx + 2.0f * st.b.x * dy);
-  }
+// Reverse step of the thread's pixel pair for a replayed entry.  cA / cB say
+// which pixels replay the entry with sigma within the skip threshold.  A
+// pixel that does not take the entry (alpha < 1/255, the forward's decision
+// in the same canonical arithmetic) gets alpha 0 below: ra = 1 and w = 0 keep
+// its state.  Writes the pair's summed contribution to gr[0..8] (x, y, ca, cb,
+// cc, o, r, g, b) and returns whether any pixel contributed.  The conic and
+// mean terms are summed over the pair before the entry's coefficients
+// multiply them: with v = dL/dsigma per pixel,
+//   dL/dx = ca*dx*S0 + cb*S1,  dL/dy = cb*dx*S0 + cc*S1,
+//   dL/dca = dx^2*S0/2,  dL/dcb = dx*S1,  dL/dcc = S2/2,
+// where S0 = sum v, S1 = sum v*dy, S2 = sum v*dy^2 (dx is shared).
+__device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, float2 ev, bool cA, bool cB,
+                                          float amin, PixB& pa, PixB& pb, float* gr) {
+  const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
+  cA = cA && !(fminf(SS_ALPHA_MAX, oe.x) < amin);
+  cB = cB && !(fminf(SS_ALPHA_MAX, oe.y) < amin);
+  if (!(cA || cB)) return false;
+  const float2 a = f2(cA ? fminf(SS_ALPHA_MAX, oe.x) : 0.0f, cB ? fminf(SS_ALPHA_MAX, oe.y) : 0.0f);
+  const float2 ra = f2(__frcp_rn(1.0f - a.x), __frcp_rn(1.0f - a.y));
+  const float2 Ti = __fmul2_rn(f2(pa.T, pb.T), ra);  // transmittance in front of the entry
+  const float2 w = __fmul2_rn(a, Ti);
+  const float2 G0 = f2(pa.g0, pb.g0), G1 = f2(pa.g1, pb.g1), G2 = f2(pa.g2, pb.g2);
+  float2 rgbg = __fmul2_rn(f2s(st.b.z), G0);
+  rgbg = __ffma2_rn(f2s(st.b.w), G1, rgbg);
+  rgbg = __ffma2_rn(f2s(st.c.x), G2, rgbg);
+  const float2 Sg = f2(pa.Sg, pb.Sg);
+  const float2 behind = __fadd2_rn(Sg, f2(pa.vTT, pb.vTT));
+  const float2 va = __ffma2_rn(Ti, rgbg, __fmul2_rn(f2(-ra.x, -ra.y), behind));  // dL/dalpha
+  const float2 Sg1 = __ffma2_rn(w, rgbg, Sg);
+  pa.Sg = Sg1.x;
+  pb.Sg = Sg1.y;
+  pa.T = Ti.x;
+  pb.T = Ti.y;
+  const float2 w0 = __fmul2_rn(w, G0), w1 = __fmul2_rn(w, G1), w2 = __fmul2_rn(w, G2);
+  gr[6] = w0.x + w0.y;
+  gr[7] = w1.x + w1.y;
+  gr[8] = w2.x + w2.y;
+  // sigma and opacity gradients only where alpha was not clamped at 0.99
+  const bool gA = cA && oe.x < SS_ALPHA_MAX, gB = cB && oe.y < SS_ALPHA_MAX;
+  const float2 vs0 = __fmul2_rn(f2(-a.x, -a.y), va);
+  const float2 ea = __fmul2_rn(ev, va);
+  const float2 v = f2(gA ? vs0.x : 0.0f, gB ? vs0.y : 0.0f);
+  gr[5] = (gA ? ea.x : 0.0f) + (gB ? ea.y : 0.0f);
+  const float2 vdy = __fmul2_rn(v, dy);
+  const float2 vdy2 = __fmul2_rn(vdy, dy);
+  const float S0 = v.x + v.y, S1 = vdy.x + vdy.y, S2 = vdy2.x + vdy2.y;
+  const float ca = 2.0f * st.a.z, cb = st.a.w, cc = 2.0f * st.b.x;  // staged halves doubled exactly
+  const float dS0 = dx * S0;
+  gr[0] = fmaf(ca, dS0, cb * S1);
+  gr[1] = fmaf(cb, dS0, cc * S1);
+  gr[2] = 0.5f * dx * dS0;
+  gr[3] = dx * S1;
+  gr[4] = 0.5f * S2;
   return true;
 }
 
@@ -542,8 +569,6 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
           const int64_t idx = b0 + k;
           const Stage& st = s_e[k];
           float gr[9];
-#pragma unroll
-          for (int t = 0; t < 9; ++t) gr[t] = 0.0f;
           bool contrib = false;
           const bool liveA = idx <= pa.last, liveB = idx <= pb.last;
           if (liveA || liveB) {
@@ -554,9 +579,12 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
             const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
             if (needA || needB) {
               const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
-              if (needA) contrib |= pixel_grad(st, dx, dy.x, ev.x, amin, pa, gr);
-              if (needB) contrib |= pixel_grad(st, dx, dy.y, ev.y, amin, pb, gr);
+              contrib = pair_grad(st, dx, dy, ev, needA, needB, amin, pa, pb, gr);
             }
+          }
+          if (!contrib) {
+#pragma unroll
+            for (int t = 0; t < 9; ++t) gr[t] = 0.0f;
           }
           if (__any_sync(0xffffffffu, contrib)) {
             const float s8 = warp_reduce8(gr, lane);

@@ -351,13 +351,14 @@ Geo geometry(const orc_dims* d) {
 // Screen row: x, y, conic a, b, c, opacity, r, g, b, depth, 0, 0.
 template <typename R>
 struct Row {
-  R x, y, ca, cb, cc, o, rgb[3];
+  R x, y, ca, cb, cc, o, rgb[3], depth;
 };
 template <typename R>
 Row<R> load_row(const double* s) {
   Row<R> r;
   r.x = R(s[0]); r.y = R(s[1]); r.ca = R(s[2]); r.cb = R(s[3]); r.cc = R(s[4]); r.o = R(s[5]);
   r.rgb[0] = R(s[6]); r.rgb[1] = R(s[7]); r.rgb[2] = R(s[8]);
+  r.depth = R(s[9]);
   return r;
 }
 
@@ -380,11 +381,17 @@ struct Contrib {
 
 // Front-to-back compositing of one pixel over its tile list.  Records the
 // composited entries when `list` is given.
+//
+// Optional extensions (the "depth and T outputs, background blend" row): with
+// depth_out the pixel's expected depth D = sum_i w_i * depth_i is returned,
+// accumulated with the same weights w_i = alpha_i * T_i as the colour; with
+// bg (the camera's background colour) the returned colour is C + T * bg.
 template <typename R>
 void composite_pixel(const double* screen, const uint32_t* vals, int64_t beg, int64_t end, R px, R py,
                      R* rgb_out, R* T_out, int64_t* last_out, std::vector<Contrib>* list,
-                     int64_t* n_eval = nullptr, int64_t* n_comp = nullptr) {
-  R T = R(1), Cc[3] = {R(0), R(0), R(0)};
+                     int64_t* n_eval = nullptr, int64_t* n_comp = nullptr, R* depth_out = nullptr,
+                     const double* bg = nullptr) {
+  R T = R(1), Cc[3] = {R(0), R(0), R(0)}, D = R(0);
   int64_t last = -1;
   const R alpha_min = R(1) / R(255);
   for (int64_t i = beg; i < end; ++i) {
@@ -401,20 +408,28 @@ void composite_pixel(const double* screen, const uint32_t* vals, int64_t beg, in
     if (Tn < R(1e-4)) break;
     R w = alpha * T;
     for (int ch = 0; ch < 3; ++ch) Cc[ch] = fmaR(g.rgb[ch], w, Cc[ch]);
+    D = fmaR(g.depth, w, D);
     T = Tn;
     last = i;
     if (n_comp) ++*n_comp;
     if (list) list->push_back({i, !(oe < R(0.99))});
   }
-  for (int ch = 0; ch < 3; ++ch) rgb_out[ch] = Cc[ch];
+  for (int ch = 0; ch < 3; ++ch) rgb_out[ch] = bg ? fmaR(T, R(bg[ch]), Cc[ch]) : Cc[ch];
   *T_out = T;
   *last_out = last;
+  if (depth_out) *depth_out = D;
 }
 
 // Gradient of one pixel (fp64) given the composited list decided in the
 // forward precision.  Accumulates into v_screen rows (fp64, 12 per row).
+// With the extensions: gD = dL/dD for the expected depth (the depth is a
+// fourth "channel" composited with the same weights, so it enters dL/dalpha
+// like a colour and adds w_i * gD to the row's depth gradient), and bg adds
+// sum_ch g_ch * bg_ch to dL/dT_final (img = C + T_final * bg).
 void pixel_backward(const double* screen, const uint32_t* vals, const std::vector<Contrib>& list, double px,
-                    double py, const double* g, double vT, double* v_screen) {
+                    double py, const double* g, double vT, double* v_screen, double gD = 0.0,
+                    const double* bg = nullptr) {
+  if (bg) vT += g[0] * bg[0] + g[1] * bg[1] + g[2] * bg[2];
   size_t n = list.size();
   std::vector<double> alpha(n), e(n), T(n + 1);
   T[0] = 1.0;
@@ -427,7 +442,7 @@ void pixel_backward(const double* screen, const uint32_t* vals, const std::vecto
     T[j + 1] = T[j] * (1.0 - alpha[j]);
   }
   double Tfin = T[n];
-  double S[3] = {0.0, 0.0, 0.0};
+  double S[3] = {0.0, 0.0, 0.0}, Sd = 0.0;
   for (size_t jj = n; jj-- > 0;) {
     int64_t row = vals[list[jj].idx];
     Row<double> gr = load_row<double>(screen + row * kRow);
@@ -439,8 +454,11 @@ void pixel_backward(const double* screen, const uint32_t* vals, const std::vecto
       vr[6 + ch] += a * Ti * g[ch];
       v_alpha += g[ch] * (gr.rgb[ch] * Ti - S[ch] / (1.0 - a));
     }
+    vr[9] += a * Ti * gD;
+    v_alpha += gD * (gr.depth * Ti - Sd / (1.0 - a));
     v_alpha -= vT * Tfin / (1.0 - a);
     for (int ch = 0; ch < 3; ++ch) S[ch] += gr.rgb[ch] * a * Ti;
+    Sd += gr.depth * a * Ti;
     if (list[jj].clamped) continue;
     double v_o = e[jj] * v_alpha;
     double v_sig = -gr.o * e[jj] * v_alpha;
@@ -841,9 +859,11 @@ int orc_tile_ranges(const uint64_t* keys, int64_t n, int64_t n_tiles, int64_t* t
 // last_id [C][H][W].  precision 0: fp32 (canonical), 1: fp64.
 // Optional evals[npix]: entries each pixel evaluated (up to and including the
 // one that stopped it); comps[npix]: entries composited.
+// depth (nullable): expected depth per pixel; bg (nullable): [C][3]
+// background colours blended as img = C + T_final * bg.
 int orc_rasterize_fwd(const orc_dims* d, const double* screen, const uint32_t* vals, const int64_t* tile_off,
                       int precision, double* img, double* T_final, int64_t* last_id, int64_t* evals,
-                      int64_t* comps, int nthreads) {
+                      int64_t* comps, int nthreads, double* depth, const double* bg) {
   set_threads(nthreads);
   Geo geo = geometry(d);
   const int64_t npix = (int64_t)d->C * d->H * d->W;
@@ -857,18 +877,21 @@ int orc_rasterize_fwd(const orc_dims* d, const double* screen, const uint32_t* v
     int64_t j = rem / d->W, i = rem % d->W;
     int64_t t = c * geo.tiles_per_cam + (j / kTile) * geo.tiles_x + (i / kTile);
     int64_t last;
+    const double* bgc = bg ? bg + 3 * c : nullptr;
     if (precision == 0) {
-      float rgb[3], T;
+      float rgb[3], T, D;
       composite_pixel<float>(screen, vals, tile_off[t], tile_off[t + 1], (float)i + 0.5f, (float)j + 0.5f, rgb, &T,
-                             &last, nullptr, ev, cp);
+                             &last, nullptr, ev, cp, &D, bgc);
       for (int ch = 0; ch < 3; ++ch) img[3 * p + ch] = rgb[ch];
       T_final[p] = T;
+      if (depth) depth[p] = D;
     } else {
-      double rgb[3], T;
+      double rgb[3], T, D;
       composite_pixel<double>(screen, vals, tile_off[t], tile_off[t + 1], (double)i + 0.5, (double)j + 0.5, rgb,
-                              &T, &last, nullptr, ev, cp);
+                              &T, &last, nullptr, ev, cp, &D, bgc);
       for (int ch = 0; ch < 3; ++ch) img[3 * p + ch] = rgb[ch];
       T_final[p] = T;
+      if (depth) depth[p] = D;
     }
     last_id[p] = last;
   }
@@ -880,9 +903,10 @@ int orc_rasterize_fwd(const orc_dims* d, const double* screen, const uint32_t* v
 // v_T may be NULL.  Pixels are visited serially (deterministic sums); with
 // nthreads > 1 cameras/pixel blocks are split over per-thread fp64 buffers
 // that are added in thread order.
+// v_depth (nullable): dL/d(expected depth) per pixel; bg (nullable): [C][3].
 int orc_rasterize_bwd(const orc_dims* d, const double* screen, const uint32_t* vals, const int64_t* tile_off,
                       const double* v_img, const double* v_T, int precision, int64_t nnz, double* v_screen,
-                      int nthreads) {
+                      int nthreads, const double* v_depth, const double* bg) {
   set_threads(nthreads);
   Geo geo = geometry(d);
   const int64_t npix = (int64_t)d->C * d->H * d->W;
@@ -918,7 +942,8 @@ int orc_rasterize_bwd(const orc_dims* d, const double* screen, const uint32_t* v
       }
       double g[3] = {v_img[3 * p], v_img[3 * p + 1], v_img[3 * p + 2]};
       double vT = v_T ? v_T[p] : 0.0;
-      pixel_backward(screen, vals, list, (double)i + 0.5, (double)j + 0.5, g, vT, acc.data());
+      pixel_backward(screen, vals, list, (double)i + 0.5, (double)j + 0.5, g, vT, acc.data(),
+                     v_depth ? v_depth[p] : 0.0, bg ? bg + 3 * c : nullptr);
     }
   }
   for (int64_t q = 0; q < nnz * kRow; ++q) {

@@ -52,8 +52,8 @@ def lib():
         L.orc_intersect.argtypes = [P, P, P, P, i64, i32, P, P, i64, P]
         L.orc_sort.argtypes = [P, P, i64]
         L.orc_tile_ranges.argtypes = [P, i64, i64, P]
-        L.orc_rasterize_fwd.argtypes = [P, P, P, P, i32, P, P, P, P, P, i32]
-        L.orc_rasterize_bwd.argtypes = [P, P, P, P, P, P, i32, i64, P, i32]
+        L.orc_rasterize_fwd.argtypes = [P, P, P, P, i32, P, P, P, P, P, i32, P, P]
+        L.orc_rasterize_bwd.argtypes = [P, P, P, P, P, P, i32, i64, P, i32, P, P]
         L.orc_project_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i64, P, i32, P, P, P, P, P]
         L.orc_tile_counts.argtypes = [P, P, P, i64, P]
         L.orc_tile_lists.argtypes = [P, P, P, P, i64, P, i64, P, P, P, i64]
@@ -210,30 +210,35 @@ def tile_ranges(keys, n_tiles: int) -> np.ndarray:
 
 
 def rasterize_fwd(scene, screen, vals_sorted, tile_off, precision: int = 0, nthreads: int = 0,
-                  evals: bool = False):
+                  evals: bool = False, bg=None, depth: bool = False):
+    """img, T, last (then ev, cp with evals, then the expected depth with
+    depth=True).  bg: [C][3] background blended as img = C + T * bg."""
     d = dims_of(scene)
     img = np.zeros((scene.C, scene.H, scene.W, 3))
     T = np.zeros((scene.C, scene.H, scene.W))
     last = np.zeros((scene.C, scene.H, scene.W), np.int64)
     ev = np.zeros((scene.C, scene.H, scene.W), np.int64) if evals else None
     cp = np.zeros((scene.C, scene.H, scene.W), np.int64) if evals else None
+    D = np.zeros((scene.C, scene.H, scene.W)) if depth else None
+    bgc = None if bg is None else _c(np.asarray(bg, np.float64).reshape(scene.C, 3), np.float64)
     lib().orc_rasterize_fwd(ct.byref(d), _p(_c(screen, np.float64)), _p(_c(vals_sorted, np.uint32)),
                             _p(_c(tile_off, np.int64)), precision, _p(img), _p(T), _p(last), _p(ev), _p(cp),
-                            nthreads)
-    if evals:
-        return img, T, last, ev, cp
-    return img, T, last
+                            nthreads, _p(D), _p(bgc))
+    out = (img, T, last) + ((ev, cp) if evals else ()) + ((D,) if depth else ())
+    return out
 
 
 def rasterize_bwd(scene, screen, vals_sorted, tile_off, v_img, v_T=None, precision: int = 0,
-                  nthreads: int = 0) -> np.ndarray:
+                  nthreads: int = 0, v_depth=None, bg=None) -> np.ndarray:
     d = dims_of(scene)
     n = len(screen)
     vs = np.zeros((max(n, 1), ROW))
     vT = None if v_T is None else _c(v_T, np.float64)
+    vD = None if v_depth is None else _c(v_depth, np.float64)
+    bgc = None if bg is None else _c(np.asarray(bg, np.float64).reshape(scene.C, 3), np.float64)
     lib().orc_rasterize_bwd(ct.byref(d), _p(_c(screen, np.float64)), _p(_c(vals_sorted, np.uint32)),
                             _p(_c(tile_off, np.int64)), _p(_c(v_img, np.float64)), _p(vT), precision, n,
-                            _p(vs), nthreads)
+                            _p(vs), nthreads, _p(vD), _p(bgc))
     return vs[:n]
 
 
@@ -259,24 +264,29 @@ def upstream(scene, img) -> np.ndarray:
     return (np.sign(np.asarray(img, np.float64) - scene.target) * scene.l1_scale).astype(np.float32)
 
 
-def forward(scene, precision: int = 0, nthreads: int = 0) -> dict:
+def forward(scene, precision: int = 0, nthreads: int = 0, bg=None, depth: bool = False) -> dict:
     g = geometry(scene)
     proj = project(scene, precision, nthreads)
     isect = intersect(scene, proj)
     ks, vs = sort(isect["keys"], isect["vals"])
     toff = tile_ranges(ks, g["n_tiles"])
-    img, T, last = rasterize_fwd(scene, proj["screen"], vs, toff, precision, nthreads)
-    return dict(proj=proj, isect=isect, keys_sorted=ks, vals_sorted=vs, tile_off=toff, img=img, T=T,
-                last=last, geo=g)
+    r = rasterize_fwd(scene, proj["screen"], vs, toff, precision, nthreads, bg=bg, depth=depth)
+    f = dict(proj=proj, isect=isect, keys_sorted=ks, vals_sorted=vs, tile_off=toff, img=r[0], T=r[1],
+             last=r[2], geo=g)
+    if depth:
+        f["depth"] = r[3]
+    return f
 
 
-def step(scene, precision: int = 0, nthreads: int = 0, v_img=None, v_T=None) -> dict:
-    """One forward+backward pass; gradients in fp64."""
-    f = forward(scene, precision, nthreads)
+def step(scene, precision: int = 0, nthreads: int = 0, v_img=None, v_T=None, v_depth=None, bg=None) -> dict:
+    """One forward+backward pass; gradients in fp64.  With v_depth the
+    forward also returns the expected depth and the backward takes its
+    gradient; bg blends a background colour per camera."""
+    f = forward(scene, precision, nthreads, bg=bg, depth=v_depth is not None)
     if v_img is None:
         v_img = upstream(scene, f["img"])
     v_screen = rasterize_bwd(scene, f["proj"]["screen"], f["vals_sorted"], f["tile_off"], v_img, v_T, precision,
-                             nthreads)
+                             nthreads, v_depth=v_depth, bg=bg)
     grads = project_bwd(scene, f["proj"], v_screen, precision)
     f.update(v_img=v_img, v_screen=v_screen, grads=grads)
     return f

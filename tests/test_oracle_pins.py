@@ -17,8 +17,11 @@ in the oracle (a dropped term, a wrong sign or index, a transposed operand):
                grow by at most one tile per side;
 * sort/ranges: numpy's stable lexsort and bincount;
 * rasterizer:  closed form of one Gaussian, telescoping sum, the 0.99 clamp
-               hand count;
-* backward:    central finite differences of the fp64 instantiation.
+               hand count; expected depth and background: the one-Gaussian
+               closed form and, for Gaussians at one camera depth z0, the
+               telescoped depth z0 * (1 - T);
+* backward:    central finite differences of the fp64 instantiation, with and
+               without the depth output and a background colour.
 """
 import math
 
@@ -338,6 +341,39 @@ def test_clamped_opacity_stops_after_one():
     np.testing.assert_allclose(f["img"][0], 0.5 * 0.99, rtol=1e-6)
 
 
+def test_single_gaussian_depth_and_background():
+    """One Gaussian at camera depth z: D = alpha * z and img = 0.5 alpha + (1 - alpha) bg
+    where it is composited; D = 0 and img = bg elsewhere."""
+    fx = fy = 50.0
+    W = H = 48
+    z, o = 2.5, 0.8
+    bg = np.array([[0.2, 0.6, 0.9]])
+    sc = make([[0.1, -0.05, z]], [[1.0, 0.0, 0.0, 0.0]], [[0.04, 0.03, 0.05]], [o], [[0.0, 0.0, 0.0]],
+              [ident_cam(fx, fy, 24.0, 24.0)], W, H)
+    for prec, tol in ((0, 2e-6), (1, 1e-12)):
+        f = orc.forward(sc, prec, bg=bg, depth=True)
+        alpha = 1.0 - f["T"][0]  # one composited entry: T = 1 - alpha
+        comp = f["last"][0] >= 0
+        np.testing.assert_allclose(f["depth"][0][comp], (alpha * z)[comp], rtol=tol, atol=tol)
+        assert np.all(f["depth"][0][~comp] == 0.0)
+        for ch in range(3):
+            want = np.where(comp, 0.5 * alpha + (1.0 - alpha) * bg[0, ch], bg[0, ch])
+            np.testing.assert_allclose(f["img"][0, ..., ch], want, atol=10 * tol)
+
+
+def test_coplanar_depth_telescopes():
+    """All Gaussians at one camera depth z0: the weights sum to 1 - T, so the
+    expected depth is z0 * (1 - T) at every pixel."""
+    rng = np.random.default_rng(9)
+    N, z0 = 80, 3.0
+    means = np.concatenate([rng.uniform(-0.6, 0.6, (N, 2)), np.full((N, 1), z0)], 1)
+    for prec, tol in ((0, 3e-5), (1, 1e-12)):
+        sc = make(means, rng.normal(size=(N, 4)), np.exp(rng.uniform(-3.5, -2.0, (N, 3))),
+                  rng.uniform(0.2, 0.95, N), rng.uniform(0.0, 1.0, (N, 3)), [ident_cam(40, 40, 24, 20)], 48, 40)
+        f = orc.forward(sc, prec, depth=True)
+        np.testing.assert_allclose(f["depth"], z0 * (1.0 - f["T"]), atol=tol * z0)
+
+
 def test_fp32_forward_close_to_fp64():
     sc = scenes.make_scene(1)
     a = render(sc, 0)
@@ -348,13 +384,19 @@ def test_fp32_forward_close_to_fp64():
 
 
 # ---------------------------------------------------------------- backward vs finite differences
-def loss(sc, v_img, v_T):
-    f = orc.forward(sc, precision=1)
-    return float(np.sum(f["img"] * v_img) + np.sum(f["T"] * v_T))
+def loss(sc, v_img, v_T, v_D=None, bg=None):
+    f = orc.forward(sc, precision=1, bg=bg, depth=v_D is not None)
+    L = float(np.sum(f["img"] * v_img) + np.sum(f["T"] * v_T))
+    if v_D is not None:
+        L += float(np.sum(f["depth"] * v_D))
+    return L
 
 
-@pytest.mark.parametrize("seed", range(8))
-def test_backward_central_differences(seed):
+@pytest.mark.parametrize("seed,ext", [(s, False) for s in range(8)] + [(s, True) for s in (8, 9, 10, 11)])
+def test_backward_central_differences(seed, ext):
+    """ext: the loss also weighs the expected depth and the colour carries a
+    background (the depth gradient then reaches the means through the camera
+    depth, and the background through dL/dT)."""
     sc = scenes.random_tiny(seed, N=5, W=32, H=32, C=2 if seed % 2 else 1, sh_degree=seed % 4,
                             opacity_range=(0.1, 0.9))
     # fp64 parameters so the differences are not quantised to fp32
@@ -363,7 +405,9 @@ def test_backward_central_differences(seed):
     rng = np.random.default_rng(seed)
     v_img = rng.uniform(-1, 1, (sc.C, sc.H, sc.W, 3))
     v_T = rng.uniform(-1, 1, (sc.C, sc.H, sc.W))
-    r = orc.step(sc, precision=1, v_img=v_img, v_T=v_T)
+    v_D = rng.uniform(-1, 1, (sc.C, sc.H, sc.W)) if ext else None
+    bg = rng.uniform(0, 1, (sc.C, 3)) if ext else None
+    r = orc.step(sc, precision=1, v_img=v_img, v_T=v_T, v_depth=v_D, bg=bg)
     gr = r["grads"]
     names = {"means": "v_means", "quats": "v_quats", "scales": "v_scales", "opacities": "v_opacities",
              "sh": "v_sh"}
@@ -378,9 +422,9 @@ def test_backward_central_differences(seed):
             for h in (1e-6, 5e-7):
                 hh = h * max(1.0, abs(x0))
                 flat[i] = x0 + hh
-                lp = loss(sc, v_img, v_T)
+                lp = loss(sc, v_img, v_T, v_D, bg)
                 flat[i] = x0 - hh
-                lm = loss(sc, v_img, v_T)
+                lm = loss(sc, v_img, v_T, v_D, bg)
                 flat[i] = x0
                 vals.append((lp - lm) / (2 * hh))
             # two step sizes that disagree mean a threshold (1/255, 3-sigma tile edge) was crossed

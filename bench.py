@@ -181,12 +181,20 @@ def run_ours(args):
     d = ss.scene_dims(sc)
     inputs = ss.scene_tensors(sc, dev)
     step = ss.PackedStep(d, dev)
-    step.forward(*inputs)
+    # optional depth output + background blend (forward) and depth gradient
+    # (backward), seeded inputs
+    fkw, bkw, bg_t, v_D = {}, {}, None, None
+    if args.depth_bg:
+        g_ext = torch.Generator(device="cpu").manual_seed(1234)
+        bg_t = torch.rand((d.C, 3), generator=g_ext).to(dev)
+        v_D = ((torch.rand((d.C, d.H, d.W), generator=g_ext) * 2 - 1) / (d.W * d.H)).to(dev)
+        fkw, bkw = dict(bg=bg_t, depth=True), dict(v_depth=v_D)
+    step.forward(*inputs, **fkw)
     torch.cuda.synchronize()
     # capacities with headroom, then the upstream gradient from this forward
     step._rows(int(step.nnz * 1.05) + 1)
     step._isects(int(step.n_isects * 1.05) + 1)
-    img = step.forward(*inputs)
+    img = step.forward(*inputs, **fkw)
     if sc.upstream == "l1":
         target = torch.from_numpy(sc.target).to(dev)
         v_img = (torch.sign(img - target) * sc.l1_scale).contiguous()
@@ -201,12 +209,12 @@ def run_ours(args):
     def run_step(ev=None):
         if ev is not None:
             ev[0].record(st)
-        step.forward(*inputs, stream=None) if ev is None else _timed_forward(ev)
+        step.forward(*inputs, stream=None, **fkw) if ev is None else _timed_forward(ev)
         if ev is None:
-            step.backward(v_img)
+            step.backward(v_img, **bkw)
         else:
             ss.ss_rasterize_bwd(d, step.screen, step.vals, step.tile_off, step.T, step.last, v_img, None,
-                                step.v_screen, step.nnz)
+                                step.v_screen, step.nnz, v_depth=v_D, bg=bg_t)
             ev[5].record(st)
             ss.ss_project_bwd(d, *inputs, step.mask, step.block_off, step.v_screen, step.v_means, step.v_quats,
                               step.v_scales, step.v_opacities, step.v_sh)
@@ -224,13 +232,14 @@ def run_ours(args):
                                  step.tile_off)
         step.vals = step.vals_b if in_b else step.vals_a
         ev[3].record(st)
-        ss.ss_rasterize_fwd(d, step.screen, step.vals, step.tile_off, step.img, step.T, step.last)
+        ss.ss_rasterize_fwd(d, step.screen, step.vals, step.tile_off, step.img, step.T, step.last,
+                            step.depth if args.depth_bg else None, bg_t)
         ev[4].record(st)
         step.nnz, step.n_isects = nnz, n
 
     for _ in range(args.warmup):
-        step.forward(*inputs)
-        step.backward(v_img)
+        step.forward(*inputs, **fkw)
+        step.backward(v_img, **bkw)
     torch.cuda.synchronize()
 
     # ---- headline: K whole steps, device-timed, max over ranks
@@ -243,8 +252,8 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(st)
     for _ in range(args.steps):
-        step.forward(*inputs)
-        step.backward(v_img)
+        step.forward(*inputs, **fkw)
+        step.backward(v_img, **bkw)
     t1.record(st)
     torch.cuda.synchronize()
     if world > 1:
@@ -286,8 +295,8 @@ def run_ours(args):
             for a, b in zip(dev_in, host_in):
                 a.copy_(b, non_blocking=True)
             dev_vimg.copy_(host_vimg, non_blocking=True)
-            step.forward(*dev_in)
-            g = step.backward(dev_vimg)
+            step.forward(*dev_in, **fkw)
+            g = step.backward(dev_vimg, **bkw)
             for k, h in host_out.items():
                 h.copy_(g[k], non_blocking=True)
 
@@ -333,6 +342,12 @@ def run_ours(args):
         f_alu = alu / fp32_peak_instr_per_s(sm_mhz) if ins else 0.0
         stages[nm] = dict(ms=round(stage_ms[nm], 4), hbm_gbs=round(hbm, 1), hbm_frac=round(f_hbm, 4),
                           alu_frac=round(f_alu, 4), bound="alu" if f_alu > f_hbm else "hbm")
+    # whole-step fraction: sum over stages of the roofline time (the slower of
+    # bytes at the HBM peak and FP32 instructions at the FP32 peak) over the
+    # sum of measured stage times
+    t_roof = sum(max(model[nm]["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                     model[nm]["instr"] / fp32_peak_instr_per_s(sm_mhz)) for nm in names)
+    step_frac = t_roof / (sum(stage_ms.values()) / 1e3)
     dom = max(names, key=lambda k: stage_ms[k])
     sd = stages[dom]
     if sd["bound"] == "hbm":
@@ -352,8 +367,10 @@ def run_ours(args):
                config=dict(workload=f"config {args.config}: {sc.name}", C=d.C, N=d.N, W=d.W, H=d.H,
                            sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
                            sort_passes=passes, l2="inputs larger than L2 (3.5 GB parameters), no flush",
-                           parallelism=f"replicas x{world}"),
-               pairs_per_s=world * d.C * d.N / (ms / 1e3), raster_work=out_work, stages=stages, roofline=roof,
+                           parallelism=f"replicas x{world}", depth_and_background=bool(args.depth_bg)),
+               pairs_per_s=world * d.C * d.N / (ms / 1e3),
+               pixel_gaussian_evals_per_s=world * work["evals"] / (stage_ms["rasterize_fwd"] / 1e3),
+               step_roofline_frac=round(step_frac, 4), raster_work=out_work, stages=stages, roofline=roof,
                clocks=clocks,
                e2e=e2e, gpu_launches=launches)
     if not args.no_cpu_baseline:
@@ -423,6 +440,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=300_000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--depth-bg", action="store_true",
+                    help="also render the expected depth over a background colour and back-propagate a depth gradient")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -12,6 +12,7 @@ thread_local std::string g_last_error;
 void set_error(const std::string& msg) { g_last_error = msg; }
 
 size_t sort_temp_bytes(int64_t n);
+size_t isect_temp_bytes(int64_t nnz);
 
 }  // namespace ss
 
@@ -36,7 +37,7 @@ extern "C" size_t ss_workspace_bytes(const ss_dims* dims, int which, int64_t cou
   const Geo g = geometry(*dims);
   switch (which) {
     case SS_WS_PROJECT: return scan_temp_bytes(max64(g.mask_blocks, 1));
-    case SS_WS_INTERSECT: return scan_temp_bytes(max64(count, 1));
+    case SS_WS_INTERSECT: return isect_temp_bytes(max64(count, 1));
     case SS_WS_SORT: return sort_temp_bytes(max64(count, 1));
     default: return 0;
   }

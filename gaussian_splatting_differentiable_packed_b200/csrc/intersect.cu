@@ -6,9 +6,11 @@
 // Count: per-row tiles from the AABB16 by integer arithmetic, CTA sums and a
 // single-CTA scan of the sums give the exact int64 total (no atomics, so the
 // total is deterministic).  Offsets: block scan per 4096 rows.  Write: load
-// balanced over output slots — each thread owns 8 consecutive slots, finds
-// the row of its first slot by binary search in the offsets and walks on, so
-// stores are contiguous whatever the per-row tile counts.
+// balanced over output slots — each thread owns 8 consecutive slots of a
+// 2048-slot chunk, finds the row of its first slot by binary search in the
+// chunk's row range (each chunk's first row comes from one pass over the
+// rows) and walks on; the chunk is staged in shared memory and stored
+// contiguously, whatever the per-row tile counts.
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 
@@ -36,20 +38,11 @@ __device__ __forceinline__ int find_cam(const int64_t* block_off, int64_t blocks
   return lo;
 }
 
-__global__ __launch_bounds__(kWrThreads) void k_isect_write(Geo g, const float* __restrict__ screen,
-                                                            const uint32_t* __restrict__ aabb16,
-                                                            const int64_t* __restrict__ block_off,
-                                                            const int64_t* __restrict__ off, int64_t nnz,
-                                                            int64_t limit, uint64_t* __restrict__ keys,
-                                                            uint32_t* __restrict__ vals) {
-  __shared__ int64_t s_lo, s_hi;
-  const int64_t s0 = (int64_t)blockIdx.x * kWrTile;
-  if (threadIdx.x == 0) s_lo = find_row(off, 0, nnz, s0);
-  if (threadIdx.x == 1) s_hi = find_row(off, 0, nnz, min(s0 + kWrTile, limit) - 1) + 1;
-  __syncthreads();
-  int64_t s = s0 + (int64_t)threadIdx.x * kWrItems;
-  if (s >= limit) return;
-  int64_t r = find_row(off, s_lo, s_hi, s);
+// Slots [s, s_stop) of rows starting at row r, into the CTA's staging arrays.
+__device__ __forceinline__ void slot_run(const Geo& g, const float* __restrict__ screen,
+                                         const uint32_t* __restrict__ aabb16, const int64_t* __restrict__ block_off,
+                                         const int64_t* __restrict__ off, int64_t r, int64_t s, int64_t s_stop,
+                                         int64_t s0, uint64_t* s_key, uint32_t* s_val) {
   int c = find_cam(block_off, g.blocks_per_cam, g.C, r);
   int64_t r_end = off[r + 1];
   int tx0, tx1, ty0, ty1, w;
@@ -63,7 +56,6 @@ __global__ __launch_bounds__(kWrThreads) void k_isect_write(Geo g, const float* 
   };
   decode(r);
   int64_t k = s - off[r];
-  const int64_t s_stop = min(s + kWrItems, limit);
   for (; s < s_stop; ++s, ++k) {
     while (s >= r_end) {  // next row with at least one tile
       ++r;
@@ -74,9 +66,56 @@ __global__ __launch_bounds__(kWrThreads) void k_isect_write(Geo g, const float* 
     }
     const int ty = ty0 + (int)(k / w), tx = tx0 + (int)(k % w);
     const uint64_t tile = (uint64_t)c * (uint64_t)g.tiles_per_cam + (uint64_t)ty * g.tiles_x + (uint64_t)tx;
-    keys[s] = (tile << 32) | dbits;
-    vals[s] = (uint32_t)r;
+    const int64_t i = s - s0;
+    s_key[i + i / kWrItems] = (tile << 32) | dbits;
+    s_val[i + i / kWrItems] = (uint32_t)r;
   }
+}
+
+// first[k] = the row holding slot k * kWrTile, for every chunk start below
+// limit (one thread per row; a row spanning several chunk starts writes each).
+__global__ void k_chunk_first(const int64_t* __restrict__ off, int64_t nnz, int64_t limit,
+                              int64_t* __restrict__ first) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= nnz) return;
+  const int64_t a = off[r], b = min64(off[r + 1], limit);
+  for (int64_t k = (a + kWrTile - 1) / kWrTile; k * kWrTile < b; ++k) first[k] = r;
+}
+
+// One CTA per 2048-slot chunk; the chunk's rows are first[blk] .. first[blk+1].
+__global__ __launch_bounds__(kWrThreads) void k_isect_write(Geo g, const float* __restrict__ screen,
+                                                            const uint32_t* __restrict__ aabb16,
+                                                            const int64_t* __restrict__ block_off,
+                                                            const int64_t* __restrict__ off, int64_t nnz,
+                                                            int64_t limit, const int64_t* __restrict__ first,
+                                                            uint64_t* __restrict__ keys, uint32_t* __restrict__ vals) {
+  // the chunk's slots, written back coalesced; one pad word after every
+  // kWrItems so that a thread's run of kWrItems slots does not share banks
+  // with its neighbours' runs
+  __shared__ uint64_t s_key[kWrTile + kWrThreads];
+  __shared__ uint32_t s_val[kWrTile + kWrThreads];
+  const int64_t blk = blockIdx.x;
+  const int64_t nch = (limit + kWrTile - 1) / kWrTile;
+  const int64_t s0 = blk * kWrTile;
+  const int64_t s_end = min64(s0 + kWrTile, limit);
+  const int64_t lo = first[blk], hi = blk + 1 < nch ? first[blk + 1] + 1 : nnz;
+  const int64_t s = s0 + (int64_t)threadIdx.x * kWrItems;
+  if (s < s_end)
+    slot_run(g, screen, aabb16, block_off, off, find_row(off, lo, hi, s), s, min64(s + kWrItems, s_end), s0, s_key,
+             s_val);
+  __syncthreads();
+  const int cnt = (int)(s_end - s0);
+  for (int i = threadIdx.x; i < cnt; i += kWrThreads) {
+    keys[s0 + i] = s_key[i + i / kWrItems];
+    vals[s0 + i] = s_val[i + i / kWrItems];
+  }
+}
+
+// Workspace: the scan's scratch, then first[] for the largest chunk count
+// (n_isects < 2^31).
+constexpr int64_t kMaxChunks = ((int64_t(1) << 31) + kWrTile - 1) / kWrTile;
+size_t isect_temp_bytes(int64_t nnz) {
+  return scan_temp_bytes(nnz) + align_up((size_t)(kMaxChunks + 1) * sizeof(int64_t), 256);
 }
 
 }  // namespace ss
@@ -126,7 +165,10 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* screen
   if (total == 0) return SS_OK;
   if (!keys || !vals) return invalid("null keys/vals");
   const int64_t limit = min64(total, cap_isects);
-  const unsigned grid = (unsigned)ceil_div(limit, kWrTile);
-  k_isect_write<<<grid, kWrThreads, 0, st>>>(g, screen, aabb16, block_off, isect_off, nnz, limit, keys, vals);
+  const int64_t nch = ceil_div(limit, kWrTile);
+  int64_t* first = reinterpret_cast<int64_t*>(reinterpret_cast<char*>(temp) + scan_temp_bytes(nnz));
+  k_chunk_first<<<(unsigned)ceil_div(nnz, 256), 256, 0, st>>>(isect_off, nnz, limit, first);
+  k_isect_write<<<(unsigned)nch, kWrThreads, 0, st>>>(g, screen, aabb16, block_off, isect_off, nnz, limit, first, keys,
+                                                      vals);
   return cuda_status(cudaGetLastError(), "intersect write");
 }

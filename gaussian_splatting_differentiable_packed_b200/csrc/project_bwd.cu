@@ -104,13 +104,39 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   const int64_t n = n0 + threadIdx.x;
   const bool valid = n < g.N;
   const int cnt = (int)min64(kBlock, g.N - n0);
-  // coalesced staging of the CTA's contiguous SH block
+  // coalesced staging of the CTA's contiguous SH block: full blocks with all
+  // 16-byte loads in flight at once (the block starts 16-byte aligned: 128*K3
+  // floats per block), the ragged last block word by word
   {
     const float* src = sh + n0 * K3;
-    for (int f = threadIdx.x; f < kBlock * K3; f += kBlock) {
-      const int gi = f / K3, q = f - gi * K3;
-      sh_s[gi * KP + q] = f < cnt * K3 ? src[f] : 0.0f;
-      gsh_s[gi * KP + q] = 0.0f;
+    if (cnt == kBlock) {
+      constexpr int kV = kBlock * K3 / 4;
+      constexpr int kPer = (kV + kBlock - 1) / kBlock;
+      float4 buf[kPer];
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int v = threadIdx.x + r * kBlock;
+        if (v < kV) buf[r] = reinterpret_cast<const float4*>(src)[v];
+      }
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int v = threadIdx.x + r * kBlock;
+        if (v < kV) {
+          const float e[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int f = 4 * v + u, gi = f / K3, q = f - gi * K3;
+            sh_s[gi * KP + q] = e[u];
+            gsh_s[gi * KP + q] = 0.0f;
+          }
+        }
+      }
+    } else {
+      for (int f = threadIdx.x; f < kBlock * K3; f += kBlock) {
+        const int gi = f / K3, q = f - gi * K3;
+        sh_s[gi * KP + q] = f < cnt * K3 ? src[f] : 0.0f;
+        gsh_s[gi * KP + q] = 0.0f;
+      }
     }
   }
   const float* shn = sh_s + threadIdx.x * KP;
@@ -143,12 +169,30 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     // its busiest Gaussian has cameras, not one round per camera of the chunk.
     uint32_t vis = 0;
     for (int cc = 0; cc < nc; ++cc) vis |= ((s_word[cc][warp] >> lane) & 1u) << cc;
+    // the gradient row of the next visible camera is loaded one round ahead
+    // (x, y, ca, cb | cc, o, r, g | b, depth)
+    const uint32_t below = (1u << lane) - 1u;
+    float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
+    float2 n2 = make_float2(0.f, 0.f);
+    if (vis) {
+      const int cc = __ffs(vis) - 1;
+      const float* rp = v_screen + (s_row0[cc][warp] + __popc(s_word[cc][warp] & below)) * kRowF;
+      n0 = reinterpret_cast<const float4*>(rp)[0];
+      n1 = reinterpret_cast<const float4*>(rp)[1];
+      n2 = reinterpret_cast<const float2*>(rp)[4];
+    }
     while (vis) {
       const int cc = __ffs(vis) - 1;
       vis &= vis - 1;
-      const int64_t row = s_row0[cc][warp] + __popc(s_word[cc][warp] & ((1u << lane) - 1u));
-      const float4* vrp = reinterpret_cast<const float4*>(v_screen + row * kRowF);
-      const float4 v0 = vrp[0], v1 = vrp[1], v2 = vrp[2];
+      const float4 v0 = n0, v1 = n1;
+      const float2 v2 = n2;
+      if (vis) {
+        const int cn = __ffs(vis) - 1;
+        const float* rp = v_screen + (s_row0[cn][warp] + __popc(s_word[cn][warp] & below)) * kRowF;
+        n0 = reinterpret_cast<const float4*>(rp)[0];
+        n1 = reinterpret_cast<const float4*>(rp)[1];
+        n2 = reinterpret_cast<const float2*>(rp)[4];
+      }
       const Cam& k = scam[cc];
       const float* R = k.R;
       // camera point and the projection's gating decision in canonical arithmetic
@@ -292,11 +336,24 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     v_opac[n] = go;
   }
   __syncthreads();
-  // coalesced write-back of the CTA's SH gradient block
+  // coalesced write-back of the CTA's SH gradient block (16-byte stores for a
+  // full block)
   float* dst = v_sh + n0 * K3;
-  for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-    const int gi = f / K3, q = f - gi * K3;
-    dst[f] = gsh_s[gi * KP + q];
+  if (cnt == kBlock) {
+    for (int v = threadIdx.x; v < kBlock * K3 / 4; v += kBlock) {
+      float e[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int f = 4 * v + u, gi = f / K3, q = f - gi * K3;
+        e[u] = gsh_s[gi * KP + q];
+      }
+      reinterpret_cast<float4*>(dst)[v] = make_float4(e[0], e[1], e[2], e[3]);
+    }
+  } else {
+    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+      const int gi = f / K3, q = f - gi * K3;
+      dst[f] = gsh_s[gi * KP + q];
+    }
   }
 }
 
@@ -328,8 +385,9 @@ extern "C" ss_status ss_project_bwd(const ss_dims* dims, const float* cams, cons
   if (g.N == 0) return SS_OK;
   if (!cams || !means || !quats || !scales || !sh || !mask || !block_off || !v_screen) return invalid("null input");
   if (!v_means || !v_quats || !v_scales || !v_opacities || !v_sh) return invalid("null output");
-  if (((uintptr_t)quats & 15) || ((uintptr_t)v_quats & 15) || ((uintptr_t)v_screen & 15))
-    return invalid("quats, v_quats and v_screen must be 16-byte aligned");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)v_quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15) ||
+      ((uintptr_t)v_sh & 15))
+    return invalid("quats, v_quats, v_screen, sh and v_sh must be 16-byte aligned");
   (void)opacities;
   cudaStream_t st = as_stream(stream);
   const unsigned grid = (unsigned)g.blocks_per_cam;

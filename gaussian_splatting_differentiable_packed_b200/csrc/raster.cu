@@ -10,8 +10,13 @@
 // pair is rounded exactly like the scalar operation, so the canonical order is
 // kept bit for bit).  Warp w owns the 16x4 region of rows 4w..4w+3.  Each batch
 // of 256 sorted entries is gathered once into shared memory (three 16-byte
-// loads per 48-byte screen row) and each warp builds its own candidate list by
-// ballot, skipping entries that provably miss its region (see warp_culled).
+// loads per 48-byte screen row).  Per block of 32 staged entries each lane
+// computes which of its warp's 64 pixels one entry can reach (outward-rounded
+// ellipse chords, see entry_coverage) and a warp bit-transpose hands every
+// lane the candidate entries of its own two pixels: the forward walks its own
+// list, the backward steps its warp through the union of the lists (it needs
+// the warp together for the gradient reduction).  The counting forward culls
+// by region box (warp_culled).
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 
@@ -52,7 +57,7 @@ struct Stage {
   float4 b;  // 0.5*cc, o, r, g
   float4 c;  // b, hx, hy, kterm = |ha| + |hc| + |cb|
   float4 d;  // thr, row (bits), P = 2*ca*kCullT, dql
-  float4 e;  // 1/ca, cb/ca, bounded (1/0), 0
+  float4 e;  // 1/ca, cb/ca, bounded (1/0), depth
 };
 
 __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint32_t r, Stage& st) {
@@ -77,7 +82,7 @@ __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint
   const float kterm = 0.5f * fabsf(ca) + 0.5f * fabsf(cc) + fabsf(cb);
   st.c = make_float4(r2.x, hx, hy, kterm);
   st.d = make_float4(o <= 1.0f ? SS_SIGMA_SKIP : inf, __uint_as_float(r), P, dql);
-  st.e = make_float4(ica, cbr, bounded, 0.0f);
+  st.e = make_float4(ica, cbr, bounded, r2.y);
 }
 
 // Warp culling.  For an entry with o <= 1 every pixel whose computed sigma
@@ -127,9 +132,12 @@ __device__ __forceinline__ float2 exp_neg_pair(float2 x) {
   return e;
 }
 
-// One pixel's front-to-back step for an entry whose sigma passed the tests.
+// One pixel's front-to-back step for an entry whose sigma passed the tests;
+// with EXT also the expected depth, accumulated with the colour's weight.
+template <bool EXT = false>
 __device__ __forceinline__ void composite(const Stage& st, float oe, float amin, int64_t idx, float& T, float& C0,
-                                          float& C1, float& C2, int64_t& last, bool& done, unsigned long long& ncomp) {
+                                          float& C1, float& C2, float& D, int64_t& last, bool& done,
+                                          unsigned long long& ncomp) {
   const float alpha = fminf(SS_ALPHA_MAX, oe);
   if (alpha < amin) return;
   const float Tn = mul(T, sub(1.0f, alpha));
@@ -141,6 +149,7 @@ __device__ __forceinline__ void composite(const Stage& st, float oe, float amin,
   C0 = fma_(st.b.z, w, C0);
   C1 = fma_(st.b.w, w, C1);
   C2 = fma_(st.c.x, w, C2);
+  if (EXT) D = fma_(st.e.w, w, D);
   T = Tn;
   last = idx;
   ++ncomp;
@@ -170,7 +179,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd(Geo g, const float* __
   const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f, y_hi = y_lo + 3.0f;
   const int64_t beg = tile_off[tile], end = tile_off[tile + 1];
   const float amin = alpha_min();
-  float TA = 1.0f, A0 = 0.0f, A1 = 0.0f, A2 = 0.0f, TB = 1.0f, B0 = 0.0f, B1 = 0.0f, B2 = 0.0f;
+  float TA = 1.0f, A0 = 0.0f, A1 = 0.0f, A2 = 0.0f, TB = 1.0f, B0 = 0.0f, B1 = 0.0f, B2 = 0.0f, DA = 0.0f,
+        DB = 0.0f;
   int64_t lastA = -1, lastB = -1;
   bool doneA = !inA, doneB = !inB;
   unsigned long long n_eval = 0, n_exp = 0, n_comp = 0, n_expA_last = 0, n_expB_last = 0, n_expA = 0, n_expB = 0;
@@ -206,7 +216,7 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd(Geo g, const float* __
             ++n_expA;
           }
           const int64_t before = lastA;
-          composite(st, oe.x, amin, idx, TA, A0, A1, A2, lastA, doneA, n_comp);
+          composite(st, oe.x, amin, idx, TA, A0, A1, A2, DA, lastA, doneA, n_comp);
           if (COUNT && lastA != before) n_expA_last = n_expA;
         }
         if (needB) {
@@ -215,7 +225,7 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd(Geo g, const float* __
             ++n_expB;
           }
           const int64_t before = lastB;
-          composite(st, oe.y, amin, idx, TB, B0, B1, B2, lastB, doneB, n_comp);
+          composite(st, oe.y, amin, idx, TB, B0, B1, B2, DB, lastB, doneB, n_comp);
           if (COUNT && lastB != before) n_expB_last = n_expB;
         }
       }
@@ -328,11 +338,16 @@ __device__ __forceinline__ void entry_coverage(const Stage& st, float x_lo, floa
   covB = s1 | (s3 << 16);
 }
 
+// EXT: also the expected depth (depth, nullable) and a background colour per
+// camera (bg [C][3], nullable) blended as img = C + T_final * bg.
+template <bool EXT>
 __global__ __launch_bounds__(kRThreads) void k_raster_fwd_masked(Geo g, const float* __restrict__ screen,
                                                                  const uint32_t* __restrict__ vals,
                                                                  const int64_t* __restrict__ tile_off,
                                                                  float* __restrict__ img, float* __restrict__ T_final,
-                                                                 int32_t* __restrict__ last_id) {
+                                                                 int32_t* __restrict__ last_id,
+                                                                 float* __restrict__ depth,
+                                                                 const float* __restrict__ bg) {
   __shared__ Stage s_e[kBatch];
   const int lane = threadIdx.x & 31;
   const int64_t tile = blockIdx.x;
@@ -345,7 +360,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd_masked(Geo g, const fl
   const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f;
   const int64_t beg = tile_off[tile], end = tile_off[tile + 1];
   const float amin = alpha_min();
-  float TA = 1.0f, A0 = 0.0f, A1 = 0.0f, A2 = 0.0f, TB = 1.0f, B0 = 0.0f, B1 = 0.0f, B2 = 0.0f;
+  float TA = 1.0f, A0 = 0.0f, A1 = 0.0f, A2 = 0.0f, TB = 1.0f, B0 = 0.0f, B1 = 0.0f, B2 = 0.0f, DA = 0.0f,
+        DB = 0.0f;
   int64_t lastA = -1, lastB = -1;
   bool doneA = !inA, doneB = !inB;
   unsigned long long ncomp = 0;
@@ -380,19 +396,29 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd_masked(Geo g, const fl
         const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
         const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
         const int64_t idx = b0 + k;
-        if (needA) composite(st, oe.x, amin, idx, TA, A0, A1, A2, lastA, doneA, ncomp);
-        if (needB) composite(st, oe.y, amin, idx, TB, B0, B1, B2, lastB, doneB, ncomp);
+        if (needA) composite<EXT>(st, oe.x, amin, idx, TA, A0, A1, A2, DA, lastA, doneA, ncomp);
+        if (needB) composite<EXT>(st, oe.y, amin, idx, TB, B0, B1, B2, DB, lastB, doneB, ncomp);
       }
       if (__all_sync(0xffffffffu, doneA && doneB)) break;
     }
   }
   const int64_t pixA = ((int64_t)c * g.H + j) * g.W + i;
+  if (EXT && bg) {
+    const float b0 = bg[3 * c], b1 = bg[3 * c + 1], b2 = bg[3 * c + 2];
+    A0 = fma_(TA, b0, A0);
+    A1 = fma_(TA, b1, A1);
+    A2 = fma_(TA, b2, A2);
+    B0 = fma_(TB, b0, B0);
+    B1 = fma_(TB, b1, B1);
+    B2 = fma_(TB, b2, B2);
+  }
   if (inA) {
     img[3 * pixA] = A0;
     img[3 * pixA + 1] = A1;
     img[3 * pixA + 2] = A2;
     T_final[pixA] = TA;
     last_id[pixA] = (int32_t)lastA;
+    if (EXT && depth) depth[pixA] = DA;
   }
   if (inB) {
     const int64_t pixB = pixA + g.W;
@@ -401,6 +427,7 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd_masked(Geo g, const fl
     img[3 * pixB + 2] = B2;
     T_final[pixB] = TB;
     last_id[pixB] = (int32_t)lastB;
+    if (EXT && depth) depth[pixB] = DB;
   }
 }
 
@@ -440,9 +467,17 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Per-pixel backward state.
 struct PixB {
-  float T, Sg, g0, g1, g2, vTT;
+  float T, Sg, g0, g1, g2, vTT, gD;  // gD: dL/d(expected depth), 0 unless requested
   int64_t last;
 };
+
+// Entries [qb, qb + 32) that a pixel with last composited entry `last`
+// replays: bit b set when qb + b <= last.
+__device__ __forceinline__ uint32_t live_bits(int64_t last, int64_t qb) {
+  if (last < qb) return 0u;
+  const int64_t d = last - qb;
+  return d >= 31 ? 0xFFFFFFFFu : (2u << (int)d) - 1u;
+}
 
 // Reverse step of the thread's pixel pair for a replayed entry.  cA / cB say
 // which pixels replay the entry with sigma within the skip threshold.  A
@@ -455,6 +490,11 @@ struct PixB {
 //   dL/dx = ca*dx*S0 + cb*S1,  dL/dy = cb*dx*S0 + cc*S1,
 //   dL/dca = dx^2*S0/2,  dL/dcb = dx*S1,  dL/dcc = S2/2,
 // where S0 = sum v, S1 = sum v*dy, S2 = sum v*dy^2 (dx is shared).
+//
+// EXT: the expected depth is a fourth channel composited with the same
+// weights, so depth * gD joins the colour term of dL/dalpha and
+// gr[9] = sum w * gD is the row's depth gradient.
+template <bool EXT>
 __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, float2 ev, bool cA, bool cB,
                                           float amin, PixB& pa, PixB& pb, float* gr) {
   const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
@@ -469,6 +509,7 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
   float2 rgbg = __fmul2_rn(f2s(st.b.z), G0);
   rgbg = __ffma2_rn(f2s(st.b.w), G1, rgbg);
   rgbg = __ffma2_rn(f2s(st.c.x), G2, rgbg);
+  if (EXT) rgbg = __ffma2_rn(f2s(st.e.w), f2(pa.gD, pb.gD), rgbg);
   const float2 Sg = f2(pa.Sg, pb.Sg);
   const float2 behind = __fadd2_rn(Sg, f2(pa.vTT, pb.vTT));
   const float2 va = __ffma2_rn(Ti, rgbg, __fmul2_rn(f2(-ra.x, -ra.y), behind));  // dL/dalpha
@@ -481,6 +522,10 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
   gr[6] = w0.x + w0.y;
   gr[7] = w1.x + w1.y;
   gr[8] = w2.x + w2.y;
+  if (EXT) {
+    const float2 wd = __fmul2_rn(w, f2(pa.gD, pb.gD));
+    gr[9] = wd.x + wd.y;
+  }
   // sigma and opacity gradients only where alpha was not clamped at 0.99
   const bool gA = cA && oe.x < SS_ALPHA_MAX, gB = cB && oe.y < SS_ALPHA_MAX;
   const float2 vs0 = __fmul2_rn(f2(-a.x, -a.y), va);
@@ -500,6 +545,9 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
   return true;
 }
 
+// EXT: v_depth (nullable, per pixel) and bg (nullable, [C][3]; the blend
+// img = C + T_final * bg adds g . bg to dL/dT_final).
+template <bool EXT>
 __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __restrict__ screen,
                                                           const uint32_t* __restrict__ vals,
                                                           const int64_t* __restrict__ tile_off,
@@ -507,6 +555,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
                                                           const int32_t* __restrict__ last_id,
                                                           const float* __restrict__ v_img,
                                                           const float* __restrict__ v_T,
+                                                          const float* __restrict__ v_depth,
+                                                          const float* __restrict__ bg,
                                                           float* __restrict__ v_screen) {
   __shared__ Stage s_e[kBatch];
   __shared__ __align__(16) float red[kBatch][kRedF];  // per-entry sums over the CTA's warps
@@ -519,15 +569,15 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
   const bool inA = i < g.W && j < g.H, inB = i < g.W && j + 1 < g.H;
   const float px = add((float)i, 0.5f);
   const float2 npy = f2(-add((float)j, 0.5f), -add((float)(j + 1), 0.5f));
-  const float x_lo = (float)tx0 + 0.5f, x_hi = x_lo + 15.0f;
-  const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f, y_hi = y_lo + 3.0f;
+  const float x_lo = (float)tx0 + 0.5f;
+  const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f;
   const int64_t beg = tile_off[tile];
   const float amin = alpha_min();
   for (int t = threadIdx.x; t < kBatch * kRedF; t += kRThreads) (&red[0][0])[t] = 0.0f;
   for (int t = threadIdx.x; t < kBatch; t += kRThreads) s_any[t] = 0u;
   if (threadIdx.x == 0) s_maxlast = -1;
   __syncthreads();
-  PixB pa{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1}, pb{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1};
+  PixB pa{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1}, pb{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1};
   const int64_t pixA = ((int64_t)c * g.H + j) * g.W + i, pixB = pixA + g.W;
   if (inA) {
     pa.last = last_id[pixA];
@@ -535,7 +585,10 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
     pa.g0 = v_img[3 * pixA];
     pa.g1 = v_img[3 * pixA + 1];
     pa.g2 = v_img[3 * pixA + 2];
-    pa.vTT = mul(v_T ? v_T[pixA] : 0.0f, pa.T);
+    float vt = v_T ? v_T[pixA] : 0.0f;
+    if (EXT && bg) vt += pa.g0 * bg[3 * c] + pa.g1 * bg[3 * c + 1] + pa.g2 * bg[3 * c + 2];
+    if (EXT && v_depth) pa.gD = v_depth[pixA];
+    pa.vTT = mul(vt, pa.T);
     if (pa.last >= 0) atomicMax(&s_maxlast, (int)pa.last);
   }
   if (inB) {
@@ -544,7 +597,10 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
     pb.g0 = v_img[3 * pixB];
     pb.g1 = v_img[3 * pixB + 1];
     pb.g2 = v_img[3 * pixB + 2];
-    pb.vTT = mul(v_T ? v_T[pixB] : 0.0f, pb.T);
+    float vt = v_T ? v_T[pixB] : 0.0f;
+    if (EXT && bg) vt += pb.g0 * bg[3 * c] + pb.g1 * bg[3 * c + 1] + pb.g2 * bg[3 * c + 2];
+    if (EXT && v_depth) pb.gD = v_depth[pixB];
+    pb.vTT = mul(vt, pb.T);
     if (pb.last >= 0) atomicMax(&s_maxlast, (int)pb.last);
   }
   __syncthreads();
@@ -560,17 +616,24 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
     if (b0 <= wlast) {
       for (int q = (cnt - 1) / 32; q >= 0; --q) {
         const int e = q * 32 + lane;
-        uint32_t bits = __ballot_sync(0xffffffffu, e < cnt && b0 + e <= wlast &&
-                                                      !warp_culled(s_e[e], x_lo, x_hi, y_lo, y_hi));
+        const int64_t qb = b0 + q * 32;
+        if (qb > wlast) continue;  // warp-uniform: no pixel of the warp replays the block
+        // candidate masks as in the forward: bit b of mA (mB) set when entry
+        // qb + b can reach this lane's upper (lower) pixel and the pixel
+        // replays it; the warp steps through the union of its lanes' masks
+        uint32_t covA = 0u, covB = 0u;
+        if (e < cnt) entry_coverage(s_e[e], x_lo, y_lo, covA, covB);
+        const uint32_t mA = warp_transpose32(covA, lane) & live_bits(pa.last, qb);
+        const uint32_t mB = warp_transpose32(covB, lane) & live_bits(pb.last, qb);
+        uint32_t bits = __reduce_or_sync(0xffffffffu, mA | mB);
         while (bits) {
           const int hb = 31 - __clz(bits);
           bits &= ~(1u << hb);
           const int k = q * 32 + hb;
-          const int64_t idx = b0 + k;
           const Stage& st = s_e[k];
-          float gr[9];
+          float gr[10];
           bool contrib = false;
-          const bool liveA = idx <= pa.last, liveB = idx <= pb.last;
+          const bool liveA = (mA >> hb) & 1u, liveB = (mB >> hb) & 1u;
           if (liveA || liveB) {
             const float dx = sub(st.a.x, px);
             const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
@@ -579,20 +642,22 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
             const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
             if (needA || needB) {
               const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
-              contrib = pair_grad(st, dx, dy, ev, needA, needB, amin, pa, pb, gr);
+              contrib = pair_grad<EXT>(st, dx, dy, ev, needA, needB, amin, pa, pb, gr);
             }
           }
           if (!contrib) {
 #pragma unroll
-            for (int t = 0; t < 9; ++t) gr[t] = 0.0f;
+            for (int t = 0; t < 10; ++t) gr[t] = 0.0f;
           }
           if (__any_sync(0xffffffffu, contrib)) {
             const float s8 = warp_reduce8(gr, lane);
             const float sb = warp_sum(gr[8]);
+            const float sd = EXT ? warp_sum(gr[9]) : 0.0f;
             if ((lane & 3) == 0)
               atomicAdd(&red[k][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)], s8);
             if (lane == 0) {
               atomicAdd(&red[k][8], sb);
+              if (EXT) atomicAdd(&red[k][9], sd);
               s_any[k] = 1u;
             }
           }
@@ -620,13 +685,19 @@ using namespace ss;
 
 extern "C" ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, const uint32_t* vals,
                                       const int64_t* tile_off, float* img, float* T_final, int32_t* last_id,
-                                      void* stream) {
+                                      float* depth, const float* bg, void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (!tile_off || !img || !T_final || !last_id) return invalid("null pointer");
   if (((uintptr_t)screen & 15) != 0) return invalid("screen must be 16-byte aligned");
   const Geo g = geometry(*dims);
   cudaStream_t st = as_stream(stream);
-  k_raster_fwd_masked<<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, img, T_final, last_id);
+  if (depth || bg) {
+    k_raster_fwd_masked<true><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, img, T_final,
+                                                                         last_id, depth, bg);
+  } else {
+    k_raster_fwd_masked<false><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, img, T_final,
+                                                                          last_id, nullptr, nullptr);
+  }
   return cuda_status(cudaGetLastError(), "rasterize fwd");
 }
 
@@ -647,8 +718,8 @@ extern "C" ss_status ss_rasterize_fwd_counts(const ss_dims* dims, const float* s
 
 extern "C" ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, const uint32_t* vals,
                                       const int64_t* tile_off, const float* T_final, const int32_t* last_id,
-                                      const float* v_img, const float* v_T, float* v_screen, int64_t nnz,
-                                      void* stream) {
+                                      const float* v_img, const float* v_T, const float* v_depth,
+                                      const float* bg, float* v_screen, int64_t nnz, void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (nnz < 0) return invalid("nnz < 0");
   if (!tile_off || !T_final || !last_id || !v_img || (nnz > 0 && !v_screen)) return invalid("null pointer");
@@ -659,7 +730,12 @@ extern "C" ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, 
     ss_status s = cuda_status(cudaMemsetAsync(v_screen, 0, (size_t)nnz * kRowF * sizeof(float), st), "memset");
     if (s) return s;
   }
-  k_raster_bwd<<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, T_final, last_id, v_img, v_T,
-                                                         v_screen);
+  if (v_depth || bg) {
+    k_raster_bwd<true><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, T_final, last_id, v_img,
+                                                                  v_T, v_depth, bg, v_screen);
+  } else {
+    k_raster_bwd<false><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, T_final, last_id,
+                                                                   v_img, v_T, nullptr, nullptr, v_screen);
+  }
   return cuda_status(cudaGetLastError(), "rasterize bwd");
 }

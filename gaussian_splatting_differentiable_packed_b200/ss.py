@@ -69,9 +69,9 @@ def lib() -> ct.CDLL:
         L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
         L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, P, sz, P, ct.POINTER(i32), P]
         L.ss_sort_isects_noalloc.argtypes = [D, P, P, P, P, i64, P, ct.POINTER(i32), P]
-        L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P]
+        L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P]
         L.ss_rasterize_fwd_counts.argtypes = [D, P, P, P, P, P, P, P, P]
-        L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, i64, P]
+        L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, i64, P]
         L.ss_project_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
         for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc",
                   "ss_rasterize_fwd",
@@ -158,9 +158,9 @@ def ss_sort_isects_noalloc(d, keys_a, vals_a, keys_b, vals_b, n, tile_off, strea
     return bool(in_b.value)
 
 
-def ss_rasterize_fwd(d, screen, vals, tile_off, img, T_final, last_id, stream=None):
+def ss_rasterize_fwd(d, screen, vals, tile_off, img, T_final, last_id, depth=None, bg=None, stream=None):
     _check(lib().ss_rasterize_fwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(img), _p(T_final),
-                                  _p(last_id), _stream(stream)), "ss_rasterize_fwd")
+                                  _p(last_id), _p(depth), _p(bg), _stream(stream)), "ss_rasterize_fwd")
 
 
 def ss_rasterize_fwd_counts(d, screen, vals, tile_off, img, T_final, last_id, counts, stream=None):
@@ -177,9 +177,11 @@ def raster_work(d, step) -> dict:
     return dict(evals=c[0], exps=c[1], comps=c[2], bwd_evals=c[3], bwd_exps=c[4])
 
 
-def ss_rasterize_bwd(d, screen, vals, tile_off, T_final, last_id, v_img, v_T, v_screen, nnz, stream=None):
+def ss_rasterize_bwd(d, screen, vals, tile_off, T_final, last_id, v_img, v_T, v_screen, nnz, stream=None,
+                     v_depth=None, bg=None):
     _check(lib().ss_rasterize_bwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(T_final), _p(last_id),
-                                  _p(v_img), _p(v_T), _p(v_screen), int(nnz), _stream(stream)), "ss_rasterize_bwd")
+                                  _p(v_img), _p(v_T), _p(v_depth), _p(bg), _p(v_screen), int(nnz), _stream(stream)),
+           "ss_rasterize_bwd")
 
 
 def ss_project_bwd(d, cams, means, quats, scales, opacities, sh, mask, block_off, v_screen, v_means, v_quats,
@@ -198,8 +200,10 @@ class PackedStep:
 
     forward() runs ss_project_packed, ss_intersect_tiles, ss_sort_isects and
     ss_rasterize_fwd; backward(v_img, v_T=None) runs ss_rasterize_bwd and
-    ss_project_bwd.  Intermediate buffers are kept as attributes so callers
-    (tests) can inspect every stage.
+    ss_project_bwd.  forward(..., bg=, depth=True) also blends a background
+    colour per camera and renders the expected depth (self.depth);
+    backward(..., v_depth=) then takes its gradient.  Intermediate buffers are
+    kept as attributes so callers (tests) can inspect every stage.
     """
 
     def __init__(self, d: ss_dims, device="cuda", cap_rows: int = 0, cap_isects: int = 0, headroom: float = 1.25):
@@ -257,8 +261,9 @@ class PackedStep:
         self.temp_sort = torch.empty(workspace_bytes(self.d, WS_SORT, cap), dtype=torch.uint8, device=dev)
         self.cap_isects = cap
 
-    def forward(self, cams, means, quats, scales, opacities, sh, stream=None):
+    def forward(self, cams, means, quats, scales, opacities, sh, stream=None, bg=None, depth=False):
         self.inputs = (cams, means, quats, scales, opacities, sh)
+        self.bg = bg
         d = self.d
         try:
             nnz = ss_project_packed(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_count,
@@ -288,14 +293,17 @@ class PackedStep:
                                           self.tile_off, stream)
         self.keys = self.keys_b if self.result_in_b else self.keys_a
         self.vals = self.vals_b if self.result_in_b else self.vals_a
-        ss_rasterize_fwd(d, self.screen, self.vals, self.tile_off, self.img, self.T, self.last, stream)
+        if depth and getattr(self, "depth", None) is None:
+            self.depth = torch.empty((d.C, d.H, d.W), dtype=torch.float32, device=self.dev)
+        ss_rasterize_fwd(d, self.screen, self.vals, self.tile_off, self.img, self.T, self.last,
+                         self.depth if depth else None, bg, stream)
         return self.img
 
-    def backward(self, v_img, v_T=None, stream=None):
+    def backward(self, v_img, v_T=None, stream=None, v_depth=None):
         cams, means, quats, scales, opacities, sh = self.inputs
         d = self.d
         ss_rasterize_bwd(d, self.screen, self.vals, self.tile_off, self.T, self.last, v_img, v_T, self.v_screen,
-                         self.nnz, stream)
+                         self.nnz, stream, v_depth=v_depth, bg=self.bg)
         ss_project_bwd(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_off, self.v_screen,
                        self.v_means, self.v_quats, self.v_scales, self.v_opacities, self.v_sh, stream)
         return dict(v_means=self.v_means, v_quats=self.v_quats, v_scales=self.v_scales,
@@ -320,16 +328,21 @@ def sort_passes(d: ss_dims) -> int:
     return 4 + (tb + 7) // 8
 
 
+def sort_launches(d: ss_dims, n_isects: int) -> int:
+    """Kernels of one ss_sort_isects call: histogram, digit bases, one onesweep
+    kernel per pass, tile ranges."""
+    return 0 if n_isects == 0 else sort_passes(d) + 3
+
+
 def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
     """Kernels libss launches in one forward+backward step (memsets excluded):
-    projection 5 (pass 1, three scan kernels, pass 2), intersection 4 (three
-    scan kernels, write), sort 5 per pass + tile ranges, rasterizer 1 + 1,
-    projection backward 1."""
+    projection 5 (pass 1, three scan kernels, pass 2), intersection 5 (three
+    scan kernels, chunk first rows, write), the sort (sort_launches),
+    rasterizer 1 + 1, projection backward 1."""
     if d.N == 0:
         return 0
     n = 5
     if nnz > 0:
-        n += 4 if n_isects > 0 else 3
-    if n_isects > 0:
-        n += 5 * sort_passes(d) + 1
+        n += 5 if n_isects > 0 else 3
+    n += sort_launches(d, n_isects)
     return n + 3

@@ -93,7 +93,8 @@ typedef struct ss_dims {
 int64_t ss_size(const ss_dims* dims, int what);
 
 /* Scratch bytes needed by a call: which = SS_WS_PROJECT (count ignored),
- * SS_WS_INTERSECT (count = nnz), SS_WS_SORT (count = number of keys). */
+ * SS_WS_INTERSECT (count = nnz; includes 8 MiB for the write pass's per-chunk
+ * row index), SS_WS_SORT (count = number of keys). */
 #define SS_WS_PROJECT 0
 #define SS_WS_INTERSECT 1
 #define SS_WS_SORT 2
@@ -117,6 +118,7 @@ const char* ss_last_error(void);
  * re-projects the survivors only: row = block_off[block] + set bits before the
  * pair, writing the screen row (SH colour evaluated toward the camera centre)
  * and the 16-bit AABB.  Rows are ordered camera-major, Gaussian-minor.
+ * quats and sh must be 16-byte aligned (SS_ERR_INVALID_ARG otherwise).
  */
 ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float* means, const float* quats,
                             const float* scales, const float* opacities, const float* sh, uint32_t* mask,
@@ -143,11 +145,13 @@ ss_status ss_intersect_tiles(const ss_dims* dims, const float* screen, const uin
 
 /*
  * Stable LSD radix sort of n (key, value) pairs by key, 8-bit digits over the
- * 31 depth bits and the tile-id bits only ("Spirula Studio VRAM deep-dive",
+ * 32 depth bits and the tile-id bits only ("Spirula Studio VRAM deep-dive",
  * buffer table: double-buffered isect.ids_a/b).  Ping-pongs between (keys_a,
  * vals_a) and (keys_b, vals_b); *result_in_b_out (host) says which pair holds
- * the result (known from dims alone; no sync).  Then writes tile_off[n_tiles+1].
+ * the result (an odd pass count: b; known from dims alone).  Then writes
+ * tile_off[n_tiles+1].
  * n >= 2^31 returns SS_ERR_OVERFLOW.  Equal keys keep their input order.
+ * Synchronises the stream at the end (reads the look-back error flag).
  */
 ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
                          uint32_t* vals_b, int64_t n, void* temp, size_t temp_bytes, int64_t* tile_off,
@@ -179,11 +183,19 @@ ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_a, uint32_t
  * its transmittance for the backward pass).  One CTA per 16x16 tile, front to
  * back over the tile's sorted entries: alpha = min(0.99, o*exp(-sigma)),
  * entries with alpha < 1/255 skipped, stop before the entry that would take
- * T below 1e-4.  Writes img, T_final and last_id (the sorted index of the last
- * composited entry, -1 if none).  vals are the sorted values.
+ * T below 1e-4.  Writes img[C][H][W][3], T_final[C][H][W] and
+ * last_id[C][H][W] (the sorted index of the last composited entry, -1 if
+ * none).  vals are the sorted values.
+ *
+ * Optional outputs (the pages' depth/T render outputs and background blend;
+ * pass NULL to leave them out, which runs the plain kernel):
+ *   depth  [C][H][W] device float, the expected depth sum_i alpha_i T_i d_i
+ *          with d_i the row's camera depth (not normalised by 1 - T_final);
+ *   bg     [C][3] device float, a background colour per camera; img becomes
+ *          C + T_final * bg.
  */
 ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, const uint32_t* vals, const int64_t* tile_off,
-                           float* img, float* T_final, int32_t* last_id, void* stream);
+                           float* img, float* T_final, int32_t* last_id, float* depth, const float* bg, void* stream);
 
 /*
  * Measurement helper, not part of the step: ss_rasterize_fwd plus exact work
@@ -202,11 +214,14 @@ ss_status ss_rasterize_fwd_counts(const ss_dims* dims, const float* screen, cons
  * reverse replay from last_id using the saved state (no re-intersection),
  * splitting v_img (and v_T, may be NULL) by each entry's alpha contribution.
  * Gradients are reduced over the tile's pixels and added with atomics into
- * v_screen[nnz][12], which the call zeroes first.
+ * v_screen[nnz][12], which the call zeroes first.  v_depth ([C][H][W], may be
+ * NULL) is the gradient of the expected depth of ss_rasterize_fwd and fills
+ * the rows' depth gradient (column 9); bg ([C][3], may be NULL) must be the
+ * background the forward blended.
  */
 ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, const uint32_t* vals, const int64_t* tile_off,
                            const float* T_final, const int32_t* last_id, const float* v_img, const float* v_T,
-                           float* v_screen, int64_t nnz, void* stream);
+                           const float* v_depth, const float* bg, float* v_screen, int64_t nnz, void* stream);
 
 /*
  * Projection backward ("Spirula Studio backward pass", section 5): for each
@@ -214,6 +229,8 @@ ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, const uint3
  * taken back through the conic, the EWA Jacobian, the camera transform, the
  * covariance and the SH colour.  Deterministic (one thread per Gaussian, no
  * atomics).  Writes every element of the five outputs (zero where invisible).
+ * quats, v_quats, v_screen, sh and v_sh must be 16-byte aligned
+ * (SS_ERR_INVALID_ARG otherwise).
  */
 ss_status ss_project_bwd(const ss_dims* dims, const float* cams, const float* means, const float* quats,
                          const float* scales, const float* opacities, const float* sh, const uint32_t* mask,

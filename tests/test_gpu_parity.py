@@ -228,3 +228,44 @@ def test_rasterizer_work_counts_match_oracle():
     replay = np.where(last >= 0, last - o["tile_off"][t] + 1, 0)
     assert w["bwd_evals"] == int(replay.sum())
     np.testing.assert_array_equal(step.last.cpu().numpy(), o["last"])
+
+
+# ---------------------------------------------------------------- depth output and background
+def depth_bg_parity(scene, seed):
+    """Forward with a background per camera and the expected depth, backward
+    with v_T and v_depth: images, depth, T and last_id against the oracle,
+    every screen-row gradient including the depth column, and the Gaussian
+    gradients (the depth gradient reaches the means through the camera z)."""
+    rng = np.random.default_rng(700 + seed)
+    shp = (scene.C, scene.H, scene.W)
+    bg = rng.uniform(0.0, 1.0, (scene.C, 3)).astype(np.float32)
+    v_img = (rng.uniform(-1, 1, shp + (3,)) / (3.0 * scene.W * scene.H)).astype(np.float32)
+    v_T = (rng.uniform(-1, 1, shp) / (scene.W * scene.H)).astype(np.float32)
+    v_D = (rng.uniform(-1, 1, shp) / (scene.W * scene.H)).astype(np.float32)
+    o = orc.step(scene, precision=0, nthreads=ORACLE_THREADS, v_img=v_img, v_T=v_T, v_depth=v_D, bg=bg)
+    step = ss.PackedStep(ss.scene_dims(scene), "cuda")
+    step.forward(*ss.scene_tensors(scene), bg=torch.from_numpy(bg).cuda(), depth=True)
+    step.backward(torch.from_numpy(v_img).cuda(), torch.from_numpy(v_T).cuda(), v_depth=torch.from_numpy(v_D).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(step.last.cpu().numpy(), o["last"])
+    assert np.abs(step.T.cpu().numpy() - o["T"]).max() <= 1e-5
+    assert np.abs(step.img.cpu().numpy() - o["img"]).max() <= 1e-5
+    D = step.depth.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(D - o["depth"]) <= 1e-5 * np.maximum(1.0, np.abs(o["depth"])))
+    n = o["proj"]["nnz"]
+    vs = step.v_screen[:n].cpu().numpy()
+    grad_close("v_screen", vs[:, :10], o["v_screen"][:, :10])
+    assert np.abs(o["v_screen"][:, 9]).max() > 0  # the depth column is exercised
+    for k, ref in o["grads"].items():
+        grad_close(k, getattr(step, k).cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_depth_and_background_random_tiny(seed):
+    sc = scenes.random_tiny(50 + seed, N=400 + 37 * seed, W=41 + 8 * seed, H=33 + 3 * seed, C=1 + seed % 2,
+                            sh_degree=(seed + 1) % 4)
+    depth_bg_parity(sc, seed)
+
+
+def test_depth_and_background_config2():
+    depth_bg_parity(scenes.make_scene(2), 9)

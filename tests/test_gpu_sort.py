@@ -1,0 +1,81 @@
+"""Direct parity of ss_sort_isects with the oracle's stable sort on seeded
+synthetic (tile << 32 | depth) keys with skewed tile populations (uniform
+tiles, a few tiles holding thousands of keys as the heavy tiles of the large
+workloads do), and a tile count needing three tile-id bytes (odd pass count:
+the result ends in the second buffer pair).
+Depths repeat (ties must keep input order) and values are not ordered by
+position, so only a stable sort by key matches.  Keys, values and tile
+offsets must be bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gaussian_splatting_differentiable_packed_b200 import ss
+from oracle import oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+
+def make_keys(rng, n_tiles, n, hot=()):
+    """n keys over uniform tiles plus `hot` = [(tile, count), ...] extra keys;
+    depths drawn from a small pool half of the time so that many tie."""
+    tiles = [rng.integers(0, n_tiles, n)]
+    for t, c in hot:
+        tiles.append(np.full(c, t))
+    tiles = np.concatenate(tiles).astype(np.uint64)
+    rng.shuffle(tiles)
+    m = len(tiles)
+    pool = rng.uniform(0.2, 50.0, 40).astype(np.float32)
+    depth = np.where(rng.random(m) < 0.5, rng.choice(pool, m), rng.uniform(0.2, 50.0, m).astype(np.float32))
+    bits = depth.astype(np.float32).view(np.uint32).astype(np.uint64)
+    keys = (tiles << np.uint64(32)) | bits
+    vals = rng.permutation(m).astype(np.uint32) * np.uint32(7) + np.uint32(3)
+    return keys, vals
+
+
+def run_sort(d, keys, vals):
+    n = len(keys)
+    ka = torch.from_numpy(keys.view(np.int64).copy()).cuda()
+    va = torch.from_numpy(vals.view(np.int32).copy()).cuda()
+    kb = torch.empty_like(ka)
+    vb = torch.empty_like(va)
+    n_tiles = ss.size(d, ss.SIZE_N_TILES)
+    tile_off = torch.empty(n_tiles + 1, dtype=torch.int64, device="cuda")
+    temp = torch.empty(ss.workspace_bytes(d, ss.WS_SORT, n), dtype=torch.uint8, device="cuda")
+    in_b = ss.ss_sort_isects(d, ka, va, kb, vb, n, temp, tile_off)
+    torch.cuda.synchronize()
+    k, v = (kb, vb) if in_b else (ka, va)
+    return in_b, k.cpu().numpy().view(np.uint64), v.cpu().numpy().view(np.uint32), tile_off.cpu().numpy()
+
+
+@pytest.mark.parametrize("case", ["small", "large", "lsd", "three_tile_bytes"])
+def test_sort_paths(case):
+    rng = np.random.default_rng({"small": 11, "large": 12, "lsd": 13, "three_tile_bytes": 14}[case])
+    if case == "three_tile_bytes":
+        d = ss.make_dims(5, 2048, 2048, 0, 1, 0.01, 1e10)  # 81920 tiles: 17 tile-id bits
+    else:
+        d = ss.make_dims(1, 1024, 1024, 0, 1, 0.01, 1e10)  # 4096 tiles
+    n_tiles = ss.size(d, ss.SIZE_N_TILES)
+    hot = {"small": [], "large": [(17, 9000), (4000, 2100)], "lsd": [(5, 20000), (6, 3000)],
+           "three_tile_bytes": [(81919, 2500)]}[case]
+    keys, vals = make_keys(rng, n_tiles, 300_000, hot)
+    in_b, gk, gv, toff = run_sort(d, keys, vals)
+    assert in_b == bool(ss.sort_passes(d) & 1)
+    ok, ov = orc.sort(keys, vals)
+    np.testing.assert_array_equal(gk, ok)
+    np.testing.assert_array_equal(gv, ov)
+    np.testing.assert_array_equal(toff, orc.tile_ranges(ok, n_tiles))
+
+
+def test_sort_single_bucket_and_tiny():
+    """Every key in one tile (one 1500-key bucket), and a 3-key input."""
+    d = ss.make_dims(1, 64, 64, 0, 1, 0.01, 1e10)
+    n_tiles = ss.size(d, ss.SIZE_N_TILES)
+    rng = np.random.default_rng(15)
+    for keys, vals in [make_keys(rng, 1, 1500), make_keys(rng, n_tiles, 3)]:
+        in_b, gk, gv, toff = run_sort(d, keys, vals)
+        ok, ov = orc.sort(keys, vals)
+        np.testing.assert_array_equal(gk, ok)
+        np.testing.assert_array_equal(gv, ov)
+        np.testing.assert_array_equal(toff, orc.tile_ranges(ok, n_tiles))

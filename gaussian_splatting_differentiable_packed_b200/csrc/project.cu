@@ -122,16 +122,42 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   const int64_t n0 = blk * kBlock;
   const int64_t n = n0 + threadIdx.x;
   const int cnt = (int)min64(kBlock, g.N - n0);
-  {
-    const float* src = sh + n0 * K3;
-    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-      const int gi = f / K3, qq = f - gi * K3;
-      sh_s[gi * KP + qq] = src[f];
-    }
-  }
   if (n < g.N) {
     s_g[threadIdx.x] = load_gauss(means, quats, scales, n);
     s_o[threadIdx.x] = opacities[n];
+  }
+  // the CTA's contiguous SH block: a full block with all 16-byte loads in
+  // flight at once (it starts 16-byte aligned: 128*K3 floats per block), the
+  // ragged last block word by word
+  {
+    const float* src = sh + n0 * K3;
+    if (cnt == kBlock) {
+      constexpr int kV = kBlock * K3 / 4;
+      constexpr int kPer = (kV + kBlock - 1) / kBlock;
+      float4 buf[kPer];
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int v = threadIdx.x + r * kBlock;
+        if (v < kV) buf[r] = reinterpret_cast<const float4*>(src)[v];
+      }
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int v = threadIdx.x + r * kBlock;
+        if (v < kV) {
+          const float e[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int f = 4 * v + u, gi = f / K3, qq = f - gi * K3;
+            sh_s[gi * KP + qq] = e[u];
+          }
+        }
+      }
+    } else {
+      for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+        const int gi = f / K3, qq = f - gi * K3;
+        sh_s[gi * KP + qq] = src[f];
+      }
+    }
   }
   if (threadIdx.x == 0) q_len = 0;
   auto process = [&](const RowItem& it) {
@@ -242,7 +268,7 @@ extern "C" ss_status ss_project_packed(const ss_dims* dims, const float* cams, c
     return SS_OK;
   }
   if (!cams || !means || !quats || !scales || !mask || !block_count) return invalid("null input");
-  if (((uintptr_t)quats & 15) != 0) return invalid("quats must be 16-byte aligned");
+  if (((uintptr_t)quats & 15) != 0 || ((uintptr_t)sh & 15) != 0) return invalid("quats and sh must be 16-byte aligned");
   if (!temp || temp_bytes < ss_workspace_bytes(dims, SS_WS_PROJECT, 0)) return invalid("temp too small");
   const unsigned grid = (unsigned)g.blocks_per_cam;
   k_project_mask<<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, mask, block_count);

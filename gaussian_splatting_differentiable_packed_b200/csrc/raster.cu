@@ -24,6 +24,9 @@ namespace ss {
 
 constexpr int kRThreads = 128;
 constexpr int kBatch = 256;
+// The backward stages half as many entries per batch: 17 KB of shared memory
+// and at most 64 registers per thread let 8 CTAs share an SM.
+constexpr int kBatchB = 128;
 constexpr int kRedF = 12;
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
@@ -548,7 +551,7 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
 // EXT: v_depth (nullable, per pixel) and bg (nullable, [C][3]; the blend
 // img = C + T_final * bg adds g . bg to dL/dT_final).
 template <bool EXT>
-__global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __restrict__ screen,
+__global__ __launch_bounds__(kRThreads, 8) void k_raster_bwd(Geo g, const float* __restrict__ screen,
                                                           const uint32_t* __restrict__ vals,
                                                           const int64_t* __restrict__ tile_off,
                                                           const float* __restrict__ T_final,
@@ -558,9 +561,9 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
                                                           const float* __restrict__ v_depth,
                                                           const float* __restrict__ bg,
                                                           float* __restrict__ v_screen) {
-  __shared__ Stage s_e[kBatch];
-  __shared__ __align__(16) float red[kBatch][kRedF];  // per-entry sums over the CTA's warps
-  __shared__ uint32_t s_any[kBatch];
+  __shared__ Stage s_e[kBatchB];
+  __shared__ __align__(16) float red[kBatchB][kRedF];  // per-entry sums over the CTA's warps
+  __shared__ uint32_t s_any[kBatchB];
   __shared__ int s_maxlast;
   const int lane = threadIdx.x & 31;
   const int64_t tile = blockIdx.x;
@@ -573,8 +576,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
   const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f;
   const int64_t beg = tile_off[tile];
   const float amin = alpha_min();
-  for (int t = threadIdx.x; t < kBatch * kRedF; t += kRThreads) (&red[0][0])[t] = 0.0f;
-  for (int t = threadIdx.x; t < kBatch; t += kRThreads) s_any[t] = 0u;
+  for (int t = threadIdx.x; t < kBatchB * kRedF; t += kRThreads) (&red[0][0])[t] = 0.0f;
+  for (int t = threadIdx.x; t < kBatchB; t += kRThreads) s_any[t] = 0u;
   if (threadIdx.x == 0) s_maxlast = -1;
   __syncthreads();
   PixB pa{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1}, pb{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1};
@@ -608,8 +611,8 @@ __global__ __launch_bounds__(kRThreads) void k_raster_bwd(Geo g, const float* __
   int64_t wlast = max64(pa.last, pb.last);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wlast = max64(wlast, __shfl_xor_sync(0xffffffffu, wlast, o));
-  for (int64_t b1 = stop; b1 > beg; b1 -= kBatch) {
-    const int64_t b0 = max64(beg, b1 - kBatch);
+  for (int64_t b1 = stop; b1 > beg; b1 -= kBatchB) {
+    const int64_t b0 = max64(beg, b1 - kBatchB);
     const int cnt = (int)(b1 - b0);
     for (int t = threadIdx.x; t < cnt; t += kRThreads) stage_row(screen, vals[b0 + t], s_e[t]);
     __syncthreads();

@@ -18,9 +18,6 @@
 // flag (reported by the call as SS_ERR_DEVICE_CHECK) and goes on.  Tiles are
 // handed out by ticket, so every tile a CTA waits on belongs to a CTA that is
 // already running and never waits on a later tile.
-//
-// The per-pass reduce-then-scan kernels below (k_radix_hist, k_radix_scatter)
-// are the simpler variant kept for reference; they are not launched.
 #include <algorithm>
 #include <mutex>
 #include <utility>
@@ -35,120 +32,6 @@ constexpr int kSortTile = kSortThreads * kSortItems;  // 4096 keys per CTA
 constexpr int kRadix = 256;
 constexpr int kSortWarps = kSortThreads / 32;
 
-__global__ __launch_bounds__(kSortThreads) void k_radix_hist(const uint64_t* __restrict__ keys, int64_t n, int shift,
-                                                             uint32_t* __restrict__ counts, int64_t ntiles) {
-  __shared__ uint32_t h[kSortWarps][kRadix];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kSortWarps * kRadix; i += kSortThreads) (&h[0][0])[i] = 0;
-  __syncthreads();
-  const int64_t base = (int64_t)blockIdx.x * kSortTile + warp * (kSortTile / kSortWarps);
-#pragma unroll 4
-  for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = base + r * 32 + lane;
-    const bool valid = i < n;
-    const uint32_t d = valid ? (uint32_t)(keys[i] >> shift) & 0xFFu : 0x100u;
-    const uint32_t peers = __match_any_sync(0xffffffffu, d);
-    if (valid && lane == 31 - __clz(peers)) h[warp][d] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  uint32_t s = 0;
-#pragma unroll
-  for (int w = 0; w < kSortWarps; ++w) s += h[w][threadIdx.x];
-  counts[(int64_t)threadIdx.x * ntiles + blockIdx.x] = s;
-}
-
-struct ScatterSmem {
-  uint32_t wcnt[kSortWarps][kRadix];
-  uint32_t dstart[kRadix];
-  uint32_t gbase[kRadix];
-  uint32_t wtot[kSortWarps + 1];
-  uint64_t k[kSortTile];
-  uint32_t v[kSortTile];
-};
-
-__global__ __launch_bounds__(kSortThreads) void k_radix_scatter(const uint64_t* __restrict__ kin,
-                                                                const uint32_t* __restrict__ vin,
-                                                                uint64_t* __restrict__ kout,
-                                                                uint32_t* __restrict__ vout, int64_t n, int shift,
-                                                                const uint32_t* __restrict__ offs, int64_t ntiles) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  ScatterSmem& S = *reinterpret_cast<ScatterSmem*>(smem_raw);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kSortWarps * kRadix; i += kSortThreads) (&S.wcnt[0][0])[i] = 0;
-  __syncthreads();
-  const int64_t tile0 = (int64_t)blockIdx.x * kSortTile;
-  const int64_t base = tile0 + warp * (kSortTile / kSortWarps);
-  const uint32_t lt = (1u << lane) - 1u;
-  uint64_t kk[kSortItems];
-  uint32_t vv[kSortItems];
-  uint32_t pos[kSortItems];
-#pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = base + r * 32 + lane;
-    const bool valid = i < n;
-    kk[r] = valid ? kin[i] : 0ull;
-    vv[r] = valid ? vin[i] : 0u;
-    const uint32_t d = valid ? (uint32_t)(kk[r] >> shift) & 0xFFu : 0x100u;
-    const uint32_t peers = __match_any_sync(0xffffffffu, d);
-    const uint32_t before = valid ? S.wcnt[warp][d] : 0u;
-    __syncwarp();
-    if (valid && lane == 31 - __clz(peers)) S.wcnt[warp][d] = before + __popc(peers);
-    __syncwarp();
-    pos[r] = valid ? before + __popc(peers & lt) : 0xFFFFFFFFu;
-  }
-  __syncthreads();
-  // per digit: exclusive prefix over warps, digit totals, then exclusive scan over digits
-  {
-    const int d = threadIdx.x;
-    uint32_t run = 0;
-#pragma unroll
-    for (int w = 0; w < kSortWarps; ++w) {
-      const uint32_t t = S.wcnt[w][d];
-      S.wcnt[w][d] = run;
-      run += t;
-    }
-    // block exclusive scan of run over the 256 digits
-    uint32_t inc = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += x;
-    }
-    if (lane == 31) S.wtot[warp] = inc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      uint32_t a = 0;
-      for (int w = 0; w < kSortWarps; ++w) {
-        const uint32_t t = S.wtot[w];
-        S.wtot[w] = a;
-        a += t;
-      }
-    }
-    __syncthreads();
-    S.dstart[d] = S.wtot[warp] + inc - run;
-    S.gbase[d] = offs[(int64_t)d * ntiles + blockIdx.x];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
-    if (pos[r] == 0xFFFFFFFFu) continue;
-    const uint32_t d = (uint32_t)(kk[r] >> shift) & 0xFFu;
-    const uint32_t lp = S.dstart[d] + S.wcnt[warp][d] + pos[r];
-    S.k[lp] = kk[r];
-    S.v[lp] = vv[r];
-  }
-  __syncthreads();
-  const int cnt = (int)min64(kSortTile, n - tile0);
-  for (int i = threadIdx.x; i < cnt; i += kSortThreads) {
-    const uint64_t key = S.k[i];
-    const uint32_t d = (uint32_t)(key >> shift) & 0xFFu;
-    const int64_t gpos = (int64_t)S.gbase[d] + (i - (int64_t)S.dstart[d]);
-    kout[gpos] = key;
-    vout[gpos] = S.v[i];
-  }
-}
-
 constexpr int kMaxPasses = 8;
 constexpr uint64_t kFlagAgg = 1ull << 54;
 constexpr uint64_t kFlagPre = 2ull << 54;
@@ -160,12 +43,21 @@ struct SortPlan {
   int shift[kMaxPasses];
 };
 
-__global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __restrict__ keys, int64_t n, SortPlan plan,
+// Digit histograms of every pass in one read of the keys.  PASSES is a
+// template argument so every digit is a constant byte of the key's low or
+// high word.  Each warp counts into its own copy (dynamic shared memory,
+// [warp][pass][digit]), so warps do not contend for the bins of common digits
+// (the tile bytes of a region); the copies are summed at the end and added to
+// the global histogram.
+template <int PASSES>
+__global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __restrict__ keys, int64_t n,
                                                            uint32_t* __restrict__ hist) {
-  __shared__ uint32_t h[kMaxPasses][kRadix];
-  const int lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kMaxPasses * kRadix; i += kSortThreads) (&h[0][0])[i] = 0;
+  extern __shared__ uint32_t hw[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kPerWarp = PASSES * kRadix;
+  for (int i = threadIdx.x; i < kSortWarps * kPerWarp; i += kSortThreads) hw[i] = 0;
   __syncthreads();
+  uint32_t* mine = hw + warp * kPerWarp;
   // coalesced: a warp reads 32 consecutive keys; neighbouring keys share
   // digits (a row's keys share the depth and neighbouring tile ids), so each
   // run of equal digits is counted by its first lane with one shared atomic
@@ -174,24 +66,36 @@ __global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __res
     const int64_t i = base + threadIdx.x;
     const bool valid = i < n;
     const uint64_t k = valid ? keys[i] : 0ull;
+    const uint32_t lo = (uint32_t)k, hi = (uint32_t)(k >> 32);
     const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-    for (int p = 0; p < plan.passes; ++p) {
-      const uint32_t d = (uint32_t)(k >> plan.shift[p]) & 0xFFu;
+    const uint32_t end_all = 32u - (uint32_t)__clz(vmask);
+    const uint32_t above = ~((2u << lane) - 1u);  // lanes above this one
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+      const uint32_t d = ((p < 4 ? lo >> (8 * p) : hi >> (8 * (p - 4)))) & 0xFFu;
       const uint32_t prev = __shfl_up_sync(0xffffffffu, d, 1);
       const bool head = valid && (lane == 0 || d != prev);
-      const uint32_t heads = __ballot_sync(0xffffffffu, head);
-      if (head) {
-        const uint32_t after = heads & ~((2u << lane) - 1u);  // heads above this lane
-        const uint32_t end_lane = after ? (uint32_t)(__ffs(after) - 1) : (uint32_t)(32 - __clz(vmask));
-        atomicAdd(&h[p][d], end_lane - (uint32_t)lane);
-      }
+      const uint32_t after = __ballot_sync(0xffffffffu, head) & above;
+      if (head) atomicAdd(&mine[p * kRadix + d], (after ? (uint32_t)(__ffs(after) - 1) : end_all) - (uint32_t)lane);
     }
   }
   __syncthreads();
-  for (int p = 0; p < plan.passes; ++p) {
-    const uint32_t v = h[p][threadIdx.x];
-    if (v) atomicAdd(&hist[p * kRadix + threadIdx.x], v);
+  for (int i = threadIdx.x; i < kPerWarp; i += kSortThreads) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) v += hw[w * kPerWarp + i];
+    if (v) atomicAdd(&hist[i], v);
   }
+}
+
+template <int PASSES>
+ss_status launch_hist(unsigned grid, cudaStream_t st, const uint64_t* keys, int64_t n, uint32_t* hist) {
+  const size_t smem = sizeof(uint32_t) * kSortWarps * PASSES * kRadix;
+  ss_status s = cuda_status(
+      cudaFuncSetAttribute(k_hist_all<PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "smem attr");
+  if (s) return s;
+  k_hist_all<PASSES><<<grid, kSortThreads, smem, st>>>(keys, n, hist);
+  return cuda_status(cudaGetLastError(), "radix histogram");
 }
 
 // hist[p][d] -> exclusive scan over d, in place (one CTA of 256 threads).
@@ -423,7 +327,14 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   plan.passes = passes;
   for (int p = 0; p < passes; ++p) plan.shift[p] = p < 4 ? 8 * p : 32 + 8 * (p - 4);
   const unsigned hgrid = (unsigned)min64(tiles, 148 * 8);
-  k_hist_all<<<hgrid, kSortThreads, 0, st>>>(keys_a, n, plan, hist);
+  switch (passes) {
+    case 4: s = launch_hist<4>(hgrid, st, keys_a, n, hist); break;
+    case 5: s = launch_hist<5>(hgrid, st, keys_a, n, hist); break;
+    case 6: s = launch_hist<6>(hgrid, st, keys_a, n, hist); break;
+    case 7: s = launch_hist<7>(hgrid, st, keys_a, n, hist); break;
+    default: s = launch_hist<8>(hgrid, st, keys_a, n, hist); break;
+  }
+  if (s) return s;
   k_bases<<<1, kRadix, 0, st>>>(hist, passes);
   s = cuda_status(cudaGetLastError(), "radix histogram");
   if (s) return s;

@@ -346,3 +346,83 @@ def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
         n += 5 if n_isects > 0 else 3
     n += sort_launches(d, n_isects)
     return n + 3
+
+
+class HostPipeline:
+    """PackedStep steps over inputs and gradients that live in pinned host
+    memory, with the transfers overlapped: while step k's kernels run on the
+    compute stream, step k+1's inputs go host -> device on one copy stream and
+    step k-1's gradients go device -> host on another.  Device inputs and
+    gradient outputs are double-buffered (2 x parameters + 2 x gradients of
+    device memory); events order every reuse of a buffer.
+
+    run(host_steps) takes a list of (inputs, v_img, outputs) per step: inputs
+    are the six pinned host tensors of PackedStep.forward, v_img the pinned
+    upstream gradient, outputs a dict of pinned host tensors named like the
+    gradients (v_means, v_quats, v_scales, v_opacities, v_sh) that receive the
+    step's gradients.  Returns an event recorded after the last gradient
+    copy (on the copy stream) once everything has been enqueued; synchronize
+    on it (or call sync()) before reading the outputs.  With start (an event
+    recorded on the compute stream) the first upload waits for it, so a timed
+    region bracketed by start and the returned event holds every copy.
+    """
+
+    GRADS = ("v_means", "v_quats", "v_scales", "v_opacities", "v_sh")
+
+    def __init__(self, step: "PackedStep", example_inputs, example_v_img):
+        self.step = step
+        dev = step.dev
+        self.compute = torch.cuda.current_stream(dev)
+        self.up = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        self.dev_in = [[torch.empty(t.shape, dtype=t.dtype, device=dev) for t in example_inputs] for _ in range(2)]
+        self.dev_vimg = [torch.empty(example_v_img.shape, dtype=example_v_img.dtype, device=dev) for _ in range(2)]
+        self.dev_out = [{k: torch.empty_like(getattr(step, k)) for k in self.GRADS} for _ in range(2)]
+        self.in_free = [None, None]   # compute finished reading buffer p
+        self.out_free = [None, None]  # device -> host copy of buffer p finished
+
+    def _upload(self, k, inputs, v_img, after=None):
+        p = k % 2
+        ev = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.up):
+            if after is not None:
+                self.up.wait_event(after)
+            if self.in_free[p] is not None:
+                self.up.wait_event(self.in_free[p])
+            for dst, src in zip(self.dev_in[p], inputs):
+                dst.copy_(src, non_blocking=True)
+            self.dev_vimg[p].copy_(v_img, non_blocking=True)
+            ev.record(self.up)
+        return ev
+
+    def run(self, host_steps, start=None):
+        step = self.step
+        if not host_steps:
+            return None
+        uploaded = self._upload(0, host_steps[0][0], host_steps[0][1], after=start)
+        for k, (inputs, v_img, outputs) in enumerate(host_steps):
+            p = k % 2
+            self.compute.wait_event(uploaded)
+            if k + 1 < len(host_steps):
+                nxt = host_steps[k + 1]
+                uploaded = self._upload(k + 1, nxt[0], nxt[1])
+            if self.out_free[p] is not None:
+                self.compute.wait_event(self.out_free[p])
+            for name in self.GRADS:
+                setattr(step, name, self.dev_out[p][name])
+            step.forward(*self.dev_in[p])
+            step.backward(self.dev_vimg[p])
+            done = torch.cuda.Event()
+            done.record(self.compute)
+            self.in_free[p] = done
+            fin = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(self.down):
+                self.down.wait_event(done)
+                for name in self.GRADS:
+                    outputs[name].copy_(self.dev_out[p][name], non_blocking=True)
+                fin.record(self.down)
+            self.out_free[p] = fin
+        return self.out_free[(len(host_steps) - 1) % 2]
+
+    def sync(self):
+        torch.cuda.synchronize(self.step.dev)

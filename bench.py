@@ -165,6 +165,25 @@ def fp32_peak_instr_per_s(sm_mhz: float) -> float:
     return 148 * 128 * sm_mhz * 1e6
 
 
+# ---------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, device) -> float:
+    """Largest x over all ranks (a replicated step's time is its slowest
+    rank's); x itself when no process group is running."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput of `world` replicas each processing
+    units_per_rank in a step whose slowest rank took ms."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 # ---------------------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -263,11 +282,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = t0.elapsed_time(t1) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
 
     # ---- per-stage times (separate pass, events between the calls)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
@@ -333,11 +348,8 @@ def run_ours(args):
             a1.record(st)
             torch.cuda.synchronize()
             e_ms = a0.elapsed_time(a1) / ke
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = dict(value=world * step.n_isects / (e_ms / 1e3), unit="isects/s", ms_per_step=e_ms,
+        e_ms = max_over_ranks(e_ms, dev)
+        e2e = dict(value=job_throughput(step.n_isects, world, e_ms), unit="isects/s", ms_per_step=e_ms,
                    h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h))
 
     if world > 1:
@@ -382,7 +394,7 @@ def run_ours(args):
                     peak_source=f"148 SMs x 128 FP32 lanes x {sm_mhz:.0f} MHz (median SM clock under load)")
     launches = ss.launches_per_step(d, step.nnz, step.n_isects) * args.steps
     out_work = dict(work)
-    out = dict(metric=METRIC, value=world * step.n_isects / (ms / 1e3), unit="isects/s", n_gpus=world,
+    out = dict(metric=METRIC, value=job_throughput(step.n_isects, world, ms), unit="isects/s", n_gpus=world,
                steps=args.steps, warmup=args.warmup, ms_per_step=round(ms, 4), higher_is_better=True,
                scaling="weak", vs_baseline=None, dtype="f32", data="synthetic",
                config=dict(workload=f"config {args.config}: {sc.name}", C=d.C, N=d.N, W=d.W, H=d.H,

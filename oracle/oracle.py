@@ -359,3 +359,40 @@ def project_bwd_rows(scene, proj, rows, v_rows) -> np.ndarray:
                                _p(_c(proj["row_gauss"][rows], np.int64)), len(rows), _p(_c(v_rows, np.float64)),
                                _p(out))
     return out
+
+
+# ---------------------------------------------------------------------------- fused optimizer step
+ADAM_GROUPS = ("means", "quats", "log_scales", "logit_opacities", "sh")
+
+
+def raw_gradients(grads: dict, scales, opacities) -> dict:
+    """Gradients of the raw parameters from the activated ones: means and
+    quaternions unchanged, log-scales through s = exp(log s) (ds/dlog s = s),
+    logit-opacities through o = sigmoid(logit) (do/dlogit = o (1 - o))."""
+    s = np.asarray(scales, np.float64)
+    o = np.asarray(opacities, np.float64)
+    return dict(means=grads["v_means"], quats=grads["v_quats"], log_scales=grads["v_scales"] * s,
+                logit_opacities=grads["v_opacities"] * o * (1.0 - o), sh=grads["v_sh"])
+
+
+def adam_step(params: dict, grads: dict, m: dict, v: dict, lr: dict, beta1: float, beta2: float, eps: float,
+              t: int):
+    """One Adam update with bias correction, element by element (fp64):
+    m = b1 m + (1 - b1) g, v = b2 v + (1 - b2) g^2,
+    p = p - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps).
+    lr maps each group to its rate; "sh" may be a pair (DC rate, rest rate)
+    applied to coefficient 0 and to the others.  Returns new (params, m, v)."""
+    P, M, V = {}, {}, {}
+    for k in params:
+        g = np.asarray(grads[k], np.float64)
+        m1 = beta1 * np.asarray(m[k], np.float64) + (1.0 - beta1) * g
+        v1 = beta2 * np.asarray(v[k], np.float64) + (1.0 - beta2) * g * g
+        step = (m1 / (1.0 - beta1 ** t)) / (np.sqrt(v1 / (1.0 - beta2 ** t)) + eps)
+        rate = lr[k]
+        if k == "sh" and isinstance(rate, tuple):
+            r = np.full(step.shape, rate[1])
+            r[:, 0, :] = rate[0]
+            rate = r
+        P[k] = np.asarray(params[k], np.float64) - rate * step
+        M[k], V[k] = m1, v1
+    return P, M, V

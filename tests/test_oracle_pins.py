@@ -434,3 +434,79 @@ def test_backward_central_differences(seed, ext):
             checked += 1
             assert abs(vals[0] - an[i]) <= 1e-4 * max(1.0, abs(an[i])), (pname, i, vals, an[i])
     assert checked > 10 * skipped
+
+
+# ---------------------------------------------------------------- fused optimizer step
+def test_adam_matches_library_adam():
+    """The oracle's Adam against torch.optim.Adam (fp64, CPU) over three steps
+    with changing gradients, per group learning rates."""
+    import torch
+    rng = np.random.default_rng(21)
+    shapes = dict(means=(7, 3), quats=(7, 4), log_scales=(7, 3), logit_opacities=(7,), sh=(7, 4, 3))
+    lr = dict(means=1e-3, quats=2e-3, log_scales=5e-3, logit_opacities=5e-2, sh=2.5e-3)
+    b1, b2, eps = 0.9, 0.999, 1e-8
+    p0 = {k: rng.normal(size=s) for k, s in shapes.items()}
+    tp = {k: torch.tensor(p0[k], dtype=torch.float64, requires_grad=True) for k in shapes}
+    opt = torch.optim.Adam([{"params": [tp[k]], "lr": lr[k]} for k in shapes], betas=(b1, b2), eps=eps)
+    P = dict(p0)
+    M = {k: np.zeros(s) for k, s in shapes.items()}
+    V = {k: np.zeros(s) for k, s in shapes.items()}
+    for t in (1, 2, 3):
+        g = {k: rng.normal(size=s) * 10.0 ** rng.uniform(-4, 0) for k, s in shapes.items()}
+        for k in shapes:
+            tp[k].grad = torch.tensor(g[k], dtype=torch.float64)
+        opt.step()
+        P, M, V = orc.adam_step(P, g, M, V, lr, b1, b2, eps, t)
+        for k in shapes:
+            np.testing.assert_allclose(P[k], tp[k].detach().numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_adam_first_step_closed_form():
+    """From zero moments, step 1 moves every element by lr * g / (|g| + eps)."""
+    rng = np.random.default_rng(22)
+    g = {"means": rng.normal(size=(5, 3))}
+    p = {"means": rng.normal(size=(5, 3))}
+    z = {"means": np.zeros((5, 3))}
+    P, M, V = orc.adam_step(p, g, z, z, {"means": 0.01}, 0.9, 0.999, 1e-6, 1)
+    np.testing.assert_allclose(P["means"], p["means"] - 0.01 * g["means"] / (np.abs(g["means"]) + 1e-6), rtol=1e-12)
+    np.testing.assert_allclose(M["means"], 0.1 * g["means"], rtol=1e-14)
+    np.testing.assert_allclose(V["means"], 0.001 * g["means"] ** 2, rtol=1e-12)
+
+
+def test_raw_gradients_central_differences():
+    """d L / d log s = s * dL/ds and d L / d logit = o (1 - o) dL/do, against
+    central differences of the fp64 oracle in the raw parameters."""
+    sc = scenes.random_tiny(13, N=5, W=32, H=32, C=1, sh_degree=1, opacity_range=(0.2, 0.8))
+    for name in ("means", "quats", "scales", "opacities", "sh"):
+        setattr(sc, name, getattr(sc, name).astype(np.float64))
+    rng = np.random.default_rng(13)
+    v_img = rng.uniform(-1, 1, (sc.C, sc.H, sc.W, 3))
+    v_T = rng.uniform(-1, 1, (sc.C, sc.H, sc.W))
+    r = orc.step(sc, precision=1, v_img=v_img, v_T=v_T)
+    raw = orc.raw_gradients(r["grads"], sc.scales, sc.opacities)
+    log_s, logit = np.log(sc.scales), np.log(sc.opacities / (1.0 - sc.opacities))
+    checked = 0
+    for arr, act, key in ((log_s, lambda x: np.exp(x), "log_scales"),
+                          (logit, lambda x: 1.0 / (1.0 + np.exp(-x)), "logit_opacities")):
+        flat = arr.reshape(-1)
+        an = raw[key].reshape(-1)
+        for i in range(flat.size):
+            x0 = flat[i]
+            vals = []
+            for h in (1e-6, 5e-7):
+                out = []
+                for sgn in (1, -1):
+                    flat[i] = x0 + sgn * h
+                    if key == "log_scales":
+                        sc.scales = act(log_s)
+                    else:
+                        sc.opacities = act(logit)
+                    out.append(loss(sc, v_img, v_T))
+                flat[i] = x0
+                vals.append((out[0] - out[1]) / (2 * h))
+            sc.scales, sc.opacities = np.exp(log_s), 1.0 / (1.0 + np.exp(-logit))
+            if abs(vals[0] - vals[1]) > 1e-5 * max(1.0, abs(vals[0])):
+                continue
+            checked += 1
+            assert abs(vals[0] - an[i]) <= 1e-4 * max(1.0, abs(an[i])), (key, i, vals, an[i])
+    assert checked >= 15

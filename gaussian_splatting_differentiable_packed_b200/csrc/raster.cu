@@ -24,8 +24,8 @@ namespace ss {
 
 constexpr int kRThreads = 128;
 constexpr int kBatch = 256;
-// The backward stages half as many entries per batch: 17 KB of shared memory
-// and at most 64 registers per thread let 8 CTAs share an SM.
+// The backward stages half as many entries per batch (35 KB of shared memory
+// with the per-warp sums, at most 64 registers per thread).
 constexpr int kBatchB = 128;
 constexpr int kRedF = 12;
 
@@ -551,7 +551,7 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
 // EXT: v_depth (nullable, per pixel) and bg (nullable, [C][3]; the blend
 // img = C + T_final * bg adds g . bg to dL/dT_final).
 template <bool EXT>
-__global__ __launch_bounds__(kRThreads, 8) void k_raster_bwd(Geo g, const float* __restrict__ screen,
+__global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float* __restrict__ screen,
                                                           const uint32_t* __restrict__ vals,
                                                           const int64_t* __restrict__ tile_off,
                                                           const float* __restrict__ T_final,
@@ -562,7 +562,9 @@ __global__ __launch_bounds__(kRThreads, 8) void k_raster_bwd(Geo g, const float*
                                                           const float* __restrict__ bg,
                                                           float* __restrict__ v_screen) {
   __shared__ Stage s_e[kBatchB];
-  __shared__ __align__(16) float red[kBatchB][kRedF];  // per-entry sums over the CTA's warps
+  // each warp's per-entry sums (plain stores: a warp visits an entry at most
+  // once per batch), added up over the warps at the flush
+  __shared__ __align__(16) float red[kRThreads / 32][kBatchB][kRedF];
   __shared__ uint32_t s_any[kBatchB];
   __shared__ int s_maxlast;
   const int lane = threadIdx.x & 31;
@@ -576,7 +578,7 @@ __global__ __launch_bounds__(kRThreads, 8) void k_raster_bwd(Geo g, const float*
   const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f;
   const int64_t beg = tile_off[tile];
   const float amin = alpha_min();
-  for (int t = threadIdx.x; t < kBatchB * kRedF; t += kRThreads) (&red[0][0])[t] = 0.0f;
+  for (int t = threadIdx.x; t < (kRThreads / 32) * kBatchB * kRedF; t += kRThreads) (&red[0][0][0])[t] = 0.0f;
   for (int t = threadIdx.x; t < kBatchB; t += kRThreads) s_any[t] = 0u;
   if (threadIdx.x == 0) s_maxlast = -1;
   __syncthreads();
@@ -656,11 +658,11 @@ __global__ __launch_bounds__(kRThreads, 8) void k_raster_bwd(Geo g, const float*
             const float s8 = warp_reduce8(gr, lane);
             const float sb = warp_sum(gr[8]);
             const float sd = EXT ? warp_sum(gr[9]) : 0.0f;
-            if ((lane & 3) == 0)
-              atomicAdd(&red[k][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)], s8);
+            const int warp = threadIdx.x >> 5;
+            if ((lane & 3) == 0) red[warp][k][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = s8;
             if (lane == 0) {
-              atomicAdd(&red[k][8], sb);
-              if (EXT) atomicAdd(&red[k][9], sd);
+              red[warp][k][8] = sb;
+              if (EXT) red[warp][k][9] = sd;
               s_any[k] = 1u;
             }
           }
@@ -668,13 +670,22 @@ __global__ __launch_bounds__(kRThreads, 8) void k_raster_bwd(Geo g, const float*
       }
     }
     __syncthreads();
-    // one vector atomic per (entry, 16-byte quarter); the buffer is re-zeroed
+    // one vector atomic per (entry, 16-byte group) with the warps' sums
+    // added up; the buffers are re-zeroed
     for (int t = threadIdx.x; t < cnt * 3; t += kRThreads) {
       const int k = t / 3, q = t - 3 * k;
       if (!s_any[k]) continue;
-      float4* src = reinterpret_cast<float4*>(&red[k][4 * q]);
-      const float4 v = *src;
-      *src = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kRThreads / 32; ++w) {
+        float4* src = reinterpret_cast<float4*>(&red[w][k][4 * q]);
+        const float4 x = *src;
+        *src = make_float4(0.f, 0.f, 0.f, 0.f);
+        v.x += x.x;
+        v.y += x.y;
+        v.z += x.z;
+        v.w += x.w;
+      }
       atomicAdd(reinterpret_cast<float4*>(v_screen + (int64_t)__float_as_uint(s_e[k].d.y) * kRowF + 4 * q), v);
     }
     __syncthreads();

@@ -157,6 +157,11 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work):
                               instr=work["bwd_evals"] * 11.0 + work["bwd_exps"] * 17.0 + work["comps"] * 30.0)
     m["project_bwd"] = dict(bytes=(par + shb) * N + row * nnz + P / 8 + P / 16 + (par + 4 + shb) * N,
                             instr=nnz * 700.0)
+    # fused with Adam: parameters, activated copies and both moments read and
+    # written once, no gradient arrays
+    pa = par + 4 + shb
+    m["project_bwd_adam"] = dict(bytes=(pa + 16) * N + 2 * pa * N + row * nnz + P / 8 + P / 16
+                                 + (pa + 16) * N + 2 * pa * N, instr=nnz * 700.0)
     return m
 
 
@@ -227,7 +232,36 @@ def run_ours(args):
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
 
-    names = ["project_packed", "intersect_tiles", "sort_isects", "rasterize_fwd", "rasterize_bwd", "project_bwd"]
+    # optional fused projection backward + Adam: raw parameters, activated
+    # copies and moments on the device, updated in place every step
+    trainer = None
+    if args.adam:
+        cams, means, quats, scales, opac, sh = inputs
+        trainer = ss.AdamTrainer(step, cams, means, quats, torch.log(scales).contiguous(),
+                                 torch.log(opac / (1.0 - opac)).contiguous(), sh, eps=1e-8)
+        inputs = (cams, means, quats, trainer.scales, trainer.opacities, sh)
+
+    last_stage = "project_bwd_adam" if args.adam else "project_bwd"
+    names = ["project_packed", "intersect_tiles", "sort_isects", "rasterize_fwd", "rasterize_bwd", last_stage]
+
+    def backward_rest():
+        if trainer is None:
+            ss.ss_project_bwd(d, *inputs, step.mask, step.block_off, step.v_screen, step.v_means, step.v_quats,
+                              step.v_scales, step.v_opacities, step.v_sh)
+        else:
+            trainer.hp.step += 1
+            ss.ss_project_bwd_adam(d, trainer.cams, trainer.means, trainer.quats, trainer.log_scales,
+                                   trainer.scales, trainer.logit_opacities, trainer.opacities, trainer.sh, step.mask,
+                                   step.block_off, step.v_screen, trainer.state, trainer.hp)
+
+    def whole_step():
+        step.forward(*inputs, **fkw)
+        if trainer is None:
+            step.backward(v_img, **bkw)
+        else:
+            ss.ss_rasterize_bwd(d, step.screen, step.vals, step.tile_off, step.T, step.last, v_img, None,
+                                step.v_screen, step.nnz)
+            backward_rest()
 
     def run_step(ev=None):
         if ev is not None:
@@ -239,8 +273,7 @@ def run_ours(args):
             ss.ss_rasterize_bwd(d, step.screen, step.vals, step.tile_off, step.T, step.last, v_img, None,
                                 step.v_screen, step.nnz, v_depth=v_D, bg=bg_t)
             ev[5].record(st)
-            ss.ss_project_bwd(d, *inputs, step.mask, step.block_off, step.v_screen, step.v_means, step.v_quats,
-                              step.v_scales, step.v_opacities, step.v_sh)
+            backward_rest()
             ev[6].record(st)
 
     def _timed_forward(ev):
@@ -261,8 +294,7 @@ def run_ours(args):
         step.nnz, step.n_isects = nnz, n
 
     for _ in range(args.warmup):
-        step.forward(*inputs, **fkw)
-        step.backward(v_img, **bkw)
+        whole_step()
     torch.cuda.synchronize()
 
     # ---- headline: K whole steps, device-timed, max over ranks
@@ -275,8 +307,7 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(st)
     for _ in range(args.steps):
-        step.forward(*inputs, **fkw)
-        step.backward(v_img, **bkw)
+        whole_step()
     t1.record(st)
     torch.cuda.synchronize()
     if world > 1:
@@ -299,7 +330,7 @@ def run_ours(args):
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.adam:  # the training run keeps its state on the device
         host_in = [t.cpu().pin_memory() for t in inputs]
         host_vimg = v_img.cpu().pin_memory()
         host_out = {k: torch.empty(tuple(getattr(step, k).shape), dtype=torch.float32).pin_memory()
@@ -400,7 +431,8 @@ def run_ours(args):
                config=dict(workload=f"config {args.config}: {sc.name}", C=d.C, N=d.N, W=d.W, H=d.H,
                            sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
                            sort_passes=passes, l2="inputs larger than L2 (3.5 GB parameters), no flush",
-                           parallelism=f"replicas x{world}", depth_and_background=bool(args.depth_bg)),
+                           parallelism=f"replicas x{world}", depth_and_background=bool(args.depth_bg),
+                           fused_adam=bool(args.adam)),
                pairs_per_s=world * d.C * d.N / (ms / 1e3),
                pixel_gaussian_evals_per_s=world * work["evals"] / (stage_ms["rasterize_fwd"] / 1e3),
                step_roofline_frac=round(step_frac, 4), raster_work=out_work, stages=stages, roofline=roof,
@@ -473,6 +505,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=300_000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--adam", action="store_true",
+                    help="train: the projection backward fused with an Adam step updates the parameters in place")
     ap.add_argument("--depth-bg", action="store_true",
                     help="also render the expected depth over a background colour and back-propagate a depth gradient")
     args = ap.parse_args()

@@ -12,6 +12,8 @@
 // Deterministic: no atomics.  Decisions that gate gradients (the Jacobian's
 // off-axis clamp, the colour clamp) are re-taken with the forward's
 // canonical arithmetic.
+#include <cmath>
+
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 
@@ -76,7 +78,28 @@ __host__ __device__ constexpr int sh_stride() {
   return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
 }
 
-template <int DEG>
+// Fused optimizer step (the pages' "fused projection backward + optimizer":
+// the gradient sums never leave registers / shared memory).  Adam with bias
+// correction on the raw parameters: means, quaternions, log-scales,
+// logit-opacities and SH coefficients; the kernel also refreshes the activated
+// copies (scales = exp, opacities = sigmoid) that the next forward reads.
+struct AdamArgs {
+  float *m_means, *v_means, *m_quats, *v_quats, *m_scales, *v_scales, *m_opac, *v_opac, *m_sh, *v_sh;
+  float *means, *quats, *log_scales, *scales, *logit_opac, *opac, *sh;  // updated in place
+  float lr_means, lr_quats, lr_scales, lr_opac, lr_sh_dc, lr_sh_rest;
+  float b1, b2, eps;
+  float ibc1;   // 1 / (1 - beta1^t)
+  float ibc2s;  // 1 / sqrt(1 - beta2^t)
+};
+
+// One Adam update of parameter p with gradient g; m and v are updated in place.
+__device__ __forceinline__ float adam_update(float p, float g, float& m, float& v, float lr, const AdamArgs& a) {
+  m = a.b1 * m + (1.0f - a.b1) * g;
+  v = a.b2 * v + (1.0f - a.b2) * g * g;
+  return p - lr * (m * a.ibc1) / (sqrtf(v) * a.ibc2s + a.eps);
+}
+
+template <int DEG, bool ADAM>
 __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* __restrict__ cams,
                                                            const float* __restrict__ means,
                                                            const float* __restrict__ quats,
@@ -87,7 +110,8 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
                                                            const float* __restrict__ v_screen,
                                                            float* __restrict__ v_means, float* __restrict__ v_quats,
                                                            float* __restrict__ v_scales, float* __restrict__ v_opac,
-                                                           float* __restrict__ v_sh) {
+                                                           float* __restrict__ v_sh, const float* __restrict__ opacities,
+                                                           AdamArgs adam) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = 3 * K;
   constexpr int KP = sh_stride<DEG>();
@@ -325,17 +349,73 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     vx += -4.f * x * GR[8]; vy += -4.f * y * GR[8];
     const double dq = w * vw + x * vx + y * vy + z * vz;
     const double qi = qr.inv;
-    v_means[3 * n] = gmu[0];
-    v_means[3 * n + 1] = gmu[1];
-    v_means[3 * n + 2] = gmu[2];
-    reinterpret_cast<float4*>(v_quats)[n] = make_float4((float)((vw - w * dq) * qi), (float)((vx - x * dq) * qi),
-                                                        (float)((vy - y * dq) * qi), (float)((vz - z * dq) * qi));
-    v_scales[3 * n] = (float)gsc[0];
-    v_scales[3 * n + 1] = (float)gsc[1];
-    v_scales[3 * n + 2] = (float)gsc[2];
-    v_opac[n] = go;
+    const float gq[4] = {(float)((vw - w * dq) * qi), (float)((vx - x * dq) * qi), (float)((vy - y * dq) * qi),
+                         (float)((vz - z * dq) * qi)};
+    if (!ADAM) {
+      v_means[3 * n] = gmu[0];
+      v_means[3 * n + 1] = gmu[1];
+      v_means[3 * n + 2] = gmu[2];
+      reinterpret_cast<float4*>(v_quats)[n] = make_float4(gq[0], gq[1], gq[2], gq[3]);
+      v_scales[3 * n] = (float)gsc[0];
+      v_scales[3 * n + 1] = (float)gsc[1];
+      v_scales[3 * n + 2] = (float)gsc[2];
+      v_opac[n] = go;
+    } else {
+      // means and raw quaternions take their gradients directly; log-scales
+      // and logit-opacities through the activations (ds/dlog s = s,
+      // do/dlogit = o (1 - o))
+      const float mu[3] = {mx, my, mz};
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+        float m = adam.m_means[3 * n + i], v = adam.v_means[3 * n + i];
+        adam.means[3 * n + i] = adam_update(mu[i], gmu[i], m, v, adam.lr_means, adam);
+        adam.m_means[3 * n + i] = m;
+        adam.v_means[3 * n + i] = v;
+      }
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+      float qn[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float m = adam.m_quats[4 * n + i], v = adam.v_quats[4 * n + i];
+        qn[i] = adam_update(qv[i], gq[i], m, v, adam.lr_quats, adam);
+        adam.m_quats[4 * n + i] = m;
+        adam.v_quats[4 * n + i] = v;
+      }
+      reinterpret_cast<float4*>(adam.quats)[n] = make_float4(qn[0], qn[1], qn[2], qn[3]);
+      const float sc[3] = {s0, s1, s2};
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+        float m = adam.m_scales[3 * n + i], v = adam.v_scales[3 * n + i];
+        const float ls = adam_update(adam.log_scales[3 * n + i], (float)gsc[i] * sc[i], m, v, adam.lr_scales, adam);
+        adam.log_scales[3 * n + i] = ls;
+        adam.scales[3 * n + i] = expf(ls);
+        adam.m_scales[3 * n + i] = m;
+        adam.v_scales[3 * n + i] = v;
+      }
+      const float o = opacities[n];
+      float m = adam.m_opac[n], v = adam.v_opac[n];
+      const float lo = adam_update(adam.logit_opac[n], go * o * (1.0f - o), m, v, adam.lr_opac, adam);
+      adam.logit_opac[n] = lo;
+      adam.opac[n] = 1.0f / (1.0f + expf(-lo));
+      adam.m_opac[n] = m;
+      adam.v_opac[n] = v;
+    }
   }
   __syncthreads();
+  if (ADAM) {
+    // the CTA's SH block: Adam on each coefficient (DC with its own rate),
+    // the staged values are the parameters, coalesced over the block
+    const int64_t b0 = n0 * K3;
+    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+      const int gi = f / K3, q = f - gi * K3;
+      float m = adam.m_sh[b0 + f], v = adam.v_sh[b0 + f];
+      adam.sh[b0 + f] = adam_update(sh_s[gi * KP + q], gsh_s[gi * KP + q], m, v,
+                                    q < 3 ? adam.lr_sh_dc : adam.lr_sh_rest, adam);
+      adam.m_sh[b0 + f] = m;
+      adam.v_sh[b0 + f] = v;
+    }
+    return;
+  }
   // coalesced write-back of the CTA's SH gradient block (16-byte stores for a
   // full block)
   float* dst = v_sh + n0 * K3;
@@ -357,18 +437,39 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   }
 }
 
-template <int DEG>
+template <int DEG, bool ADAM>
 ss_status launch_pbwd(const Geo& g, unsigned grid, cudaStream_t st, const float* cams, const float* means,
                       const float* quats, const float* scales, const float* sh, const uint32_t* mask,
                       const int64_t* block_off, const float* v_screen, float* v_means, float* v_quats,
-                      float* v_scales, float* v_opacities, float* v_sh) {
+                      float* v_scales, float* v_opacities, float* v_sh, const float* opacities,
+                      const AdamArgs& adam) {
   const size_t smem = 2 * sizeof(float) * kBlock * sh_stride<DEG>();
-  ss_status s = cuda_status(
-      cudaFuncSetAttribute(k_project_bwd<DEG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "smem attr");
+  ss_status s = cuda_status(cudaFuncSetAttribute(k_project_bwd<DEG, ADAM>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                            "smem attr");
   if (s) return s;
-  k_project_bwd<DEG><<<grid, kBlock, smem, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                                 v_means, v_quats, v_scales, v_opacities, v_sh);
+  k_project_bwd<DEG, ADAM><<<grid, kBlock, smem, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                                       v_means, v_quats, v_scales, v_opacities, v_sh, opacities,
+                                                       adam);
   return cuda_status(cudaGetLastError(), "project bwd");
+}
+
+template <bool ADAM>
+ss_status dispatch_pbwd(const Geo& g, cudaStream_t st, const float* cams, const float* means, const float* quats,
+                        const float* scales, const float* sh, const uint32_t* mask, const int64_t* block_off,
+                        const float* v_screen, float* v_means, float* v_quats, float* v_scales, float* v_opacities,
+                        float* v_sh, const float* opacities, const AdamArgs& adam) {
+  const unsigned grid = (unsigned)g.blocks_per_cam;
+  switch (g.deg) {
+    case 0: return launch_pbwd<0, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                        v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
+    case 1: return launch_pbwd<1, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                        v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
+    case 2: return launch_pbwd<2, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                        v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
+    default: return launch_pbwd<3, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                         v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
+  }
 }
 
 }  // namespace ss
@@ -388,17 +489,42 @@ extern "C" ss_status ss_project_bwd(const ss_dims* dims, const float* cams, cons
   if (((uintptr_t)quats & 15) || ((uintptr_t)v_quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15) ||
       ((uintptr_t)v_sh & 15))
     return invalid("quats, v_quats, v_screen, sh and v_sh must be 16-byte aligned");
-  (void)opacities;
   cudaStream_t st = as_stream(stream);
-  const unsigned grid = (unsigned)g.blocks_per_cam;
-  switch (g.deg) {
-    case 0: return launch_pbwd<0>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
-                                  v_quats, v_scales, v_opacities, v_sh);
-    case 1: return launch_pbwd<1>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
-                                  v_quats, v_scales, v_opacities, v_sh);
-    case 2: return launch_pbwd<2>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
-                                  v_quats, v_scales, v_opacities, v_sh);
-    default: return launch_pbwd<3>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
-                                   v_quats, v_scales, v_opacities, v_sh);
-  }
+  return dispatch_pbwd<false>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means, v_quats,
+                              v_scales, v_opacities, v_sh, opacities, AdamArgs{});
+}
+
+extern "C" ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams, float* means, float* quats,
+                                         float* log_scales, float* scales, float* logit_opacities, float* opacities,
+                                         float* sh, const uint32_t* mask, const int64_t* block_off,
+                                         const float* v_screen, const ss_adam_state* state, const ss_adam* hp,
+                                         void* stream) {
+  if (!dims_ok(dims)) return invalid("dims");
+  const Geo g = geometry(*dims);
+  if (g.N == 0) return SS_OK;
+  if (!state || !hp) return invalid("null state or hyper-parameters");
+  if (!cams || !means || !quats || !log_scales || !scales || !logit_opacities || !opacities || !sh || !mask ||
+      !block_off || !v_screen)
+    return invalid("null input");
+  const ss_adam_state& S = *state;
+  if (!S.m_means || !S.v_means || !S.m_quats || !S.v_quats || !S.m_scales || !S.v_scales || !S.m_opacities ||
+      !S.v_opacities || !S.m_sh || !S.v_sh)
+    return invalid("null optimizer state");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15))
+    return invalid("quats, v_screen and sh must be 16-byte aligned");
+  if (hp->step < 1) return invalid("adam step must be >= 1");
+  AdamArgs a{};
+  a.m_means = S.m_means; a.v_means = S.v_means; a.m_quats = S.m_quats; a.v_quats = S.v_quats;
+  a.m_scales = S.m_scales; a.v_scales = S.v_scales; a.m_opac = S.m_opacities; a.v_opac = S.v_opacities;
+  a.m_sh = S.m_sh; a.v_sh = S.v_sh;
+  a.means = means; a.quats = quats; a.log_scales = log_scales; a.scales = scales; a.logit_opac = logit_opacities;
+  a.opac = opacities; a.sh = sh;
+  a.lr_means = hp->lr_means; a.lr_quats = hp->lr_quats; a.lr_scales = hp->lr_scales;
+  a.lr_opac = hp->lr_opacities; a.lr_sh_dc = hp->lr_sh_dc; a.lr_sh_rest = hp->lr_sh_rest;
+  a.b1 = hp->beta1; a.b2 = hp->beta2; a.eps = hp->eps;
+  a.ibc1 = (float)(1.0 / (1.0 - std::pow((double)hp->beta1, (double)hp->step)));
+  a.ibc2s = (float)(1.0 / std::sqrt(1.0 - std::pow((double)hp->beta2, (double)hp->step)));
+  cudaStream_t st = as_stream(stream);
+  return dispatch_pbwd<true>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, opacities, a);
 }

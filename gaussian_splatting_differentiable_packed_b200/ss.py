@@ -30,7 +30,18 @@ TILE = 16
 EXPORTS = ("ss_size", "ss_workspace_bytes", "ss_status_string", "ss_last_error", "ss_project_packed",
            "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc", "ss_rasterize_fwd",
            "ss_rasterize_fwd_counts",
-           "ss_rasterize_bwd", "ss_project_bwd")
+           "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam")
+
+
+class ss_adam(ct.Structure):
+    _fields_ = [("lr_means", ct.c_float), ("lr_quats", ct.c_float), ("lr_scales", ct.c_float),
+                ("lr_opacities", ct.c_float), ("lr_sh_dc", ct.c_float), ("lr_sh_rest", ct.c_float),
+                ("beta1", ct.c_float), ("beta2", ct.c_float), ("eps", ct.c_float), ("step", ct.c_int32)]
+
+
+class ss_adam_state(ct.Structure):
+    _fields_ = [(n, ct.c_void_p) for n in ("m_means", "v_means", "m_quats", "v_quats", "m_scales", "v_scales",
+                                           "m_opacities", "v_opacities", "m_sh", "v_sh")]
 
 
 class ss_dims(ct.Structure):
@@ -73,9 +84,11 @@ def lib() -> ct.CDLL:
         L.ss_rasterize_fwd_counts.argtypes = [D, P, P, P, P, P, P, P, P]
         L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, i64, P]
         L.ss_project_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.ss_project_bwd_adam.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, ct.POINTER(ss_adam_state),
+                                          ct.POINTER(ss_adam), P]
         for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc",
                   "ss_rasterize_fwd",
-                  "ss_rasterize_fwd_counts", "ss_rasterize_bwd", "ss_project_bwd"):
+                  "ss_rasterize_fwd_counts", "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -189,6 +202,52 @@ def ss_project_bwd(d, cams, means, quats, scales, opacities, sh, mask, block_off
     _check(lib().ss_project_bwd(ct.byref(d), _p(cams), _p(means), _p(quats), _p(scales), _p(opacities), _p(sh),
                                 _p(mask), _p(block_off), _p(v_screen), _p(v_means), _p(v_quats), _p(v_scales),
                                 _p(v_opacities), _p(v_sh), _stream(stream)), "ss_project_bwd")
+
+
+def ss_project_bwd_adam(d, cams, means, quats, log_scales, scales, logit_opacities, opacities, sh, mask, block_off,
+                        v_screen, state: dict, hp: ss_adam, stream=None):
+    """Fused projection backward + Adam.  state maps m_/v_ + (means, quats,
+    scales, opacities, sh) to device tensors shaped like the parameters."""
+    st = ss_adam_state(*[_p(state[n]) for n, _ in ss_adam_state._fields_])
+    _check(lib().ss_project_bwd_adam(ct.byref(d), _p(cams), _p(means), _p(quats), _p(log_scales), _p(scales),
+                                     _p(logit_opacities), _p(opacities), _p(sh), _p(mask), _p(block_off),
+                                     _p(v_screen), ct.byref(st), ct.byref(hp), _stream(stream)),
+           "ss_project_bwd_adam")
+
+
+class AdamTrainer:
+    """Training steps on one PackedStep with the fused projection backward +
+    Adam: the parameters (means, raw quats, log-scales, logit-opacities, SH),
+    their activated copies and the moments live on the device and are updated
+    in place each step; no gradient arrays are written.
+
+    step(v_img_fn) runs forward, the rasterizer backward with the upstream
+    gradient v_img_fn(img) and the fused update, and returns the image."""
+
+    def __init__(self, step: "PackedStep", cams, means, quats, log_scales, logit_opacities, sh,
+                 lr=(1.6e-4, 1e-3, 5e-3, 5e-2, 2.5e-3, 1.25e-4), beta1=0.9, beta2=0.999, eps=1e-15):
+        self.step_obj = step
+        self.cams, self.means, self.quats, self.sh = cams, means, quats, sh
+        self.log_scales, self.logit_opacities = log_scales, logit_opacities
+        self.scales = torch.exp(log_scales).contiguous()
+        self.opacities = torch.sigmoid(logit_opacities).contiguous()
+        self.state = {}
+        for name, ref in (("means", means), ("quats", quats), ("scales", log_scales),
+                          ("opacities", logit_opacities), ("sh", sh)):
+            self.state["m_" + name] = torch.zeros_like(ref)
+            self.state["v_" + name] = torch.zeros_like(ref)
+        self.hp = ss_adam(*lr, beta1, beta2, eps, 0)
+
+    def step(self, v_img_fn, stream=None):
+        s = self.step_obj
+        img = s.forward(self.cams, self.means, self.quats, self.scales, self.opacities, self.sh, stream)
+        v_img = v_img_fn(img)
+        ss_rasterize_bwd(s.d, s.screen, s.vals, s.tile_off, s.T, s.last, v_img, None, s.v_screen, s.nnz, stream)
+        self.hp.step += 1
+        ss_project_bwd_adam(s.d, self.cams, self.means, self.quats, self.log_scales, self.scales,
+                            self.logit_opacities, self.opacities, self.sh, s.mask, s.block_off, s.v_screen,
+                            self.state, self.hp, stream)
+        return img
 
 
 def _u32(n, dev):

@@ -11,6 +11,7 @@
  *   ss_rasterize_bwd    per-pixel reverse replay -> screen-space gradients
  *   ss_project_bwd      screen-space gradients -> means, quats, scales,
  *                       opacities, SH coefficients
+ *   ss_project_bwd_adam the same, fused with an Adam step on the parameters
  *
  * Conventions (all entry points):
  *   - Every array pointer is a DEVICE pointer owned by the caller unless the
@@ -18,9 +19,11 @@
  *     or frees memory and keeps no state between calls.  Calls that need
  *     scratch take (temp, temp_bytes), sized by ss_workspace_bytes().
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
- *     legacy default stream).  Only ss_project_packed and ss_intersect_tiles
- *     synchronise the stream, to return the counts that size later buffers.
- *   - Outputs are overwritten, never accumulated into.
+ *     legacy default stream).  ss_project_packed and ss_intersect_tiles
+ *     synchronise the stream to return the counts that size later buffers,
+ *     ss_sort_isects to read its device-side check flag.
+ *   - Outputs are overwritten, never accumulated into (ss_project_bwd_adam
+ *     updates its parameters and optimizer state in place).
  *   - Floating point is IEEE fp32; integer outputs are deterministic.
  *   - Errors are returned as ss_status; a failing call writes no element
  *     outside the caller's stated capacities.  Device-side checks never trap.
@@ -156,6 +159,43 @@ ss_status ss_intersect_tiles(const ss_dims* dims, const float* screen, const uin
 ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
                          uint32_t* vals_b, int64_t n, void* temp, size_t temp_bytes, int64_t* tile_off,
                          int* result_in_b_out, void* stream);
+
+/*
+ * Projection backward fused with an Adam step (the pages' fused projection
+ * backward + optimizer, "Spirula Studio backward pass", section 6: the
+ * world-space gradient sums go straight into the optimizer, so no gradient
+ * arrays are written).  Same gradient chain as ss_project_bwd; then, per
+ * element, Adam with bias correction on the raw parameters
+ *   m = b1 m + (1 - b1) g,  v = b2 v + (1 - b2) g^2,
+ *   p = p - lr * (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * where the raw parameters are means, quats (unnormalised), log_scales,
+ * logit_opacities and sh, and g for log-scales / logit-opacities is the
+ * activated gradient times s / o (1 - o).  Updates in place: means, quats,
+ * log_scales, logit_opacities, sh and the moments; refreshes the activated
+ * copies scales = exp(log_scales) and opacities = sigmoid(logit_opacities)
+ * that the forward reads (scales and opacities are read first as the
+ * activated values the forward used).  All arrays are device memory laid out
+ * like the parameters; state and hp are host structs.  quats, v_screen and sh
+ * must be 16-byte aligned; hp->step >= 1.
+ */
+typedef struct ss_adam {
+  float lr_means, lr_quats, lr_scales, lr_opacities, lr_sh_dc, lr_sh_rest;
+  float beta1, beta2, eps;
+  int32_t step; /* t of this update, >= 1 */
+} ss_adam;
+
+typedef struct ss_adam_state {
+  float *m_means, *v_means;         /* [N][3] */
+  float *m_quats, *v_quats;         /* [N][4] */
+  float *m_scales, *v_scales;       /* [N][3], of the log-scales */
+  float *m_opacities, *v_opacities; /* [N], of the logit-opacities */
+  float *m_sh, *v_sh;               /* [N][K][3] */
+} ss_adam_state;
+
+ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams, float* means, float* quats, float* log_scales,
+                              float* scales, float* logit_opacities, float* opacities, float* sh,
+                              const uint32_t* mask, const int64_t* block_off, const float* v_screen,
+                              const ss_adam_state* state, const ss_adam* hp, void* stream);
 
 /*
  * Allocation-free variant of ss_sort_isects (the pages have no counterpart:

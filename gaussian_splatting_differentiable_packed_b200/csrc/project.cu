@@ -90,13 +90,15 @@ struct RowItem {
   int cam;  // camera within the current chunk
   int g;    // Gaussian within the CTA
 };
-constexpr int kQueue = 2 * kBlock;
 
-// Pass 2 keeps its 128 threads busy whatever the visibility pattern: the
-// visible pairs of the CTA's Gaussians are appended camera by camera to a
-// shared queue (row = block_off of the camera's block + rank among the set
-// bits) and processed 128 at a time by any thread, with the Gaussians'
-// parameters and SH blocks in shared memory.
+// Pass 2 keeps its 128 threads busy whatever the visibility pattern.  For a
+// chunk of cameras the CTA stages each warp's mask word per camera and an
+// exclusive prefix of their popcounts in camera-major order; the chunk's
+// visible pairs are then items 0..total-1 of a virtual list, and thread t
+// decodes item i (t, t + 128, ...) by itself: the (camera, warp) slot by
+// binary search in the prefix, the lane as the rank-th set bit of the slot's
+// word, the row as the camera's block offset plus the rank among the
+// camera's set bits.  Consecutive items are consecutive rows.
 template <int DEG>
 __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __restrict__ cams,
                                                          const float* __restrict__ means,
@@ -110,13 +112,15 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = 3 * K;
   constexpr int KP = rows_sh_stride<DEG>();
+  constexpr int kWarps = kBlock / 32;
+  constexpr int kSlots = kCamChunk * kWarps;
   __shared__ Cam scam[kCamChunk];
   __shared__ float sh_s[kBlock * KP];
   __shared__ GaussIn s_g[kBlock];
   __shared__ float s_o[kBlock];
-  __shared__ RowItem q[kQueue];
-  __shared__ int q_len;
-  __shared__ uint32_t s_wc[kBlock / 32];
+  __shared__ uint32_t s_word[kSlots];  // [camera][warp]
+  __shared__ int s_pre[kSlots + 1];    // exclusive prefix of the words' popcounts
+  __shared__ int64_t s_row0[kCamChunk];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t blk = blockIdx.x;
   const int64_t n0 = blk * kBlock;
@@ -159,7 +163,6 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
       }
     }
   }
-  if (threadIdx.x == 0) q_len = 0;
   auto process = [&](const RowItem& it) {
     const Cam& k = scam[it.cam];
     const GaussIn& gi = s_g[it.g];
@@ -194,48 +197,57 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   };
   for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
     const int nc = min(kCamChunk, g.C - c0);
+    const int ns = nc * kWarps;
     __syncthreads();
-    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
-    __syncthreads();
-    for (int cc = 0; cc < nc; ++cc) {
-      const int64_t c = c0 + cc;
-      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
-      const uint32_t word = mask[wbase + warp];
-      if (lane == 0) s_wc[warp] = __popc(word);
-      __syncthreads();
-      int before = 0, total = 0;
-#pragma unroll
-      for (int w = 0; w < kBlock / 32; ++w) {
-        before += w < warp ? (int)s_wc[w] : 0;
-        total += (int)s_wc[w];
-      }
-      const int base = q_len;
-      if ((word >> lane) & 1u) {
-        const int r = before + __popc(word & ((1u << lane) - 1u));
-        RowItem it;
-        it.row = block_off[c * g.blocks_per_cam + blk] + r;
-        it.cam = cc;
-        it.g = threadIdx.x;
-        q[base + r] = it;
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) q_len = base + total;
-      __syncthreads();
-      if (q_len >= kBlock) {  // a full round: every thread takes one item
-        const int len = q_len;
-        process(q[threadIdx.x]);
-        __syncthreads();
-        for (int t = kBlock + threadIdx.x; t < len; t += kBlock) q[t - kBlock] = q[t];
-        __syncthreads();
-        if (threadIdx.x == 0) q_len = len - kBlock;
-        __syncthreads();
-      }
+    if (threadIdx.x < nc) {
+      scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
+      s_row0[threadIdx.x] = block_off[(int64_t)(c0 + threadIdx.x) * g.blocks_per_cam + blk];
     }
-    // the queue refers to this chunk's cameras: drain it before the next chunk
-    const int len = q_len;
-    if (threadIdx.x < len) process(q[threadIdx.x]);
+    if (threadIdx.x < ns) {
+      const int64_t c = c0 + threadIdx.x / kWarps;
+      s_word[threadIdx.x] = mask[(c * g.n_pad + blk * kBlock) / 32 + threadIdx.x % kWarps];
+    }
     __syncthreads();
-    if (threadIdx.x == 0) q_len = 0;
+    if (warp == 0) {
+      // exclusive prefix over the ns <= 128 slots, 4 consecutive slots a lane
+      int v[4], sum = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int sl = 4 * lane + u;
+        v[u] = sl < ns ? __popc(s_word[sl]) : 0;
+        sum += v[u];
+      }
+      int inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+      }
+      int run = inc - sum;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int sl = 4 * lane + u;
+        if (sl < ns) s_pre[sl] = run;
+        run += v[u];
+      }
+      if (lane == 31) s_pre[ns] = inc;  // the chunk's total
+    }
+    __syncthreads();
+    const int total = s_pre[ns];
+    for (int i = threadIdx.x; i < total; i += kBlock) {
+      int lo = 0, hi = ns;  // largest slot j with s_pre[j] <= i
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_pre[mid] <= i) lo = mid; else hi = mid;
+      }
+      const int cc = lo / kWarps, w = lo - cc * kWarps;
+      const int rank = i - s_pre[lo];
+      RowItem it;
+      it.cam = cc;
+      it.g = w * 32 + (int)__fns(s_word[lo], 0, rank + 1);
+      it.row = s_row0[cc] + (s_pre[lo] - s_pre[cc * kWarps]) + rank;
+      process(it);
+    }
   }
 }
 

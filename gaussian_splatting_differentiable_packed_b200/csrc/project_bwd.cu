@@ -404,15 +404,51 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   __syncthreads();
   if (ADAM) {
     // the CTA's SH block: Adam on each coefficient (DC with its own rate),
-    // the staged values are the parameters, coalesced over the block
+    // the staged values are the parameters.  A full block moves the moments
+    // and parameters in 16-byte vectors, kChunk of them in flight per thread
+    // (the block starts 16-byte aligned); the ragged last block word by word.
     const int64_t b0 = n0 * K3;
-    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-      const int gi = f / K3, q = f - gi * K3;
-      float m = adam.m_sh[b0 + f], v = adam.v_sh[b0 + f];
-      adam.sh[b0 + f] = adam_update(sh_s[gi * KP + q], gsh_s[gi * KP + q], m, v,
-                                    q < 3 ? adam.lr_sh_dc : adam.lr_sh_rest, adam);
-      adam.m_sh[b0 + f] = m;
-      adam.v_sh[b0 + f] = v;
+    if (cnt == kBlock) {
+      constexpr int kV = kBlock * K3 / 4;
+      constexpr int kChunk = 4;
+      float4* m4 = reinterpret_cast<float4*>(adam.m_sh + b0);
+      float4* v4 = reinterpret_cast<float4*>(adam.v_sh + b0);
+      float4* p4 = reinterpret_cast<float4*>(adam.sh + b0);
+      for (int v0 = threadIdx.x; v0 < kV; v0 += kChunk * kBlock) {
+        float4 mb[kChunk], vb[kChunk];
+#pragma unroll
+        for (int r = 0; r < kChunk; ++r) {
+          const int vv = v0 + r * kBlock;
+          if (vv < kV) {
+            mb[r] = m4[vv];
+            vb[r] = v4[vv];
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < kChunk; ++r) {
+          const int vv = v0 + r * kBlock;
+          if (vv >= kV) continue;
+          float me[4] = {mb[r].x, mb[r].y, mb[r].z, mb[r].w}, ve[4] = {vb[r].x, vb[r].y, vb[r].z, vb[r].w}, pe[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int f = 4 * vv + u, gi = f / K3, q = f - gi * K3;
+            pe[u] = adam_update(sh_s[gi * KP + q], gsh_s[gi * KP + q], me[u], ve[u],
+                                q < 3 ? adam.lr_sh_dc : adam.lr_sh_rest, adam);
+          }
+          p4[vv] = make_float4(pe[0], pe[1], pe[2], pe[3]);
+          m4[vv] = make_float4(me[0], me[1], me[2], me[3]);
+          v4[vv] = make_float4(ve[0], ve[1], ve[2], ve[3]);
+        }
+      }
+    } else {
+      for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+        const int gi = f / K3, q = f - gi * K3;
+        float m = adam.m_sh[b0 + f], v = adam.v_sh[b0 + f];
+        adam.sh[b0 + f] = adam_update(sh_s[gi * KP + q], gsh_s[gi * KP + q], m, v,
+                                      q < 3 ? adam.lr_sh_dc : adam.lr_sh_rest, adam);
+        adam.m_sh[b0 + f] = m;
+        adam.v_sh[b0 + f] = v;
+      }
     }
     return;
   }
@@ -510,8 +546,9 @@ extern "C" ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams,
   if (!S.m_means || !S.v_means || !S.m_quats || !S.v_quats || !S.m_scales || !S.v_scales || !S.m_opacities ||
       !S.v_opacities || !S.m_sh || !S.v_sh)
     return invalid("null optimizer state");
-  if (((uintptr_t)quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15))
-    return invalid("quats, v_screen and sh must be 16-byte aligned");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15) || ((uintptr_t)S.m_sh & 15) ||
+      ((uintptr_t)S.v_sh & 15))
+    return invalid("quats, v_screen, sh and the SH moments must be 16-byte aligned");
   if (hp->step < 1) return invalid("adam step must be >= 1");
   AdamArgs a{};
   a.m_means = S.m_means; a.v_means = S.v_means; a.m_quats = S.m_quats; a.v_quats = S.v_quats;

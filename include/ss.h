@@ -175,8 +175,8 @@ ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a
  * copies scales = exp(log_scales) and opacities = sigmoid(logit_opacities)
  * that the forward reads (scales and opacities are read first as the
  * activated values the forward used).  All arrays are device memory laid out
- * like the parameters; state and hp are host structs.  quats, v_screen and sh
- * must be 16-byte aligned; hp->step >= 1.
+ * like the parameters; state and hp are host structs.  quats, v_screen, sh
+ * and the SH moments must be 16-byte aligned; hp->step >= 1.
  */
 typedef struct ss_adam {
   float lr_means, lr_quats, lr_scales, lr_opacities, lr_sh_dc, lr_sh_rest;

@@ -410,7 +410,7 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     const int64_t b0 = n0 * K3;
     if (cnt == kBlock) {
       constexpr int kV = kBlock * K3 / 4;
-      constexpr int kChunk = 4;
+      constexpr int kChunk = (kV + kBlock - 1) / kBlock;  // every vector of the thread in flight
       float4* m4 = reinterpret_cast<float4*>(adam.m_sh + b0);
       float4* v4 = reinterpret_cast<float4*>(adam.v_sh + b0);
       float4* p4 = reinterpret_cast<float4*>(adam.sh + b0);

@@ -141,6 +141,12 @@ def test_many_cameras_ragged():
     full_parity(scenes.random_tiny(40, N=517, W=45, H=23, C=33, sh_degree=2))
 
 
+def test_opacity_above_one():
+    # opacities in (0.5, 1.6): entries with o > 1 take no skip threshold and no
+    # culling (every pixel evaluates them), the alpha clamp at 0.99 is hit
+    full_parity(scenes.random_tiny(41, N=600, W=48, H=40, C=2, sh_degree=1, opacity_range=(0.5, 1.6)))
+
+
 def test_empty_scene():
     sc = scenes.random_tiny(1, N=0, W=40, H=24)
     o = orc.step(sc)

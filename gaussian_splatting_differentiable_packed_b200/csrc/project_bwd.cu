@@ -92,6 +92,14 @@ struct AdamArgs {
   float ibc2s;  // 1 / sqrt(1 - beta2^t)
 };
 
+// Asks L2 to fetch [p, p + bytes) ahead of use (bulk prefetch, no data
+// returned to the SM; bytes is rounded down to the 16-byte granule).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  bytes &= ~15u;
+  if (bytes == 0 || ((uintptr_t)p & 15)) return;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // One Adam update of parameter p with gradient g; m and v are updated in place.
 __device__ __forceinline__ float adam_update(float p, float g, float& m, float& v, float lr, const AdamArgs& a) {
   m = a.b1 * m + (1.0f - a.b1) * g;
@@ -128,6 +136,19 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   const int64_t n = n0 + threadIdx.x;
   const bool valid = n < g.N;
   const int cnt = (int)min64(kBlock, g.N - n0);
+  if (ADAM && threadIdx.x == 0) {
+    // the optimizer state is only touched after the camera loop: have L2 fetch
+    // the CTA's moment blocks now, so the update reads them from L2
+    prefetch_l2(adam.m_sh + n0 * K3, (uint32_t)(cnt * K3 * 4));
+    prefetch_l2(adam.v_sh + n0 * K3, (uint32_t)(cnt * K3 * 4));
+    prefetch_l2(adam.m_means + 3 * n0, (uint32_t)(cnt * 12));
+    prefetch_l2(adam.v_means + 3 * n0, (uint32_t)(cnt * 12));
+    prefetch_l2(adam.m_quats + 4 * n0, (uint32_t)(cnt * 16));
+    prefetch_l2(adam.v_quats + 4 * n0, (uint32_t)(cnt * 16));
+    prefetch_l2(adam.m_scales + 3 * n0, (uint32_t)(cnt * 12));
+    prefetch_l2(adam.v_scales + 3 * n0, (uint32_t)(cnt * 12));
+    prefetch_l2(adam.log_scales + 3 * n0, (uint32_t)(cnt * 12));
+  }
   // coalesced staging of the CTA's contiguous SH block: full blocks with all
   // 16-byte loads in flight at once (the block starts 16-byte aligned: 128*K3
   // floats per block), the ragged last block word by word

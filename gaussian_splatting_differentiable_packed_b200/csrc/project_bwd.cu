@@ -136,6 +136,14 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   const int64_t n = n0 + threadIdx.x;
   const bool valid = n < g.N;
   const int cnt = (int)min64(kBlock, g.N - n0);
+  // the CTA's gradient rows of camera c are the contiguous rows
+  // block_off[c][blk] .. block_off[c][blk + 1]: have L2 fetch them now, the
+  // camera loop reads them one pair at a time
+  for (int c = threadIdx.x; c < g.C; c += kBlock) {
+    const int64_t r0 = block_off[(int64_t)c * g.blocks_per_cam + blk];
+    const int64_t r1 = block_off[(int64_t)c * g.blocks_per_cam + blk + 1];
+    prefetch_l2(v_screen + r0 * kRowF, (uint32_t)((r1 - r0) * kRowF * 4));
+  }
   if (ADAM && threadIdx.x == 0) {
     // the optimizer state is only touched after the camera loop: have L2 fetch
     // the CTA's moment blocks now, so the update reads them from L2

@@ -108,7 +108,8 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
                                                          const float* __restrict__ sh,
                                                          const uint32_t* __restrict__ mask,
                                                          const int64_t* __restrict__ block_off,
-                                                         float* __restrict__ screen, uint32_t* __restrict__ aabb16) {
+                                                         float* __restrict__ screen, uint32_t* __restrict__ aabb16,
+                                                         int64_t ahead) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = 3 * K;
   constexpr int KP = rows_sh_stride<DEG>();
@@ -126,6 +127,16 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   const int64_t n0 = blk * kBlock;
   const int64_t n = n0 + threadIdx.x;
   const int cnt = (int)min64(kBlock, g.N - n0);
+  if (threadIdx.x == 0 && ahead > 0 && blk + ahead < (int64_t)gridDim.x) {
+    // the parameters of the block that starts about a wave later, into L2
+    const int64_t m0 = (blk + ahead) * kBlock;
+    const int mc = (int)min64(kBlock, g.N - m0);
+    prefetch_l2(sh + m0 * K3, (uint32_t)(mc * K3 * 4));
+    prefetch_l2(means + 3 * m0, (uint32_t)(mc * 12));
+    prefetch_l2(quats + 4 * m0, (uint32_t)(mc * 16));
+    prefetch_l2(scales + 3 * m0, (uint32_t)(mc * 12));
+    prefetch_l2(opacities + m0, (uint32_t)(mc * 4));
+  }
   if (n < g.N) {
     s_g[threadIdx.x] = load_gauss(means, quats, scales, n);
     s_o[threadIdx.x] = opacities[n];
@@ -255,8 +266,9 @@ template <int DEG>
 void launch_rows(const Geo& g, unsigned grid, cudaStream_t st, const float* cams, const float* means,
                  const float* quats, const float* scales, const float* opacities, const float* sh,
                  const uint32_t* mask, const int64_t* block_off, float* screen, uint32_t* aabb16) {
+  const int64_t ahead = wave_blocks(k_project_rows<DEG>, kBlock, 0);
   k_project_rows<DEG><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, opacities, sh, mask, block_off, screen,
-                                               aabb16);
+                                               aabb16, ahead);
 }
 
 }  // namespace ss

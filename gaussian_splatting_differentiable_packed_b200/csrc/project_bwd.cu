@@ -92,14 +92,6 @@ struct AdamArgs {
   float ibc2s;  // 1 / sqrt(1 - beta2^t)
 };
 
-// Asks L2 to fetch [p, p + bytes) ahead of use (bulk prefetch, no data
-// returned to the SM; bytes is rounded down to the 16-byte granule).
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  bytes &= ~15u;
-  if (bytes == 0 || ((uintptr_t)p & 15)) return;
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // One Adam update of parameter p with gradient g; m and v are updated in place.
 __device__ __forceinline__ float adam_update(float p, float g, float& m, float& v, float lr, const AdamArgs& a) {
   m = a.b1 * m + (1.0f - a.b1) * g;

@@ -77,6 +77,26 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
+// Asks L2 to fetch [p, p + bytes) ahead of use (bulk prefetch, no data
+// returned to the SM; bytes is rounded down to the 16-byte granule).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  bytes &= ~15u;
+  if (bytes == 0 || ((uintptr_t)p & 15)) return;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Resident CTAs of a kernel over the whole GPU (SMs x CTAs per SM): the
+// distance, in blocks, between a CTA and the one that starts about a wave
+// later.  0 if the query fails (then nothing is prefetched ahead).
+template <typename K>
+inline int64_t wave_blocks(K kernel, int threads, size_t smem) {
+  int dev = 0, sms = 0, per = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, threads, smem) != cudaSuccess) return 0;
+  return (int64_t)sms * per;
+}
+
 // ----- generic exclusive scan (int64 totals), defined in scan.cu -----
 // Items are produced by a "counter" selected by kind:
 enum ScanKind { SCAN_U32 = 0, SCAN_TILES = 1 };

@@ -428,7 +428,8 @@ def run_ours(args):
     out = dict(metric=METRIC, value=job_throughput(step.n_isects, world, ms), unit="isects/s", n_gpus=world,
                steps=args.steps, warmup=args.warmup, ms_per_step=round(ms, 4), higher_is_better=True,
                scaling="weak", vs_baseline=None, dtype="f32", data="synthetic",
-               config=dict(workload=f"config {args.config}: {sc.name}", C=d.C, N=d.N, W=d.W, H=d.H,
+               config=dict(workload=sc.name if args.n is None else f"{sc.name}, N overridden to {d.N}",
+                           C=d.C, N=d.N, W=d.W, H=d.H,
                            sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
                            sort_passes=passes, l2="inputs larger than L2 (3.5 GB parameters), no flush",
                            parallelism=f"replicas x{world}", depth_and_background=bool(args.depth_bg),
@@ -462,7 +463,7 @@ def cpu_baseline(config: int, n_sample: int, repeats: int = 1):
         isects += r["isect"]["n_isects"]
     dt = time.perf_counter() - t
     return dict(value=isects / dt, unit="isects/s", cores=cores, kind="oracle",
-                sample=f"config {config} distributions and cameras with N={n_sample} Gaussians "
+                sample=f"the workload's distributions and cameras ({sc.name}) with N={n_sample} Gaussians "
                        f"({r['isect']['n_isects']} intersections, full image size), {repeats} step(s) "
                        f"in {dt:.1f} s")
 
@@ -487,9 +488,9 @@ def run_reference(args):
     out = dict(impl="reference", metric=METRIC, value=v, unit="isects/s", n_gpus=world, steps=args.steps,
                warmup=args.warmup, ms_per_step=1e3 * dt / args.steps, higher_is_better=True, scaling="weak",
                vs_baseline=None, dtype="f32", data="synthetic",
-               config=dict(workload=f"config {args.config} (bounded sample, N={args.cpu_sample})"),
+               config=dict(workload=f"{sc.name}: bounded sample with N={sc.N} Gaussians"),
                cpu_baseline=dict(value=v, unit="isects/s", cores=cores, kind="oracle",
-                                 sample=f"config {args.config} with N={args.cpu_sample} Gaussians per step"),
+                                 sample=f"{sc.name} with N={sc.N} Gaussians per step"),
                e2e=dict(value=v, unit="isects/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(out))
 

@@ -111,7 +111,7 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
                                                            float* __restrict__ v_means, float* __restrict__ v_quats,
                                                            float* __restrict__ v_scales, float* __restrict__ v_opac,
                                                            float* __restrict__ v_sh, const float* __restrict__ opacities,
-                                                           AdamArgs adam) {
+                                                           AdamArgs adam, int64_t ahead) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = 3 * K;
   constexpr int KP = sh_stride<DEG>();
@@ -135,6 +135,11 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     const int64_t r0 = block_off[(int64_t)c * g.blocks_per_cam + blk];
     const int64_t r1 = block_off[(int64_t)c * g.blocks_per_cam + blk + 1];
     prefetch_l2(v_screen + r0 * kRowF, (uint32_t)((r1 - r0) * kRowF * 4));
+  }
+  if (threadIdx.x == 0 && ahead > 0 && blk + ahead < (int64_t)gridDim.x) {
+    // the SH block of the CTA that starts about a wave later, into L2
+    const int64_t m0 = (blk + ahead) * kBlock;
+    prefetch_l2(sh + m0 * K3, (uint32_t)(min64(kBlock, g.N - m0) * K3 * 4));
   }
   if (ADAM && threadIdx.x == 0) {
     // the optimizer state is only touched after the camera loop: have L2 fetch
@@ -505,9 +510,10 @@ ss_status launch_pbwd(const Geo& g, unsigned grid, cudaStream_t st, const float*
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                             "smem attr");
   if (s) return s;
+  const int64_t ahead = wave_blocks(k_project_bwd<DEG, ADAM>, kBlock, smem);
   k_project_bwd<DEG, ADAM><<<grid, kBlock, smem, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
                                                        v_means, v_quats, v_scales, v_opacities, v_sh, opacities,
-                                                       adam);
+                                                       adam, ahead);
   return cuda_status(cudaGetLastError(), "project bwd");
 }
 

@@ -462,6 +462,63 @@ __device__ __forceinline__ float warp_reduce8(float* a, int lane) {
   return a[0];
 }
 
+// Two entries' eight sums reduced together: the exchange across lane bit 4
+// leaves the first entry's partial sums in lanes 0-15 and the second's in
+// lanes 16-31, and each half finishes as warp_reduce8 does over lane bits
+// 3..1.  Lane l returns value 4*b3 + 2*b2 + b1 of entry b4 (bn: bit n of
+// l), in 16 shuffles where two single reductions take 18.
+__device__ __forceinline__ float warp_reduce8x2(float* a, const float* b, int lane) {
+  bool up = lane & 16;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float send = up ? a[q] : b[q];
+    const float keep = up ? b[q] : a[q];
+    a[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+  up = lane & 8;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float send = up ? a[q] : a[q + 4];
+    const float keep = up ? a[q + 4] : a[q];
+    a[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  up = lane & 4;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const float send = up ? a[q] : a[q + 2];
+    const float keep = up ? a[q + 2] : a[q];
+    a[q] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  up = lane & 2;
+  {
+    const float send = up ? a[0] : a[1];
+    const float keep = up ? a[1] : a[0];
+    a[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  a[0] += __shfl_xor_sync(0xffffffffu, a[0], 1);
+  return a[0];
+}
+
+// Warp sums of (a0, a1) for one entry and (b0, b1) for another: lane l
+// returns value b3 of entry b4 (value 0: a0 or b0, value 1: a1 or b1).
+// With `two` false only value 0 is reduced (lanes 0-15: a0, 16-31: b0).
+template <bool two>
+__device__ __forceinline__ float warp_sum_x2(float a0, float a1, float b0, float b1, int lane) {
+  bool up = lane & 16;
+  float v = (up ? b0 : a0) + __shfl_xor_sync(0xffffffffu, up ? a0 : b0, 16);
+  if (two) {
+    const float v1 = (up ? b1 : a1) + __shfl_xor_sync(0xffffffffu, up ? a1 : b1, 16);
+    up = lane & 8;
+    v = (up ? v1 : v) + __shfl_xor_sync(0xffffffffu, up ? v : v1, 8);
+  } else {
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+  }
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -548,6 +605,32 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
   return true;
 }
 
+// One replayed entry (bit hb of the lanes' candidate masks mA, mB) for the
+// thread's pixel pair: sigma and exp where a pixel is a candidate, then the
+// reverse step.  gr[0..9] is zero when neither pixel contributes.
+template <bool EXT>
+__device__ __forceinline__ bool entry_grad(const Stage& st, uint32_t mA, uint32_t mB, int hb, float px, float2 npy,
+                                           float amin, PixB& pa, PixB& pb, float* gr) {
+  bool contrib = false;
+  const bool liveA = (mA >> hb) & 1u, liveB = (mB >> hb) & 1u;
+  if (liveA || liveB) {
+    const float dx = sub(st.a.x, px);
+    const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
+    const float2 sig = sigma_pair(st, dx, dy);
+    const bool needA = liveA && !(sig.x < 0.0f) && !(sig.x > st.d.x);
+    const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
+    if (needA || needB) {
+      const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
+      contrib = pair_grad<EXT>(st, dx, dy, ev, needA, needB, amin, pa, pb, gr);
+    }
+  }
+  if (!contrib) {
+#pragma unroll
+    for (int t = 0; t < 10; ++t) gr[t] = 0.0f;
+  }
+  return contrib;
+}
+
 // EXT: v_depth (nullable, per pixel) and bg (nullable, [C][3]; the blend
 // img = C + T_final * bg adds g . bg to dL/dT_final).
 template <bool EXT>
@@ -631,39 +714,50 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
         const uint32_t mA = warp_transpose32(covA, lane) & live_bits(pa.last, qb);
         const uint32_t mB = warp_transpose32(covB, lane) & live_bits(pb.last, qb);
         uint32_t bits = __reduce_or_sync(0xffffffffu, mA | mB);
+        const int warp = threadIdx.x >> 5;
         while (bits) {
           const int hb = 31 - __clz(bits);
           bits &= ~(1u << hb);
-          const int k = q * 32 + hb;
-          const Stage& st = s_e[k];
+          int kA = q * 32 + hb;
           float gr[10];
-          bool contrib = false;
-          const bool liveA = (mA >> hb) & 1u, liveB = (mB >> hb) & 1u;
-          if (liveA || liveB) {
-            const float dx = sub(st.a.x, px);
-            const float2 dy = __fadd2_rn(f2s(st.a.y), npy);
-            const float2 sig = sigma_pair(st, dx, dy);
-            const bool needA = liveA && !(sig.x < 0.0f) && !(sig.x > st.d.x);
-            const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
-            if (needA || needB) {
-              const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
-              contrib = pair_grad<EXT>(st, dx, dy, ev, needA, needB, amin, pa, pb, gr);
+          bool anyA = __any_sync(0xffffffffu, entry_grad<EXT>(s_e[kA], mA, mB, hb, px, npy, amin, pa, pb, gr));
+          if (bits) {
+            // the next candidate of the warp: its pixel step follows this
+            // one's, and the two entries' sums are reduced together
+            const int hb2 = 31 - __clz(bits);
+            bits &= ~(1u << hb2);
+            const int kB = q * 32 + hb2;
+            float gr2[10];
+            const bool anyB =
+                __any_sync(0xffffffffu, entry_grad<EXT>(s_e[kB], mA, mB, hb2, px, npy, amin, pa, pb, gr2));
+            if (anyA && anyB) {
+              const float s8 = warp_reduce8x2(gr, gr2, lane);
+              const float s2 = warp_sum_x2<EXT>(gr[8], gr[9], gr2[8], gr2[9], lane);
+              const int kl = (lane & 16) ? kB : kA;
+              if ((lane & 1) == 0) red[warp][kl][((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = s8;
+              if ((lane & 15) == 0) {
+                red[warp][kl][8] = s2;
+                s_any[kl] = 1u;
+              }
+              if (EXT && (lane & 15) == 8) red[warp][kl][9] = s2;
+              continue;
+            }
+            if (anyB) {
+#pragma unroll
+              for (int t = 0; t < 10; ++t) gr[t] = gr2[t];
+              kA = kB;
+              anyA = true;
             }
           }
-          if (!contrib) {
-#pragma unroll
-            for (int t = 0; t < 10; ++t) gr[t] = 0.0f;
-          }
-          if (__any_sync(0xffffffffu, contrib)) {
+          if (anyA) {
             const float s8 = warp_reduce8(gr, lane);
             const float sb = warp_sum(gr[8]);
             const float sd = EXT ? warp_sum(gr[9]) : 0.0f;
-            const int warp = threadIdx.x >> 5;
-            if ((lane & 3) == 0) red[warp][k][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = s8;
+            if ((lane & 3) == 0) red[warp][kA][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = s8;
             if (lane == 0) {
-              red[warp][k][8] = sb;
-              if (EXT) red[warp][k][9] = sd;
-              s_any[k] = 1u;
+              red[warp][kA][8] = sb;
+              if (EXT) red[warp][kA][9] = sd;
+              s_any[kA] = 1u;
             }
           }
         }

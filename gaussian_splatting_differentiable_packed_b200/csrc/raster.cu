@@ -605,6 +605,33 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
   return true;
 }
 
+// One vector atomic per (touched entry, 16-byte group) of a batch with the
+// warps' sums added up, one thread per entry; the sums and the entry's flag
+// are re-zeroed for the batch after next.
+__device__ __forceinline__ void flush_sums(float (*red)[kBatchB][kRedF], const uint32_t* rows, uint32_t* any, int cnt,
+                                           float* __restrict__ v_screen) {
+  for (int k = threadIdx.x; k < cnt; k += kRThreads) {
+    if (!any[k]) continue;
+    any[k] = 0u;
+    float* dst = v_screen + (int64_t)rows[k] * kRowF;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kRThreads / 32; ++w) {
+        float4* src = reinterpret_cast<float4*>(&red[w][k][4 * q]);
+        const float4 x = *src;
+        *src = make_float4(0.f, 0.f, 0.f, 0.f);
+        v.x += x.x;
+        v.y += x.y;
+        v.z += x.z;
+        v.w += x.w;
+      }
+      atomicAdd(reinterpret_cast<float4*>(dst + 4 * q), v);
+    }
+  }
+}
+
 // One replayed entry (bit hb of the lanes' candidate masks mA, mB) for the
 // thread's pixel pair: sigma and exp where a pixel is a candidate, then the
 // reverse step.  gr[0..9] is zero when neither pixel contributes.
@@ -648,7 +675,11 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
   // each warp's per-entry sums (plain stores: a warp visits an entry at most
   // once per batch), added up over the warps at the flush
   __shared__ __align__(16) float red[kRThreads / 32][kBatchB][kRedF];
-  __shared__ uint32_t s_any[kBatchB];
+  // row ids and touched flags of the batch in work and of the one being
+  // flushed (double-buffered: the flush of a batch runs beside the staging
+  // of the next one)
+  __shared__ uint32_t s_row[2][kBatchB];
+  __shared__ uint32_t s_any[2][kBatchB];
   __shared__ int s_maxlast;
   const int lane = threadIdx.x & 31;
   const int64_t tile = blockIdx.x;
@@ -662,7 +693,7 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
   const int64_t beg = tile_off[tile];
   const float amin = alpha_min();
   for (int t = threadIdx.x; t < (kRThreads / 32) * kBatchB * kRedF; t += kRThreads) (&red[0][0][0])[t] = 0.0f;
-  for (int t = threadIdx.x; t < kBatchB; t += kRThreads) s_any[t] = 0u;
+  for (int t = threadIdx.x; t < 2 * kBatchB; t += kRThreads) (&s_any[0][0])[t] = 0u;
   if (threadIdx.x == 0) s_maxlast = -1;
   __syncthreads();
   PixB pa{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1}, pb{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1};
@@ -696,11 +727,19 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
   int64_t wlast = max64(pa.last, pb.last);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wlast = max64(wlast, __shfl_xor_sync(0xffffffffu, wlast, o));
-  for (int64_t b1 = stop; b1 > beg; b1 -= kBatchB) {
+  int par = 0, prev_cnt = 0;
+  for (int64_t b1 = stop; b1 > beg; b1 -= kBatchB, par ^= 1) {
     const int64_t b0 = max64(beg, b1 - kBatchB);
     const int cnt = (int)(b1 - b0);
-    for (int t = threadIdx.x; t < cnt; t += kRThreads) stage_row(screen, vals[b0 + t], s_e[t]);
+    for (int t = threadIdx.x; t < cnt; t += kRThreads) {
+      const uint32_t r = vals[b0 + t];
+      s_row[par][t] = r;
+      stage_row(screen, r, s_e[t]);
+    }
+    flush_sums(red, s_row[par ^ 1], s_any[par ^ 1], prev_cnt, v_screen);
+    prev_cnt = cnt;
     __syncthreads();
+    uint32_t* any = s_any[par];
     if (b0 <= wlast) {
       for (int q = (cnt - 1) / 32; q >= 0; --q) {
         const int e = q * 32 + lane;
@@ -737,7 +776,7 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
               if ((lane & 1) == 0) red[warp][kl][((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = s8;
               if ((lane & 15) == 0) {
                 red[warp][kl][8] = s2;
-                s_any[kl] = 1u;
+                any[kl] = 1u;
               }
               if (EXT && (lane & 15) == 8) red[warp][kl][9] = s2;
               continue;
@@ -757,34 +796,15 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
             if (lane == 0) {
               red[warp][kA][8] = sb;
               if (EXT) red[warp][kA][9] = sd;
-              s_any[kA] = 1u;
+              any[kA] = 1u;
             }
           }
         }
       }
     }
     __syncthreads();
-    // one vector atomic per (entry, 16-byte group) with the warps' sums
-    // added up; the buffers are re-zeroed
-    for (int t = threadIdx.x; t < cnt * 3; t += kRThreads) {
-      const int k = t / 3, q = t - 3 * k;
-      if (!s_any[k]) continue;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < kRThreads / 32; ++w) {
-        float4* src = reinterpret_cast<float4*>(&red[w][k][4 * q]);
-        const float4 x = *src;
-        *src = make_float4(0.f, 0.f, 0.f, 0.f);
-        v.x += x.x;
-        v.y += x.y;
-        v.z += x.z;
-        v.w += x.w;
-      }
-      atomicAdd(reinterpret_cast<float4*>(v_screen + (int64_t)__float_as_uint(s_e[k].d.y) * kRowF + 4 * q), v);
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < cnt; t += kRThreads) s_any[t] = 0u;
   }
+  flush_sums(red, s_row[par ^ 1], s_any[par ^ 1], prev_cnt, v_screen);
 }
 
 }  // namespace ss

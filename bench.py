@@ -3,7 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
 
 A step is one pass of the whole path over the workload: ss_project_packed,
-ss_intersect_tiles, ss_sort_isects, ss_rasterize_fwd, ss_rasterize_bwd,
+ss_intersect_tiles, ss_sort_isects, ss_tile_order, ss_rasterize_fwd, ss_rasterize_bwd,
 ss_project_bwd.  The upstream dL/dimage is an input of the step (the L1
 gradient against the workload's seeded target, computed once from the forward
 image before timing; the step's work does not depend on its values).
@@ -260,7 +260,7 @@ def run_ours(args):
             step.backward(v_img, **bkw)
         else:
             ss.ss_rasterize_bwd(d, step.screen, step.vals, step.tile_off, step.T, step.last, v_img, None,
-                                step.v_screen, step.nnz)
+                                step.v_screen, step.nnz, tile_order=step.tile_order)
             backward_rest()
 
     def run_step(ev=None):
@@ -271,7 +271,7 @@ def run_ours(args):
             step.backward(v_img, **bkw)
         else:
             ss.ss_rasterize_bwd(d, step.screen, step.vals, step.tile_off, step.T, step.last, v_img, None,
-                                step.v_screen, step.nnz, v_depth=v_D, bg=bg_t)
+                                step.v_screen, step.nnz, v_depth=v_D, bg=bg_t, tile_order=step.tile_order)
             ev[5].record(st)
             backward_rest()
             ev[6].record(st)
@@ -288,8 +288,10 @@ def run_ours(args):
                                  step.tile_off)
         step.vals = step.vals_b if in_b else step.vals_a
         ev[3].record(st)
+        # the rasterizers' tile order is part of the forward rasterizer's stage
+        ss.ss_tile_order(d, step.tile_off, step.tile_order, step.temp_order)
         ss.ss_rasterize_fwd(d, step.screen, step.vals, step.tile_off, step.img, step.T, step.last,
-                            step.depth if args.depth_bg else None, bg_t)
+                            step.depth if args.depth_bg else None, bg_t, tile_order=step.tile_order)
         ev[4].record(st)
         step.nnz, step.n_isects = nnz, n
 

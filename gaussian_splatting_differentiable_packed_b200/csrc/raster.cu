@@ -350,10 +350,12 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd_masked(Geo g, const fl
                                                                  float* __restrict__ img, float* __restrict__ T_final,
                                                                  int32_t* __restrict__ last_id,
                                                                  float* __restrict__ depth,
-                                                                 const float* __restrict__ bg) {
+                                                                 const float* __restrict__ bg,
+                                                                 const uint32_t* __restrict__ tile_order) {
   __shared__ Stage s_e[kBatch];
   const int lane = threadIdx.x & 31;
-  const int64_t tile = blockIdx.x;
+  const int64_t tile = tile_order ? (int64_t)tile_order[blockIdx.x] : (int64_t)blockIdx.x;
+  if (tile >= g.n_tiles) return;  // not a tile index: nothing to draw
   int c, tx0, ty0, i, j;
   tile_coords(g, tile, c, tx0, ty0, i, j);
   const bool inA = i < g.W && j < g.H, inB = i < g.W && j + 1 < g.H;
@@ -670,6 +672,7 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
                                                           const float* __restrict__ v_T,
                                                           const float* __restrict__ v_depth,
                                                           const float* __restrict__ bg,
+                                                          const uint32_t* __restrict__ tile_order,
                                                           float* __restrict__ v_screen) {
   __shared__ Stage s_e[kBatchB];
   // each warp's per-entry sums (plain stores: a warp visits an entry at most
@@ -682,7 +685,8 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
   __shared__ uint32_t s_any[2][kBatchB];
   __shared__ int s_maxlast;
   const int lane = threadIdx.x & 31;
-  const int64_t tile = blockIdx.x;
+  const int64_t tile = tile_order ? (int64_t)tile_order[blockIdx.x] : (int64_t)blockIdx.x;
+  if (tile >= g.n_tiles) return;  // not a tile index: nothing to replay
   int c, tx0, ty0, i, j;
   tile_coords(g, tile, c, tx0, ty0, i, j);
   const bool inA = i < g.W && j < g.H, inB = i < g.W && j + 1 < g.H;
@@ -807,13 +811,99 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
   flush_sums(red, s_row[par ^ 1], s_any[par ^ 1], prev_cnt, v_screen);
 }
 
+// ----- tile order: heaviest tiles first ------------------------------------
+// The rasterizers take one CTA per tile, and tiles differ in their entry
+// counts by orders of magnitude (most are empty, a few hold thousands of
+// entries).  The block scheduler hands out CTAs in index order, so a heavy
+// tile that comes late runs on after the rest have finished; taking tiles in
+// decreasing order of entry count (longest first) keeps the SMs busy to the
+// end.  The order is a counting sort over bins of the count: four bins per
+// power of two (the two bits below the leading one), heavier bins first,
+// empty tiles last; the order inside a bin is the order the atomic cursor
+// hands out (any order draws the same images).
+constexpr int kOrderBins = 128;
+
+__device__ __forceinline__ int order_bin(int64_t cnt) {
+  if (cnt <= 0) return kOrderBins - 1;
+  const int msb = 63 - __clzll((long long)cnt);
+  const int key = msb < 2 ? (int)cnt : 4 * msb + (int)((cnt >> (msb - 2)) & 3);  // non-decreasing in cnt
+  return max(0, kOrderBins - 2 - key);
+}
+
+__global__ __launch_bounds__(256) void k_order_hist(const int64_t* __restrict__ tile_off, int64_t n_tiles,
+                                                    uint32_t* __restrict__ hist) {
+  __shared__ uint32_t h[kOrderBins];
+  for (int i = threadIdx.x; i < kOrderBins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_tiles; t += (int64_t)gridDim.x * blockDim.x)
+    atomicAdd(&h[order_bin(tile_off[t + 1] - tile_off[t])], 1u);
+  __syncthreads();
+  for (int i = threadIdx.x; i < kOrderBins; i += blockDim.x)
+    if (h[i]) atomicAdd(&hist[i], h[i]);
+}
+
+// hist -> exclusive prefix in place (the bins' write cursors); one warp.
+__global__ void k_order_scan(uint32_t* __restrict__ hist) {
+  const int lane = threadIdx.x;
+  uint32_t carry = 0;
+  for (int b0 = 0; b0 < kOrderBins; b0 += 32) {
+    const uint32_t v = hist[b0 + lane];
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += x;
+    }
+    hist[b0 + lane] = carry + inc - v;
+    carry += __shfl_sync(0xffffffffu, inc, 31);
+  }
+}
+
+// One cursor atomic per (warp, bin): lanes with equal bins share it.
+__global__ __launch_bounds__(256) void k_order_scatter(const int64_t* __restrict__ tile_off, int64_t n_tiles,
+                                                       uint32_t* __restrict__ cursor,
+                                                       uint32_t* __restrict__ tile_order) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < n_tiles; base += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = base + threadIdx.x;
+    const bool valid = t < n_tiles;
+    const int bin = valid ? order_bin(tile_off[t + 1] - tile_off[t]) : -1 - lane;
+    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+    const int leader = __ffs(peers) - 1;
+    uint32_t first = 0;
+    if (valid && lane == leader) first = atomicAdd(&cursor[bin], (uint32_t)__popc(peers));
+    first = __shfl_sync(0xffffffffu, first, leader);
+    if (valid) tile_order[first + __popc(peers & ((1u << lane) - 1u))] = (uint32_t)t;
+  }
+}
+
+size_t tile_order_temp_bytes() { return kOrderBins * sizeof(uint32_t); }
+
 }  // namespace ss
 
 using namespace ss;
 
+extern "C" ss_status ss_tile_order(const ss_dims* dims, const int64_t* tile_off, uint32_t* tile_order, void* temp,
+                                   size_t temp_bytes, void* stream) {
+  if (!dims_ok(dims)) return invalid("dims");
+  if (!tile_off || !tile_order) return invalid("null pointer");
+  if (!temp || temp_bytes < tile_order_temp_bytes()) return invalid("temp too small");
+  const Geo g = geometry(*dims);
+  cudaStream_t st = as_stream(stream);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(temp);
+  ss_status s = cuda_status(cudaMemsetAsync(hist, 0, tile_order_temp_bytes(), st), "memset");
+  if (s) return s;
+  const unsigned grid = (unsigned)max64(1, min64(ceil_div(g.n_tiles, 256), 148 * 4));
+  k_order_hist<<<grid, 256, 0, st>>>(tile_off, g.n_tiles, hist);
+  k_order_scan<<<1, 32, 0, st>>>(hist);
+  k_order_scatter<<<grid, 256, 0, st>>>(tile_off, g.n_tiles, hist, tile_order);
+  return cuda_status(cudaGetLastError(), "tile order");
+}
+
 extern "C" ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, const uint32_t* vals,
-                                      const int64_t* tile_off, float* img, float* T_final, int32_t* last_id,
-                                      float* depth, const float* bg, void* stream) {
+                                      const int64_t* tile_off, const uint32_t* tile_order, float* img,
+                                      float* T_final, int32_t* last_id, float* depth, const float* bg,
+                                      void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (!tile_off || !img || !T_final || !last_id) return invalid("null pointer");
   if (((uintptr_t)screen & 15) != 0) return invalid("screen must be 16-byte aligned");
@@ -821,10 +911,10 @@ extern "C" ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, 
   cudaStream_t st = as_stream(stream);
   if (depth || bg) {
     k_raster_fwd_masked<true><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, img, T_final,
-                                                                         last_id, depth, bg);
+                                                                         last_id, depth, bg, tile_order);
   } else {
     k_raster_fwd_masked<false><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, img, T_final,
-                                                                          last_id, nullptr, nullptr);
+                                                                          last_id, nullptr, nullptr, tile_order);
   }
   return cuda_status(cudaGetLastError(), "rasterize fwd");
 }
@@ -845,9 +935,10 @@ extern "C" ss_status ss_rasterize_fwd_counts(const ss_dims* dims, const float* s
 }
 
 extern "C" ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, const uint32_t* vals,
-                                      const int64_t* tile_off, const float* T_final, const int32_t* last_id,
-                                      const float* v_img, const float* v_T, const float* v_depth,
-                                      const float* bg, float* v_screen, int64_t nnz, void* stream) {
+                                      const int64_t* tile_off, const uint32_t* tile_order, const float* T_final,
+                                      const int32_t* last_id, const float* v_img, const float* v_T,
+                                      const float* v_depth, const float* bg, float* v_screen, int64_t nnz,
+                                      void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (nnz < 0) return invalid("nnz < 0");
   if (!tile_off || !T_final || !last_id || !v_img || (nnz > 0 && !v_screen)) return invalid("null pointer");
@@ -860,10 +951,11 @@ extern "C" ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, 
   }
   if (v_depth || bg) {
     k_raster_bwd<true><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, T_final, last_id, v_img,
-                                                                  v_T, v_depth, bg, v_screen);
+                                                                  v_T, v_depth, bg, tile_order, v_screen);
   } else {
     k_raster_bwd<false><<<(unsigned)g.n_tiles, kRThreads, 0, st>>>(g, screen, vals, tile_off, T_final, last_id,
-                                                                   v_img, v_T, nullptr, nullptr, v_screen);
+                                                                   v_img, v_T, nullptr, nullptr, tile_order,
+                                                                   v_screen);
   }
   return cuda_status(cudaGetLastError(), "rasterize bwd");
 }

@@ -22,13 +22,13 @@ LIB_PATH = os.path.join(_HERE, "libss.so")
 
 SS_OK, SS_ERR_INVALID_ARG, SS_ERR_CAPACITY, SS_ERR_OVERFLOW, SS_ERR_CUDA, SS_ERR_DEVICE_CHECK = range(6)
 SIZE_MASK_WORDS, SIZE_MASK_BLOCKS, SIZE_TILES_X, SIZE_TILES_Y, SIZE_N_TILES, SIZE_N_PAD = range(6)
-WS_PROJECT, WS_INTERSECT, WS_SORT = range(3)
+WS_PROJECT, WS_INTERSECT, WS_SORT, WS_TILE_ORDER = range(4)
 ROW = 12
 PMASK_BLOCK = 128
 TILE = 16
 
 EXPORTS = ("ss_size", "ss_workspace_bytes", "ss_status_string", "ss_last_error", "ss_project_packed",
-           "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc", "ss_rasterize_fwd",
+           "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc", "ss_tile_order", "ss_rasterize_fwd",
            "ss_rasterize_fwd_counts",
            "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam")
 
@@ -80,14 +80,15 @@ def lib() -> ct.CDLL:
         L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
         L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, P, sz, P, ct.POINTER(i32), P]
         L.ss_sort_isects_noalloc.argtypes = [D, P, P, P, P, i64, P, ct.POINTER(i32), P]
-        L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P]
+        L.ss_tile_order.argtypes = [D, P, P, P, sz, P]
+        L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P]
         L.ss_rasterize_fwd_counts.argtypes = [D, P, P, P, P, P, P, P, P]
-        L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, i64, P]
+        L.ss_rasterize_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, i64, P]
         L.ss_project_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.ss_project_bwd_adam.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, ct.POINTER(ss_adam_state),
                                           ct.POINTER(ss_adam), P]
         for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc",
-                  "ss_rasterize_fwd",
+                  "ss_tile_order", "ss_rasterize_fwd",
                   "ss_rasterize_fwd_counts", "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam"):
             getattr(L, f).restype = i32
         _lib = L
@@ -171,9 +172,16 @@ def ss_sort_isects_noalloc(d, keys_a, vals_a, keys_b, vals_b, n, tile_off, strea
     return bool(in_b.value)
 
 
-def ss_rasterize_fwd(d, screen, vals, tile_off, img, T_final, last_id, depth=None, bg=None, stream=None):
-    _check(lib().ss_rasterize_fwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(img), _p(T_final),
-                                  _p(last_id), _p(depth), _p(bg), _stream(stream)), "ss_rasterize_fwd")
+def ss_tile_order(d, tile_off, tile_order, temp, stream=None):
+    _check(lib().ss_tile_order(ct.byref(d), _p(tile_off), _p(tile_order), _p(temp),
+                               0 if temp is None else temp.numel() * temp.element_size(), _stream(stream)),
+           "ss_tile_order")
+
+
+def ss_rasterize_fwd(d, screen, vals, tile_off, img, T_final, last_id, depth=None, bg=None, stream=None,
+                     tile_order=None):
+    _check(lib().ss_rasterize_fwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(tile_order), _p(img),
+                                  _p(T_final), _p(last_id), _p(depth), _p(bg), _stream(stream)), "ss_rasterize_fwd")
 
 
 def ss_rasterize_fwd_counts(d, screen, vals, tile_off, img, T_final, last_id, counts, stream=None):
@@ -191,9 +199,10 @@ def raster_work(d, step) -> dict:
 
 
 def ss_rasterize_bwd(d, screen, vals, tile_off, T_final, last_id, v_img, v_T, v_screen, nnz, stream=None,
-                     v_depth=None, bg=None):
-    _check(lib().ss_rasterize_bwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(T_final), _p(last_id),
-                                  _p(v_img), _p(v_T), _p(v_depth), _p(bg), _p(v_screen), int(nnz), _stream(stream)),
+                     v_depth=None, bg=None, tile_order=None):
+    _check(lib().ss_rasterize_bwd(ct.byref(d), _p(screen), _p(vals), _p(tile_off), _p(tile_order), _p(T_final),
+                                  _p(last_id), _p(v_img), _p(v_T), _p(v_depth), _p(bg), _p(v_screen), int(nnz),
+                                  _stream(stream)),
            "ss_rasterize_bwd")
 
 
@@ -242,7 +251,8 @@ class AdamTrainer:
         s = self.step_obj
         img = s.forward(self.cams, self.means, self.quats, self.scales, self.opacities, self.sh, stream)
         v_img = v_img_fn(img)
-        ss_rasterize_bwd(s.d, s.screen, s.vals, s.tile_off, s.T, s.last, v_img, None, s.v_screen, s.nnz, stream)
+        ss_rasterize_bwd(s.d, s.screen, s.vals, s.tile_off, s.T, s.last, v_img, None, s.v_screen, s.nnz, stream,
+                         tile_order=s.tile_order)
         self.hp.step += 1
         ss_project_bwd_adam(s.d, self.cams, self.means, self.quats, self.log_scales, self.scales,
                             self.logit_opacities, self.opacities, self.sh, s.mask, s.block_off, s.v_screen,
@@ -257,8 +267,8 @@ def _u32(n, dev):
 class PackedStep:
     """One forward+backward step over fixed dims, buffers owned by torch.
 
-    forward() runs ss_project_packed, ss_intersect_tiles, ss_sort_isects and
-    ss_rasterize_fwd; backward(v_img, v_T=None) runs ss_rasterize_bwd and
+    forward() runs ss_project_packed, ss_intersect_tiles, ss_sort_isects,
+    ss_tile_order and ss_rasterize_fwd; backward(v_img, v_T=None) runs ss_rasterize_bwd and
     ss_project_bwd.  forward(..., bg=, depth=True) also blends a background
     colour per camera and renders the expected depth (self.depth);
     backward(..., v_depth=) then takes its gradient.  Intermediate buffers are
@@ -280,6 +290,8 @@ class PackedStep:
         self.block_off = torch.empty(self.mask_blocks + 1, dtype=torch.int64, device=dev)
         self.temp_project = torch.empty(workspace_bytes(d, WS_PROJECT), dtype=torch.uint8, device=dev)
         self.tile_off = torch.empty(self.n_tiles + 1, dtype=torch.int64, device=dev)
+        self.tile_order = _u32(self.n_tiles, dev)
+        self.temp_order = torch.empty(workspace_bytes(d, WS_TILE_ORDER), dtype=torch.uint8, device=dev)
         self.img = torch.empty((C, d.H, d.W, 3), dtype=torch.float32, device=dev)
         self.T = torch.empty((C, d.H, d.W), dtype=torch.float32, device=dev)
         self.last = torch.empty((C, d.H, d.W), dtype=torch.int32, device=dev)
@@ -352,17 +364,18 @@ class PackedStep:
                                           self.tile_off, stream)
         self.keys = self.keys_b if self.result_in_b else self.keys_a
         self.vals = self.vals_b if self.result_in_b else self.vals_a
+        ss_tile_order(d, self.tile_off, self.tile_order, self.temp_order, stream)
         if depth and getattr(self, "depth", None) is None:
             self.depth = torch.empty((d.C, d.H, d.W), dtype=torch.float32, device=self.dev)
         ss_rasterize_fwd(d, self.screen, self.vals, self.tile_off, self.img, self.T, self.last,
-                         self.depth if depth else None, bg, stream)
+                         self.depth if depth else None, bg, stream, tile_order=self.tile_order)
         return self.img
 
     def backward(self, v_img, v_T=None, stream=None, v_depth=None):
         cams, means, quats, scales, opacities, sh = self.inputs
         d = self.d
         ss_rasterize_bwd(d, self.screen, self.vals, self.tile_off, self.T, self.last, v_img, v_T, self.v_screen,
-                         self.nnz, stream, v_depth=v_depth, bg=self.bg)
+                         self.nnz, stream, v_depth=v_depth, bg=self.bg, tile_order=self.tile_order)
         ss_project_bwd(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_off, self.v_screen,
                        self.v_means, self.v_quats, self.v_scales, self.v_opacities, self.v_sh, stream)
         return dict(v_means=self.v_means, v_quats=self.v_quats, v_scales=self.v_scales,
@@ -396,15 +409,16 @@ def sort_launches(d: ss_dims, n_isects: int) -> int:
 def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
     """Kernels libss launches in one forward+backward step (memsets excluded):
     projection 5 (pass 1, three scan kernels, pass 2), intersection 5 (three
-    scan kernels, chunk first rows, write), the sort (sort_launches),
-    rasterizer 1 + 1, projection backward 1."""
+    scan kernels, chunk first rows, write), the sort (sort_launches), tile
+    order 3 (histogram, scan, scatter), rasterizer 1 + 1, projection
+    backward 1."""
     if d.N == 0:
         return 0
     n = 5
     if nnz > 0:
         n += 5 if n_isects > 0 else 3
     n += sort_launches(d, n_isects)
-    return n + 3
+    return n + 3 + 3
 
 
 class HostPipeline:

@@ -7,6 +7,7 @@
  *                       compaction into screen rows and 16-bit AABBs)
  *   ss_intersect_tiles  tile intersections with an exact 64-bit count
  *   ss_sort_isects      radix sort of (tile_id << 32 | depth) keys + tile ranges
+ *   ss_tile_order       tiles by decreasing entry count (rasterizer scheduling)
  *   ss_rasterize_fwd    16x16-tile front-to-back alpha compositing
  *   ss_rasterize_bwd    per-pixel reverse replay -> screen-space gradients
  *   ss_project_bwd      screen-space gradients -> means, quats, scales,
@@ -97,10 +98,12 @@ int64_t ss_size(const ss_dims* dims, int what);
 
 /* Scratch bytes needed by a call: which = SS_WS_PROJECT (count ignored),
  * SS_WS_INTERSECT (count = nnz; includes 8 MiB for the write pass's per-chunk
- * row index), SS_WS_SORT (count = number of keys). */
+ * row index), SS_WS_SORT (count = number of keys), SS_WS_TILE_ORDER (count
+ * ignored). */
 #define SS_WS_PROJECT 0
 #define SS_WS_INTERSECT 1
 #define SS_WS_SORT 2
+#define SS_WS_TILE_ORDER 3
 size_t ss_workspace_bytes(const ss_dims* dims, int which, int64_t count);
 
 const char* ss_status_string(ss_status status);
@@ -218,6 +221,19 @@ ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_a, uint32_t
                                  void* stream);
 
 /*
+ * Scheduling order of the rasterizers' tiles: a permutation of [0, n_tiles)
+ * into tile_order[n_tiles] (device uint32), tiles with more entries first
+ * (tile_off[t+1] - tile_off[t], binned four bins per power of two; empty tiles
+ * last; the order inside a bin is unspecified).  The rasterizers run one CTA
+ * per tile and the block scheduler starts CTAs in index order, so a heavy
+ * tile late in index order would run on alone at the end; longest first
+ * keeps every SM busy until the work runs out.  temp: ss_workspace_bytes
+ * (SS_WS_TILE_ORDER) bytes.
+ */
+ss_status ss_tile_order(const ss_dims* dims, const int64_t* tile_off, uint32_t* tile_order, void* temp,
+                        size_t temp_bytes, void* stream);
+
+/*
  * Forward rasterizer ("Spirula Studio backward pass", section 4: the forward
  * keeps tile offsets, the intersection list, each pixel's last Gaussian and
  * its transmittance for the backward pass).  One CTA per 16x16 tile, front to
@@ -233,9 +249,13 @@ ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_a, uint32_t
  *          with d_i the row's camera depth (not normalised by 1 - T_final);
  *   bg     [C][3] device float, a background colour per camera; img becomes
  *          C + T_final * bg.
+ * tile_order (may be NULL: tile index order) is the order the CTAs take the
+ * tiles in, as written by ss_tile_order; it changes only the scheduling (the
+ * outputs are the same).  An entry >= n_tiles is skipped.
  */
 ss_status ss_rasterize_fwd(const ss_dims* dims, const float* screen, const uint32_t* vals, const int64_t* tile_off,
-                           float* img, float* T_final, int32_t* last_id, float* depth, const float* bg, void* stream);
+                           const uint32_t* tile_order, float* img, float* T_final, int32_t* last_id, float* depth,
+                           const float* bg, void* stream);
 
 /*
  * Measurement helper, not part of the step: ss_rasterize_fwd plus exact work
@@ -257,11 +277,13 @@ ss_status ss_rasterize_fwd_counts(const ss_dims* dims, const float* screen, cons
  * v_screen[nnz][12], which the call zeroes first.  v_depth ([C][H][W], may be
  * NULL) is the gradient of the expected depth of ss_rasterize_fwd and fills
  * the rows' depth gradient (column 9); bg ([C][3], may be NULL) must be the
- * background the forward blended.
+ * background the forward blended.  tile_order as for ss_rasterize_fwd (the
+ * rows' float sums are then added in another order: equal up to rounding).
  */
 ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, const uint32_t* vals, const int64_t* tile_off,
-                           const float* T_final, const int32_t* last_id, const float* v_img, const float* v_T,
-                           const float* v_depth, const float* bg, float* v_screen, int64_t nnz, void* stream);
+                           const uint32_t* tile_order, const float* T_final, const int32_t* last_id,
+                           const float* v_img, const float* v_T, const float* v_depth, const float* bg,
+                           float* v_screen, int64_t nnz, void* stream);
 
 /*
  * Projection backward ("Spirula Studio backward pass", section 5): for each

@@ -141,6 +141,42 @@ def test_many_cameras_ragged():
     full_parity(scenes.random_tiny(40, N=517, W=45, H=23, C=33, sh_degree=2))
 
 
+def test_non_rigid_viewmat_and_edge_gaussians():
+    # view matrices whose 3x3 part is scaled and sheared (rows of unequal norm,
+    # row 0 not orthogonal to row 2) and Gaussians spread across and past the
+    # image edges: the projection's conservative pre-test must keep every pair
+    # the exact test accepts, so the mask stays bit-exact
+    sc = scenes.random_tiny(42, N=900, W=53, H=41, C=3, sh_degree=1)
+    rng = np.random.default_rng(42)
+    sc.means = rng.uniform(-2.2, 2.2, (sc.N, 3)).astype(np.float32)
+    cams = sc.cams.copy()
+    for c in range(sc.C):
+        R = cams[c, :12].reshape(3, 4)[:, :3].astype(np.float64)
+        R2 = R.copy()
+        R2[0] = 1.25 * R[0] + 0.1 * R[2]
+        R2[1] = 0.8 * R[1] - 0.07 * R[2]
+        R2[2] = 1.1 * R[2]
+        m = cams[c, :12].reshape(3, 4).copy()
+        m[:, :3] = R2
+        cams[c, :12] = m.reshape(-1)
+    sc.cams = cams.astype(np.float32)
+    o = orc.step(sc, precision=0, nthreads=ORACLE_THREADS)
+    assert 0 < o["proj"]["nnz"] < sc.C * sc.N
+    step = run_gpu(sc, o["v_img"])
+    check_forward(sc, o, step)
+    check_unsorted(sc, o, step)
+    vs = step.v_screen[: o["proj"]["nnz"]].cpu().numpy()
+    grad_close("v_screen", vs[:, :9], o["v_screen"][:, :9])
+    # Parameter gradients: a few Gaussians here sum camera terms that cancel
+    # (v_means[520, 2] = 0.34 from terms of size ~3), where the float oracle
+    # itself is 2e-4 of the largest gradient away from the fp64 oracle; so
+    # the bound is relative to each gradient's scale.
+    for k, ref in o["grads"].items():
+        gpu = np.asarray(getattr(step, k).cpu().numpy(), np.float64)
+        err = np.abs(gpu - np.asarray(ref, np.float64))
+        assert err.max() <= 1e-3 * max(float(np.abs(ref).max()), 1e-30), (k, float(err.max()))
+
+
 def test_opacity_above_one():
     # opacities in (0.5, 1.6): entries with o > 1 take no skip threshold and no
     # culling (every pixel evaluates them), the alpha clamp at 0.99 is hit

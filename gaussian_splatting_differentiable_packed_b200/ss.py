@@ -411,9 +411,10 @@ def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
     projection 5 (pass 1, three scan kernels, pass 2), intersection 5 (three
     scan kernels, chunk first rows, write), the sort (sort_launches), tile
     order 3 (histogram, scan, scatter), rasterizer 1 + 1, projection
-    backward 1."""
+    backward 1.  With no Gaussians only the tile order and the two
+    rasterizers launch (they still write the empty images)."""
     if d.N == 0:
-        return 0
+        return 3 + 2
     n = 5
     if nnz > 0:
         n += 5 if n_isects > 0 else 3

@@ -78,6 +78,22 @@ __host__ __device__ constexpr int sh_stride() {
   return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
 }
 
+// Gaussian gi and coefficient q of word u (0..3) of the SH block's 16-byte
+// vector v (word f = 4v + u: gi = f / K3, q = f mod K3).  When K3 is a
+// multiple of 4 no vector straddles two Gaussians, so the division is taken
+// once per vector rather than once per word.
+template <int K3>
+__device__ __forceinline__ void sh_word(int v, int u, int& gi, int& q) {
+  if constexpr (K3 % 4 == 0) {
+    gi = v / (K3 / 4);
+    q = 4 * (v - gi * (K3 / 4)) + u;
+  } else {
+    const int f = 4 * v + u;
+    gi = f / K3;
+    q = f - gi * K3;
+  }
+}
+
 // Fused optimizer step (the pages' "fused projection backward + optimizer":
 // the gradient sums never leave registers / shared memory).  Adam with bias
 // correction on the raw parameters: means, quaternions, log-scales,
@@ -175,7 +191,8 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
           const float e[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int f = 4 * v + u, gi = f / K3, q = f - gi * K3;
+            int gi, q;
+            sh_word<K3>(v, u, gi, q);
             sh_s[gi * KP + q] = e[u];
             gsh_s[gi * KP + q] = 0.0f;
           }
@@ -457,7 +474,8 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
           float me[4] = {mb[r].x, mb[r].y, mb[r].z, mb[r].w}, ve[4] = {vb[r].x, vb[r].y, vb[r].z, vb[r].w}, pe[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int f = 4 * vv + u, gi = f / K3, q = f - gi * K3;
+            int gi, q;
+            sh_word<K3>(vv, u, gi, q);
             pe[u] = adam_update(sh_s[gi * KP + q], gsh_s[gi * KP + q], me[u], ve[u],
                                 q < 3 ? adam.lr_sh_dc : adam.lr_sh_rest, adam);
           }
@@ -486,7 +504,8 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
       float e[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int f = 4 * v + u, gi = f / K3, q = f - gi * K3;
+        int gi, q;
+        sh_word<K3>(v, u, gi, q);
         e[u] = gsh_s[gi * KP + q];
       }
       reinterpret_cast<float4*>(dst)[v] = make_float4(e[0], e[1], e[2], e[3]);

@@ -137,6 +137,21 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     prefetch_l2(scales + 3 * m0, (uint32_t)(mc * 12));
     prefetch_l2(opacities + m0, (uint32_t)(mc * 4));
   }
+  // A chunk's cameras, first rows and each warp's mask word per camera.  The
+  // first chunk is loaded before the parameters and the SH block so that its
+  // loads are in flight together with theirs.
+  auto load_chunk = [&](int c0) {
+    const int nc = min(kCamChunk, g.C - c0);
+    if (threadIdx.x < nc) {
+      scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
+      s_row0[threadIdx.x] = block_off[(int64_t)(c0 + threadIdx.x) * g.blocks_per_cam + blk];
+    }
+    if (threadIdx.x < nc * kWarps) {
+      const int64_t c = c0 + threadIdx.x / kWarps;
+      s_word[threadIdx.x] = mask[(c * g.n_pad + blk * kBlock) / 32 + threadIdx.x % kWarps];
+    }
+  };
+  load_chunk(0);
   if (n < g.N) {
     s_g[threadIdx.x] = load_gauss(means, quats, scales, n);
     s_o[threadIdx.x] = opacities[n];
@@ -209,14 +224,9 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
     const int nc = min(kCamChunk, g.C - c0);
     const int ns = nc * kWarps;
-    __syncthreads();
-    if (threadIdx.x < nc) {
-      scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
-      s_row0[threadIdx.x] = block_off[(int64_t)(c0 + threadIdx.x) * g.blocks_per_cam + blk];
-    }
-    if (threadIdx.x < ns) {
-      const int64_t c = c0 + threadIdx.x / kWarps;
-      s_word[threadIdx.x] = mask[(c * g.n_pad + blk * kBlock) / 32 + threadIdx.x % kWarps];
+    if (c0 > 0) {  // the first chunk was loaded before the parameters
+      __syncthreads();
+      load_chunk(c0);
     }
     __syncthreads();
     if (warp == 0) {

@@ -170,24 +170,6 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     prefetch_l2(adam.v_scales + 3 * n0, (uint32_t)(cnt * 12));
     prefetch_l2(adam.log_scales + 3 * n0, (uint32_t)(cnt * 12));
   }
-  // The cameras of a chunk, each warp's mask word per camera and the warp's
-  // first row per camera (block offset plus the popcounts of the earlier
-  // warps' words).  The first chunk is staged before the SH block so that its
-  // loads are in flight together with the SH loads.
-  auto stage_chunk = [&](int c0) {
-    const int nc = min(kCamChunkB, g.C - c0);
-    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
-    if (threadIdx.x < nc * kWarps) {
-      const int cc = threadIdx.x / kWarps, w = threadIdx.x % kWarps;
-      const int64_t c = c0 + cc;
-      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
-      int64_t row = block_off[c * g.blocks_per_cam + blk];
-      for (int w2 = 0; w2 < w; ++w2) row += __popc(mask[wbase + w2]);
-      s_word[cc][w] = mask[wbase + w];
-      s_row0[cc][w] = row;
-    }
-  };
-  stage_chunk(0);
   // coalesced staging of the CTA's contiguous SH block: full blocks with all
   // 16-byte loads in flight at once (the block starts 16-byte aligned: 128*K3
   // floats per block), the ragged last block word by word
@@ -236,9 +218,17 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   double gS[6] = {0., 0., 0., 0., 0., 0.};  // dL/dSigma, full-matrix convention (00 01 02 11 12 22)
   for (int c0 = 0; c0 < g.C; c0 += kCamChunkB) {
     const int nc = min(kCamChunkB, g.C - c0);
-    if (c0 > 0) {  // the first chunk's cameras were staged before the SH block
-      __syncthreads();
-      stage_chunk(c0);
+    __syncthreads();
+    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
+    if (threadIdx.x < nc * kWarps) {
+      // each warp's mask word and first row, per camera of the chunk
+      const int cc = threadIdx.x / kWarps, w = threadIdx.x % kWarps;
+      const int64_t c = c0 + cc;
+      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
+      int64_t row = block_off[c * g.blocks_per_cam + blk];
+      for (int w2 = 0; w2 < w; ++w2) row += __popc(mask[wbase + w2]);
+      s_word[cc][w] = mask[wbase + w];
+      s_row0[cc][w] = row;
     }
     __syncthreads();
     if (!valid) continue;

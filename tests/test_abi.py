@@ -40,8 +40,23 @@ def test_sizes_match_layout(L):
     assert ss.size(d, ss.SIZE_MASK_BLOCKS) == 5 * n_pad // 128
     assert ss.size(d, ss.SIZE_TILES_X) == 100 and ss.size(d, ss.SIZE_TILES_Y) == 67
     assert ss.size(d, ss.SIZE_N_TILES) == 5 * 100 * 67
-    for which, count in ((ss.WS_PROJECT, 0), (ss.WS_INTERSECT, 15_000_000), (ss.WS_SORT, 30_000_000)):
+    for which, count in ((ss.WS_PROJECT, 0), (ss.WS_INTERSECT, 15_000_000), (ss.WS_SORT, 30_000_000),
+                         (ss.WS_TILE_ORDER, 0)):
         assert ss.workspace_bytes(d, which, count) > 0
+
+
+def test_tile_order_rejects_bad_arguments_on_host(L):
+    """ss_tile_order checks its pointers and scratch size before any device
+    work (the fake pointers are never dereferenced)."""
+    d = ss.make_dims(1, 64, 64, 0, 10)
+    fake = ct.c_void_p(256)
+    need = ss.workspace_bytes(d, ss.WS_TILE_ORDER, 0)
+    assert L.ss_tile_order(ct.byref(d), None, fake, fake, need, None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_tile_order(ct.byref(d), fake, None, fake, need, None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_tile_order(ct.byref(d), fake, fake, fake, need - 1, None) == ss.SS_ERR_INVALID_ARG
+    assert b"temp" in L.ss_last_error()
+    bad = ss.make_dims(1, 0, 64, 0, 10)
+    assert L.ss_tile_order(ct.byref(bad), fake, fake, fake, need, None) == ss.SS_ERR_INVALID_ARG
 
 
 def test_oracle_and_library_agree_on_geometry(L):

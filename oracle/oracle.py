@@ -11,6 +11,8 @@ Every function restates one step of the packed 3DGS step in plain serial form
   sort         std::stable_sort by key
   tile_ranges  per-tile [start, end) by counting
   rasterize_fwd / rasterize_bwd / project_bwd  one pixel / one row at a time
+  raw_gradients, adam_step                      the fused optimizer step (numpy, fp64)
+  gq_quantise, gq_decode, gq_accumulate         block-quantised gradient accumulation (numpy)
 """
 from __future__ import annotations
 
@@ -396,3 +398,64 @@ def adam_step(params: dict, grads: dict, m: dict, v: dict, lr: dict, beta1: floa
         P[k] = np.asarray(params[k], np.float64) - rate * step
         M[k], V[k] = m1, v1
     return P, M, V
+
+
+# ---------------------------------------------------------------------------- block-quantised gradient accumulation
+# "Spirula Studio backward pass", section 6, technique 1 (grad-quant): each
+# attribute's gradient accumulator is kept as 16-bit codes in blocks of 256
+# Gaussians; for every sub-batch the projection backward decodes the
+# accumulator, adds the sub-batch's gradient and quantises again.  The page
+# names the block size and the code width only.  Readings: one scale per
+# (attribute, block) = the block's largest magnitude / 32767, codes =
+# round-half-even(x / scale) (so the largest element maps to +-32767 and no
+# clamp is ever needed), an all-zero block has scale 0 and codes 0; the six
+# attributes are the page's gradient outputs (means, quaternions, scales,
+# opacities, DC colour, higher SH coefficients).
+GQ_BLOCK = 256
+GQ_MAX = 32767
+
+
+def gq_attributes(grads: dict) -> dict:
+    """The six accumulated attributes, [N, width] each, from the gradient
+    dict of project_bwd (v_sh split into its DC and higher coefficients)."""
+    N = np.asarray(grads["v_means"]).shape[0]
+    sh = np.asarray(grads["v_sh"], np.float64)
+    return dict(means=np.asarray(grads["v_means"], np.float64).reshape(N, -1),
+                quats=np.asarray(grads["v_quats"], np.float64).reshape(N, -1),
+                scales=np.asarray(grads["v_scales"], np.float64).reshape(N, -1),
+                opacities=np.asarray(grads["v_opacities"], np.float64).reshape(N, 1),
+                sh_dc=sh[:, :1, :].reshape(N, -1), sh_rest=sh[:, 1:, :].reshape(N, -1))
+
+
+def gq_quantise(x) -> tuple[np.ndarray, np.ndarray]:
+    """Codes [N, w] (int16) and per-block scales [ceil(N/256)] of x [N, w]."""
+    x = np.asarray(x, np.float64)
+    N = x.shape[0]
+    nb = (N + GQ_BLOCK - 1) // GQ_BLOCK
+    codes = np.zeros(x.shape, np.int16)
+    scales = np.zeros(nb, np.float64)
+    for b in range(nb):
+        blk = x[b * GQ_BLOCK:(b + 1) * GQ_BLOCK]
+        m = float(np.abs(blk).max()) if blk.size else 0.0
+        if m > 0.0:
+            scales[b] = m / GQ_MAX
+            codes[b * GQ_BLOCK:(b + 1) * GQ_BLOCK] = np.rint(blk / scales[b]).astype(np.int16)
+    return codes, scales
+
+
+def gq_decode(codes, scales) -> np.ndarray:
+    """Values [N, w] of an accumulator: code times its block's scale."""
+    codes = np.asarray(codes)
+    N = codes.shape[0]
+    per_row = np.repeat(np.asarray(scales, np.float64), GQ_BLOCK)[:N]
+    return codes.astype(np.float64) * per_row.reshape((N,) + (1,) * (codes.ndim - 1))
+
+
+def gq_accumulate(acc: dict | None, grads: dict) -> dict:
+    """One sub-batch: decode the accumulator (None: start from zero), add the
+    sub-batch's gradients, quantise again.  Returns {attribute: (codes, scales)}."""
+    out = {}
+    for name, g in gq_attributes(grads).items():
+        x = g if acc is None else gq_decode(*acc[name]) + g
+        out[name] = gq_quantise(x)
+    return out

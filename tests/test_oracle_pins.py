@@ -21,7 +21,12 @@ in the oracle (a dropped term, a wrong sign or index, a transposed operand):
                closed form and, for Gaussians at one camera depth z0, the
                telescoped depth z0 * (1 - T);
 * backward:    central finite differences of the fp64 instantiation, with and
-               without the depth output and a background colour.
+               without the depth output and a background colour;
+* grad-quant:  where the full code lands (every 256th Gaussian of a ramp, so
+               the block size and the scale are pinned), the half-step error
+               bound, exact round trips of code multiples, zero blocks, sign
+               symmetry of the rounding, the two-sub-batch error bound and
+               the split of the SH gradient into its DC and higher parts.
 """
 import math
 
@@ -510,3 +515,86 @@ def test_raw_gradients_central_differences():
             checked += 1
             assert abs(vals[0] - an[i]) <= 1e-4 * max(1.0, abs(an[i])), (key, i, vals, an[i])
     assert checked >= 15
+
+
+# ---------------------------------------------------------------------------- block-quantised accumulation
+def test_gq_full_code_at_each_blocks_largest_element():
+    """A ramp x[g] = g + 1 over 700 Gaussians: each block's largest element is
+    its last Gaussian, so the full code 32767 appears exactly at 255, 511 and
+    699 (a wrong block size or one scale for all blocks moves it), and the
+    scale is that element over 32767 (a divisor of 32768 or 65535 leaves no
+    full code)."""
+    x = (np.arange(700, dtype=np.float64) + 1.0).reshape(700, 1)
+    codes, scales = orc.gq_quantise(x)
+    assert codes.dtype == np.int16 and scales.shape == (3,)
+    assert np.flatnonzero(codes[:, 0] == 32767).tolist() == [255, 511, 699]
+    assert np.all(codes > 0)
+    dec = orc.gq_decode(codes, scales)
+    assert np.allclose(dec[[255, 511, 699], 0], [256.0, 512.0, 700.0], rtol=1e-12, atol=0)
+
+
+def test_gq_half_step_error_bound_and_exact_multiples():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((1000, 4)) * np.exp(rng.uniform(-3, 3, (1000, 1)))
+    codes, scales = orc.gq_quantise(x)
+    err = np.abs(orc.gq_decode(codes, scales) - x)
+    step = np.repeat(scales, orc.GQ_BLOCK)[:1000].reshape(1000, 1)
+    assert np.all(err <= 0.5 * step * (1 + 1e-12))
+    # integer multiples of one block's step come back exactly
+    k = rng.integers(-32767, 32768, (256, 3)).astype(np.float64)
+    k[17, 1] = 32767.0
+    y = k * (3.25 / 32767.0)
+    c2, s2 = orc.gq_quantise(y)
+    assert np.array_equal(c2.astype(np.float64), k)
+    assert np.allclose(orc.gq_decode(c2, s2), y, rtol=1e-15, atol=0)
+
+
+def test_gq_zero_block_and_sign_symmetry():
+    x = np.zeros((512, 2))
+    x[300, 1] = -2.5e-7
+    codes, scales = orc.gq_quantise(x)
+    assert scales[0] == 0.0 and np.all(codes[:256] == 0)
+    assert codes[300, 1] == -32767 and np.count_nonzero(codes[256:]) == 1
+    rng = np.random.default_rng(8)
+    y = rng.standard_normal((300, 3))
+    y[5, 0] = 0.5 * (abs(y).max() / 32767.0) * 3  # an exact half step: ties go to even
+    cp, sp = orc.gq_quantise(y)
+    cn, sn = orc.gq_quantise(-y)
+    assert np.array_equal(sp, sn) and np.array_equal(cn, -cp)
+
+
+def test_gq_two_sub_batches_error_bound():
+    """decode(acc2) differs from g1 + g2 by at most half a step of each
+    quantisation; g2 is 50x larger than g1 so that keeping the first scale, or
+    adding codes instead of values, breaks the bound."""
+    rng = np.random.default_rng(9)
+    N, K = 600, 16
+    def grads(scale):
+        return dict(v_means=rng.standard_normal((N, 3)) * scale, v_quats=rng.standard_normal((N, 4)) * scale,
+                    v_scales=rng.standard_normal((N, 3)) * scale, v_opacities=rng.standard_normal(N) * scale,
+                    v_sh=rng.standard_normal((N, K, 3)) * scale)
+    g1, g2 = grads(1e-3), grads(5e-2)
+    acc1 = orc.gq_accumulate(None, g1)
+    acc2 = orc.gq_accumulate(acc1, g2)
+    a1, a2 = orc.gq_attributes(g1), orc.gq_attributes(g2)
+    for name in a1:
+        s1 = np.repeat(acc1[name][1], orc.GQ_BLOCK)[:N].reshape(N, 1)
+        s2 = np.repeat(acc2[name][1], orc.GQ_BLOCK)[:N].reshape(N, 1)
+        err = np.abs(orc.gq_decode(*acc2[name]) - (a1[name] + a2[name]))
+        assert np.all(err <= 0.5 * (s1 + s2) * (1 + 1e-9)), name
+        c, s = orc.gq_quantise(a1[name])
+        assert np.array_equal(acc1[name][0], c) and np.array_equal(acc1[name][1], s)
+
+
+def test_gq_attribute_split():
+    N, K = 3, 9
+    sh = np.zeros((N, K, 3))
+    for k in range(K):
+        for c in range(3):
+            sh[:, k, c] = 100 * k + c
+    a = orc.gq_attributes(dict(v_means=np.zeros((N, 3)), v_quats=np.zeros((N, 4)), v_scales=np.zeros((N, 3)),
+                               v_opacities=np.arange(N, dtype=float), v_sh=sh))
+    assert [a[k].shape[1] for k in ("means", "quats", "scales", "opacities", "sh_dc", "sh_rest")] == [3, 4, 3, 1, 3, 24]
+    assert a["sh_dc"][0].tolist() == [0, 1, 2]
+    assert a["sh_rest"][0, :4].tolist() == [100, 101, 102, 200]
+    assert a["opacities"][:, 0].tolist() == [0, 1, 2]

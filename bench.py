@@ -162,6 +162,11 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work):
     pa = par + 4 + shb
     m["project_bwd_adam"] = dict(bytes=(pa + 16) * N + 2 * pa * N + row * nnz + P / 8 + P / 16
                                  + (pa + 16) * N + 2 * pa * N, instr=nnz * 700.0)
+    # with block-quantised accumulators: parameters and SH read once, the
+    # 16-bit codes read and written (2 bytes per gradient element), scales
+    q = 2 * (11 + 3 * K)
+    m["project_bwd_gq"] = dict(bytes=(par + 4 + shb) * N + row * nnz + P / 8 + P / 16 + 2 * q * N + 2 * 6 * 4 * N / 256,
+                               instr=nnz * 700.0)
     return m
 
 
@@ -241,11 +246,19 @@ def run_ours(args):
                                  torch.log(opac / (1.0 - opac)).contiguous(), sh, eps=1e-8)
         inputs = (cams, means, quats, trainer.scales, trainer.opacities, sh)
 
-    last_stage = "project_bwd_adam" if args.adam else "project_bwd"
+    # optional block-quantised gradient accumulation: every step after the
+    # first decodes, adds and re-quantises (the sub-batch update)
+    gq = ss.GradQuantAccum(d.N, (d.sh_degree + 1) ** 2, dev) if args.grad_quant else None
+    gq_first = [True]
+
+    last_stage = "project_bwd_adam" if args.adam else ("project_bwd_gq" if gq is not None else "project_bwd")
     names = ["project_packed", "intersect_tiles", "sort_isects", "rasterize_fwd", "rasterize_bwd", last_stage]
 
     def backward_rest():
-        if trainer is None:
+        if gq is not None:
+            ss.ss_project_bwd_gq(d, *inputs, step.mask, step.block_off, step.v_screen, gq, first=gq_first[0])
+            gq_first[0] = False
+        elif trainer is None:
             ss.ss_project_bwd(d, *inputs, step.mask, step.block_off, step.v_screen, step.v_means, step.v_quats,
                               step.v_scales, step.v_opacities, step.v_sh)
         else:
@@ -256,7 +269,7 @@ def run_ours(args):
 
     def whole_step():
         step.forward(*inputs, **fkw)
-        if trainer is None:
+        if trainer is None and gq is None:
             step.backward(v_img, **bkw)
         else:
             ss.ss_rasterize_bwd(d, step.screen, step.vals, step.tile_off, step.T, step.last, v_img, None,
@@ -332,7 +345,7 @@ def run_ours(args):
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e and not args.adam:  # the training run keeps its state on the device
+    if not args.no_e2e and not args.adam and not args.grad_quant:  # those keep their state on the device
         host_in = [t.cpu().pin_memory() for t in inputs]
         host_vimg = v_img.cpu().pin_memory()
         host_out = {k: torch.empty(tuple(getattr(step, k).shape), dtype=torch.float32).pin_memory()
@@ -435,7 +448,7 @@ def run_ours(args):
                            sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
                            sort_passes=passes, l2="inputs larger than L2 (3.5 GB parameters), no flush",
                            parallelism=f"replicas x{world}", depth_and_background=bool(args.depth_bg),
-                           fused_adam=bool(args.adam)),
+                           fused_adam=bool(args.adam), grad_quant=bool(args.grad_quant)),
                pairs_per_s=world * d.C * d.N / (ms / 1e3),
                pixel_gaussian_evals_per_s=world * work["evals"] / (stage_ms["rasterize_fwd"] / 1e3),
                step_roofline_frac=round(step_frac, 4), raster_work=out_work, stages=stages, roofline=roof,
@@ -510,6 +523,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--adam", action="store_true",
                     help="train: the projection backward fused with an Adam step updates the parameters in place")
+    ap.add_argument("--grad-quant", action="store_true",
+                    help="accumulate the projection backward's gradients into block-quantised 16-bit accumulators")
     ap.add_argument("--depth-bg", action="store_true",
                     help="also render the expected depth over a background colour and back-propagate a depth gradient")
     args = ap.parse_args()

@@ -14,6 +14,8 @@
 // canonical arithmetic.
 #include <cmath>
 
+#include <cooperative_groups.h>
+
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 
@@ -115,7 +117,65 @@ __device__ __forceinline__ float adam_update(float p, float g, float& m, float& 
   return p - lr * (m * a.ibc1) / (sqrtf(v) * a.ibc2s + a.eps);
 }
 
-template <int DEG, bool ADAM>
+// Block-quantised gradient accumulation ("Spirula Studio backward pass",
+// section 6, technique 1: each attribute's accumulator is kept as 16-bit
+// codes in blocks of 256 Gaussians, and every sub-batch's projection
+// backward decodes it, adds the sub-batch's gradient and quantises again, so
+// no fp32 gradient array exists).  One scale per (attribute, block) = the
+// block's largest magnitude / 32767 and codes = nearest-even(x / scale); an
+// all-zero block has scale 0.  A block of 256 Gaussians is two CTAs, launched
+// as a cluster of two that exchange their maxima through distributed shared
+// memory.  Attributes: means [N][3], quats [N][4], scales [N][3], opacities
+// [N], SH DC [N][3], higher SH [N][K-1][3].
+constexpr int kGqAttr = 6;
+constexpr int64_t kGqBlock = 256;
+constexpr float kGqMax = 32767.0f;
+
+struct GqArgs {
+  int16_t* code[kGqAttr];
+  float* scale;  // [kGqAttr][ceil(N / 256)]
+  int first;     // the accumulators start from zero (their contents are ignored)
+};
+
+__device__ __forceinline__ int16_t gq_code(float x, float s) {
+  if (!(s > 0.0f)) return 0;
+  return (int16_t)__float2int_rn(fminf(fmaxf(x / s, -kGqMax), kGqMax));
+}
+
+// Largest value of v over the CTA for each attribute (a < kGqAttr), into out.
+__device__ __forceinline__ void gq_cta_max(const float (&v)[kGqAttr], float (*wmax)[kBlock / 32], float* out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int a = 0; a < kGqAttr; ++a) {
+    float m = v[a];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) wmax[a][warp] = m;
+  }
+  __syncthreads();
+  if (threadIdx.x < kGqAttr) {
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kBlock / 32; ++w) m = fmaxf(m, wmax[threadIdx.x][w]);
+    out[threadIdx.x] = m;
+  }
+}
+
+// The pair's maxima: both CTAs of the cluster have written theirs to amax;
+// every thread reads the partner's and returns the block's scales.  The
+// second cluster barrier keeps a CTA's maxima alive until its partner has
+// read them.  Every thread of both CTAs calls this exactly once.
+__device__ __forceinline__ void gq_exchange(float* amax, float (&scale)[kGqAttr]) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  cl.sync();
+  const float* other = cl.map_shared_rank(amax, (int)(cl.block_rank() ^ 1u));
+#pragma unroll
+  for (int a = 0; a < kGqAttr; ++a) scale[a] = fmaxf(amax[a], other[a]) / kGqMax;
+  cl.sync();
+}
+
+template <int DEG, bool ADAM, bool GQ>
 __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* __restrict__ cams,
                                                            const float* __restrict__ means,
                                                            const float* __restrict__ quats,
@@ -127,11 +187,13 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
                                                            float* __restrict__ v_means, float* __restrict__ v_quats,
                                                            float* __restrict__ v_scales, float* __restrict__ v_opac,
                                                            float* __restrict__ v_sh, const float* __restrict__ opacities,
-                                                           AdamArgs adam, int64_t ahead) {
+                                                           AdamArgs adam, int64_t ahead, GqArgs gqa) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = 3 * K;
   constexpr int KP = sh_stride<DEG>();
   constexpr int kWarps = kBlock / 32;
+  __shared__ float s_gq_wmax[GQ ? kGqAttr : 1][kWarps];
+  __shared__ float s_gq_amax[GQ ? kGqAttr : 1];
   __shared__ Cam scam[kCamChunkB];
   __shared__ uint32_t s_word[kCamChunkB][kWarps];
   __shared__ int64_t s_row0[kCamChunkB][kWarps];
@@ -144,6 +206,16 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   const int64_t n = n0 + threadIdx.x;
   const bool valid = n < g.N;
   const int cnt = (int)min64(kBlock, g.N - n0);
+  if constexpr (GQ) {
+    if (blk >= g.blocks_per_cam) {
+      // the cluster's second CTA past the last block of Gaussians (an odd
+      // block count): no Gaussians, but it takes part in the pair's exchange
+      if (threadIdx.x < kGqAttr) s_gq_amax[threadIdx.x] = 0.0f;
+      float scale[kGqAttr];
+      gq_exchange(s_gq_amax, scale);
+      return;
+    }
+  }
   // the CTA's gradient rows of camera c are the contiguous rows
   // block_off[c][blk] .. block_off[c][blk + 1]: have L2 fetch them now, the
   // camera loop reads them one pair at a time
@@ -152,7 +224,8 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     const int64_t r1 = block_off[(int64_t)c * g.blocks_per_cam + blk + 1];
     prefetch_l2(v_screen + r0 * kRowF, (uint32_t)((r1 - r0) * kRowF * 4));
   }
-  if (threadIdx.x == 0 && ahead > 0 && blk + ahead < (int64_t)gridDim.x) {
+  // (blocks_per_cam, not the grid: a grad-quant grid may hold one CTA more)
+  if (threadIdx.x == 0 && ahead > 0 && blk + ahead < (GQ ? g.blocks_per_cam : (int64_t)gridDim.x)) {
     // the SH block of the CTA that starts about a wave later, into L2
     const int64_t m0 = (blk + ahead) * kBlock;
     prefetch_l2(sh + m0 * K3, (uint32_t)(min64(kBlock, g.N - m0) * K3 * 4));
@@ -216,6 +289,7 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   const Cov3 S = cov3(qr, s0, s1, s2);
   float gmu[3] = {0.f, 0.f, 0.f}, go = 0.f;
   double gS[6] = {0., 0., 0., 0., 0., 0.};  // dL/dSigma, full-matrix convention (00 01 02 11 12 22)
+  float gx[GQ ? 11 : 1] = {};  // GQ: this Gaussian's means, quats, scales and opacity gradients
   for (int c0 = 0; c0 < g.C; c0 += kCamChunkB) {
     const int nc = min(kCamChunkB, g.C - c0);
     __syncthreads();
@@ -394,7 +468,16 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     const double qi = qr.inv;
     const float gq[4] = {(float)((vw - w * dq) * qi), (float)((vx - x * dq) * qi), (float)((vy - y * dq) * qi),
                          (float)((vz - z * dq) * qi)};
-    if (!ADAM) {
+    if constexpr (GQ) {
+      gx[0] = gmu[0];
+      gx[1] = gmu[1];
+      gx[2] = gmu[2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) gx[3 + i] = gq[i];
+#pragma unroll
+      for (int i = 0; i < 3; ++i) gx[7 + i] = (float)gsc[i];
+      gx[10] = go;
+    } else if (!ADAM) {
       v_means[3 * n] = gmu[0];
       v_means[3 * n + 1] = gmu[1];
       v_means[3 * n + 2] = gmu[2];
@@ -496,6 +579,62 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     }
     return;
   }
+  if constexpr (GQ) {
+    // decode the accumulators, add this sub-batch's gradients, and quantise
+    // the sums with the block's new scales
+    const int64_t qb = blk >> 1;
+    const int64_t nqb = (g.N + kGqBlock - 1) / kGqBlock;
+    constexpr int kW[4] = {3, 4, 3, 1};  // widths of the per-thread attributes
+    constexpr int kOff[4] = {0, 3, 7, 10};
+    float old[kGqAttr];
+#pragma unroll
+    for (int a = 0; a < kGqAttr; ++a) old[a] = gqa.first ? 0.0f : gqa.scale[a * nqb + qb];
+    float vmax[kGqAttr] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (valid) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int i = 0; i < kW[a]; ++i) {
+          float x = gx[kOff[a] + i];
+          if (!gqa.first) x += (float)gqa.code[a][kW[a] * n + i] * old[a];
+          gx[kOff[a] + i] = x;
+          vmax[a] = fmaxf(vmax[a], fabsf(x));
+        }
+    }
+    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+      const int gi = f / K3, q = f - gi * K3;
+      const int64_t m = n0 + gi;
+      float x = gsh_s[gi * KP + q];
+      if (!gqa.first)
+        x += q < 3 ? (float)gqa.code[4][3 * m + q] * old[4] : (float)gqa.code[5][(K3 - 3) * m + (q - 3)] * old[5];
+      gsh_s[gi * KP + q] = x;
+      if (q < 3) vmax[4] = fmaxf(vmax[4], fabsf(x)); else vmax[5] = fmaxf(vmax[5], fabsf(x));
+    }
+    gq_cta_max(vmax, s_gq_wmax, s_gq_amax);
+    float scale[kGqAttr];
+    gq_exchange(s_gq_amax, scale);  // the cluster barrier also orders the gsh_s updates above
+    if (valid) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int i = 0; i < kW[a]; ++i) gqa.code[a][kW[a] * n + i] = gq_code(gx[kOff[a] + i], scale[a]);
+    }
+    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+      const int gi = f / K3, q = f - gi * K3;
+      const int64_t m = n0 + gi;
+      const float x = gsh_s[gi * KP + q];
+      if (q < 3) gqa.code[4][3 * m + q] = gq_code(x, scale[4]);
+      else gqa.code[5][(K3 - 3) * m + (q - 3)] = gq_code(x, scale[5]);
+    }
+    if ((blk & 1) == 0 && threadIdx.x < kGqAttr) {
+      float sc = 0.0f;
+#pragma unroll
+      for (int a = 0; a < kGqAttr; ++a)
+        if (a == (int)threadIdx.x) sc = scale[a];
+      gqa.scale[threadIdx.x * nqb + qb] = sc;
+    }
+    return;
+  }
   // coalesced write-back of the CTA's SH gradient block (16-byte stores for a
   // full block)
   float* dst = v_sh + n0 * K3;
@@ -518,39 +657,57 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   }
 }
 
-template <int DEG, bool ADAM>
-ss_status launch_pbwd(const Geo& g, unsigned grid, cudaStream_t st, const float* cams, const float* means,
-                      const float* quats, const float* scales, const float* sh, const uint32_t* mask,
-                      const int64_t* block_off, const float* v_screen, float* v_means, float* v_quats,
-                      float* v_scales, float* v_opacities, float* v_sh, const float* opacities,
-                      const AdamArgs& adam) {
+template <int DEG, bool ADAM, bool GQ>
+ss_status launch_pbwd(const Geo& g, cudaStream_t st, const float* cams, const float* means, const float* quats,
+                      const float* scales, const float* sh, const uint32_t* mask, const int64_t* block_off,
+                      const float* v_screen, float* v_means, float* v_quats, float* v_scales, float* v_opacities,
+                      float* v_sh, const float* opacities, const AdamArgs& adam, const GqArgs& gqa) {
   const size_t smem = 2 * sizeof(float) * kBlock * sh_stride<DEG>();
-  ss_status s = cuda_status(cudaFuncSetAttribute(k_project_bwd<DEG, ADAM>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+  auto kernel = k_project_bwd<DEG, ADAM, GQ>;
+  ss_status s = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                             "smem attr");
   if (s) return s;
-  const int64_t ahead = wave_blocks(k_project_bwd<DEG, ADAM>, kBlock, smem);
-  k_project_bwd<DEG, ADAM><<<grid, kBlock, smem, st>>>(g, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                                       v_means, v_quats, v_scales, v_opacities, v_sh, opacities,
-                                                       adam, ahead);
-  return cuda_status(cudaGetLastError(), "project bwd");
+  const int64_t ahead = wave_blocks(kernel, kBlock, smem);
+  if constexpr (!GQ) {
+    kernel<<<(unsigned)g.blocks_per_cam, kBlock, smem, st>>>(g, cams, means, quats, scales, sh, mask, block_off,
+                                                              v_screen, v_means, v_quats, v_scales, v_opacities, v_sh,
+                                                              opacities, adam, ahead, gqa);
+    return cuda_status(cudaGetLastError(), "project bwd");
+  } else {
+    // clusters of two CTAs (one quantisation block of 256 Gaussians); an odd
+    // block count gets one more CTA, which holds no Gaussians
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(g.blocks_per_cam + (g.blocks_per_cam & 1)));
+    cfg.blockDim = dim3(kBlock);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kernel, g, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                          v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam, ahead, gqa),
+                       "project bwd (grad-quant)");
+  }
 }
 
-template <bool ADAM>
+template <bool ADAM, bool GQ>
 ss_status dispatch_pbwd(const Geo& g, cudaStream_t st, const float* cams, const float* means, const float* quats,
                         const float* scales, const float* sh, const uint32_t* mask, const int64_t* block_off,
                         const float* v_screen, float* v_means, float* v_quats, float* v_scales, float* v_opacities,
-                        float* v_sh, const float* opacities, const AdamArgs& adam) {
-  const unsigned grid = (unsigned)g.blocks_per_cam;
+                        float* v_sh, const float* opacities, const AdamArgs& adam, const GqArgs& gqa = GqArgs{}) {
   switch (g.deg) {
-    case 0: return launch_pbwd<0, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                        v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
-    case 1: return launch_pbwd<1, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                        v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
-    case 2: return launch_pbwd<2, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                        v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
-    default: return launch_pbwd<3, ADAM>(g, grid, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
-                                         v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam);
+    case 0: return launch_pbwd<0, ADAM, GQ>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                            v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam, gqa);
+    case 1: return launch_pbwd<1, ADAM, GQ>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                            v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam, gqa);
+    case 2: return launch_pbwd<2, ADAM, GQ>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                            v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam, gqa);
+    default: return launch_pbwd<3, ADAM, GQ>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen,
+                                             v_means, v_quats, v_scales, v_opacities, v_sh, opacities, adam, gqa);
   }
 }
 
@@ -572,8 +729,8 @@ extern "C" ss_status ss_project_bwd(const ss_dims* dims, const float* cams, cons
       ((uintptr_t)v_sh & 15))
     return invalid("quats, v_quats, v_screen, sh and v_sh must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
-  return dispatch_pbwd<false>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means, v_quats,
-                              v_scales, v_opacities, v_sh, opacities, AdamArgs{});
+  return dispatch_pbwd<false, false>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
+                                     v_quats, v_scales, v_opacities, v_sh, opacities, AdamArgs{});
 }
 
 extern "C" ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams, float* means, float* quats,
@@ -608,6 +765,33 @@ extern "C" ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams,
   a.ibc1 = (float)(1.0 / (1.0 - std::pow((double)hp->beta1, (double)hp->step)));
   a.ibc2s = (float)(1.0 / std::sqrt(1.0 - std::pow((double)hp->beta2, (double)hp->step)));
   cudaStream_t st = as_stream(stream);
-  return dispatch_pbwd<true>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, nullptr, nullptr,
-                             nullptr, nullptr, nullptr, opacities, a);
+  return dispatch_pbwd<true, false>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, nullptr,
+                                    nullptr, nullptr, nullptr, nullptr, opacities, a);
+}
+
+extern "C" ss_status ss_project_bwd_gq(const ss_dims* dims, const float* cams, const float* means, const float* quats,
+                                       const float* scales, const float* opacities, const float* sh,
+                                       const uint32_t* mask, const int64_t* block_off, const float* v_screen,
+                                       const ss_gq_accum* acc, int first, void* stream) {
+  if (!dims_ok(dims)) return invalid("dims");
+  const Geo g = geometry(*dims);
+  if (g.N == 0) return SS_OK;
+  if (!cams || !means || !quats || !scales || !sh || !mask || !block_off || !v_screen) return invalid("null input");
+  if (!acc || !acc->means || !acc->quats || !acc->scales || !acc->opacities || !acc->sh_dc || !acc->block_scale ||
+      (g.deg > 0 && !acc->sh_rest))
+    return invalid("null accumulator");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15))
+    return invalid("quats, v_screen and sh must be 16-byte aligned");
+  GqArgs q{};
+  q.code[0] = acc->means;
+  q.code[1] = acc->quats;
+  q.code[2] = acc->scales;
+  q.code[3] = acc->opacities;
+  q.code[4] = acc->sh_dc;
+  q.code[5] = acc->sh_rest;
+  q.scale = acc->block_scale;
+  q.first = first ? 1 : 0;
+  cudaStream_t st = as_stream(stream);
+  return dispatch_pbwd<false, true>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, nullptr,
+                                    nullptr, nullptr, nullptr, nullptr, opacities, AdamArgs{}, q);
 }

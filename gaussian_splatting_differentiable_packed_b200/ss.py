@@ -30,7 +30,7 @@ TILE = 16
 EXPORTS = ("ss_size", "ss_workspace_bytes", "ss_status_string", "ss_last_error", "ss_project_packed",
            "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc", "ss_tile_order", "ss_rasterize_fwd",
            "ss_rasterize_fwd_counts",
-           "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam")
+           "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam", "ss_project_bwd_gq")
 
 
 class ss_adam(ct.Structure):
@@ -42,6 +42,11 @@ class ss_adam(ct.Structure):
 class ss_adam_state(ct.Structure):
     _fields_ = [(n, ct.c_void_p) for n in ("m_means", "v_means", "m_quats", "v_quats", "m_scales", "v_scales",
                                            "m_opacities", "v_opacities", "m_sh", "v_sh")]
+
+
+class ss_gq_accum(ct.Structure):
+    _fields_ = [(n, ct.c_void_p) for n in ("means", "quats", "scales", "opacities", "sh_dc", "sh_rest",
+                                           "block_scale")]
 
 
 class ss_dims(ct.Structure):
@@ -87,9 +92,11 @@ def lib() -> ct.CDLL:
         L.ss_project_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
         L.ss_project_bwd_adam.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, ct.POINTER(ss_adam_state),
                                           ct.POINTER(ss_adam), P]
+        L.ss_project_bwd_gq.argtypes = [D, P, P, P, P, P, P, P, P, P, ct.POINTER(ss_gq_accum), i32, P]
         for f in ("ss_project_packed", "ss_intersect_tiles", "ss_sort_isects", "ss_sort_isects_noalloc",
                   "ss_tile_order", "ss_rasterize_fwd",
-                  "ss_rasterize_fwd_counts", "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam"):
+                  "ss_rasterize_fwd_counts", "ss_rasterize_bwd", "ss_project_bwd", "ss_project_bwd_adam",
+                  "ss_project_bwd_gq"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -222,6 +229,48 @@ def ss_project_bwd_adam(d, cams, means, quats, log_scales, scales, logit_opaciti
                                      _p(logit_opacities), _p(opacities), _p(sh), _p(mask), _p(block_off),
                                      _p(v_screen), ct.byref(st), ct.byref(hp), _stream(stream)),
            "ss_project_bwd_adam")
+
+
+GQ_BLOCK = 256
+GQ_ATTRS = ("means", "quats", "scales", "opacities", "sh_dc", "sh_rest")
+
+
+class GradQuantAccum:
+    """Block-quantised gradient accumulators of N Gaussians (ss_project_bwd_gq):
+    int16 codes per attribute and the [6, ceil(N/256)] block scales, on the
+    device.  decoded() gives the accumulated values (code * block scale) for
+    inspection; the step itself never decodes outside the kernel."""
+
+    def __init__(self, N: int, K: int, device="cuda"):
+        self.N, self.K = int(N), int(K)
+        widths = dict(means=3, quats=4, scales=3, opacities=1, sh_dc=3, sh_rest=3 * (self.K - 1))
+        dev = torch.device(device)
+        self.codes = {a: torch.zeros((self.N, max(w, 1)), dtype=torch.int16, device=dev) for a, w in widths.items()}
+        self.widths = widths
+        self.nb = (self.N + GQ_BLOCK - 1) // GQ_BLOCK
+        self.block_scale = torch.zeros((len(GQ_ATTRS), max(self.nb, 1)), dtype=torch.float32, device=dev)
+
+    def struct(self) -> ss_gq_accum:
+        ptr = [_p(self.codes[a]) if self.widths[a] > 0 else None for a in GQ_ATTRS]
+        return ss_gq_accum(*ptr, _p(self.block_scale))
+
+    def decoded(self) -> dict:
+        out = {}
+        for i, a in enumerate(GQ_ATTRS):
+            per_row = self.block_scale[i].repeat_interleave(GQ_BLOCK)[: self.N].double().unsqueeze(1)
+            out[a] = (self.codes[a][:, : self.widths[a]].double() * per_row).cpu().numpy()
+        return out
+
+
+def ss_project_bwd_gq(d, cams, means, quats, scales, opacities, sh, mask, block_off, v_screen,
+                      acc: GradQuantAccum, first: bool, stream=None):
+    """Projection backward that adds its gradients into block-quantised
+    accumulators (first=True starts them from zero)."""
+    st = acc.struct()
+    _check(lib().ss_project_bwd_gq(ct.byref(d), _p(cams), _p(means), _p(quats), _p(scales), _p(opacities), _p(sh),
+                                   _p(mask), _p(block_off), _p(v_screen), ct.byref(st), 1 if first else 0,
+                                   _stream(stream)),
+           "ss_project_bwd_gq")
 
 
 class AdamTrainer:

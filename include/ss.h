@@ -13,6 +13,8 @@
  *   ss_project_bwd      screen-space gradients -> means, quats, scales,
  *                       opacities, SH coefficients
  *   ss_project_bwd_adam the same, fused with an Adam step on the parameters
+ *   ss_project_bwd_gq   the same, accumulating into block-quantised 16-bit
+ *                       gradient accumulators
  *
  * Conventions (all entry points):
  *   - Every array pointer is a DEVICE pointer owned by the caller unless the
@@ -199,6 +201,42 @@ ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams, float* mea
                               float* scales, float* logit_opacities, float* opacities, float* sh,
                               const uint32_t* mask, const int64_t* block_off, const float* v_screen,
                               const ss_adam_state* state, const ss_adam* hp, void* stream);
+
+/*
+ * Projection backward with block-quantised gradient accumulation ("Spirula
+ * Studio backward pass", section 6, technique 1): instead of fp32 gradient
+ * arrays, each attribute's gradient accumulator is held as 16-bit codes in
+ * blocks of 256 Gaussians (index n / 256), one fp32 scale per attribute and
+ * block; the call decodes the accumulator (code * scale), adds this
+ * sub-batch's gradient (the same gradient ss_project_bwd computes for the
+ * cameras of dims) and quantises the sums again: scale = the block's largest
+ * magnitude / 32767, code = nearest-even(x / scale), 0 for an all-zero block.
+ * first != 0 starts from zero (the accumulator's contents are ignored), as
+ * for a step's first sub-batch.  Accumulator layout (device, owned by the
+ * caller, updated in place):
+ *   means [N][3], quats [N][4], scales [N][3], opacities [N], sh_dc [N][3]
+ *   (SH coefficient 0), sh_rest [N][K-1][3] (NULL allowed when K == 1) as
+ *   int16; block_scale [6][ceil(N/256)] float in that attribute order.
+ * 118 B per Gaussian at SH degree 3 against 236 for the fp32 gradients.
+ * quats, v_screen and sh must be 16-byte aligned (SS_ERR_INVALID_ARG
+ * otherwise).  Two CTAs of 128 Gaussians form one block; they run as a
+ * thread-block cluster of two and exchange their maxima through distributed
+ * shared memory.
+ */
+typedef struct ss_gq_accum {
+  int16_t* means;
+  int16_t* quats;
+  int16_t* scales;
+  int16_t* opacities;
+  int16_t* sh_dc;
+  int16_t* sh_rest;
+  float* block_scale;
+} ss_gq_accum;
+
+ss_status ss_project_bwd_gq(const ss_dims* dims, const float* cams, const float* means, const float* quats,
+                            const float* scales, const float* opacities, const float* sh, const uint32_t* mask,
+                            const int64_t* block_off, const float* v_screen, const ss_gq_accum* acc, int first,
+                            void* stream);
 
 /*
  * Allocation-free variant of ss_sort_isects (the pages have no counterpart:

@@ -601,12 +601,51 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
           vmax[a] = fmaxf(vmax[a], fabsf(x));
         }
     }
+    // the block's SH codes: DC [128][3] and higher [128][K3-3] int16, each
+    // contiguous and 16-byte aligned for a full block; decoded into the SH
+    // staging area (the coefficients are not needed after the camera walk)
+    // with every 16-byte load in flight, word by word for the ragged block
+    constexpr int kDcV = kBlock * 3 * 2 / 16;
+    constexpr int kRestV = kBlock * (K3 - 3) * 2 / 16;
+    constexpr int kPerV = (kDcV + kRestV + kBlock - 1) / kBlock;
+    const bool vec = cnt == kBlock;
+    if (!gqa.first && vec) {
+      const int4* dc4 = reinterpret_cast<const int4*>(gqa.code[4] + 3 * n0);
+      const int4* rest4 = reinterpret_cast<const int4*>(gqa.code[5] + (K3 - 3) * n0);
+      int4 buf[kPerV];
+#pragma unroll
+      for (int r = 0; r < kPerV; ++r) {
+        const int v = threadIdx.x + r * kBlock;
+        if (v < kDcV) buf[r] = dc4[v];
+        else if (v < kDcV + kRestV) buf[r] = rest4[v - kDcV];
+      }
+#pragma unroll
+      for (int r = 0; r < kPerV; ++r) {
+        const int v = threadIdx.x + r * kBlock;
+        if (v >= kDcV + kRestV) continue;
+        const uint32_t w[4] = {(uint32_t)buf[r].x, (uint32_t)buf[r].y, (uint32_t)buf[r].z, (uint32_t)buf[r].w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float c = (float)(int16_t)(w[u >> 1] >> (16 * (u & 1)));
+          if (v < kDcV) {
+            const int e = 8 * v + u, gi = e / 3;
+            sh_s[gi * KP + (e - 3 * gi)] = c * old[4];
+          } else {
+            const int e = 8 * (v - kDcV) + u, gi = e / (K3 - 3 > 0 ? K3 - 3 : 1);
+            sh_s[gi * KP + 3 + (e - (K3 - 3) * gi)] = c * old[5];
+          }
+        }
+      }
+      __syncthreads();
+    }
     for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
       const int gi = f / K3, q = f - gi * K3;
       const int64_t m = n0 + gi;
       float x = gsh_s[gi * KP + q];
-      if (!gqa.first)
-        x += q < 3 ? (float)gqa.code[4][3 * m + q] * old[4] : (float)gqa.code[5][(K3 - 3) * m + (q - 3)] * old[5];
+      if (!gqa.first) {
+        if (vec) x += sh_s[gi * KP + q];
+        else x += q < 3 ? (float)gqa.code[4][3 * m + q] * old[4] : (float)gqa.code[5][(K3 - 3) * m + (q - 3)] * old[5];
+      }
       gsh_s[gi * KP + q] = x;
       if (q < 3) vmax[4] = fmaxf(vmax[4], fabsf(x)); else vmax[5] = fmaxf(vmax[5], fabsf(x));
     }
@@ -619,12 +658,35 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
 #pragma unroll
         for (int i = 0; i < kW[a]; ++i) gqa.code[a][kW[a] * n + i] = gq_code(gx[kOff[a] + i], scale[a]);
     }
-    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-      const int gi = f / K3, q = f - gi * K3;
-      const int64_t m = n0 + gi;
-      const float x = gsh_s[gi * KP + q];
-      if (q < 3) gqa.code[4][3 * m + q] = gq_code(x, scale[4]);
-      else gqa.code[5][(K3 - 3) * m + (q - 3)] = gq_code(x, scale[5]);
+    if (vec) {
+      // 16-byte stores of eight codes each, the same vectors as the loads
+      int4* dc4 = reinterpret_cast<int4*>(gqa.code[4] + 3 * n0);
+      int4* rest4 = reinterpret_cast<int4*>(gqa.code[5] + (K3 - 3) * n0);
+      for (int v = threadIdx.x; v < kDcV + kRestV; v += kBlock) {
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          int16_t c;
+          if (v < kDcV) {
+            const int e = 8 * v + u, gi = e / 3;
+            c = gq_code(gsh_s[gi * KP + (e - 3 * gi)], scale[4]);
+          } else {
+            const int e = 8 * (v - kDcV) + u, gi = e / (K3 - 3 > 0 ? K3 - 3 : 1);
+            c = gq_code(gsh_s[gi * KP + 3 + (e - (K3 - 3) * gi)], scale[5]);
+          }
+          w[u >> 1] |= (uint32_t)(uint16_t)c << (16 * (u & 1));
+        }
+        const int4 o = make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
+        if (v < kDcV) dc4[v] = o; else rest4[v - kDcV] = o;
+      }
+    } else {
+      for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+        const int gi = f / K3, q = f - gi * K3;
+        const int64_t m = n0 + gi;
+        const float x = gsh_s[gi * KP + q];
+        if (q < 3) gqa.code[4][3 * m + q] = gq_code(x, scale[4]);
+        else gqa.code[5][(K3 - 3) * m + (q - 3)] = gq_code(x, scale[5]);
+      }
     }
     if ((blk & 1) == 0 && threadIdx.x < kGqAttr) {
       float sc = 0.0f;
@@ -782,6 +844,8 @@ extern "C" ss_status ss_project_bwd_gq(const ss_dims* dims, const float* cams, c
     return invalid("null accumulator");
   if (((uintptr_t)quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15))
     return invalid("quats, v_screen and sh must be 16-byte aligned");
+  if (((uintptr_t)acc->sh_dc & 15) || ((uintptr_t)acc->sh_rest & 15))
+    return invalid("the SH code arrays must be 16-byte aligned");
   GqArgs q{};
   q.code[0] = acc->means;
   q.code[1] = acc->quats;

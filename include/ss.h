@@ -218,8 +218,8 @@ ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams, float* mea
  *   (SH coefficient 0), sh_rest [N][K-1][3] (NULL allowed when K == 1) as
  *   int16; block_scale [6][ceil(N/256)] float in that attribute order.
  * 118 B per Gaussian at SH degree 3 against 236 for the fp32 gradients.
- * quats, v_screen and sh must be 16-byte aligned (SS_ERR_INVALID_ARG
- * otherwise).  Two CTAs of 128 Gaussians form one block; they run as a
+ * quats, v_screen, sh, sh_dc and sh_rest must be 16-byte aligned
+ * (SS_ERR_INVALID_ARG otherwise).  Two CTAs of 128 Gaussians form one block; they run as a
  * thread-block cluster of two and exchange their maxima through distributed
  * shared memory.
  */

@@ -93,6 +93,21 @@ def test_sort_overflow_rejected_before_device_work(L):
     assert L.ss_status_string(st) == b"count overflows 32-bit indices"
 
 
+def test_grad_quant_rejects_bad_arguments_on_host(L):
+    """ss_project_bwd_gq checks its accumulator before any device work (the
+    fake pointers are never dereferenced)."""
+    d = ss.make_dims(1, 64, 64, 3, 1000)
+    f = ct.c_void_p(256)
+    args = [ct.byref(d)] + [f] * 9
+    assert L.ss_project_bwd_gq(*args, None, 1, None) == ss.SS_ERR_INVALID_ARG
+    acc = ss.ss_gq_accum(256, 256, 256, 256, 256, None, 256)  # degree 3 needs the higher-SH codes
+    assert L.ss_project_bwd_gq(*args, ct.byref(acc), 1, None) == ss.SS_ERR_INVALID_ARG
+    assert b"accumulator" in L.ss_last_error()
+    acc = ss.ss_gq_accum(256, 256, 256, 256, 256 + 2, 256, 256)  # DC codes off a 16-byte boundary
+    assert L.ss_project_bwd_gq(*args, ct.byref(acc), 1, None) == ss.SS_ERR_INVALID_ARG
+    assert b"16-byte" in L.ss_last_error()
+
+
 def test_null_and_short_temp_rejected(L):
     d = ss.make_dims(1, 64, 64, 0, 10)
     nnz = ct.c_int64(0)

@@ -462,9 +462,14 @@ def run_ours(args):
 
 
 # ---------------------------------------------------------------------------- CPU oracle
+# Gaussian count of each workload (the sample never exceeds the workload)
+WORKLOAD_N = {1: 2_000, 2: 100_000, 3: 1_000_000, 4: 15_000_000, 5: 13_000_000}
+
+
 def oracle_sample(config: int, n: int):
     from gaussian_splatting_differentiable_packed_b200 import scenes
-    return scenes.make_scene(config, n=n)
+    full = WORKLOAD_N.get(config)
+    return scenes.make_scene(config, n=None if full is not None and n >= full else n)
 
 
 def cpu_baseline(config: int, n_sample: int, repeats: int = 1):

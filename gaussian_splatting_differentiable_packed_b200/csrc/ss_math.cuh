@@ -5,7 +5,7 @@
 // outputs (visibility, AABB16, keys, last_id) are decided by these values.
 //
 // EWA splatting as named on the "Spirula Studio backward pass" page, section 5
-// (projection through intrinsics/extrinsics), with the task's constants: 0.3
+// (projection through intrinsics/extrinsics), with the method's constants: 0.3
 // dilation, 3-sigma radius, alpha clamp 0.99, skip below 1/255, stop below
 // T = 1e-4.
 #pragma once

@@ -1,0 +1,68 @@
+"""Host-side logic of bench.py and the binding that the bench line rests on
+(no GPU needed): the traffic record's guards, the per-step launch count, the
+oracle sample bound and the stage model's bytes."""
+import json
+import os
+
+import pytest
+
+import bench
+from gaussian_splatting_differentiable_packed_b200 import ss
+
+
+def test_traffic_record_guards(tmp_path, monkeypatch):
+    rec = json.load(open(bench.TRAFFIC_FILE))
+    stage = "rasterize_bwd"
+    wl = rec["_workload"]
+    assert bench.recorded_traffic(stage, wl["config"], wl["n"]) == float(rec[stage]["dram_bytes_per_launch"])
+    # another workload: no traffic
+    assert bench.recorded_traffic(stage, 3, None) is None
+    assert bench.recorded_traffic(stage, wl["config"], 3_000_000) is None
+    # sources that differ from the capture's: no traffic
+    bad = dict(rec)
+    bad[stage] = dict(rec[stage], sha256="0" * 64)
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps(bad))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
+    assert bench.recorded_traffic(stage, wl["config"], wl["n"]) is None
+    # a missing stage or file: no traffic
+    assert bench.recorded_traffic("no_such_stage", wl["config"], wl["n"]) is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.recorded_traffic(stage, wl["config"], wl["n"]) is None
+
+
+def test_launches_per_step():
+    """projection 5, intersection 5 (3 without intersections), the sort's
+    histogram, bases, one pass per digit and tile ranges, the tile order 3,
+    rasterizers 2, projection backward 1."""
+    d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)
+    passes = ss.sort_passes(d)
+    assert passes == 6  # 33,500 tiles: 16 tile-id bits, 2 digits over them
+    assert ss.launches_per_step(d, 15_000_000, 33_000_000) == 5 + 5 + (passes + 3) + 3 + 2 + 1
+    assert ss.launches_per_step(d, 15_000_000, 0) == 5 + 3 + 0 + 3 + 2 + 1
+    assert ss.launches_per_step(d, 0, 0) == 5 + 0 + 0 + 3 + 2 + 1
+    assert ss.launches_per_step(ss.make_dims(1, 64, 64, 0, 0), 0, 0) == 3 + 2
+
+
+def test_oracle_sample_never_exceeds_the_workload():
+    assert bench.oracle_sample(1, 300_000).N == 2_000
+    assert bench.oracle_sample(2, 300_000).N == 100_000
+    assert bench.oracle_sample(3, 300_000).N == 300_000
+
+
+def test_stage_model_counts_every_stage():
+    d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)
+    work = dict(evals=1.6e9, exps=1.1e8, comps=9e7, bwd_evals=1.6e9, bwd_exps=1.1e8)
+    m = bench.stage_model(d, 16, 15_000_000, 33_000_000, 6, 33_500, work)
+    for name in ("project_packed", "intersect_tiles", "sort_isects", "rasterize_fwd", "rasterize_bwd", "project_bwd",
+                 "project_bwd_adam", "project_bwd_gq"):
+        assert m[name]["bytes"] > 0, name
+    # the projection backward reads and writes 236 B per Gaussian at SH 3,
+    # plus the screen rows and the mask
+    assert m["project_bwd"]["bytes"] > 2 * 236 * 15_000_000
+    # the 16-bit accumulators are read and written (118 B each way per
+    # Gaussian) where the plain call writes 236 B of fp32 gradients: about
+    # the same traffic, half the memory; the fused Adam moves far more
+    gq, plain = m["project_bwd_gq"]["bytes"], m["project_bwd"]["bytes"]
+    assert abs(gq - plain) < 0.02 * plain
+    assert plain < m["project_bwd_adam"]["bytes"]

@@ -6,9 +6,13 @@ on a non-zero status.  No step of the splatting path runs in Python or on the
 CPU: if libss.so is missing the import of the library fails loudly.
 PyTorch only allocates device memory and provides the stream.
 
-`PackedStep` strings the six calls into one forward+backward step with
-buffers owned by torch (the counts returned by the two synchronising calls
-size the later buffers; capacities grow with headroom when exceeded).
+`PackedStep` strings the calls into one forward+backward step with buffers
+owned by torch (the counts returned by the two synchronising calls size the
+later buffers; capacities grow with headroom when exceeded).  Around it:
+`HostPipeline` (steps over pinned host inputs and gradients, copies
+overlapped with the kernels), `AdamTrainer` (the projection backward fused
+with Adam) and `GradQuantAccum` (16-bit block-quantised gradient
+accumulators for ss_project_bwd_gq).
 """
 from __future__ import annotations
 

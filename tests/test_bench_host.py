@@ -14,16 +14,20 @@ def test_traffic_record_guards(tmp_path, monkeypatch):
     rec = json.load(open(bench.TRAFFIC_FILE))
     stage = "rasterize_bwd"
     wl = rec["_workload"]
+    # a record whose digest matches the sources as they are now is reported
+    good = dict(rec)
+    good[stage] = dict(rec[stage], sha256=bench.source_digest(rec[stage]["sources"]))
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps(good))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
     assert bench.recorded_traffic(stage, wl["config"], wl["n"]) == float(rec[stage]["dram_bytes_per_launch"])
     # another workload: no traffic
     assert bench.recorded_traffic(stage, 3, None) is None
-    assert bench.recorded_traffic(stage, wl["config"], 3_000_000) is None
+    assert bench.recorded_traffic(stage, wl["config"], 3_000_001) is None
     # sources that differ from the capture's: no traffic
     bad = dict(rec)
     bad[stage] = dict(rec[stage], sha256="0" * 64)
-    p = tmp_path / "traffic.json"
     p.write_text(json.dumps(bad))
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
     assert bench.recorded_traffic(stage, wl["config"], wl["n"]) is None
     # a missing stage or file: no traffic
     assert bench.recorded_traffic("no_such_stage", wl["config"], wl["n"]) is None

@@ -6,7 +6,7 @@ rows are bit-identical too), AABB16, n_isects, per-row offsets, keys and
 values before and after the sort, tile ranges, last_id.  Images and final
 transmittance within 1e-5 absolute.  Gradients within 1e-3 relative +
 1e-5 absolute of the oracle's fp64 gradients (atomic order varies), plus a
-scale-aware bound (error / max|reference| <= 1e-3) so that small-valued
+scale-aware bound (error / max|reference| <= 1e-4) so that small-valued
 gradient fields are not passed by the absolute term alone.
 """
 import numpy as np
@@ -38,7 +38,7 @@ def run_gpu(scene, v_img=None, v_T=None, **kw):
     return step
 
 
-def grad_close(name, gpu, ref, rtol=1e-3, atol=1e-5, scale_tol=1e-3):
+def grad_close(name, gpu, ref, rtol=1e-3, atol=1e-5, scale_tol=1e-4):
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     assert gpu.shape == ref.shape, name
@@ -132,8 +132,14 @@ def test_config2_100k():
 
 
 def test_config3_reduced():
-    # config 3's distributions and cameras with 1/10 of the Gaussians
+    # the 1M x 4 workload's distributions and cameras with 1/10 of the Gaussians
     full_parity(scenes.make_scene(3, n=100_000), with_unsorted=False)
+
+
+def test_config3_full_size():
+    # the 1M-Gaussian, 4-camera 1280x720 workload, every output compared whole
+    o, step = full_parity(scenes.make_scene(3), with_unsorted=False)
+    assert o["proj"]["nnz"] > 1_000_000
 
 
 def test_many_cameras_ragged():
@@ -144,8 +150,8 @@ def test_many_cameras_ragged():
 def test_non_rigid_viewmat_and_edge_gaussians():
     # view matrices whose 3x3 part is scaled and sheared (rows of unequal norm,
     # row 0 not orthogonal to row 2) and Gaussians spread across and past the
-    # image edges: the projection's conservative pre-test must keep every pair
-    # the exact test accepts, so the mask stays bit-exact
+    # image edges: the visibility decisions near the edges and with a
+    # non-orthonormal camera rotation must stay bit-exact
     sc = scenes.random_tiny(42, N=900, W=53, H=41, C=3, sh_degree=1)
     rng = np.random.default_rng(42)
     sc.means = rng.uniform(-2.2, 2.2, (sc.N, 3)).astype(np.float32)

@@ -589,6 +589,36 @@ Gates decide_gates(const double* cam20, const orc_dims* d, const double* mu, con
   return gt;
 }
 
+// Order of opacities for the visible cap: the IEEE total order of the fp32
+// value (for the activated opacities in (0, 1) this is the numeric order).
+uint32_t opacity_order_key(double o) {
+  float f = (float)o;
+  uint32_t b;
+  std::memcpy(&b, &f, 4);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Per-image visible cap ("Spirula Studio VRAM deep-dive", practical guide:
+// --cap-max, the per-image visible splat cap that holds down nnz).  The page
+// gives no selection rule; reading: in each camera whose visible pairs
+// exceed cap_max, keep the cap_max of highest opacity, ties going to the
+// lower Gaussian index, and drop the others.  Written as a plain
+// sort-and-truncate of each camera's visible list.
+void apply_visible_cap(std::vector<uint8_t>& vis, const double* opac, int64_t C, int64_t N, int64_t cap_max) {
+  if (cap_max < 0) return;
+  std::vector<int64_t> list;
+  for (int64_t c = 0; c < C; ++c) {
+    list.clear();
+    for (int64_t n = 0; n < N; ++n)
+      if (vis[c * N + n]) list.push_back(n);
+    if ((int64_t)list.size() <= cap_max) continue;
+    std::stable_sort(list.begin(), list.end(), [&](int64_t a, int64_t b) {
+      return opacity_order_key(opac[a]) > opacity_order_key(opac[b]);
+    });
+    for (size_t k = (size_t)cap_max; k < list.size(); ++k) vis[c * N + list[k]] = 0;
+  }
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -622,10 +652,12 @@ void orc_geometry(const orc_dims* d, int64_t* out) {
 // (nnz_out is still exact).  precision: 0 = fp32 decisions and values (inputs
 // must then be fp32-representable), 1 = fp64 throughout.  Screen rows are
 // stored in fp64: x, y, conic a, b, c, opacity, r, g, b, depth, 0, 0.
+// cap_max < 0: no visible cap.
 int orc_project(const orc_dims* d, const double* cams, const double* means, const double* quats,
                 const double* scales, const double* opac, const double* sh, int precision, uint32_t* mask,
                 uint32_t* block_count, int64_t* block_off, int64_t* nnz_out, double* screen, uint32_t* aabb,
-                int32_t* row_cam, int64_t* row_gauss, uint8_t* rgb_clamped, int64_t cap_rows, int nthreads) {
+                int32_t* row_cam, int64_t* row_gauss, uint8_t* rgb_clamped, int64_t cap_rows, int nthreads,
+                int64_t cap_max) {
   set_threads(nthreads);
   const int64_t N = d->N, C = d->C;
   const int K = (d->sh_degree + 1) * (d->sh_degree + 1);
@@ -650,6 +682,7 @@ int orc_project(const orc_dims* d, const double* cams, const double* means, cons
     }
     vis[i] = v ? 1 : 0;
   }
+  apply_visible_cap(vis, opac, C, N, cap_max);
   // (a) plain compaction
   std::vector<int64_t> slot_a((size_t)(C * N));
   int64_t run = 0;

@@ -48,7 +48,7 @@ def lib():
         L.orc_sh_basis_f64.argtypes = [i32, ct.c_double, ct.c_double, ct.c_double, P]
         L.orc_sh_basis_grad_f64.argtypes = [i32, ct.c_double, ct.c_double, ct.c_double, P]
         L.orc_geometry.argtypes = [P, P]
-        L.orc_project.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, P, P, P, P, P, i64, i32]
+        L.orc_project.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, P, P, P, P, P, i64, i32, i64]
         L.orc_row_boxes.argtypes = [P, P, P, P, P, P, P, P, i64, P]
         L.orc_count_tiles.argtypes = [P, P, i64, P, P]
         L.orc_intersect.argtypes = [P, P, P, P, i64, i32, P, P, i64, P]
@@ -125,7 +125,10 @@ def _inputs(scene):
                 opac=_c(scene.opacities, np.float64), sh=_c(scene.sh, np.float64))
 
 
-def project(scene, precision: int = 0, nthreads: int = 0, rows: bool = True) -> dict:
+def project(scene, precision: int = 0, nthreads: int = 0, rows: bool = True, cap_max: int | None = None) -> dict:
+    """Packed projection.  cap_max (per-image visible cap): in each camera
+    with more visible pairs, keep the cap_max of highest opacity (ties to the
+    lower Gaussian index)."""
     g = geometry(scene)
     d = dims_of(scene)
     x = _inputs(scene)
@@ -136,7 +139,8 @@ def project(scene, precision: int = 0, nthreads: int = 0, rows: bool = True) -> 
     L = lib()
     args = [ct.byref(d), _p(x["cams"]), _p(x["means"]), _p(x["quats"]), _p(x["scales"]), _p(x["opac"]),
             _p(x["sh"]), precision, _p(mask), _p(bc), _p(bo), ct.byref(nnz)]
-    rc = L.orc_project(*args, None, None, None, None, None, 0, nthreads)
+    cap = -1 if cap_max is None else int(cap_max)
+    rc = L.orc_project(*args, None, None, None, None, None, 0, nthreads, cap)
     if rc != 0:
         raise RuntimeError(f"oracle projection: compactions disagree (rc={rc})")
     out = dict(mask=mask, block_count=bc, block_off=bo, nnz=int(nnz.value))
@@ -148,7 +152,7 @@ def project(scene, precision: int = 0, nthreads: int = 0, rows: bool = True) -> 
     row_cam = np.zeros(max(n, 1), np.int32)
     row_gauss = np.zeros(max(n, 1), np.int64)
     rgb_cl = np.zeros((max(n, 1), 3), np.uint8)
-    rc = L.orc_project(*args, _p(screen), _p(aabb), _p(row_cam), _p(row_gauss), _p(rgb_cl), n, nthreads)
+    rc = L.orc_project(*args, _p(screen), _p(aabb), _p(row_cam), _p(row_gauss), _p(rgb_cl), n, nthreads, cap)
     if rc != 0:
         raise RuntimeError(f"oracle projection failed (rc={rc})")
     out.update(screen=screen[:n], aabb=aabb[:n], row_cam=row_cam[:n], row_gauss=row_gauss[:n],
@@ -266,9 +270,10 @@ def upstream(scene, img) -> np.ndarray:
     return (np.sign(np.asarray(img, np.float64) - scene.target) * scene.l1_scale).astype(np.float32)
 
 
-def forward(scene, precision: int = 0, nthreads: int = 0, bg=None, depth: bool = False) -> dict:
+def forward(scene, precision: int = 0, nthreads: int = 0, bg=None, depth: bool = False,
+            cap_max: int | None = None) -> dict:
     g = geometry(scene)
-    proj = project(scene, precision, nthreads)
+    proj = project(scene, precision, nthreads, cap_max=cap_max)
     isect = intersect(scene, proj)
     ks, vs = sort(isect["keys"], isect["vals"])
     toff = tile_ranges(ks, g["n_tiles"])
@@ -280,11 +285,13 @@ def forward(scene, precision: int = 0, nthreads: int = 0, bg=None, depth: bool =
     return f
 
 
-def step(scene, precision: int = 0, nthreads: int = 0, v_img=None, v_T=None, v_depth=None, bg=None) -> dict:
+def step(scene, precision: int = 0, nthreads: int = 0, v_img=None, v_T=None, v_depth=None, bg=None,
+         cap_max: int | None = None) -> dict:
     """One forward+backward pass; gradients in fp64.  With v_depth the
     forward also returns the expected depth and the backward takes its
-    gradient; bg blends a background colour per camera."""
-    f = forward(scene, precision, nthreads, bg=bg, depth=v_depth is not None)
+    gradient; bg blends a background colour per camera; cap_max applies the
+    per-image visible cap (see project)."""
+    f = forward(scene, precision, nthreads, bg=bg, depth=v_depth is not None, cap_max=cap_max)
     if v_img is None:
         v_img = upstream(scene, f["img"])
     v_screen = rasterize_bwd(scene, f["proj"]["screen"], f["vals_sorted"], f["tile_off"], v_img, v_T, precision,

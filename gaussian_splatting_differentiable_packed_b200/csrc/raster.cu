@@ -45,21 +45,35 @@ __device__ __forceinline__ void tile_coords(const Geo& g, int64_t tile, int& c, 
 }
 
 // ---------------------------------------------------------------------------
-// Staged entry.  thr = 5.6 when o <= 1 (then sigma > 5.6 implies
-// o*exp(-sigma) < 1/255: the pixel skips the entry without the exp), +inf
-// otherwise.  The remaining fields bound where the entry can matter, all
-// computed in fp32 and rounded outward: dql underestimates ca*cc - cb^2 (the
-// fma error bound subtracted), so (hx, hy) over-cover the ellipse
-// {sigma <= 5.8} of the stored conic and the row chords below over-cover it
-// too; +inf / "everything" when o > 1 or the conic is not safely positive
-// definite.
-constexpr float kCullT = 5.8f;
+// Staged entry.  thr is the entry's skip threshold: a pixel whose canonical
+// sigma exceeds thr cannot reach alpha >= 1/255, so it skips the entry
+// without the exp (the per-pixel definition skips it too).  For o <= 1 it is
+// ln(255 o) plus a small margin, verified in the canonical arithmetic
+// (o * E(-thr) < 1/255; E is monotone, so every larger sigma fails too) and
+// capped at 5.6 (E(-5.6) < 1/255 holds for every o <= 1); -1 when o < 1/255
+// (alpha <= o can never reach 1/255); +inf when o > 1.  The remaining fields
+// bound where the entry can matter, all computed in fp32 and rounded outward:
+// dql underestimates ca*cc - cb^2 (the fma error bound subtracted), so
+// (hx, hy) over-cover the ellipse {sigma <= thr + kCullMargin} of the stored
+// conic and the row chords below over-cover it too; +inf / "everything" when
+// o > 1 or the conic is not safely positive definite.  The margin covers the
+// fp32 rounding of the canonical sigma (at most 0.04 where the coverage is
+// used, see warp_culled and entry_coverage).
+constexpr float kCullMargin = 0.2f;
+
+__device__ __forceinline__ float entry_threshold(float o, float amin) {
+  if (!(o <= 1.0f)) return __int_as_float(0x7f800000);
+  if (!(o >= amin)) return -1.0f;
+  float thr = fminf(SS_SIGMA_SKIP, __logf(255.0f * o) + 2e-3f);
+  if (!(mul(o, exp_neg(-thr)) < amin)) thr = SS_SIGMA_SKIP;
+  return thr;
+}
 
 struct Stage {
   float4 a;  // x, y, 0.5*ca, cb
   float4 b;  // 0.5*cc, o, r, g
   float4 c;  // b, hx, hy, kterm = |ha| + |hc| + |cb|
-  float4 d;  // thr, row (bits), P = 2*ca*kCullT, dql
+  float4 d;  // thr, row (bits), P = 2*ca*(thr + margin), dql
   float4 e;  // 1/ca, cb/ca, bounded (1/0), depth
 };
 
@@ -70,31 +84,39 @@ __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint
   st.a = make_float4(r0.x, r0.y, mul(0.5f, ca), cb);
   st.b = make_float4(mul(0.5f, cc), o, r1.z, r1.w);
   const float inf = __int_as_float(0x7f800000);
+  const float thr = entry_threshold(o, alpha_min());
   const float bb = cb * cb;
   const float dq = fmaf(ca, cc, -bb);
   const float dql = dq - 2e-7f * (bb + fabsf(dq)) - 1e-30f;
   float hx = inf, hy = inf, P = 0.0f, ica = 0.0f, cbr = 0.0f, bounded = 0.0f;
-  if (o <= 1.0f && ca > 0.0f && cc > 0.0f && dql > 0.0f) {
-    hx = sqrtf(2.0f * kCullT * cc / dql) * 1.00001f + 1e-3f;
-    hy = sqrtf(2.0f * kCullT * ca / dql) * 1.00001f + 1e-3f;
-    P = 2.0f * kCullT * ca;
+  if (thr < 0.0f) {
+    // never composited: an empty box
+    hx = hy = -1.0f;
+    P = -1.0f;
+    bounded = 1.0f;
+  } else if (o <= 1.0f && ca > 0.0f && cc > 0.0f && dql > 0.0f) {
+    const float L = thr + kCullMargin;
+    hx = sqrtf(2.0f * L * cc / dql) * 1.00001f + 1e-3f;
+    hy = sqrtf(2.0f * L * ca / dql) * 1.00001f + 1e-3f;
+    P = 2.0f * L * ca;
     ica = 1.0f / ca;
     cbr = cb * ica;
     bounded = 1.0f;
   }
   const float kterm = 0.5f * fabsf(ca) + 0.5f * fabsf(cc) + fabsf(cb);
   st.c = make_float4(r2.x, hx, hy, kterm);
-  st.d = make_float4(o <= 1.0f ? SS_SIGMA_SKIP : inf, __uint_as_float(r), P, dql);
+  st.d = make_float4(thr, __uint_as_float(r), P, dql);
   st.e = make_float4(ica, cbr, bounded, r2.y);
 }
 
 // Warp culling.  For an entry with o <= 1 every pixel whose computed sigma
-// exceeds 5.6 skips the entry.  A region outside the box (hx, hy) of the
-// ellipse {sigma <= 5.8} has exact sigma > 5.8 at every pixel centre; when
-// kterm*(Dx^2 + Dy^2) <= 8e4 (D: largest offset from the mean to the region)
-// the canonical fp32 sigma differs from the exact one by less than 0.04, so
-// every pixel of the region computes sigma > 5.6 and would skip the entry:
-// skipping it for the whole warp takes exactly the per-pixel decision.
+// exceeds thr skips the entry.  A region outside the box (hx, hy) of the
+// ellipse {sigma <= thr + 0.2} has exact sigma > thr + 0.2 at every pixel
+// centre; when kterm*(Dx^2 + Dy^2) <= 8e4 (D: largest offset from the mean to
+// the region) the canonical fp32 sigma differs from the exact one by less
+// than 0.04, so every pixel of the region computes sigma > thr and would skip
+// the entry: skipping it for the whole warp takes exactly the per-pixel
+// decision.
 __device__ __forceinline__ bool warp_culled(const Stage& st, float x_lo, float x_hi, float y_lo, float y_hi) {
   const float mx = st.a.x, my = st.a.y;
   const float ex = fmaxf(fmaxf(x_lo - mx, mx - x_hi), 0.0f);
@@ -268,9 +290,9 @@ __global__ __launch_bounds__(kRThreads) void k_raster_fwd(Geo g, const float* __
 // ---------------------------------------------------------------------------
 // Per-pixel candidate masks.  For a block of 32 staged entries (one per lane)
 // each lane computes which of the warp's 64 pixels its entry can reach: a
-// pixel is left out only if its computed sigma provably exceeds 5.6 for an
-// entry with o <= 1 (exact sigma > 5.7 outside the fp64 chord of the ellipse
-// {sigma <= 5.7}, widened by 1e-3 px, and kterm*D^2 <= 8e4 bounds the fp32
+// pixel is left out only if its computed sigma provably exceeds the entry's
+// threshold thr (exact sigma > thr + 0.2 outside the outward-rounded chord of
+// the ellipse {sigma <= thr + 0.2}, and kterm*D^2 <= 8e4 bounds the fp32
 // rounding of the canonical sigma by 0.04); such pixels skip the entry in the
 // per-pixel definition too.  A 32x32 bit transpose across the warp then gives
 // each lane the entries of the block that reach each of its two pixels.
@@ -291,10 +313,10 @@ __device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
 }
 
 // 16-bit column mask of the pixels of row centre yc (columns x_lo + c,
-// c = 0..15) inside the outward-rounded chord of {sigma <= 5.8}: for a pixel
-// row at offset dy the chord is centred at mx + (cb/ca)*dy with half-width
-// sqrt(2*ca*5.8 - dq*dy^2)/ca; dql <= dq and the margins make every fp32
-// rounding widen it.
+// c = 0..15) inside the outward-rounded chord of {sigma <= L}, L = thr + 0.2:
+// for a pixel row at offset dy the chord is centred at mx + (cb/ca)*dy with
+// half-width sqrt(2*ca*L - dq*dy^2)/ca; dql <= dq and the margins make every
+// fp32 rounding widen it.
 __device__ __forceinline__ uint32_t chord_span(const Stage& st, float yc, float x_lo) {
   const float dy = st.a.y - yc;
   const float q = st.d.w * dy * dy;
@@ -316,9 +338,9 @@ __device__ __forceinline__ uint32_t chord_span(const Stage& st, float yc, float 
 
 // Coverage of this lane's entry over the warp's region: bit L of covA (covB)
 // set when the entry can reach lane L's upper (lower) pixel.  A pixel left
-// out has exact sigma > 5.8, and kterm*D^2 <= 8e4 bounds the rounding of the
-// canonical fp32 sigma by 0.04, so its computed sigma exceeds 5.6: it skips
-// the entry in the per-pixel definition as well.
+// out has exact sigma > thr + 0.2, and kterm*D^2 <= 8e4 bounds the rounding
+// of the canonical fp32 sigma by 0.04, so its computed sigma exceeds thr: it
+// skips the entry in the per-pixel definition as well.
 __device__ __forceinline__ void entry_coverage(const Stage& st, float x_lo, float y_lo, uint32_t& covA,
                                                uint32_t& covB) {
   const float x_hi = x_lo + 15.0f, y_hi = y_lo + 3.0f;
@@ -541,6 +563,17 @@ __device__ __forceinline__ uint32_t live_bits(int64_t last, int64_t qb) {
   return d >= 31 ? 0xFFFFFFFFu : (2u << (int)d) - 1u;
 }
 
+// exp(x) of a pair through the hardware's fast exponential (relative error
+// about 1e-6 on the sigma range the replay evaluates); see pair_grad for
+// where the canonical E takes over.
+__device__ __forceinline__ float2 exp_fast_pair(float2 x) { return f2(__expf(x.x), __expf(x.y)); }
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Reverse step of the thread's pixel pair for a replayed entry.  cA / cB say
 // which pixels replay the entry with sigma within the skip threshold.  A
 // pixel that does not take the entry (alpha < 1/255, the forward's decision
@@ -553,18 +586,33 @@ __device__ __forceinline__ uint32_t live_bits(int64_t last, int64_t qb) {
 //   dL/dca = dx^2*S0/2,  dL/dcb = dx*S1,  dL/dcc = S2/2,
 // where S0 = sum v, S1 = sum v*dy, S2 = sum v*dy^2 (dx is shared).
 //
+// The exponential comes from the fast hardware path; only the two decisions
+// the forward took on it must come out the same (alpha >= 1/255, and
+// whether o*E reached the 0.99 clamp), so wherever o*exp lies within 1e-5
+// (relative) of either threshold, ten times the fast path's error, the pair
+// is recomputed with the canonical E.  Elsewhere alpha and the recovered
+// transmittance (an approximate reciprocal) differ from the forward's by a
+// few ulps, which moves the gradients by about 1e-6 relative.
+//
 // EXT: the expected depth is a fourth channel composited with the same
 // weights, so depth * gD joins the colour term of dL/dalpha and
 // gr[9] = sum w * gD is the row's depth gradient.
 template <bool EXT>
-__device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, float2 ev, bool cA, bool cB,
+__device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, float2 sig, bool cA, bool cB,
                                           float amin, PixB& pa, PixB& pb, float* gr) {
-  const float2 oe = __fmul2_rn(f2s(st.b.y), ev);
+  float2 ev = exp_fast_pair(f2(-sig.x, -sig.y));
+  float2 oe = __fmul2_rn(f2s(st.b.y), ev);
+  const bool nearA = fabsf(oe.x - amin) <= 1e-5f * amin || fabsf(oe.x - SS_ALPHA_MAX) <= 1e-5f;
+  const bool nearB = fabsf(oe.y - amin) <= 1e-5f * amin || fabsf(oe.y - SS_ALPHA_MAX) <= 1e-5f;
+  if ((cA && nearA) || (cB && nearB)) {
+    ev = exp_neg_pair(f2(-sig.x, -sig.y));
+    oe = __fmul2_rn(f2s(st.b.y), ev);
+  }
   cA = cA && !(fminf(SS_ALPHA_MAX, oe.x) < amin);
   cB = cB && !(fminf(SS_ALPHA_MAX, oe.y) < amin);
   if (!(cA || cB)) return false;
   const float2 a = f2(cA ? fminf(SS_ALPHA_MAX, oe.x) : 0.0f, cB ? fminf(SS_ALPHA_MAX, oe.y) : 0.0f);
-  const float2 ra = f2(__frcp_rn(1.0f - a.x), __frcp_rn(1.0f - a.y));
+  const float2 ra = f2(rcp_approx(1.0f - a.x), rcp_approx(1.0f - a.y));
   const float2 Ti = __fmul2_rn(f2(pa.T, pb.T), ra);  // transmittance in front of the entry
   const float2 w = __fmul2_rn(a, Ti);
   const float2 G0 = f2(pa.g0, pb.g0), G1 = f2(pa.g1, pb.g1), G2 = f2(pa.g2, pb.g2);
@@ -634,6 +682,16 @@ __device__ __forceinline__ void flush_sums(float (*red)[kBatchB][kRedF], const u
   }
 }
 
+// The warp's sums of an entry when a single lane contributed: that lane's
+// values, stored by it (the row's pad words stay zero).
+template <bool EXT>
+__device__ __forceinline__ void store_sums(float* row, const float* gr, uint32_t* any) {
+  reinterpret_cast<float4*>(row)[0] = make_float4(gr[0], gr[1], gr[2], gr[3]);
+  reinterpret_cast<float4*>(row)[1] = make_float4(gr[4], gr[5], gr[6], gr[7]);
+  reinterpret_cast<float2*>(row)[4] = make_float2(gr[8], EXT ? gr[9] : 0.0f);
+  *any = 1u;
+}
+
 // One replayed entry (bit hb of the lanes' candidate masks mA, mB) for the
 // thread's pixel pair: sigma and exp where a pixel is a candidate, then the
 // reverse step.  gr[0..9] is zero when neither pixel contributes.
@@ -648,10 +706,7 @@ __device__ __forceinline__ bool entry_grad(const Stage& st, uint32_t mA, uint32_
     const float2 sig = sigma_pair(st, dx, dy);
     const bool needA = liveA && !(sig.x < 0.0f) && !(sig.x > st.d.x);
     const bool needB = liveB && !(sig.y < 0.0f) && !(sig.y > st.d.x);
-    if (needA || needB) {
-      const float2 ev = exp_neg_pair(f2(-sig.x, -sig.y));
-      contrib = pair_grad<EXT>(st, dx, dy, ev, needA, needB, amin, pa, pb, gr);
-    }
+    if (needA || needB) contrib = pair_grad<EXT>(st, dx, dy, sig, needA, needB, amin, pa, pb, gr);
   }
   if (!contrib) {
 #pragma unroll
@@ -763,7 +818,9 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
           bits &= ~(1u << hb);
           int kA = q * 32 + hb;
           float gr[10];
-          bool anyA = __any_sync(0xffffffffu, entry_grad<EXT>(s_e[kA], mA, mB, hb, px, npy, amin, pa, pb, gr));
+          bool cA;
+          uint32_t balA;
+          const uint32_t mAB = mA | mB;
           if (bits) {
             // the next candidate of the warp: its pixel step follows this
             // one's, and the two entries' sums are reduced together
@@ -771,9 +828,36 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
             bits &= ~(1u << hb2);
             const int kB = q * 32 + hb2;
             float gr2[10];
-            const bool anyB =
-                __any_sync(0xffffffffu, entry_grad<EXT>(s_e[kB], mA, mB, hb2, px, npy, amin, pa, pb, gr2));
-            if (anyA && anyB) {
+            bool cB;
+            const bool inA = (mAB >> hb) & 1u, inB = (mAB >> hb2) & 1u;
+            if (!__any_sync(0xffffffffu, inA && inB)) {
+              // no pixel pair of the warp is a candidate of both entries:
+              // each lane steps through the one entry it has (if any), so
+              // both entries take one pixel step between them
+              const int hx = inA ? hb : hb2;
+              float g1[10];
+              const bool c1 = entry_grad<EXT>(s_e[q * 32 + hx], mA, mB, hx, px, npy, amin, pa, pb, g1);
+              cA = inA && c1;
+              cB = !inA && c1;
+#pragma unroll
+              for (int t = 0; t < 10; ++t) {
+                gr[t] = inA ? g1[t] : 0.0f;
+                gr2[t] = inA ? 0.0f : g1[t];
+              }
+            } else {
+              cA = entry_grad<EXT>(s_e[kA], mA, mB, hb, px, npy, amin, pa, pb, gr);
+              cB = entry_grad<EXT>(s_e[kB], mA, mB, hb2, px, npy, amin, pa, pb, gr2);
+            }
+            balA = __ballot_sync(0xffffffffu, cA);
+            const uint32_t balB = __ballot_sync(0xffffffffu, cB);
+            if ((balA & (balA - 1u)) == 0u && (balB & (balB - 1u)) == 0u) {
+              // at most one lane contributes to each entry: its pixel pair's
+              // sums are the warp's, stored as they are
+              if (cA) store_sums<EXT>(red[warp][kA], gr, any + kA);
+              if (cB) store_sums<EXT>(red[warp][kB], gr2, any + kB);
+              continue;
+            }
+            if (balA && balB) {
               const float s8 = warp_reduce8x2(gr, gr2, lane);
               const float s2 = warp_sum_x2<EXT>(gr[8], gr[9], gr2[8], gr2[9], lane);
               const int kl = (lane & 16) ? kB : kA;
@@ -785,14 +869,20 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
               if (EXT && (lane & 15) == 8) red[warp][kl][9] = s2;
               continue;
             }
-            if (anyB) {
+            if (balB) {
 #pragma unroll
               for (int t = 0; t < 10; ++t) gr[t] = gr2[t];
               kA = kB;
-              anyA = true;
+              cA = cB;
+              balA = balB;
             }
+          } else {
+            cA = entry_grad<EXT>(s_e[kA], mA, mB, hb, px, npy, amin, pa, pb, gr);
+            balA = __ballot_sync(0xffffffffu, cA);
           }
-          if (anyA) {
+          if ((balA & (balA - 1u)) == 0u) {
+            if (cA) store_sums<EXT>(red[warp][kA], gr, any + kA);
+          } else {
             const float s8 = warp_reduce8(gr, lane);
             const float sb = warp_sum(gr[8]);
             const float sd = EXT ? warp_sum(gr[9]) : 0.0f;

@@ -23,55 +23,69 @@ namespace ss {
 
 constexpr int kCamChunkB = 32;
 
+// dL/d(coefficient k, channel ch) += b_k v_ch where the channel was not
+// clamped (vm holds v with the clamped channels zeroed).
 template <int DEG>
-__device__ __forceinline__ void sh_grads(float X, float Y, float Z, const float* __restrict__ shn, const float vr[3],
-                                         const bool cl[3], float* gsh, float vdir[3]) {
+__device__ __forceinline__ void sh_coef_grads(float X, float Y, float Z, const float vm[3], const bool cl[3],
+                                              float* gsh) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   float b[16];
   sh_basis(DEG, X, Y, Z, b);
-  // d b_k / d(X, Y, Z)
-  float dX[16], dY[16], dZ[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) dX[k] = dY[k] = dZ[k] = 0.0f;
+  for (int k = 0; k < K; ++k)
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch)
+      if (!cl[ch]) gsh[3 * k + ch] += b[k] * vm[ch];
+}
+
+// The view direction's gradient sum_k w_k db_k/d(X, Y, Z) with
+// w_k = sum_ch coefficient(k, ch) v_ch (one weight per basis function; only
+// the derivatives that are not identically zero are taken).
+template <int DEG>
+__device__ __forceinline__ void sh_dir_grads(float X, float Y, float Z, const float* __restrict__ shn,
+                                             const float vm[3], float vdir[3]) {
+  constexpr int K = (DEG + 1) * (DEG + 1);
+  float w[16];
+#pragma unroll
+  for (int k = 0; k < K; ++k)
+    w[k] = k == 0 ? 0.0f : shn[3 * k] * vm[0] + shn[3 * k + 1] * vm[1] + shn[3 * k + 2] * vm[2];
+  float gX = 0.0f, gY = 0.0f, gZ = 0.0f;
   if (DEG >= 1) {
-    dY[1] = -SS_SH_C1; dZ[2] = SS_SH_C1; dX[3] = -SS_SH_C1;
+    gY -= SS_SH_C1 * w[1];
+    gZ += SS_SH_C1 * w[2];
+    gX -= SS_SH_C1 * w[3];
   }
   if (DEG >= 2) {
-    dX[4] = SS_SH_C2A * Y; dY[4] = SS_SH_C2A * X;
-    dY[5] = -SS_SH_C2A * Z; dZ[5] = -SS_SH_C2A * Y;
-    dX[6] = -2.0f * SS_SH_C2C * X; dY[6] = -2.0f * SS_SH_C2C * Y; dZ[6] = 4.0f * SS_SH_C2C * Z;
-    dX[7] = -SS_SH_C2A * Z; dZ[7] = -SS_SH_C2A * X;
-    dX[8] = 2.0f * SS_SH_C2E * X; dY[8] = -2.0f * SS_SH_C2E * Y;
+    gX += SS_SH_C2A * (Y * w[4] - Z * w[7]) + 2.0f * SS_SH_C2E * X * w[8] - 2.0f * SS_SH_C2C * X * w[6];
+    gY += SS_SH_C2A * (X * w[4] - Z * w[5]) - 2.0f * SS_SH_C2E * Y * w[8] - 2.0f * SS_SH_C2C * Y * w[6];
+    gZ += -SS_SH_C2A * (Y * w[5] + X * w[7]) + 4.0f * SS_SH_C2C * Z * w[6];
   }
   if (DEG >= 3) {
     const float XX = X * X, YY = Y * Y, ZZ = Z * Z;
-    dX[9] = -SS_SH_C3A * 6.0f * X * Y; dY[9] = -SS_SH_C3A * (3.0f * XX - 3.0f * YY);
-    dX[10] = SS_SH_C3B * Y * Z; dY[10] = SS_SH_C3B * X * Z; dZ[10] = SS_SH_C3B * X * Y;
-    dX[11] = 2.0f * SS_SH_C3C * X * Y; dY[11] = -SS_SH_C3C * (4.0f * ZZ - XX - 3.0f * YY);
-    dZ[11] = -8.0f * SS_SH_C3C * Y * Z;
-    dX[12] = -6.0f * SS_SH_C3D * X * Z; dY[12] = -6.0f * SS_SH_C3D * Y * Z;
-    dZ[12] = SS_SH_C3D * (6.0f * ZZ - 3.0f * XX - 3.0f * YY);
-    dX[13] = -SS_SH_C3C * (4.0f * ZZ - 3.0f * XX - YY); dY[13] = 2.0f * SS_SH_C3C * X * Y;
-    dZ[13] = -8.0f * SS_SH_C3C * X * Z;
-    dX[14] = 2.0f * SS_SH_C3F * X * Z; dY[14] = -2.0f * SS_SH_C3F * Y * Z; dZ[14] = SS_SH_C3F * (XX - YY);
-    dX[15] = -SS_SH_C3A * (3.0f * XX - 3.0f * YY); dY[15] = SS_SH_C3A * 6.0f * X * Y;
+    gX += -SS_SH_C3A * 6.0f * X * Y * w[9] + SS_SH_C3B * Y * Z * w[10] + 2.0f * SS_SH_C3C * X * Y * w[11] -
+          6.0f * SS_SH_C3D * X * Z * w[12] - SS_SH_C3C * (4.0f * ZZ - 3.0f * XX - YY) * w[13] +
+          2.0f * SS_SH_C3F * X * Z * w[14] - SS_SH_C3A * (3.0f * XX - 3.0f * YY) * w[15];
+    gY += -SS_SH_C3A * (3.0f * XX - 3.0f * YY) * w[9] + SS_SH_C3B * X * Z * w[10] -
+          SS_SH_C3C * (4.0f * ZZ - XX - 3.0f * YY) * w[11] - 6.0f * SS_SH_C3D * Y * Z * w[12] +
+          2.0f * SS_SH_C3C * X * Y * w[13] - 2.0f * SS_SH_C3F * Y * Z * w[14] + SS_SH_C3A * 6.0f * X * Y * w[15];
+    gZ += SS_SH_C3B * X * Y * w[10] - 8.0f * SS_SH_C3C * Y * Z * w[11] +
+          SS_SH_C3D * (6.0f * ZZ - 3.0f * XX - 3.0f * YY) * w[12] - 8.0f * SS_SH_C3C * X * Z * w[13] +
+          SS_SH_C3F * (XX - YY) * w[14];
   }
-#pragma unroll
-  for (int ch = 0; ch < 3; ++ch) {
-    if (cl[ch]) continue;
-    const float v = vr[ch];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      gsh[3 * k + ch] += b[k] * v;
-      if (DEG >= 1) {
-        const float sv = shn[3 * k + ch] * v;
-        vdir[0] += sv * dX[k];
-        vdir[1] += sv * dY[k];
-        vdir[2] += sv * dZ[k];
-      }
-    }
-  }
+  vdir[0] = gX;
+  vdir[1] = gY;
+  vdir[2] = gZ;
 }
+
+// Whether any camera sees Gaussian m (a set bit in one of its C mask words).
+__device__ __forceinline__ bool any_camera_sees(const Geo& g, const uint32_t* __restrict__ mask, int64_t m) {
+  uint32_t u = 0;
+  for (int c = 0; c < g.C && !u; ++c) u = (mask[((int64_t)c * g.n_pad + m) / 32] >> (m & 31)) & 1u;
+  return u != 0;
+}
+
+// Bit gi of the CTA's per-warp visibility words.
+__device__ __forceinline__ bool seen(const uint32_t* s_seen, int gi) { return (s_seen[gi >> 5] >> (gi & 31)) & 1u; }
 
 // Shared-memory stride per Gaussian for SH blocks (odd, so that thread t's
 // word k sits in bank (t*stride + k) mod 32: conflict-free across a warp).
@@ -137,9 +151,11 @@ struct GqArgs {
   int first;     // the accumulators start from zero (their contents are ignored)
 };
 
-__device__ __forceinline__ int16_t gq_code(float x, float s) {
-  if (!(s > 0.0f)) return 0;
-  return (int16_t)__float2int_rn(fminf(fmaxf(x / s, -kGqMax), kGqMax));
+// Code of x at a block scale s, given is = 1/s (0 when s is 0): the quotient
+// x/s is taken as x * is, at most about 1.5 ulp of the quotient (0.005 of a
+// step at full scale) from the correctly rounded one.
+__device__ __forceinline__ int16_t gq_code(float x, float is) {
+  return (int16_t)__float2int_rn(fminf(fmaxf(x * is, -kGqMax), kGqMax));
 }
 
 // Largest value of v over the CTA for each attribute (a < kGqAttr), into out.
@@ -197,6 +213,13 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   __shared__ Cam scam[kCamChunkB];
   __shared__ uint32_t s_word[kCamChunkB][kWarps];
   __shared__ int64_t s_row0[kCamChunkB][kWarps];
+  __shared__ float s_margin[kBlock][3];
+  __shared__ uint32_t s_seen[kWarps];  // per warp: its Gaussians seen by some camera
+  // the optimizer updates every parameter and the accumulators are decoded
+  // into the SH staging area, so only the plain backward skips unseen rows
+  constexpr bool kSkipUnseen = !ADAM && !GQ;
+  __shared__ __align__(16) float s_pf[kWarps][32][4];  // a round's pair sums: mean (3), opacity
+  __shared__ double s_pd[kWarps][32][6];               // and dL/dSigma
   extern __shared__ float smem[];
   float* sh_s = smem;                 // [kBlock][KP] SH coefficients of the CTA's Gaussians
   float* gsh_s = smem + kBlock * KP;  // [kBlock][KP] their gradient accumulators
@@ -225,10 +248,34 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     prefetch_l2(v_screen + r0 * kRowF, (uint32_t)((r1 - r0) * kRowF * 4));
   }
   // (blocks_per_cam, not the grid: a grad-quant grid may hold one CTA more)
-  if (threadIdx.x == 0 && ahead > 0 && blk + ahead < (GQ ? g.blocks_per_cam : (int64_t)gridDim.x)) {
-    // the SH block of the CTA that starts about a wave later, into L2
+  if (ahead > 0 && blk + ahead < (GQ ? g.blocks_per_cam : (int64_t)gridDim.x)) {
+    // the SH block of the CTA that starts about a wave later, into L2; the
+    // plain backward reads only the rows of Gaussians some camera sees
     const int64_t m0 = (blk + ahead) * kBlock;
-    prefetch_l2(sh + m0 * K3, (uint32_t)(min64(kBlock, g.N - m0) * K3 * 4));
+    const int mc = (int)min64(kBlock, g.N - m0);
+    if (kSkipUnseen) {
+      if (threadIdx.x < mc && any_camera_sees(g, mask, m0 + threadIdx.x))
+        prefetch_l2(sh + (m0 + threadIdx.x) * K3, (uint32_t)(K3 * 4));
+    } else if (threadIdx.x == 0) {
+      prefetch_l2(sh + m0 * K3, (uint32_t)(mc * K3 * 4));
+    }
+  }
+  if (kSkipUnseen) {
+    // which of the CTA's Gaussians any camera sees (per warp, one word)
+    uint32_t u = 0;
+    for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + n0) / 32 + warp];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
+    if (lane == 0) s_seen[warp] = u;
+    __syncthreads();
+  }
+  if (GQ && !gqa.first && threadIdx.x == 0) {
+    // the accumulator codes are read after the camera loop: have L2 fetch
+    // the CTA's now
+    constexpr int kWidths[kGqAttr] = {3, 4, 3, 1, 3, K3 - 3};
+#pragma unroll
+    for (int a = 0; a < kGqAttr; ++a)
+      if (kWidths[a] > 0) prefetch_l2(gqa.code[a] + kWidths[a] * n0, (uint32_t)(cnt * kWidths[a] * 2));
   }
   if (ADAM && threadIdx.x == 0) {
     // the optimizer state is only touched after the camera loop: have L2 fetch
@@ -245,7 +292,10 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   }
   // coalesced staging of the CTA's contiguous SH block: full blocks with all
   // 16-byte loads in flight at once (the block starts 16-byte aligned: 128*K3
-  // floats per block), the ragged last block word by word
+  // floats per block), the ragged last block word by word.  The plain
+  // backward skips the rows of Gaussians no camera sees: their gradients
+  // are zero and their coefficients are never read (a third of the
+  // Gaussians of the 15M-Gaussian workload)
   {
     const float* src = sh + n0 * K3;
     if (cnt == kBlock) {
@@ -255,7 +305,10 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
         const int v = threadIdx.x + r * kBlock;
-        if (v < kV) buf[r] = reinterpret_cast<const float4*>(src)[v];
+        if (v < kV && (!kSkipUnseen || seen(s_seen, (4 * v) / K3) || seen(s_seen, (4 * v + 3) / K3)))
+          buf[r] = reinterpret_cast<const float4*>(src)[v];
+        else
+          buf[r] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
@@ -274,19 +327,35 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     } else {
       for (int f = threadIdx.x; f < kBlock * K3; f += kBlock) {
         const int gi = f / K3, q = f - gi * K3;
-        sh_s[gi * KP + q] = f < cnt * K3 ? src[f] : 0.0f;
+        sh_s[gi * KP + q] = f < cnt * K3 && (!kSkipUnseen || seen(s_seen, gi)) ? src[f] : 0.0f;
         gsh_s[gi * KP + q] = 0.0f;
       }
     }
   }
-  const float* shn = sh_s + threadIdx.x * KP;
-  float* gsh = gsh_s + threadIdx.x * KP;
+  __syncthreads();  // the staged SH block is read below
+  {
+    // Bound on how far 0.5 + sum_k sh_k b_k can move with the summation
+    // order: each order's rounding is below 17 * 2^-24 * (0.5 + sum_k |sh_k
+    // b_k|) and |b_k| <= 2 on the unit sphere for degree <= 3; the margin is
+    // ten times that.  One per Gaussian and channel, read by the lane that
+    // takes the pair.
+    const float* shn = sh_s + threadIdx.x * KP;
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) {
+      float a = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < K; ++kk) a += fabsf(shn[3 * kk + ch]);
+      s_margin[threadIdx.x][ch] = 1e-5f * (1.0f + 2.0f * a);
+    }
+  }
   const int64_t nn = valid ? n : 0;
   const float mx = means[3 * nn], my = means[3 * nn + 1], mz = means[3 * nn + 2];
-  const float4 q4 = reinterpret_cast<const float4*>(quats)[nn];
-  const QuatRot qr = quat_rot(q4.x, q4.y, q4.z, q4.w);
-  const float s0 = scales[3 * nn], s1 = scales[3 * nn + 1], s2 = scales[3 * nn + 2];
-  const Cov3 S = cov3(qr, s0, s1, s2);
+  Cov3 S;
+  {
+    const float4 q = reinterpret_cast<const float4*>(quats)[nn];
+    const QuatRot qr = quat_rot(q.x, q.y, q.z, q.w);
+    S = cov3(qr, scales[3 * nn], scales[3 * nn + 1], scales[3 * nn + 2]);
+  }
   float gmu[3] = {0.f, 0.f, 0.f}, go = 0.f;
   double gS[6] = {0., 0., 0., 0., 0., 0.};  // dL/dSigma, full-matrix convention (00 01 02 11 12 22)
   float gx[GQ ? 11 : 1] = {};  // GQ: this Gaussian's means, quats, scales and opacity gradients
@@ -305,137 +374,209 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
       s_row0[cc][w] = row;
     }
     __syncthreads();
-    if (!valid) continue;
-    // Each lane walks its own visible cameras: a warp runs as many rounds as
-    // its busiest Gaussian has cameras, not one round per camera of the chunk.
+    // The warp's (Gaussian, camera) pairs of this chunk, numbered Gaussian by
+    // Gaussian (lane order) and camera by camera, are dealt to the lanes 32 at
+    // a time, so a warp runs ceil(pairs / 32) rounds rather than as many as
+    // its busiest Gaussian has cameras.  The lane that takes a pair reads its
+    // owner's data from the owner lane (shuffles) and shared memory; the
+    // owner adds its pairs' sums in camera order (deterministic).
     uint32_t vis = 0;
-    for (int cc = 0; cc < nc; ++cc) vis |= ((s_word[cc][warp] >> lane) & 1u) << cc;
-    // the gradient row of the next visible camera is loaded one round ahead
-    // (x, y, ca, cb | cc, o, r, g | b, depth)
-    const uint32_t below = (1u << lane) - 1u;
-    float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
-    float2 n2 = make_float2(0.f, 0.f);
-    if (vis) {
-      const int cc = __ffs(vis) - 1;
-      const float* rp = v_screen + (s_row0[cc][warp] + __popc(s_word[cc][warp] & below)) * kRowF;
-      n0 = reinterpret_cast<const float4*>(rp)[0];
-      n1 = reinterpret_cast<const float4*>(rp)[1];
-      n2 = reinterpret_cast<const float2*>(rp)[4];
+    if (valid)
+      for (int cc = 0; cc < nc; ++cc) vis |= ((s_word[cc][warp] >> lane) & 1u) << cc;
+    const int nv = __popc(vis);
+    int incl = nv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
     }
-    while (vis) {
-      const int cc = __ffs(vis) - 1;
-      vis &= vis - 1;
-      const float4 v0 = n0, v1 = n1;
-      const float2 v2 = n2;
-      if (vis) {
-        const int cn = __ffs(vis) - 1;
-        const float* rp = v_screen + (s_row0[cn][warp] + __popc(s_word[cn][warp] & below)) * kRowF;
-        n0 = reinterpret_cast<const float4*>(rp)[0];
-        n1 = reinterpret_cast<const float4*>(rp)[1];
-        n2 = reinterpret_cast<const float2*>(rp)[4];
+    const int excl = incl - nv;
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    for (int r0 = 0; r0 < total; r0 += 32) {
+      const int i = r0 + lane;
+      const bool has = i < total;
+      // owner: the last lane whose first pair is at or before i
+      int o = 0;
+#pragma unroll
+      for (int step = 16; step >= 1; step >>= 1) {
+        const int cand = o + step;
+        const int pe = __shfl_sync(0xffffffffu, excl, cand & 31);
+        if (cand < 32 && pe <= i) o = cand;
       }
-      const Cam& k = scam[cc];
-      const float* R = k.R;
-      // camera point and the projection's gating decision in canonical arithmetic
-      float px, py, pz;
-      cam_point(k, mx, my, mz, px, py, pz);
-      const float izc = div_(1.0f, pz);
-      const float u = mul(px, izc), v = mul(py, izc);
-      const bool clx = (u < -k.limx) || (u > k.limx);
-      const bool cly = (v < -k.limy) || (v > k.limy);
-      const float ux = fminf(fmaxf(u, -k.limx), k.limx), uy = fminf(fmaxf(v, -k.limy), k.limy);
-      // gradient arithmetic (any rounding order)
-      const float iz = 1.0f / pz, iz2 = iz * iz;
-      const float j00 = k.fx * iz, j02 = -j00 * ux, j11 = k.fy * iz, j12 = -j11 * uy;
-      float T[6];
+      const uint32_t vo = __shfl_sync(0xffffffffu, vis, o);
+      const int eo = __shfl_sync(0xffffffffu, excl, o);
+      const float omx = __shfl_sync(0xffffffffu, mx, o), omy = __shfl_sync(0xffffffffu, my, o),
+                  omz = __shfl_sync(0xffffffffu, mz, o);
+      Cov3 oS;
+      oS.s00 = __shfl_sync(0xffffffffu, S.s00, o);
+      oS.s01 = __shfl_sync(0xffffffffu, S.s01, o);
+      oS.s02 = __shfl_sync(0xffffffffu, S.s02, o);
+      oS.s11 = __shfl_sync(0xffffffffu, S.s11, o);
+      oS.s12 = __shfl_sync(0xffffffffu, S.s12, o);
+      oS.s22 = __shfl_sync(0xffffffffu, S.s22, o);
+      const int og = warp * 32 + o;  // owner within the CTA
+      const float* shn = sh_s + og * KP;
+      float pg[4] = {0.f, 0.f, 0.f, 0.f};  // the pair's mean (3) and opacity gradients
+      double pS[6] = {0., 0., 0., 0., 0., 0.};
+      int seg = 0;  // rank of the pair among its owner's pairs of this round
+      float X = 0.f, Y = 0.f, Z = 0.f;
+      float vm[3] = {0.f, 0.f, 0.f};
+      bool cl[3] = {true, true, true};
+      if (has) {
+        const int rank = i - eo;
+        seg = i - max(eo, r0);
+        const int cc = (int)__fns(vo, 0, rank + 1);
+        const float* rp = v_screen + (s_row0[cc][warp] + __popc(s_word[cc][warp] & ((1u << o) - 1u))) * kRowF;
+        const float4 v0 = reinterpret_cast<const float4*>(rp)[0];
+        const float4 v1 = reinterpret_cast<const float4*>(rp)[1];
+        const float2 v2 = reinterpret_cast<const float2*>(rp)[4];
+        const Cam& k = scam[cc];
+        const float* R = k.R;
+        // camera point and the projection's gating decision in canonical arithmetic
+        float px, py, pz;
+        cam_point(k, omx, omy, omz, px, py, pz);
+        const float izc = div_(1.0f, pz);
+        const float u = mul(px, izc), v = mul(py, izc);
+        const bool clx = (u < -k.limx) || (u > k.limx);
+        const bool cly = (v < -k.limy) || (v > k.limy);
+        const float ux = fminf(fmaxf(u, -k.limx), k.limx), uy = fminf(fmaxf(v, -k.limy), k.limy);
+        // gradient arithmetic (any rounding order)
+        const float iz = 1.0f / pz, iz2 = iz * iz;
+        const float j00 = k.fx * iz, j02 = -j00 * ux, j11 = k.fy * iz, j12 = -j11 * uy;
+        float T[6];
 #pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        T[m] = j00 * R[m] + j02 * R[6 + m];
-        T[3 + m] = j11 * R[3 + m] + j12 * R[6 + m];
-      }
-      // conic -> 2D covariance -> (T, Sigma) in fp64: the terms are of size
-      // (f/z)^2 * |V2| and cancel down to small rotation/scale gradients
-      const double Sm[3][3] = {{S.s00, S.s01, S.s02}, {S.s01, S.s11, S.s12}, {S.s02, S.s12, S.s22}};
-      double Td[6];
-#pragma unroll
-      for (int m = 0; m < 6; ++m) Td[m] = T[m];
-      double TS[2][3];
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int m = 0; m < 3; ++m)
-          TS[r][m] = Td[3 * r] * Sm[0][m] + Td[3 * r + 1] * Sm[1][m] + Td[3 * r + 2] * Sm[2][m];
-      const double a = TS[0][0] * Td[0] + TS[0][1] * Td[1] + TS[0][2] * Td[2] + 0.3;
-      const double b = TS[0][0] * Td[3] + TS[0][1] * Td[4] + TS[0][2] * Td[5];
-      const double cq = TS[1][0] * Td[3] + TS[1][1] * Td[4] + TS[1][2] * Td[5] + 0.3;
-      // conic (c, -b, a)/det -> dilated covariance (a, b, c)
-      const double id = 1.0 / (a * cq - b * b), id2 = id * id;
-      const double vca = v0.z, vcb = v0.w, vcc = v1.x;
-      const double va = (-vca * cq * cq + vcb * b * cq - vcc * b * b) * id2;
-      const double vb = (2.0 * vca * b * cq - vcb * (a * cq + b * b) + 2.0 * vcc * a * b) * id2;
-      const double vc = (-vca * b * b + vcb * a * b - vcc * a * a) * id2;
-      const double hb = 0.5 * vb;
-      // dL/dT = 2 V2 T Sigma;  dL/dSigma += T^T V2 T
-      float GT[2][3];
-      double VT[2][3];
-#pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        GT[0][m] = (float)(2.0 * (va * TS[0][m] + hb * TS[1][m]));
-        GT[1][m] = (float)(2.0 * (hb * TS[0][m] + vc * TS[1][m]));
-        VT[0][m] = va * Td[m] + hb * Td[3 + m];
-        VT[1][m] = hb * Td[m] + vc * Td[3 + m];
-      }
-      gS[0] += Td[0] * VT[0][0] + Td[3] * VT[1][0];
-      gS[1] += Td[0] * VT[0][1] + Td[3] * VT[1][1];
-      gS[2] += Td[0] * VT[0][2] + Td[3] * VT[1][2];
-      gS[3] += Td[1] * VT[0][1] + Td[4] * VT[1][1];
-      gS[4] += Td[1] * VT[0][2] + Td[4] * VT[1][2];
-      gS[5] += Td[2] * VT[0][2] + Td[5] * VT[1][2];
-      // T = J R -> dL/dJ = dL/dT R^T (entries 00, 02, 11, 12)
-      const float gj00 = GT[0][0] * R[0] + GT[0][1] * R[1] + GT[0][2] * R[2];
-      const float gj02 = GT[0][0] * R[6] + GT[0][1] * R[7] + GT[0][2] * R[8];
-      const float gj11 = GT[1][0] * R[3] + GT[1][1] * R[4] + GT[1][2] * R[5];
-      const float gj12 = GT[1][0] * R[6] + GT[1][1] * R[7] + GT[1][2] * R[8];
-      float gx = 0.f, gy = 0.f;
-      float gz = -k.fx * iz2 * gj00 + k.fx * ux * iz2 * gj02 - k.fy * iz2 * gj11 + k.fy * uy * iz2 * gj12;
-      const float gux = -k.fx * iz * gj02, guy = -k.fy * iz * gj12;
-      if (!clx) { gx += gux * iz; gz -= gux * px * iz2; }
-      if (!cly) { gy += guy * iz; gz -= guy * py * iz2; }
-      const float vmx = v0.x, vmy = v0.y;
-      gx += vmx * k.fx * iz; gz -= vmx * k.fx * px * iz2;
-      gy += vmy * k.fy * iz; gz -= vmy * k.fy * py * iz2;
-      gz += v2.y;  // depth
-      gmu[0] += R[0] * gx + R[3] * gy + R[6] * gz;
-      gmu[1] += R[1] * gx + R[4] * gy + R[7] * gz;
-      gmu[2] += R[2] * gx + R[5] * gy + R[8] * gz;
-      go += v1.y;
-      // colour: clamp decisions in the forward's canonical arithmetic
-      float X = 0.f, Y = 0.f, Z = 0.f, il = 0.f;
-      if (DEG > 0) view_dir(k, mx, my, mz, X, Y, Z, il);
-      bool cl[3];
-      {
-        float bb[16];
-        sh_basis(DEG, X, Y, Z, bb);
-#pragma unroll
-        for (int ch = 0; ch < 3; ++ch) {
-          float acc = mul(shn[ch], bb[0]);
-#pragma unroll
-          for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], bb[kk]));
-          cl[ch] = !(add(acc, 0.5f) >= 0.0f);
+        for (int m = 0; m < 3; ++m) {
+          T[m] = j00 * R[m] + j02 * R[6 + m];
+          T[3 + m] = j11 * R[3 + m] + j12 * R[6 + m];
         }
+        // conic -> 2D covariance -> (T, Sigma) in fp64: the terms are of size
+        // (f/z)^2 * |V2| and cancel down to small rotation/scale gradients
+        const double Sm[3][3] = {{oS.s00, oS.s01, oS.s02}, {oS.s01, oS.s11, oS.s12}, {oS.s02, oS.s12, oS.s22}};
+        double Td[6];
+#pragma unroll
+        for (int m = 0; m < 6; ++m) Td[m] = T[m];
+        double TS[2][3];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int m = 0; m < 3; ++m)
+            TS[r][m] = Td[3 * r] * Sm[0][m] + Td[3 * r + 1] * Sm[1][m] + Td[3 * r + 2] * Sm[2][m];
+        const double a = TS[0][0] * Td[0] + TS[0][1] * Td[1] + TS[0][2] * Td[2] + 0.3;
+        const double b = TS[0][0] * Td[3] + TS[0][1] * Td[4] + TS[0][2] * Td[5];
+        const double cq = TS[1][0] * Td[3] + TS[1][1] * Td[4] + TS[1][2] * Td[5] + 0.3;
+        // conic (c, -b, a)/det -> dilated covariance (a, b, c)
+        const double id = 1.0 / (a * cq - b * b), id2 = id * id;
+        const double vca = v0.z, vcb = v0.w, vcc = v1.x;
+        const double va = (-vca * cq * cq + vcb * b * cq - vcc * b * b) * id2;
+        const double vb = (2.0 * vca * b * cq - vcb * (a * cq + b * b) + 2.0 * vcc * a * b) * id2;
+        const double vc = (-vca * b * b + vcb * a * b - vcc * a * a) * id2;
+        const double hb = 0.5 * vb;
+        // dL/dT = 2 V2 T Sigma;  dL/dSigma = T^T V2 T
+        float GT[2][3];
+        double VT[2][3];
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          GT[0][m] = (float)(2.0 * (va * TS[0][m] + hb * TS[1][m]));
+          GT[1][m] = (float)(2.0 * (hb * TS[0][m] + vc * TS[1][m]));
+          VT[0][m] = va * Td[m] + hb * Td[3 + m];
+          VT[1][m] = hb * Td[m] + vc * Td[3 + m];
+        }
+        pS[0] = Td[0] * VT[0][0] + Td[3] * VT[1][0];
+        pS[1] = Td[0] * VT[0][1] + Td[3] * VT[1][1];
+        pS[2] = Td[0] * VT[0][2] + Td[3] * VT[1][2];
+        pS[3] = Td[1] * VT[0][1] + Td[4] * VT[1][1];
+        pS[4] = Td[1] * VT[0][2] + Td[4] * VT[1][2];
+        pS[5] = Td[2] * VT[0][2] + Td[5] * VT[1][2];
+        // T = J R -> dL/dJ = dL/dT R^T (entries 00, 02, 11, 12)
+        const float gj00 = GT[0][0] * R[0] + GT[0][1] * R[1] + GT[0][2] * R[2];
+        const float gj02 = GT[0][0] * R[6] + GT[0][1] * R[7] + GT[0][2] * R[8];
+        const float gj11 = GT[1][0] * R[3] + GT[1][1] * R[4] + GT[1][2] * R[5];
+        const float gj12 = GT[1][0] * R[6] + GT[1][1] * R[7] + GT[1][2] * R[8];
+        float gx_ = 0.f, gy = 0.f;
+        float gz = -k.fx * iz2 * gj00 + k.fx * ux * iz2 * gj02 - k.fy * iz2 * gj11 + k.fy * uy * iz2 * gj12;
+        const float gux = -k.fx * iz * gj02, guy = -k.fy * iz * gj12;
+        if (!clx) { gx_ += gux * iz; gz -= gux * px * iz2; }
+        if (!cly) { gy += guy * iz; gz -= guy * py * iz2; }
+        const float vmx = v0.x, vmy = v0.y;
+        gx_ += vmx * k.fx * iz; gz -= vmx * k.fx * px * iz2;
+        gy += vmy * k.fy * iz; gz -= vmy * k.fy * py * iz2;
+        gz += v2.y;  // depth
+        pg[0] = R[0] * gx_ + R[3] * gy + R[6] * gz;
+        pg[1] = R[1] * gx_ + R[4] * gy + R[7] * gz;
+        pg[2] = R[2] * gx_ + R[5] * gy + R[8] * gz;
+        pg[3] = v1.y;
+        // colour: the clamp decisions of the forward.  The sum is taken in
+        // any order first; only where 0.5 + sum lies within the owner's
+        // margin (ten times the rounding bound of either order) of zero is it
+        // redone in the forward's canonical order, so the decision is always
+        // the forward's
+        float il = 0.f;
+        if (DEG > 0) view_dir(k, omx, omy, omz, X, Y, Z, il);
+        {
+          float bb[16];
+          sh_basis(DEG, X, Y, Z, bb);
+#pragma unroll
+          for (int ch = 0; ch < 3; ++ch) {
+            float f = 0.5f;
+#pragma unroll
+            for (int kk = 0; kk < K; ++kk) f = fmaf(shn[3 * kk + ch], bb[kk], f);
+            bool c = !(f >= 0.0f);
+            if (fabsf(f) <= s_margin[og][ch]) {
+              float acc = mul(shn[ch], bb[0]);
+#pragma unroll
+              for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], bb[kk]));
+              c = !(add(acc, 0.5f) >= 0.0f);
+            }
+            cl[ch] = c;
+          }
+        }
+        const float vr[3] = {v1.z, v1.w, v2.x};
+#pragma unroll
+        for (int ch = 0; ch < 3; ++ch) vm[ch] = cl[ch] ? 0.0f : vr[ch];
+        if (DEG > 0) {
+          float vdir[3];
+          sh_dir_grads<DEG>(X, Y, Z, shn, vm, vdir);
+          const float dd = X * vdir[0] + Y * vdir[1] + Z * vdir[2];
+          pg[0] += (vdir[0] - X * dd) * il;
+          pg[1] += (vdir[1] - Y * dd) * il;
+          pg[2] += (vdir[2] - Z * dd) * il;
+        }
+        // the owner's first pair of the round adds its SH coefficient
+        // gradients now; the others wait their turn below
+        if (seg == 0) sh_coef_grads<DEG>(X, Y, Z, vm, cl, gsh_s + og * KP);
       }
-      const float vr[3] = {v1.z, v1.w, v2.x};
-      float vdir[3] = {0.f, 0.f, 0.f};
-      sh_grads<DEG>(X, Y, Z, shn, vr, cl, gsh, vdir);
-      if (DEG > 0) {
-        const float dd = X * vdir[0] + Y * vdir[1] + Z * vdir[2];
-        gmu[0] += (vdir[0] - X * dd) * il;
-        gmu[1] += (vdir[1] - Y * dd) * il;
-        gmu[2] += (vdir[2] - Z * dd) * il;
+      // an owner's further pairs of this round, one rank at a time (each
+      // rank holds at most one pair per owner, so no two lanes of a rank
+      // touch the same row), in camera order
+      const int maxseg = __reduce_max_sync(0xffffffffu, has ? (unsigned)seg : 0u);
+      for (int j = 1; j <= maxseg; ++j) {
+        __syncwarp();
+        if (has && seg == j) sh_coef_grads<DEG>(X, Y, Z, vm, cl, gsh_s + og * KP);
       }
+      // the pairs' sums to their owners, added in camera order
+      reinterpret_cast<float4*>(&s_pf[warp][lane][0])[0] = make_float4(pg[0], pg[1], pg[2], pg[3]);
+#pragma unroll
+      for (int m = 0; m < 6; ++m) s_pd[warp][lane][m] = pS[m];
+      __syncwarp();
+      const int l0 = max(excl, r0) - r0, l1 = min(excl + nv, r0 + 32) - r0;
+      for (int l = l0; l < l1; ++l) {
+        const float4 f = reinterpret_cast<const float4*>(&s_pf[warp][l][0])[0];
+        gmu[0] += f.x;
+        gmu[1] += f.y;
+        gmu[2] += f.z;
+        go += f.w;
+#pragma unroll
+        for (int m = 0; m < 6; ++m) gS[m] += s_pd[warp][l][m];
+      }
+      __syncwarp();
     }
   }
   if (valid) {
+    // the rotation and scales again (read back rather than kept live across
+    // the camera rounds)
+    const float4 q4 = reinterpret_cast<const float4*>(quats)[n];
+    const float s0 = scales[3 * n], s1 = scales[3 * n + 1], s2 = scales[3 * n + 2];
+    const QuatRot qr = quat_rot(q4.x, q4.y, q4.z, q4.w);
     // Sigma = M M^T: dL/dM = 2 gS M, M = R_q diag(s)  (fp64, see above)
     const double Gs[3][3] = {{gS[0], gS[1], gS[2]}, {gS[1], gS[3], gS[4]}, {gS[2], gS[4], gS[5]}};
     const double sv[3] = {s0, s1, s2};
@@ -650,13 +791,15 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
       if (q < 3) vmax[4] = fmaxf(vmax[4], fabsf(x)); else vmax[5] = fmaxf(vmax[5], fabsf(x));
     }
     gq_cta_max(vmax, s_gq_wmax, s_gq_amax);
-    float scale[kGqAttr];
+    float scale[kGqAttr], iscale[kGqAttr];
     gq_exchange(s_gq_amax, scale);  // the cluster barrier also orders the gsh_s updates above
+#pragma unroll
+    for (int a = 0; a < kGqAttr; ++a) iscale[a] = scale[a] > 0.0f ? 1.0f / scale[a] : 0.0f;
     if (valid) {
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int i = 0; i < kW[a]; ++i) gqa.code[a][kW[a] * n + i] = gq_code(gx[kOff[a] + i], scale[a]);
+        for (int i = 0; i < kW[a]; ++i) gqa.code[a][kW[a] * n + i] = gq_code(gx[kOff[a] + i], iscale[a]);
     }
     if (vec) {
       // 16-byte stores of eight codes each, the same vectors as the loads
@@ -669,10 +812,10 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
           int16_t c;
           if (v < kDcV) {
             const int e = 8 * v + u, gi = e / 3;
-            c = gq_code(gsh_s[gi * KP + (e - 3 * gi)], scale[4]);
+            c = gq_code(gsh_s[gi * KP + (e - 3 * gi)], iscale[4]);
           } else {
             const int e = 8 * (v - kDcV) + u, gi = e / (K3 - 3 > 0 ? K3 - 3 : 1);
-            c = gq_code(gsh_s[gi * KP + 3 + (e - (K3 - 3) * gi)], scale[5]);
+            c = gq_code(gsh_s[gi * KP + 3 + (e - (K3 - 3) * gi)], iscale[5]);
           }
           w[u >> 1] |= (uint32_t)(uint16_t)c << (16 * (u & 1));
         }
@@ -684,8 +827,8 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
         const int gi = f / K3, q = f - gi * K3;
         const int64_t m = n0 + gi;
         const float x = gsh_s[gi * KP + q];
-        if (q < 3) gqa.code[4][3 * m + q] = gq_code(x, scale[4]);
-        else gqa.code[5][(K3 - 3) * m + (q - 3)] = gq_code(x, scale[5]);
+        if (q < 3) gqa.code[4][3 * m + q] = gq_code(x, iscale[4]);
+        else gqa.code[5][(K3 - 3) * m + (q - 3)] = gq_code(x, iscale[5]);
       }
     }
     if ((blk & 1) == 0 && threadIdx.x < kGqAttr) {

@@ -1,12 +1,18 @@
 // Stable LSD radix sort of (key, value) pairs on the (tile_id << 32 | depth)
 // keys ("Spirula Studio VRAM deep-dive", buffer-cost table: double-buffered
 // isect.ids_a/b; the reference's CUDA backend calls a library sort, this one is
-// written here).  8-bit digits over the 31 depth bits (depth > 0, so bit 31 is
-// zero) and over the bits the tile ids need.
+// written here).  8-bit digits: the four bytes of the depth and the bytes the
+// tile ids need.  A digit that is the same in every key (for example the top
+// byte of depths whose exponents share their high bits) cannot change the
+// order, so its pass is skipped; the histograms show which ones, and the
+// device keeps the plan, so the host launches the full plan's kernels and
+// the skipped ones return at once.
 //
 //   k_hist_all   one read of the keys: the global digit histogram of every pass
 //                (a permutation does not change them)
-//   k_bases      exclusive scan of each pass's 256 counts
+//   k_plan       which passes run (a digit whose histogram holds every key in
+//                one bin is skipped), and the exclusive scan of each running
+//                pass's 256 counts
 //   k_onesweep   per pass, one kernel: each CTA takes the next 4096-key tile by
 //                ticket, ranks its keys stably among equal digits (warp match +
 //                per-warp counters), publishes its digit counts and looks back
@@ -20,6 +26,7 @@
 // already running and never waits on a later tile.
 #include <algorithm>
 #include <mutex>
+#include <string>
 #include <utility>
 
 #include "ss_common.cuh"
@@ -38,8 +45,10 @@ constexpr uint64_t kFlagPre = 2ull << 54;
 constexpr uint64_t kValMask = (1ull << 54) - 1;
 constexpr int kSpinLimit = 1 << 20;
 
-struct SortPlan {
-  int passes;
+// The passes that run, written by k_plan: shift[k] is the key bit of the k-th
+// running pass's digit, count the number of running passes.
+struct DevPlan {
+  int count;
   int shift[kMaxPasses];
 };
 
@@ -98,25 +107,40 @@ ss_status launch_hist(unsigned grid, cudaStream_t st, const uint64_t* keys, int6
   return cuda_status(cudaGetLastError(), "radix histogram");
 }
 
-// hist[p][d] -> exclusive scan over d, in place (one CTA of 256 threads).
-__global__ __launch_bounds__(kRadix) void k_bases(uint32_t* __restrict__ hist, int passes) {
+// Which passes run and their digit bases (one CTA of 256 threads): pass p is
+// skipped when one bin of its histogram holds all n keys; the running passes'
+// histograms are scanned (exclusive) and moved to the front, in order, so
+// running pass k reads hist[k] and the digit at key bit plan->shift[k].
+__global__ __launch_bounds__(kRadix) void k_plan(uint32_t* __restrict__ hist, int passes, int64_t n,
+                                                 DevPlan* __restrict__ plan) {
   __shared__ uint32_t wt[kRadix / 32];
+  __shared__ int s_full;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int k = 0;
   for (int p = 0; p < passes; ++p) {
-    const uint32_t v = hist[p * kRadix + threadIdx.x];
-    uint32_t inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += x;
-    }
-    if (lane == 31) wt[warp] = inc;
+    if (threadIdx.x == 0) s_full = 0;
     __syncthreads();
-    uint32_t before = 0;
-    for (int w = 0; w < warp; ++w) before += wt[w];
-    hist[p * kRadix + threadIdx.x] = before + inc - v;
+    const uint32_t v = hist[p * kRadix + threadIdx.x];
+    if ((int64_t)v == n) s_full = 1;
+    __syncthreads();
+    if (s_full == 0) {
+      uint32_t inc = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+      }
+      if (lane == 31) wt[warp] = inc;
+      __syncthreads();
+      uint32_t before = 0;
+      for (int w = 0; w < warp; ++w) before += wt[w];
+      hist[k * kRadix + threadIdx.x] = before + inc - v;  // k <= p, and row p was read above
+      if (threadIdx.x == 0) plan->shift[k] = p < 4 ? 8 * p : 32 + 8 * (p - 4);
+      ++k;
+    }
     __syncthreads();
   }
+  if (threadIdx.x == 0) plan->count = k;
 }
 
 struct OnesweepSmem {
@@ -136,12 +160,14 @@ __device__ __forceinline__ uint64_t ld_status(const uint64_t* p) {
 __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __restrict__ kin,
                                                            const uint32_t* __restrict__ vin,
                                                            uint64_t* __restrict__ kout, uint32_t* __restrict__ vout,
-                                                           int64_t n, int shift, uint64_t epoch,
-                                                           const uint32_t* __restrict__ bases,
+                                                           int64_t n, int pass, const DevPlan* __restrict__ plan,
+                                                           uint64_t epoch, const uint32_t* __restrict__ bases,
                                                            uint64_t* __restrict__ status,
                                                            uint32_t* __restrict__ ticket, uint32_t* __restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   OnesweepSmem& S = *reinterpret_cast<OnesweepSmem*>(smem_raw);
+  if (pass >= plan->count) return;  // a skipped digit: nothing moves
+  const int shift = plan->shift[pass];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) S.tile = atomicAdd(ticket, 1u);
   for (int i = threadIdx.x; i < kSortWarps * kRadix; i += kSortThreads) (&S.wcnt[0][0])[i] = 0;
@@ -264,8 +290,10 @@ __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __res
 }
 
 // tile_off[t] = first sorted index whose tile id is >= t; tile_off[ntiles] = n.
-__global__ void k_tile_ranges(const uint64_t* __restrict__ keys, int64_t n, int64_t ntiles,
-                              int64_t* __restrict__ tile_off) {
+// The sorted keys are in keys_b after an odd number of running passes.
+__global__ void k_tile_ranges(const uint64_t* __restrict__ keys_a, const uint64_t* __restrict__ keys_b, int64_t n,
+                              int64_t ntiles, const DevPlan* __restrict__ plan, int64_t* __restrict__ tile_off) {
+  const uint64_t* keys = (plan->count & 1) ? keys_b : keys_a;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i > n) return;
   const int64_t prev = i == 0 ? -1 : (int64_t)(keys[i - 1] >> 32);
@@ -282,13 +310,15 @@ int tile_bits(int64_t ntiles) {
 int sort_passes(int64_t ntiles) { return 4 + (tile_bits(ntiles) + 7) / 8; }
 
 // Scratch layout: hist [kMaxPasses][256] u32 | tickets [kMaxPasses] u32 |
-// error flag u32 | look-back status [tiles][256] u64.
-size_t sort_status_offset() { return align_up(kMaxPasses * kRadix * 4 + kMaxPasses * 4 + 4, 256); }
+// error flag u32 | plan | look-back status [tiles][256] u64.
+constexpr size_t sort_plan_offset() { return align_up(kMaxPasses * kRadix * 4 + kMaxPasses * 4 + 4, 16); }
+constexpr size_t sort_status_offset() { return align_up(sort_plan_offset() + sizeof(DevPlan), 256); }
 
-size_t sort_temp_bytes(int64_t n) {
-  const int64_t tiles = ceil_div(max64(n, 1), kSortTile);
-  return sort_status_offset() + (size_t)tiles * kRadix * 8;
+constexpr size_t sort_scratch_bytes(int64_t n) {
+  return sort_status_offset() + (size_t)ceil_div(n > 1 ? n : 1, kSortTile) * kRadix * 8;
 }
+
+size_t sort_temp_bytes(int64_t n) { return sort_scratch_bytes(n); }
 
 }  // namespace ss
 
@@ -306,8 +336,7 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   }
   const Geo g = geometry(*dims);
   cudaStream_t st = as_stream(stream);
-  const int passes = sort_passes(g.n_tiles);
-  *result_in_b_out = passes & 1;
+  *result_in_b_out = 0;
   if (n == 0) return cuda_status(cudaMemsetAsync(tile_off, 0, sizeof(int64_t) * (g.n_tiles + 1), st), "memset");
   if (!keys_a || !vals_a || !keys_b || !vals_b) return invalid("null keys/vals");
   if (!temp || temp_bytes < sort_temp_bytes(n)) return invalid("temp too small");
@@ -320,12 +349,13 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   uint32_t* hist = reinterpret_cast<uint32_t*>(tb);
   uint32_t* tickets = hist + kMaxPasses * kRadix;
   uint32_t* err = tickets + kMaxPasses;
+  DevPlan* dplan = reinterpret_cast<DevPlan*>(tb + sort_plan_offset());
   uint64_t* status = reinterpret_cast<uint64_t*>(tb + sort_status_offset());
   s = cuda_status(cudaMemsetAsync(temp, 0, sort_status_offset() + (size_t)tiles * kRadix * 8, st), "memset");
   if (s) return s;
-  SortPlan plan{};
-  plan.passes = passes;
-  for (int p = 0; p < passes; ++p) plan.shift[p] = p < 4 ? 8 * p : 32 + 8 * (p - 4);
+  // the full plan: every byte of the depth and the bytes of the tile ids;
+  // k_plan drops the bytes that do not vary
+  const int passes = sort_passes(g.n_tiles);
   const unsigned hgrid = (unsigned)min64(tiles, 148 * 8);
   switch (passes) {
     case 4: s = launch_hist<4>(hgrid, st, keys_a, n, hist); break;
@@ -335,8 +365,8 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
     default: s = launch_hist<8>(hgrid, st, keys_a, n, hist); break;
   }
   if (s) return s;
-  k_bases<<<1, kRadix, 0, st>>>(hist, passes);
-  s = cuda_status(cudaGetLastError(), "radix histogram");
+  k_plan<<<1, kRadix, 0, st>>>(hist, passes, n, dplan);
+  s = cuda_status(cudaGetLastError(), "radix plan");
   if (s) return s;
   uint64_t* kin = keys_a;
   uint32_t* vin = vals_a;
@@ -345,22 +375,27 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   for (int p = 0; p < passes; ++p) {
     const uint64_t epoch = (uint64_t)(p + 1) << 56;
     k_onesweep<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
-        kin, vin, kout, vout, n, plan.shift[p], epoch, hist + p * kRadix, status, tickets + p, err);
+        kin, vin, kout, vout, n, p, dplan, epoch, hist + p * kRadix, status, tickets + p, err);
     s = cuda_status(cudaGetLastError(), "radix pass");
     if (s) return s;
     std::swap(kin, kout);
     std::swap(vin, vout);
   }
   const unsigned grid = (unsigned)ceil_div(n + 1, 256);
-  k_tile_ranges<<<grid, 256, 0, st>>>(kin, n, g.n_tiles, tile_off);
+  k_tile_ranges<<<grid, 256, 0, st>>>(keys_a, keys_b, n, g.n_tiles, dplan, tile_off);
   s = cuda_status(cudaGetLastError(), "tile ranges");
   if (s) return s;
-  uint32_t herr = 0;
-  s = cuda_status(cudaMemcpyAsync(&herr, err, 4, cudaMemcpyDeviceToHost, st), "copy sort flag");
+  // the error flag and the plan's pass count, read together
+  uint32_t hbuf[2] = {0u, 0u};
+  s = cuda_status(cudaMemcpyAsync(&hbuf[0], err, 4, cudaMemcpyDeviceToHost, st), "copy sort flag");
+  if (s) return s;
+  int count = 0;
+  s = cuda_status(cudaMemcpyAsync(&count, &dplan->count, sizeof(int), cudaMemcpyDeviceToHost, st), "copy sort plan");
   if (s) return s;
   s = cuda_status(cudaStreamSynchronize(st), "sort");
   if (s) return s;
-  if (herr) {
+  *result_in_b_out = count & 1;
+  if (hbuf[0]) {
     set_error("ss_sort_isects: look-back wait exceeded its limit");
     return SS_ERR_DEVICE_CHECK;
   }
@@ -368,22 +403,54 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
 }
 
 // ---------------------------------------------------------------------------
-// Allocation-free variant.  Some callers cannot call cudaMalloc at all (for
-// example code running inside another runtime's allocator callbacks, or a
-// host that hands out only fixed device buffers), so this entry point keeps
-// the sort's scratch in a file-scope device array instead of a caller buffer.
+// Allocation-free variant.  Some callers cannot call cudaMalloc at all: code
+// that runs inside another runtime's allocator callbacks or memory-pool hooks
+// (a nested cudaMalloc would re-enter that allocator), or a host that hands
+// out only fixed, pre-sized device buffers.  This entry point keeps the
+// sort's scratch in a file-scope device array instead of a caller buffer.
 // The array is part of the loaded module: every GPU that loads the library
 // holds it until the process exits.
 
 namespace ss {
 
 constexpr size_t kNoAllocScratchBytes = size_t(24) << 20;  // 24 MiB
+// Largest key count whose scratch fits: whole 4096-key tiles of look-back
+// status after the fixed header.
+constexpr int64_t kNoAllocMaxKeys =
+    (int64_t)((kNoAllocScratchBytes - sort_status_offset()) / (kRadix * 8)) * kSortTile;
+static_assert(sort_scratch_bytes(kNoAllocMaxKeys) <= kNoAllocScratchBytes, "limit must fit the scratch");
+static_assert(sort_scratch_bytes(kNoAllocMaxKeys + 1) > kNoAllocScratchBytes, "limit must be the largest that fits");
+
 __device__ __align__(256) unsigned char g_sort_scratch[kNoAllocScratchBytes];
 
 // Host code may not use g_sort_scratch as a device address: the symbol's host
-// side is only a stand-in.  The device address is looked up once per device.
+// side is only a stand-in.  The device address is looked up with
+// cudaGetSymbolAddress once per device and context (the module, and so the
+// array, is loaded again in a new context, e.g. after cudaDeviceReset).
+typedef int (*CtxGetCurrentFn)(void**);
 std::mutex g_scratch_mu;
-void* g_scratch_addr[256] = {};
+struct ScratchSlot {
+  void* ctx;
+  void* addr;
+};
+ScratchSlot g_scratch_slot[256] = {};
+
+// The context current on this thread (NULL before the runtime has made one).
+ss_status current_context(void** ctx) {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    ss_status s = cuda_status(cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q),
+                              "cudaGetDriverEntryPoint");
+    if (s) return s;
+    if (!f || q != cudaDriverEntryPointSuccess) return invalid("cuCtxGetCurrent not found");
+    fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  }
+  *ctx = nullptr;
+  if (fn(ctx) != 0) *ctx = nullptr;
+  return SS_OK;
+}
 
 ss_status noalloc_scratch(void** out) {
   int dev = 0;
@@ -391,13 +458,21 @@ ss_status noalloc_scratch(void** out) {
   if (s) return s;
   if (dev < 0 || dev >= 256) return invalid("device ordinal out of range");
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  void* ctx = nullptr;
+  s = current_context(&ctx);
+  if (s) return s;
+  ScratchSlot& slot = g_scratch_slot[dev];
+  if (!ctx || slot.ctx != ctx || !slot.addr) {
+    // the lookup also makes the runtime's context current if none was
     void* p = nullptr;
     s = cuda_status(cudaGetSymbolAddress(&p, g_sort_scratch), "cudaGetSymbolAddress");
     if (s) return s;
-    g_scratch_addr[dev] = p;
+    s = current_context(&ctx);
+    if (s) return s;
+    slot.ctx = ctx;
+    slot.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = slot.addr;
   return SS_OK;
 }
 
@@ -407,8 +482,10 @@ extern "C" ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_
                                             uint64_t* keys_b, uint32_t* vals_b, int64_t n, int64_t* tile_off,
                                             int* result_in_b_out, void* stream) {
   if (n < 0) return invalid("n < 0");
-  if (n > 0 && sort_temp_bytes(n) > kNoAllocScratchBytes) {
-    set_error("ss_sort_isects_noalloc: n exceeds the 24 MiB static scratch (at most 50311168 keys)");
+  if (n > kNoAllocMaxKeys) {
+    set_error("ss_sort_isects_noalloc: n = " + std::to_string(n) + " exceeds the " +
+              std::to_string(kNoAllocScratchBytes >> 20) + " MiB static scratch (at most " +
+              std::to_string(kNoAllocMaxKeys) + " keys)");
     return SS_ERR_INVALID_ARG;
   }
   void* scratch = nullptr;

@@ -74,8 +74,8 @@ inline ss_status invalid(const char* what) {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
-inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+constexpr size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
 // Asks L2 to fetch [p, p + bytes) ahead of use (bulk prefetch, no data
 // returned to the SM; bytes is rounded down to the 16-byte granule).

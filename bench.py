@@ -60,19 +60,29 @@ def source_digest(paths) -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(stage: str, config: int, n):
+def recorded_traffic(stage: str, config: int, n, units=None):
     """DRAM bytes per launch of the stage's kernel from a recorded ncu capture,
     or None when there is none, it was taken on another workload, or the
-    kernel's sources changed since."""
+    kernel's sources changed since.  A capture of a smaller case of the same
+    workload (fewer Gaussians) is scaled to this launch by the units the
+    kernel processes (record["units"]: the unit's name and its count in the
+    capture; `units` maps names to this run's counts), when the record says
+    that its traffic grows in proportion to them."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
         rec = t[stage]
-        if t["_workload"] != {"config": config, "n": n}:
-            return None
+        wl = rec.get("workload", t["_workload"])
         if source_digest(rec["sources"]) != rec["sha256"]:
             return None
-        return float(rec["dram_bytes_per_launch"])
+        if wl == {"config": config, "n": n}:
+            return float(rec["dram_bytes_per_launch"])
+        if wl.get("config") != config or "units" not in rec or not units:
+            return None
+        name, captured = rec["units"]["name"], float(rec["units"]["value"])
+        if name not in units or captured <= 0:
+            return None
+        return float(rec["dram_bytes_per_launch"]) * float(units[name]) / captured
     except Exception:
         return None
 
@@ -129,13 +139,17 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- roofline model
-def stage_model(d, K, nnz, n_isects, passes, n_tiles, work):
+def stage_model(d, K, nnz, n_isects, passes, n_tiles, work, n_seen=None):
     """Algorithmic bytes (HBM) and FP32 instruction counts per call.
 
-    bytes: every input read once and every output written once, at the
-    stage's own layout; instr: FP32-pipe instructions of the canonical
-    per-item sequences (counted from the source), for the ALU-bound stages.
+    bytes: every input the stage needs read once and every output written
+    once, at the stage's own layout (the SH coefficients only of the n_seen
+    Gaussians some camera sees: the colour of the others is never
+    evaluated); instr: FP32-pipe instructions of the canonical per-item
+    sequences (counted from the source), for the ALU-bound stages.
     """
+    if n_seen is None:
+        n_seen = d.N
     C, N, W, H = d.C, d.N, d.W, d.H
     P = C * N
     X = C * W * H
@@ -143,19 +157,27 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work):
     par = 40  # means 12 + quats 16 + scales 12
     shb = 12 * K
     m = {}
-    m["project_packed"] = dict(bytes=par * N + P / 8 + P / 32 + P / 16 + (par + 4 + shb) * N + (row + 8) * nnz,
-                               instr=P * 140.0 + nnz * 160.0)
+    m["project_packed"] = dict(bytes=par * N + P / 8 + P / 32 + P / 16 + (par + 4) * N + shb * n_seen
+                               + (row + 8 + 4) * nnz, instr=P * 140.0 + nnz * 160.0)
     m["intersect_tiles"] = dict(bytes=8 * nnz * 2 + 8 * nnz + 4 * nnz + 12 * n_isects, instr=0.0)
-    m["sort_isects"] = dict(bytes=n_isects * (8 + 24) * passes + 8 * (n_tiles + 1), instr=0.0)
+    # histogram (one read), 12 B read + 12 B written per key per digit pass
+    # that runs, tile offsets
+    m["sort_isects"] = dict(bytes=n_isects * (8 + 24 * passes) + 8 * (n_tiles + 1), instr=0.0)
     # per-pixel FP32 instructions of the canonical sequences: 11 per evaluated
     # entry (offsets, sigma, tests), 16 per exp (range reduction, degree-7
     # polynomial, scaling, alpha), 7 per composite; backward: 11 per replayed
     # entry, 17 per exp, 30 per contributing entry (T recovery, nine gradients)
+    # second model, the measurement plan's FLOP counts: forward E * (12 + 1
+    # exp) + C * 10 over the evaluated entries E and composited entries C; the
+    # backward about three times that on the replayed entries (against 2
+    # FLOPs per FMA lane per clock)
     m["rasterize_fwd"] = dict(bytes=n_isects * (4 + row) + X * 20 + 8 * (n_tiles + 1),
-                              instr=work["evals"] * 11.0 + work["exps"] * 16.0 + work["comps"] * 7.0)
+                              instr=work["evals"] * 11.0 + work["exps"] * 16.0 + work["comps"] * 7.0,
+                              flops=work["evals"] * 13.0 + work["comps"] * 10.0)
     m["rasterize_bwd"] = dict(bytes=n_isects * (4 + row) + X * 24 + nnz * row * 2,
-                              instr=work["bwd_evals"] * 11.0 + work["bwd_exps"] * 17.0 + work["comps"] * 30.0)
-    m["project_bwd"] = dict(bytes=(par + shb) * N + row * nnz + P / 8 + P / 16 + (par + 4 + shb) * N,
+                              instr=work["bwd_evals"] * 11.0 + work["bwd_exps"] * 17.0 + work["comps"] * 30.0,
+                              flops=3.0 * (work["bwd_evals"] * 13.0 + work["comps"] * 10.0))
+    m["project_bwd"] = dict(bytes=par * N + shb * n_seen + row * nnz + P / 8 + P / 16 + (par + 4 + shb) * N,
                             instr=nnz * 700.0)
     # fused with Adam: parameters, activated copies and both moments read and
     # written once, no gradient arrays
@@ -173,6 +195,11 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work):
 def fp32_peak_instr_per_s(sm_mhz: float) -> float:
     # 148 SMs x 128 FP32 lanes, one instruction per lane per clock
     return 148 * 128 * sm_mhz * 1e6
+
+
+def fp32_peak_flops(sm_mhz: float) -> float:
+    # the same lanes counted as 2 FLOPs per FMA
+    return 2.0 * fp32_peak_instr_per_s(sm_mhz)
 
 
 # ---------------------------------------------------------------------------- ranks
@@ -292,9 +319,10 @@ def run_ours(args):
     def _timed_forward(ev):
         cams, means, quats, scales, opac, sh = inputs
         nnz = ss.ss_project_packed(d, cams, means, quats, scales, opac, sh, step.mask, step.block_count,
-                                   step.block_off, step.screen, step.aabb16, step.cap_rows, step.temp_project)
+                                   step.block_off, step.screen, step.aabb16, step.row_depth, step.cap_rows,
+                                   step.temp_project)
         ev[1].record(st)
-        n = ss.ss_intersect_tiles(d, step.screen, step.aabb16, step.block_off, nnz, step.isect_off, step.keys_a,
+        n = ss.ss_intersect_tiles(d, step.row_depth, step.aabb16, step.block_off, nnz, step.isect_off, step.keys_a,
                                   step.vals_a, step.cap_isects, step.temp_isect)
         ev[2].record(st)
         in_b = ss.ss_sort_isects(d, step.keys_a, step.vals_a, step.keys_b, step.vals_b, n, step.temp_sort,
@@ -406,9 +434,10 @@ def run_ours(args):
         return
 
     peaks = load_peaks()
-    passes = ss.sort_passes(d)
+    passes = ss.sort_passes_for(step.keys[: step.n_isects], d)
+    n_seen = ss.seen_gaussians(d, step.mask)
     model = stage_model(d, (d.sh_degree + 1) ** 2, step.nnz, step.n_isects, passes, ss.size(d, ss.SIZE_N_TILES),
-                        work)
+                        work, n_seen)
     sm_mhz = clocks["sm_mhz"] or peaks["sm_max_mhz"]
     stages = {}
     for nm in names:
@@ -421,23 +450,36 @@ def run_ours(args):
         f_alu = alu / fp32_peak_instr_per_s(sm_mhz) if ins else 0.0
         stages[nm] = dict(ms=round(stage_ms[nm], 4), hbm_gbs=round(hbm, 1), hbm_frac=round(f_hbm, 4),
                           alu_frac=round(f_alu, 4), bound="alu" if f_alu > f_hbm else "hbm")
+        if "flops" in model[nm]:
+            stages[nm]["flop_frac"] = round(model[nm]["flops"] / t / fp32_peak_flops(sm_mhz), 4)
     # whole-step fraction: sum over stages of the roofline time (the slower of
     # bytes at the HBM peak and FP32 instructions at the FP32 peak) over the
     # sum of measured stage times
     t_roof = sum(max(model[nm]["bytes"] / (peaks["hbm_gbs"] * 1e9),
                      model[nm]["instr"] / fp32_peak_instr_per_s(sm_mhz)) for nm in names)
     step_frac = t_roof / (sum(stage_ms.values()) / 1e3)
+    # the same with the rasterizers priced by the FLOP model
+    t_roof_fl = sum(max(model[nm]["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                        model[nm].get("flops", model[nm]["instr"] * 2.0) / fp32_peak_flops(sm_mhz)) for nm in names)
+    step_frac_fl = t_roof_fl / (sum(stage_ms.values()) / 1e3)
     dom = max(names, key=lambda k: stage_ms[k])
+    units = dict(N=d.N, nnz=step.nnz, n_isects=step.n_isects, pixels=d.C * d.W * d.H)
     sd = stages[dom]
     if sd["bound"] == "hbm":
         roof = dict(bound="hbm", achieved=sd["hbm_gbs"], peak=peaks["hbm_gbs"], unit="GB/s", frac=sd["hbm_frac"],
-                    traffic=recorded_traffic(dom, args.config, args.n), kernel=dom, peak_source=peaks["src"])
+                    traffic=recorded_traffic(dom, args.config, args.n, units), kernel=dom, peak_source=peaks["src"])
     else:
         ach = model[dom]["instr"] / (stage_ms[dom] / 1e3) / 1e12
         pk = fp32_peak_instr_per_s(sm_mhz) / 1e12
         roof = dict(bound="alu", achieved=round(ach, 3), peak=round(pk, 3), unit="T FP32 instr/s",
-                    frac=round(ach / pk, 4), traffic=recorded_traffic(dom, args.config, args.n), kernel=dom,
-                    peak_source=f"148 SMs x 128 FP32 lanes x {sm_mhz:.0f} MHz (median SM clock under load)")
+                    frac=round(ach / pk, 4), traffic=recorded_traffic(dom, args.config, args.n, units), kernel=dom,
+                    peak_source=f"148 SMs x 128 FP32 lanes x {sm_mhz:.0f} MHz (median SM clock under load)",
+                    model="FP32 instructions of the canonical per-pixel sequences")
+        if "flops" in model[dom]:
+            fa = model[dom]["flops"] / (stage_ms[dom] / 1e3) / 1e12
+            fp = fp32_peak_flops(sm_mhz) / 1e12
+            roof["flop_model"] = dict(achieved=round(fa, 3), peak=round(fp, 3), unit="TFLOP/s", frac=round(fa / fp, 4),
+                                      model="E * (12 + 1 exp) + C * 10 per pass, x3 for the backward")
     launches = ss.launches_per_step(d, step.nnz, step.n_isects) * args.steps
     out_work = dict(work)
     out = dict(metric=METRIC, value=job_throughput(step.n_isects, world, ms), unit="isects/s", n_gpus=world,
@@ -446,12 +488,13 @@ def run_ours(args):
                config=dict(workload=sc.name if args.n is None else f"{sc.name}, N overridden to {d.N}",
                            C=d.C, N=d.N, W=d.W, H=d.H,
                            sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
-                           sort_passes=passes, l2="inputs larger than L2 (3.5 GB parameters), no flush",
+                           sort_passes=passes, gaussians_seen=n_seen, l2="inputs larger than L2 (3.5 GB parameters), no flush",
                            parallelism=f"replicas x{world}", depth_and_background=bool(args.depth_bg),
                            fused_adam=bool(args.adam), grad_quant=bool(args.grad_quant)),
                pairs_per_s=world * d.C * d.N / (ms / 1e3),
                pixel_gaussian_evals_per_s=world * work["evals"] / (stage_ms["rasterize_fwd"] / 1e3),
-               step_roofline_frac=round(step_frac, 4), raster_work=out_work, stages=stages, roofline=roof,
+               step_roofline_frac=round(step_frac, 4), step_roofline_frac_flop_model=round(step_frac_fl, 4),
+               raster_work=out_work, stages=stages, roofline=roof,
                clocks=clocks,
                e2e=e2e, gpu_launches=launches)
     if not args.no_cpu_baseline:

@@ -14,6 +14,7 @@ void set_error(const std::string& msg) { g_last_error = msg; }
 size_t sort_temp_bytes(int64_t n);
 size_t isect_temp_bytes(int64_t nnz);
 size_t tile_order_temp_bytes();
+size_t project_temp_bytes(const Geo& g);
 
 }  // namespace ss
 
@@ -37,7 +38,7 @@ extern "C" size_t ss_workspace_bytes(const ss_dims* dims, int which, int64_t cou
   if (!dims_ok(dims)) return 0;
   const Geo g = geometry(*dims);
   switch (which) {
-    case SS_WS_PROJECT: return scan_temp_bytes(max64(g.mask_blocks, 1));
+    case SS_WS_PROJECT: return project_temp_bytes(g);
     case SS_WS_INTERSECT: return isect_temp_bytes(max64(count, 1));
     case SS_WS_SORT: return sort_temp_bytes(max64(count, 1));
     case SS_WS_TILE_ORDER: return tile_order_temp_bytes();

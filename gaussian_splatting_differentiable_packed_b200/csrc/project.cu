@@ -84,6 +84,16 @@ __host__ __device__ constexpr int rows_sh_stride() {
   return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
 }
 
+// Whether any camera sees Gaussian m (a set bit in one of its C mask words).
+__device__ __forceinline__ bool any_camera_sees(const Geo& g, const uint32_t* __restrict__ mask, int64_t m) {
+  uint32_t u = 0;
+  for (int c = 0; c < g.C && !u; ++c) u = (mask[((int64_t)c * g.n_pad + m) / 32] >> (m & 31)) & 1u;
+  return u != 0;
+}
+
+// Bit gi of the CTA's per-warp visibility words.
+__device__ __forceinline__ bool seen(const uint32_t* s_seen, int gi) { return (s_seen[gi >> 5] >> (gi & 31)) & 1u; }
+
 // A visible (camera, Gaussian) pair waiting in the CTA's work queue.
 struct RowItem {
   int64_t row;
@@ -109,7 +119,7 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
                                                          const uint32_t* __restrict__ mask,
                                                          const int64_t* __restrict__ block_off,
                                                          float* __restrict__ screen, uint32_t* __restrict__ aabb16,
-                                                         int64_t ahead) {
+                                                         float* __restrict__ row_depth, int64_t ahead) {
   constexpr int K = (DEG + 1) * (DEG + 1);
   constexpr int K3 = 3 * K;
   constexpr int KP = rows_sh_stride<DEG>();
@@ -122,20 +132,26 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   __shared__ uint32_t s_word[kSlots];  // [camera][warp]
   __shared__ int s_pre[kSlots + 1];    // exclusive prefix of the words' popcounts
   __shared__ int64_t s_row0[kCamChunk];
+  __shared__ uint32_t s_seen[kWarps];  // per warp: its Gaussians seen by some camera
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t blk = blockIdx.x;
   const int64_t n0 = blk * kBlock;
   const int64_t n = n0 + threadIdx.x;
   const int cnt = (int)min64(kBlock, g.N - n0);
-  if (threadIdx.x == 0 && ahead > 0 && blk + ahead < (int64_t)gridDim.x) {
-    // the parameters of the block that starts about a wave later, into L2
+  if (ahead > 0 && blk + ahead < (int64_t)gridDim.x) {
+    // the parameters of the block that starts about a wave later, into L2;
+    // SH rows only of the Gaussians some camera sees (the others are never
+    // read)
     const int64_t m0 = (blk + ahead) * kBlock;
     const int mc = (int)min64(kBlock, g.N - m0);
-    prefetch_l2(sh + m0 * K3, (uint32_t)(mc * K3 * 4));
-    prefetch_l2(means + 3 * m0, (uint32_t)(mc * 12));
-    prefetch_l2(quats + 4 * m0, (uint32_t)(mc * 16));
-    prefetch_l2(scales + 3 * m0, (uint32_t)(mc * 12));
-    prefetch_l2(opacities + m0, (uint32_t)(mc * 4));
+    if (threadIdx.x == 0) {
+      prefetch_l2(means + 3 * m0, (uint32_t)(mc * 12));
+      prefetch_l2(quats + 4 * m0, (uint32_t)(mc * 16));
+      prefetch_l2(scales + 3 * m0, (uint32_t)(mc * 12));
+      prefetch_l2(opacities + m0, (uint32_t)(mc * 4));
+    }
+    if (threadIdx.x < mc && any_camera_sees(g, mask, m0 + threadIdx.x))
+      prefetch_l2(sh + (m0 + threadIdx.x) * K3, (uint32_t)(K3 * 4));
   }
   // A chunk's cameras, first rows and each warp's mask word per camera.  The
   // first chunk is loaded before the parameters and the SH block so that its
@@ -156,6 +172,17 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     s_g[threadIdx.x] = load_gauss(means, quats, scales, n);
     s_o[threadIdx.x] = opacities[n];
   }
+  // which of the CTA's Gaussians any camera sees: only their SH rows are
+  // staged (a third of the Gaussians of the 15M-Gaussian workload are seen
+  // by no camera)
+  {
+    uint32_t u = 0;
+    for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + n0) / 32 + warp];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
+    if (lane == 0) s_seen[warp] = u;
+  }
+  __syncthreads();
   // the CTA's contiguous SH block: a full block with all 16-byte loads in
   // flight at once (it starts 16-byte aligned: 128*K3 floats per block), the
   // ragged last block word by word
@@ -168,12 +195,13 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
         const int v = threadIdx.x + r * kBlock;
-        if (v < kV) buf[r] = reinterpret_cast<const float4*>(src)[v];
+        if (v < kV && (seen(s_seen, (4 * v) / K3) || seen(s_seen, (4 * v + 3) / K3)))
+          buf[r] = reinterpret_cast<const float4*>(src)[v];
       }
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
         const int v = threadIdx.x + r * kBlock;
-        if (v < kV) {
+        if (v < kV && (seen(s_seen, (4 * v) / K3) || seen(s_seen, (4 * v + 3) / K3))) {
           const float e[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -185,7 +213,7 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     } else {
       for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
         const int gi = f / K3, qq = f - gi * K3;
-        sh_s[gi * KP + qq] = src[f];
+        if (seen(s_seen, gi)) sh_s[gi * KP + qq] = src[f];
       }
     }
   }
@@ -220,6 +248,7 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     qq.x = q16_floor(x0, g.W) | (q16_floor(y0, g.H) << 16);
     qq.y = q16_ceil(x1, g.W) | (q16_ceil(y1, g.H) << 16);
     reinterpret_cast<uint2*>(aabb16)[it.row] = qq;
+    row_depth[it.row] = P.pz;
   };
   for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
     const int nc = min(kCamChunk, g.C - c0);
@@ -275,10 +304,19 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
 template <int DEG>
 void launch_rows(const Geo& g, unsigned grid, cudaStream_t st, const float* cams, const float* means,
                  const float* quats, const float* scales, const float* opacities, const float* sh,
-                 const uint32_t* mask, const int64_t* block_off, float* screen, uint32_t* aabb16) {
+                 const uint32_t* mask, const int64_t* block_off, float* screen, uint32_t* aabb16,
+                 float* row_depth) {
   const int64_t ahead = wave_blocks(k_project_rows<DEG>, kBlock, 0);
   k_project_rows<DEG><<<grid, kBlock, 0, st>>>(g, cams, means, quats, scales, opacities, sh, mask, block_off, screen,
-                                               aabb16, ahead);
+                                               aabb16, row_depth, ahead);
+}
+
+size_t cap_temp_bytes(int C);
+ss_status apply_visible_cap(const Geo& g, const float* opacities, uint32_t* mask, uint32_t* block_count,
+                            const int64_t* block_off, int64_t cap, void* temp, cudaStream_t st, bool* changed);
+
+size_t project_temp_bytes(const Geo& g) {
+  return scan_temp_bytes(max64(g.mask_blocks, 1)) + cap_temp_bytes(g.C);
 }
 
 }  // namespace ss
@@ -288,7 +326,8 @@ using namespace ss;
 extern "C" ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float* means,
                                        const float* quats, const float* scales, const float* opacities,
                                        const float* sh, uint32_t* mask, uint32_t* block_count, int64_t* block_off,
-                                       float* screen, uint32_t* aabb16, int64_t cap_rows, void* temp,
+                                       float* screen, uint32_t* aabb16, float* row_depth, int64_t cap_rows,
+                                       int64_t cap_visible, void* temp,
                                        size_t temp_bytes, int64_t* nnz_out, void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (!nnz_out) return invalid("nnz_out is NULL");
@@ -315,6 +354,20 @@ extern "C" ss_status ss_project_packed(const ss_dims* dims, const float* cams, c
   if (s) return s;
   s = scan_phase2<int64_t>(src, g.mask_blocks, temp, block_off, st);
   if (s) return s;
+  if (cap_visible >= 0) {
+    if (!opacities) return invalid("the visible cap needs the opacities");
+    if (g.N > (int64_t(1) << 32)) return invalid("the visible cap needs N <= 2^32");
+    bool changed = false;
+    void* cap_temp = reinterpret_cast<char*>(temp) + scan_temp_bytes(max64(g.mask_blocks, 1));
+    s = apply_visible_cap(g, opacities, mask, block_count, block_off, cap_visible, cap_temp, st, &changed);
+    if (s) return s;
+    if (changed) {
+      s = scan_phase1(src, g.mask_blocks, temp, block_off + g.mask_blocks, st);
+      if (s) return s;
+      s = scan_phase2<int64_t>(src, g.mask_blocks, temp, block_off, st);
+      if (s) return s;
+    }
+  }
   int64_t nnz = 0;
   s = cuda_status(cudaMemcpyAsync(&nnz, block_off + g.mask_blocks, sizeof(int64_t), cudaMemcpyDeviceToHost, st),
                   "copy nnz");
@@ -327,16 +380,20 @@ extern "C" ss_status ss_project_packed(const ss_dims* dims, const float* cams, c
     set_error("ss_project_packed: nnz exceeds cap_rows");
     return SS_ERR_CAPACITY;
   }
-  if (!opacities || !sh || !aabb16) return invalid("null row input/output");
+  if (!opacities || !sh || !aabb16 || !row_depth) return invalid("null row input/output");
   if (((uintptr_t)screen & 15) != 0 || ((uintptr_t)aabb16 & 7) != 0) return invalid("row buffers misaligned");
   switch (g.deg) {
-    case 0: launch_rows<0>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+    case 0: launch_rows<0>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16,
+                            row_depth);
             break;
-    case 1: launch_rows<1>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+    case 1: launch_rows<1>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16,
+                            row_depth);
             break;
-    case 2: launch_rows<2>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+    case 2: launch_rows<2>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16,
+                            row_depth);
             break;
-    default: launch_rows<3>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16);
+    default: launch_rows<3>(g, grid, st, cams, means, quats, scales, opacities, sh, mask, block_off, screen, aabb16,
+                            row_depth);
   }
   return cuda_status(cudaGetLastError(), "project pass 2");
 }

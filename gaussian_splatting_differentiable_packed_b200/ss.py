@@ -85,7 +85,7 @@ def lib() -> ct.CDLL:
         L.ss_status_string.restype = ct.c_char_p
         L.ss_last_error.argtypes = []
         L.ss_last_error.restype = ct.c_char_p
-        L.ss_project_packed.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, i64, P, sz, ct.POINTER(i64), P]
+        L.ss_project_packed.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, i64, i64, P, sz, ct.POINTER(i64), P]
         L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
         L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, P, sz, P, ct.POINTER(i32), P]
         L.ss_sort_isects_noalloc.argtypes = [D, P, P, P, P, i64, P, ct.POINTER(i32), P]
@@ -144,20 +144,22 @@ def workspace_bytes(d: ss_dims, which: int, count: int = 0) -> int:
 
 
 def ss_project_packed(d, cams, means, quats, scales, opacities, sh, mask, block_count, block_off, screen, aabb16,
-                      cap_rows, temp, stream=None) -> int:
+                      row_depth, cap_rows, temp, stream=None, cap_visible=None) -> int:
+    """cap_visible: the per-image visible cap (None: no cap)."""
     nnz = ct.c_int64(0)
     st = lib().ss_project_packed(ct.byref(d), _p(cams), _p(means), _p(quats), _p(scales), _p(opacities), _p(sh),
-                                 _p(mask), _p(block_count), _p(block_off), _p(screen), _p(aabb16), int(cap_rows),
+                                 _p(mask), _p(block_count), _p(block_off), _p(screen), _p(aabb16), _p(row_depth),
+                                 int(cap_rows), -1 if cap_visible is None else int(cap_visible),
                                  _p(temp), 0 if temp is None else temp.numel() * temp.element_size(),
                                  ct.byref(nnz), _stream(stream))
     _check(st, "ss_project_packed", int(nnz.value))
     return int(nnz.value)
 
 
-def ss_intersect_tiles(d, screen, aabb16, block_off, nnz, isect_off, keys, vals, cap_isects, temp,
+def ss_intersect_tiles(d, row_depth, aabb16, block_off, nnz, isect_off, keys, vals, cap_isects, temp,
                        stream=None) -> int:
     n = ct.c_uint64(0)
-    st = lib().ss_intersect_tiles(ct.byref(d), _p(screen), _p(aabb16), _p(block_off), int(nnz), _p(isect_off),
+    st = lib().ss_intersect_tiles(ct.byref(d), _p(row_depth), _p(aabb16), _p(block_off), int(nnz), _p(isect_off),
                                   _p(keys), _p(vals), int(cap_isects), _p(temp),
                                   0 if temp is None else temp.numel() * temp.element_size(), ct.byref(n),
                                   _stream(stream))
@@ -324,12 +326,15 @@ class PackedStep:
     ss_tile_order and ss_rasterize_fwd; backward(v_img, v_T=None) runs ss_rasterize_bwd and
     ss_project_bwd.  forward(..., bg=, depth=True) also blends a background
     colour per camera and renders the expected depth (self.depth);
-    backward(..., v_depth=) then takes its gradient.  Intermediate buffers are
-    kept as attributes so callers (tests) can inspect every stage.
+    backward(..., v_depth=) then takes its gradient.  cap_visible applies the
+    per-image visible cap of ss_project_packed (None: no cap).  Intermediate
+    buffers are kept as attributes so callers (tests) can inspect every stage.
     """
 
-    def __init__(self, d: ss_dims, device="cuda", cap_rows: int = 0, cap_isects: int = 0, headroom: float = 1.25):
+    def __init__(self, d: ss_dims, device="cuda", cap_rows: int = 0, cap_isects: int = 0, headroom: float = 1.25,
+                 cap_visible: int | None = None):
         self.d = d
+        self.cap_visible = cap_visible
         self.dev = torch.device(device)
         self.headroom = headroom
         C, N = d.C, d.N
@@ -368,6 +373,7 @@ class PackedStep:
         dev = self.dev
         self.screen = torch.empty((cap, ROW), dtype=torch.float32, device=dev)
         self.aabb16 = torch.empty((cap, 2), dtype=torch.int32, device=dev)
+        self.row_depth = torch.empty(cap, dtype=torch.float32, device=dev)
         self.isect_off = torch.empty(cap + 1, dtype=torch.int64, device=dev)
         self.v_screen = torch.empty((cap, ROW), dtype=torch.float32, device=dev)
         self.temp_isect = torch.empty(workspace_bytes(self.d, WS_INTERSECT, cap), dtype=torch.uint8, device=dev)
@@ -391,25 +397,25 @@ class PackedStep:
         d = self.d
         try:
             nnz = ss_project_packed(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_count,
-                                    self.block_off, self.screen, self.aabb16, self.cap_rows, self.temp_project,
-                                    stream)
+                                    self.block_off, self.screen, self.aabb16, self.row_depth, self.cap_rows,
+                                    self.temp_project, stream, cap_visible=self.cap_visible)
         except SSError as e:
             if e.status != SS_ERR_CAPACITY:
                 raise
             self._rows(int(e.count * self.headroom) + 1)
             nnz = ss_project_packed(d, cams, means, quats, scales, opacities, sh, self.mask, self.block_count,
-                                    self.block_off, self.screen, self.aabb16, self.cap_rows, self.temp_project,
-                                    stream)
+                                    self.block_off, self.screen, self.aabb16, self.row_depth, self.cap_rows,
+                                    self.temp_project, stream, cap_visible=self.cap_visible)
         self.nnz = nnz
         try:
-            n = ss_intersect_tiles(d, self.screen, self.aabb16, self.block_off, nnz, self.isect_off, self.keys_a,
-                                   self.vals_a, self.cap_isects, self.temp_isect, stream)
+            n = ss_intersect_tiles(d, self.row_depth, self.aabb16, self.block_off, nnz, self.isect_off,
+                                   self.keys_a, self.vals_a, self.cap_isects, self.temp_isect, stream)
         except SSError as e:
             if e.status != SS_ERR_CAPACITY:
                 raise
             self._isects(int(e.count * self.headroom) + 1)
-            n = ss_intersect_tiles(d, self.screen, self.aabb16, self.block_off, nnz, self.isect_off, self.keys_a,
-                                   self.vals_a, self.cap_isects, self.temp_isect, stream)
+            n = ss_intersect_tiles(d, self.row_depth, self.aabb16, self.block_off, nnz, self.isect_off,
+                                   self.keys_a, self.vals_a, self.cap_isects, self.temp_isect, stream)
         self.n_isects = n
         self.unsorted_keys = self.keys_a
         self.unsorted_vals = self.vals_a
@@ -445,32 +451,60 @@ def scene_dims(scene) -> ss_dims:
     return make_dims(scene.C, scene.W, scene.H, scene.sh_degree, scene.N, scene.near, scene.far)
 
 
-def sort_passes(d: ss_dims) -> int:
-    """8-bit digit passes of ss_sort_isects: 4 over the 31 depth bits, then
-    ceil(bits(n_tiles) / 8) over the tile id."""
-    n_tiles = size(d, SIZE_N_TILES)
-    tb = max(0, (n_tiles - 1).bit_length())
-    return 4 + (tb + 7) // 8
+def sort_passes_for(keys, d: ss_dims) -> int:
+    """Digit passes ss_sort_isects runs on these (unsorted or sorted) keys:
+    one per byte of the depth and per byte the tile ids need, less the bytes
+    that are equal in every key.  Measurement helper (torch reductions); not
+    part of any step."""
+    if keys.numel() == 0:
+        return 0
+    k = keys.to(torch.int64)
+    tb = max(0, (size(d, SIZE_N_TILES) - 1).bit_length())
+    shifts = [0, 8, 16, 24] + [32 + 8 * i for i in range((tb + 7) // 8)]
+    n = 0
+    for sh in shifts:
+        dig = (k >> sh) & 0xFF
+        n += int(dig.min().item()) != int(dig.max().item())
+    return n
+
+
+def seen_gaussians(d: ss_dims, mask) -> int:
+    """Gaussians that some camera sees (a set bit in one of their mask words).
+    Measurement helper (torch reductions); not part of any step."""
+    words = size(d, SIZE_MASK_WORDS) // d.C
+    m = mask[: d.C * words].view(d.C, words)
+    u = m[0].clone()
+    for c in range(1, d.C):
+        u |= m[c]
+    b = u.view(torch.uint8).to(torch.int32)
+    pop = torch.zeros_like(b)
+    for k in range(8):
+        pop += (b >> k) & 1
+    return int(pop.sum().item())
 
 
 def sort_launches(d: ss_dims, n_isects: int) -> int:
-    """Kernels of one ss_sort_isects call: histogram, digit bases, one onesweep
-    kernel per pass, tile ranges."""
-    return 0 if n_isects == 0 else sort_passes(d) + 3
+    """Kernels of one ss_sort_isects call: histogram, plan, one onesweep
+    kernel per byte of the full plan (a skipped byte's kernel returns at
+    once), tile ranges."""
+    if n_isects == 0:
+        return 0
+    tb = max(0, (size(d, SIZE_N_TILES) - 1).bit_length())
+    return 2 + 4 + (tb + 7) // 8 + 1
 
 
 def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
     """Kernels libss launches in one forward+backward step (memsets excluded):
-    projection 5 (pass 1, three scan kernels, pass 2), intersection 5 (three
-    scan kernels, chunk first rows, write), the sort (sort_launches), tile
-    order 3 (histogram, scan, scatter), rasterizer 1 + 1, projection
-    backward 1.  With no Gaussians only the tile order and the two
+    projection 5 (pass 1, three scan kernels, pass 2), intersection 3 (two
+    count kernels, the fused offsets-and-write kernel), the sort
+    (sort_launches), tile order 3 (histogram, scan, scatter), rasterizer
+    1 + 1, projection backward 1.  With no Gaussians only the tile order and the two
     rasterizers launch (they still write the empty images)."""
     if d.N == 0:
         return 3 + 2
     n = 5
     if nnz > 0:
-        n += 5 if n_isects > 0 else 3
+        n += 3
     n += sort_launches(d, n_isects)
     return n + 3 + 3
 

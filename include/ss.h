@@ -47,6 +47,8 @@
  *             r, g, b, depth, 0, 0 (48-byte rows: three 16-byte vectors)
  *   aabb16    uint32 [cap_rows][2]: word0 = qx0 | qy0 << 16, word1 = qx1 | qy1 << 16,
  *             edges on the grid extent/65535, min floored, max ceiled
+ *   row_depth float [cap_rows]: the row's camera depth (the screen row's depth,
+ *             stored compactly for the intersection pass's keys)
  *   keys      uint64 [cap_isects]: (c*tiles_per_cam + ty*tiles_x + tx) << 32 | bits(depth)
  *   vals      uint32 [cap_isects]: screen row index
  *   tile_off  int64 [n_tiles + 1]: tile t owns sorted entries [tile_off[t], tile_off[t+1])
@@ -99,9 +101,8 @@ typedef struct ss_dims {
 int64_t ss_size(const ss_dims* dims, int what);
 
 /* Scratch bytes needed by a call: which = SS_WS_PROJECT (count ignored),
- * SS_WS_INTERSECT (count = nnz; includes 8 MiB for the write pass's per-chunk
- * row index), SS_WS_SORT (count = number of keys), SS_WS_TILE_ORDER (count
- * ignored). */
+ * SS_WS_INTERSECT (count = nnz), SS_WS_SORT (count = number of keys),
+ * SS_WS_TILE_ORDER (count ignored). */
 #define SS_WS_PROJECT 0
 #define SS_WS_INTERSECT 1
 #define SS_WS_SORT 2
@@ -124,14 +125,29 @@ const char* ss_last_error(void);
  * is NULL the call stops there (count-only).  If nnz > cap_rows it returns
  * SS_ERR_CAPACITY with *nnz_out exact and writes no row.  Otherwise pass 2
  * re-projects the survivors only: row = block_off[block] + set bits before the
- * pair, writing the screen row (SH colour evaluated toward the camera centre)
- * and the 16-bit AABB.  Rows are ordered camera-major, Gaussian-minor.
- * quats and sh must be 16-byte aligned (SS_ERR_INVALID_ARG otherwise).
+ * pair, writing the screen row (SH colour evaluated toward the camera centre),
+ * the 16-bit AABB and the row's depth into row_depth (4 bytes a row: the
+ * intersection pass reads it instead of the 48-byte screen row).  Rows are
+ * ordered camera-major, Gaussian-minor.  quats and sh must be 16-byte aligned
+ * (SS_ERR_INVALID_ARG otherwise).
+ *
+ * cap_visible ("Spirula Studio VRAM deep-dive", practical guide: --cap-max,
+ * the per-image visible splat cap that holds down nnz): < 0 for no cap.
+ * Otherwise, in every camera with more than cap_visible visible pairs, only
+ * the cap_visible of highest opacity stay visible (opacity ordered by its
+ * fp32 value, IEEE total order; ties go to the lower Gaussian index; the page
+ * names the cap but no selection rule, this is this library's reading); the
+ * mask, block counts, block_off and nnz describe the capped set, so every
+ * later call (and the projection backward) sees only the kept pairs.  Needs
+ * opacities (even in count-only mode) and N <= 2^32; when the cap binds it
+ * costs one more small copy and stream sync and 8 selection passes over the
+ * mask.
  */
 ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float* means, const float* quats,
                             const float* scales, const float* opacities, const float* sh, uint32_t* mask,
                             uint32_t* block_count, int64_t* block_off, float* screen, uint32_t* aabb16,
-                            int64_t cap_rows, void* temp, size_t temp_bytes, int64_t* nnz_out, void* stream);
+                            float* row_depth, int64_t cap_rows, int64_t cap_visible, void* temp, size_t temp_bytes,
+                            int64_t* nnz_out, void* stream);
 
 /*
  * Tile intersections ("Spirula Studio VRAM deep-dive", section "4 GiB rule and
@@ -143,10 +159,11 @@ ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float*
  * Returns SS_ERR_CAPACITY if the total exceeds cap_isects and
  * SS_ERR_OVERFLOW if it is >= 2^31, writing nothing else in either case.
  * Otherwise writes isect_off[nnz+1] (exclusive per-row offsets) and one
- * (key, row) per covered tile, row-major over (row, ty, tx).  block_off is the
- * array ss_project_packed wrote (it gives each camera's first row).
+ * (key, row) per covered tile, row-major over (row, ty, tx); the key's depth
+ * bits come from row_depth.  block_off, aabb16 and row_depth are the arrays
+ * ss_project_packed wrote (block_off gives each camera's first row).
  */
-ss_status ss_intersect_tiles(const ss_dims* dims, const float* screen, const uint32_t* aabb16,
+ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_depth, const uint32_t* aabb16,
                              const int64_t* block_off, int64_t nnz, int64_t* isect_off, uint64_t* keys,
                              uint32_t* vals, int64_t cap_isects, void* temp, size_t temp_bytes,
                              uint64_t* n_isects_out, void* stream);
@@ -154,10 +171,11 @@ ss_status ss_intersect_tiles(const ss_dims* dims, const float* screen, const uin
 /*
  * Stable LSD radix sort of n (key, value) pairs by key, 8-bit digits over the
  * 32 depth bits and the tile-id bits only ("Spirula Studio VRAM deep-dive",
- * buffer table: double-buffered isect.ids_a/b).  Ping-pongs between (keys_a,
- * vals_a) and (keys_b, vals_b); *result_in_b_out (host) says which pair holds
- * the result (an odd pass count: b; known from dims alone).  Then writes
- * tile_off[n_tiles+1].
+ * buffer table: double-buffered isect.ids_a/b); a digit that is equal in
+ * every key is skipped (it cannot change the order).  Ping-pongs between
+ * (keys_a, vals_a) and (keys_b, vals_b); *result_in_b_out (host) says which
+ * pair holds the result (b after an odd number of digit passes, which depends
+ * on the keys).  Then writes tile_off[n_tiles+1].
  * n >= 2^31 returns SS_ERR_OVERFLOW.  Equal keys keep their input order.
  * Synchronises the stream at the end (reads the look-back error flag).
  */
@@ -210,7 +228,8 @@ ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams, float* mea
  * block; the call decodes the accumulator (code * scale), adds this
  * sub-batch's gradient (the same gradient ss_project_bwd computes for the
  * cameras of dims) and quantises the sums again: scale = the block's largest
- * magnitude / 32767, code = nearest-even(x / scale), 0 for an all-zero block.
+ * magnitude / 32767, code = nearest-even(x * (1 / scale)) in fp32 (within
+ * 0.005 of a step of the exact quotient), 0 for an all-zero block.
  * first != 0 starts from zero (the accumulator's contents are ignored), as
  * for a step's first sub-batch.  Accumulator layout (device, owned by the
  * caller, updated in place):
@@ -240,19 +259,23 @@ ss_status ss_project_bwd_gq(const ss_dims* dims, const float* cams, const float*
 
 /*
  * Allocation-free variant of ss_sort_isects (the pages have no counterpart:
- * this is an addition of this library).  For callers that cannot allocate
- * device memory themselves (code that runs inside another runtime's
- * allocator or capture, or a host that only hands out fixed buffers): the
- * sort's scratch lives in a file-scope device array of 24 MiB that the
- * library holds on every GPU that loads it, until the process exits.  The
- * caller still passes the key/value buffers and tile_off; no cudaMalloc,
- * cudaFree or allocating routine is called.  n may be at most 50,311,168
- * keys; a larger n returns SS_ERR_INVALID_ARG before any device work.  The
- * first call on a device looks up the array's device address
+ * this is an addition of this library).  For callers that cannot call
+ * cudaMalloc themselves: code that runs inside another runtime's allocator
+ * callbacks or memory-pool hooks, where a nested cudaMalloc would re-enter
+ * that allocator, or a host that hands out only fixed, pre-sized device
+ * buffers.  The sort's scratch lives in a file-scope device array of 24 MiB
+ * that the library holds on every GPU that loads it, until the process exits.
+ * The caller still passes the key/value buffers and tile_off; no cudaMalloc,
+ * cudaFree or allocating routine is called.  n may be at most 50,311,168 keys
+ * (the whole 4096-key tiles of look-back state that fit in the 24 MiB after
+ * a fixed header); a larger n returns SS_ERR_INVALID_ARG before any device work.  The
+ * first call on a device (and context) looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  Every call shares the one array (cleared at the
  * start of each call), so calls that overlap on the GPU race with each other:
- * serialise them, e.g. on one stream.  Results equal ss_sort_isects'.
+ * serialise them, e.g. on one stream.  Like ss_sort_isects, the call
+ * synchronises the stream at the end to read the sort's device-side check
+ * flag.  Results equal ss_sort_isects'.
  */
 ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
                                  uint32_t* vals_b, int64_t n, int64_t* tile_off, int* result_in_b_out,

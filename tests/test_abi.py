@@ -80,7 +80,7 @@ def test_invalid_dims_rejected_on_host(L, bad):
     assert L.ss_size(ct.byref(d), 0) == -1
     assert L.ss_workspace_bytes(ct.byref(d), 0, 0) == 0
     nnz = ct.c_int64(0)
-    st = L.ss_project_packed(ct.byref(d), *([None] * 11), 0, None, 0, ct.byref(nnz), None)
+    st = L.ss_project_packed(ct.byref(d), *([None] * 12), 0, -1, None, 0, ct.byref(nnz), None)
     assert st == ss.SS_ERR_INVALID_ARG
     assert b"dims" in L.ss_last_error()
 
@@ -112,9 +112,24 @@ def test_null_and_short_temp_rejected(L):
     d = ss.make_dims(1, 64, 64, 0, 10)
     nnz = ct.c_int64(0)
     fake = ct.c_void_p(256)  # never dereferenced: the temp size check fails first
-    st = L.ss_project_packed(ct.byref(d), fake, fake, fake, fake, fake, fake, fake, fake, fake, None, None, 0,
-                             fake, 1, ct.byref(nnz), None)
+    st = L.ss_project_packed(ct.byref(d), fake, fake, fake, fake, fake, fake, fake, fake, fake, None, None, None, 0,
+                             -1, fake, 1, ct.byref(nnz), None)
     assert st == ss.SS_ERR_INVALID_ARG
     n = ct.c_uint64(0)
     st = L.ss_intersect_tiles(ct.byref(d), fake, fake, fake, 5, fake, fake, fake, 100, fake, 1, ct.byref(n), None)
     assert st == ss.SS_ERR_INVALID_ARG
+
+
+def test_noalloc_sort_limit_on_host(L):
+    """The allocation-free sort's key limit is the largest count whose sort
+    scratch fits its 24 MiB static array: the workspace query agrees at the
+    boundary, and one key more is refused with the limit in the message."""
+    d = ss.make_dims(1, 64, 64, 0, 10)
+    limit = 50_311_168
+    assert ss.workspace_bytes(d, ss.WS_SORT, limit) <= 24 << 20
+    assert ss.workspace_bytes(d, ss.WS_SORT, limit + 1) > 24 << 20
+    in_b = ct.c_int(0)
+    fake = ct.c_void_p(256)  # never dereferenced: the size check comes first
+    st = L.ss_sort_isects_noalloc(ct.byref(d), fake, fake, fake, fake, limit + 1, fake, ct.byref(in_b), None)
+    assert st == ss.SS_ERR_INVALID_ARG
+    assert f"at most {limit} keys".encode() in L.ss_last_error()

@@ -29,6 +29,15 @@ def test_traffic_record_guards(tmp_path, monkeypatch):
     bad[stage] = dict(rec[stage], sha256="0" * 64)
     p.write_text(json.dumps(bad))
     assert bench.recorded_traffic(stage, wl["config"], wl["n"]) is None
+    # a capture of a smaller case scales by the units the kernel processes
+    small = dict(rec)
+    small[stage] = dict(rec[stage], sha256=bench.source_digest(rec[stage]["sources"]),
+                        workload={"config": wl["config"], "n": 3_000_000}, units={"name": "n_isects", "value": 1000})
+    p.write_text(json.dumps(small))
+    got = bench.recorded_traffic(stage, wl["config"], None, dict(n_isects=3000))
+    assert got == 3 * float(rec[stage]["dram_bytes_per_launch"])
+    assert bench.recorded_traffic(stage, wl["config"], None, dict(nnz=3000)) is None
+    assert bench.recorded_traffic(stage, 3, None, dict(n_isects=3000)) is None
     # a missing stage or file: no traffic
     assert bench.recorded_traffic("no_such_stage", wl["config"], wl["n"]) is None
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
@@ -36,16 +45,27 @@ def test_traffic_record_guards(tmp_path, monkeypatch):
 
 
 def test_launches_per_step():
-    """projection 5, intersection 5 (3 without intersections), the sort's
-    histogram, bases, one pass per digit and tile ranges, the tile order 3,
-    rasterizers 2, projection backward 1."""
-    d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)
-    passes = ss.sort_passes(d)
-    assert passes == 6  # 33,500 tiles: 16 tile-id bits, 2 digits over them
-    assert ss.launches_per_step(d, 15_000_000, 33_000_000) == 5 + 5 + (passes + 3) + 3 + 2 + 1
+    """projection 5, intersection 3 (two count kernels, the fused write), the
+    sort's histogram, plan, one kernel per byte of the full plan and tile
+    ranges, the tile order 3, rasterizers 2, projection backward 1."""
+    d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)  # 33,500 tiles: 16 tile-id bits, 2 bytes
+    assert ss.launches_per_step(d, 15_000_000, 33_000_000) == 5 + 3 + (2 + 6 + 1) + 3 + 2 + 1
     assert ss.launches_per_step(d, 15_000_000, 0) == 5 + 3 + 0 + 3 + 2 + 1
     assert ss.launches_per_step(d, 0, 0) == 5 + 0 + 0 + 3 + 2 + 1
     assert ss.launches_per_step(ss.make_dims(1, 64, 64, 0, 0), 0, 0) == 3 + 2
+
+
+def test_sort_passes_skip_constant_bytes():
+    """A byte equal in every key takes no pass: 16 tile-id bits and depths
+    whose top byte is fixed take 5 of the 6 byte passes; keys that differ in
+    one low bit take one; equal keys none."""
+    import torch
+    d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)
+    tiles = torch.arange(0, 33_500, dtype=torch.int64)
+    depth = torch.full_like(tiles, 0x41000000) + (tiles * 1237) % (1 << 23)
+    assert ss.sort_passes_for((tiles << 32) | depth, d) == 5
+    assert ss.sort_passes_for(torch.tensor([7, 6], dtype=torch.int64), d) == 1
+    assert ss.sort_passes_for(torch.tensor([5, 5], dtype=torch.int64), d) == 0
 
 
 def test_oracle_sample_never_exceeds_the_workload():

@@ -42,6 +42,8 @@ def grad_close(name, gpu, ref, rtol=1e-3, atol=1e-5, scale_tol=1e-4):
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     assert gpu.shape == ref.shape, name
+    if ref.size == 0:
+        return
     err = np.abs(gpu - ref)
     bad = err > atol + rtol * np.abs(ref)
     assert not bad.any(), (name, int(bad.sum()), float(err[bad].max()), np.argwhere(bad)[:5].tolist())
@@ -85,7 +87,7 @@ def check_unsorted(scene, o, step):
     I = it["n_isects"]
     keys = torch.empty(max(I, 1), dtype=torch.int64, device="cuda")
     vals = torch.empty(max(I, 1), dtype=torch.int32, device="cuda")
-    n = ss.ss_intersect_tiles(step.d, step.screen, step.aabb16, step.block_off, step.nnz, step.isect_off, keys, vals,
+    n = ss.ss_intersect_tiles(step.d, step.row_depth, step.aabb16, step.block_off, step.nnz, step.isect_off, keys, vals,
                               I, step.temp_isect)
     torch.cuda.synchronize()
     assert n == I
@@ -217,16 +219,16 @@ def test_capacity_errors_report_exact_counts():
     step = ss.PackedStep(d, "cuda", cap_rows=10, cap_isects=10)
     with pytest.raises(ss.SSError) as e:
         ss.ss_project_packed(d, *t, step.mask, step.block_count, step.block_off, step.screen, step.aabb16,
-                             step.cap_rows, step.temp_project)
+                             step.row_depth, step.cap_rows, step.temp_project)
     assert e.value.status == ss.SS_ERR_CAPACITY and e.value.count == o["proj"]["nnz"]
     # count-only mode
-    assert ss.ss_project_packed(d, *t, step.mask, step.block_count, step.block_off, None, None, 0,
+    assert ss.ss_project_packed(d, *t, step.mask, step.block_count, step.block_off, None, None, None, 0,
                                 step.temp_project) == o["proj"]["nnz"]
     step._rows(o["proj"]["nnz"])
     nnz = ss.ss_project_packed(d, *t, step.mask, step.block_count, step.block_off, step.screen, step.aabb16,
-                               step.cap_rows, step.temp_project)
+                               step.row_depth, step.cap_rows, step.temp_project)
     with pytest.raises(ss.SSError) as e:
-        ss.ss_intersect_tiles(d, step.screen, step.aabb16, step.block_off, nnz, step.isect_off, step.keys_a,
+        ss.ss_intersect_tiles(d, step.row_depth, step.aabb16, step.block_off, nnz, step.isect_off, step.keys_a,
                               step.vals_a, 10, step.temp_isect)
     assert e.value.status == ss.SS_ERR_CAPACITY and e.value.count == o["isect"]["n_isects"]
 
@@ -250,10 +252,10 @@ def test_counts_past_2_pow_32_are_exact():
     t = ss.scene_tensors(sc)
     step = ss.PackedStep(d, "cuda", cap_rows=N, cap_isects=1)
     nnz = ss.ss_project_packed(d, *t, step.mask, step.block_count, step.block_off, step.screen, step.aabb16,
-                               step.cap_rows, step.temp_project)
+                               step.row_depth, step.cap_rows, step.temp_project)
     assert nnz == p["nnz"] == N
     with pytest.raises(ss.SSError) as e:
-        ss.ss_intersect_tiles(d, step.screen, step.aabb16, step.block_off, nnz, step.isect_off, None, None,
+        ss.ss_intersect_tiles(d, step.row_depth, step.aabb16, step.block_off, nnz, step.isect_off, None, None,
                               2**62, step.temp_isect)
     assert e.value.status == ss.SS_ERR_OVERFLOW
     assert e.value.count == total

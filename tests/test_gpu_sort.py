@@ -1,8 +1,9 @@
 """Direct parity of ss_sort_isects with the oracle's stable sort on seeded
 synthetic (tile << 32 | depth) keys with skewed tile populations (uniform
 tiles, a few tiles holding thousands of keys as the heavy tiles of the large
-workloads do), and a tile count needing three tile-id bytes (odd pass count:
-the result ends in the second buffer pair).
+workloads do), and a tile count needing 17 tile-id bits.  The sort skips
+the digit bytes that are equal in every key, so the pass count (and the
+buffer pair that ends up holding the result) follows from the keys.
 Depths repeat (ties must keep input order) and values are not ordered by
 position, so only a stable sort by key matches.  Keys, values and tile
 offsets must be bit-exact.
@@ -61,7 +62,7 @@ def test_sort_paths(case):
            "three_tile_bytes": [(81919, 2500)]}[case]
     keys, vals = make_keys(rng, n_tiles, 300_000, hot)
     in_b, gk, gv, toff = run_sort(d, keys, vals)
-    assert in_b == bool(ss.sort_passes(d) & 1)
+    assert in_b == bool(ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d) & 1)
     ok, ov = orc.sort(keys, vals)
     np.testing.assert_array_equal(gk, ok)
     np.testing.assert_array_equal(gv, ov)
@@ -75,6 +76,32 @@ def test_sort_single_bucket_and_tiny():
     rng = np.random.default_rng(15)
     for keys, vals in [make_keys(rng, 1, 1500), make_keys(rng, n_tiles, 3)]:
         in_b, gk, gv, toff = run_sort(d, keys, vals)
+        ok, ov = orc.sort(keys, vals)
+        np.testing.assert_array_equal(gk, ok)
+        np.testing.assert_array_equal(gv, ov)
+        np.testing.assert_array_equal(toff, orc.tile_ranges(ok, n_tiles))
+
+
+def test_sort_skipped_digit_plans():
+    """Digit bytes equal in every key are skipped: every key equal (no pass,
+    the result stays in the first pair), keys differing in one low bit (one
+    pass), depths sharing their top byte (one pass fewer), and full 32-bit
+    low words with the top bit set (every pass)."""
+    d = ss.make_dims(1, 1024, 1024, 0, 1, 0.01, 1e10)
+    n_tiles = ss.size(d, ss.SIZE_N_TILES)
+    rng = np.random.default_rng(16)
+    same = np.full(5000, (np.uint64(77) << np.uint64(32)) | np.uint64(0x40a00000), np.uint64)
+    one_bit = same ^ rng.integers(0, 2, 5000).astype(np.uint64)
+    top = (rng.integers(0, n_tiles, 100_000).astype(np.uint64) << np.uint64(32)) | \
+        (np.uint64(0x41000000) + rng.integers(0, 1 << 23, 100_000).astype(np.uint64))
+    full = (rng.integers(0, n_tiles, 200_000).astype(np.uint64) << np.uint64(32)) | \
+        rng.integers(0, 2**32, 200_000, dtype=np.uint64)
+    for keys, passes in ((same, 0), (one_bit, 1), (top, 5), (full, 6)):
+        vals = rng.permutation(len(keys)).astype(np.uint32)
+        p = ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d)
+        assert p == passes
+        in_b, gk, gv, toff = run_sort(d, keys, vals)
+        assert in_b == bool(p & 1)
         ok, ov = orc.sort(keys, vals)
         np.testing.assert_array_equal(gk, ok)
         np.testing.assert_array_equal(gv, ov)

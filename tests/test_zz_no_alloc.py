@@ -1,9 +1,10 @@
 """The allocation-free sort entry point (ss_sort_isects_noalloc).
 
 It exists for callers that cannot call cudaMalloc themselves (code running
-inside another runtime's allocator or capture, or hosts that hand out only
-fixed device buffers): its scratch is a static device array inside libss.so,
-so the caller passes only the key/value buffers and tile_off.
+inside another runtime's allocator callbacks, where a nested cudaMalloc would
+re-enter that allocator, or hosts that hand out only fixed device buffers):
+its scratch is a static device array inside libss.so, so the caller passes
+only the key/value buffers and tile_off.
 
 Checked here through the C ABI: two calls in a row give exactly the results of
 the allocating ss_sort_isects (integer outputs, so the tolerance is equality),
@@ -20,7 +21,16 @@ from gaussian_splatting_differentiable_packed_b200 import scenes, ss
 
 pytestmark = pytest.mark.gpu
 
-MAX_KEYS = 50_311_168
+SCRATCH_BYTES = 24 << 20
+
+
+def max_keys(d):
+    """Largest key count whose sort scratch fits the 24 MiB static array."""
+    lo, hi = 1, 1 << 31
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if ss.workspace_bytes(d, ss.WS_SORT, mid) <= SCRATCH_BYTES else (lo, mid)
+    return lo
 
 
 def unsorted_keys(cfg):
@@ -32,7 +42,7 @@ def unsorted_keys(cfg):
     # the intersection pass alone: keys/values in row-major order
     keys = torch.empty(n, dtype=torch.int64, device="cuda")
     vals = torch.empty(n, dtype=torch.int32, device="cuda")
-    ss.ss_intersect_tiles(d, step.screen, step.aabb16, step.block_off, step.nnz, step.isect_off, keys, vals, n,
+    ss.ss_intersect_tiles(d, step.row_depth, step.aabb16, step.block_off, step.nnz, step.isect_off, keys, vals, n,
                           step.temp_isect)
     torch.cuda.synchronize()
     return d, keys, vals, n
@@ -65,9 +75,11 @@ def test_noalloc_sort_matches_allocating_sort_twice(cfg):
 
 def test_noalloc_sort_rejects_more_than_its_limit():
     d = ss.make_dims(1, 64, 64, 0, 10)
+    limit = max_keys(d)
+    assert limit == 50_311_168  # the limit the header states
     in_b = ct.c_int(0)
     fake = ct.c_void_p(256)  # never dereferenced: the size check comes first
-    st = ss.lib().ss_sort_isects_noalloc(ct.byref(d), fake, fake, fake, fake, MAX_KEYS + 1, fake, ct.byref(in_b),
+    st = ss.lib().ss_sort_isects_noalloc(ct.byref(d), fake, fake, fake, fake, limit + 1, fake, ct.byref(in_b),
                                          None)
     assert st == ss.SS_ERR_INVALID_ARG
-    assert b"static scratch" in ss.lib().ss_last_error()
+    assert f"at most {limit} keys".encode() in ss.lib().ss_last_error()

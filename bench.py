@@ -139,7 +139,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- roofline model
-def stage_model(d, K, nnz, n_isects, passes, n_tiles, work, n_seen=None):
+def stage_model(d, K, nnz, n_isects, passes, n_tiles, work, n_seen=None, depth_passes=4):
     """Algorithmic bytes (HBM) and FP32 instruction counts per call.
 
     bytes: every input the stage needs read once and every output written
@@ -159,9 +159,12 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work, n_seen=None):
     m = {}
     m["project_packed"] = dict(bytes=par * N + P / 8 + P / 32 + P / 16 + (par + 4) * N + shb * n_seen
                                + (row + 8 + 4) * nnz, instr=P * 140.0 + nnz * 160.0)
-    m["intersect_tiles"] = dict(bytes=8 * nnz * 2 + 8 * nnz + 4 * nnz + 12 * n_isects, instr=0.0)
+    # depth keys of the rows (4 B read, 12 B written), their sort (histogram 8
+    # B, 24 B per byte pass), the count in depth order (row id 4 B, AABB 8 B),
+    # the write (row id, depth key, AABB: 20 B; offsets 8 B; 12 B per key)
+    m["intersect_tiles"] = dict(bytes=nnz * (16 + 8 + 24 * depth_passes + 12 + 28) + 12 * n_isects, instr=0.0)
     # histogram (one read), 12 B read + 12 B written per key per digit pass
-    # that runs, tile offsets
+    # that runs (the tile-id bytes: the keys arrive in depth order), tile offsets
     m["sort_isects"] = dict(bytes=n_isects * (8 + 24 * passes) + 8 * (n_tiles + 1), instr=0.0)
     # per-pixel FP32 instructions of the canonical sequences: 11 per evaluated
     # entry (offsets, sigma, tests), 16 per exp (range reduction, degree-7
@@ -326,7 +329,7 @@ def run_ours(args):
                                   step.vals_a, step.cap_isects, step.temp_isect)
         ev[2].record(st)
         in_b = ss.ss_sort_isects(d, step.keys_a, step.vals_a, step.keys_b, step.vals_b, n, step.temp_sort,
-                                 step.tile_off)
+                                 step.tile_off, presorted_depth=True)
         step.vals = step.vals_b if in_b else step.vals_a
         ev[3].record(st)
         # the rasterizers' tile order is part of the forward rasterizer's stage
@@ -436,8 +439,9 @@ def run_ours(args):
     peaks = load_peaks()
     passes = ss.sort_passes_for(step.keys[: step.n_isects], d)
     n_seen = ss.seen_gaussians(d, step.mask)
+    depth_passes = ss.depth_sort_passes(step.row_depth[: step.nnz])
     model = stage_model(d, (d.sh_degree + 1) ** 2, step.nnz, step.n_isects, passes, ss.size(d, ss.SIZE_N_TILES),
-                        work, n_seen)
+                        work, n_seen, depth_passes)
     sm_mhz = clocks["sm_mhz"] or peaks["sm_max_mhz"]
     stages = {}
     for nm in names:
@@ -488,7 +492,7 @@ def run_ours(args):
                config=dict(workload=sc.name if args.n is None else f"{sc.name}, N overridden to {d.N}",
                            C=d.C, N=d.N, W=d.W, H=d.H,
                            sh_degree=d.sh_degree, pairs=d.C * d.N, nnz=step.nnz, n_isects=step.n_isects,
-                           sort_passes=passes, gaussians_seen=n_seen, l2="inputs larger than L2 (3.5 GB parameters), no flush",
+                           sort_passes=passes, depth_sort_passes=depth_passes, gaussians_seen=n_seen, l2="inputs larger than L2 (3.5 GB parameters), no flush",
                            parallelism=f"replicas x{world}", depth_and_background=bool(args.depth_bg),
                            fused_adam=bool(args.adam), grad_quant=bool(args.grad_quant)),
                pairs_per_s=world * d.C * d.N / (ms / 1e3),

@@ -60,7 +60,7 @@ struct DevPlan {
 // the global histogram.
 template <int PASSES>
 __global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __restrict__ keys, int64_t n,
-                                                           uint32_t* __restrict__ hist) {
+                                                           int lo_bytes, uint32_t* __restrict__ hist) {
   extern __shared__ uint32_t hw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int kPerWarp = PASSES * kRadix;
@@ -81,7 +81,7 @@ __global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __res
     const uint32_t above = ~((2u << lane) - 1u);  // lanes above this one
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
-      const uint32_t d = ((p < 4 ? lo >> (8 * p) : hi >> (8 * (p - 4)))) & 0xFFu;
+      const uint32_t d = ((p < lo_bytes ? lo >> (8 * p) : hi >> (8 * (p - lo_bytes)))) & 0xFFu;
       const uint32_t prev = __shfl_up_sync(0xffffffffu, d, 1);
       const bool head = valid && (lane == 0 || d != prev);
       const uint32_t after = __ballot_sync(0xffffffffu, head) & above;
@@ -98,12 +98,12 @@ __global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __res
 }
 
 template <int PASSES>
-ss_status launch_hist(unsigned grid, cudaStream_t st, const uint64_t* keys, int64_t n, uint32_t* hist) {
+ss_status launch_hist(unsigned grid, cudaStream_t st, const uint64_t* keys, int64_t n, int lo_bytes, uint32_t* hist) {
   const size_t smem = sizeof(uint32_t) * kSortWarps * PASSES * kRadix;
   ss_status s = cuda_status(
       cudaFuncSetAttribute(k_hist_all<PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "smem attr");
   if (s) return s;
-  k_hist_all<PASSES><<<grid, kSortThreads, smem, st>>>(keys, n, hist);
+  k_hist_all<PASSES><<<grid, kSortThreads, smem, st>>>(keys, n, lo_bytes, hist);
   return cuda_status(cudaGetLastError(), "radix histogram");
 }
 
@@ -111,7 +111,7 @@ ss_status launch_hist(unsigned grid, cudaStream_t st, const uint64_t* keys, int6
 // skipped when one bin of its histogram holds all n keys; the running passes'
 // histograms are scanned (exclusive) and moved to the front, in order, so
 // running pass k reads hist[k] and the digit at key bit plan->shift[k].
-__global__ __launch_bounds__(kRadix) void k_plan(uint32_t* __restrict__ hist, int passes, int64_t n,
+__global__ __launch_bounds__(kRadix) void k_plan(uint32_t* __restrict__ hist, int passes, int lo_bytes, int64_t n,
                                                  DevPlan* __restrict__ plan) {
   __shared__ uint32_t wt[kRadix / 32];
   __shared__ int s_full;
@@ -135,7 +135,7 @@ __global__ __launch_bounds__(kRadix) void k_plan(uint32_t* __restrict__ hist, in
       uint32_t before = 0;
       for (int w = 0; w < warp; ++w) before += wt[w];
       hist[k * kRadix + threadIdx.x] = before + inc - v;  // k <= p, and row p was read above
-      if (threadIdx.x == 0) plan->shift[k] = p < 4 ? 8 * p : 32 + 8 * (p - 4);
+      if (threadIdx.x == 0) plan->shift[k] = p < lo_bytes ? 8 * p : 32 + 8 * (p - lo_bytes);
       ++k;
     }
     __syncthreads();
@@ -307,12 +307,16 @@ int tile_bits(int64_t ntiles) {
   return b;
 }
 
-int sort_passes(int64_t ntiles) { return 4 + (tile_bits(ntiles) + 7) / 8; }
 
 // Scratch layout: hist [kMaxPasses][256] u32 | tickets [kMaxPasses] u32 |
 // error flag u32 | plan | look-back status [tiles][256] u64.
 constexpr size_t sort_plan_offset() { return align_up(kMaxPasses * kRadix * 4 + kMaxPasses * 4 + 4, 16); }
 constexpr size_t sort_status_offset() { return align_up(sort_plan_offset() + sizeof(DevPlan), 256); }
+
+inline DevPlan* sort_plan(void* temp) { return reinterpret_cast<DevPlan*>(reinterpret_cast<char*>(temp) + sort_plan_offset()); }
+inline const DevPlan* sort_plan(const void* temp) {
+  return reinterpret_cast<const DevPlan*>(reinterpret_cast<const char*>(temp) + sort_plan_offset());
+}
 
 constexpr size_t sort_scratch_bytes(int64_t n) {
   return sort_status_offset() + (size_t)ceil_div(n > 1 ? n : 1, kSortTile) * kRadix * 8;
@@ -324,9 +328,90 @@ size_t sort_temp_bytes(int64_t n) { return sort_scratch_bytes(n); }
 
 using namespace ss;
 
+namespace ss {
+
+// Stable LSD sort of n (key, value) pairs over byte digits: the low word's
+// lo_bytes bytes (4, or 0 when the keys already arrive in the order of their
+// low words, ties in the order to keep), then the high word's hi_bytes bytes.
+// Digits equal in every key are skipped (device plan); the result is in
+// (kb, vb) after an odd number of running passes: plan->count & 1, on the
+// device.  temp: sort_temp_bytes(n), cleared here.  No host synchronisation.
+ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
+                           int hi_bytes, void* temp, cudaStream_t st) {
+  ss_status s = cuda_status(cudaFuncSetAttribute(k_onesweep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)sizeof(OnesweepSmem)),
+                            "set smem attribute");
+  if (s) return s;
+  const int64_t tiles = ceil_div(n, kSortTile);
+  char* tb = reinterpret_cast<char*>(temp);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(tb);
+  uint32_t* tickets = hist + kMaxPasses * kRadix;
+  uint32_t* err = tickets + kMaxPasses;
+  DevPlan* dplan = sort_plan(temp);
+  uint64_t* status = reinterpret_cast<uint64_t*>(tb + sort_status_offset());
+  s = cuda_status(cudaMemsetAsync(temp, 0, sort_status_offset() + (size_t)tiles * kRadix * 8, st), "memset");
+  if (s) return s;
+  (void)err;
+  const int passes = lo_bytes + hi_bytes;
+  if (passes < 1 || passes > kMaxPasses) return invalid("sort digit count");
+  const unsigned hgrid = (unsigned)min64(tiles, 148 * 8);
+  switch (passes) {
+    case 1: s = launch_hist<1>(hgrid, st, ka, n, lo_bytes, hist); break;
+    case 2: s = launch_hist<2>(hgrid, st, ka, n, lo_bytes, hist); break;
+    case 3: s = launch_hist<3>(hgrid, st, ka, n, lo_bytes, hist); break;
+    case 4: s = launch_hist<4>(hgrid, st, ka, n, lo_bytes, hist); break;
+    case 5: s = launch_hist<5>(hgrid, st, ka, n, lo_bytes, hist); break;
+    case 6: s = launch_hist<6>(hgrid, st, ka, n, lo_bytes, hist); break;
+    case 7: s = launch_hist<7>(hgrid, st, ka, n, lo_bytes, hist); break;
+    default: s = launch_hist<8>(hgrid, st, ka, n, lo_bytes, hist); break;
+  }
+  if (s) return s;
+  k_plan<<<1, kRadix, 0, st>>>(hist, passes, lo_bytes, n, dplan);
+  s = cuda_status(cudaGetLastError(), "radix plan");
+  if (s) return s;
+  uint64_t* kin = ka;
+  uint32_t* vin = va;
+  uint64_t* kout = kb;
+  uint32_t* vout = vb;
+  for (int p = 0; p < passes; ++p) {
+    const uint64_t epoch = (uint64_t)(p + 1) << 56;
+    k_onesweep<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
+        kin, vin, kout, vout, n, p, dplan, epoch, hist + p * kRadix, status, tickets + p, err);
+    s = cuda_status(cudaGetLastError(), "radix pass");
+    if (s) return s;
+    std::swap(kin, kout);
+    std::swap(vin, vout);
+  }
+  return SS_OK;
+}
+
+// The device-side count of a sort's running passes (its result is in the
+// second buffer pair when odd).
+const int* sort_passes_run(const void* temp) { return &sort_plan(temp)->count; }
+
+// Reads back a finished sort's look-back flag and pass count (stream sync).
+ss_status radix_sort_result(const void* temp, cudaStream_t st, int* passes_run, bool* flagged) {
+  const char* tb = reinterpret_cast<const char*>(temp);
+  const uint32_t* err = reinterpret_cast<const uint32_t*>(tb) + kMaxPasses * kRadix + kMaxPasses;
+  uint32_t herr = 0;
+  int count = 0;
+  ss_status s = cuda_status(cudaMemcpyAsync(&herr, err, 4, cudaMemcpyDeviceToHost, st), "copy sort flag");
+  if (s) return s;
+  s = cuda_status(cudaMemcpyAsync(&count, &sort_plan(temp)->count, sizeof(int), cudaMemcpyDeviceToHost, st),
+                  "copy sort plan");
+  if (s) return s;
+  s = cuda_status(cudaStreamSynchronize(st), "sort");
+  if (s) return s;
+  *passes_run = count;
+  *flagged = herr != 0;
+  return SS_OK;
+}
+
+}  // namespace ss
+
 extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
-                                    uint32_t* vals_b, int64_t n, void* temp, size_t temp_bytes, int64_t* tile_off,
-                                    int* result_in_b_out, void* stream) {
+                                    uint32_t* vals_b, int64_t n, int presorted_depth, void* temp, size_t temp_bytes,
+                                    int64_t* tile_off, int* result_in_b_out, void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (!result_in_b_out || !tile_off) return invalid("null output");
   if (n < 0) return invalid("n < 0");
@@ -340,62 +425,22 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   if (n == 0) return cuda_status(cudaMemsetAsync(tile_off, 0, sizeof(int64_t) * (g.n_tiles + 1), st), "memset");
   if (!keys_a || !vals_a || !keys_b || !vals_b) return invalid("null keys/vals");
   if (!temp || temp_bytes < sort_temp_bytes(n)) return invalid("temp too small");
-  ss_status s = cuda_status(cudaFuncSetAttribute(k_onesweep, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)sizeof(OnesweepSmem)),
-                            "set smem attribute");
+  // every byte of the depth (none when the keys arrive in depth order) and
+  // the bytes of the tile ids; the plan drops the bytes that do not vary
+  const int lo_bytes = presorted_depth ? 0 : 4;
+  const int hi_bytes = max((tile_bits(g.n_tiles) + 7) / 8, lo_bytes ? 0 : 1);
+  ss_status s = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, n, lo_bytes, hi_bytes, temp, st);
   if (s) return s;
-  const int64_t tiles = ceil_div(n, kSortTile);
-  char* tb = reinterpret_cast<char*>(temp);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(tb);
-  uint32_t* tickets = hist + kMaxPasses * kRadix;
-  uint32_t* err = tickets + kMaxPasses;
-  DevPlan* dplan = reinterpret_cast<DevPlan*>(tb + sort_plan_offset());
-  uint64_t* status = reinterpret_cast<uint64_t*>(tb + sort_status_offset());
-  s = cuda_status(cudaMemsetAsync(temp, 0, sort_status_offset() + (size_t)tiles * kRadix * 8, st), "memset");
-  if (s) return s;
-  // the full plan: every byte of the depth and the bytes of the tile ids;
-  // k_plan drops the bytes that do not vary
-  const int passes = sort_passes(g.n_tiles);
-  const unsigned hgrid = (unsigned)min64(tiles, 148 * 8);
-  switch (passes) {
-    case 4: s = launch_hist<4>(hgrid, st, keys_a, n, hist); break;
-    case 5: s = launch_hist<5>(hgrid, st, keys_a, n, hist); break;
-    case 6: s = launch_hist<6>(hgrid, st, keys_a, n, hist); break;
-    case 7: s = launch_hist<7>(hgrid, st, keys_a, n, hist); break;
-    default: s = launch_hist<8>(hgrid, st, keys_a, n, hist); break;
-  }
-  if (s) return s;
-  k_plan<<<1, kRadix, 0, st>>>(hist, passes, n, dplan);
-  s = cuda_status(cudaGetLastError(), "radix plan");
-  if (s) return s;
-  uint64_t* kin = keys_a;
-  uint32_t* vin = vals_a;
-  uint64_t* kout = keys_b;
-  uint32_t* vout = vals_b;
-  for (int p = 0; p < passes; ++p) {
-    const uint64_t epoch = (uint64_t)(p + 1) << 56;
-    k_onesweep<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
-        kin, vin, kout, vout, n, p, dplan, epoch, hist + p * kRadix, status, tickets + p, err);
-    s = cuda_status(cudaGetLastError(), "radix pass");
-    if (s) return s;
-    std::swap(kin, kout);
-    std::swap(vin, vout);
-  }
   const unsigned grid = (unsigned)ceil_div(n + 1, 256);
-  k_tile_ranges<<<grid, 256, 0, st>>>(keys_a, keys_b, n, g.n_tiles, dplan, tile_off);
+  k_tile_ranges<<<grid, 256, 0, st>>>(keys_a, keys_b, n, g.n_tiles, sort_plan(temp), tile_off);
   s = cuda_status(cudaGetLastError(), "tile ranges");
   if (s) return s;
-  // the error flag and the plan's pass count, read together
-  uint32_t hbuf[2] = {0u, 0u};
-  s = cuda_status(cudaMemcpyAsync(&hbuf[0], err, 4, cudaMemcpyDeviceToHost, st), "copy sort flag");
-  if (s) return s;
   int count = 0;
-  s = cuda_status(cudaMemcpyAsync(&count, &dplan->count, sizeof(int), cudaMemcpyDeviceToHost, st), "copy sort plan");
-  if (s) return s;
-  s = cuda_status(cudaStreamSynchronize(st), "sort");
+  bool flagged = false;
+  s = radix_sort_result(temp, st, &count, &flagged);
   if (s) return s;
   *result_in_b_out = count & 1;
-  if (hbuf[0]) {
+  if (flagged) {
     set_error("ss_sort_isects: look-back wait exceeded its limit");
     return SS_ERR_DEVICE_CHECK;
   }
@@ -493,6 +538,6 @@ extern "C" ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_
     ss_status s = noalloc_scratch(&scratch);
     if (s) return s;
   }
-  return ss_sort_isects(dims, keys_a, vals_a, keys_b, vals_b, n, scratch, kNoAllocScratchBytes, tile_off,
+  return ss_sort_isects(dims, keys_a, vals_a, keys_b, vals_b, n, 0, scratch, kNoAllocScratchBytes, tile_off,
                         result_in_b_out, stream);
 }

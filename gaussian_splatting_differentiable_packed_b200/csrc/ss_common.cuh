@@ -99,11 +99,16 @@ inline int64_t wave_blocks(K kernel, int threads, size_t smem) {
 
 // ----- generic exclusive scan (int64 totals), defined in scan.cu -----
 // Items are produced by a "counter" selected by kind:
-enum ScanKind { SCAN_U32 = 0, SCAN_TILES = 1 };
+enum ScanKind { SCAN_U32 = 0, SCAN_TILES = 1, SCAN_TILES_ORDERED = 2 };
 struct ScanSrc {
   int kind;
   const uint32_t* u32;     // SCAN_U32: counts
   const uint32_t* aabb16;  // SCAN_TILES: per-row AABB16, count = tiles covered
+  // SCAN_TILES_ORDERED: item i is row order[i], order = rows_b when the
+  // sort that wrote it ran an odd number of passes (*passes_run), else rows_a
+  const uint32_t* rows_a;
+  const uint32_t* rows_b;
+  const int* passes_run;
   int W, H, tiles_x, tiles_y;
 };
 constexpr int kScanItems = 16;

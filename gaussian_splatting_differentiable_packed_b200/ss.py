@@ -87,7 +87,7 @@ def lib() -> ct.CDLL:
         L.ss_last_error.restype = ct.c_char_p
         L.ss_project_packed.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, i64, i64, P, sz, ct.POINTER(i64), P]
         L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
-        L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, P, sz, P, ct.POINTER(i32), P]
+        L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, i32, P, sz, P, ct.POINTER(i32), P]
         L.ss_sort_isects_noalloc.argtypes = [D, P, P, P, P, i64, P, ct.POINTER(i32), P]
         L.ss_tile_order.argtypes = [D, P, P, P, sz, P]
         L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P]
@@ -167,9 +167,12 @@ def ss_intersect_tiles(d, row_depth, aabb16, block_off, nnz, isect_off, keys, va
     return int(n.value)
 
 
-def ss_sort_isects(d, keys_a, vals_a, keys_b, vals_b, n, temp, tile_off, stream=None) -> bool:
+def ss_sort_isects(d, keys_a, vals_a, keys_b, vals_b, n, temp, tile_off, stream=None, presorted_depth=False) -> bool:
+    """presorted_depth: the keys arrive in depth order (as ss_intersect_tiles
+    writes them), so only the tile-id bytes are sorted."""
     in_b = ct.c_int(0)
-    st = lib().ss_sort_isects(ct.byref(d), _p(keys_a), _p(vals_a), _p(keys_b), _p(vals_b), int(n), _p(temp),
+    st = lib().ss_sort_isects(ct.byref(d), _p(keys_a), _p(vals_a), _p(keys_b), _p(vals_b), int(n),
+                              1 if presorted_depth else 0, _p(temp),
                               0 if temp is None else temp.numel() * temp.element_size(), _p(tile_off),
                               ct.byref(in_b), _stream(stream))
     _check(st, "ss_sort_isects")
@@ -420,7 +423,7 @@ class PackedStep:
         self.unsorted_keys = self.keys_a
         self.unsorted_vals = self.vals_a
         self.result_in_b = ss_sort_isects(d, self.keys_a, self.vals_a, self.keys_b, self.vals_b, n, self.temp_sort,
-                                          self.tile_off, stream)
+                                          self.tile_off, stream, presorted_depth=True)
         self.keys = self.keys_b if self.result_in_b else self.keys_a
         self.vals = self.vals_b if self.result_in_b else self.vals_a
         ss_tile_order(d, self.tile_off, self.tile_order, self.temp_order, stream)
@@ -451,21 +454,33 @@ def scene_dims(scene) -> ss_dims:
     return make_dims(scene.C, scene.W, scene.H, scene.sh_degree, scene.N, scene.near, scene.far)
 
 
-def sort_passes_for(keys, d: ss_dims) -> int:
-    """Digit passes ss_sort_isects runs on these (unsorted or sorted) keys:
-    one per byte of the depth and per byte the tile ids need, less the bytes
-    that are equal in every key.  Measurement helper (torch reductions); not
-    part of any step."""
-    if keys.numel() == 0:
-        return 0
-    k = keys.to(torch.int64)
-    tb = max(0, (size(d, SIZE_N_TILES) - 1).bit_length())
-    shifts = [0, 8, 16, 24] + [32 + 8 * i for i in range((tb + 7) // 8)]
+def _varying_bytes(k, shifts) -> int:
     n = 0
     for sh in shifts:
         dig = (k >> sh) & 0xFF
         n += int(dig.min().item()) != int(dig.max().item())
     return n
+
+
+def sort_passes_for(keys, d: ss_dims, presorted_depth: bool = True) -> int:
+    """Digit passes ss_sort_isects runs on these (unsorted or sorted) keys:
+    one per byte the tile ids need and, unless the keys arrive in depth order,
+    per byte of the depth, less the bytes that are equal in every key.
+    Measurement helper (torch reductions); not part of any step."""
+    if keys.numel() == 0:
+        return 0
+    k = keys.to(torch.int64)
+    tb = max(0, (size(d, SIZE_N_TILES) - 1).bit_length())
+    hi = [32 + 8 * i for i in range(max((tb + 7) // 8, 1 if presorted_depth else 0))]
+    return _varying_bytes(k, ([] if presorted_depth else [0, 8, 16, 24]) + hi)
+
+
+def depth_sort_passes(row_depth) -> int:
+    """Digit passes of the intersection's depth sort of its rows: the bytes of
+    the rows' depth bits that are not equal in every row.  Measurement helper."""
+    if row_depth.numel() == 0:
+        return 0
+    return _varying_bytes(row_depth.view(torch.int32).to(torch.int64) & 0xFFFFFFFF, [0, 8, 16, 24])
 
 
 def seen_gaussians(d: ss_dims, mask) -> int:
@@ -483,20 +498,21 @@ def seen_gaussians(d: ss_dims, mask) -> int:
     return int(pop.sum().item())
 
 
-def sort_launches(d: ss_dims, n_isects: int) -> int:
+def sort_launches(d: ss_dims, n_isects: int, presorted_depth: bool = True) -> int:
     """Kernels of one ss_sort_isects call: histogram, plan, one onesweep
     kernel per byte of the full plan (a skipped byte's kernel returns at
     once), tile ranges."""
     if n_isects == 0:
         return 0
     tb = max(0, (size(d, SIZE_N_TILES) - 1).bit_length())
-    return 2 + 4 + (tb + 7) // 8 + 1
+    return 2 + (0 if presorted_depth else 4) + max((tb + 7) // 8, 1 if presorted_depth else 0) + 1
 
 
 def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
     """Kernels libss launches in one forward+backward step (memsets excluded):
-    projection 5 (pass 1, three scan kernels, pass 2), intersection 3 (two
-    count kernels, the fused offsets-and-write kernel), the sort
+    projection 5 (pass 1, three scan kernels, pass 2), intersection 10 (row
+    depth keys, the depth sort's histogram, plan and 4 byte passes, two count
+    kernels, the fused offsets-and-write kernel), the sort
     (sort_launches), tile order 3 (histogram, scan, scatter), rasterizer
     1 + 1, projection backward 1.  With no Gaussians only the tile order and the two
     rasterizers launch (they still write the empty images)."""
@@ -504,7 +520,7 @@ def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
         return 3 + 2
     n = 5
     if nnz > 0:
-        n += 3
+        n += 10
     n += sort_launches(d, n_isects)
     return n + 3 + 3
 

@@ -157,11 +157,15 @@ ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float*
  * Counts the tiles of each row from its AABB16 (integer arithmetic), sums them
  * exactly in 64 bits and returns the total in *n_isects_out (stream sync).
  * Returns SS_ERR_CAPACITY if the total exceeds cap_isects and
- * SS_ERR_OVERFLOW if it is >= 2^31, writing nothing else in either case.
- * Otherwise writes isect_off[nnz+1] (exclusive per-row offsets) and one
- * (key, row) per covered tile, row-major over (row, ty, tx); the key's depth
- * bits come from row_depth.  block_off, aabb16 and row_depth are the arrays
- * ss_project_packed wrote (block_off gives each camera's first row).
+ * SS_ERR_OVERFLOW if it is >= 2^31, writing no key in either case.
+ * Otherwise writes one (key, row) per covered tile, the rows taken in order
+ * of their depth (the IEEE bits of row_depth, ties by row index), each row's
+ * tiles row-major over (ty, tx), so that ss_sort_isects can sort the tile
+ * ids alone (presorted_depth); isect_off[nnz+1] holds the exclusive offsets
+ * of the rows in that order.  block_off, aabb16 and row_depth are the arrays
+ * ss_project_packed wrote (block_off gives each camera's first row).  temp:
+ * ss_workspace_bytes(SS_WS_INTERSECT, nnz) bytes (it holds the depth order
+ * of the rows).
  */
 ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_depth, const uint32_t* aabb16,
                              const int64_t* block_off, int64_t nnz, int64_t* isect_off, uint64_t* keys,
@@ -172,16 +176,19 @@ ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_depth, const 
  * Stable LSD radix sort of n (key, value) pairs by key, 8-bit digits over the
  * 32 depth bits and the tile-id bits only ("Spirula Studio VRAM deep-dive",
  * buffer table: double-buffered isect.ids_a/b); a digit that is equal in
- * every key is skipped (it cannot change the order).  Ping-pongs between
- * (keys_a, vals_a) and (keys_b, vals_b); *result_in_b_out (host) says which
- * pair holds the result (b after an odd number of digit passes, which depends
- * on the keys).  Then writes tile_off[n_tiles+1].
+ * every key is skipped (it cannot change the order).  presorted_depth != 0
+ * says the keys arrive in ascending order of their low words (the depths),
+ * ties in the order to keep, as ss_intersect_tiles writes them: the tile-id
+ * bytes alone are then sorted, which yields the same order.  Ping-pongs
+ * between (keys_a, vals_a) and (keys_b, vals_b); *result_in_b_out (host)
+ * says which pair holds the result (b after an odd number of digit passes,
+ * which depends on the keys).  Then writes tile_off[n_tiles+1].
  * n >= 2^31 returns SS_ERR_OVERFLOW.  Equal keys keep their input order.
  * Synchronises the stream at the end (reads the look-back error flag).
  */
 ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
-                         uint32_t* vals_b, int64_t n, void* temp, size_t temp_bytes, int64_t* tile_off,
-                         int* result_in_b_out, void* stream);
+                         uint32_t* vals_b, int64_t n, int presorted_depth, void* temp, size_t temp_bytes,
+                         int64_t* tile_off, int* result_in_b_out, void* stream);
 
 /*
  * Projection backward fused with an Adam step (the pages' fused projection

@@ -807,20 +807,36 @@ int orc_count_tiles(const orc_dims* d, const uint32_t* aabb, int64_t nnz, int64_
 // float box by less than one quantisation step).  Writes (key, row) in
 // row-major order over (row, ty, tx).  Returns 0, -1 on a disagreement, -2 if
 // the capacity is short (the total is still exact).
+// Intersection keys.  Rows are visited in order of their depth (the IEEE bits
+// of the fp32 camera-space depth, ties by row index), each row's tiles
+// row-major over (ty, tx); order_out (nullable) receives the visiting order.
+// Write order is a layout choice (the keys themselves are the page's); with
+// the rows in depth order, a stable sort by tile id alone yields the key order.
 int orc_intersect(const orc_dims* d, const double* screen, const uint32_t* aabb, const int32_t* row_cam, int64_t nnz,
-                  int all_pairs, uint64_t* keys, uint32_t* vals, int64_t cap, uint64_t* total_out) {
+                  int all_pairs, uint64_t* keys, uint32_t* vals, int64_t cap, uint64_t* total_out, int64_t* order_out) {
   Geo geo = geometry(d);
   std::vector<int64_t> per_row((size_t)nnz);
   uint64_t total = 0;
   orc_count_tiles(d, aabb, nnz, per_row.data(), &total);
   *total_out = total;
   if ((int64_t)total > cap) return -2;
+  std::vector<uint32_t> dbits_of((size_t)nnz);
+  for (int64_t r = 0; r < nnz; ++r) {
+    float depth32 = (float)screen[r * kRow + 9];
+    std::memcpy(&dbits_of[r], &depth32, 4);
+  }
+  std::vector<int64_t> order((size_t)nnz);
+  for (int64_t r = 0; r < nnz; ++r) order[r] = r;
+  std::stable_sort(order.begin(), order.end(), [&](int64_t a, int64_t b) { return dbits_of[a] < dbits_of[b]; });
+  if (order_out)
+    for (int64_t p = 0; p < nnz; ++p) order_out[p] = order[p];
   std::vector<int64_t> off((size_t)nnz + 1);
   off[0] = 0;
-  for (int64_t r = 0; r < nnz; ++r) off[r + 1] = off[r] + per_row[r];
+  for (int64_t p = 0; p < nnz; ++p) off[p + 1] = off[p] + per_row[order[p]];
   int bad = 0;
 #pragma omp parallel for schedule(dynamic, 256) reduction(| : bad)
-  for (int64_t r = 0; r < nnz; ++r) {
+  for (int64_t p = 0; p < nnz; ++p) {
+    const int64_t r = order[p];
     uint32_t qx0 = aabb[2 * r] & 0xFFFFu, qx1 = aabb[2 * r + 1] & 0xFFFFu;
     uint32_t qy0 = aabb[2 * r] >> 16, qy1 = aabb[2 * r + 1] >> 16;
     int64_t tx0, tx1, ty0, ty1;
@@ -836,11 +852,9 @@ int orc_intersect(const orc_dims* d, const double* screen, const uint32_t* aabb,
       wy0 = std::max<int64_t>(0, (int64_t)std::floor(fy0 / kTile) - 1);
       wy1 = std::min<int64_t>(geo.tiles_y, (int64_t)std::ceil(fy1 / kTile) + 1);
     }
-    int64_t w = off[r];
+    int64_t w = off[p];
     // key low word: IEEE bits of the fp32 camera-space depth
-    float depth32 = (float)screen[r * kRow + 9];
-    uint32_t dbits;
-    std::memcpy(&dbits, &depth32, 4);
+    const uint32_t dbits = dbits_of[r];
     const uint64_t cam_base = (uint64_t)row_cam[r] * (uint64_t)geo.tiles_per_cam;
     int64_t found = 0;
     for (int64_t ty = wy0; ty < wy1; ++ty) {

@@ -51,7 +51,7 @@ def lib():
         L.orc_project.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, P, P, P, P, P, i64, i32, i64]
         L.orc_row_boxes.argtypes = [P, P, P, P, P, P, P, P, i64, P]
         L.orc_count_tiles.argtypes = [P, P, i64, P, P]
-        L.orc_intersect.argtypes = [P, P, P, P, i64, i32, P, P, i64, P]
+        L.orc_intersect.argtypes = [P, P, P, P, i64, i32, P, P, i64, P, P]
         L.orc_sort.argtypes = [P, P, i64]
         L.orc_tile_ranges.argtypes = [P, i64, i64, P]
         L.orc_rasterize_fwd.argtypes = [P, P, P, P, i32, P, P, P, P, P, i32, P, P]
@@ -183,6 +183,8 @@ def count_tiles(scene, aabb) -> tuple[np.ndarray, int]:
 
 
 def intersect(scene, proj, all_pairs: bool | None = None) -> dict:
+    """Intersection keys and values, rows visited in order of depth (ties by
+    row index), each row's tiles row-major; `order` is that visiting order."""
     g = geometry(scene)
     d = dims_of(scene)
     n = proj["nnz"]
@@ -191,13 +193,14 @@ def intersect(scene, proj, all_pairs: bool | None = None) -> dict:
         all_pairs = n * g["tiles_per_cam"] <= 200_000_000
     keys = np.zeros(max(total, 1), np.uint64)
     vals = np.zeros(max(total, 1), np.uint32)
+    order = np.zeros(max(n, 1), np.int64)
     tot = ct.c_uint64(0)
     rc = lib().orc_intersect(ct.byref(d), _p(_c(proj["screen"], np.float64)), _p(_c(proj["aabb"], np.uint32)),
                              _p(_c(proj["row_cam"], np.int32)), n, int(all_pairs), _p(keys), _p(vals), total,
-                             ct.byref(tot))
+                             ct.byref(tot), _p(order))
     if rc != 0:
         raise RuntimeError(f"oracle intersect: range form and overlap test disagree (rc={rc})")
-    return dict(keys=keys[:total], vals=vals[:total], n_isects=int(tot.value))
+    return dict(keys=keys[:total], vals=vals[:total], n_isects=int(tot.value), order=order[:n])
 
 
 def sort(keys, vals) -> tuple[np.ndarray, np.ndarray]:

@@ -45,12 +45,13 @@ def test_traffic_record_guards(tmp_path, monkeypatch):
 
 
 def test_launches_per_step():
-    """projection 5, intersection 3 (two count kernels, the fused write), the
-    sort's histogram, plan, one kernel per byte of the full plan and tile
-    ranges, the tile order 3, rasterizers 2, projection backward 1."""
+    """projection 5, intersection 10 (row depth keys, the depth sort's
+    histogram, plan and 4 byte passes, two count kernels, the fused write),
+    the sort's histogram, plan, one kernel per tile-id byte and tile ranges,
+    the tile order 3, rasterizers 2, projection backward 1."""
     d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)  # 33,500 tiles: 16 tile-id bits, 2 bytes
-    assert ss.launches_per_step(d, 15_000_000, 33_000_000) == 5 + 3 + (2 + 6 + 1) + 3 + 2 + 1
-    assert ss.launches_per_step(d, 15_000_000, 0) == 5 + 3 + 0 + 3 + 2 + 1
+    assert ss.launches_per_step(d, 15_000_000, 33_000_000) == 5 + 10 + (2 + 2 + 1) + 3 + 2 + 1
+    assert ss.launches_per_step(d, 15_000_000, 0) == 5 + 10 + 0 + 3 + 2 + 1
     assert ss.launches_per_step(d, 0, 0) == 5 + 0 + 0 + 3 + 2 + 1
     assert ss.launches_per_step(ss.make_dims(1, 64, 64, 0, 0), 0, 0) == 3 + 2
 
@@ -63,9 +64,12 @@ def test_sort_passes_skip_constant_bytes():
     d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)
     tiles = torch.arange(0, 33_500, dtype=torch.int64)
     depth = torch.full_like(tiles, 0x41000000) + (tiles * 1237) % (1 << 23)
-    assert ss.sort_passes_for((tiles << 32) | depth, d) == 5
-    assert ss.sort_passes_for(torch.tensor([7, 6], dtype=torch.int64), d) == 1
-    assert ss.sort_passes_for(torch.tensor([5, 5], dtype=torch.int64), d) == 0
+    assert ss.sort_passes_for((tiles << 32) | depth, d, presorted_depth=False) == 5
+    assert ss.sort_passes_for(torch.tensor([7, 6], dtype=torch.int64), d, presorted_depth=False) == 1
+    assert ss.sort_passes_for(torch.tensor([5, 5], dtype=torch.int64), d, presorted_depth=False) == 0
+    # keys in depth order: the tile-id bytes only
+    assert ss.sort_passes_for((tiles << 32) | depth, d) == 2
+    assert ss.depth_sort_passes(torch.tensor([1.5, 2.5, 3.0])) == 2
 
 
 def test_oracle_sample_never_exceeds_the_workload():

@@ -67,7 +67,9 @@ def check_forward(scene, o, step):
     I = o["isect"]["n_isects"]
     assert step.n_isects == I
     per, _ = orc.count_tiles(scene, p["aabb"])
-    np.testing.assert_array_equal(step.isect_off[: n + 1].cpu().numpy(), np.concatenate([[0], np.cumsum(per)]))
+    # rows are written in depth order: the offsets follow that order
+    order = o["isect"]["order"]
+    np.testing.assert_array_equal(step.isect_off[: n + 1].cpu().numpy(), np.concatenate([[0], np.cumsum(per[order])]))
     if I:
         np.testing.assert_array_equal(step.keys[:I].cpu().numpy().view(np.uint64), o["keys_sorted"])
         np.testing.assert_array_equal(u32(step.vals[:I]), o["vals_sorted"])

@@ -35,7 +35,7 @@ def make_keys(rng, n_tiles, n, hot=()):
     return keys, vals
 
 
-def run_sort(d, keys, vals):
+def run_sort(d, keys, vals, presorted_depth=False):
     n = len(keys)
     ka = torch.from_numpy(keys.view(np.int64).copy()).cuda()
     va = torch.from_numpy(vals.view(np.int32).copy()).cuda()
@@ -44,7 +44,7 @@ def run_sort(d, keys, vals):
     n_tiles = ss.size(d, ss.SIZE_N_TILES)
     tile_off = torch.empty(n_tiles + 1, dtype=torch.int64, device="cuda")
     temp = torch.empty(ss.workspace_bytes(d, ss.WS_SORT, n), dtype=torch.uint8, device="cuda")
-    in_b = ss.ss_sort_isects(d, ka, va, kb, vb, n, temp, tile_off)
+    in_b = ss.ss_sort_isects(d, ka, va, kb, vb, n, temp, tile_off, presorted_depth=presorted_depth)
     torch.cuda.synchronize()
     k, v = (kb, vb) if in_b else (ka, va)
     return in_b, k.cpu().numpy().view(np.uint64), v.cpu().numpy().view(np.uint32), tile_off.cpu().numpy()
@@ -62,7 +62,7 @@ def test_sort_paths(case):
            "three_tile_bytes": [(81919, 2500)]}[case]
     keys, vals = make_keys(rng, n_tiles, 300_000, hot)
     in_b, gk, gv, toff = run_sort(d, keys, vals)
-    assert in_b == bool(ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d) & 1)
+    assert in_b == bool(ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d, presorted_depth=False) & 1)
     ok, ov = orc.sort(keys, vals)
     np.testing.assert_array_equal(gk, ok)
     np.testing.assert_array_equal(gv, ov)
@@ -98,7 +98,7 @@ def test_sort_skipped_digit_plans():
         rng.integers(0, 2**32, 200_000, dtype=np.uint64)
     for keys, passes in ((same, 0), (one_bit, 1), (top, 5), (full, 6)):
         vals = rng.permutation(len(keys)).astype(np.uint32)
-        p = ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d)
+        p = ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d, presorted_depth=False)
         assert p == passes
         in_b, gk, gv, toff = run_sort(d, keys, vals)
         assert in_b == bool(p & 1)
@@ -106,3 +106,23 @@ def test_sort_skipped_digit_plans():
         np.testing.assert_array_equal(gk, ok)
         np.testing.assert_array_equal(gv, ov)
         np.testing.assert_array_equal(toff, orc.tile_ranges(ok, n_tiles))
+
+
+@pytest.mark.parametrize("case", ["tiles4096", "tiles81920"])
+def test_sort_presorted_depth(case):
+    """Keys that arrive in depth order (ties in the order to keep), as the
+    intersection writes them: sorting the tile-id bytes alone gives the full
+    stable key order."""
+    rng = np.random.default_rng(17)
+    d = ss.make_dims(1, 1024, 1024, 0, 1, 0.01, 1e10) if case == "tiles4096" else \
+        ss.make_dims(5, 2048, 2048, 0, 1, 0.01, 1e10)
+    n_tiles = ss.size(d, ss.SIZE_N_TILES)
+    keys, vals = make_keys(rng, n_tiles, 300_000, [(n_tiles - 1, 3000), (3, 9000)])
+    order = np.argsort((keys & np.uint64(0xFFFFFFFF)).astype(np.uint32), kind="stable")
+    keys, vals = keys[order], vals[order]
+    in_b, gk, gv, toff = run_sort(d, keys, vals, presorted_depth=True)
+    assert in_b == bool(ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d, presorted_depth=True) & 1)
+    ok, ov = orc.sort(keys, vals)
+    np.testing.assert_array_equal(gk, ok)
+    np.testing.assert_array_equal(gv, ov)
+    np.testing.assert_array_equal(toff, orc.tile_ranges(ok, n_tiles))

@@ -266,11 +266,26 @@ def test_keys_layout_and_sort_against_lexsort():
     np.testing.assert_array_equal(cams, pr["row_cam"][v])
     depth = (k & np.uint64(0xFFFFFFFF)).astype(np.uint32).view(np.float32)
     np.testing.assert_array_equal(depth, pr["screen"][v, 9].astype(np.float32))
-    assert np.all(np.diff(v.astype(np.int64)) >= 0)  # written row-major
+    # written row by row in order of depth (ties by row index), each row's
+    # tiles contiguous
+    dbits = (k & np.uint64(0xFFFFFFFF)).astype(np.uint32)
+    assert np.all(np.diff(dbits.astype(np.int64)) >= 0)
+    runs = v[np.concatenate([[True], v[1:] != v[:-1]])]
+    np.testing.assert_array_equal(runs, it["order"][np.isin(it["order"], v)])
+    assert len(np.unique(runs)) == len(runs)
+    rd = pr["screen"][:, 9].astype(np.float32).view(np.uint32)
+    np.testing.assert_array_equal(it["order"], np.lexsort((np.arange(pr["nnz"]), rd)))
     ks, vs = orc.sort(k, v)
     order = np.lexsort((np.arange(len(k)), k))
     np.testing.assert_array_equal(ks, k[order])
     np.testing.assert_array_equal(vs, v[order])
+    # the sorted order is (tile, depth, row); with the rows written in depth
+    # order a stable sort by the tile id alone reaches it
+    by_tile = np.argsort(tiles, kind="stable")
+    np.testing.assert_array_equal(k[by_tile], ks)
+    np.testing.assert_array_equal(v[by_tile], vs)
+    full = np.lexsort((v.astype(np.int64), dbits, tiles))
+    np.testing.assert_array_equal(v[full], vs)
     off = orc.tile_ranges(ks, g["n_tiles"])
     np.testing.assert_array_equal(np.diff(off), np.bincount(tiles, minlength=g["n_tiles"]))
 

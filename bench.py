@@ -484,7 +484,7 @@ def run_ours(args):
             fp = fp32_peak_flops(sm_mhz) / 1e12
             roof["flop_model"] = dict(achieved=round(fa, 3), peak=round(fp, 3), unit="TFLOP/s", frac=round(fa / fp, 4),
                                       model="E * (12 + 1 exp) + C * 10 per pass, x3 for the backward")
-    launches = ss.launches_per_step(d, step.nnz, step.n_isects) * args.steps
+    launches = ss.launches_per_step(d, step.nnz, step.n_isects, passes, depth_passes) * args.steps
     out_work = dict(work)
     out = dict(metric=METRIC, value=job_throughput(step.n_isects, world, ms), unit="isects/s", n_gpus=world,
                steps=args.steps, warmup=args.warmup, ms_per_step=round(ms, 4), higher_is_better=True,

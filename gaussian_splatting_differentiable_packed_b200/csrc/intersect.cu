@@ -12,8 +12,7 @@
 // workload, 59 on the 7680^2 one).
 //
 //   k_row_keys      (depth bits, row) of every row
-//   radix sort      stable, by depth (sort.cu), result in either buffer pair
-//                   (the parity is read on the device)
+//   radix sort      stable, by depth (sort.cu)
 //   count           per-row tiles from the AABB16 by integer arithmetic, in
 //                   depth order: CTA sums per 4096 rows and a single-CTA scan
 //                   give the exact int64 total (no atomics: deterministic)
@@ -33,9 +32,8 @@ namespace ss {
 
 size_t sort_temp_bytes(int64_t n);
 ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
-                           int hi_bytes, void* temp, cudaStream_t st);
-ss_status radix_sort_result(const void* temp, cudaStream_t st, int* passes_run, bool* flagged);
-const int* sort_passes_run(const void* temp);
+                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b);
+ss_status radix_sort_flag(const void* temp, cudaStream_t st, bool* flagged);
 
 constexpr int kIxThreads = 512;
 constexpr int kIxRows = (int)kScanTile;  // rows per CTA: the count pass's tiling
@@ -69,11 +67,8 @@ __device__ __forceinline__ int camera_of_row(const int64_t* __restrict__ block_o
   return lo;
 }
 
-__global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_t* __restrict__ dkeys_a,
-                                                            const uint64_t* __restrict__ dkeys_b,
-                                                            const uint32_t* __restrict__ rows_a,
-                                                            const uint32_t* __restrict__ rows_b,
-                                                            const int* __restrict__ passes_run,
+__global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_t* __restrict__ dkeys,
+                                                            const uint32_t* __restrict__ rows,
                                                             const uint32_t* __restrict__ aabb16,
                                                             const int64_t* __restrict__ block_off,
                                                             const int64_t* __restrict__ partial, int64_t nnz,
@@ -83,9 +78,6 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
   extern __shared__ __align__(16) unsigned char ix_raw[];
   IxSmem& S = *reinterpret_cast<IxSmem*>(ix_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool in_b = (*passes_run) & 1;
-  const uint64_t* dkeys = in_b ? dkeys_b : dkeys_a;
-  const uint32_t* rows = in_b ? rows_b : rows_a;
   const int64_t p0 = (int64_t)blockIdx.x * kIxRows;
   const int nr = (int)min64(kIxRows, nnz - p0);
   // decode the rows of positions p0 .. p0 + nr of the depth order, coalesced
@@ -220,16 +212,16 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   k_row_keys<<<(unsigned)ceil_div(nnz, 256), 256, 0, st>>>(row_depth, nnz, t.dk_a, t.rows_a);
   ss_status s = cuda_status(cudaGetLastError(), "row keys");
   if (s) return s;
-  s = radix_sort_pairs(t.dk_a, t.rows_a, t.dk_b, t.rows_b, nnz, 4, 0, t.sort, st);
+  bool in_b = false;
+  s = radix_sort_pairs(t.dk_a, t.rows_a, t.dk_b, t.rows_b, nnz, 4, 0, t.sort, st, &in_b);
   if (s) return s;
-  const int* passes_run = sort_passes_run(t.sort);
+  const uint64_t* dkeys = in_b ? t.dk_b : t.dk_a;
+  const uint32_t* rows = in_b ? t.rows_b : t.rows_a;
   // the exact total, counted in that order
   ScanSrc src{};
   src.kind = SCAN_TILES_ORDERED;
   src.aabb16 = aabb16;
-  src.rows_a = t.rows_a;
-  src.rows_b = t.rows_b;
-  src.passes_run = passes_run;
+  src.rows = rows;
   src.W = g.W; src.H = g.H; src.tiles_x = g.tiles_x; src.tiles_y = g.tiles_y;
   s = scan_phase1(src, nnz, t.scan, isect_off + nnz, st);
   if (s) return s;
@@ -237,9 +229,8 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   s = cuda_status(cudaMemcpyAsync(&total, isect_off + nnz, sizeof(int64_t), cudaMemcpyDeviceToHost, st),
                   "copy n_isects");
   if (s) return s;
-  int passes = 0;
   bool flagged = false;
-  s = radix_sort_result(t.sort, st, &passes, &flagged);  // synchronises the stream
+  s = radix_sort_flag(t.sort, st, &flagged);  // synchronises the stream
   if (s) return s;
   if (flagged) {
     set_error("ss_intersect_tiles: the depth sort's look-back wait exceeded its limit");
@@ -262,7 +253,6 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
                   "set smem attribute");
   if (s) return s;
   k_isect_fused<<<(unsigned)ceil_div(nnz, kIxRows), kIxThreads, sizeof(IxSmem), st>>>(
-      g, t.dk_a, t.dk_b, t.rows_a, t.rows_b, passes_run, aabb16, block_off, partial, nnz, limit, isect_off, keys,
-      vals);
+      g, dkeys, rows, aabb16, block_off, partial, nnz, limit, isect_off, keys, vals);
   return cuda_status(cudaGetLastError(), "intersect write");
 }

@@ -84,11 +84,18 @@ __host__ __device__ constexpr int rows_sh_stride() {
   return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
 }
 
-// Whether any camera sees Gaussian m (a set bit in one of its C mask words).
-__device__ __forceinline__ bool any_camera_sees(const Geo& g, const uint32_t* __restrict__ mask, int64_t m) {
+// L2 prefetch of the SH rows of block m0's Gaussians that some camera sees:
+// each warp ORs its 32 Gaussians' mask words over the cameras (lane c loads
+// camera c's, all in flight together) and each lane prefetches its row.
+__device__ __forceinline__ void prefetch_seen_rows(const Geo& g, const uint32_t* __restrict__ mask,
+                                                   const float* __restrict__ sh, int64_t m0, int K3) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t u = 0;
-  for (int c = 0; c < g.C && !u; ++c) u = (mask[((int64_t)c * g.n_pad + m) / 32] >> (m & 31)) & 1u;
-  return u != 0;
+  for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + m0) / 32 + warp];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
+  const int64_t m = m0 + threadIdx.x;
+  if (((u >> lane) & 1u) && m < g.N) prefetch_l2(sh + m * K3, (uint32_t)(K3 * 4));
 }
 
 // Bit gi of the CTA's per-warp visibility words.
@@ -138,20 +145,16 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   const int64_t n0 = blk * kBlock;
   const int64_t n = n0 + threadIdx.x;
   const int cnt = (int)min64(kBlock, g.N - n0);
-  if (ahead > 0 && blk + ahead < (int64_t)gridDim.x) {
-    // the parameters of the block that starts about a wave later, into L2;
-    // SH rows only of the Gaussians some camera sees (the others are never
-    // read)
+  const bool prefetch_ahead = ahead > 0 && blk + ahead < (int64_t)gridDim.x;
+  if (prefetch_ahead && threadIdx.x == 0) {
+    // the parameters of the block that starts about a wave later, into L2
+    // (its SH rows follow once this block's own loads are in flight)
     const int64_t m0 = (blk + ahead) * kBlock;
     const int mc = (int)min64(kBlock, g.N - m0);
-    if (threadIdx.x == 0) {
-      prefetch_l2(means + 3 * m0, (uint32_t)(mc * 12));
-      prefetch_l2(quats + 4 * m0, (uint32_t)(mc * 16));
-      prefetch_l2(scales + 3 * m0, (uint32_t)(mc * 12));
-      prefetch_l2(opacities + m0, (uint32_t)(mc * 4));
-    }
-    if (threadIdx.x < mc && any_camera_sees(g, mask, m0 + threadIdx.x))
-      prefetch_l2(sh + (m0 + threadIdx.x) * K3, (uint32_t)(K3 * 4));
+    prefetch_l2(means + 3 * m0, (uint32_t)(mc * 12));
+    prefetch_l2(quats + 4 * m0, (uint32_t)(mc * 16));
+    prefetch_l2(scales + 3 * m0, (uint32_t)(mc * 12));
+    prefetch_l2(opacities + m0, (uint32_t)(mc * 4));
   }
   // A chunk's cameras, first rows and each warp's mask word per camera.  The
   // first chunk is loaded before the parameters and the SH block so that its
@@ -174,13 +177,17 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   }
   // which of the CTA's Gaussians any camera sees: only their SH rows are
   // staged (a third of the Gaussians of the 15M-Gaussian workload are seen
-  // by no camera)
-  {
+  // by no camera).  With every camera in the first chunk the words are the
+  // ones just staged; otherwise every row is staged.
+  __syncthreads();
+  if (threadIdx.x < kWarps) {
     uint32_t u = 0;
-    for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + n0) / 32 + warp];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
-    if (lane == 0) s_seen[warp] = u;
+    if (g.C <= kCamChunk) {
+      for (int c = 0; c < g.C; ++c) u |= s_word[c * kWarps + threadIdx.x];
+    } else {
+      u = 0xFFFFFFFFu;
+    }
+    s_seen[threadIdx.x] = u;
   }
   __syncthreads();
   // the CTA's contiguous SH block: a full block with all 16-byte loads in
@@ -198,6 +205,7 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
         if (v < kV && (seen(s_seen, (4 * v) / K3) || seen(s_seen, (4 * v + 3) / K3)))
           buf[r] = reinterpret_cast<const float4*>(src)[v];
       }
+      if (prefetch_ahead) prefetch_seen_rows(g, mask, sh, (blk + ahead) * kBlock, K3);
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
         const int v = threadIdx.x + r * kBlock;

@@ -77,11 +77,18 @@ __device__ __forceinline__ void sh_dir_grads(float X, float Y, float Z, const fl
   vdir[2] = gZ;
 }
 
-// Whether any camera sees Gaussian m (a set bit in one of its C mask words).
-__device__ __forceinline__ bool any_camera_sees(const Geo& g, const uint32_t* __restrict__ mask, int64_t m) {
+// L2 prefetch of the SH rows of block m0's Gaussians that some camera sees:
+// each warp ORs its 32 Gaussians' mask words over the cameras (lane c loads
+// camera c's, all in flight together) and each lane prefetches its row.
+__device__ __forceinline__ void prefetch_seen_rows(const Geo& g, const uint32_t* __restrict__ mask,
+                                                   const float* __restrict__ sh, int64_t m0, int K3) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t u = 0;
-  for (int c = 0; c < g.C && !u; ++c) u = (mask[((int64_t)c * g.n_pad + m) / 32] >> (m & 31)) & 1u;
-  return u != 0;
+  for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + m0) / 32 + warp];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
+  const int64_t m = m0 + threadIdx.x;
+  if (((u >> lane) & 1u) && m < g.N) prefetch_l2(sh + m * K3, (uint32_t)(K3 * 4));
 }
 
 // Bit gi of the CTA's per-warp visibility words.
@@ -218,8 +225,6 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   // the optimizer updates every parameter and the accumulators are decoded
   // into the SH staging area, so only the plain backward skips unseen rows
   constexpr bool kSkipUnseen = !ADAM && !GQ;
-  __shared__ __align__(16) float s_pf[kWarps][32][4];  // a round's pair sums: mean (3), opacity
-  __shared__ double s_pd[kWarps][32][6];               // and dL/dSigma
   extern __shared__ float smem[];
   float* sh_s = smem;                 // [kBlock][KP] SH coefficients of the CTA's Gaussians
   float* gsh_s = smem + kBlock * KP;  // [kBlock][KP] their gradient accumulators
@@ -248,25 +253,42 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     prefetch_l2(v_screen + r0 * kRowF, (uint32_t)((r1 - r0) * kRowF * 4));
   }
   // (blocks_per_cam, not the grid: a grad-quant grid may hold one CTA more)
-  if (ahead > 0 && blk + ahead < (GQ ? g.blocks_per_cam : (int64_t)gridDim.x)) {
-    // the SH block of the CTA that starts about a wave later, into L2; the
-    // plain backward reads only the rows of Gaussians some camera sees
+  const bool prefetch_ahead = ahead > 0 && blk + ahead < (GQ ? g.blocks_per_cam : (int64_t)gridDim.x);
+  if (!kSkipUnseen && prefetch_ahead && threadIdx.x == 0) {
+    // the SH block of the CTA that starts about a wave later, into L2
     const int64_t m0 = (blk + ahead) * kBlock;
-    const int mc = (int)min64(kBlock, g.N - m0);
-    if (kSkipUnseen) {
-      if (threadIdx.x < mc && any_camera_sees(g, mask, m0 + threadIdx.x))
-        prefetch_l2(sh + (m0 + threadIdx.x) * K3, (uint32_t)(K3 * 4));
-    } else if (threadIdx.x == 0) {
-      prefetch_l2(sh + m0 * K3, (uint32_t)(mc * K3 * 4));
-    }
+    prefetch_l2(sh + m0 * K3, (uint32_t)(min64(kBlock, g.N - m0) * K3 * 4));
   }
+  // The camera chunk of the first cameras: each warp's mask word and first
+  // row per camera (loaded before the SH block, so the plain backward knows
+  // which Gaussians some camera sees; later chunks are loaded in the loop).
+  auto load_chunk = [&](int c0) {
+    const int nc = min(kCamChunkB, g.C - c0);
+    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
+    if (threadIdx.x < nc * kWarps) {
+      const int cc = threadIdx.x / kWarps, w = threadIdx.x % kWarps;
+      const int64_t c = c0 + cc;
+      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
+      int64_t row = block_off[c * g.blocks_per_cam + blk];
+      for (int w2 = 0; w2 < w; ++w2) row += __popc(mask[wbase + w2]);
+      s_word[cc][w] = mask[wbase + w];
+      s_row0[cc][w] = row;
+    }
+  };
+  load_chunk(0);
   if (kSkipUnseen) {
-    // which of the CTA's Gaussians any camera sees (per warp, one word)
-    uint32_t u = 0;
-    for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + n0) / 32 + warp];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
-    if (lane == 0) s_seen[warp] = u;
+    // which of the CTA's Gaussians any camera sees: with every camera in the
+    // first chunk, from the words just staged; otherwise every row is read
+    __syncthreads();
+    if (threadIdx.x < kWarps) {
+      uint32_t u = 0;
+      if (g.C <= kCamChunkB) {
+        for (int c = 0; c < g.C; ++c) u |= s_word[c][threadIdx.x];
+      } else {
+        u = 0xFFFFFFFFu;
+      }
+      s_seen[threadIdx.x] = u;
+    }
     __syncthreads();
   }
   if (GQ && !gqa.first && threadIdx.x == 0) {
@@ -310,6 +332,7 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
         else
           buf[r] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      if (kSkipUnseen && prefetch_ahead) prefetch_seen_rows(g, mask, sh, (blk + ahead) * kBlock, K3);
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
         const int v = threadIdx.x + r * kBlock;
@@ -362,218 +385,143 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   for (int c0 = 0; c0 < g.C; c0 += kCamChunkB) {
     const int nc = min(kCamChunkB, g.C - c0);
     __syncthreads();
-    if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
-    if (threadIdx.x < nc * kWarps) {
-      // each warp's mask word and first row, per camera of the chunk
-      const int cc = threadIdx.x / kWarps, w = threadIdx.x % kWarps;
-      const int64_t c = c0 + cc;
-      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
-      int64_t row = block_off[c * g.blocks_per_cam + blk];
-      for (int w2 = 0; w2 < w; ++w2) row += __popc(mask[wbase + w2]);
-      s_word[cc][w] = mask[wbase + w];
-      s_row0[cc][w] = row;
-    }
+    if (c0 > 0) load_chunk(c0);  // the first chunk was loaded before the SH block
     __syncthreads();
-    // The warp's (Gaussian, camera) pairs of this chunk, numbered Gaussian by
-    // Gaussian (lane order) and camera by camera, are dealt to the lanes 32 at
-    // a time, so a warp runs ceil(pairs / 32) rounds rather than as many as
-    // its busiest Gaussian has cameras.  The lane that takes a pair reads its
-    // owner's data from the owner lane (shuffles) and shared memory; the
-    // owner adds its pairs' sums in camera order (deterministic).
+    if (!valid) continue;
+    // each lane walks the cameras of the chunk that see its Gaussian, in
+    // camera order, with the next pair's gradient row loaded one pair ahead
     uint32_t vis = 0;
-    if (valid)
-      for (int cc = 0; cc < nc; ++cc) vis |= ((s_word[cc][warp] >> lane) & 1u) << cc;
-    const int nv = __popc(vis);
-    int incl = nv;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int x = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += x;
+    for (int cc = 0; cc < nc; ++cc) vis |= ((s_word[cc][warp] >> lane) & 1u) << cc;
+    const uint32_t below = (1u << lane) - 1u;
+    const float* shn = sh_s + threadIdx.x * KP;
+    float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
+    float2 n2 = make_float2(0.f, 0.f);
+    if (vis) {
+      const int cc = __ffs(vis) - 1;
+      const float* rp = v_screen + (s_row0[cc][warp] + __popc(s_word[cc][warp] & below)) * kRowF;
+      n0 = reinterpret_cast<const float4*>(rp)[0];
+      n1 = reinterpret_cast<const float4*>(rp)[1];
+      n2 = reinterpret_cast<const float2*>(rp)[4];
     }
-    const int excl = incl - nv;
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    for (int r0 = 0; r0 < total; r0 += 32) {
-      const int i = r0 + lane;
-      const bool has = i < total;
-      // owner: the last lane whose first pair is at or before i
-      int o = 0;
-#pragma unroll
-      for (int step = 16; step >= 1; step >>= 1) {
-        const int cand = o + step;
-        const int pe = __shfl_sync(0xffffffffu, excl, cand & 31);
-        if (cand < 32 && pe <= i) o = cand;
+    while (vis) {
+      const int cc = __ffs(vis) - 1;
+      vis &= vis - 1;
+      const float4 v0 = n0, v1 = n1;
+      const float2 v2 = n2;
+      if (vis) {
+        const int cn = __ffs(vis) - 1;
+        const float* rp = v_screen + (s_row0[cn][warp] + __popc(s_word[cn][warp] & below)) * kRowF;
+        n0 = reinterpret_cast<const float4*>(rp)[0];
+        n1 = reinterpret_cast<const float4*>(rp)[1];
+        n2 = reinterpret_cast<const float2*>(rp)[4];
       }
-      const uint32_t vo = __shfl_sync(0xffffffffu, vis, o);
-      const int eo = __shfl_sync(0xffffffffu, excl, o);
-      const float omx = __shfl_sync(0xffffffffu, mx, o), omy = __shfl_sync(0xffffffffu, my, o),
-                  omz = __shfl_sync(0xffffffffu, mz, o);
-      Cov3 oS;
-      oS.s00 = __shfl_sync(0xffffffffu, S.s00, o);
-      oS.s01 = __shfl_sync(0xffffffffu, S.s01, o);
-      oS.s02 = __shfl_sync(0xffffffffu, S.s02, o);
-      oS.s11 = __shfl_sync(0xffffffffu, S.s11, o);
-      oS.s12 = __shfl_sync(0xffffffffu, S.s12, o);
-      oS.s22 = __shfl_sync(0xffffffffu, S.s22, o);
-      const int og = warp * 32 + o;  // owner within the CTA
-      const float* shn = sh_s + og * KP;
-      float pg[4] = {0.f, 0.f, 0.f, 0.f};  // the pair's mean (3) and opacity gradients
-      double pS[6] = {0., 0., 0., 0., 0., 0.};
-      int seg = 0;  // rank of the pair among its owner's pairs of this round
-      float X = 0.f, Y = 0.f, Z = 0.f;
-      float vm[3] = {0.f, 0.f, 0.f};
-      bool cl[3] = {true, true, true};
-      if (has) {
-        const int rank = i - eo;
-        seg = i - max(eo, r0);
-        const int cc = (int)__fns(vo, 0, rank + 1);
-        const float* rp = v_screen + (s_row0[cc][warp] + __popc(s_word[cc][warp] & ((1u << o) - 1u))) * kRowF;
-        const float4 v0 = reinterpret_cast<const float4*>(rp)[0];
-        const float4 v1 = reinterpret_cast<const float4*>(rp)[1];
-        const float2 v2 = reinterpret_cast<const float2*>(rp)[4];
-        const Cam& k = scam[cc];
-        const float* R = k.R;
-        // camera point and the projection's gating decision in canonical arithmetic
-        float px, py, pz;
-        cam_point(k, omx, omy, omz, px, py, pz);
-        const float izc = div_(1.0f, pz);
-        const float u = mul(px, izc), v = mul(py, izc);
-        const bool clx = (u < -k.limx) || (u > k.limx);
-        const bool cly = (v < -k.limy) || (v > k.limy);
-        const float ux = fminf(fmaxf(u, -k.limx), k.limx), uy = fminf(fmaxf(v, -k.limy), k.limy);
-        // gradient arithmetic (any rounding order)
-        const float iz = 1.0f / pz, iz2 = iz * iz;
-        const float j00 = k.fx * iz, j02 = -j00 * ux, j11 = k.fy * iz, j12 = -j11 * uy;
-        float T[6];
+      const Cam& k = scam[cc];
+      const float* R = k.R;
+      float px, py, pz;
+      cam_point(k, mx, my, mz, px, py, pz);
+      const float izc = div_(1.0f, pz);
+      const float u = mul(px, izc), v = mul(py, izc);
+      const bool clx = (u < -k.limx) || (u > k.limx);
+      const bool cly = (v < -k.limy) || (v > k.limy);
+      const float ux = fminf(fmaxf(u, -k.limx), k.limx), uy = fminf(fmaxf(v, -k.limy), k.limy);
+      const float iz = 1.0f / pz, iz2 = iz * iz;
+      const float j00 = k.fx * iz, j02 = -j00 * ux, j11 = k.fy * iz, j12 = -j11 * uy;
+      float T[6];
 #pragma unroll
-        for (int m = 0; m < 3; ++m) {
-          T[m] = j00 * R[m] + j02 * R[6 + m];
-          T[3 + m] = j11 * R[3 + m] + j12 * R[6 + m];
-        }
-        // conic -> 2D covariance -> (T, Sigma) in fp64: the terms are of size
-        // (f/z)^2 * |V2| and cancel down to small rotation/scale gradients
-        const double Sm[3][3] = {{oS.s00, oS.s01, oS.s02}, {oS.s01, oS.s11, oS.s12}, {oS.s02, oS.s12, oS.s22}};
-        double Td[6];
+      for (int m = 0; m < 3; ++m) {
+        T[m] = j00 * R[m] + j02 * R[6 + m];
+        T[3 + m] = j11 * R[3 + m] + j12 * R[6 + m];
+      }
+      const double Sm[3][3] = {{S.s00, S.s01, S.s02}, {S.s01, S.s11, S.s12}, {S.s02, S.s12, S.s22}};
+      double Td[6];
 #pragma unroll
-        for (int m = 0; m < 6; ++m) Td[m] = T[m];
-        double TS[2][3];
+      for (int m = 0; m < 6; ++m) Td[m] = T[m];
+      double TS[2][3];
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
+      for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int m = 0; m < 3; ++m)
-            TS[r][m] = Td[3 * r] * Sm[0][m] + Td[3 * r + 1] * Sm[1][m] + Td[3 * r + 2] * Sm[2][m];
-        const double a = TS[0][0] * Td[0] + TS[0][1] * Td[1] + TS[0][2] * Td[2] + 0.3;
-        const double b = TS[0][0] * Td[3] + TS[0][1] * Td[4] + TS[0][2] * Td[5];
-        const double cq = TS[1][0] * Td[3] + TS[1][1] * Td[4] + TS[1][2] * Td[5] + 0.3;
-        // conic (c, -b, a)/det -> dilated covariance (a, b, c)
-        const double id = 1.0 / (a * cq - b * b), id2 = id * id;
-        const double vca = v0.z, vcb = v0.w, vcc = v1.x;
-        const double va = (-vca * cq * cq + vcb * b * cq - vcc * b * b) * id2;
-        const double vb = (2.0 * vca * b * cq - vcb * (a * cq + b * b) + 2.0 * vcc * a * b) * id2;
-        const double vc = (-vca * b * b + vcb * a * b - vcc * a * a) * id2;
-        const double hb = 0.5 * vb;
-        // dL/dT = 2 V2 T Sigma;  dL/dSigma = T^T V2 T
-        float GT[2][3];
-        double VT[2][3];
+        for (int m = 0; m < 3; ++m)
+          TS[r][m] = Td[3 * r] * Sm[0][m] + Td[3 * r + 1] * Sm[1][m] + Td[3 * r + 2] * Sm[2][m];
+      const double a = TS[0][0] * Td[0] + TS[0][1] * Td[1] + TS[0][2] * Td[2] + 0.3;
+      const double b = TS[0][0] * Td[3] + TS[0][1] * Td[4] + TS[0][2] * Td[5];
+      const double cq = TS[1][0] * Td[3] + TS[1][1] * Td[4] + TS[1][2] * Td[5] + 0.3;
+      const double id = 1.0 / (a * cq - b * b), id2 = id * id;
+      const double vca = v0.z, vcb = v0.w, vcc = v1.x;
+      const double va = (-vca * cq * cq + vcb * b * cq - vcc * b * b) * id2;
+      const double vb = (2.0 * vca * b * cq - vcb * (a * cq + b * b) + 2.0 * vcc * a * b) * id2;
+      const double vc = (-vca * b * b + vcb * a * b - vcc * a * a) * id2;
+      const double hb = 0.5 * vb;
+      float GT[2][3];
+      double VT[2][3];
 #pragma unroll
-        for (int m = 0; m < 3; ++m) {
-          GT[0][m] = (float)(2.0 * (va * TS[0][m] + hb * TS[1][m]));
-          GT[1][m] = (float)(2.0 * (hb * TS[0][m] + vc * TS[1][m]));
-          VT[0][m] = va * Td[m] + hb * Td[3 + m];
-          VT[1][m] = hb * Td[m] + vc * Td[3 + m];
-        }
-        pS[0] = Td[0] * VT[0][0] + Td[3] * VT[1][0];
-        pS[1] = Td[0] * VT[0][1] + Td[3] * VT[1][1];
-        pS[2] = Td[0] * VT[0][2] + Td[3] * VT[1][2];
-        pS[3] = Td[1] * VT[0][1] + Td[4] * VT[1][1];
-        pS[4] = Td[1] * VT[0][2] + Td[4] * VT[1][2];
-        pS[5] = Td[2] * VT[0][2] + Td[5] * VT[1][2];
-        // T = J R -> dL/dJ = dL/dT R^T (entries 00, 02, 11, 12)
-        const float gj00 = GT[0][0] * R[0] + GT[0][1] * R[1] + GT[0][2] * R[2];
-        const float gj02 = GT[0][0] * R[6] + GT[0][1] * R[7] + GT[0][2] * R[8];
-        const float gj11 = GT[1][0] * R[3] + GT[1][1] * R[4] + GT[1][2] * R[5];
-        const float gj12 = GT[1][0] * R[6] + GT[1][1] * R[7] + GT[1][2] * R[8];
-        float gx_ = 0.f, gy = 0.f;
-        float gz = -k.fx * iz2 * gj00 + k.fx * ux * iz2 * gj02 - k.fy * iz2 * gj11 + k.fy * uy * iz2 * gj12;
-        const float gux = -k.fx * iz * gj02, guy = -k.fy * iz * gj12;
-        if (!clx) { gx_ += gux * iz; gz -= gux * px * iz2; }
-        if (!cly) { gy += guy * iz; gz -= guy * py * iz2; }
-        const float vmx = v0.x, vmy = v0.y;
-        gx_ += vmx * k.fx * iz; gz -= vmx * k.fx * px * iz2;
-        gy += vmy * k.fy * iz; gz -= vmy * k.fy * py * iz2;
-        gz += v2.y;  // depth
-        pg[0] = R[0] * gx_ + R[3] * gy + R[6] * gz;
-        pg[1] = R[1] * gx_ + R[4] * gy + R[7] * gz;
-        pg[2] = R[2] * gx_ + R[5] * gy + R[8] * gz;
-        pg[3] = v1.y;
-        // colour: the clamp decisions of the forward.  The sum is taken in
-        // any order first; only where 0.5 + sum lies within the owner's
-        // margin (ten times the rounding bound of either order) of zero is it
-        // redone in the forward's canonical order, so the decision is always
-        // the forward's
-        float il = 0.f;
-        if (DEG > 0) view_dir(k, omx, omy, omz, X, Y, Z, il);
-        {
-          float bb[16];
-          sh_basis(DEG, X, Y, Z, bb);
+      for (int m = 0; m < 3; ++m) {
+        GT[0][m] = (float)(2.0 * (va * TS[0][m] + hb * TS[1][m]));
+        GT[1][m] = (float)(2.0 * (hb * TS[0][m] + vc * TS[1][m]));
+        VT[0][m] = va * Td[m] + hb * Td[3 + m];
+        VT[1][m] = hb * Td[m] + vc * Td[3 + m];
+      }
+      gS[0] += Td[0] * VT[0][0] + Td[3] * VT[1][0];
+      gS[1] += Td[0] * VT[0][1] + Td[3] * VT[1][1];
+      gS[2] += Td[0] * VT[0][2] + Td[3] * VT[1][2];
+      gS[3] += Td[1] * VT[0][1] + Td[4] * VT[1][1];
+      gS[4] += Td[1] * VT[0][2] + Td[4] * VT[1][2];
+      gS[5] += Td[2] * VT[0][2] + Td[5] * VT[1][2];
+      const float gj00 = GT[0][0] * R[0] + GT[0][1] * R[1] + GT[0][2] * R[2];
+      const float gj02 = GT[0][0] * R[6] + GT[0][1] * R[7] + GT[0][2] * R[8];
+      const float gj11 = GT[1][0] * R[3] + GT[1][1] * R[4] + GT[1][2] * R[5];
+      const float gj12 = GT[1][0] * R[6] + GT[1][1] * R[7] + GT[1][2] * R[8];
+      float gx_ = 0.f, gy = 0.f;
+      float gz = -k.fx * iz2 * gj00 + k.fx * ux * iz2 * gj02 - k.fy * iz2 * gj11 + k.fy * uy * iz2 * gj12;
+      const float gux = -k.fx * iz * gj02, guy = -k.fy * iz * gj12;
+      if (!clx) { gx_ += gux * iz; gz -= gux * px * iz2; }
+      if (!cly) { gy += guy * iz; gz -= guy * py * iz2; }
+      const float vmx = v0.x, vmy = v0.y;
+      gx_ += vmx * k.fx * iz; gz -= vmx * k.fx * px * iz2;
+      gy += vmy * k.fy * iz; gz -= vmy * k.fy * py * iz2;
+      gz += v2.y;
+      gmu[0] += R[0] * gx_ + R[3] * gy + R[6] * gz;
+      gmu[1] += R[1] * gx_ + R[4] * gy + R[7] * gz;
+      gmu[2] += R[2] * gx_ + R[5] * gy + R[8] * gz;
+      go += v1.y;
+      float X = 0.f, Y = 0.f, Z = 0.f, il = 0.f;
+      if (DEG > 0) view_dir(k, mx, my, mz, X, Y, Z, il);
+      bool cl[3];
+      {
+        float bb[16];
+        sh_basis(DEG, X, Y, Z, bb);
 #pragma unroll
-          for (int ch = 0; ch < 3; ++ch) {
-            float f = 0.5f;
+        for (int ch = 0; ch < 3; ++ch) {
+          float f = 0.5f;
 #pragma unroll
-            for (int kk = 0; kk < K; ++kk) f = fmaf(shn[3 * kk + ch], bb[kk], f);
-            bool c = !(f >= 0.0f);
-            if (fabsf(f) <= s_margin[og][ch]) {
-              float acc = mul(shn[ch], bb[0]);
+          for (int kk = 0; kk < K; ++kk) f = fmaf(shn[3 * kk + ch], bb[kk], f);
+          bool c = !(f >= 0.0f);
+          if (fabsf(f) <= s_margin[threadIdx.x][ch]) {
+            float acc = mul(shn[ch], bb[0]);
 #pragma unroll
-              for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], bb[kk]));
-              c = !(add(acc, 0.5f) >= 0.0f);
-            }
-            cl[ch] = c;
+            for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], bb[kk]));
+            c = !(add(acc, 0.5f) >= 0.0f);
           }
+          cl[ch] = c;
         }
-        const float vr[3] = {v1.z, v1.w, v2.x};
-#pragma unroll
-        for (int ch = 0; ch < 3; ++ch) vm[ch] = cl[ch] ? 0.0f : vr[ch];
-        if (DEG > 0) {
-          float vdir[3];
-          sh_dir_grads<DEG>(X, Y, Z, shn, vm, vdir);
-          const float dd = X * vdir[0] + Y * vdir[1] + Z * vdir[2];
-          pg[0] += (vdir[0] - X * dd) * il;
-          pg[1] += (vdir[1] - Y * dd) * il;
-          pg[2] += (vdir[2] - Z * dd) * il;
-        }
-        // the owner's first pair of the round adds its SH coefficient
-        // gradients now; the others wait their turn below
-        if (seg == 0) sh_coef_grads<DEG>(X, Y, Z, vm, cl, gsh_s + og * KP);
       }
-      // an owner's further pairs of this round, one rank at a time (each
-      // rank holds at most one pair per owner, so no two lanes of a rank
-      // touch the same row), in camera order
-      const int maxseg = __reduce_max_sync(0xffffffffu, has ? (unsigned)seg : 0u);
-      for (int j = 1; j <= maxseg; ++j) {
-        __syncwarp();
-        if (has && seg == j) sh_coef_grads<DEG>(X, Y, Z, vm, cl, gsh_s + og * KP);
-      }
-      // the pairs' sums to their owners, added in camera order
-      reinterpret_cast<float4*>(&s_pf[warp][lane][0])[0] = make_float4(pg[0], pg[1], pg[2], pg[3]);
+      const float vr[3] = {v1.z, v1.w, v2.x};
+      float vm[3];
 #pragma unroll
-      for (int m = 0; m < 6; ++m) s_pd[warp][lane][m] = pS[m];
-      __syncwarp();
-      const int l0 = max(excl, r0) - r0, l1 = min(excl + nv, r0 + 32) - r0;
-      for (int l = l0; l < l1; ++l) {
-        const float4 f = reinterpret_cast<const float4*>(&s_pf[warp][l][0])[0];
-        gmu[0] += f.x;
-        gmu[1] += f.y;
-        gmu[2] += f.z;
-        go += f.w;
-#pragma unroll
-        for (int m = 0; m < 6; ++m) gS[m] += s_pd[warp][l][m];
+      for (int ch = 0; ch < 3; ++ch) vm[ch] = cl[ch] ? 0.0f : vr[ch];
+      sh_coef_grads<DEG>(X, Y, Z, vm, cl, gsh_s + threadIdx.x * KP);
+      if (DEG > 0) {
+        float vdir[3];
+        sh_dir_grads<DEG>(X, Y, Z, shn, vm, vdir);
+        const float dd = X * vdir[0] + Y * vdir[1] + Z * vdir[2];
+        gmu[0] += (vdir[0] - X * dd) * il;
+        gmu[1] += (vdir[1] - Y * dd) * il;
+        gmu[2] += (vdir[2] - Z * dd) * il;
       }
-      __syncwarp();
     }
   }
   if (valid) {
     // the rotation and scales again (read back rather than kept live across
-    // the camera rounds)
+    // the camera walk)
     const float4 q4 = reinterpret_cast<const float4*>(quats)[n];
     const float s0 = scales[3 * n], s1 = scales[3 * n + 1], s2 = scales[3 * n + 2];
     const QuatRot qr = quat_rot(q4.x, q4.y, q4.z, q4.w);

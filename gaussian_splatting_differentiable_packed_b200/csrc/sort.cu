@@ -4,15 +4,12 @@
 // written here).  8-bit digits: the four bytes of the depth and the bytes the
 // tile ids need.  A digit that is the same in every key (for example the top
 // byte of depths whose exponents share their high bits) cannot change the
-// order, so its pass is skipped; the histograms show which ones, and the
-// device keeps the plan, so the host launches the full plan's kernels and
-// the skipped ones return at once.
+// order, so its pass is skipped: the host reads the histograms (one small
+// copy) and launches only the passes whose digits vary.
 //
 //   k_hist_all   one read of the keys: the global digit histogram of every pass
 //                (a permutation does not change them)
-//   k_plan       which passes run (a digit whose histogram holds every key in
-//                one bin is skipped), and the exclusive scan of each running
-//                pass's 256 counts
+//   k_bases      the exclusive scan of each pass's 256 counts
 //   k_onesweep   per pass, one kernel: each CTA takes the next 4096-key tile by
 //                ticket, ranks its keys stably among equal digits (warp match +
 //                per-warp counters), publishes its digit counts and looks back
@@ -44,13 +41,6 @@ constexpr uint64_t kFlagAgg = 1ull << 54;
 constexpr uint64_t kFlagPre = 2ull << 54;
 constexpr uint64_t kValMask = (1ull << 54) - 1;
 constexpr int kSpinLimit = 1 << 20;
-
-// The passes that run, written by k_plan: shift[k] is the key bit of the k-th
-// running pass's digit, count the number of running passes.
-struct DevPlan {
-  int count;
-  int shift[kMaxPasses];
-};
 
 // Digit histograms of every pass in one read of the keys.  PASSES is a
 // template argument so every digit is a constant byte of the key's low or
@@ -107,40 +97,25 @@ ss_status launch_hist(unsigned grid, cudaStream_t st, const uint64_t* keys, int6
   return cuda_status(cudaGetLastError(), "radix histogram");
 }
 
-// Which passes run and their digit bases (one CTA of 256 threads): pass p is
-// skipped when one bin of its histogram holds all n keys; the running passes'
-// histograms are scanned (exclusive) and moved to the front, in order, so
-// running pass k reads hist[k] and the digit at key bit plan->shift[k].
-__global__ __launch_bounds__(kRadix) void k_plan(uint32_t* __restrict__ hist, int passes, int lo_bytes, int64_t n,
-                                                 DevPlan* __restrict__ plan) {
+// hist[p][d] -> exclusive scan over d, in place (one CTA of 256 threads).
+__global__ __launch_bounds__(kRadix) void k_bases(uint32_t* __restrict__ hist, int passes) {
   __shared__ uint32_t wt[kRadix / 32];
-  __shared__ int s_full;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int k = 0;
   for (int p = 0; p < passes; ++p) {
-    if (threadIdx.x == 0) s_full = 0;
-    __syncthreads();
     const uint32_t v = hist[p * kRadix + threadIdx.x];
-    if ((int64_t)v == n) s_full = 1;
-    __syncthreads();
-    if (s_full == 0) {
-      uint32_t inc = v;
+    uint32_t inc = v;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += x;
-      }
-      if (lane == 31) wt[warp] = inc;
-      __syncthreads();
-      uint32_t before = 0;
-      for (int w = 0; w < warp; ++w) before += wt[w];
-      hist[k * kRadix + threadIdx.x] = before + inc - v;  // k <= p, and row p was read above
-      if (threadIdx.x == 0) plan->shift[k] = p < lo_bytes ? 8 * p : 32 + 8 * (p - lo_bytes);
-      ++k;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += x;
     }
+    if (lane == 31) wt[warp] = inc;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += wt[w];
+    hist[p * kRadix + threadIdx.x] = before + inc - v;
     __syncthreads();
   }
-  if (threadIdx.x == 0) plan->count = k;
 }
 
 struct OnesweepSmem {
@@ -160,14 +135,12 @@ __device__ __forceinline__ uint64_t ld_status(const uint64_t* p) {
 __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __restrict__ kin,
                                                            const uint32_t* __restrict__ vin,
                                                            uint64_t* __restrict__ kout, uint32_t* __restrict__ vout,
-                                                           int64_t n, int pass, const DevPlan* __restrict__ plan,
-                                                           uint64_t epoch, const uint32_t* __restrict__ bases,
+                                                           int64_t n, int shift, uint64_t epoch,
+                                                           const uint32_t* __restrict__ bases,
                                                            uint64_t* __restrict__ status,
                                                            uint32_t* __restrict__ ticket, uint32_t* __restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   OnesweepSmem& S = *reinterpret_cast<OnesweepSmem*>(smem_raw);
-  if (pass >= plan->count) return;  // a skipped digit: nothing moves
-  const int shift = plan->shift[pass];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) S.tile = atomicAdd(ticket, 1u);
   for (int i = threadIdx.x; i < kSortWarps * kRadix; i += kSortThreads) (&S.wcnt[0][0])[i] = 0;
@@ -290,10 +263,8 @@ __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __res
 }
 
 // tile_off[t] = first sorted index whose tile id is >= t; tile_off[ntiles] = n.
-// The sorted keys are in keys_b after an odd number of running passes.
-__global__ void k_tile_ranges(const uint64_t* __restrict__ keys_a, const uint64_t* __restrict__ keys_b, int64_t n,
-                              int64_t ntiles, const DevPlan* __restrict__ plan, int64_t* __restrict__ tile_off) {
-  const uint64_t* keys = (plan->count & 1) ? keys_b : keys_a;
+__global__ void k_tile_ranges(const uint64_t* __restrict__ keys, int64_t n, int64_t ntiles,
+                              int64_t* __restrict__ tile_off) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i > n) return;
   const int64_t prev = i == 0 ? -1 : (int64_t)(keys[i - 1] >> 32);
@@ -309,14 +280,8 @@ int tile_bits(int64_t ntiles) {
 
 
 // Scratch layout: hist [kMaxPasses][256] u32 | tickets [kMaxPasses] u32 |
-// error flag u32 | plan | look-back status [tiles][256] u64.
-constexpr size_t sort_plan_offset() { return align_up(kMaxPasses * kRadix * 4 + kMaxPasses * 4 + 4, 16); }
-constexpr size_t sort_status_offset() { return align_up(sort_plan_offset() + sizeof(DevPlan), 256); }
-
-inline DevPlan* sort_plan(void* temp) { return reinterpret_cast<DevPlan*>(reinterpret_cast<char*>(temp) + sort_plan_offset()); }
-inline const DevPlan* sort_plan(const void* temp) {
-  return reinterpret_cast<const DevPlan*>(reinterpret_cast<const char*>(temp) + sort_plan_offset());
-}
+// error flag u32 | look-back status [tiles][256] u64.
+constexpr size_t sort_status_offset() { return align_up(kMaxPasses * kRadix * 4 + kMaxPasses * 4 + 4, 256); }
 
 constexpr size_t sort_scratch_bytes(int64_t n) {
   return sort_status_offset() + (size_t)ceil_div(n > 1 ? n : 1, kSortTile) * kRadix * 8;
@@ -333,11 +298,13 @@ namespace ss {
 // Stable LSD sort of n (key, value) pairs over byte digits: the low word's
 // lo_bytes bytes (4, or 0 when the keys already arrive in the order of their
 // low words, ties in the order to keep), then the high word's hi_bytes bytes.
-// Digits equal in every key are skipped (device plan); the result is in
-// (kb, vb) after an odd number of running passes: plan->count & 1, on the
-// device.  temp: sort_temp_bytes(n), cleared here.  No host synchronisation.
+// The histograms are read back (one small copy, stream sync) and a digit
+// equal in every key is skipped.  *in_b: the result is in (kb, vb).  temp:
+// sort_temp_bytes(n), cleared here.  The look-back flag is left in temp
+// (radix_sort_flag).
 ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
-                           int hi_bytes, void* temp, cudaStream_t st) {
+                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b) {
+  *in_b = false;
   ss_status s = cuda_status(cudaFuncSetAttribute(k_onesweep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)sizeof(OnesweepSmem)),
                             "set smem attribute");
@@ -347,11 +314,9 @@ ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* v
   uint32_t* hist = reinterpret_cast<uint32_t*>(tb);
   uint32_t* tickets = hist + kMaxPasses * kRadix;
   uint32_t* err = tickets + kMaxPasses;
-  DevPlan* dplan = sort_plan(temp);
   uint64_t* status = reinterpret_cast<uint64_t*>(tb + sort_status_offset());
   s = cuda_status(cudaMemsetAsync(temp, 0, sort_status_offset() + (size_t)tiles * kRadix * 8, st), "memset");
   if (s) return s;
-  (void)err;
   const int passes = lo_bytes + hi_bytes;
   if (passes < 1 || passes > kMaxPasses) return invalid("sort digit count");
   const unsigned hgrid = (unsigned)min64(tiles, 148 * 8);
@@ -366,43 +331,47 @@ ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* v
     default: s = launch_hist<8>(hgrid, st, ka, n, lo_bytes, hist); break;
   }
   if (s) return s;
-  k_plan<<<1, kRadix, 0, st>>>(hist, passes, lo_bytes, n, dplan);
-  s = cuda_status(cudaGetLastError(), "radix plan");
+  // which digits vary: a pass whose histogram holds all n keys in one bin
+  // keeps the order as it is
+  uint32_t h[kMaxPasses * kRadix];
+  s = cuda_status(cudaMemcpyAsync(h, hist, (size_t)passes * kRadix * 4, cudaMemcpyDeviceToHost, st), "copy histograms");
+  if (s) return s;
+  s = cuda_status(cudaStreamSynchronize(st), "radix histogram");
+  if (s) return s;
+  k_bases<<<1, kRadix, 0, st>>>(hist, passes);
+  s = cuda_status(cudaGetLastError(), "radix bases");
   if (s) return s;
   uint64_t* kin = ka;
   uint32_t* vin = va;
   uint64_t* kout = kb;
   uint32_t* vout = vb;
+  int run = 0;
   for (int p = 0; p < passes; ++p) {
-    const uint64_t epoch = (uint64_t)(p + 1) << 56;
+    bool one_bin = false;
+    for (int d = 0; d < kRadix; ++d) one_bin = one_bin || (int64_t)h[p * kRadix + d] == n;
+    if (one_bin) continue;
+    const int shift = p < lo_bytes ? 8 * p : 32 + 8 * (p - lo_bytes);
+    const uint64_t epoch = (uint64_t)(run + 1) << 56;
     k_onesweep<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
-        kin, vin, kout, vout, n, p, dplan, epoch, hist + p * kRadix, status, tickets + p, err);
+        kin, vin, kout, vout, n, shift, epoch, hist + p * kRadix, status, tickets + run, err);
     s = cuda_status(cudaGetLastError(), "radix pass");
     if (s) return s;
     std::swap(kin, kout);
     std::swap(vin, vout);
+    ++run;
   }
+  *in_b = run & 1;
   return SS_OK;
 }
 
-// The device-side count of a sort's running passes (its result is in the
-// second buffer pair when odd).
-const int* sort_passes_run(const void* temp) { return &sort_plan(temp)->count; }
-
-// Reads back a finished sort's look-back flag and pass count (stream sync).
-ss_status radix_sort_result(const void* temp, cudaStream_t st, int* passes_run, bool* flagged) {
-  const char* tb = reinterpret_cast<const char*>(temp);
-  const uint32_t* err = reinterpret_cast<const uint32_t*>(tb) + kMaxPasses * kRadix + kMaxPasses;
+// Whether a sort's look-back wait ran out (stream sync).
+ss_status radix_sort_flag(const void* temp, cudaStream_t st, bool* flagged) {
+  const uint32_t* err = reinterpret_cast<const uint32_t*>(temp) + kMaxPasses * kRadix + kMaxPasses;
   uint32_t herr = 0;
-  int count = 0;
   ss_status s = cuda_status(cudaMemcpyAsync(&herr, err, 4, cudaMemcpyDeviceToHost, st), "copy sort flag");
-  if (s) return s;
-  s = cuda_status(cudaMemcpyAsync(&count, &sort_plan(temp)->count, sizeof(int), cudaMemcpyDeviceToHost, st),
-                  "copy sort plan");
   if (s) return s;
   s = cuda_status(cudaStreamSynchronize(st), "sort");
   if (s) return s;
-  *passes_run = count;
   *flagged = herr != 0;
   return SS_OK;
 }
@@ -429,17 +398,17 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   // the bytes of the tile ids; the plan drops the bytes that do not vary
   const int lo_bytes = presorted_depth ? 0 : 4;
   const int hi_bytes = max((tile_bits(g.n_tiles) + 7) / 8, lo_bytes ? 0 : 1);
-  ss_status s = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, n, lo_bytes, hi_bytes, temp, st);
+  bool in_b = false;
+  ss_status s = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, n, lo_bytes, hi_bytes, temp, st, &in_b);
   if (s) return s;
   const unsigned grid = (unsigned)ceil_div(n + 1, 256);
-  k_tile_ranges<<<grid, 256, 0, st>>>(keys_a, keys_b, n, g.n_tiles, sort_plan(temp), tile_off);
+  k_tile_ranges<<<grid, 256, 0, st>>>(in_b ? keys_b : keys_a, n, g.n_tiles, tile_off);
   s = cuda_status(cudaGetLastError(), "tile ranges");
   if (s) return s;
-  int count = 0;
   bool flagged = false;
-  s = radix_sort_result(temp, st, &count, &flagged);
+  s = radix_sort_flag(temp, st, &flagged);
   if (s) return s;
-  *result_in_b_out = count & 1;
+  *result_in_b_out = in_b ? 1 : 0;
   if (flagged) {
     set_error("ss_sort_isects: look-back wait exceeded its limit");
     return SS_ERR_DEVICE_CHECK;

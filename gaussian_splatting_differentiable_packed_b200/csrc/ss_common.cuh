@@ -104,11 +104,7 @@ struct ScanSrc {
   int kind;
   const uint32_t* u32;     // SCAN_U32: counts
   const uint32_t* aabb16;  // SCAN_TILES: per-row AABB16, count = tiles covered
-  // SCAN_TILES_ORDERED: item i is row order[i], order = rows_b when the
-  // sort that wrote it ran an odd number of passes (*passes_run), else rows_a
-  const uint32_t* rows_a;
-  const uint32_t* rows_b;
-  const int* passes_run;
+  const uint32_t* rows;  // SCAN_TILES_ORDERED: item i is row rows[i]
   int W, H, tiles_x, tiles_y;
 };
 constexpr int kScanItems = 16;

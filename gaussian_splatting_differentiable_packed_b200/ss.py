@@ -498,30 +498,26 @@ def seen_gaussians(d: ss_dims, mask) -> int:
     return int(pop.sum().item())
 
 
-def sort_launches(d: ss_dims, n_isects: int, presorted_depth: bool = True) -> int:
-    """Kernels of one ss_sort_isects call: histogram, plan, one onesweep
-    kernel per byte of the full plan (a skipped byte's kernel returns at
-    once), tile ranges."""
-    if n_isects == 0:
-        return 0
-    tb = max(0, (size(d, SIZE_N_TILES) - 1).bit_length())
-    return 2 + (0 if presorted_depth else 4) + max((tb + 7) // 8, 1 if presorted_depth else 0) + 1
+def sort_launches(n_isects: int, passes: int) -> int:
+    """Kernels of one ss_sort_isects call: histogram, digit bases, one
+    onesweep kernel per digit pass that runs, tile ranges."""
+    return 0 if n_isects == 0 else 3 + passes
 
 
-def launches_per_step(d: ss_dims, nnz: int, n_isects: int) -> int:
+def launches_per_step(d: ss_dims, nnz: int, n_isects: int, sort_passes: int, depth_passes: int) -> int:
     """Kernels libss launches in one forward+backward step (memsets excluded):
-    projection 5 (pass 1, three scan kernels, pass 2), intersection 10 (row
-    depth keys, the depth sort's histogram, plan and 4 byte passes, two count
-    kernels, the fused offsets-and-write kernel), the sort
+    projection 5 (pass 1, three scan kernels, pass 2), intersection 6 plus
+    one per depth-sort pass (row depth keys, the depth sort's histogram and
+    bases, two count kernels, the fused offsets-and-write kernel), the sort
     (sort_launches), tile order 3 (histogram, scan, scatter), rasterizer
-    1 + 1, projection backward 1.  With no Gaussians only the tile order and the two
-    rasterizers launch (they still write the empty images)."""
+    1 + 1, projection backward 1.  With no Gaussians only the tile order and
+    the two rasterizers launch (they still write the empty images)."""
     if d.N == 0:
         return 3 + 2
     n = 5
     if nnz > 0:
-        n += 10
-    n += sort_launches(d, n_isects)
+        n += 6 + depth_passes
+    n += sort_launches(n_isects, sort_passes)
     return n + 3 + 3
 
 

@@ -45,15 +45,14 @@ def test_traffic_record_guards(tmp_path, monkeypatch):
 
 
 def test_launches_per_step():
-    """projection 5, intersection 10 (row depth keys, the depth sort's
-    histogram, plan and 4 byte passes, two count kernels, the fused write),
-    the sort's histogram, plan, one kernel per tile-id byte and tile ranges,
+    """projection 5, intersection 6 plus one per depth-sort pass, the sort's
+    histogram, bases, one kernel per digit pass that runs and tile ranges,
     the tile order 3, rasterizers 2, projection backward 1."""
-    d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)  # 33,500 tiles: 16 tile-id bits, 2 bytes
-    assert ss.launches_per_step(d, 15_000_000, 33_000_000) == 5 + 10 + (2 + 2 + 1) + 3 + 2 + 1
-    assert ss.launches_per_step(d, 15_000_000, 0) == 5 + 10 + 0 + 3 + 2 + 1
-    assert ss.launches_per_step(d, 0, 0) == 5 + 0 + 0 + 3 + 2 + 1
-    assert ss.launches_per_step(ss.make_dims(1, 64, 64, 0, 0), 0, 0) == 3 + 2
+    d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)
+    assert ss.launches_per_step(d, 15_000_000, 33_000_000, 2, 3) == 5 + (6 + 3) + (3 + 2) + 3 + 2 + 1
+    assert ss.launches_per_step(d, 15_000_000, 0, 0, 3) == 5 + (6 + 3) + 0 + 3 + 2 + 1
+    assert ss.launches_per_step(d, 0, 0, 0, 0) == 5 + 0 + 0 + 3 + 2 + 1
+    assert ss.launches_per_step(ss.make_dims(1, 64, 64, 0, 0), 0, 0, 0, 0) == 3 + 2
 
 
 def test_sort_passes_skip_constant_bytes():

@@ -7,24 +7,26 @@
 // then depth, then row; a row's keys all carry its depth, so if the rows are
 // visited in (depth, row) order, every tile's keys come out in the right
 // order and the key sort needs only the tile-id bytes: a stable sort of the
-// nnz rows' 32-bit depths (4 byte passes over 12 bytes a row) replaces the 4
-// depth passes over the 12-byte keys (2.2 keys a row on the 15M-Gaussian
-// workload, 59 on the 7680^2 one).
+// nnz rows' 32-bit depths replaces the depth passes over the keys (2.2 keys a
+// row on the 15M-Gaussian workload, 59 on the 7680^2 one).
 //
-//   k_row_keys      (depth bits, row) of every row
-//   radix sort      stable, by depth (sort.cu)
-//   count           per-row tiles from the AABB16 by integer arithmetic, in
-//                   depth order: CTA sums per 4096 rows and a single-CTA scan
-//                   give the exact int64 total (no atomics: deterministic)
-//   k_isect_fused   (after the host check) one CTA per 4096 rows of the depth
-//                   order: decodes its rows once into shared memory (first
-//                   tile id, tile columns, depth bits), scans their tile
-//                   counts into offsets (written to isect_off with the block's
-//                   base from the count), then expands the block's slots: slot
-//                   s belongs to the last row whose offset is <= s (binary
-//                   search in shared memory), and consecutive threads write
-//                   consecutive slots, so every store is coalesced whatever
-//                   the per-row counts.
+//   k_row_keys      (depth bits << 32 | row) of every row, and the exact
+//                   int64 total of tiles covered (integer atomics: the sum
+//                   is the same in any order)
+//   radix sort      keys only, by the depth word (sort.cu; the row index in
+//                   the low word rides along, ties stay in row order)
+//   (host)          checks the total against the capacity and 2^31
+//   k_isect_fused   one CTA per 4096 positions of the depth order, blocks
+//                   taken by ticket: decodes its rows once into shared memory
+//                   (first tile id, tile columns, depth bits, row id, from
+//                   the row's AABB16), scans their tile counts, publishes the
+//                   block's total and looks back over earlier blocks for its
+//                   base (decoupled look-back, bounded spin), writes the
+//                   rows' offsets to isect_off, then expands the block's
+//                   slots: slot s belongs to the last row whose offset is
+//                   <= s (binary search in shared memory), and consecutive
+//                   threads write consecutive slots, so every store is
+//                   coalesced whatever the per-row counts.
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 
@@ -36,9 +38,16 @@ ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* v
 ss_status radix_sort_flag(const void* temp, cudaStream_t st, bool* flagged);
 
 constexpr int kIxThreads = 512;
-constexpr int kIxRows = (int)kScanTile;  // rows per CTA: the count pass's tiling
+constexpr int kIxRows = 4096;  // positions of the depth order per CTA
 constexpr int kIxPer = kIxRows / kIxThreads;
 static_assert(kIxRows % kIxThreads == 0, "rows per thread");
+constexpr int kRowKeyThreads = 256;
+
+// Block status of the look-back: flag in the top two bits, count below.
+constexpr uint64_t kIxAgg = 1ull << 62;
+constexpr uint64_t kIxPre = 2ull << 62;
+constexpr uint64_t kIxVal = (1ull << 62) - 1;
+constexpr int kIxSpinLimit = 1 << 20;
 
 struct IxSmem {
   uint32_t off[kIxRows + 1];  // slot offset of each row within the block
@@ -47,14 +56,76 @@ struct IxSmem {
   uint32_t row[kIxRows];      // row index
   uint16_t w[kIxRows];        // tile columns of the row's range
   uint32_t wsum[kIxThreads / 32];
+  int64_t base;
+  uint32_t blk;
 };
 
-__global__ void k_row_keys(const float* __restrict__ row_depth, int64_t nnz, uint64_t* __restrict__ keys,
-                           uint32_t* __restrict__ rows) {
-  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= nnz) return;
-  keys[r] = (uint64_t)__float_as_uint(row_depth[r]);
-  rows[r] = (uint32_t)r;
+// Scratch: total (int64) | ticket (u32) | error flag (u32) | block status
+// (u64 per block), then the keys' two buffers and the sort's scratch.
+struct IxTemp {
+  int64_t* total;
+  uint32_t* ticket;
+  uint32_t* err;
+  uint64_t* status;
+  size_t head_bytes;  // total .. status, cleared per call
+  uint64_t *dk_a, *dk_b;
+  void* sort;
+};
+
+IxTemp isect_temp(void* temp, int64_t nnz) {
+  char* p = reinterpret_cast<char*>(temp);
+  IxTemp t;
+  t.total = reinterpret_cast<int64_t*>(p);
+  t.ticket = reinterpret_cast<uint32_t*>(p + 8);
+  t.err = reinterpret_cast<uint32_t*>(p + 12);
+  t.status = reinterpret_cast<uint64_t*>(p + 16);
+  t.head_bytes = align_up(16 + (size_t)ceil_div(nnz, kIxRows) * 8, 256);
+  p += t.head_bytes;
+  t.dk_a = reinterpret_cast<uint64_t*>(p);
+  p += align_up((size_t)nnz * 8, 256);
+  t.dk_b = reinterpret_cast<uint64_t*>(p);
+  p += align_up((size_t)nnz * 8, 256);
+  t.sort = p;
+  return t;
+}
+
+size_t isect_temp_bytes(int64_t nnz) {
+  return align_up(16 + (size_t)ceil_div(nnz, kIxRows) * 8, 256) + 2 * align_up((size_t)nnz * 8, 256) +
+         sort_temp_bytes(nnz);
+}
+
+__device__ __forceinline__ uint32_t row_tiles(const Geo& g, uint2 q, int& tx0, int& ty0, int& w) {
+  int tx1, ty1;
+  tile_span(q.x & 0xFFFFu, q.y & 0xFFFFu, g.W, g.tiles_x, tx0, tx1);
+  tile_span(q.x >> 16, q.y >> 16, g.H, g.tiles_y, ty0, ty1);
+  w = tx1 - tx0;
+  return (uint32_t)w * (uint32_t)(ty1 - ty0);
+}
+
+__global__ __launch_bounds__(kRowKeyThreads) void k_row_keys(Geo g, const float* __restrict__ row_depth,
+                                                             const uint32_t* __restrict__ aabb16, int64_t nnz,
+                                                             uint64_t* __restrict__ keys,
+                                                             int64_t* __restrict__ total) {
+  __shared__ uint32_t ws[kRowKeyThreads / 32];
+  const int64_t r = (int64_t)blockIdx.x * kRowKeyThreads + threadIdx.x;
+  uint32_t cnt = 0;
+  if (r < nnz) {
+    keys[r] = ((uint64_t)__float_as_uint(row_depth[r]) << 32) | (uint64_t)r;
+    int tx0, ty0, w;
+    cnt = row_tiles(g, reinterpret_cast<const uint2*>(aabb16)[r], tx0, ty0, w);
+  }
+  // a row covers at most 4096 x 4096 tiles (16-bit image extents), so a
+  // warp's sum fits 32 bits; the warps' sums are added in 64 bits
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long s = 0;
+#pragma unroll
+    for (int w = 0; w < kRowKeyThreads / 32; ++w) s += ws[w];
+    if (s) atomicAdd(reinterpret_cast<unsigned long long*>(total), s);
+  }
 }
 
 __device__ __forceinline__ int camera_of_row(const int64_t* __restrict__ block_off, int64_t blocks_per_cam, int C,
@@ -67,18 +138,27 @@ __device__ __forceinline__ int camera_of_row(const int64_t* __restrict__ block_o
   return lo;
 }
 
+__device__ __forceinline__ uint64_t ld_volatile(const uint64_t* p) {
+  return *reinterpret_cast<const volatile unsigned long long*>(p);
+}
+
 __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_t* __restrict__ dkeys,
-                                                            const uint32_t* __restrict__ rows,
                                                             const uint32_t* __restrict__ aabb16,
-                                                            const int64_t* __restrict__ block_off,
-                                                            const int64_t* __restrict__ partial, int64_t nnz,
-                                                            int64_t limit, int64_t* __restrict__ isect_off,
+                                                            const int64_t* __restrict__ block_off, int64_t nnz,
+                                                            int64_t limit, uint64_t* __restrict__ status,
+                                                            uint32_t* __restrict__ ticket, uint32_t* __restrict__ err,
+                                                            int64_t* __restrict__ isect_off,
                                                             uint64_t* __restrict__ keys,
                                                             uint32_t* __restrict__ vals) {
   extern __shared__ __align__(16) unsigned char ix_raw[];
   IxSmem& S = *reinterpret_cast<IxSmem*>(ix_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t p0 = (int64_t)blockIdx.x * kIxRows;
+  // blocks by ticket: every block this one looks back on belongs to a CTA
+  // that is already running
+  if (tid == 0) S.blk = atomicAdd(ticket, 1u);
+  __syncthreads();
+  const int64_t blk = S.blk;
+  const int64_t p0 = blk * kIxRows;
   const int nr = (int)min64(kIxRows, nnz - p0);
   // decode the rows of positions p0 .. p0 + nr of the depth order, coalesced
   // in position (row i = k * kIxThreads + tid); counts go to S.off for the scan
@@ -87,17 +167,14 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
     const int i = k * kIxThreads + tid;
     uint32_t cnt = 0;
     if (i < nr) {
-      const uint32_t r = rows[p0 + i];
-      const uint2 q = reinterpret_cast<const uint2*>(aabb16)[r];
-      int tx0, tx1, ty0, ty1;
-      tile_span(q.x & 0xFFFFu, q.y & 0xFFFFu, g.W, g.tiles_x, tx0, tx1);
-      tile_span(q.x >> 16, q.y >> 16, g.H, g.tiles_y, ty0, ty1);
+      const uint64_t key = dkeys[p0 + i];
+      const uint32_t r = (uint32_t)key;
+      int tx0, ty0, w;
+      cnt = row_tiles(g, reinterpret_cast<const uint2*>(aabb16)[r], tx0, ty0, w);
       const int c = camera_of_row(block_off, g.blocks_per_cam, g.C, (int64_t)r);
-      const int w = tx1 - tx0;
-      cnt = (uint32_t)w * (uint32_t)(ty1 - ty0);
       S.t0[i] = (uint32_t)((uint64_t)c * (uint64_t)g.tiles_per_cam + (uint64_t)ty0 * g.tiles_x + (uint64_t)tx0);
       S.w[i] = (uint16_t)w;
-      S.dep[i] = (uint32_t)dkeys[p0 + i];
+      S.dep[i] = (uint32_t)(key >> 32);
       S.row[i] = r;
     }
     S.off[i] = cnt;
@@ -133,13 +210,56 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
     run += v[k];
   }
   if (tid == 0) S.off[kIxRows] = total;
+  if (warp == 0) {
+    // publish the block's total, then look back: lane j reads block
+    // blk - 1 - j of the current window; the nearest inclusive prefix ends
+    // the walk, a block that has not published makes the warp wait (bounded)
+    if (lane == 0)
+      atomicExch(reinterpret_cast<unsigned long long*>(status + blk), (blk == 0 ? kIxPre : kIxAgg) | total);
+    int64_t prefix = 0;
+    if (blk > 0) {
+      int64_t t = blk - 1;
+      int spins = 0;
+      while (true) {
+        const int64_t b = t - lane;
+        const uint64_t sv = b >= 0 ? ld_volatile(status + b) : kIxPre;  // before block 0: prefix 0
+        const uint32_t pre = __ballot_sync(0xffffffffu, (sv & kIxPre) != 0);
+        const uint32_t none = __ballot_sync(0xffffffffu, (sv & (kIxPre | kIxAgg)) == 0);
+        // lanes up to the first inclusive one, if no lane before it is unpublished
+        const int first_pre = pre ? __ffs(pre) - 1 : 32;
+        const int first_none = none ? __ffs(none) - 1 : 32;
+        // the published counts before the first unpublished block, up to and
+        // including the first inclusive prefix (64-bit sums: prefixes pass 2^32)
+        const int take = first_none < first_pre ? first_none : first_pre + 1;
+        uint64_t s = lane < take && b >= 0 ? (sv & kIxVal) : 0ull;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        prefix += (int64_t)s;
+        if (first_none < first_pre) {
+          // block t - first_none has not published yet: wait for it (bounded)
+          t -= first_none;
+          if (++spins > kIxSpinLimit) {
+            if (lane == 0) atomicOr(err, 1u);
+            break;
+          }
+          __nanosleep(64);
+          continue;
+        }
+        if (first_pre < 32) break;
+        t -= 32;
+      }
+      if (lane == 0)
+        atomicExch(reinterpret_cast<unsigned long long*>(status + blk), kIxPre | (uint64_t)(prefix + total));
+    }
+    if (lane == 0) S.base = prefix;
+  }
   __syncthreads();
-  const int64_t base = partial[blockIdx.x];
+  const int64_t base = S.base;
   for (int i = tid; i < nr; i += kIxThreads) isect_off[p0 + i] = base + (int64_t)S.off[i];
   // expand the block's slots; positions past nr have offset == total and are
   // never found for s < total
-  const uint32_t stop = (uint32_t)min64((int64_t)total, limit - base);
-  for (uint32_t s = tid; (int64_t)s < (int64_t)stop; s += kIxThreads) {
+  const uint32_t stop = (uint32_t)max64(0, min64((int64_t)total, limit - base));
+  for (uint32_t s = tid; s < stop; s += kIxThreads) {
     int lo = 0, hi = nr;  // largest i with S.off[i] <= s
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -151,37 +271,6 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
     keys[base + s] = (tile << 32) | S.dep[lo];
     vals[base + s] = S.row[lo];
   }
-}
-
-// Workspace: the count's scratch | row depth keys a, b (u64) | row ids a, b
-// (u32) | the row sort's scratch.
-struct IxTemp {
-  void* scan;
-  uint64_t *dk_a, *dk_b;
-  uint32_t *rows_a, *rows_b;
-  void* sort;
-};
-
-IxTemp isect_temp(void* temp, int64_t nnz) {
-  char* p = reinterpret_cast<char*>(temp);
-  IxTemp t;
-  t.scan = p;
-  p += scan_temp_bytes(nnz);
-  t.dk_a = reinterpret_cast<uint64_t*>(p);
-  p += align_up((size_t)nnz * 8, 256);
-  t.dk_b = reinterpret_cast<uint64_t*>(p);
-  p += align_up((size_t)nnz * 8, 256);
-  t.rows_a = reinterpret_cast<uint32_t*>(p);
-  p += align_up((size_t)nnz * 4, 256);
-  t.rows_b = reinterpret_cast<uint32_t*>(p);
-  p += align_up((size_t)nnz * 4, 256);
-  t.sort = p;
-  return t;
-}
-
-size_t isect_temp_bytes(int64_t nnz) {
-  return scan_temp_bytes(nnz) + 2 * align_up((size_t)nnz * 8, 256) + 2 * align_up((size_t)nnz * 4, 256) +
-         sort_temp_bytes(nnz);
 }
 
 }  // namespace ss
@@ -208,26 +297,21 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   if (((uintptr_t)aabb16 & 7) != 0) return invalid("aabb16 must be 8-byte aligned");
   if (!temp || temp_bytes < ss_workspace_bytes(dims, SS_WS_INTERSECT, nnz)) return invalid("temp too small");
   const IxTemp t = isect_temp(temp, nnz);
-  // the rows in depth order (ties by row index: the sort is stable)
-  k_row_keys<<<(unsigned)ceil_div(nnz, 256), 256, 0, st>>>(row_depth, nnz, t.dk_a, t.rows_a);
-  ss_status s = cuda_status(cudaGetLastError(), "row keys");
+  ss_status s = cuda_status(cudaMemsetAsync(t.total, 0, t.head_bytes, st), "memset");
   if (s) return s;
+  // the rows' depth keys and the exact total
+  k_row_keys<<<(unsigned)ceil_div(nnz, kRowKeyThreads), kRowKeyThreads, 0, st>>>(g, row_depth, aabb16, nnz, t.dk_a,
+                                                                                t.total);
+  s = cuda_status(cudaGetLastError(), "row keys");
+  if (s) return s;
+  // the rows in depth order (ties by row index: the sort is stable and the
+  // row index is the key's low word)
   bool in_b = false;
-  s = radix_sort_pairs(t.dk_a, t.rows_a, t.dk_b, t.rows_b, nnz, 4, 0, t.sort, st, &in_b);
+  s = radix_sort_pairs(t.dk_a, nullptr, t.dk_b, nullptr, nnz, 0, 4, t.sort, st, &in_b);
   if (s) return s;
   const uint64_t* dkeys = in_b ? t.dk_b : t.dk_a;
-  const uint32_t* rows = in_b ? t.rows_b : t.rows_a;
-  // the exact total, counted in that order
-  ScanSrc src{};
-  src.kind = SCAN_TILES_ORDERED;
-  src.aabb16 = aabb16;
-  src.rows = rows;
-  src.W = g.W; src.H = g.H; src.tiles_x = g.tiles_x; src.tiles_y = g.tiles_y;
-  s = scan_phase1(src, nnz, t.scan, isect_off + nnz, st);
-  if (s) return s;
   int64_t total = 0;
-  s = cuda_status(cudaMemcpyAsync(&total, isect_off + nnz, sizeof(int64_t), cudaMemcpyDeviceToHost, st),
-                  "copy n_isects");
+  s = cuda_status(cudaMemcpyAsync(&total, t.total, sizeof(int64_t), cudaMemcpyDeviceToHost, st), "copy n_isects");
   if (s) return s;
   bool flagged = false;
   s = radix_sort_flag(t.sort, st, &flagged);  // synchronises the stream
@@ -247,12 +331,23 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   }
   if (total > 0 && (!keys || !vals)) return invalid("null keys/vals");
   const int64_t limit = min64(total, cap_isects);
-  const int64_t* partial = reinterpret_cast<const int64_t*>(t.scan);
   s = cuda_status(cudaFuncSetAttribute(k_isect_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sizeof(IxSmem)),
                   "set smem attribute");
   if (s) return s;
   k_isect_fused<<<(unsigned)ceil_div(nnz, kIxRows), kIxThreads, sizeof(IxSmem), st>>>(
-      g, dkeys, rows, aabb16, block_off, partial, nnz, limit, isect_off, keys, vals);
-  return cuda_status(cudaGetLastError(), "intersect write");
+      g, dkeys, aabb16, block_off, nnz, limit, t.status, t.ticket, t.err, isect_off, keys, vals);
+  s = cuda_status(cudaGetLastError(), "intersect write");
+  if (s) return s;
+  // the write's look-back flag (stream sync)
+  uint32_t herr = 0;
+  s = cuda_status(cudaMemcpyAsync(&herr, t.err, 4, cudaMemcpyDeviceToHost, st), "copy flag");
+  if (s) return s;
+  s = cuda_status(cudaStreamSynchronize(st), "intersect write");
+  if (s) return s;
+  if (herr) {
+    set_error("ss_intersect_tiles: the write's look-back wait exceeded its limit");
+    return SS_ERR_DEVICE_CHECK;
+  }
+  return SS_OK;
 }

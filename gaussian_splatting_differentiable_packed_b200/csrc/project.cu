@@ -84,20 +84,6 @@ __host__ __device__ constexpr int rows_sh_stride() {
   return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
 }
 
-// L2 prefetch of the SH rows of block m0's Gaussians that some camera sees:
-// each warp ORs its 32 Gaussians' mask words over the cameras (lane c loads
-// camera c's, all in flight together) and each lane prefetches its row.
-__device__ __forceinline__ void prefetch_seen_rows(const Geo& g, const uint32_t* __restrict__ mask,
-                                                   const float* __restrict__ sh, int64_t m0, int K3) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t u = 0;
-  for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + m0) / 32 + warp];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
-  const int64_t m = m0 + threadIdx.x;
-  if (((u >> lane) & 1u) && m < g.N) prefetch_l2(sh + m * K3, (uint32_t)(K3 * 4));
-}
-
 // Bit gi of the CTA's per-warp visibility words.
 __device__ __forceinline__ bool seen(const uint32_t* s_seen, int gi) { return (s_seen[gi >> 5] >> (gi & 31)) & 1u; }
 
@@ -147,14 +133,15 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   const int cnt = (int)min64(kBlock, g.N - n0);
   const bool prefetch_ahead = ahead > 0 && blk + ahead < (int64_t)gridDim.x;
   if (prefetch_ahead && threadIdx.x == 0) {
-    // the parameters of the block that starts about a wave later, into L2
-    // (its SH rows follow once this block's own loads are in flight)
+    // the parameters and the SH block of the block that starts about a wave
+    // later, into L2
     const int64_t m0 = (blk + ahead) * kBlock;
     const int mc = (int)min64(kBlock, g.N - m0);
     prefetch_l2(means + 3 * m0, (uint32_t)(mc * 12));
     prefetch_l2(quats + 4 * m0, (uint32_t)(mc * 16));
     prefetch_l2(scales + 3 * m0, (uint32_t)(mc * 12));
     prefetch_l2(opacities + m0, (uint32_t)(mc * 4));
+    prefetch_l2(sh + m0 * K3, (uint32_t)(mc * K3 * 4));
   }
   // A chunk's cameras, first rows and each warp's mask word per camera.  The
   // first chunk is loaded before the parameters and the SH block so that its
@@ -190,40 +177,18 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     s_seen[threadIdx.x] = u;
   }
   __syncthreads();
-  // the CTA's contiguous SH block: a full block with all 16-byte loads in
-  // flight at once (it starts 16-byte aligned: 128*K3 floats per block), the
-  // ragged last block word by word
+  // the CTA's contiguous SH block, copied word by word into its padded
+  // shared layout by asynchronous copies: all in flight together and no
+  // register staging (which would cap the CTAs per SM); consecutive threads
+  // copy consecutive words
   {
     const float* src = sh + n0 * K3;
-    if (cnt == kBlock) {
-      constexpr int kV = kBlock * K3 / 4;
-      constexpr int kPer = (kV + kBlock - 1) / kBlock;
-      float4 buf[kPer];
-#pragma unroll
-      for (int r = 0; r < kPer; ++r) {
-        const int v = threadIdx.x + r * kBlock;
-        if (v < kV && (seen(s_seen, (4 * v) / K3) || seen(s_seen, (4 * v + 3) / K3)))
-          buf[r] = reinterpret_cast<const float4*>(src)[v];
-      }
-      if (prefetch_ahead) prefetch_seen_rows(g, mask, sh, (blk + ahead) * kBlock, K3);
-#pragma unroll
-      for (int r = 0; r < kPer; ++r) {
-        const int v = threadIdx.x + r * kBlock;
-        if (v < kV && (seen(s_seen, (4 * v) / K3) || seen(s_seen, (4 * v + 3) / K3))) {
-          const float e[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int f = 4 * v + u, gi = f / K3, qq = f - gi * K3;
-            sh_s[gi * KP + qq] = e[u];
-          }
-        }
-      }
-    } else {
-      for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-        const int gi = f / K3, qq = f - gi * K3;
-        if (seen(s_seen, gi)) sh_s[gi * KP + qq] = src[f];
-      }
+#pragma unroll 8
+    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+      const int gi = f / K3, qq = f - gi * K3;
+      if (seen(s_seen, gi)) cp_async4(&sh_s[gi * KP + qq], src + f);
     }
+    cp_async_wait_all();
   }
   auto process = [&](const RowItem& it) {
     const Cam& k = scam[it.cam];

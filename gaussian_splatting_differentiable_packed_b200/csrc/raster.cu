@@ -24,9 +24,6 @@ namespace ss {
 
 constexpr int kRThreads = 128;
 constexpr int kBatch = 256;
-// The backward stages half as many entries per batch (35 KB of shared memory
-// with the per-warp sums, at most 64 registers per thread).
-constexpr int kBatchB = 128;
 constexpr int kRedF = 12;
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
@@ -77,9 +74,8 @@ struct Stage {
   float4 e;  // 1/ca, cb/ca, bounded (1/0), depth
 };
 
-__device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint32_t r, Stage& st) {
-  const float4* row = reinterpret_cast<const float4*>(screen + (int64_t)r * kRowF);
-  const float4 r0 = row[0], r1 = row[1], r2 = row[2];
+// The staged form of screen row r (r0..r2: its three 16-byte words).
+__device__ __forceinline__ void stage_from(const float4 r0, const float4 r1, const float4 r2, uint32_t r, Stage& st) {
   const float ca = r0.z, cb = r0.w, cc = r1.x, o = r1.y;
   st.a = make_float4(r0.x, r0.y, mul(0.5f, ca), cb);
   st.b = make_float4(mul(0.5f, cc), o, r1.z, r1.w);
@@ -107,6 +103,11 @@ __device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint
   st.c = make_float4(r2.x, hx, hy, kterm);
   st.d = make_float4(thr, __uint_as_float(r), P, dql);
   st.e = make_float4(ica, cbr, bounded, r2.y);
+}
+
+__device__ __forceinline__ void stage_row(const float* __restrict__ screen, uint32_t r, Stage& st) {
+  const float4* row = reinterpret_cast<const float4*>(screen + (int64_t)r * kRowF);
+  stage_from(row[0], row[1], row[2], r, st);
 }
 
 // Warp culling.  For an entry with o <= 1 every pixel whose computed sigma
@@ -655,41 +656,13 @@ __device__ __forceinline__ bool pair_grad(const Stage& st, float dx, float2 dy, 
   return true;
 }
 
-// One vector atomic per (touched entry, 16-byte group) of a batch with the
-// warps' sums added up, one thread per entry; the sums and the entry's flag
-// are re-zeroed for the batch after next.
-__device__ __forceinline__ void flush_sums(float (*red)[kBatchB][kRedF], const uint32_t* rows, uint32_t* any, int cnt,
-                                           float* __restrict__ v_screen) {
-  for (int k = threadIdx.x; k < cnt; k += kRThreads) {
-    if (!any[k]) continue;
-    any[k] = 0u;
-    float* dst = v_screen + (int64_t)rows[k] * kRowF;
-#pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < kRThreads / 32; ++w) {
-        float4* src = reinterpret_cast<float4*>(&red[w][k][4 * q]);
-        const float4 x = *src;
-        *src = make_float4(0.f, 0.f, 0.f, 0.f);
-        v.x += x.x;
-        v.y += x.y;
-        v.z += x.z;
-        v.w += x.w;
-      }
-      atomicAdd(reinterpret_cast<float4*>(dst + 4 * q), v);
-    }
-  }
-}
-
 // The warp's sums of an entry when a single lane contributed: that lane's
 // values, stored by it (the row's pad words stay zero).
 template <bool EXT>
-__device__ __forceinline__ void store_sums(float* row, const float* gr, uint32_t* any) {
+__device__ __forceinline__ void store_sums(float* row, const float* gr) {
   reinterpret_cast<float4*>(row)[0] = make_float4(gr[0], gr[1], gr[2], gr[3]);
   reinterpret_cast<float4*>(row)[1] = make_float4(gr[4], gr[5], gr[6], gr[7]);
   reinterpret_cast<float2*>(row)[4] = make_float2(gr[8], EXT ? gr[9] : 0.0f);
-  *any = 1u;
 }
 
 // One replayed entry (bit hb of the lanes' candidate masks mA, mB) for the
@@ -717,6 +690,15 @@ __device__ __forceinline__ bool entry_grad(const Stage& st, uint32_t mA, uint32_
 
 // EXT: v_depth (nullable, per pixel) and bg (nullable, [C][3]; the blend
 // img = C + T_final * bg adds g . bg to dL/dT_final).
+//
+// Each warp replays its own 16x4 region independently (no CTA barrier): it
+// walks the tile's entries from the last one any of its pixels composited
+// down to the tile's first, 32 at a time, lane l holding entry
+// top - 32k - 31 + l of block k.  The screen rows of block k + 1 are copied
+// into the warp's second row buffer (asynchronous 16-byte copies) while
+// block k runs, with the row ids of block k + 2 loaded meanwhile.  A
+// touched entry's warp sums go to v_screen with three 16-byte atomics from
+// the lane that holds the entry.
 template <bool EXT>
 __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float* __restrict__ screen,
                                                           const uint32_t* __restrict__ vals,
@@ -729,17 +711,13 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
                                                           const float* __restrict__ bg,
                                                           const uint32_t* __restrict__ tile_order,
                                                           float* __restrict__ v_screen) {
-  __shared__ Stage s_e[kBatchB];
-  // each warp's per-entry sums (plain stores: a warp visits an entry at most
-  // once per batch), added up over the warps at the flush
-  __shared__ __align__(16) float red[kRThreads / 32][kBatchB][kRedF];
-  // row ids and touched flags of the batch in work and of the one being
-  // flushed (double-buffered: the flush of a batch runs beside the staging
-  // of the next one)
-  __shared__ uint32_t s_row[2][kBatchB];
-  __shared__ uint32_t s_any[2][kBatchB];
-  __shared__ int s_maxlast;
-  const int lane = threadIdx.x & 31;
+  constexpr int kWarps = kRThreads / 32;
+  __shared__ __align__(16) float s_raw[kWarps][2][32][kRowF];  // rows of the block in work and the next
+  __shared__ Stage s_e[kWarps][32];
+  // the warp's sums of each entry of the block (plain stores: a warp visits
+  // an entry once; slots 10 and 11, and 9 without EXT, stay zero)
+  __shared__ __align__(16) float red[kWarps][32][kRedF];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t tile = tile_order ? (int64_t)tile_order[blockIdx.x] : (int64_t)blockIdx.x;
   if (tile >= g.n_tiles) return;  // not a tile index: nothing to replay
   int c, tx0, ty0, i, j;
@@ -751,10 +729,9 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
   const float y_lo = (float)(j - 2 * (lane >> 4)) + 0.5f;
   const int64_t beg = tile_off[tile];
   const float amin = alpha_min();
-  for (int t = threadIdx.x; t < (kRThreads / 32) * kBatchB * kRedF; t += kRThreads) (&red[0][0][0])[t] = 0.0f;
-  for (int t = threadIdx.x; t < 2 * kBatchB; t += kRThreads) (&s_any[0][0])[t] = 0u;
-  if (threadIdx.x == 0) s_maxlast = -1;
-  __syncthreads();
+  float* rw = &red[warp][lane][0];
+#pragma unroll
+  for (int t = 0; t < kRedF; ++t) rw[t] = 0.0f;
   PixB pa{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1}, pb{1.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, -1};
   const int64_t pixA = ((int64_t)c * g.H + j) * g.W + i, pixB = pixA + g.W;
   if (inA) {
@@ -767,7 +744,6 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
     if (EXT && bg) vt += pa.g0 * bg[3 * c] + pa.g1 * bg[3 * c + 1] + pa.g2 * bg[3 * c + 2];
     if (EXT && v_depth) pa.gD = v_depth[pixA];
     pa.vTT = mul(vt, pa.T);
-    if (pa.last >= 0) atomicMax(&s_maxlast, (int)pa.last);
   }
   if (inB) {
     pb.last = last_id[pixB];
@@ -779,126 +755,141 @@ __global__ __launch_bounds__(kRThreads, 6) void k_raster_bwd(Geo g, const float*
     if (EXT && bg) vt += pb.g0 * bg[3 * c] + pb.g1 * bg[3 * c + 1] + pb.g2 * bg[3 * c + 2];
     if (EXT && v_depth) pb.gD = v_depth[pixB];
     pb.vTT = mul(vt, pb.T);
-    if (pb.last >= 0) atomicMax(&s_maxlast, (int)pb.last);
   }
-  __syncthreads();
-  const int64_t stop = (int64_t)s_maxlast + 1;  // entries [beg, stop) can matter
-  int64_t wlast = max64(pa.last, pb.last);
+  int64_t top = max64(pa.last, pb.last);  // the warp's last replayed entry
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wlast = max64(wlast, __shfl_xor_sync(0xffffffffu, wlast, o));
-  int par = 0, prev_cnt = 0;
-  for (int64_t b1 = stop; b1 > beg; b1 -= kBatchB, par ^= 1) {
-    const int64_t b0 = max64(beg, b1 - kBatchB);
-    const int cnt = (int)(b1 - b0);
-    for (int t = threadIdx.x; t < cnt; t += kRThreads) {
-      const uint32_t r = vals[b0 + t];
-      s_row[par][t] = r;
-      stage_row(screen, r, s_e[t]);
+  for (int o = 16; o > 0; o >>= 1) top = max64(top, __shfl_xor_sync(0xffffffffu, top, o));
+  if (top < beg) return;
+  const int nblk = (int)((top - beg) / 32 + 1);
+  // row id of this lane's entry in block k (~0u: none)
+  auto row_of = [&](int k) -> uint32_t {
+    const int64_t e = top - 32 * (int64_t)k - 31 + lane;
+    return (k < nblk && e >= beg) ? vals[e] : ~0u;
+  };
+  auto fetch = [&](int k, uint32_t r) {
+    if (r != ~0u) {
+      const float* src = screen + (int64_t)r * kRowF;
+      float* dst = &s_raw[warp][k & 1][lane][0];
+      cp_async16(dst, src);
+      cp_async16(dst + 4, src + 4);
+      cp_async16(dst + 8, src + 8);
     }
-    flush_sums(red, s_row[par ^ 1], s_any[par ^ 1], prev_cnt, v_screen);
-    prev_cnt = cnt;
-    __syncthreads();
-    uint32_t* any = s_any[par];
-    if (b0 <= wlast) {
-      for (int q = (cnt - 1) / 32; q >= 0; --q) {
-        const int e = q * 32 + lane;
-        const int64_t qb = b0 + q * 32;
-        if (qb > wlast) continue;  // warp-uniform: no pixel of the warp replays the block
-        // candidate masks as in the forward: bit b of mA (mB) set when entry
-        // qb + b can reach this lane's upper (lower) pixel and the pixel
-        // replays it; the warp steps through the union of its lanes' masks
-        uint32_t covA = 0u, covB = 0u;
-        if (e < cnt) entry_coverage(s_e[e], x_lo, y_lo, covA, covB);
-        const uint32_t mA = warp_transpose32(covA, lane) & live_bits(pa.last, qb);
-        const uint32_t mB = warp_transpose32(covB, lane) & live_bits(pb.last, qb);
-        uint32_t bits = __reduce_or_sync(0xffffffffu, mA | mB);
-        const int warp = threadIdx.x >> 5;
-        while (bits) {
-          const int hb = 31 - __clz(bits);
-          bits &= ~(1u << hb);
-          int kA = q * 32 + hb;
-          float gr[10];
-          bool cA;
-          uint32_t balA;
-          const uint32_t mAB = mA | mB;
-          if (bits) {
-            // the next candidate of the warp: its pixel step follows this
-            // one's, and the two entries' sums are reduced together
-            const int hb2 = 31 - __clz(bits);
-            bits &= ~(1u << hb2);
-            const int kB = q * 32 + hb2;
-            float gr2[10];
-            bool cB;
-            const bool inA = (mAB >> hb) & 1u, inB = (mAB >> hb2) & 1u;
-            if (!__any_sync(0xffffffffu, inA && inB)) {
-              // no pixel pair of the warp is a candidate of both entries:
-              // each lane steps through the one entry it has (if any), so
-              // both entries take one pixel step between them
-              const int hx = inA ? hb : hb2;
-              float g1[10];
-              const bool c1 = entry_grad<EXT>(s_e[q * 32 + hx], mA, mB, hx, px, npy, amin, pa, pb, g1);
-              cA = inA && c1;
-              cB = !inA && c1;
+    cp_async_commit();
+  };
+  uint32_t rcur = row_of(0);
+  fetch(0, rcur);
+  uint32_t rnext = row_of(1);
+  for (int k = 0; k < nblk; ++k) {
+    const uint32_t rnext2 = row_of(k + 2);
+    fetch(k + 1, rnext);
+    cp_async_wait_group<1>();  // this lane's rows of block k have landed
+    const int64_t qb = top - 32 * (int64_t)k - 31;
+    uint32_t covA = 0u, covB = 0u;
+    if (rcur != ~0u) {
+      const float4* raw = reinterpret_cast<const float4*>(&s_raw[warp][k & 1][lane][0]);
+      Stage st;
+      stage_from(raw[0], raw[1], raw[2], rcur, st);
+      s_e[warp][lane] = st;
+      entry_coverage(st, x_lo, y_lo, covA, covB);
+    }
+    __syncwarp();
+    // candidate masks as in the forward: bit b of mA (mB) set when entry
+    // qb + b can reach this lane's upper (lower) pixel and the pixel replays
+    // it; the warp steps through the union of its lanes' masks
+    const uint32_t mA = warp_transpose32(covA, lane) & live_bits(pa.last, qb);
+    const uint32_t mB = warp_transpose32(covB, lane) & live_bits(pb.last, qb);
+    uint32_t bits = __reduce_or_sync(0xffffffffu, mA | mB);
+    uint32_t touched = 0u;  // warp-uniform: entries whose sums were stored
+    while (bits) {
+      int hb = 31 - __clz(bits);
+      bits &= ~(1u << hb);
+      float gr[10];
+      bool cA;
+      uint32_t balA;
+      const uint32_t mAB = mA | mB;
+      if (bits) {
+        // the next candidate of the warp: its pixel step follows this
+        // one's, and the two entries' sums are reduced together
+        const int hb2 = 31 - __clz(bits);
+        bits &= ~(1u << hb2);
+        float gr2[10];
+        bool cB;
+        const bool inA2 = (mAB >> hb) & 1u, inB2 = (mAB >> hb2) & 1u;
+        if (!__any_sync(0xffffffffu, inA2 && inB2)) {
+          // no pixel pair of the warp is a candidate of both entries: each
+          // lane steps through the one entry it has (if any), so both
+          // entries take one pixel step between them
+          const int hx = inA2 ? hb : hb2;
+          float g1[10];
+          const bool c1 = entry_grad<EXT>(s_e[warp][hx], mA, mB, hx, px, npy, amin, pa, pb, g1);
+          cA = inA2 && c1;
+          cB = !inA2 && c1;
 #pragma unroll
-              for (int t = 0; t < 10; ++t) {
-                gr[t] = inA ? g1[t] : 0.0f;
-                gr2[t] = inA ? 0.0f : g1[t];
-              }
-            } else {
-              cA = entry_grad<EXT>(s_e[kA], mA, mB, hb, px, npy, amin, pa, pb, gr);
-              cB = entry_grad<EXT>(s_e[kB], mA, mB, hb2, px, npy, amin, pa, pb, gr2);
-            }
-            balA = __ballot_sync(0xffffffffu, cA);
-            const uint32_t balB = __ballot_sync(0xffffffffu, cB);
-            if ((balA & (balA - 1u)) == 0u && (balB & (balB - 1u)) == 0u) {
-              // at most one lane contributes to each entry: its pixel pair's
-              // sums are the warp's, stored as they are
-              if (cA) store_sums<EXT>(red[warp][kA], gr, any + kA);
-              if (cB) store_sums<EXT>(red[warp][kB], gr2, any + kB);
-              continue;
-            }
-            if (balA && balB) {
-              const float s8 = warp_reduce8x2(gr, gr2, lane);
-              const float s2 = warp_sum_x2<EXT>(gr[8], gr[9], gr2[8], gr2[9], lane);
-              const int kl = (lane & 16) ? kB : kA;
-              if ((lane & 1) == 0) red[warp][kl][((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = s8;
-              if ((lane & 15) == 0) {
-                red[warp][kl][8] = s2;
-                any[kl] = 1u;
-              }
-              if (EXT && (lane & 15) == 8) red[warp][kl][9] = s2;
-              continue;
-            }
-            if (balB) {
+          for (int t = 0; t < 10; ++t) {
+            gr[t] = inA2 ? g1[t] : 0.0f;
+            gr2[t] = inA2 ? 0.0f : g1[t];
+          }
+        } else {
+          cA = entry_grad<EXT>(s_e[warp][hb], mA, mB, hb, px, npy, amin, pa, pb, gr);
+          cB = entry_grad<EXT>(s_e[warp][hb2], mA, mB, hb2, px, npy, amin, pa, pb, gr2);
+        }
+        balA = __ballot_sync(0xffffffffu, cA);
+        const uint32_t balB = __ballot_sync(0xffffffffu, cB);
+        touched |= (balA ? 1u << hb : 0u) | (balB ? 1u << hb2 : 0u);
+        if ((balA & (balA - 1u)) == 0u && (balB & (balB - 1u)) == 0u) {
+          // at most one lane contributes to each entry: its pixel pair's
+          // sums are the warp's, stored as they are
+          if (cA) store_sums<EXT>(red[warp][hb], gr);
+          if (cB) store_sums<EXT>(red[warp][hb2], gr2);
+          continue;
+        }
+        if (balA && balB) {
+          const float s8 = warp_reduce8x2(gr, gr2, lane);
+          const float s2 = warp_sum_x2<EXT>(gr[8], gr[9], gr2[8], gr2[9], lane);
+          const int kl = (lane & 16) ? hb2 : hb;
+          if ((lane & 1) == 0) red[warp][kl][((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = s8;
+          if ((lane & 15) == 0) red[warp][kl][8] = s2;
+          if (EXT && (lane & 15) == 8) red[warp][kl][9] = s2;
+          continue;
+        }
+        if (balB) {
 #pragma unroll
-              for (int t = 0; t < 10; ++t) gr[t] = gr2[t];
-              kA = kB;
-              cA = cB;
-              balA = balB;
-            }
-          } else {
-            cA = entry_grad<EXT>(s_e[kA], mA, mB, hb, px, npy, amin, pa, pb, gr);
-            balA = __ballot_sync(0xffffffffu, cA);
-          }
-          if ((balA & (balA - 1u)) == 0u) {
-            if (cA) store_sums<EXT>(red[warp][kA], gr, any + kA);
-          } else {
-            const float s8 = warp_reduce8(gr, lane);
-            const float sb = warp_sum(gr[8]);
-            const float sd = EXT ? warp_sum(gr[9]) : 0.0f;
-            if ((lane & 3) == 0) red[warp][kA][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = s8;
-            if (lane == 0) {
-              red[warp][kA][8] = sb;
-              if (EXT) red[warp][kA][9] = sd;
-              any[kA] = 1u;
-            }
-          }
+          for (int t = 0; t < 10; ++t) gr[t] = gr2[t];
+          hb = hb2;
+          cA = cB;
+          balA = balB;
+        }
+      } else {
+        cA = entry_grad<EXT>(s_e[warp][hb], mA, mB, hb, px, npy, amin, pa, pb, gr);
+        balA = __ballot_sync(0xffffffffu, cA);
+        touched |= balA ? 1u << hb : 0u;
+      }
+      if ((balA & (balA - 1u)) == 0u) {
+        if (cA) store_sums<EXT>(red[warp][hb], gr);
+      } else {
+        const float s8 = warp_reduce8(gr, lane);
+        const float sb = warp_sum(gr[8]);
+        const float sd = EXT ? warp_sum(gr[9]) : 0.0f;
+        if ((lane & 3) == 0) red[warp][hb][((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)] = s8;
+        if (lane == 0) {
+          red[warp][hb][8] = sb;
+          if (EXT) red[warp][hb][9] = sd;
         }
       }
     }
-    __syncthreads();
+    __syncwarp();
+    if ((touched >> lane) & 1u) {
+      const float4* src = reinterpret_cast<const float4*>(rw);
+      float4* dst = reinterpret_cast<float4*>(v_screen + (int64_t)rcur * kRowF);
+      atomicAdd(dst, src[0]);
+      atomicAdd(dst + 1, src[1]);
+      atomicAdd(dst + 2, src[2]);
+    }
+    __syncwarp();
+    rcur = rnext;
+    rnext = rnext2;
   }
-  flush_sums(red, s_row[par ^ 1], s_any[par ^ 1], prev_cnt, v_screen);
+  cp_async_wait_group<0>();
 }
 
 // ----- tile order: heaviest tiles first ------------------------------------

@@ -13,7 +13,6 @@ namespace ss {
 
 __device__ __forceinline__ int64_t item_count(const ScanSrc& s, int64_t i) {
   if (s.kind == SCAN_U32) return (int64_t)s.u32[i];
-  if (s.kind == SCAN_TILES_ORDERED) i = s.rows[i];
   uint32_t w0 = s.aabb16[2 * i], w1 = s.aabb16[2 * i + 1];
   int tx0, tx1, ty0, ty1;
   tile_span(w0 & 0xFFFFu, w1 & 0xFFFFu, s.W, s.tiles_x, tx0, tx1);

@@ -35,6 +35,7 @@ constexpr int kSortItems = 16;
 constexpr int kSortTile = kSortThreads * kSortItems;  // 4096 keys per CTA
 constexpr int kRadix = 256;
 constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kHistItems = 8;  // keys per thread per histogram round
 
 constexpr int kMaxPasses = 8;
 constexpr uint64_t kFlagAgg = 1ull << 54;
@@ -57,25 +58,33 @@ __global__ __launch_bounds__(kSortThreads) void k_hist_all(const uint64_t* __res
   for (int i = threadIdx.x; i < kSortWarps * kPerWarp; i += kSortThreads) hw[i] = 0;
   __syncthreads();
   uint32_t* mine = hw + warp * kPerWarp;
-  // coalesced: a warp reads 32 consecutive keys; neighbouring keys share
-  // digits (a row's keys share the depth and neighbouring tile ids), so each
-  // run of equal digits is counted by its first lane with one shared atomic
-  const int64_t stride = (int64_t)gridDim.x * kSortThreads;
-  for (int64_t base = (int64_t)blockIdx.x * kSortThreads; base < n; base += stride) {
-    const int64_t i = base + threadIdx.x;
-    const bool valid = i < n;
-    const uint64_t k = valid ? keys[i] : 0ull;
-    const uint32_t lo = (uint32_t)k, hi = (uint32_t)(k >> 32);
-    const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-    const uint32_t end_all = 32u - (uint32_t)__clz(vmask);
-    const uint32_t above = ~((2u << lane) - 1u);  // lanes above this one
+  // coalesced: a warp reads kHistItems runs of 32 consecutive keys, all in
+  // flight together; neighbouring keys share digits (a row's keys share the
+  // depth and neighbouring tile ids), so each run of equal digits is counted
+  // by its first lane with one shared atomic
+  const int64_t stride = (int64_t)gridDim.x * kSortThreads * kHistItems;
+  for (int64_t base = ((int64_t)blockIdx.x * kSortWarps + warp) * 32 * kHistItems; base < n; base += stride) {
+    uint64_t kr[kHistItems];
 #pragma unroll
-    for (int p = 0; p < PASSES; ++p) {
-      const uint32_t d = ((p < lo_bytes ? lo >> (8 * p) : hi >> (8 * (p - lo_bytes)))) & 0xFFu;
-      const uint32_t prev = __shfl_up_sync(0xffffffffu, d, 1);
-      const bool head = valid && (lane == 0 || d != prev);
-      const uint32_t after = __ballot_sync(0xffffffffu, head) & above;
-      if (head) atomicAdd(&mine[p * kRadix + d], (after ? (uint32_t)(__ffs(after) - 1) : end_all) - (uint32_t)lane);
+    for (int r = 0; r < kHistItems; ++r) {
+      const int64_t i = base + r * 32 + lane;
+      kr[r] = i < n ? keys[i] : 0ull;
+    }
+#pragma unroll
+    for (int r = 0; r < kHistItems; ++r) {
+      const bool valid = base + r * 32 + lane < n;
+      const uint32_t lo = (uint32_t)kr[r], hi = (uint32_t)(kr[r] >> 32);
+      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+      const uint32_t end_all = 32u - (uint32_t)__clz(vmask);
+      const uint32_t above = ~((2u << lane) - 1u);  // lanes above this one
+#pragma unroll
+      for (int p = 0; p < PASSES; ++p) {
+        const uint32_t d = ((p < lo_bytes ? lo >> (8 * p) : hi >> (8 * (p - lo_bytes)))) & 0xFFu;
+        const uint32_t prev = __shfl_up_sync(0xffffffffu, d, 1);
+        const bool head = valid && (lane == 0 || d != prev);
+        const uint32_t after = __ballot_sync(0xffffffffu, head) & above;
+        if (head) atomicAdd(&mine[p * kRadix + d], (after ? (uint32_t)(__ffs(after) - 1) : end_all) - (uint32_t)lane);
+      }
     }
   }
   __syncthreads();
@@ -132,6 +141,7 @@ __device__ __forceinline__ uint64_t ld_status(const uint64_t* p) {
   return *reinterpret_cast<const volatile unsigned long long*>(p);
 }
 
+template <bool VALS>
 __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __restrict__ kin,
                                                            const uint32_t* __restrict__ vin,
                                                            uint64_t* __restrict__ kout, uint32_t* __restrict__ vout,
@@ -157,7 +167,7 @@ __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __res
     const int64_t i = base + r * 32 + lane;
     const bool valid = i < n;
     kk[r] = valid ? kin[i] : 0ull;
-    vv[r] = valid ? vin[i] : 0u;
+    if (VALS) vv[r] = valid ? vin[i] : 0u;
     const uint32_t d = valid ? (uint32_t)(kk[r] >> shift) & 0xFFu : 0x100u;
     const uint32_t peers = __match_any_sync(0xffffffffu, d);
     const uint32_t before = valid ? S.wcnt[warp][d] : 0u;
@@ -249,7 +259,7 @@ __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __res
     const uint32_t d = (uint32_t)(kk[r] >> shift) & 0xFFu;
     const uint32_t lp = S.dstart[d] + S.wcnt[warp][d] + pos[r];
     S.k[lp] = kk[r];
-    S.v[lp] = vv[r];
+    if (VALS) S.v[lp] = vv[r];
   }
   __syncthreads();
   const int cnt = (int)min64(kSortTile, n - tile0);
@@ -258,7 +268,7 @@ __global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __res
     const uint32_t d = (uint32_t)(key >> shift) & 0xFFu;
     const int64_t gpos = S.gbase[d] + (i - (int64_t)S.dstart[d]);
     kout[gpos] = key;
-    vout[gpos] = S.v[i];
+    if (VALS) vout[gpos] = S.v[i];
   }
 }
 
@@ -299,13 +309,15 @@ namespace ss {
 // lo_bytes bytes (4, or 0 when the keys already arrive in the order of their
 // low words, ties in the order to keep), then the high word's hi_bytes bytes.
 // The histograms are read back (one small copy, stream sync) and a digit
-// equal in every key is skipped.  *in_b: the result is in (kb, vb).  temp:
-// sort_temp_bytes(n), cleared here.  The look-back flag is left in temp
-// (radix_sort_flag).
+// equal in every key is skipped.  va and vb null: keys only.  *in_b: the
+// result is in (kb, vb).  temp: sort_temp_bytes(n), cleared here.  The
+// look-back flag is left in temp (radix_sort_flag).
 ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
                            int hi_bytes, void* temp, cudaStream_t st, bool* in_b) {
   *in_b = false;
-  ss_status s = cuda_status(cudaFuncSetAttribute(k_onesweep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool vals = va != nullptr;
+  ss_status s = cuda_status(cudaFuncSetAttribute(vals ? k_onesweep<true> : k_onesweep<false>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)sizeof(OnesweepSmem)),
                             "set smem attribute");
   if (s) return s;
@@ -352,7 +364,7 @@ ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* v
     if (one_bin) continue;
     const int shift = p < lo_bytes ? 8 * p : 32 + 8 * (p - lo_bytes);
     const uint64_t epoch = (uint64_t)(run + 1) << 56;
-    k_onesweep<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
+    (vals ? k_onesweep<true> : k_onesweep<false>)<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
         kin, vin, kout, vout, n, shift, epoch, hist + p * kRadix, status, tickets + run, err);
     s = cuda_status(cudaGetLastError(), "radix pass");
     if (s) return s;

@@ -85,6 +85,23 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// Asynchronous 4-byte copy global -> shared (no register holds the word;
+// the copies of a thread complete at cp_async_wait_all).
+__device__ __forceinline__ void cp_async4(float* smem_dst, const float* gsrc) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gsrc) : "memory");
+}
+// Asynchronous 16-byte copy global -> shared (both 16-byte aligned), L2 only.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N of the thread's committed copy groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Resident CTAs of a kernel over the whole GPU (SMs x CTAs per SM): the
 // distance, in blocks, between a CTA and the one that starts about a wave
 // later.  0 if the query fails (then nothing is prefetched ahead).
@@ -99,12 +116,11 @@ inline int64_t wave_blocks(K kernel, int threads, size_t smem) {
 
 // ----- generic exclusive scan (int64 totals), defined in scan.cu -----
 // Items are produced by a "counter" selected by kind:
-enum ScanKind { SCAN_U32 = 0, SCAN_TILES = 1, SCAN_TILES_ORDERED = 2 };
+enum ScanKind { SCAN_U32 = 0, SCAN_TILES = 1 };
 struct ScanSrc {
   int kind;
   const uint32_t* u32;     // SCAN_U32: counts
   const uint32_t* aabb16;  // SCAN_TILES: per-row AABB16, count = tiles covered
-  const uint32_t* rows;  // SCAN_TILES_ORDERED: item i is row rows[i]
   int W, H, tiles_x, tiles_y;
 };
 constexpr int kScanItems = 16;

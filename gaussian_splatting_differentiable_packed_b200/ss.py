@@ -506,9 +506,9 @@ def sort_launches(n_isects: int, passes: int) -> int:
 
 def launches_per_step(d: ss_dims, nnz: int, n_isects: int, sort_passes: int, depth_passes: int) -> int:
     """Kernels libss launches in one forward+backward step (memsets excluded):
-    projection 5 (pass 1, three scan kernels, pass 2), intersection 6 plus
-    one per depth-sort pass (row depth keys, the depth sort's histogram and
-    bases, two count kernels, the fused offsets-and-write kernel), the sort
+    projection 5 (pass 1, three scan kernels, pass 2), intersection 4 plus
+    one per depth-sort pass (row depth keys with the count, the depth sort's
+    histogram and bases, the fused offsets-and-write kernel), the sort
     (sort_launches), tile order 3 (histogram, scan, scatter), rasterizer
     1 + 1, projection backward 1.  With no Gaussians only the tile order and
     the two rasterizers launch (they still write the empty images)."""
@@ -516,7 +516,7 @@ def launches_per_step(d: ss_dims, nnz: int, n_isects: int, sort_passes: int, dep
         return 3 + 2
     n = 5
     if nnz > 0:
-        n += 6 + depth_passes
+        n += 4 + depth_passes
     n += sort_launches(n_isects, sort_passes)
     return n + 3 + 3
 

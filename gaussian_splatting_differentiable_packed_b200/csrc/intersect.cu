@@ -11,8 +11,8 @@
 // row on the 15M-Gaussian workload, 59 on the 7680^2 one).
 //
 //   k_row_keys      (depth bits << 32 | row) of every row, and the exact
-//                   int64 total of tiles covered (integer atomics: the sum
-//                   is the same in any order)
+//                   int64 total of tiles covered (integer atomics, one per
+//                   CTA: the sum is the same in any order)
 //   radix sort      keys only, by the depth word (sort.cu; the row index in
 //                   the low word rides along, ties stay in row order)
 //   (host)          checks the total against the capacity and 2^31
@@ -102,20 +102,20 @@ __device__ __forceinline__ uint32_t row_tiles(const Geo& g, uint2 q, int& tx0, i
   return (uint32_t)w * (uint32_t)(ty1 - ty0);
 }
 
+// Grid-stride over the rows (a few CTAs per SM): one 64-bit atomic per CTA
+// for the total, not one per 256 rows.
 __global__ __launch_bounds__(kRowKeyThreads) void k_row_keys(Geo g, const float* __restrict__ row_depth,
                                                              const uint32_t* __restrict__ aabb16, int64_t nnz,
                                                              uint64_t* __restrict__ keys,
                                                              int64_t* __restrict__ total) {
-  __shared__ uint32_t ws[kRowKeyThreads / 32];
-  const int64_t r = (int64_t)blockIdx.x * kRowKeyThreads + threadIdx.x;
-  uint32_t cnt = 0;
-  if (r < nnz) {
+  __shared__ unsigned long long ws[kRowKeyThreads / 32];
+  unsigned long long cnt = 0;
+  for (int64_t r = (int64_t)blockIdx.x * kRowKeyThreads + threadIdx.x; r < nnz;
+       r += (int64_t)gridDim.x * kRowKeyThreads) {
     keys[r] = ((uint64_t)__float_as_uint(row_depth[r]) << 32) | (uint64_t)r;
     int tx0, ty0, w;
-    cnt = row_tiles(g, reinterpret_cast<const uint2*>(aabb16)[r], tx0, ty0, w);
+    cnt += row_tiles(g, reinterpret_cast<const uint2*>(aabb16)[r], tx0, ty0, w);
   }
-  // a row covers at most 4096 x 4096 tiles (16-bit image extents), so a
-  // warp's sum fits 32 bits; the warps' sums are added in 64 bits
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
   if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = cnt;
@@ -256,6 +256,7 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
   __syncthreads();
   const int64_t base = S.base;
   for (int i = tid; i < nr; i += kIxThreads) isect_off[p0 + i] = base + (int64_t)S.off[i];
+  if (tid == 0 && p0 + nr == nnz) isect_off[nnz] = base + (int64_t)total;  // the last block: the total
   // expand the block's slots; positions past nr have offset == total and are
   // never found for s < total
   const uint32_t stop = (uint32_t)max64(0, min64((int64_t)total, limit - base));
@@ -266,7 +267,12 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
       if (S.off[mid] <= s) lo = mid; else hi = mid;
     }
     const uint32_t k = s - S.off[lo], w = S.w[lo];
-    const uint32_t ty = k / w, tx = k - ty * w;
+    // k / w through the approximate reciprocal: k < 2^24, so the estimate is
+    // off by at most one, and one correction each way makes it exact
+    uint32_t ty = (uint32_t)__fmul_rz((float)k, __frcp_rn((float)w));
+    if (ty * w > k) --ty;
+    if ((ty + 1) * w <= k) ++ty;
+    const uint32_t tx = k - ty * w;
     const uint64_t tile = (uint64_t)S.t0[lo] + (uint64_t)ty * (uint64_t)g.tiles_x + tx;
     keys[base + s] = (tile << 32) | S.dep[lo];
     vals[base + s] = S.row[lo];
@@ -300,8 +306,8 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   ss_status s = cuda_status(cudaMemsetAsync(t.total, 0, t.head_bytes, st), "memset");
   if (s) return s;
   // the rows' depth keys and the exact total
-  k_row_keys<<<(unsigned)ceil_div(nnz, kRowKeyThreads), kRowKeyThreads, 0, st>>>(g, row_depth, aabb16, nnz, t.dk_a,
-                                                                                t.total);
+  k_row_keys<<<(unsigned)min64(ceil_div(nnz, kRowKeyThreads), 148 * 8), kRowKeyThreads, 0, st>>>(
+      g, row_depth, aabb16, nnz, t.dk_a, t.total);
   s = cuda_status(cudaGetLastError(), "row keys");
   if (s) return s;
   // the rows in depth order (ties by row index: the sort is stable and the

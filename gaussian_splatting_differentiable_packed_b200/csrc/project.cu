@@ -78,10 +78,21 @@ __global__ __launch_bounds__(kBlock) void k_project_mask(Geo g, const float* __r
   }
 }
 
-// Shared-memory stride per Gaussian for an SH block (odd: conflict-free).
+// Shared-memory layout of a CTA's SH block.  With 3(D+1)^2 a multiple of 4
+// (degrees 1 and 3) a row is copied and read in 16-byte words and its stride
+// is an odd number of them, so the 8 lanes of a quarter-warp that read 16
+// bytes each from 8 different rows hit 8 different bank groups.  Otherwise
+// the stride is an odd number of words (word accesses of 32 rows conflict-
+// free).
+template <int DEG>
+__host__ __device__ constexpr bool rows_sh_vec() {
+  return (3 * (DEG + 1) * (DEG + 1)) % 4 == 0;
+}
 template <int DEG>
 __host__ __device__ constexpr int rows_sh_stride() {
-  return ((3 * (DEG + 1) * (DEG + 1)) % 2 == 0) ? 3 * (DEG + 1) * (DEG + 1) + 1 : 3 * (DEG + 1) * (DEG + 1);
+  constexpr int K3 = 3 * (DEG + 1) * (DEG + 1);
+  if (rows_sh_vec<DEG>()) return ((K3 / 4) % 2 == 1) ? K3 : K3 + 4;
+  return (K3 % 2 == 0) ? K3 + 1 : K3;
 }
 
 // Bit gi of the CTA's per-warp visibility words.
@@ -119,7 +130,7 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   constexpr int kWarps = kBlock / 32;
   constexpr int kSlots = kCamChunk * kWarps;
   __shared__ Cam scam[kCamChunk];
-  __shared__ float sh_s[kBlock * KP];
+  __shared__ __align__(16) float sh_s[kBlock * KP];
   __shared__ GaussIn s_g[kBlock];
   __shared__ float s_o[kBlock];
   __shared__ uint32_t s_word[kSlots];  // [camera][warp]
@@ -177,16 +188,25 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     s_seen[threadIdx.x] = u;
   }
   __syncthreads();
-  // the CTA's contiguous SH block, copied word by word into its padded
-  // shared layout by asynchronous copies: all in flight together and no
-  // register staging (which would cap the CTAs per SM); consecutive threads
-  // copy consecutive words
+  // the CTA's contiguous SH block (16-byte aligned: 128 * K3 floats a block)
+  // into its padded shared layout by asynchronous copies: all in flight
+  // together and no register staging (which would cap the CTAs per SM);
+  // consecutive threads copy consecutive 16-byte (or 4-byte) words
   {
     const float* src = sh + n0 * K3;
+    if constexpr (rows_sh_vec<DEG>()) {
+      constexpr int Q = K3 / 4;  // 16-byte words a row
+#pragma unroll 4
+      for (int v = threadIdx.x; v < cnt * Q; v += kBlock) {
+        const int gi = v / Q, qq = v - gi * Q;
+        if (seen(s_seen, gi)) cp_async16(&sh_s[gi * KP + 4 * qq], src + 4 * v);
+      }
+    } else {
 #pragma unroll 8
-    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-      const int gi = f / K3, qq = f - gi * K3;
-      if (seen(s_seen, gi)) cp_async4(&sh_s[gi * KP + qq], src + f);
+      for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+        const int gi = f / K3, qq = f - gi * K3;
+        if (seen(s_seen, gi)) cp_async4(&sh_s[gi * KP + qq], src + f);
+      }
     }
     cp_async_wait_all();
   }
@@ -204,12 +224,31 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     if (DEG > 0) view_dir(k, gi.mx, gi.my, gi.mz, X, Y, Z, il);
     sh_basis(DEG, X, Y, Z, b);
     float rgb[3];
+    if constexpr (rows_sh_vec<DEG>()) {
+      // coefficient e = 3 kk + ch in increasing e: each channel's terms come
+      // in increasing kk, the canonical order
+      float acc[3] = {0.0f, 0.0f, 0.0f};
+      const float4* sh4 = reinterpret_cast<const float4*>(shn);
 #pragma unroll
-    for (int ch = 0; ch < 3; ++ch) {
-      float acc = mul(shn[ch], b[0]);
+      for (int q = 0; q < K3 / 4; ++q) {
+        const float4 w = sh4[q];
+        const float e4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], b[kk]));
-      rgb[ch] = fmaxf(add(acc, 0.5f), 0.0f);
+        for (int u = 0; u < 4; ++u) {
+          const int e = 4 * q + u, kk = e / 3, ch = e - 3 * kk;
+          acc[ch] = kk == 0 ? mul(e4[u], b[0]) : add(acc[ch], mul(e4[u], b[kk]));
+        }
+      }
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) rgb[ch] = fmaxf(add(acc[ch], 0.5f), 0.0f);
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) {
+        float acc = mul(shn[ch], b[0]);
+#pragma unroll
+        for (int kk = 1; kk < K; ++kk) acc = add(acc, mul(shn[3 * kk + ch], b[kk]));
+        rgb[ch] = fmaxf(add(acc, 0.5f), 0.0f);
+      }
     }
     float4* out = reinterpret_cast<float4*>(screen + it.row * kRowF);
     out[0] = make_float4(P.mx, P.my, ca, cb);

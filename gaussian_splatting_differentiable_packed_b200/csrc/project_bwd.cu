@@ -77,20 +77,6 @@ __device__ __forceinline__ void sh_dir_grads(float X, float Y, float Z, const fl
   vdir[2] = gZ;
 }
 
-// L2 prefetch of the SH rows of block m0's Gaussians that some camera sees:
-// each warp ORs its 32 Gaussians' mask words over the cameras (lane c loads
-// camera c's, all in flight together) and each lane prefetches its row.
-__device__ __forceinline__ void prefetch_seen_rows(const Geo& g, const uint32_t* __restrict__ mask,
-                                                   const float* __restrict__ sh, int64_t m0, int K3) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t u = 0;
-  for (int c = lane; c < g.C; c += 32) u |= mask[((int64_t)c * g.n_pad + m0) / 32 + warp];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) u |= __shfl_xor_sync(0xffffffffu, u, o);
-  const int64_t m = m0 + threadIdx.x;
-  if (((u >> lane) & 1u) && m < g.N) prefetch_l2(sh + m * K3, (uint32_t)(K3 * 4));
-}
-
 // Bit gi of the CTA's per-warp visibility words.
 __device__ __forceinline__ bool seen(const uint32_t* s_seen, int gi) { return (s_seen[gi >> 5] >> (gi & 31)) & 1u; }
 
@@ -254,7 +240,7 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   }
   // (blocks_per_cam, not the grid: a grad-quant grid may hold one CTA more)
   const bool prefetch_ahead = ahead > 0 && blk + ahead < (GQ ? g.blocks_per_cam : (int64_t)gridDim.x);
-  if (!kSkipUnseen && prefetch_ahead && threadIdx.x == 0) {
+  if (prefetch_ahead && threadIdx.x == 0) {
     // the SH block of the CTA that starts about a wave later, into L2
     const int64_t m0 = (blk + ahead) * kBlock;
     prefetch_l2(sh + m0 * K3, (uint32_t)(min64(kBlock, g.N - m0) * K3 * 4));
@@ -332,7 +318,6 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
         else
           buf[r] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      if (kSkipUnseen && prefetch_ahead) prefetch_seen_rows(g, mask, sh, (blk + ahead) * kBlock, K3);
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
         const int v = threadIdx.x + r * kBlock;

@@ -118,10 +118,14 @@ struct AdamArgs {
 };
 
 // One Adam update of parameter p with gradient g; m and v are updated in place.
+// The square root and the quotient come from the hardware's approximate
+// reciprocal square root and divide (a few ulp on the step, far inside the
+// update's tolerance; v >= 0, and v = 0 gives the root 0).
 __device__ __forceinline__ float adam_update(float p, float g, float& m, float& v, float lr, const AdamArgs& a) {
   m = a.b1 * m + (1.0f - a.b1) * g;
   v = a.b2 * v + (1.0f - a.b2) * g * g;
-  return p - lr * (m * a.ibc1) / (sqrtf(v) * a.ibc2s + a.eps);
+  const float root = v > 0.0f ? v * rsqrtf(v) : 0.0f;
+  return p - __fdividef(lr * (m * a.ibc1), root * a.ibc2s + a.eps);
 }
 
 // Block-quantised gradient accumulation ("Spirula Studio backward pass",
@@ -620,8 +624,8 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
         for (int r = 0; r < kChunk; ++r) {
           const int vv = v0 + r * kBlock;
           if (vv < kV) {
-            mb[r] = m4[vv];
-            vb[r] = v4[vv];
+            mb[r] = __ldcs(m4 + vv);
+            vb[r] = __ldcs(v4 + vv);
           }
         }
 #pragma unroll
@@ -636,9 +640,10 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
             pe[u] = adam_update(sh_s[gi * KP + q], gsh_s[gi * KP + q], me[u], ve[u],
                                 q < 3 ? adam.lr_sh_dc : adam.lr_sh_rest, adam);
           }
-          p4[vv] = make_float4(pe[0], pe[1], pe[2], pe[3]);
-          m4[vv] = make_float4(me[0], me[1], me[2], me[3]);
-          v4[vv] = make_float4(ve[0], ve[1], ve[2], ve[3]);
+          // streaming stores: the lines are not read again in this kernel
+          __stcs(p4 + vv, make_float4(pe[0], pe[1], pe[2], pe[3]));
+          __stcs(m4 + vv, make_float4(me[0], me[1], me[2], me[3]));
+          __stcs(v4 + vv, make_float4(ve[0], ve[1], ve[2], ve[3]));
         }
       }
     } else {

@@ -141,8 +141,9 @@ __device__ __forceinline__ uint64_t ld_status(const uint64_t* p) {
   return *reinterpret_cast<const volatile unsigned long long*>(p);
 }
 
+// Keys only: three CTAs per SM (85 registers); with values two.
 template <bool VALS>
-__global__ __launch_bounds__(kSortThreads) void k_onesweep(const uint64_t* __restrict__ kin,
+__global__ __launch_bounds__(kSortThreads, VALS ? 2 : 3) void k_onesweep(const uint64_t* __restrict__ kin,
                                                            const uint32_t* __restrict__ vin,
                                                            uint64_t* __restrict__ kout, uint32_t* __restrict__ vout,
                                                            int64_t n, int shift, uint64_t epoch,

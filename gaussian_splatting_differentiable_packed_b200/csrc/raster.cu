@@ -27,6 +27,10 @@ constexpr int kBatch = 256;
 constexpr int kRedF = 12;
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// sqrt(x) for x >= 0 through the approximate reciprocal square root (a few
+// ulp); only the culling bounds use it, widened far beyond that error.
+__device__ __forceinline__ float sqrt_approx(float x) { return x > 0.0f ? x * rsqrtf(x) : 0.0f; }
 __device__ __forceinline__ float2 f2s(float a) { return make_float2(a, a); }
 
 // Pixel-pair coordinates of this thread: column i, rows j and j+1.
@@ -92,10 +96,12 @@ __device__ __forceinline__ void stage_from(const float4 r0, const float4 r1, con
     bounded = 1.0f;
   } else if (o <= 1.0f && ca > 0.0f && cc > 0.0f && dql > 0.0f) {
     const float L = thr + kCullMargin;
-    hx = sqrtf(2.0f * L * cc / dql) * 1.00001f + 1e-3f;
-    hy = sqrtf(2.0f * L * ca / dql) * 1.00001f + 1e-3f;
+    // bounds only: the hardware's approximate root and divide (relative
+    // error below 1e-6) stay inside the 1e-5 widening
+    hx = sqrt_approx(__fdividef(2.0f * L * cc, dql)) * 1.00001f + 1e-3f;
+    hy = sqrt_approx(__fdividef(2.0f * L * ca, dql)) * 1.00001f + 1e-3f;
     P = 2.0f * L * ca;
-    ica = 1.0f / ca;
+    ica = __fdividef(1.0f, ca);
     cbr = cb * ica;
     bounded = 1.0f;
   }
@@ -324,7 +330,7 @@ __device__ __forceinline__ uint32_t chord_span(const Stage& st, float yc, float 
   const float disc = st.d.z - q + 4e-7f * (st.d.z + q);
   if (disc < 0.0f) return 0u;
   if (!(disc >= 0.0f)) return 0xFFFFu;  // NaN: nothing can be concluded
-  const float hw = sqrtf(disc) * st.e.x * 1.00001f + 2e-3f;
+  const float hw = sqrt_approx(disc) * st.e.x * 1.00001f + 2e-3f;
   const float off = st.e.y * dy;
   const float ctr = st.a.x + off;
   const float m = 1e-5f * (fabsf(st.a.x) + fabsf(off)) + 2e-3f;

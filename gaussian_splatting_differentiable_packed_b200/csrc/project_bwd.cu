@@ -77,9 +77,6 @@ __device__ __forceinline__ void sh_dir_grads(float X, float Y, float Z, const fl
   vdir[2] = gZ;
 }
 
-// Bit gi of the CTA's per-warp visibility words.
-__device__ __forceinline__ bool seen(const uint32_t* s_seen, int gi) { return (s_seen[gi >> 5] >> (gi & 31)) & 1u; }
-
 // Shared-memory stride per Gaussian for SH blocks (odd, so that thread t's
 // word k sits in bank (t*stride + k) mod 32: conflict-free across a warp).
 template <int DEG>
@@ -211,7 +208,6 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   __shared__ uint32_t s_word[kCamChunkB][kWarps];
   __shared__ int64_t s_row0[kCamChunkB][kWarps];
   __shared__ float s_margin[kBlock][3];
-  __shared__ uint32_t s_seen[kWarps];  // per warp: its Gaussians seen by some camera
   // the optimizer updates every parameter and the accumulators are decoded
   // into the SH staging area, so only the plain backward skips unseen rows
   constexpr bool kSkipUnseen = !ADAM && !GQ;
@@ -266,21 +262,11 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     }
   };
   load_chunk(0);
-  if (kSkipUnseen) {
-    // which of the CTA's Gaussians any camera sees: with every camera in the
-    // first chunk, from the words just staged; otherwise every row is read
-    __syncthreads();
-    if (threadIdx.x < kWarps) {
-      uint32_t u = 0;
-      if (g.C <= kCamChunkB) {
-        for (int c = 0; c < g.C; ++c) u |= s_word[c][threadIdx.x];
-      } else {
-        u = 0xFFFFFFFFu;
-      }
-      s_seen[threadIdx.x] = u;
-    }
-    __syncthreads();
-  }
+  __syncthreads();  // the first chunk's words and rows are read by every warp
+  // which of the warp's Gaussians any camera sees: with every camera in the
+  // first chunk, from the words just staged; otherwise every row is read
+  uint32_t seen_w = 0xFFFFFFFFu;
+  if (kSkipUnseen && g.C <= kCamChunkB) seen_w = __reduce_or_sync(0xffffffffu, lane < g.C ? s_word[lane][warp] : 0u);
   if (GQ && !gqa.first && threadIdx.x == 0) {
     // the accumulator codes are read after the camera loop: have L2 fetch
     // the CTA's now
@@ -302,49 +288,52 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     prefetch_l2(adam.v_scales + 3 * n0, (uint32_t)(cnt * 12));
     prefetch_l2(adam.log_scales + 3 * n0, (uint32_t)(cnt * 12));
   }
-  // coalesced staging of the CTA's contiguous SH block: full blocks with all
-  // 16-byte loads in flight at once (the block starts 16-byte aligned: 128*K3
-  // floats per block), the ragged last block word by word.  The plain
-  // backward skips the rows of Gaussians no camera sees: their gradients
-  // are zero and their coefficients are never read (a third of the
-  // Gaussians of the 15M-Gaussian workload)
+  // staging of the warp's 32 rows of the CTA's SH block (contiguous and
+  // 16-byte aligned: 32 * K3 floats a warp) with all 16-byte loads in flight
+  // at once, a ragged warp word by word.  The plain backward skips the rows
+  // of Gaussians no camera sees: their gradients are zero and their
+  // coefficients are never read (a third of the Gaussians of the 15M-Gaussian
+  // workload).  Each warp stages, walks and writes back its own rows, so no
+  // CTA barrier separates them.
+  const int wrows = max(0, min(32, cnt - 32 * warp));  // the warp's valid rows
+  float* const sh_w = sh_s + 32 * warp * KP;
+  float* const gsh_w = gsh_s + 32 * warp * KP;
   {
-    const float* src = sh + n0 * K3;
-    if (cnt == kBlock) {
-      constexpr int kV = kBlock * K3 / 4;
-      constexpr int kPer = (kV + kBlock - 1) / kBlock;
+    const float* src = sh + (n0 + 32 * warp) * K3;
+    if (wrows == 32) {
+      constexpr int kV = 32 * K3 / 4;
+      constexpr int kPer = (kV + 31) / 32;
       float4 buf[kPer];
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
-        const int v = threadIdx.x + r * kBlock;
-        if (v < kV && (!kSkipUnseen || seen(s_seen, (4 * v) / K3) || seen(s_seen, (4 * v + 3) / K3)))
-          buf[r] = reinterpret_cast<const float4*>(src)[v];
-        else
-          buf[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int v = lane + 32 * r;
+        const bool need = v < kV && (!kSkipUnseen || ((seen_w >> ((4 * v) / K3)) & 1u) ||
+                                     ((seen_w >> ((4 * v + 3) / K3)) & 1u));
+        buf[r] = need ? reinterpret_cast<const float4*>(src)[v] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
-        const int v = threadIdx.x + r * kBlock;
+        const int v = lane + 32 * r;
         if (v < kV) {
           const float e[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             int gi, q;
             sh_word<K3>(v, u, gi, q);
-            sh_s[gi * KP + q] = e[u];
-            gsh_s[gi * KP + q] = 0.0f;
+            sh_w[gi * KP + q] = e[u];
+            gsh_w[gi * KP + q] = 0.0f;
           }
         }
       }
     } else {
-      for (int f = threadIdx.x; f < kBlock * K3; f += kBlock) {
+      for (int f = lane; f < 32 * K3; f += 32) {
         const int gi = f / K3, q = f - gi * K3;
-        sh_s[gi * KP + q] = f < cnt * K3 && (!kSkipUnseen || seen(s_seen, gi)) ? src[f] : 0.0f;
-        gsh_s[gi * KP + q] = 0.0f;
+        sh_w[gi * KP + q] = gi < wrows && (!kSkipUnseen || ((seen_w >> gi) & 1u)) ? src[f] : 0.0f;
+        gsh_w[gi * KP + q] = 0.0f;
       }
     }
   }
-  __syncthreads();  // the staged SH block is read below
+  __syncwarp();  // the warp's staged rows are read by its lanes below
   {
     // Bound on how far 0.5 + sum_k sh_k b_k can move with the summation
     // order: each order's rounding is below 17 * 2^-24 * (0.5 + sum_k |sh_k
@@ -373,9 +362,11 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   float gx[GQ ? 11 : 1] = {};  // GQ: this Gaussian's means, quats, scales and opacity gradients
   for (int c0 = 0; c0 < g.C; c0 += kCamChunkB) {
     const int nc = min(kCamChunkB, g.C - c0);
-    __syncthreads();
-    if (c0 > 0) load_chunk(c0);  // the first chunk was loaded before the SH block
-    __syncthreads();
+    if (c0 > 0) {  // the first chunk was loaded (and the CTA synchronised) before the SH block
+      __syncthreads();
+      load_chunk(c0);
+      __syncthreads();
+    }
     if (!valid) continue;
     // each lane walks the cameras of the chunk that see its Gaussian, in
     // camera order, with the next pair's gradient row loaded one pair ahead
@@ -605,7 +596,7 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
       adam.v_opac[n] = v;
     }
   }
-  __syncthreads();
+  if (ADAM || GQ) __syncthreads();  // their epilogues run over the CTA's whole block
   if (ADAM) {
     // the CTA's SH block: Adam on each coefficient (DC with its own rate),
     // the staged values are the parameters.  A full block moves the moments
@@ -778,24 +769,26 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
     }
     return;
   }
-  // coalesced write-back of the CTA's SH gradient block (16-byte stores for a
-  // full block)
-  float* dst = v_sh + n0 * K3;
-  if (cnt == kBlock) {
-    for (int v = threadIdx.x; v < kBlock * K3 / 4; v += kBlock) {
+  // write-back of the warp's own rows of the SH gradient block (16-byte
+  // stores for a full warp; its lanes wrote the rows, so a warp barrier
+  // suffices)
+  __syncwarp();
+  float* dst = v_sh + (n0 + 32 * warp) * K3;
+  if (wrows == 32) {
+    for (int v = lane; v < 32 * K3 / 4; v += 32) {
       float e[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         int gi, q;
         sh_word<K3>(v, u, gi, q);
-        e[u] = gsh_s[gi * KP + q];
+        e[u] = gsh_w[gi * KP + q];
       }
       reinterpret_cast<float4*>(dst)[v] = make_float4(e[0], e[1], e[2], e[3]);
     }
   } else {
-    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+    for (int f = lane; f < wrows * K3; f += 32) {
       const int gi = f / K3, q = f - gi * K3;
-      dst[f] = gsh_s[gi * KP + q];
+      dst[f] = gsh_w[gi * KP + q];
     }
   }
 }

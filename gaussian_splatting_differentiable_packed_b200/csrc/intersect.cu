@@ -42,6 +42,7 @@ constexpr int kIxRows = 4096;  // positions of the depth order per CTA
 constexpr int kIxPer = kIxRows / kIxThreads;
 static_assert(kIxRows % kIxThreads == 0, "rows per thread");
 constexpr int kRowKeyThreads = 256;
+constexpr int kIxCams = 256;  // cameras whose first rows the write kernel keeps in shared memory
 
 // Block status of the look-back: flag in the top two bits, count below.
 constexpr uint64_t kIxAgg = 1ull << 62;
@@ -56,6 +57,7 @@ struct IxSmem {
   uint32_t row[kIxRows];      // row index
   uint16_t w[kIxRows];        // tile columns of the row's range
   uint32_t wsum[kIxThreads / 32];
+  int64_t cam_row0[kIxCams];  // first row of each camera
   int64_t base;
   uint32_t blk;
 };
@@ -128,12 +130,15 @@ __global__ __launch_bounds__(kRowKeyThreads) void k_row_keys(Geo g, const float*
   }
 }
 
-__device__ __forceinline__ int camera_of_row(const int64_t* __restrict__ block_off, int64_t blocks_per_cam, int C,
-                                             int64_t r) {
-  int lo = 0, hi = C;  // camera c starts at row block_off[c * blocks_per_cam]
+// Camera of row r: camera c's rows start at block_off[c * blocks_per_cam];
+// cam_row0 holds those starts in shared memory for the first kIxCams cameras.
+__device__ __forceinline__ int camera_of_row(const int64_t* __restrict__ block_off, const int64_t* cam_row0,
+                                             int64_t blocks_per_cam, int C, int64_t r) {
+  int lo = 0, hi = C;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (block_off[(int64_t)mid * blocks_per_cam] <= r) lo = mid; else hi = mid;
+    const int64_t start = mid < kIxCams ? cam_row0[mid] : block_off[(int64_t)mid * blocks_per_cam];
+    if (start <= r) lo = mid; else hi = mid;
   }
   return lo;
 }
@@ -156,6 +161,7 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
   // blocks by ticket: every block this one looks back on belongs to a CTA
   // that is already running
   if (tid == 0) S.blk = atomicAdd(ticket, 1u);
+  for (int c = tid; c < min(g.C, kIxCams); c += kIxThreads) S.cam_row0[c] = block_off[(int64_t)c * g.blocks_per_cam];
   __syncthreads();
   const int64_t blk = S.blk;
   const int64_t p0 = blk * kIxRows;
@@ -171,7 +177,7 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
       const uint32_t r = (uint32_t)key;
       int tx0, ty0, w;
       cnt = row_tiles(g, reinterpret_cast<const uint2*>(aabb16)[r], tx0, ty0, w);
-      const int c = camera_of_row(block_off, g.blocks_per_cam, g.C, (int64_t)r);
+      const int c = camera_of_row(block_off, S.cam_row0, g.blocks_per_cam, g.C, (int64_t)r);
       S.t0[i] = (uint32_t)((uint64_t)c * (uint64_t)g.tiles_per_cam + (uint64_t)ty0 * g.tiles_x + (uint64_t)tx0);
       S.w[i] = (uint16_t)w;
       S.dep[i] = (uint32_t)(key >> 32);

@@ -248,9 +248,17 @@ __device__ __forceinline__ uint32_t q16_ceil(float v, int extent) {
 
 // Tile range [t0, t1) of a decoded 16-bit edge pair (integers only).
 __device__ __forceinline__ void tile_span(uint32_t q0, uint32_t q1, int extent, int ntiles, int& t0, int& t1) {
-  const int64_t den = 65535LL * 16;
-  int64_t a = ((int64_t)q0 * extent) / den;
-  int64_t b = ((int64_t)q1 * extent + den - 1) / den;
+  constexpr uint32_t kDen = 65535u * 16u;
+  int64_t a, b;
+  if (extent <= 65535) {
+    // q * extent < 2^32: the same quotients in 32-bit arithmetic
+    const uint32_t x0 = q0 * (uint32_t)extent, x1 = q1 * (uint32_t)extent;
+    a = x0 / kDen;
+    b = x1 / kDen + (x1 % kDen != 0u ? 1 : 0);
+  } else {
+    a = ((int64_t)q0 * extent) / kDen;
+    b = ((int64_t)q1 * extent + kDen - 1) / kDen;
+  }
   t0 = (int)min64(max64(a, 0), ntiles);
   t1 = (int)min64(max64(b, 0), ntiles);
 }

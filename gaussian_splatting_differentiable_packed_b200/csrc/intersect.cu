@@ -23,10 +23,11 @@
 //                   block's total and looks back over earlier blocks for its
 //                   base (decoupled look-back, bounded spin), writes the
 //                   rows' offsets to isect_off, then expands the block's
-//                   slots: slot s belongs to the last row whose offset is
-//                   <= s (binary search in shared memory), and consecutive
-//                   threads write consecutive slots, so every store is
-//                   coalesced whatever the per-row counts.
+//                   slots 8192 at a time: slot s belongs to the last row
+//                   whose offset is <= s (a binary search in shared memory
+//                   between the rows of its 64-slot cell, found first), and
+//                   consecutive threads write consecutive slots, so every
+//                   store is coalesced whatever the per-row counts.
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 
@@ -43,6 +44,8 @@ constexpr int kIxPer = kIxRows / kIxThreads;
 static_assert(kIxRows % kIxThreads == 0, "rows per thread");
 constexpr int kRowKeyThreads = 256;
 constexpr int kIxCams = 256;  // cameras whose first rows the write kernel keeps in shared memory
+constexpr int kIxChunk = 8192;  // slots expanded per round of the write kernel
+constexpr int kIxCell = 64;     // slots per search cell
 
 // Block status of the look-back: flag in the top two bits, count below.
 constexpr uint64_t kIxAgg = 1ull << 62;
@@ -58,6 +61,7 @@ struct IxSmem {
   uint16_t w[kIxRows];        // tile columns of the row's range
   uint32_t wsum[kIxThreads / 32];
   int64_t cam_row0[kIxCams];  // first row of each camera
+  uint32_t cell[kIxChunk / kIxCell + 1];  // row of every kIxCell-th slot of the chunk
   int64_t base;
   uint32_t blk;
 };
@@ -263,25 +267,44 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
   const int64_t base = S.base;
   for (int i = tid; i < nr; i += kIxThreads) isect_off[p0 + i] = base + (int64_t)S.off[i];
   if (tid == 0 && p0 + nr == nnz) isect_off[nnz] = base + (int64_t)total;  // the last block: the total
-  // expand the block's slots; positions past nr have offset == total and are
-  // never found for s < total
+  // expand the block's slots, kIxChunk at a time.  A slot's row is the last
+  // row whose offset is <= the slot; every kIxCell-th slot of the chunk has
+  // its row found first (one binary search per cell over the whole block),
+  // so a slot searches only between its cell's bounding rows (about 29 rows
+  // on the 15M-Gaussian workload, one or two on the 7680^2 one).  Positions
+  // past nr have offset == total and are never found for s < total.
   const uint32_t stop = (uint32_t)max64(0, min64((int64_t)total, limit - base));
-  for (uint32_t s = tid; s < stop; s += kIxThreads) {
-    int lo = 0, hi = nr;  // largest i with S.off[i] <= s
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (S.off[mid] <= s) lo = mid; else hi = mid;
+  for (uint32_t c0 = 0; c0 < stop; c0 += kIxChunk) {
+    __syncthreads();  // the previous chunk's cells are read no more
+    for (int j = tid; j <= kIxChunk / kIxCell; j += kIxThreads) {
+      const uint32_t sc = min(c0 + (uint32_t)(j * kIxCell), total - 1u);
+      int lo = 0, hi = nr;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (S.off[mid] <= sc) lo = mid; else hi = mid;
+      }
+      S.cell[j] = (uint32_t)lo;
     }
-    const uint32_t k = s - S.off[lo], w = S.w[lo];
-    // k / w through the approximate reciprocal: k < 2^24, so the estimate is
-    // off by at most one, and one correction each way makes it exact
-    uint32_t ty = (uint32_t)__fmul_rz((float)k, __frcp_rn((float)w));
-    if (ty * w > k) --ty;
-    if ((ty + 1) * w <= k) ++ty;
-    const uint32_t tx = k - ty * w;
-    const uint64_t tile = (uint64_t)S.t0[lo] + (uint64_t)ty * (uint64_t)g.tiles_x + tx;
-    keys[base + s] = (tile << 32) | S.dep[lo];
-    vals[base + s] = S.row[lo];
+    __syncthreads();
+    const uint32_t c1 = min(stop, c0 + (uint32_t)kIxChunk);
+    for (uint32_t s = c0 + tid; s < c1; s += kIxThreads) {
+      const int j = (int)((s - c0) / kIxCell);
+      int lo = (int)S.cell[j], hi = (int)S.cell[j + 1];  // the row is in [lo, hi]
+      while (hi > lo) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (S.off[mid] <= s) lo = mid; else hi = mid - 1;
+      }
+      const uint32_t k = s - S.off[lo], w = S.w[lo];
+      // k / w through the approximate reciprocal: k < 2^24, so the estimate is
+      // off by at most one, and one correction each way makes it exact
+      uint32_t ty = (uint32_t)__fmul_rz((float)k, __frcp_rn((float)w));
+      if (ty * w > k) --ty;
+      if ((ty + 1) * w <= k) ++ty;
+      const uint32_t tx = k - ty * w;
+      const uint64_t tile = (uint64_t)S.t0[lo] + (uint64_t)ty * (uint64_t)g.tiles_x + tx;
+      keys[base + s] = (tile << 32) | S.dep[lo];
+      vals[base + s] = S.row[lo];
+    }
   }
 }
 

@@ -217,7 +217,7 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     Proj P;
     cam_point(k, gi.mx, gi.my, gi.mz, P.px, P.py, P.pz);
     project_rest(k, gi.S, g.W, g.H, P);
-    const float idet = div_(1.0f, P.det);
+    const float idet = rcp_(P.det);
     const float ca = mul(P.c, idet), cb = -mul(P.b, idet), cc2 = mul(P.a, idet);
     float b[16];
     float X = 0.0f, Y = 0.0f, Z = 0.0f, il;

@@ -399,7 +399,7 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
       const float* R = k.R;
       float px, py, pz;
       cam_point(k, mx, my, mz, px, py, pz);
-      const float izc = div_(1.0f, pz);
+      const float izc = rcp_(pz);
       const float u = mul(px, izc), v = mul(py, izc);
       const bool clx = (u < -k.limx) || (u > k.limx);
       const bool cly = (v < -k.limy) || (v > k.limy);

@@ -19,12 +19,17 @@ __device__ __forceinline__ float mul(float a, float b) { return __fmul_rn(a, b);
 __device__ __forceinline__ float add(float a, float b) { return __fadd_rn(a, b); }
 __device__ __forceinline__ float sub(float a, float b) { return __fsub_rn(a, b); }
 __device__ __forceinline__ float div_(float a, float b) { return __fdiv_rn(a, b); }
+// 1/b correctly rounded: the same value as div_(1.0f, b) (both are the exact
+// quotient rounded to nearest even), through the reciprocal intrinsic.
+__device__ __forceinline__ float rcp_(float b) { return __frcp_rn(b); }
 __device__ __forceinline__ float sqrt_(float a) { return __fsqrt_rn(a); }
 __device__ __forceinline__ float fma_(float a, float b, float c) { return __fmaf_rn(a, b, c); }
 
 // Camera constants, computed per camera (identical wherever computed).
-struct Cam {
-  float R[9], t[3], fx, fy, cx, cy, limx, limy, cpos[3];
+// 16-byte aligned and padded to six 16-byte words, so that a warp's read of
+// a camera from shared memory can use 16-byte loads.
+struct __align__(16) Cam {
+  float R[9], t[3], fx, fy, cx, cy, limx, limy, cpos[3], pad[3];
 };
 
 __device__ __forceinline__ Cam load_cam(const float* c20, int W, int H) {
@@ -57,7 +62,7 @@ struct QuatRot {
 __device__ __forceinline__ QuatRot quat_rot(float qw, float qx, float qy, float qz) {
   QuatRot o;
   float n2 = add(add(add(mul(qw, qw), mul(qx, qx)), mul(qy, qy)), mul(qz, qz));
-  o.inv = div_(1.0f, sqrt_(n2));
+  o.inv = rcp_(sqrt_(n2));
   float w = mul(qw, o.inv), x = mul(qx, o.inv), y = mul(qy, o.inv), z = mul(qz, o.inv);
   o.w = w; o.x = x; o.y = y; o.z = z;
   float xx = mul(x, x), yy = mul(y, y), zz = mul(z, z);
@@ -113,7 +118,7 @@ __device__ __forceinline__ void cam_point(const Cam& k, float mx, float my, floa
 // Full EWA projection after the depth test passed.  vis covers det > 0 and the
 // image-overlap test; the caller has checked near < z < far.
 __device__ __forceinline__ void project_rest(const Cam& k, const Cov3& S, int W, int H, Proj& o) {
-  float iz = div_(1.0f, o.pz);
+  float iz = rcp_(o.pz);
   o.u = mul(o.px, iz);
   o.v = mul(o.py, iz);
   o.ux = fminf(fmaxf(o.u, -k.limx), k.limx);
@@ -193,7 +198,7 @@ __device__ __forceinline__ void view_dir(const Cam& k, float mx, float my, float
                                          float& il) {
   float d0 = sub(mx, k.cpos[0]), d1 = sub(my, k.cpos[1]), d2 = sub(mz, k.cpos[2]);
   float l2 = add(add(mul(d0, d0), mul(d1, d1)), mul(d2, d2));
-  il = div_(1.0f, sqrt_(l2));
+  il = rcp_(sqrt_(l2));
   X = mul(d0, il); Y = mul(d1, il); Z = mul(d2, il);
 }
 

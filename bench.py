@@ -530,7 +530,7 @@ def cpu_baseline(config: int, n_sample: int, repeats: int = 1):
         isects += r["isect"]["n_isects"]
     dt = time.perf_counter() - t
     return dict(value=isects / dt, unit="isects/s", cores=cores, kind="oracle",
-                sample=f"the workload's distributions and cameras ({sc.name}) with N={n_sample} Gaussians "
+                sample=f"the workload's distributions and cameras ({sc.name}) with N={sc.N} Gaussians "
                        f"({r['isect']['n_isects']} intersections, full image size), {repeats} step(s) "
                        f"in {dt:.1f} s")
 

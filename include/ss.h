@@ -165,7 +165,9 @@ ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float*
  * of the rows in that order.  block_off, aabb16 and row_depth are the arrays
  * ss_project_packed wrote (block_off gives each camera's first row).  temp:
  * ss_workspace_bytes(SS_WS_INTERSECT, nnz) bytes (it holds the depth order
- * of the rows).
+ * of the rows).  The call synchronises the stream once more after the write
+ * and returns SS_ERR_DEVICE_CHECK if a bounded look-back wait (the depth
+ * sort's or the write's offsets) ran out.
  */
 ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_depth, const uint32_t* aabb16,
                              const int64_t* block_off, int64_t nnz, int64_t* isect_off, uint64_t* keys,

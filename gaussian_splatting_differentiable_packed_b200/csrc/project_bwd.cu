@@ -248,17 +248,20 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
   // The camera chunk of the first cameras: each warp's mask word and first
   // row per camera (loaded before the SH block, so the plain backward knows
   // which Gaussians some camera sees; later chunks are loaded in the loop).
+  // Every warp loads its own words and first rows (lane cc: camera c0 + cc,
+  // the CTA's four mask words of that camera in one 16-byte load, so a
+  // warp's rows need no chain of loads); warp 0 also loads the cameras.
+  static_assert(kWarps == 4, "one 16-byte load holds a CTA's mask words of a camera");
   auto load_chunk = [&](int c0) {
     const int nc = min(kCamChunkB, g.C - c0);
     if (threadIdx.x < nc) scam[threadIdx.x] = load_cam(cams + 20 * (int64_t)(c0 + threadIdx.x), g.W, g.H);
-    if (threadIdx.x < nc * kWarps) {
-      const int cc = threadIdx.x / kWarps, w = threadIdx.x % kWarps;
-      const int64_t c = c0 + cc;
-      const int64_t wbase = (c * g.n_pad + blk * kBlock) / 32;
-      int64_t row = block_off[c * g.blocks_per_cam + blk];
-      for (int w2 = 0; w2 < w; ++w2) row += __popc(mask[wbase + w2]);
-      s_word[cc][w] = mask[wbase + w];
-      s_row0[cc][w] = row;
+    if (lane < nc) {
+      const int64_t c = c0 + lane;
+      const uint4 wv = reinterpret_cast<const uint4*>(mask)[(c * g.n_pad + blk * kBlock) / 128];
+      const int64_t row = block_off[c * g.blocks_per_cam + blk] + (warp > 0 ? __popc(wv.x) : 0) +
+                          (warp > 1 ? __popc(wv.y) : 0) + (warp > 2 ? __popc(wv.z) : 0);
+      s_word[lane][warp] = warp == 0 ? wv.x : warp == 1 ? wv.y : warp == 2 ? wv.z : wv.w;
+      s_row0[lane][warp] = row;
     }
   };
   load_chunk(0);
@@ -861,9 +864,9 @@ extern "C" ss_status ss_project_bwd(const ss_dims* dims, const float* cams, cons
   if (g.N == 0) return SS_OK;
   if (!cams || !means || !quats || !scales || !sh || !mask || !block_off || !v_screen) return invalid("null input");
   if (!v_means || !v_quats || !v_scales || !v_opacities || !v_sh) return invalid("null output");
-  if (((uintptr_t)quats & 15) || ((uintptr_t)v_quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15) ||
-      ((uintptr_t)v_sh & 15))
-    return invalid("quats, v_quats, v_screen, sh and v_sh must be 16-byte aligned");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)mask & 15) || ((uintptr_t)v_quats & 15) ||
+      ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15) || ((uintptr_t)v_sh & 15))
+    return invalid("quats, mask, v_quats, v_screen, sh and v_sh must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
   return dispatch_pbwd<false, false>(g, st, cams, means, quats, scales, sh, mask, block_off, v_screen, v_means,
                                      v_quats, v_scales, v_opacities, v_sh, opacities, AdamArgs{});
@@ -885,9 +888,9 @@ extern "C" ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams,
   if (!S.m_means || !S.v_means || !S.m_quats || !S.v_quats || !S.m_scales || !S.v_scales || !S.m_opacities ||
       !S.v_opacities || !S.m_sh || !S.v_sh)
     return invalid("null optimizer state");
-  if (((uintptr_t)quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15) || ((uintptr_t)S.m_sh & 15) ||
-      ((uintptr_t)S.v_sh & 15))
-    return invalid("quats, v_screen, sh and the SH moments must be 16-byte aligned");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)mask & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15) ||
+      ((uintptr_t)S.m_sh & 15) || ((uintptr_t)S.v_sh & 15))
+    return invalid("quats, mask, v_screen, sh and the SH moments must be 16-byte aligned");
   if (hp->step < 1) return invalid("adam step must be >= 1");
   AdamArgs a{};
   a.m_means = S.m_means; a.v_means = S.v_means; a.m_quats = S.m_quats; a.v_quats = S.v_quats;
@@ -916,8 +919,8 @@ extern "C" ss_status ss_project_bwd_gq(const ss_dims* dims, const float* cams, c
   if (!acc || !acc->means || !acc->quats || !acc->scales || !acc->opacities || !acc->sh_dc || !acc->block_scale ||
       (g.deg > 0 && !acc->sh_rest))
     return invalid("null accumulator");
-  if (((uintptr_t)quats & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15))
-    return invalid("quats, v_screen and sh must be 16-byte aligned");
+  if (((uintptr_t)quats & 15) || ((uintptr_t)mask & 15) || ((uintptr_t)v_screen & 15) || ((uintptr_t)sh & 15))
+    return invalid("quats, mask, v_screen and sh must be 16-byte aligned");
   if (((uintptr_t)acc->sh_dc & 15) || ((uintptr_t)acc->sh_rest & 15))
     return invalid("the SH code arrays must be 16-byte aligned");
   GqArgs q{};

@@ -207,8 +207,8 @@ ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a
  * copies scales = exp(log_scales) and opacities = sigmoid(logit_opacities)
  * that the forward reads (scales and opacities are read first as the
  * activated values the forward used).  All arrays are device memory laid out
- * like the parameters; state and hp are host structs.  quats, v_screen, sh
- * and the SH moments must be 16-byte aligned; hp->step >= 1.
+ * like the parameters; state and hp are host structs.  quats, mask, v_screen,
+ * sh and the SH moments must be 16-byte aligned; hp->step >= 1.
  */
 typedef struct ss_adam {
   float lr_means, lr_quats, lr_scales, lr_opacities, lr_sh_dc, lr_sh_rest;
@@ -246,7 +246,7 @@ ss_status ss_project_bwd_adam(const ss_dims* dims, const float* cams, float* mea
  *   (SH coefficient 0), sh_rest [N][K-1][3] (NULL allowed when K == 1) as
  *   int16; block_scale [6][ceil(N/256)] float in that attribute order.
  * 118 B per Gaussian at SH degree 3 against 236 for the fp32 gradients.
- * quats, v_screen, sh, sh_dc and sh_rest must be 16-byte aligned
+ * quats, mask, v_screen, sh, sh_dc and sh_rest must be 16-byte aligned
  * (SS_ERR_INVALID_ARG otherwise).  Two CTAs of 128 Gaussians form one block; they run as a
  * thread-block cluster of two and exchange their maxima through distributed
  * shared memory.
@@ -361,7 +361,7 @@ ss_status ss_rasterize_bwd(const ss_dims* dims, const float* screen, const uint3
  * taken back through the conic, the EWA Jacobian, the camera transform, the
  * covariance and the SH colour.  Deterministic (one thread per Gaussian, no
  * atomics).  Writes every element of the five outputs (zero where invisible).
- * quats, v_quats, v_screen, sh and v_sh must be 16-byte aligned
+ * quats, mask, v_quats, v_screen, sh and v_sh must be 16-byte aligned
  * (SS_ERR_INVALID_ARG otherwise).
  */
 ss_status ss_project_bwd(const ss_dims* dims, const float* cams, const float* means, const float* quats,

@@ -95,9 +95,6 @@ __host__ __device__ constexpr int rows_sh_stride() {
   return (K3 % 2 == 0) ? K3 + 1 : K3;
 }
 
-// Bit gi of the CTA's per-warp visibility words.
-__device__ __forceinline__ bool seen(const uint32_t* s_seen, int gi) { return (s_seen[gi >> 5] >> (gi & 31)) & 1u; }
-
 // A visible (camera, Gaussian) pair waiting in the CTA's work queue.
 struct RowItem {
   int64_t row;
@@ -136,7 +133,6 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   __shared__ uint32_t s_word[kSlots];  // [camera][warp]
   __shared__ int s_pre[kSlots + 1];    // exclusive prefix of the words' popcounts
   __shared__ int64_t s_row0[kCamChunk];
-  __shared__ uint32_t s_seen[kWarps];  // per warp: its Gaussians seen by some camera
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t blk = blockIdx.x;
   const int64_t n0 = blk * kBlock;
@@ -173,43 +169,64 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
     s_g[threadIdx.x] = load_gauss(means, quats, scales, n);
     s_o[threadIdx.x] = opacities[n];
   }
-  // which of the CTA's Gaussians any camera sees: only their SH rows are
-  // staged (a third of the Gaussians of the 15M-Gaussian workload are seen
-  // by no camera).  With every camera in the first chunk the words are the
-  // ones just staged; otherwise every row is staged.
-  __syncthreads();
-  if (threadIdx.x < kWarps) {
-    uint32_t u = 0;
-    if (g.C <= kCamChunk) {
-      for (int c = 0; c < g.C; ++c) u |= s_word[c * kWarps + threadIdx.x];
-    } else {
-      u = 0xFFFFFFFFu;
+  // exclusive prefix of the chunk's ns <= 128 slot popcounts into s_pre,
+  // 4 consecutive slots a lane (one warp)
+  auto chunk_prefix = [&](int ns) {
+    int v[4], sum = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sl = 4 * lane + u;
+      v[u] = sl < ns ? __popc(s_word[sl]) : 0;
+      sum += v[u];
     }
-    s_seen[threadIdx.x] = u;
-  }
-  __syncthreads();
-  // the CTA's contiguous SH block (16-byte aligned: 128 * K3 floats a block)
-  // into its padded shared layout by asynchronous copies: all in flight
-  // together and no register staging (which would cap the CTAs per SM);
-  // consecutive threads copy consecutive 16-byte (or 4-byte) words
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += x;
+    }
+    int run = inc - sum;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sl = 4 * lane + u;
+      if (sl < ns) s_pre[sl] = run;
+      run += v[u];
+    }
+    if (lane == 31) s_pre[ns] = inc;  // the chunk's total
+  };
+  __syncthreads();  // the first chunk's cameras, rows and words
+  // Each warp copies the SH rows of its own 32 Gaussians that some camera
+  // sees (a third of the Gaussians of the 15M-Gaussian workload are seen by
+  // none; with every camera in the first chunk the words just staged tell,
+  // otherwise every row is copied) into the padded shared layout by
+  // asynchronous copies: all in flight together, no register staging
+  // (which would cap the CTAs per SM), consecutive lanes on consecutive
+  // 16-byte (or 4-byte) words.  Warp 0 meanwhile scans the first chunk.
   {
-    const float* src = sh + n0 * K3;
+    const uint32_t seen_w =
+        g.C <= kCamChunk ? __reduce_or_sync(0xffffffffu, lane < g.C ? s_word[lane * kWarps + warp] : 0u)
+                         : 0xFFFFFFFFu;
+    const int wrows = max(0, min(32, cnt - 32 * warp));
+    const float* src = sh + (n0 + 32 * warp) * K3;
+    float* dst = sh_s + 32 * warp * KP;
     if constexpr (rows_sh_vec<DEG>()) {
       constexpr int Q = K3 / 4;  // 16-byte words a row
 #pragma unroll 4
-      for (int v = threadIdx.x; v < cnt * Q; v += kBlock) {
+      for (int v = lane; v < wrows * Q; v += 32) {
         const int gi = v / Q, qq = v - gi * Q;
-        if (seen(s_seen, gi)) cp_async16(&sh_s[gi * KP + 4 * qq], src + 4 * v);
+        if ((seen_w >> gi) & 1u) cp_async16(&dst[gi * KP + 4 * qq], src + 4 * v);
       }
     } else {
 #pragma unroll 8
-      for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+      for (int f = lane; f < wrows * K3; f += 32) {
         const int gi = f / K3, qq = f - gi * K3;
-        if (seen(s_seen, gi)) cp_async4(&sh_s[gi * KP + qq], src + f);
+        if ((seen_w >> gi) & 1u) cp_async4(&dst[gi * KP + qq], src + f);
       }
     }
+    if (warp == 0) chunk_prefix(min(kCamChunk, g.C) * kWarps);
     cp_async_wait_all();
   }
+  __syncthreads();  // every warp's rows, the parameters and the first chunk's prefix
   auto process = [&](const RowItem& it) {
     const Cam& k = scam[it.cam];
     const GaussIn& gi = s_g[it.g];
@@ -265,36 +282,13 @@ __global__ __launch_bounds__(kBlock) void k_project_rows(Geo g, const float* __r
   for (int c0 = 0; c0 < g.C; c0 += kCamChunk) {
     const int nc = min(kCamChunk, g.C - c0);
     const int ns = nc * kWarps;
-    if (c0 > 0) {  // the first chunk was loaded before the parameters
+    if (c0 > 0) {  // the first chunk was loaded and scanned above
       __syncthreads();
       load_chunk(c0);
+      __syncthreads();
+      if (warp == 0) chunk_prefix(ns);
+      __syncthreads();
     }
-    __syncthreads();
-    if (warp == 0) {
-      // exclusive prefix over the ns <= 128 slots, 4 consecutive slots a lane
-      int v[4], sum = 0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int sl = 4 * lane + u;
-        v[u] = sl < ns ? __popc(s_word[sl]) : 0;
-        sum += v[u];
-      }
-      int inc = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += x;
-      }
-      int run = inc - sum;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int sl = 4 * lane + u;
-        if (sl < ns) s_pre[sl] = run;
-        run += v[u];
-      }
-      if (lane == 31) s_pre[ns] = inc;  // the chunk's total
-    }
-    __syncthreads();
     const int total = s_pre[ns];
     for (int i = threadIdx.x; i < total; i += kBlock) {
       int lo = 0, hi = ns;  // largest slot j with s_pre[j] <= i

@@ -279,8 +279,8 @@ ss_status ss_project_bwd_gq(const ss_dims* dims, const float* cams, const float*
  * (the whole 4096-key tiles of look-back state that fit in the 24 MiB after
  * a fixed header); a larger n returns SS_ERR_INVALID_ARG before any device work.  The
  * first call on a device (and context) looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call shares the one array (cleared at the
+ * (cudaGetSymbolAddress) with that device current and keeps it for later
+ * calls in that context.  Every call shares the one array (cleared at the
  * start of each call), so calls that overlap on the GPU race with each other:
  * serialise them, e.g. on one stream.  Like ss_sort_isects, the call
  * synchronises the stream at the end to read the sort's device-side check

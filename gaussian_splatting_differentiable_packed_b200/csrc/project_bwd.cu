@@ -675,52 +675,57 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
         }
     }
     // the block's SH codes: DC [128][3] and higher [128][K3-3] int16, each
-    // contiguous and 16-byte aligned for a full block; decoded into the SH
-    // staging area (the coefficients are not needed after the camera walk)
-    // with every 16-byte load in flight, word by word for the ragged block
+    // contiguous and 16-byte aligned for a full block.  A full block copies
+    // them as they are into shared memory (the SH staging area: the
+    // coefficients are not needed after the camera walk) with every 16-byte
+    // load in flight, and each thread then adds its own Gaussian's row, so no
+    // code needs an index division; the ragged block goes word by word.
     constexpr int kDcV = kBlock * 3 * 2 / 16;
     constexpr int kRestV = kBlock * (K3 - 3) * 2 / 16;
     constexpr int kPerV = (kDcV + kRestV + kBlock - 1) / kBlock;
+    constexpr int kDcN = kBlock * 3;
     const bool vec = cnt == kBlock;
-    if (!gqa.first && vec) {
-      const int4* dc4 = reinterpret_cast<const int4*>(gqa.code[4] + 3 * n0);
-      const int4* rest4 = reinterpret_cast<const int4*>(gqa.code[5] + (K3 - 3) * n0);
-      int4 buf[kPerV];
-#pragma unroll
-      for (int r = 0; r < kPerV; ++r) {
-        const int v = threadIdx.x + r * kBlock;
-        if (v < kDcV) buf[r] = dc4[v];
-        else if (v < kDcV + kRestV) buf[r] = rest4[v - kDcV];
-      }
-#pragma unroll
-      for (int r = 0; r < kPerV; ++r) {
-        const int v = threadIdx.x + r * kBlock;
-        if (v >= kDcV + kRestV) continue;
-        const uint32_t w[4] = {(uint32_t)buf[r].x, (uint32_t)buf[r].y, (uint32_t)buf[r].z, (uint32_t)buf[r].w};
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float c = (float)(int16_t)(w[u >> 1] >> (16 * (u & 1)));
-          if (v < kDcV) {
-            const int e = 8 * v + u, gi = e / 3;
-            sh_s[gi * KP + (e - 3 * gi)] = c * old[4];
-          } else {
-            const int e = 8 * (v - kDcV) + u, gi = e / (K3 - 3 > 0 ? K3 - 3 : 1);
-            sh_s[gi * KP + 3 + (e - (K3 - 3) * gi)] = c * old[5];
-          }
-        }
-      }
-      __syncthreads();
-    }
-    for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
-      const int gi = f / K3, q = f - gi * K3;
-      const int64_t m = n0 + gi;
-      float x = gsh_s[gi * KP + q];
+    int16_t* code_s = reinterpret_cast<int16_t*>(sh_s);  // DC [kBlock][3], then higher [kBlock][K3 - 3]
+    if (vec) {
       if (!gqa.first) {
-        if (vec) x += sh_s[gi * KP + q];
-        else x += q < 3 ? (float)gqa.code[4][3 * m + q] * old[4] : (float)gqa.code[5][(K3 - 3) * m + (q - 3)] * old[5];
+        const int4* dc4 = reinterpret_cast<const int4*>(gqa.code[4] + 3 * n0);
+        const int4* rest4 = reinterpret_cast<const int4*>(gqa.code[5] + (K3 - 3) * n0);
+        int4* cs4 = reinterpret_cast<int4*>(code_s);
+        int4 buf[kPerV];
+#pragma unroll
+        for (int r = 0; r < kPerV; ++r) {
+          const int v = threadIdx.x + r * kBlock;
+          if (v < kDcV) buf[r] = dc4[v];
+          else if (v < kDcV + kRestV) buf[r] = rest4[v - kDcV];
+        }
+#pragma unroll
+        for (int r = 0; r < kPerV; ++r) {
+          const int v = threadIdx.x + r * kBlock;
+          if (v < kDcV + kRestV) cs4[v] = buf[r];
+        }
+        __syncthreads();
       }
-      gsh_s[gi * KP + q] = x;
-      if (q < 3) vmax[4] = fmaxf(vmax[4], fabsf(x)); else vmax[5] = fmaxf(vmax[5], fabsf(x));
+      float* gr = gsh_s + threadIdx.x * KP;
+#pragma unroll
+      for (int q = 0; q < K3; ++q) {
+        float x = gr[q];
+        if (!gqa.first) {
+          const int16_t c = q < 3 ? code_s[3 * threadIdx.x + q] : code_s[kDcN + (K3 - 3) * threadIdx.x + (q - 3)];
+          x = __fadd_rn(x, __fmul_rn((float)c, q < 3 ? old[4] : old[5]));
+        }
+        gr[q] = x;
+        if (q < 3) vmax[4] = fmaxf(vmax[4], fabsf(x)); else vmax[5] = fmaxf(vmax[5], fabsf(x));
+      }
+    } else {
+      for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {
+        const int gi = f / K3, q = f - gi * K3;
+        const int64_t m = n0 + gi;
+        float x = gsh_s[gi * KP + q];
+        if (!gqa.first)
+          x += q < 3 ? (float)gqa.code[4][3 * m + q] * old[4] : (float)gqa.code[5][(K3 - 3) * m + (q - 3)] * old[5];
+        gsh_s[gi * KP + q] = x;
+        if (q < 3) vmax[4] = fmaxf(vmax[4], fabsf(x)); else vmax[5] = fmaxf(vmax[5], fabsf(x));
+      }
     }
     gq_cta_max(vmax, s_gq_wmax, s_gq_amax);
     float scale[kGqAttr], iscale[kGqAttr];
@@ -734,25 +739,20 @@ __global__ __launch_bounds__(kBlock, 4) void k_project_bwd(Geo g, const float* _
         for (int i = 0; i < kW[a]; ++i) gqa.code[a][kW[a] * n + i] = gq_code(gx[kOff[a] + i], iscale[a]);
     }
     if (vec) {
+      // each thread quantises its own row into the shared code layout, then
       // 16-byte stores of eight codes each, the same vectors as the loads
+      const float* gr = gsh_s + threadIdx.x * KP;
+#pragma unroll
+      for (int q = 0; q < K3; ++q) {
+        const int16_t c = gq_code(gr[q], q < 3 ? iscale[4] : iscale[5]);
+        if (q < 3) code_s[3 * threadIdx.x + q] = c; else code_s[kDcN + (K3 - 3) * threadIdx.x + (q - 3)] = c;
+      }
+      __syncthreads();
       int4* dc4 = reinterpret_cast<int4*>(gqa.code[4] + 3 * n0);
       int4* rest4 = reinterpret_cast<int4*>(gqa.code[5] + (K3 - 3) * n0);
+      const int4* cs4 = reinterpret_cast<const int4*>(code_s);
       for (int v = threadIdx.x; v < kDcV + kRestV; v += kBlock) {
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          int16_t c;
-          if (v < kDcV) {
-            const int e = 8 * v + u, gi = e / 3;
-            c = gq_code(gsh_s[gi * KP + (e - 3 * gi)], iscale[4]);
-          } else {
-            const int e = 8 * (v - kDcV) + u, gi = e / (K3 - 3 > 0 ? K3 - 3 : 1);
-            c = gq_code(gsh_s[gi * KP + 3 + (e - (K3 - 3) * gi)], iscale[5]);
-          }
-          w[u >> 1] |= (uint32_t)(uint16_t)c << (16 * (u & 1));
-        }
-        const int4 o = make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
-        if (v < kDcV) dc4[v] = o; else rest4[v - kDcV] = o;
+        if (v < kDcV) dc4[v] = cs4[v]; else rest4[v - kDcV] = cs4[v];
       }
     } else {
       for (int f = threadIdx.x; f < cnt * K3; f += kBlock) {

@@ -35,7 +35,8 @@ namespace ss {
 
 size_t sort_temp_bytes(int64_t n);
 ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
-                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b);
+                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b, int64_t* tile_off,
+                           int64_t ntiles, bool* ranged);
 ss_status radix_sort_flag(const void* temp, cudaStream_t st, bool* flagged);
 
 constexpr int kIxThreads = 512;
@@ -342,7 +343,7 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   // the rows in depth order (ties by row index: the sort is stable and the
   // row index is the key's low word)
   bool in_b = false;
-  s = radix_sort_pairs(t.dk_a, nullptr, t.dk_b, nullptr, nnz, 0, 4, t.sort, st, &in_b);
+  s = radix_sort_pairs(t.dk_a, nullptr, t.dk_b, nullptr, nnz, 0, 4, t.sort, st, &in_b, nullptr, 0, nullptr);
   if (s) return s;
   const uint64_t* dkeys = in_b ? t.dk_b : t.dk_a;
   int64_t total = 0;

@@ -141,15 +141,19 @@ __device__ __forceinline__ uint64_t ld_status(const uint64_t* p) {
   return *reinterpret_cast<const volatile unsigned long long*>(p);
 }
 
-// Keys only: three CTAs per SM (85 registers); with values two.
-template <bool VALS>
+// Keys only: three CTAs per SM (85 registers); with values two.  RANGES (the
+// last pass of the key sort): a tile-id boundary between two keys of the
+// same digit run of this CTA sets the tile offsets it crosses; the runs'
+// first keys are left to k_range_starts.
+template <bool VALS, bool RANGES>
 __global__ __launch_bounds__(kSortThreads, VALS ? 2 : 3) void k_onesweep(const uint64_t* __restrict__ kin,
                                                            const uint32_t* __restrict__ vin,
                                                            uint64_t* __restrict__ kout, uint32_t* __restrict__ vout,
                                                            int64_t n, int shift, uint64_t epoch,
                                                            const uint32_t* __restrict__ bases,
                                                            uint64_t* __restrict__ status,
-                                                           uint32_t* __restrict__ ticket, uint32_t* __restrict__ err) {
+                                                           uint32_t* __restrict__ ticket, uint32_t* __restrict__ err,
+                                                           int64_t* __restrict__ tile_off) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   OnesweepSmem& S = *reinterpret_cast<OnesweepSmem*>(smem_raw);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -270,6 +274,35 @@ __global__ __launch_bounds__(kSortThreads, VALS ? 2 : 3) void k_onesweep(const u
     const int64_t gpos = S.gbase[d] + (i - (int64_t)S.dstart[d]);
     kout[gpos] = key;
     if (VALS) vout[gpos] = S.v[i];
+    if (RANGES && i != (int)S.dstart[d]) {
+      // inside this CTA's run of digit d the predecessor in the output is
+      // the previous key in shared memory
+      const int64_t prev = (int64_t)(S.k[i - 1] >> 32), cur = (int64_t)(key >> 32);
+      for (int64_t t = prev + 1; t <= cur; ++t) tile_off[t] = gpos;
+    }
+  }
+}
+
+// The first key of every (CTA tile, digit) run of the last pass: its place is
+// the digit's base plus the run's exclusive prefix (the previous tile's
+// inclusive status), its predecessor the key before it in the output; sets
+// the tile offsets that boundary crosses.  Thread (0, 0) also closes the
+// ranges after the last key.
+__global__ __launch_bounds__(kRadix) void k_range_starts(const uint64_t* __restrict__ status,
+                                                         const uint32_t* __restrict__ bases,
+                                                         const uint64_t* __restrict__ keys, int64_t n,
+                                                         int64_t ntiles, int64_t* __restrict__ tile_off) {
+  const int64_t t = blockIdx.x;
+  const int d = threadIdx.x;
+  const uint64_t incl = status[t * kRadix + d] & kValMask;
+  const uint64_t excl = t > 0 ? status[(t - 1) * kRadix + d] & kValMask : 0ull;
+  if (incl > excl) {
+    const int64_t gpos = (int64_t)bases[d] + (int64_t)excl;
+    const int64_t prev = gpos == 0 ? -1 : (int64_t)(keys[gpos - 1] >> 32), cur = (int64_t)(keys[gpos] >> 32);
+    for (int64_t u = prev + 1; u <= cur; ++u) tile_off[u] = gpos;
+  }
+  if (t == 0 && d == 0) {
+    for (int64_t u = (int64_t)(keys[n - 1] >> 32) + 1; u <= ntiles; ++u) tile_off[u] = n;
   }
 }
 
@@ -314,13 +347,20 @@ namespace ss {
 // result is in (kb, vb).  temp: sort_temp_bytes(n), cleared here.  The
 // look-back flag is left in temp (radix_sort_flag).
 ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
-                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b) {
+                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b, int64_t* tile_off,
+                           int64_t ntiles, bool* ranged) {
   *in_b = false;
+  if (ranged) *ranged = false;
   const bool vals = va != nullptr;
-  ss_status s = cuda_status(cudaFuncSetAttribute(vals ? k_onesweep<true> : k_onesweep<false>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)sizeof(OnesweepSmem)),
-                            "set smem attribute");
+  auto pass_kernel = [&](bool ranges) {
+    return vals ? (ranges ? k_onesweep<true, true> : k_onesweep<true, false>)
+                : (ranges ? k_onesweep<false, true> : k_onesweep<false, false>);
+  };
+  ss_status s = SS_OK;
+  for (int r = 0; r < 2 && !s; ++r)
+    s = cuda_status(cudaFuncSetAttribute(pass_kernel(r == 1), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(OnesweepSmem)),
+                    "set smem attribute");
   if (s) return s;
   const int64_t tiles = ceil_div(n, kSortTile);
   char* tb = reinterpret_cast<char*>(temp);
@@ -358,17 +398,30 @@ ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* v
   uint32_t* vin = va;
   uint64_t* kout = kb;
   uint32_t* vout = vb;
-  int run = 0;
+  bool varies[kMaxPasses];
+  int last = -1;
   for (int p = 0; p < passes; ++p) {
     bool one_bin = false;
     for (int d = 0; d < kRadix; ++d) one_bin = one_bin || (int64_t)h[p * kRadix + d] == n;
-    if (one_bin) continue;
+    varies[p] = !one_bin;
+    if (varies[p]) last = p;
+  }
+  int run = 0;
+  for (int p = 0; p < passes; ++p) {
+    if (!varies[p]) continue;
     const int shift = p < lo_bytes ? 8 * p : 32 + 8 * (p - lo_bytes);
     const uint64_t epoch = (uint64_t)(run + 1) << 56;
-    (vals ? k_onesweep<true> : k_onesweep<false>)<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
-        kin, vin, kout, vout, n, shift, epoch, hist + p * kRadix, status, tickets + run, err);
+    const bool ranges = tile_off != nullptr && p == last;
+    pass_kernel(ranges)<<<(unsigned)tiles, kSortThreads, sizeof(OnesweepSmem), st>>>(
+        kin, vin, kout, vout, n, shift, epoch, hist + p * kRadix, status, tickets + run, err, tile_off);
     s = cuda_status(cudaGetLastError(), "radix pass");
     if (s) return s;
+    if (ranges) {
+      k_range_starts<<<(unsigned)tiles, kRadix, 0, st>>>(status, hist + p * kRadix, kout, n, ntiles, tile_off);
+      s = cuda_status(cudaGetLastError(), "tile ranges");
+      if (s) return s;
+      *ranged = true;
+    }
     std::swap(kin, kout);
     std::swap(vin, vout);
     ++run;
@@ -411,13 +464,16 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   // the bytes of the tile ids; the plan drops the bytes that do not vary
   const int lo_bytes = presorted_depth ? 0 : 4;
   const int hi_bytes = max((tile_bits(g.n_tiles) + 7) / 8, lo_bytes ? 0 : 1);
-  bool in_b = false;
-  ss_status s = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, n, lo_bytes, hi_bytes, temp, st, &in_b);
+  bool in_b = false, ranged = false;
+  ss_status s = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, n, lo_bytes, hi_bytes, temp, st, &in_b, tile_off,
+                                 g.n_tiles, &ranged);
   if (s) return s;
-  const unsigned grid = (unsigned)ceil_div(n + 1, 256);
-  k_tile_ranges<<<grid, 256, 0, st>>>(in_b ? keys_b : keys_a, n, g.n_tiles, tile_off);
-  s = cuda_status(cudaGetLastError(), "tile ranges");
-  if (s) return s;
+  if (!ranged) {  // no pass ran: the keys were already in order
+    const unsigned grid = (unsigned)ceil_div(n + 1, 256);
+    k_tile_ranges<<<grid, 256, 0, st>>>(in_b ? keys_b : keys_a, n, g.n_tiles, tile_off);
+    s = cuda_status(cudaGetLastError(), "tile ranges");
+    if (s) return s;
+  }
   bool flagged = false;
   s = radix_sort_flag(temp, st, &flagged);
   if (s) return s;

@@ -500,7 +500,8 @@ def seen_gaussians(d: ss_dims, mask) -> int:
 
 def sort_launches(n_isects: int, passes: int) -> int:
     """Kernels of one ss_sort_isects call: histogram, digit bases, one
-    onesweep kernel per digit pass that runs, tile ranges."""
+    onesweep kernel per digit pass that runs, tile ranges (the runs' first
+    keys after the last pass, or every key when no pass runs)."""
     return 0 if n_isects == 0 else 3 + passes
 
 

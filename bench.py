@@ -163,9 +163,10 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work, n_seen=None, depth_p
     # B written), their keys-only sort (histogram 8 B, 16 B per byte pass),
     # the write (key 8 B, AABB 8 B, offsets 8 B; 12 B per key)
     m["intersect_tiles"] = dict(bytes=nnz * (20 + 8 + 16 * depth_passes + 24) + 12 * n_isects, instr=0.0)
-    # histogram (one read), 12 B read + 12 B written per key per digit pass
-    # that runs (the tile-id bytes: the keys arrive in depth order), tile offsets
-    m["sort_isects"] = dict(bytes=n_isects * (8 + 24 * passes) + 8 * (n_tiles + 1), instr=0.0)
+    # 12 B read + 12 B written per key per digit pass that runs (the tile-id
+    # bytes: the keys arrive in depth order, with their digit counts from the
+    # intersection), tile offsets
+    m["sort_isects"] = dict(bytes=n_isects * (24 * passes) + 8 * (n_tiles + 1), instr=0.0)
     # per-pixel FP32 instructions of the canonical sequences: 11 per evaluated
     # entry (offsets, sigma, tests), 16 per exp (range reduction, degree-7
     # polynomial, scaling, alpha), 7 per composite; backward: 11 per replayed
@@ -326,10 +327,10 @@ def run_ours(args):
                                    step.temp_project)
         ev[1].record(st)
         n = ss.ss_intersect_tiles(d, step.row_depth, step.aabb16, step.block_off, nnz, step.isect_off, step.keys_a,
-                                  step.vals_a, step.cap_isects, step.temp_isect)
+                                  step.vals_a, step.cap_isects, step.temp_isect, key_hist=step.key_hist)
         ev[2].record(st)
         in_b = ss.ss_sort_isects(d, step.keys_a, step.vals_a, step.keys_b, step.vals_b, n, step.temp_sort,
-                                 step.tile_off, presorted_depth=True)
+                                 step.tile_off, presorted_depth=True, key_hist=step.key_hist)
         step.vals = step.vals_b if in_b else step.vals_a
         ev[3].record(st)
         # the rasterizers' tile order is part of the forward rasterizer's stage

@@ -35,9 +35,10 @@ namespace ss {
 
 size_t sort_temp_bytes(int64_t n);
 ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
-                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b, int64_t* tile_off,
-                           int64_t ntiles, bool* ranged);
+                           int hi_bytes, const uint32_t* given_hist, void* temp, cudaStream_t st, bool* in_b,
+                           int64_t* tile_off, int64_t ntiles, bool* ranged);
 ss_status radix_sort_flag(const void* temp, cudaStream_t st, bool* flagged);
+int tile_bits(int64_t ntiles);
 
 constexpr int kIxThreads = 512;
 constexpr int kIxRows = 4096;  // positions of the depth order per CTA
@@ -57,12 +58,12 @@ constexpr int kIxSpinLimit = 1 << 20;
 struct IxSmem {
   uint32_t off[kIxRows + 1];  // slot offset of each row within the block
   uint32_t t0[kIxRows];       // first tile id of the row's range
-  uint32_t dep[kIxRows];      // depth bits
   uint32_t row[kIxRows];      // row index
   uint16_t w[kIxRows];        // tile columns of the row's range
   uint32_t wsum[kIxThreads / 32];
   int64_t cam_row0[kIxCams];  // first row of each camera
   uint32_t cell[kIxChunk / kIxCell + 1];  // row of every kIxCell-th slot of the chunk
+  uint32_t hist[4][256];  // digit counts of the written keys' tile-id bytes
   int64_t base;
   uint32_t blk;
 };
@@ -159,13 +160,16 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
                                                             uint32_t* __restrict__ ticket, uint32_t* __restrict__ err,
                                                             int64_t* __restrict__ isect_off,
                                                             uint64_t* __restrict__ keys,
-                                                            uint32_t* __restrict__ vals) {
+                                                            uint32_t* __restrict__ vals,
+                                                            uint32_t* __restrict__ key_hist, int hist_bytes) {
   extern __shared__ __align__(16) unsigned char ix_raw[];
   IxSmem& S = *reinterpret_cast<IxSmem*>(ix_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // blocks by ticket: every block this one looks back on belongs to a CTA
   // that is already running
   if (tid == 0) S.blk = atomicAdd(ticket, 1u);
+  if (key_hist)
+    for (int i = tid; i < 4 * 256; i += kIxThreads) (&S.hist[0][0])[i] = 0u;
   for (int c = tid; c < min(g.C, kIxCams); c += kIxThreads) S.cam_row0[c] = block_off[(int64_t)c * g.blocks_per_cam];
   __syncthreads();
   const int64_t blk = S.blk;
@@ -183,9 +187,10 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
       int tx0, ty0, w;
       cnt = row_tiles(g, reinterpret_cast<const uint2*>(aabb16)[r], tx0, ty0, w);
       const int c = camera_of_row(block_off, S.cam_row0, g.blocks_per_cam, g.C, (int64_t)r);
-      S.t0[i] = (uint32_t)((uint64_t)c * (uint64_t)g.tiles_per_cam + (uint64_t)ty0 * g.tiles_x + (uint64_t)tx0);
+      const uint32_t t0 =
+          (uint32_t)((uint64_t)c * (uint64_t)g.tiles_per_cam + (uint64_t)ty0 * g.tiles_x + (uint64_t)tx0);
+      S.t0[i] = t0;
       S.w[i] = (uint16_t)w;
-      S.dep[i] = (uint32_t)(key >> 32);
       S.row[i] = r;
     }
     S.off[i] = cnt;
@@ -288,23 +293,52 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
     }
     __syncthreads();
     const uint32_t c1 = min(stop, c0 + (uint32_t)kIxChunk);
-    for (uint32_t s = c0 + tid; s < c1; s += kIxThreads) {
-      const int j = (int)((s - c0) / kIxCell);
-      int lo = (int)S.cell[j], hi = (int)S.cell[j + 1];  // the row is in [lo, hi]
-      while (hi > lo) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (S.off[mid] <= s) lo = mid; else hi = mid - 1;
+    // warp-uniform rounds: a warp's lanes take 32 consecutive slots
+    for (uint32_t s0 = c0 + (uint32_t)(warp * 32); s0 < c1; s0 += kIxThreads) {
+      const uint32_t s = s0 + (uint32_t)lane;
+      const bool live = s < c1;
+      uint32_t tile32 = 0;
+      if (live) {
+        const int j = (int)((s - c0) / kIxCell);
+        int lo = (int)S.cell[j], hi = (int)S.cell[j + 1];  // the row is in [lo, hi]
+        while (hi > lo) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (S.off[mid] <= s) lo = mid; else hi = mid - 1;
+        }
+        const uint32_t k = s - S.off[lo], w = S.w[lo];
+        // k / w through the approximate reciprocal: k < 2^24, so the estimate is
+        // off by at most one, and one correction each way makes it exact
+        uint32_t ty = (uint32_t)__fmul_rz((float)k, __frcp_rn((float)w));
+        if (ty * w > k) --ty;
+        if ((ty + 1) * w <= k) ++ty;
+        const uint32_t tx = k - ty * w;
+        const uint64_t tile = (uint64_t)S.t0[lo] + (uint64_t)ty * (uint64_t)g.tiles_x + tx;
+        keys[base + s] = (tile << 32) | (dkeys[p0 + lo] >> 32);  // the row's depth bits (L1-resident)
+        vals[base + s] = S.row[lo];
+        tile32 = (uint32_t)tile;
       }
-      const uint32_t k = s - S.off[lo], w = S.w[lo];
-      // k / w through the approximate reciprocal: k < 2^24, so the estimate is
-      // off by at most one, and one correction each way makes it exact
-      uint32_t ty = (uint32_t)__fmul_rz((float)k, __frcp_rn((float)w));
-      if (ty * w > k) --ty;
-      if ((ty + 1) * w <= k) ++ty;
-      const uint32_t tx = k - ty * w;
-      const uint64_t tile = (uint64_t)S.t0[lo] + (uint64_t)ty * (uint64_t)g.tiles_x + tx;
-      keys[base + s] = (tile << 32) | S.dep[lo];
-      vals[base + s] = S.row[lo];
+      if (key_hist) {
+        // the keys' tile-id bytes, counted for the sort: neighbouring slots
+        // share their upper bytes (a row's tiles are consecutive ids), so
+        // each run of equal digits is added by its first lane
+        const uint32_t vmask = __ballot_sync(0xffffffffu, live);
+        const uint32_t end_all = 32u - (uint32_t)__clz(vmask);
+        const uint32_t above = ~((2u << lane) - 1u);
+        for (int b = 0; b < hist_bytes; ++b) {
+          const uint32_t d = (tile32 >> (8 * b)) & 0xFFu;
+          const uint32_t prev = __shfl_up_sync(0xffffffffu, d, 1);
+          const bool head = live && (lane == 0 || d != prev);
+          const uint32_t after = __ballot_sync(0xffffffffu, head) & above;
+          if (head) atomicAdd(&S.hist[b][d], (after ? (uint32_t)(__ffs(after) - 1) : end_all) - (uint32_t)lane);
+        }
+      }
+    }
+  }
+  if (key_hist) {
+    __syncthreads();
+    for (int i = tid; i < hist_bytes * 256; i += kIxThreads) {
+      const uint32_t c = (&S.hist[0][0])[i];
+      if (c) atomicAdd(key_hist + i, c);
     }
   }
 }
@@ -315,14 +349,18 @@ using namespace ss;
 
 extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_depth, const uint32_t* aabb16,
                                         const int64_t* block_off, int64_t nnz, int64_t* isect_off, uint64_t* keys,
-                                        uint32_t* vals, int64_t cap_isects, void* temp, size_t temp_bytes,
-                                        uint64_t* n_isects_out, void* stream) {
+                                        uint32_t* vals, uint32_t* key_hist, int64_t cap_isects, void* temp,
+                                        size_t temp_bytes, uint64_t* n_isects_out, void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (!n_isects_out || !isect_off) return invalid("null output");
   if (nnz < 0) return invalid("nnz < 0");
   if (nnz >= (int64_t(1) << 32)) return invalid("nnz >= 2^32 (32-bit row ids)");
   const Geo g = geometry(*dims);
   cudaStream_t st = as_stream(stream);
+  if (key_hist) {
+    ss_status s = cuda_status(cudaMemsetAsync(key_hist, 0, 4 * 256 * sizeof(uint32_t), st), "memset");
+    if (s) return s;
+  }
   if (nnz == 0) {
     ss_status s = cuda_status(cudaMemsetAsync(isect_off, 0, sizeof(int64_t), st), "memset");
     if (s) return s;
@@ -343,7 +381,8 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   // the rows in depth order (ties by row index: the sort is stable and the
   // row index is the key's low word)
   bool in_b = false;
-  s = radix_sort_pairs(t.dk_a, nullptr, t.dk_b, nullptr, nnz, 0, 4, t.sort, st, &in_b, nullptr, 0, nullptr);
+  s = radix_sort_pairs(t.dk_a, nullptr, t.dk_b, nullptr, nnz, 0, 4, nullptr, t.sort, st, &in_b, nullptr, 0,
+                       nullptr);
   if (s) return s;
   const uint64_t* dkeys = in_b ? t.dk_b : t.dk_a;
   int64_t total = 0;
@@ -372,7 +411,8 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
                   "set smem attribute");
   if (s) return s;
   k_isect_fused<<<(unsigned)ceil_div(nnz, kIxRows), kIxThreads, sizeof(IxSmem), st>>>(
-      g, dkeys, aabb16, block_off, nnz, limit, t.status, t.ticket, t.err, isect_off, keys, vals);
+      g, dkeys, aabb16, block_off, nnz, limit, t.status, t.ticket, t.err, isect_off, keys, vals, key_hist,
+      max(1, (tile_bits(g.n_tiles) + 7) / 8));
   s = cuda_status(cudaGetLastError(), "intersect write");
   if (s) return s;
   // the write's look-back flag (stream sync)

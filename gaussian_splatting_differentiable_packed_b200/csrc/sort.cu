@@ -347,8 +347,8 @@ namespace ss {
 // result is in (kb, vb).  temp: sort_temp_bytes(n), cleared here.  The
 // look-back flag is left in temp (radix_sort_flag).
 ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* vb, int64_t n, int lo_bytes,
-                           int hi_bytes, void* temp, cudaStream_t st, bool* in_b, int64_t* tile_off,
-                           int64_t ntiles, bool* ranged) {
+                           int hi_bytes, const uint32_t* given_hist, void* temp, cudaStream_t st, bool* in_b,
+                           int64_t* tile_off, int64_t ntiles, bool* ranged) {
   *in_b = false;
   if (ranged) *ranged = false;
   const bool vals = va != nullptr;
@@ -373,7 +373,10 @@ ss_status radix_sort_pairs(uint64_t* ka, uint32_t* va, uint64_t* kb, uint32_t* v
   const int passes = lo_bytes + hi_bytes;
   if (passes < 1 || passes > kMaxPasses) return invalid("sort digit count");
   const unsigned hgrid = (unsigned)min64(tiles, 148 * 8);
-  switch (passes) {
+  if (given_hist) {  // the digit counts come with the keys
+    s = cuda_status(cudaMemcpyAsync(hist, given_hist, (size_t)passes * kRadix * 4, cudaMemcpyDeviceToDevice, st),
+                    "copy histograms");
+  } else switch (passes) {
     case 1: s = launch_hist<1>(hgrid, st, ka, n, lo_bytes, hist); break;
     case 2: s = launch_hist<2>(hgrid, st, ka, n, lo_bytes, hist); break;
     case 3: s = launch_hist<3>(hgrid, st, ka, n, lo_bytes, hist); break;
@@ -445,8 +448,9 @@ ss_status radix_sort_flag(const void* temp, cudaStream_t st, bool* flagged) {
 }  // namespace ss
 
 extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
-                                    uint32_t* vals_b, int64_t n, int presorted_depth, void* temp, size_t temp_bytes,
-                                    int64_t* tile_off, int* result_in_b_out, void* stream) {
+                                    uint32_t* vals_b, int64_t n, int presorted_depth, const uint32_t* key_hist,
+                                    void* temp, size_t temp_bytes, int64_t* tile_off, int* result_in_b_out,
+                                    void* stream) {
   if (!dims_ok(dims)) return invalid("dims");
   if (!result_in_b_out || !tile_off) return invalid("null output");
   if (n < 0) return invalid("n < 0");
@@ -460,13 +464,14 @@ extern "C" ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint3
   if (n == 0) return cuda_status(cudaMemsetAsync(tile_off, 0, sizeof(int64_t) * (g.n_tiles + 1), st), "memset");
   if (!keys_a || !vals_a || !keys_b || !vals_b) return invalid("null keys/vals");
   if (!temp || temp_bytes < sort_temp_bytes(n)) return invalid("temp too small");
+  if (key_hist && !presorted_depth) return invalid("key_hist needs presorted_depth (tile-id digits only)");
   // every byte of the depth (none when the keys arrive in depth order) and
   // the bytes of the tile ids; the plan drops the bytes that do not vary
   const int lo_bytes = presorted_depth ? 0 : 4;
   const int hi_bytes = max((tile_bits(g.n_tiles) + 7) / 8, lo_bytes ? 0 : 1);
   bool in_b = false, ranged = false;
-  ss_status s = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, n, lo_bytes, hi_bytes, temp, st, &in_b, tile_off,
-                                 g.n_tiles, &ranged);
+  ss_status s = radix_sort_pairs(keys_a, vals_a, keys_b, vals_b, n, lo_bytes, hi_bytes, key_hist, temp, st, &in_b,
+                                 tile_off, g.n_tiles, &ranged);
   if (s) return s;
   if (!ranged) {  // no pass ran: the keys were already in order
     const unsigned grid = (unsigned)ceil_div(n + 1, 256);
@@ -576,6 +581,6 @@ extern "C" ss_status ss_sort_isects_noalloc(const ss_dims* dims, uint64_t* keys_
     ss_status s = noalloc_scratch(&scratch);
     if (s) return s;
   }
-  return ss_sort_isects(dims, keys_a, vals_a, keys_b, vals_b, n, 0, scratch, kNoAllocScratchBytes, tile_off,
-                        result_in_b_out, stream);
+  return ss_sort_isects(dims, keys_a, vals_a, keys_b, vals_b, n, 0, nullptr, scratch, kNoAllocScratchBytes,
+                        tile_off, result_in_b_out, stream);
 }

@@ -86,8 +86,8 @@ def lib() -> ct.CDLL:
         L.ss_last_error.argtypes = []
         L.ss_last_error.restype = ct.c_char_p
         L.ss_project_packed.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, i64, i64, P, sz, ct.POINTER(i64), P]
-        L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
-        L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, i32, P, sz, P, ct.POINTER(i32), P]
+        L.ss_intersect_tiles.argtypes = [D, P, P, P, i64, P, P, P, P, i64, P, sz, ct.POINTER(ct.c_uint64), P]
+        L.ss_sort_isects.argtypes = [D, P, P, P, P, i64, i32, P, P, sz, P, ct.POINTER(i32), P]
         L.ss_sort_isects_noalloc.argtypes = [D, P, P, P, P, i64, P, ct.POINTER(i32), P]
         L.ss_tile_order.argtypes = [D, P, P, P, sz, P]
         L.ss_rasterize_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P]
@@ -157,22 +157,26 @@ def ss_project_packed(d, cams, means, quats, scales, opacities, sh, mask, block_
 
 
 def ss_intersect_tiles(d, row_depth, aabb16, block_off, nnz, isect_off, keys, vals, cap_isects, temp,
-                       stream=None) -> int:
+                       stream=None, key_hist=None) -> int:
+    """key_hist: optional device uint32 [4*256], set to the digit counts of
+    the keys' tile-id bytes (for ss_sort_isects)."""
     n = ct.c_uint64(0)
     st = lib().ss_intersect_tiles(ct.byref(d), _p(row_depth), _p(aabb16), _p(block_off), int(nnz), _p(isect_off),
-                                  _p(keys), _p(vals), int(cap_isects), _p(temp),
+                                  _p(keys), _p(vals), _p(key_hist), int(cap_isects), _p(temp),
                                   0 if temp is None else temp.numel() * temp.element_size(), ct.byref(n),
                                   _stream(stream))
     _check(st, "ss_intersect_tiles", int(n.value))
     return int(n.value)
 
 
-def ss_sort_isects(d, keys_a, vals_a, keys_b, vals_b, n, temp, tile_off, stream=None, presorted_depth=False) -> bool:
+def ss_sort_isects(d, keys_a, vals_a, keys_b, vals_b, n, temp, tile_off, stream=None, presorted_depth=False,
+                   key_hist=None) -> bool:
     """presorted_depth: the keys arrive in depth order (as ss_intersect_tiles
-    writes them), so only the tile-id bytes are sorted."""
+    writes them), so only the tile-id bytes are sorted; key_hist: their digit
+    counts as ss_intersect_tiles wrote them (skips the histogram read)."""
     in_b = ct.c_int(0)
     st = lib().ss_sort_isects(ct.byref(d), _p(keys_a), _p(vals_a), _p(keys_b), _p(vals_b), int(n),
-                              1 if presorted_depth else 0, _p(temp),
+                              1 if presorted_depth else 0, _p(key_hist), _p(temp),
                               0 if temp is None else temp.numel() * temp.element_size(), _p(tile_off),
                               ct.byref(in_b), _stream(stream))
     _check(st, "ss_sort_isects")
@@ -351,6 +355,7 @@ class PackedStep:
         self.block_off = torch.empty(self.mask_blocks + 1, dtype=torch.int64, device=dev)
         self.temp_project = torch.empty(workspace_bytes(d, WS_PROJECT), dtype=torch.uint8, device=dev)
         self.tile_off = torch.empty(self.n_tiles + 1, dtype=torch.int64, device=dev)
+        self.key_hist = torch.empty(4 * 256, dtype=torch.int32, device=dev)  # digit counts of the keys' tile ids
         self.tile_order = _u32(self.n_tiles, dev)
         self.temp_order = torch.empty(workspace_bytes(d, WS_TILE_ORDER), dtype=torch.uint8, device=dev)
         self.img = torch.empty((C, d.H, d.W, 3), dtype=torch.float32, device=dev)
@@ -412,18 +417,20 @@ class PackedStep:
         self.nnz = nnz
         try:
             n = ss_intersect_tiles(d, self.row_depth, self.aabb16, self.block_off, nnz, self.isect_off,
-                                   self.keys_a, self.vals_a, self.cap_isects, self.temp_isect, stream)
+                                   self.keys_a, self.vals_a, self.cap_isects, self.temp_isect, stream,
+                                   key_hist=self.key_hist)
         except SSError as e:
             if e.status != SS_ERR_CAPACITY:
                 raise
             self._isects(int(e.count * self.headroom) + 1)
             n = ss_intersect_tiles(d, self.row_depth, self.aabb16, self.block_off, nnz, self.isect_off,
-                                   self.keys_a, self.vals_a, self.cap_isects, self.temp_isect, stream)
+                                   self.keys_a, self.vals_a, self.cap_isects, self.temp_isect, stream,
+                                   key_hist=self.key_hist)
         self.n_isects = n
         self.unsorted_keys = self.keys_a
         self.unsorted_vals = self.vals_a
         self.result_in_b = ss_sort_isects(d, self.keys_a, self.vals_a, self.keys_b, self.vals_b, n, self.temp_sort,
-                                          self.tile_off, stream, presorted_depth=True)
+                                          self.tile_off, stream, presorted_depth=True, key_hist=self.key_hist)
         self.keys = self.keys_b if self.result_in_b else self.keys_a
         self.vals = self.vals_b if self.result_in_b else self.vals_a
         ss_tile_order(d, self.tile_off, self.tile_order, self.temp_order, stream)
@@ -498,11 +505,12 @@ def seen_gaussians(d: ss_dims, mask) -> int:
     return int(pop.sum().item())
 
 
-def sort_launches(n_isects: int, passes: int) -> int:
-    """Kernels of one ss_sort_isects call: histogram, digit bases, one
-    onesweep kernel per digit pass that runs, tile ranges (the runs' first
-    keys after the last pass, or every key when no pass runs)."""
-    return 0 if n_isects == 0 else 3 + passes
+def sort_launches(n_isects: int, passes: int, given_hist: bool = True) -> int:
+    """Kernels of one ss_sort_isects call: histogram (none when the digit
+    counts come with the keys), digit bases, one onesweep kernel per digit
+    pass that runs, tile ranges (the runs' first keys after the last pass, or
+    every key when no pass runs)."""
+    return 0 if n_isects == 0 else (2 if given_hist else 3) + passes
 
 
 def launches_per_step(d: ss_dims, nnz: int, n_isects: int, sort_passes: int, depth_passes: int) -> int:

@@ -167,11 +167,14 @@ ss_status ss_project_packed(const ss_dims* dims, const float* cams, const float*
  * ss_workspace_bytes(SS_WS_INTERSECT, nnz) bytes (it holds the depth order
  * of the rows).  The call synchronises the stream once more after the write
  * and returns SS_ERR_DEVICE_CHECK if a bounded look-back wait (the depth
- * sort's or the write's offsets) ran out.
+ * sort's or the write's offsets) ran out.  key_hist (device, nullable):
+ * uint32 [4][256], set to the counts of each digit value of byte b of the
+ * written keys' tile ids (rows b >= the tile-id bytes stay zero), for
+ * ss_sort_isects' key_hist.
  */
 ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_depth, const uint32_t* aabb16,
                              const int64_t* block_off, int64_t nnz, int64_t* isect_off, uint64_t* keys,
-                             uint32_t* vals, int64_t cap_isects, void* temp, size_t temp_bytes,
+                             uint32_t* vals, uint32_t* key_hist, int64_t cap_isects, void* temp, size_t temp_bytes,
                              uint64_t* n_isects_out, void* stream);
 
 /*
@@ -185,12 +188,15 @@ ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_depth, const 
  * between (keys_a, vals_a) and (keys_b, vals_b); *result_in_b_out (host)
  * says which pair holds the result (b after an odd number of digit passes,
  * which depends on the keys).  Then writes tile_off[n_tiles+1].
+ * key_hist (device, nullable; only with presorted_depth != 0): the digit
+ * counts of the keys' tile-id bytes, uint32 [4][256] as ss_intersect_tiles
+ * writes them; the sort then skips its own histogram read of the keys.
  * n >= 2^31 returns SS_ERR_OVERFLOW.  Equal keys keep their input order.
  * Synchronises the stream at the end (reads the look-back error flag).
  */
 ss_status ss_sort_isects(const ss_dims* dims, uint64_t* keys_a, uint32_t* vals_a, uint64_t* keys_b,
-                         uint32_t* vals_b, int64_t n, int presorted_depth, void* temp, size_t temp_bytes,
-                         int64_t* tile_off, int* result_in_b_out, void* stream);
+                         uint32_t* vals_b, int64_t n, int presorted_depth, const uint32_t* key_hist, void* temp,
+                         size_t temp_bytes, int64_t* tile_off, int* result_in_b_out, void* stream);
 
 /*
  * Projection backward fused with an Adam step (the pages' fused projection

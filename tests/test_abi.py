@@ -88,8 +88,8 @@ def test_invalid_dims_rejected_on_host(L, bad):
 def test_sort_overflow_rejected_before_device_work(L):
     d = ss.make_dims(1, 64, 64, 0, 10)
     in_b = ct.c_int(0)
-    st = L.ss_sort_isects(ct.byref(d), None, None, None, None, 2**31, 0, None, 0, ct.c_void_p(16), ct.byref(in_b),
-                          None)
+    st = L.ss_sort_isects(ct.byref(d), None, None, None, None, 2**31, 0, None, None, 0, ct.c_void_p(16),
+                          ct.byref(in_b), None)
     assert st == ss.SS_ERR_OVERFLOW
     assert L.ss_status_string(st) == b"count overflows 32-bit indices"
 
@@ -117,7 +117,8 @@ def test_null_and_short_temp_rejected(L):
                              -1, fake, 1, ct.byref(nnz), None)
     assert st == ss.SS_ERR_INVALID_ARG
     n = ct.c_uint64(0)
-    st = L.ss_intersect_tiles(ct.byref(d), fake, fake, fake, 5, fake, fake, fake, 100, fake, 1, ct.byref(n), None)
+    st = L.ss_intersect_tiles(ct.byref(d), fake, fake, fake, 5, fake, fake, fake, None, 100, fake, 1, ct.byref(n),
+                              None)
     assert st == ss.SS_ERR_INVALID_ARG
 
 

@@ -89,13 +89,22 @@ def check_unsorted(scene, o, step):
     I = it["n_isects"]
     keys = torch.empty(max(I, 1), dtype=torch.int64, device="cuda")
     vals = torch.empty(max(I, 1), dtype=torch.int32, device="cuda")
+    hist = torch.full((4 * 256,), -1, dtype=torch.int32, device="cuda")
     n = ss.ss_intersect_tiles(step.d, step.row_depth, step.aabb16, step.block_off, step.nnz, step.isect_off, keys, vals,
-                              I, step.temp_isect)
+                              I, step.temp_isect, key_hist=hist)
     torch.cuda.synchronize()
     assert n == I
     if I:
         np.testing.assert_array_equal(keys[:I].cpu().numpy().view(np.uint64), it["keys"])
         np.testing.assert_array_equal(u32(vals[:I]), it["vals"])
+    # the digit counts of the keys' tile-id bytes it wrote for the sort (the
+    # bytes past the tile ids' width stay zero)
+    tiles = it["keys"] >> np.uint64(32)
+    nb = max(1, (int(np.ceil(np.log2(max(ss.size(step.d, ss.SIZE_N_TILES), 1)))) + 7) // 8) if I else 0
+    want = np.zeros((4, 256), np.int64)
+    for b in range(nb):
+        want[b] = np.bincount(((tiles >> np.uint64(8 * b)) & np.uint64(255)).astype(np.int64), minlength=256)
+    np.testing.assert_array_equal(hist.cpu().numpy().reshape(4, 256), want)
 
 
 def check_backward(scene, o, step):

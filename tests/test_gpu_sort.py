@@ -35,7 +35,16 @@ def make_keys(rng, n_tiles, n, hot=()):
     return keys, vals
 
 
-def run_sort(d, keys, vals, presorted_depth=False):
+def digit_hist(keys):
+    """Counts of each value of byte b of the keys' tile ids, [4][256] int32."""
+    tiles = (np.asarray(keys, np.uint64) >> np.uint64(32)).astype(np.uint64)
+    h = np.zeros((4, 256), np.int64)
+    for b in range(4):
+        h[b] = np.bincount(((tiles >> np.uint64(8 * b)) & np.uint64(255)).astype(np.int64), minlength=256)
+    return h.astype(np.int32).reshape(-1)
+
+
+def run_sort(d, keys, vals, presorted_depth=False, with_hist=False):
     n = len(keys)
     ka = torch.from_numpy(keys.view(np.int64).copy()).cuda()
     va = torch.from_numpy(vals.view(np.int32).copy()).cuda()
@@ -44,7 +53,8 @@ def run_sort(d, keys, vals, presorted_depth=False):
     n_tiles = ss.size(d, ss.SIZE_N_TILES)
     tile_off = torch.empty(n_tiles + 1, dtype=torch.int64, device="cuda")
     temp = torch.empty(ss.workspace_bytes(d, ss.WS_SORT, n), dtype=torch.uint8, device="cuda")
-    in_b = ss.ss_sort_isects(d, ka, va, kb, vb, n, temp, tile_off, presorted_depth=presorted_depth)
+    hist = torch.from_numpy(digit_hist(keys)).cuda() if with_hist else None
+    in_b = ss.ss_sort_isects(d, ka, va, kb, vb, n, temp, tile_off, presorted_depth=presorted_depth, key_hist=hist)
     torch.cuda.synchronize()
     k, v = (kb, vb) if in_b else (ka, va)
     return in_b, k.cpu().numpy().view(np.uint64), v.cpu().numpy().view(np.uint32), tile_off.cpu().numpy()
@@ -120,9 +130,12 @@ def test_sort_presorted_depth(case):
     keys, vals = make_keys(rng, n_tiles, 300_000, [(n_tiles - 1, 3000), (3, 9000)])
     order = np.argsort((keys & np.uint64(0xFFFFFFFF)).astype(np.uint32), kind="stable")
     keys, vals = keys[order], vals[order]
-    in_b, gk, gv, toff = run_sort(d, keys, vals, presorted_depth=True)
-    assert in_b == bool(ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d, presorted_depth=True) & 1)
     ok, ov = orc.sort(keys, vals)
-    np.testing.assert_array_equal(gk, ok)
-    np.testing.assert_array_equal(gv, ov)
-    np.testing.assert_array_equal(toff, orc.tile_ranges(ok, n_tiles))
+    # with the sort's own histogram read, and with the digit counts given as
+    # the intersection writes them
+    for with_hist in (False, True):
+        in_b, gk, gv, toff = run_sort(d, keys, vals, presorted_depth=True, with_hist=with_hist)
+        assert in_b == bool(ss.sort_passes_for(torch.from_numpy(keys.view(np.int64)), d, presorted_depth=True) & 1)
+        np.testing.assert_array_equal(gk, ok)
+        np.testing.assert_array_equal(gv, ov)
+        np.testing.assert_array_equal(toff, orc.tile_ranges(ok, n_tiles))

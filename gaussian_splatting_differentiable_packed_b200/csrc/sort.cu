@@ -8,7 +8,8 @@
 // copy) and launches only the passes whose digits vary.
 //
 //   k_hist_all   one read of the keys: the global digit histogram of every pass
-//                (a permutation does not change them)
+//                (a permutation does not change them); skipped when the caller
+//                passes the counts (key_hist, as the intersection writes them)
 //   k_bases      the exclusive scan of each pass's 256 counts
 //   k_onesweep   per pass, one kernel: each CTA takes the next 4096-key tile by
 //                ticket, ranks its keys stably among equal digits (warp match +
@@ -16,6 +17,9 @@
 //                over earlier tiles' published counts (decoupled look-back) for
 //                its global offsets, then writes the keys in contiguous runs
 //                from shared memory.  12 B read + 12 B written per key per pass.
+//                The last pass also sets the tile offsets at tile boundaries
+//                inside its runs; k_range_starts then takes the runs' first
+//                keys (their places follow from the look-back status).
 //
 // The look-back spin is bounded: after kSpinLimit polls it records an error
 // flag (reported by the call as SS_ERR_DEVICE_CHECK) and goes on.  Tiles are

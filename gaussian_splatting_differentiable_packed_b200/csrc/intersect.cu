@@ -306,16 +306,20 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
           if (S.off[mid] <= s) lo = mid; else hi = mid - 1;
         }
         const uint32_t k = s - S.off[lo], w = S.w[lo];
-        // k / w through the approximate reciprocal: k < 2^24, so the estimate is
-        // off by at most one, and one correction each way makes it exact
-        uint32_t ty = (uint32_t)__fmul_rz((float)k, __frcp_rn((float)w));
+        // k / w through the hardware's approximate reciprocal (relative error
+        // below 2^-22 with the product's rounding): k < 2^24 is exact in fp32
+        // and the quotient is below 2^22, so the estimate's floor is off by at
+        // most one, and one correction each way makes it exact
+        float rw;
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rw) : "f"((float)w));
+        uint32_t ty = (uint32_t)__fmul_rz((float)k, rw);
         if (ty * w > k) --ty;
         if ((ty + 1) * w <= k) ++ty;
         const uint32_t tx = k - ty * w;
-        const uint64_t tile = (uint64_t)S.t0[lo] + (uint64_t)ty * (uint64_t)g.tiles_x + tx;
-        keys[base + s] = (tile << 32) | (dkeys[p0 + lo] >> 32);  // the row's depth bits (L1-resident)
+        // tile ids fit 32 bits (a key's high word)
+        tile32 = S.t0[lo] + ty * (uint32_t)g.tiles_x + tx;
+        keys[base + s] = ((uint64_t)tile32 << 32) | (dkeys[p0 + lo] >> 32);  // the row's depth bits (L1-resident)
         vals[base + s] = S.row[lo];
-        tile32 = (uint32_t)tile;
       }
       if (key_hist) {
         // the keys' tile-id bytes, counted for the sort: neighbouring slots
@@ -324,7 +328,9 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
         const uint32_t vmask = __ballot_sync(0xffffffffu, live);
         const uint32_t end_all = 32u - (uint32_t)__clz(vmask);
         const uint32_t above = ~((2u << lane) - 1u);
-        for (int b = 0; b < hist_bytes; ++b) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          if (b >= hist_bytes) break;
           const uint32_t d = (tile32 >> (8 * b)) & 0xFFu;
           const uint32_t prev = __shfl_up_sync(0xffffffffu, d, 1);
           const bool head = live && (lane == 0 || d != prev);

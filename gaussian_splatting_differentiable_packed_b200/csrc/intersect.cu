@@ -18,8 +18,10 @@
 //   (host)          checks the total against the capacity and 2^31
 //   k_isect_fused   one CTA per 4096 positions of the depth order, blocks
 //                   taken by ticket: decodes its rows once into shared memory
-//                   (first tile id, tile columns, depth bits, row id, from
-//                   the row's AABB16), scans their tile counts, publishes the
+//                   (first tile id and tile columns, from the row's AABB16;
+//                   the depth bits and the row id are the row's depth key,
+//                   read again at the write), scans their tile counts,
+//                   publishes the
 //                   block's total and looks back over earlier blocks for its
 //                   base (decoupled look-back, bounded spin), writes the
 //                   rows' offsets to isect_off, then expands the block's
@@ -58,7 +60,6 @@ constexpr int kIxSpinLimit = 1 << 20;
 struct IxSmem {
   uint32_t off[kIxRows + 1];  // slot offset of each row within the block
   uint32_t t0[kIxRows];       // first tile id of the row's range
-  uint32_t row[kIxRows];      // row index
   uint16_t w[kIxRows];        // tile columns of the row's range
   uint32_t wsum[kIxThreads / 32];
   int64_t cam_row0[kIxCams];  // first row of each camera
@@ -191,7 +192,6 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
           (uint32_t)((uint64_t)c * (uint64_t)g.tiles_per_cam + (uint64_t)ty0 * g.tiles_x + (uint64_t)tx0);
       S.t0[i] = t0;
       S.w[i] = (uint16_t)w;
-      S.row[i] = r;
     }
     S.off[i] = cnt;
   }
@@ -318,8 +318,10 @@ __global__ __launch_bounds__(kIxThreads) void k_isect_fused(Geo g, const uint64_
         const uint32_t tx = k - ty * w;
         // tile ids fit 32 bits (a key's high word)
         tile32 = S.t0[lo] + ty * (uint32_t)g.tiles_x + tx;
-        keys[base + s] = ((uint64_t)tile32 << 32) | (dkeys[p0 + lo] >> 32);  // the row's depth bits (L1-resident)
-        vals[base + s] = S.row[lo];
+        // the row's depth key (L1-resident): depth bits and row index
+        const uint64_t dk = dkeys[p0 + lo];
+        keys[base + s] = ((uint64_t)tile32 << 32) | (dk >> 32);
+        vals[base + s] = (uint32_t)dk;
       }
       if (key_hist) {
         // the keys' tile-id bytes, counted for the sort: neighbouring slots

@@ -21,15 +21,14 @@
 //                   (first tile id and tile columns, from the row's AABB16;
 //                   the depth bits and the row id are the row's depth key,
 //                   read again at the write), scans their tile counts,
-//                   publishes the
-//                   block's total and looks back over earlier blocks for its
-//                   base (decoupled look-back, bounded spin), writes the
-//                   rows' offsets to isect_off, then expands the block's
-//                   slots 8192 at a time: slot s belongs to the last row
-//                   whose offset is <= s (a binary search in shared memory
-//                   between the rows of its 64-slot cell, found first), and
-//                   consecutive threads write consecutive slots, so every
-//                   store is coalesced whatever the per-row counts.
+//                   publishes the block's total and looks back over earlier
+//                   blocks for its base (decoupled look-back, bounded spin),
+//                   writes the rows' offsets to isect_off, then expands the
+//                   block's slots 8192 at a time: slot s belongs to the last
+//                   row whose offset is <= s (a binary search in shared
+//                   memory between the rows of its 64-slot cell, found
+//                   first), and consecutive threads write consecutive slots,
+//                   so every store is coalesced whatever the per-row counts.
 #include "ss_common.cuh"
 #include "ss_math.cuh"
 

@@ -10,9 +10,10 @@
 // nnz rows' 32-bit depths replaces the depth passes over the keys (2.2 keys a
 // row on the 15M-Gaussian workload, 59 on the 7680^2 one).
 //
-//   k_row_keys      (depth bits << 32 | row) of every row, and the exact
-//                   int64 total of tiles covered (integer atomics, one per
-//                   CTA: the sum is the same in any order)
+//   k_row_keys      (depth bits << 32 | row) of every row, the exact int64
+//                   total of tiles covered (integer atomics, one per CTA:
+//                   the sum is the same in any order) and the depth bytes'
+//                   digit counts, so the depth sort reads no histogram
 //   radix sort      keys only, by the depth word (sort.cu; the row index in
 //                   the low word rides along, ties stay in row order)
 //   (host)          checks the total against the capacity and 2^31
@@ -69,13 +70,15 @@ struct IxSmem {
 };
 
 // Scratch: total (int64) | ticket (u32) | error flag (u32) | block status
-// (u64 per block), then the keys' two buffers and the sort's scratch.
+// (u64 per block) | the depth keys' digit counts ([4][256] u32), then the
+// keys' two buffers and the sort's scratch.
 struct IxTemp {
   int64_t* total;
   uint32_t* ticket;
   uint32_t* err;
   uint64_t* status;
-  size_t head_bytes;  // total .. status, cleared per call
+  uint32_t* dhist;    // [4][256] digit counts of the depth keys' high word
+  size_t head_bytes;  // total .. dhist, cleared per call
   uint64_t *dk_a, *dk_b;
   void* sort;
 };
@@ -87,7 +90,8 @@ IxTemp isect_temp(void* temp, int64_t nnz) {
   t.ticket = reinterpret_cast<uint32_t*>(p + 8);
   t.err = reinterpret_cast<uint32_t*>(p + 12);
   t.status = reinterpret_cast<uint64_t*>(p + 16);
-  t.head_bytes = align_up(16 + (size_t)ceil_div(nnz, kIxRows) * 8, 256);
+  t.dhist = reinterpret_cast<uint32_t*>(p + 16 + (size_t)ceil_div(nnz, kIxRows) * 8);
+  t.head_bytes = align_up(16 + (size_t)ceil_div(nnz, kIxRows) * 8 + 4 * 256 * 4, 256);
   p += t.head_bytes;
   t.dk_a = reinterpret_cast<uint64_t*>(p);
   p += align_up((size_t)nnz * 8, 256);
@@ -98,7 +102,7 @@ IxTemp isect_temp(void* temp, int64_t nnz) {
 }
 
 size_t isect_temp_bytes(int64_t nnz) {
-  return align_up(16 + (size_t)ceil_div(nnz, kIxRows) * 8, 256) + 2 * align_up((size_t)nnz * 8, 256) +
+  return align_up(16 + (size_t)ceil_div(nnz, kIxRows) * 8 + 4 * 256 * 4, 256) + 2 * align_up((size_t)nnz * 8, 256) +
          sort_temp_bytes(nnz);
 }
 
@@ -115,12 +119,19 @@ __device__ __forceinline__ uint32_t row_tiles(const Geo& g, uint2 q, int& tx0, i
 __global__ __launch_bounds__(kRowKeyThreads) void k_row_keys(Geo g, const float* __restrict__ row_depth,
                                                              const uint32_t* __restrict__ aabb16, int64_t nnz,
                                                              uint64_t* __restrict__ keys,
-                                                             int64_t* __restrict__ total) {
+                                                             int64_t* __restrict__ total,
+                                                             uint32_t* __restrict__ dhist) {
   __shared__ unsigned long long ws[kRowKeyThreads / 32];
+  __shared__ uint32_t h[4][256];  // the depth bytes' digit counts, for the depth sort
+  for (int i = threadIdx.x; i < 4 * 256; i += kRowKeyThreads) (&h[0][0])[i] = 0u;
+  __syncthreads();
   unsigned long long cnt = 0;
   for (int64_t r = (int64_t)blockIdx.x * kRowKeyThreads + threadIdx.x; r < nnz;
        r += (int64_t)gridDim.x * kRowKeyThreads) {
-    keys[r] = ((uint64_t)__float_as_uint(row_depth[r]) << 32) | (uint64_t)r;
+    const uint32_t d = __float_as_uint(row_depth[r]);
+    keys[r] = ((uint64_t)d << 32) | (uint64_t)r;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) atomicAdd(&h[b][(d >> (8 * b)) & 0xFFu], 1u);
     int tx0, ty0, w;
     cnt += row_tiles(g, reinterpret_cast<const uint2*>(aabb16)[r], tx0, ty0, w);
   }
@@ -133,6 +144,10 @@ __global__ __launch_bounds__(kRowKeyThreads) void k_row_keys(Geo g, const float*
 #pragma unroll
     for (int w = 0; w < kRowKeyThreads / 32; ++w) s += ws[w];
     if (s) atomicAdd(reinterpret_cast<unsigned long long*>(total), s);
+  }
+  for (int i = threadIdx.x; i < 4 * 256; i += kRowKeyThreads) {
+    const uint32_t c = (&h[0][0])[i];
+    if (c) atomicAdd(dhist + i, c);
   }
 }
 
@@ -382,13 +397,13 @@ extern "C" ss_status ss_intersect_tiles(const ss_dims* dims, const float* row_de
   if (s) return s;
   // the rows' depth keys and the exact total
   k_row_keys<<<(unsigned)min64(ceil_div(nnz, kRowKeyThreads), 148 * 8), kRowKeyThreads, 0, st>>>(
-      g, row_depth, aabb16, nnz, t.dk_a, t.total);
+      g, row_depth, aabb16, nnz, t.dk_a, t.total, t.dhist);
   s = cuda_status(cudaGetLastError(), "row keys");
   if (s) return s;
   // the rows in depth order (ties by row index: the sort is stable and the
   // row index is the key's low word)
   bool in_b = false;
-  s = radix_sort_pairs(t.dk_a, nullptr, t.dk_b, nullptr, nnz, 0, 4, nullptr, t.sort, st, &in_b, nullptr, 0,
+  s = radix_sort_pairs(t.dk_a, nullptr, t.dk_b, nullptr, nnz, 0, 4, t.dhist, t.sort, st, &in_b, nullptr, 0,
                        nullptr);
   if (s) return s;
   const uint64_t* dkeys = in_b ? t.dk_b : t.dk_a;

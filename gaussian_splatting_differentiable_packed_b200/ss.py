@@ -515,9 +515,10 @@ def sort_launches(n_isects: int, passes: int, given_hist: bool = True) -> int:
 
 def launches_per_step(d: ss_dims, nnz: int, n_isects: int, sort_passes: int, depth_passes: int) -> int:
     """Kernels libss launches in one forward+backward step (memsets excluded):
-    projection 5 (pass 1, three scan kernels, pass 2), intersection 4 plus
-    one per depth-sort pass (row depth keys with the count, the depth sort's
-    histogram and bases, the fused offsets-and-write kernel), the sort
+    projection 5 (pass 1, three scan kernels, pass 2), intersection 3 plus
+    one per depth-sort pass (row depth keys with the count and the depth
+    bytes' digit counts, the depth sort's bases, the fused offsets-and-write
+    kernel), the sort
     (sort_launches), tile order 3 (histogram, scan, scatter), rasterizer
     1 + 1, projection backward 1.  With no Gaussians only the tile order and
     the two rasterizers launch (they still write the empty images)."""
@@ -525,7 +526,7 @@ def launches_per_step(d: ss_dims, nnz: int, n_isects: int, sort_passes: int, dep
         return 3 + 2
     n = 5
     if nnz > 0:
-        n += 4 + depth_passes
+        n += 3 + depth_passes
     n += sort_launches(n_isects, sort_passes)
     return n + 3 + 3
 

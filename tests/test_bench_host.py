@@ -45,12 +45,13 @@ def test_traffic_record_guards(tmp_path, monkeypatch):
 
 
 def test_launches_per_step():
-    """projection 5, intersection 6 plus one per depth-sort pass, the sort's
-    histogram, bases, one kernel per digit pass that runs and tile ranges,
-    the tile order 3, rasterizers 2, projection backward 1."""
+    """projection 5, intersection 3 plus one per depth-sort pass, the sort's
+    bases (its digit counts come with the keys), one kernel per digit pass
+    that runs and tile ranges, the tile order 3, rasterizers 2, projection
+    backward 1."""
     d = ss.make_dims(5, 1600, 1067, 3, 15_000_000)
-    assert ss.launches_per_step(d, 15_000_000, 33_000_000, 2, 3) == 5 + (4 + 3) + (2 + 2) + 3 + 2 + 1
-    assert ss.launches_per_step(d, 15_000_000, 0, 0, 3) == 5 + (4 + 3) + 0 + 3 + 2 + 1
+    assert ss.launches_per_step(d, 15_000_000, 33_000_000, 2, 3) == 5 + (3 + 3) + (2 + 2) + 3 + 2 + 1
+    assert ss.launches_per_step(d, 15_000_000, 0, 0, 3) == 5 + (3 + 3) + 0 + 3 + 2 + 1
     assert ss.launches_per_step(d, 0, 0, 0, 0) == 5 + 0 + 0 + 3 + 2 + 1
     assert ss.launches_per_step(ss.make_dims(1, 64, 64, 0, 0), 0, 0, 0, 0) == 3 + 2
 

@@ -159,10 +159,10 @@ def stage_model(d, K, nnz, n_isects, passes, n_tiles, work, n_seen=None, depth_p
     m = {}
     m["project_packed"] = dict(bytes=par * N + P / 8 + P / 32 + P / 16 + (par + 4) * N + shb * n_seen
                                + (row + 8 + 4) * nnz, instr=P * 140.0 + nnz * 160.0)
-    # depth keys of the rows and the count (depth 4 B and AABB 8 B read, key 8
-    # B written), their keys-only sort (histogram 8 B, 16 B per byte pass),
-    # the write (key 8 B, AABB 8 B, offsets 8 B; 12 B per key)
-    m["intersect_tiles"] = dict(bytes=nnz * (20 + 8 + 16 * depth_passes + 24) + 12 * n_isects, instr=0.0)
+    # depth keys of the rows, the count and the depth digits (depth 4 B and
+    # AABB 8 B read, key 8 B written), their keys-only sort (16 B per byte
+    # pass), the write (key 8 B, AABB 8 B, offsets 8 B; 12 B per key)
+    m["intersect_tiles"] = dict(bytes=nnz * (20 + 16 * depth_passes + 24) + 12 * n_isects, instr=0.0)
     # 12 B read + 12 B written per key per digit pass that runs (the tile-id
     # bytes: the keys arrive in depth order, with their digit counts from the
     # intersection), tile offsets
